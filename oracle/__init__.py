@@ -1,0 +1,300 @@
+"""CPU oracle for KIVI-style low-bit KV-cache decode attention -- TEST INFRASTRUCTURE.
+
+Only the tests, the smoke check and the benchmark's CPU-baseline leg may use
+this package.  It is a plain restatement of the method written from the
+pages (see ``kvq_oracle.c`` for the passages followed): the numeric core is
+plain C compiled with gcc (fp32 codes without FMA contraction or fast-math,
+fp64 attention), and this module only marshals numpy arrays into it and keeps
+the streaming bookkeeping of the KIVI residual (section 1 of "LLM系列：
+KVCache量化1 KIVI ...": new tokens go to the full-precision residual; when it
+holds R tokens it is quantized, appended to the quantized part and reset).
+
+It shares no code with the CUDA library and imports nothing from it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kvq_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+OK, EINVAL, ERANGE = 0, 1, 2
+FP16, BF16 = 0, 1
+
+
+def build(force: bool = False) -> str:
+    """Compile ``liboracle.so`` next to its source (gcc, OpenMP when available)."""
+    if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
+        return _LIB
+    base = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+            "-fno-fast-math", "-Wall"]
+    tmp = _LIB + f".tmp{os.getpid()}"
+    try:
+        subprocess.run(base + ["-fopenmp", "-o", tmp, _SRC, "-lm"], check=True,
+                       capture_output=True)
+    except subprocess.CalledProcessError:
+        subprocess.run(base + ["-o", tmp, _SRC, "-lm"], check=True)
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i64, i32 = ctypes.c_int64, ctypes.c_int
+        lib.oracle_widen.restype = ctypes.c_float
+        lib.oracle_widen.argtypes = [ctypes.c_uint16, i32]
+        lib.oracle_asym_params.restype = i32
+        lib.oracle_asym_params.argtypes = [P, i64, i64, i32, P, P]
+        lib.oracle_asym_code.restype = i32
+        lib.oracle_asym_code.argtypes = [ctypes.c_float, ctypes.c_float, ctypes.c_int32, i32]
+        lib.oracle_sym_params.restype = i32
+        lib.oracle_sym_params.argtypes = [P, i64, i64, i32, P]
+        lib.oracle_sym_code.restype = i32
+        lib.oracle_sym_code.argtypes = [ctypes.c_float, ctypes.c_float, i32]
+        lib.oracle_quantize_kv.restype = i32
+        lib.oracle_quantize_kv.argtypes = [P, P, i32, i64, i64, i32, i32, i32, i32, i32,
+                                           P, P, P, P, P, P]
+        lib.oracle_code_position.restype = None
+        lib.oracle_code_position.argtypes = [i64, i32, i32, i32, i32, P, P]
+        lib.oracle_pack.restype = i32
+        lib.oracle_pack.argtypes = [P, i64, i64, i32, i32, i32, P]
+        lib.oracle_unpack.restype = i32
+        lib.oracle_unpack.argtypes = [P, i64, i64, i32, i32, i32, P]
+        lib.oracle_dequant.restype = ctypes.c_double
+        lib.oracle_dequant.argtypes = [i32, ctypes.c_float, ctypes.c_int32]
+        lib.oracle_decode_attention.restype = i32
+        lib.oracle_decode_attention.argtypes = [P, P, P, P, P, P, i64, P, P, i64, i64, P,
+                                                i32, i64, i32, i32, i32, i32, i32, i32, i32, P]
+        lib.oracle_num_threads.restype = i32
+        lib.oracle_num_threads.argtypes = []
+        _lib = lib
+        return lib
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc: int, what: str):
+    if rc != OK:
+        raise ValueError(f"oracle {what} rejected its input (status {rc})")
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+# ----------------------------------------------------------------------------
+# scalar / small helpers
+# ----------------------------------------------------------------------------
+
+def widen(bits: np.ndarray, dtype: int) -> np.ndarray:
+    """Exact fp16/bf16 -> fp32 widening of an array of element bit patterns."""
+    lib = _load()
+    flat = np.ascontiguousarray(bits, dtype=np.uint16).ravel()
+    out = np.array([lib.oracle_widen(int(b), dtype) for b in flat], dtype=np.float32)
+    return out.reshape(np.shape(bits))
+
+
+def asym_params(x: np.ndarray, bits: int):
+    """(s, z) of one asymmetric min-max group."""
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    s = np.zeros(1, np.float32)
+    z = np.zeros(1, np.int32)
+    _check(lib.oracle_asym_params(_ptr(x), x.size, 1, bits, _ptr(s), _ptr(z)), "asym_params")
+    return float(s[0]), int(z[0])
+
+
+def asym_codes(x: np.ndarray, bits: int):
+    """(codes, s, z) of one asymmetric group."""
+    lib = _load()
+    s, z = asym_params(x, bits)
+    codes = np.array([lib.oracle_asym_code(float(v), s, z, bits)
+                      for v in np.asarray(x, np.float32)], dtype=np.int32)
+    return codes, s, z
+
+
+def sym_codes(x: np.ndarray, bits: int):
+    """(offset codes u, s) of one symmetric group."""
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    s = np.zeros(1, np.float32)
+    _check(lib.oracle_sym_params(_ptr(x), x.size, 1, bits, _ptr(s)), "sym_params")
+    codes = np.array([lib.oracle_sym_code(float(v), float(s[0]), bits) for v in x],
+                     dtype=np.int32)
+    return codes, float(s[0])
+
+
+def dequant(code: int, s: float, z: int) -> float:
+    return float(_load().oracle_dequant(int(code), float(s), int(z)))
+
+
+def code_position(t: int, c: int, is_v: bool, d: int, bits: int):
+    lib = _load()
+    w = ctypes.c_int64()
+    b = ctypes.c_int()
+    lib.oracle_code_position(t, c, int(is_v), d, bits, ctypes.byref(w), ctypes.byref(b))
+    return int(w.value), int(b.value)
+
+
+# ----------------------------------------------------------------------------
+# block quantisation, packing, attention
+# ----------------------------------------------------------------------------
+
+def quantize_kv(XK: np.ndarray, XV: np.ndarray, dtype: int, G: int, Gv: int, bits: int,
+                symmetric: bool = False) -> dict:
+    """Quantise K/V element bits shaped [BH, T, d] (KIVI: K per channel, V per token)."""
+    lib = _load()
+    XK = np.ascontiguousarray(XK, dtype=np.uint16)
+    XV = np.ascontiguousarray(XV, dtype=np.uint16)
+    BH, T, d = XK.shape
+    assert XV.shape == XK.shape
+    Kq = np.zeros((BH, T, d), np.uint8)
+    Vq = np.zeros((BH, T, d), np.uint8)
+    Ks = np.zeros((BH, T // G, d), np.float32)
+    Kz = np.zeros((BH, T // G, d), np.int16)
+    Vs = np.zeros((BH, T, d // Gv), np.float32)
+    Vz = np.zeros((BH, T, d // Gv), np.int16)
+    rc = lib.oracle_quantize_kv(_ptr(XK), _ptr(XV), dtype, BH, T, d, G, Gv, bits, int(symmetric),
+                                _ptr(Kq), _ptr(Ks), _ptr(Kz), _ptr(Vq), _ptr(Vs), _ptr(Vz))
+    _check(rc, "quantize_kv")
+    return dict(Kq=Kq, Ks=Ks, Kz=Kz, Vq=Vq, Vs=Vs, Vz=Vz)
+
+
+def pack(q: np.ndarray, bits: int, is_v: bool) -> np.ndarray:
+    """Pack codes [BH, T, d] into the tile layout -> uint32 [BH, T*d*bits/32]."""
+    lib = _load()
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    BH, T, d = q.shape
+    out = np.zeros((BH, T * d * bits // 32), np.uint32)
+    _check(lib.oracle_pack(_ptr(q), BH, T, d, bits, int(is_v), _ptr(out)), "pack")
+    return out
+
+
+def unpack(words: np.ndarray, T: int, d: int, bits: int, is_v: bool) -> np.ndarray:
+    lib = _load()
+    words = np.ascontiguousarray(words, dtype=np.uint32)
+    BH = words.shape[0]
+    q = np.zeros((BH, T, d), np.uint8)
+    _check(lib.oracle_unpack(_ptr(words), BH, T, d, bits, int(is_v), _ptr(q)), "unpack")
+    return q
+
+
+def decode_attention(qcache: dict, Tq: int, Kr: np.ndarray, Vr: np.ndarray, r: int,
+                     Q: np.ndarray, dtype: int, B: int, Hq: int, Hkv: int, d: int,
+                     G: int, Gv: int, bits: int, symmetric: bool) -> np.ndarray:
+    """fp64 decode attention of queries Q [B, Hq, d] over [deq(quantized); residual]."""
+    lib = _load()
+    Q = np.ascontiguousarray(Q, dtype=np.uint16)
+    Kr = np.ascontiguousarray(Kr, dtype=np.uint16)
+    Vr = np.ascontiguousarray(Vr, dtype=np.uint16)
+    Rcap = Kr.shape[1]
+    out = np.zeros((B, Hq, d), np.float64)
+    arrs = [np.ascontiguousarray(qcache[k]) for k in ("Kq", "Ks", "Kz", "Vq", "Vs", "Vz")]
+    rc = lib.oracle_decode_attention(*[_ptr(a) for a in arrs], Tq, _ptr(Kr), _ptr(Vr), Rcap, r,
+                                     _ptr(Q), dtype, B, Hq, Hkv, d, G, Gv, bits,
+                                     int(symmetric), _ptr(out))
+    _check(rc, "decode_attention")
+    return out
+
+
+# ----------------------------------------------------------------------------
+# streaming cache (KIVI section 1: quantized part + residual of < R tokens)
+# ----------------------------------------------------------------------------
+
+class OracleCache:
+    """Prefill / append / decode with KIVI's residual.
+
+    Prefill of T tokens quantises the first floor(T/R)*R of them and keeps the
+    rest in the residual; each append adds one token to the residual and, when
+    the residual reaches R tokens, quantises all R of them, appends them to
+    the quantized part and empties the residual.  Attention therefore always
+    sees fewer than R residual tokens.
+    """
+
+    def __init__(self, B, Hq, Hkv, d, G, Gv, R, bits, symmetric=False, dtype=BF16):
+        assert R % G == 0 and d % Gv == 0 and Hq % Hkv == 0
+        self.B, self.Hq, self.Hkv, self.d = B, Hq, Hkv, d
+        self.G, self.Gv, self.R, self.bits = G, Gv, R, bits
+        self.symmetric, self.dtype = symmetric, dtype
+        BH = B * Hkv
+        self.blocks = []                       # quantized blocks, each R*k tokens
+        self.Kr = np.zeros((BH, R, d), np.uint16)
+        self.Vr = np.zeros((BH, R, d), np.uint16)
+        self.r = 0
+        self.Tq = 0
+        self.flushes = 0
+        self._cat = None
+
+    def _quantize_block(self, XK, XV):
+        blk = quantize_kv(XK, XV, self.dtype, self.G, self.Gv, self.bits, self.symmetric)
+        self.blocks.append(blk)
+        self.Tq += XK.shape[1]
+        self._cat = None
+
+    def prefill(self, XK: np.ndarray, XV: np.ndarray):
+        """XK, XV element bits [B, Hkv, T, d]."""
+        assert self.Tq == 0 and self.r == 0
+        B, Hkv, T, d = XK.shape
+        XK = XK.reshape(B * Hkv, T, d)
+        XV = XV.reshape(B * Hkv, T, d)
+        Tq = (T // self.R) * self.R
+        if Tq:
+            self._quantize_block(XK[:, :Tq], XV[:, :Tq])
+        self.r = T - Tq
+        self.Kr[:, :self.r] = XK[:, Tq:]
+        self.Vr[:, :self.r] = XV[:, Tq:]
+
+    def append(self, tK: np.ndarray, tV: np.ndarray):
+        """tK, tV element bits [B, Hkv, d]; flushes the residual when it fills."""
+        BH = self.B * self.Hkv
+        self.Kr[:, self.r] = tK.reshape(BH, self.d)
+        self.Vr[:, self.r] = tV.reshape(BH, self.d)
+        self.r += 1
+        if self.r == self.R:
+            self._quantize_block(self.Kr.copy(), self.Vr.copy())
+            self.flushes += 1
+            self.r = 0
+
+    def quantized(self) -> dict:
+        """All quantized tokens so far, concatenated along the token axis."""
+        if self._cat is None:
+            if not self.blocks:
+                BH, d = self.B * self.Hkv, self.d
+                self._cat = dict(Kq=np.zeros((BH, 0, d), np.uint8),
+                                 Ks=np.zeros((BH, 0, d), np.float32),
+                                 Kz=np.zeros((BH, 0, d), np.int16),
+                                 Vq=np.zeros((BH, 0, d), np.uint8),
+                                 Vs=np.zeros((BH, 0, d // self.Gv), np.float32),
+                                 Vz=np.zeros((BH, 0, d // self.Gv), np.int16))
+            else:
+                self._cat = {k: np.concatenate([b[k] for b in self.blocks], axis=1)
+                             for k in self.blocks[0]}
+        return self._cat
+
+    def packed(self) -> dict:
+        """Quantized part in the library's storage format (codes packed)."""
+        qc = self.quantized()
+        return dict(Kc=pack(qc["Kq"], self.bits, False), Vc=pack(qc["Vq"], self.bits, True),
+                    Ks=qc["Ks"], Kz=qc["Kz"], Vs=qc["Vs"], Vz=qc["Vz"])
+
+    def decode(self, Q: np.ndarray) -> np.ndarray:
+        """Q element bits [B, Hq, d] -> fp64 output [B, Hq, d]."""
+        return decode_attention(self.quantized(), self.Tq, self.Kr, self.Vr, self.r, Q,
+                                self.dtype, self.B, self.Hq, self.Hkv, self.d, self.G,
+                                self.Gv, self.bits, self.symmetric)
