@@ -1,0 +1,404 @@
+"""Benchmark: decode attention over a KIVI-style low-bit KV cache on B200.
+
+One step = one full pass of the hot path over one batch: prefill-quantize the
+prompt (keys per channel, values per token, residual tail), then every decode
+step of the workload (append the new token -- flushing the residual when it
+holds R tokens -- and split-K decode attention with its log-sum-exp combine).
+The metric is KV tokens attended per second: each decode step attends to
+B * (Tq + r) cached tokens.
+
+Default workload: llama7b (B8, 32 MHA heads, d128, 4096-token prompt bf16,
+4-bit asymmetric, G = Gv = R = 128, 128 decode steps).  Multi-GPU runs are
+weak-scaled: every rank serves its own batch of 8 sequences (no data-path
+collective).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+       python bench.py --impl reference ...   (the CPU oracle, rank 0 only)
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "quantized-KV decode attn: KV tokens/s and achieved HBM GB/s vs B200 peak"
+UNIT = "KV tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--workload", default="llama7b")
+    p.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--ncu-case", action="store_true",
+                   help="run one prefill and 3 decode steps of the workload, then exit (for ncu)")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def algorithmic_bytes(w, Tq: int, r: int) -> int:
+    """Bytes one decode attention must move: packed codes, scales/zeros, residual
+    rows, the query and the fp32 output."""
+    BH = w.B * w.Hkv
+    meta = 4 if w.symmetric else 6
+    # codes of K and V, key meta amortised over its G tokens, value meta per token
+    per_tok = 2 * w.d * w.bits / 8 + w.d * meta / w.G + (w.d // w.Gv) * meta
+    return int(BH * (Tq * per_tok + r * 2 * w.d * 2) + w.B * w.Hq * w.d * (2 + 4))
+
+
+def episode_contexts(w):
+    """(Tq, r) seen by each decode step of an episode."""
+    out = []
+    Tq, r = (w.T // w.R) * w.R, w.T % w.R
+    for _ in range(w.steps):
+        r += 1
+        if r == w.R:
+            Tq, r = Tq + w.R, 0
+        out.append((Tq, r))
+    return out
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def ncu_traffic(workload: str):
+    """Per-launch DRAM bytes of the decode kernel from the committed ncu summary,
+    if it was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"decode_split_kernel_{workload}.md")
+    src = os.path.join(ROOT, "bit_kv_cache_22_b200", "csrc", "decode.cu")
+    try:
+        text = open(path).read()
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        m_sha = re.search(r"decode\.cu sha256\[:16\]:\s*([0-9a-f]{16})", text)
+        m_b = re.search(r"dram bytes per launch:\s*([0-9]+)", text)
+        if m_sha and m_b and m_sha.group(1) == sha:
+            return int(m_b.group(1))
+    except OSError:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the library arm
+# ---------------------------------------------------------------------------
+
+def run_kvq(args):
+    import torch
+    import torch.distributed as dist
+
+    from bit_kv_cache_22_b200 import kvq
+    from bit_kv_cache_22_b200 import workloads as wl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
+
+    base = wl.WORKLOADS[args.workload]
+    w = base.replace(seed=base.seed + 1000 * rank) if rank else base
+    dt = torch.float16 if w.dtype == wl.FP16 else torch.bfloat16
+
+    def to_t(bits, pin=False):
+        t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(dt)
+        return t.pin_memory() if pin else t
+
+    XK_h, XV_h = wl.prefill_bits(w)
+    tK_h, tV_h, tQ_h = wl.decode_bits(w)
+    XK, XV = to_t(XK_h).to(dev), to_t(XV_h).to(dev)
+    tK, tV, tQ = to_t(tK_h).to(dev), to_t(tV_h).to(dev), to_t(tQ_h).to(dev)
+    cache = kvq.KVQCache(w.B, w.Hq, w.Hkv, w.d, w.G, w.Gv, w.R, w.bits, w.symmetric, dt,
+                         w.capacity, dev)
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    if args.ncu_case:
+        cache.prefill_quantize(XK, XV)
+        for s in range(3):
+            cache.append(tK[s], tV[s])
+            cache.decode_attention(tQ[s], out=out)
+        torch.cuda.synchronize()
+        print(json.dumps({"ncu_case": args.workload, "state": cache.state()}))
+        return
+
+    ctx = episode_contexts(w)
+    tokens_per_episode = sum(w.B * (tq + r) for tq, r in ctx)
+    bytes_per_episode = sum(algorithmic_bytes(w, tq, r) for tq, r in ctx)
+
+    def episode(ev=None):
+        cache.reset()
+        cache.prefill_quantize(XK, XV)
+        for s in range(w.steps):
+            cache.append(tK[s], tV[s])
+            if ev is not None:
+                ev[s][0].record(stream)
+            cache.decode_attention(tQ[s], out=out)
+            if ev is not None:
+                ev[s][1].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        episode()
+    torch.cuda.synchronize()
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(w.steps)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = kvq.kernel_launches()
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for k in range(args.steps):
+            episode(evs[k])
+        stop.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    launches = kvq.kernel_launches() - launches0
+    ms = start.elapsed_time(stop)
+    decode_ms = sum(a.elapsed_time(b) for ev in evs for a, b in ev)
+    t = torch.tensor([ms, decode_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms, decode_ms = float(t[0]), float(t[1])
+
+    # ---- end to end through the public API with pinned host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        XKp, XVp = to_t(XK_h, True), to_t(XV_h, True)
+        tKp, tVp, tQp = to_t(tK_h, True), to_t(tV_h, True), to_t(tQ_h, True)
+        outs = torch.empty((w.steps, w.B, w.Hq, w.d), dtype=torch.float32).pin_memory()
+
+        def e2e_episode():
+            cache.reset()
+            cache.prefill_quantize(XKp, XVp)           # host -> device inside the call path
+            for s in range(w.steps):
+                cache.append(tKp[s], tVp[s])
+                cache.decode_attention(tQp[s], out=outs[s])   # device -> host of t_O
+        for _ in range(max(1, args.warmup)):
+            e2e_episode()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_episode()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e_ms = float(te[0])
+        h2d = XKp.numel() * 2 * 2 + w.steps * (2 * w.B * w.Hkv * w.d + w.B * w.Hq * w.d) * 2
+        d2h = w.steps * w.B * w.Hq * w.d * 4
+        e2e = {"value": tokens_per_episode * args.steps * world / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e2e_ms / args.steps}
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, budget_s=20.0)
+
+    peak, peak_kind = peaks()
+    decode_launch_ms = decode_ms / (args.steps * w.steps)
+    achieved = bytes_per_episode / w.steps / (decode_launch_ms / 1e3) / 1e9
+    traffic = ncu_traffic(args.workload)
+    line = {
+        "metric": METRIC,
+        "value": tokens_per_episode * args.steps * world / (ms / 1e3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": f"u{w.bits} codes, f32 accumulate",
+        "data": "synthetic (seeded; distributions of the workload definition)",
+        "config": {
+            "workload": w.name, "batch_per_gpu": w.B, "global_batch": w.B * world,
+            "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d, "prompt_tokens": w.T,
+            "decode_steps": w.steps, "bits": w.bits, "group_k": w.G, "group_v": w.Gv,
+            "residual": w.R, "symmetric": w.symmetric,
+            "elem": "fp16" if w.dtype == wl.FP16 else "bf16",
+            "parallelism": f"dp{world} (independent sequences per GPU)",
+            "l2": "inputs larger than L2: packed cache "
+                  f"{bytes_per_episode / w.steps / 1e6:.0f} MB per decode step, prompt "
+                  f"{2 * XK.numel() * 2 / 1e6:.0f} MB per step",
+            "splits": cache.splits(),
+        },
+        "decode_steps_per_s": w.steps * args.steps / (ms / 1e3),
+        "kv_tokens_per_s_decode_only": tokens_per_episode * args.steps * world / (decode_ms / 1e3),
+        "roofline": {
+            "kernel": "decode_attention (split-K kernel + combine), per call",
+            "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+            if peak_kind == "measured" else "fallback 6.65 TB/s",
+            "algorithmic_bytes_per_launch": bytes_per_episode / w.steps,
+            "avg_launch_us": decode_launch_ms * 1e3,
+            "traffic": traffic,
+        },
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (cpu_baseline leg and --impl reference)
+# ---------------------------------------------------------------------------
+
+def cpu_baseline(w, budget_s=20.0, steps=None):
+    """Time the oracle (as it stands) on a bounded sample of the workload: one
+    sequence (all of its kv heads), its prompt prefill and the first decode
+    steps, stopping after ~budget_s seconds.  Returns KV tokens/s for that sample."""
+    import oracle
+    from bit_kv_cache_22_b200 import workloads as wl
+    XK, XV = wl.prefill_bits(w, bs=[0])
+    tK, tV, tQ = wl.decode_bits(w, bs=[0])
+    t0 = time.perf_counter()
+    c = oracle.OracleCache(1, w.Hq, w.Hkv, w.d, w.G, w.Gv, w.R, w.bits, w.symmetric, w.dtype)
+    c.prefill(XK, XV)
+    tokens, done = 0, 0
+    limit = w.steps if steps is None else steps
+    for s in range(limit):
+        c.append(tK[s], tV[s])
+        c.decode(tQ[s])
+        tokens += c.Tq + c.r
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    el = time.perf_counter() - t0
+    return {"value": tokens / el, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"1 of {w.B} sequences (all {w.Hkv} kv heads): prefill of {w.T} tokens + "
+                      f"{done} of {w.steps} decode steps, {el:.1f} s, fp64 C oracle with OpenMP"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from bit_kv_cache_22_b200 import workloads as wl
+    w = wl.WORKLOADS[args.workload]
+    budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_baseline(w, budget_s=budget)
+    vals = [cpu_baseline(w, budget_s=budget) for _ in range(args.steps)]
+    v = statistics.mean(x["value"] for x in vals)
+    line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "impl": "reference", "dtype": "f64",
+            "data": "synthetic (seeded)",
+            "config": {"workload": w.name, "global_batch": w.B, "note": "CPU oracle, rank 0"},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": vals[0]["cores"],
+                             "kind": "oracle", "sample": vals[0]["sample"]},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def main():
+    args = _args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_kvq(args)
+
+
+if __name__ == "__main__":
+    main()

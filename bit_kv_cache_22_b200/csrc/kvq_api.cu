@@ -1,0 +1,374 @@
+// kvq_api.cu -- the C ABI of include/kvq.h: validation, host-side cache state and launches.
+//
+// The handle keeps only geometry, the caller's device pointers and the two
+// counters of the KIVI cache ("LLM系列：KVCache量化1 KIVI ...", section 1):
+// Tq quantized tokens and r < R residual tokens.  Every branch of the
+// streaming logic (when to flush, where a token goes) is decided here on the
+// host from those counters, so the kernels need no device-side control flow
+// and a sequence of calls never waits on the device.
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <atomic>
+#include <new>
+#include <string>
+
+#include "../../include/kvq.h"
+#include "kvq_internal.cuh"
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}  // namespace
+
+void kvq::count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
+
+namespace {
+
+thread_local std::string g_last_error;
+
+kvq_status fail(kvq_status st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+kvq_status fail(kvq_status st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+kvq_status ok() {
+    g_last_error.clear();
+    return KVQ_OK;
+}
+
+kvq_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(KVQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kMaxSplits = 64;
+constexpr int kMinTilesPerSplit = 4;
+
+kvq_status validate(const kvq_config *c) {
+    if (!c) return fail(KVQ_ERR_INVALID_ARG, "config is NULL");
+    if (c->batch < 1 || c->q_heads < 1 || c->kv_heads < 1)
+        return fail(KVQ_ERR_INVALID_ARG, "batch, q_heads and kv_heads must be >= 1");
+    if (c->q_heads % c->kv_heads != 0)
+        return fail(KVQ_ERR_INVALID_ARG, "q_heads (%d) must be a multiple of kv_heads (%d)",
+                    c->q_heads, c->kv_heads);
+    if (static_cast<int64_t>(c->batch) * c->kv_heads > 65535 ||
+        static_cast<int64_t>(c->batch) > 65535 || c->q_heads > 65535)
+        return fail(KVQ_ERR_UNSUPPORTED, "batch * kv_heads must be <= 65535");
+    if (c->bits != 2 && c->bits != 4)
+        return fail(KVQ_ERR_UNSUPPORTED, "bits must be 2 or 4 (got %d)", c->bits);
+    if (c->head_dim != 64 && c->head_dim != 128)
+        return fail(KVQ_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", c->head_dim);
+    if (c->group_k < 16 || c->group_k % 16 != 0 || c->group_k > 256 ||
+        c->group_k * c->head_dim > 32768)
+        return fail(KVQ_ERR_INVALID_ARG,
+                    "group_k must be a multiple of 16, <= 256, with group_k*head_dim <= 32768");
+    if (!(c->group_v == 16 || c->group_v == 32 || c->group_v == 64 || c->group_v == 128) ||
+        c->group_v > c->head_dim)
+        return fail(KVQ_ERR_INVALID_ARG, "group_v must be 16, 32, 64 or 128 and <= head_dim");
+    if (c->residual < c->group_k || c->residual % c->group_k != 0)
+        return fail(KVQ_ERR_INVALID_ARG, "residual (%d) must be a positive multiple of group_k (%d)",
+                    c->residual, c->group_k);
+    if (c->symmetric != 0 && c->symmetric != 1)
+        return fail(KVQ_ERR_INVALID_ARG, "symmetric must be 0 or 1");
+    if (c->dtype != KVQ_FP16 && c->dtype != KVQ_BF16)
+        return fail(KVQ_ERR_INVALID_ARG, "dtype must be KVQ_FP16 or KVQ_BF16");
+    if (c->capacity < c->residual || c->capacity % c->residual != 0)
+        return fail(KVQ_ERR_INVALID_ARG, "capacity must be a positive multiple of residual");
+    if (c->capacity / 16 > (int64_t{1} << 30))
+        return fail(KVQ_ERR_UNSUPPORTED, "capacity too large");
+    return KVQ_OK;
+}
+
+int max_splits(const kvq_config *c) {
+    const int64_t tiles = c->capacity / 16 + c->residual / 16;
+    return static_cast<int>(tiles < kMaxSplits ? tiles : kMaxSplits);
+}
+
+}  // namespace
+
+struct kvq_cache {
+    kvq_config cfg;
+    kvq_buffers buf;
+    int64_t Tq = 0;
+    int32_t r = 0;
+    int num_sms = 148;
+    int ctas_per_sm = 4;
+    int split_limit = 64;
+};
+
+namespace {
+
+// Split count for the current cache length: enough CTAs to fill the GPU once,
+// at least kMinTilesPerSplit tiles each, at most kMaxSplits.
+void plan_splits(const kvq_cache *h, int *S_out, int *tiles_per_split) {
+    const kvq_config &c = h->cfg;
+    const int64_t tiles = h->Tq / 16 + (h->r + 15) / 16;
+    const int64_t units = static_cast<int64_t>(c.batch) * c.q_heads;
+    const int64_t target = static_cast<int64_t>(h->num_sms) * h->ctas_per_sm;
+    int64_t S = (target + units - 1) / units;
+    const int64_t by_tiles = (tiles + kMinTilesPerSplit - 1) / kMinTilesPerSplit;
+    if (S > by_tiles) S = by_tiles;
+    if (S > max_splits(&c)) S = max_splits(&c);
+    if (S > h->split_limit) S = h->split_limit;
+    if (S < 1) S = 1;
+    int64_t per = (tiles + S - 1) / S;
+    if (per < 1) per = 1;
+    S = (tiles + per - 1) / per;
+    if (S < 1) S = 1;
+    *S_out = static_cast<int>(S);
+    *tiles_per_split = static_cast<int>(per);
+}
+
+kvq::DecodeArgs decode_args(const kvq_cache *h) {
+    const kvq_config &c = h->cfg;
+    kvq::DecodeArgs a{};
+    a.kc = static_cast<const uint32_t *>(h->buf.k_codes);
+    a.vc = static_cast<const uint32_t *>(h->buf.v_codes);
+    a.ks = h->buf.k_scales;
+    a.vs = h->buf.v_scales;
+    a.kz = h->buf.k_zeros;
+    a.vz = h->buf.v_zeros;
+    a.kr = static_cast<const uint16_t *>(h->buf.k_residual);
+    a.vr = static_cast<const uint16_t *>(h->buf.v_residual);
+    a.cap = c.capacity;
+    a.B = c.batch;
+    a.Hq = c.q_heads;
+    a.Hkv = c.kv_heads;
+    a.d = c.head_dim;
+    a.G = c.group_k;
+    a.Gv = c.group_v;
+    a.R = c.residual;
+    a.bits = c.bits;
+    a.sym = c.symmetric != 0;
+    a.bf16 = c.dtype == KVQ_BF16;
+    a.qscale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c.head_dim)));
+    return a;
+}
+
+kvq::QuantizeArgs quantize_args(const kvq_cache *h) {
+    const kvq_config &c = h->cfg;
+    kvq::QuantizeArgs q{};
+    q.BH = static_cast<int64_t>(c.batch) * c.kv_heads;
+    q.d = c.head_dim;
+    q.G = c.group_k;
+    q.Gv = c.group_v;
+    q.bits = c.bits;
+    q.sym = c.symmetric != 0;
+    q.bf16 = c.dtype == KVQ_BF16;
+    q.kc = static_cast<uint32_t *>(h->buf.k_codes);
+    q.vc = static_cast<uint32_t *>(h->buf.v_codes);
+    q.ks = h->buf.k_scales;
+    q.vs = h->buf.v_scales;
+    q.kz = h->buf.k_zeros;
+    q.vz = h->buf.v_zeros;
+    q.cap = c.capacity;
+    return q;
+}
+
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_get_sizes(const kvq_config *cfg, kvq_sizes *out) {
+    if (!out) return fail(KVQ_ERR_INVALID_ARG, "out is NULL");
+    kvq_status st = validate(cfg);
+    if (st != KVQ_OK) return st;
+    const int64_t BH = static_cast<int64_t>(cfg->batch) * cfg->kv_heads;
+    const int64_t cap = cfg->capacity;
+    const int64_t d = cfg->head_dim;
+    std::memset(out, 0, sizeof *out);
+    out->k_codes = out->v_codes = static_cast<size_t>(BH * cap * d * cfg->bits / 8);
+    out->k_scales = static_cast<size_t>(BH * (cap / cfg->group_k) * d * 4);
+    out->k_zeros = cfg->symmetric ? 0 : static_cast<size_t>(BH * (cap / cfg->group_k) * d * 2);
+    out->v_scales = static_cast<size_t>(BH * cap * (d / cfg->group_v) * 4);
+    out->v_zeros = cfg->symmetric ? 0 : static_cast<size_t>(BH * cap * (d / cfg->group_v) * 2);
+    out->k_residual = out->v_residual = static_cast<size_t>(BH * cfg->residual * d * 2);
+    const int64_t units = static_cast<int64_t>(cfg->batch) * cfg->q_heads;
+    out->workspace = static_cast<size_t>(units * max_splits(cfg) * (d + 2) * 4);
+    return ok();
+}
+
+kvq_status kvq_create(const kvq_config *cfg, const kvq_buffers *bufs, kvq_cache **out) {
+    if (!out) return fail(KVQ_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    kvq_status st = validate(cfg);
+    if (st != KVQ_OK) return st;
+    if (!bufs) return fail(KVQ_ERR_INVALID_ARG, "buffers are NULL");
+    const void *need[] = {bufs->k_codes, bufs->k_scales, bufs->v_codes, bufs->v_scales,
+                          bufs->k_residual, bufs->v_residual};
+    for (const void *p : need)
+        if (!p || !aligned16(p))
+            return fail(KVQ_ERR_INVALID_ARG, "cache buffers must be non-NULL and 16-byte aligned");
+    if (!cfg->symmetric && (!bufs->k_zeros || !bufs->v_zeros || !aligned16(bufs->k_zeros) ||
+                            !aligned16(bufs->v_zeros)))
+        return fail(KVQ_ERR_INVALID_ARG, "asymmetric caches need 16-byte aligned zero buffers");
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "querying the current device");
+    kvq_cache *h = new (std::nothrow) kvq_cache();
+    if (!h) return fail(KVQ_ERR_INVALID_ARG, "out of host memory");
+    h->cfg = *cfg;
+    h->buf = *bufs;
+    if (cfg->symmetric) {
+        h->buf.k_zeros = nullptr;
+        h->buf.v_zeros = nullptr;
+    }
+    h->num_sms = sms > 0 ? sms : 148;
+    h->ctas_per_sm = kvq::decode_ctas_per_sm(decode_args(h));
+    *out = h;
+    return ok();
+}
+
+void kvq_destroy(kvq_cache *cache) { delete cache; }
+
+kvq_status kvq_reset(kvq_cache *cache) {
+    if (!cache) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+    cache->Tq = 0;
+    cache->r = 0;
+    return ok();
+}
+
+kvq_status kvq_prefill_quantize(kvq_cache *h, const void *X_K, const void *X_V, int64_t T,
+                                void *stream) {
+    if (!h) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+    if (T < 0) return fail(KVQ_ERR_INVALID_ARG, "T must be >= 0");
+    if (h->Tq != 0 || h->r != 0) return fail(KVQ_ERR_STATE, "prefill needs an empty cache");
+    if (T == 0) return ok();
+    if (!X_K || !X_V || !aligned16(X_K) || !aligned16(X_V))
+        return fail(KVQ_ERR_INVALID_ARG, "X_K and X_V must be non-NULL and 16-byte aligned");
+    const kvq_config &c = h->cfg;
+    const int64_t Tq = (T / c.residual) * c.residual;
+    const int64_t r = T - Tq;
+    if (Tq > c.capacity)
+        return fail(KVQ_ERR_CAPACITY, "prefill of %lld tokens exceeds capacity %lld",
+                    static_cast<long long>(Tq), static_cast<long long>(c.capacity));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    kvq::QuantizeArgs q = quantize_args(h);
+    q.xk = static_cast<const uint16_t *>(X_K);
+    q.xv = static_cast<const uint16_t *>(X_V);
+    q.in_bh_stride = T * c.head_dim;
+    q.in_tok0 = 0;
+    q.n_groups = Tq / c.group_k;
+    q.out_tok0 = 0;
+    cudaError_t e = kvq::launch_quantize(q, s);
+    if (e != cudaSuccess) return cuda_fail(e, "prefill quantize launch");
+    const int64_t BH = static_cast<int64_t>(c.batch) * c.kv_heads;
+    const int64_t rstride = static_cast<int64_t>(c.residual) * c.head_dim;
+    e = kvq::launch_copy_rows(static_cast<const uint16_t *>(X_K), T * c.head_dim, Tq,
+                              static_cast<uint16_t *>(h->buf.k_residual), rstride, 0, r, BH,
+                              c.head_dim, s);
+    if (e == cudaSuccess)
+        e = kvq::launch_copy_rows(static_cast<const uint16_t *>(X_V), T * c.head_dim, Tq,
+                                  static_cast<uint16_t *>(h->buf.v_residual), rstride, 0, r, BH,
+                                  c.head_dim, s);
+    if (e != cudaSuccess) return cuda_fail(e, "prefill residual copy launch");
+    h->Tq = Tq;
+    h->r = static_cast<int32_t>(r);
+    return ok();
+}
+
+kvq_status kvq_append(kvq_cache *h, const void *t_K, const void *t_V, void *stream) {
+    if (!h) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+    if (!t_K || !t_V || !aligned16(t_K) || !aligned16(t_V))
+        return fail(KVQ_ERR_INVALID_ARG, "t_K and t_V must be non-NULL and 16-byte aligned");
+    const kvq_config &c = h->cfg;
+    const bool flush = h->r + 1 == c.residual;
+    if (flush && h->Tq + c.residual > c.capacity)
+        return fail(KVQ_ERR_CAPACITY, "flushing the residual would exceed capacity %lld",
+                    static_cast<long long>(c.capacity));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t BH = static_cast<int64_t>(c.batch) * c.kv_heads;
+    const int64_t rstride = static_cast<int64_t>(c.residual) * c.head_dim;
+    cudaError_t e = kvq::launch_copy_rows(static_cast<const uint16_t *>(t_K), c.head_dim, 0,
+                                          static_cast<uint16_t *>(h->buf.k_residual), rstride,
+                                          h->r, 1, BH, c.head_dim, s);
+    if (e == cudaSuccess)
+        e = kvq::launch_copy_rows(static_cast<const uint16_t *>(t_V), c.head_dim, 0,
+                                  static_cast<uint16_t *>(h->buf.v_residual), rstride, h->r, 1, BH,
+                                  c.head_dim, s);
+    if (e != cudaSuccess) return cuda_fail(e, "append launch");
+    if (flush) {
+        kvq::QuantizeArgs q = quantize_args(h);
+        q.xk = static_cast<const uint16_t *>(h->buf.k_residual);
+        q.xv = static_cast<const uint16_t *>(h->buf.v_residual);
+        q.in_bh_stride = rstride;
+        q.in_tok0 = 0;
+        q.n_groups = c.residual / c.group_k;
+        q.out_tok0 = h->Tq;
+        e = kvq::launch_quantize(q, s);
+        if (e != cudaSuccess) return cuda_fail(e, "flush quantize launch");
+        h->Tq += c.residual;
+        h->r = 0;
+    } else {
+        h->r += 1;
+    }
+    return ok();
+}
+
+kvq_status kvq_set_split_limit(kvq_cache *h, int32_t max_splits) {
+    if (!h) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+    if (max_splits < 0 || max_splits > kMaxSplits)
+        return fail(KVQ_ERR_INVALID_ARG, "max_splits must be in 0..%d", kMaxSplits);
+    h->split_limit = max_splits == 0 ? kMaxSplits : max_splits;
+    return ok();
+}
+
+int32_t kvq_decode_splits(const kvq_cache *h) {
+    if (!h) return 0;
+    int S, per;
+    plan_splits(h, &S, &per);
+    return S;
+}
+
+kvq_status kvq_decode_attention(kvq_cache *h, const void *t_Q, float *t_O, void *workspace,
+                                size_t workspace_bytes, void *stream) {
+    if (!h) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+    if (!t_Q || !t_O || !workspace || !aligned16(t_Q) || !aligned16(t_O) || !aligned16(workspace))
+        return fail(KVQ_ERR_INVALID_ARG, "t_Q, t_O and workspace must be non-NULL and 16-byte aligned");
+    if (h->Tq == 0 && h->r == 0) return fail(KVQ_ERR_STATE, "the cache is empty");
+    const kvq_config &c = h->cfg;
+    kvq_sizes sz;
+    kvq_get_sizes(&c, &sz);
+    if (workspace_bytes < sz.workspace)
+        return fail(KVQ_ERR_INVALID_ARG, "workspace needs %zu bytes, got %zu", sz.workspace,
+                    workspace_bytes);
+    kvq::DecodeArgs a = decode_args(h);
+    plan_splits(h, &a.S, &a.tiles_per_split);
+    const int64_t units = static_cast<int64_t>(c.batch) * c.q_heads;
+    float *ws = static_cast<float *>(workspace);
+    a.o_part = ws;
+    a.m_part = ws + units * a.S * c.head_dim;
+    a.l_part = a.m_part + units * a.S;
+    a.q = static_cast<const uint16_t *>(t_Q);
+    a.out = t_O;
+    a.n_qtiles = static_cast<int>(h->Tq / 16);
+    a.r = h->r;
+    cudaError_t e = kvq::launch_decode(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    return ok();
+}
+
+kvq_status kvq_cache_state(const kvq_cache *h, int64_t *quantized_tokens, int32_t *residual_tokens) {
+    if (!h) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+    if (quantized_tokens) *quantized_tokens = h->Tq;
+    if (residual_tokens) *residual_tokens = h->r;
+    return ok();
+}
+
+uint64_t kvq_kernel_launches(void) { return g_launches.load(); }
+
+const char *kvq_last_error(void) { return g_last_error.c_str(); }
+
+int32_t kvq_layout_version(void) { return 1; }
+
+}  // extern "C"

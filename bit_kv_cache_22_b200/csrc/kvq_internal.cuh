@@ -1,0 +1,75 @@
+// kvq_internal.cuh -- declarations shared by the libkvq translation units.
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace kvq {
+
+constexpr int kTile = 16;          // tokens per code tile (and channels per chunk)
+
+// Words of one 16-token tile of one (batch, kv-head) slice: 16*d*n/32.
+__host__ __device__ constexpr int tile_words(int d, int n) { return d * n / 2; }
+// Words owned by each of the 32 lanes inside a tile.
+__host__ __device__ constexpr int lane_words(int d, int n) { return d * n / 64; }
+
+// fp16 / bf16 bit pattern -> float (exact).
+__device__ __forceinline__ float widen(uint16_t h, bool bf16) {
+    if (bf16) return __uint_as_float(static_cast<uint32_t>(h) << 16);
+    __half_raw r;
+    r.x = h;
+    return __half2float(__half(r));
+}
+
+// Record n kernel launches (reported by kvq_kernel_launches()).
+void count_launches(int n);
+
+// ---------------------------------------------------------------------------
+// launch helpers (implemented in quantize.cu / decode.cu); all return the
+// cudaError_t of the launch.
+// ---------------------------------------------------------------------------
+
+struct QuantizeArgs {
+    const uint16_t *xk, *xv;     // e [BH][*][d]; slice stride in elements below
+    int64_t in_bh_stride;        // elements between consecutive (b,h) slices
+    int64_t in_tok0;             // first input token
+    int64_t n_groups;            // key groups to quantize per slice
+    int64_t BH;
+    int d, G, Gv, bits;
+    bool sym, bf16;
+    uint32_t *kc, *vc;           // packed codes, [BH][cap*d*n/32]
+    float *ks, *vs;              // [BH][cap/G][d], [BH][cap][d/Gv]
+    int16_t *kz, *vz;            // same shapes (unused when sym)
+    int64_t cap;                 // token capacity per slice
+    int64_t out_tok0;            // first output token (multiple of G)
+};
+cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s);
+
+// dst[bh][dst_row0 + i][:] = src[bh][src_row0 + i][:] for i < rows (e elements)
+cudaError_t launch_copy_rows(const uint16_t *src, int64_t src_bh_stride, int64_t src_row0,
+                             uint16_t *dst, int64_t dst_bh_stride, int64_t dst_row0,
+                             int64_t rows, int64_t BH, int d, cudaStream_t s);
+
+struct DecodeArgs {
+    const uint32_t *kc, *vc;
+    const float *ks, *vs;
+    const int16_t *kz, *vz;
+    const uint16_t *kr, *vr;     // residual [BH][R][d]
+    const uint16_t *q;           // [B][Hq][d]
+    float *o_part, *m_part, *l_part;   // [B*Hq][S][d], [B*Hq][S], [B*Hq][S]
+    float *out;                  // [B][Hq][d]
+    int64_t cap;
+    int B, Hq, Hkv, d, G, Gv, R, bits;
+    bool sym, bf16;
+    int n_qtiles;                // Tq / 16
+    int r;                       // residual rows
+    int tiles_per_split;
+    int S;
+    float qscale;                // log2(e) / sqrt(d)
+};
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+// CTAs of the split kernel that fit on one SM for this configuration.
+int decode_ctas_per_sm(const DecodeArgs &a);
+
+}  // namespace kvq

@@ -1,0 +1,274 @@
+// quantize.cu -- KIVI quantize + pack (prefill and residual flush), residual copies.
+//
+// One CTA quantizes one key group of G tokens of one (batch, kv-head) slice:
+//   keys   : per channel over the G tokens ("LLM系列：KVCache量化1 KIVI ...",
+//            section 1: Key per-channel), values: per token over Gv channels
+//            (Value per-token);
+//   params : asymmetric s = (max-min)/(2^n-1), z = round(-min/s),
+//            code = clamp(round(x/s) + z, 0, 2^n-1), or symmetric
+//            s = 2 max|x|/(2^n-1), u = clamp(round(x/s), -2^(n-1), 2^(n-1)-1) + 2^(n-1)
+//            ("Atom: Low-bit Quantization ...", section 核心公式 / 量化基础, c = 1).
+// Every fp32 operation that decides a code is a single IEEE round-to-nearest
+// operation (explicit __f*_rn intrinsics, rintf = half-to-even), so codes,
+// scales and zeros are bit-identical to a plain fp32 evaluation of the
+// formulas.  A constant group takes s = |min| (1 if min = 0), which
+// reconstructs it exactly.
+//
+// Packing writes the library's tile layout (see include/kvq.h): each output
+// word is assembled from the 16x16 tensor-core A-fragment table, so writes are
+// fully coalesced and each thread produces whole words.
+#include <cfloat>
+#include <cstdint>
+
+#include "kvq_internal.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int kQuantThreads = 256;
+
+struct GroupParams {
+    float s;
+    int z;
+};
+
+__device__ __forceinline__ GroupParams asym_params(float mn, float mx, int bits) {
+    const float L = static_cast<float>((1 << bits) - 1);
+    float s;
+    if (mx > mn)
+        s = __fdiv_rn(__fsub_rn(mx, mn), L);
+    else
+        s = (mn != 0.0f) ? fabsf(mn) : 1.0f;
+    const float zf = rintf(__fdiv_rn(-mn, s));
+    return {s, static_cast<int>(zf)};
+}
+
+__device__ __forceinline__ int asym_code(float x, GroupParams p, int bits) {
+    const int L = (1 << bits) - 1;
+    int q = static_cast<int>(rintf(__fdiv_rn(x, p.s))) + p.z;
+    return min(max(q, 0), L);
+}
+
+__device__ __forceinline__ float sym_scale(float amax, int bits) {
+    const float L = static_cast<float>((1 << bits) - 1);
+    return __fdiv_rn(__fmul_rn(2.0f, amax), L);
+}
+
+__device__ __forceinline__ int sym_code(float x, float s, int bits) {
+    const int half = 1 << (bits - 1);
+    if (s == 0.0f) return half;
+    int q = static_cast<int>(rintf(__fdiv_rn(x, s)));
+    q = min(max(q, -half), half - 1);
+    return q + half;
+}
+
+// Assemble the packed words of `ntiles` 16-token tiles from byte codes
+// codes[t * d + c] (t relative to the first tile) and store them at dst.
+__device__ void pack_tiles(const uint8_t *codes, int ntiles, int d, int bits, bool is_v,
+                           uint32_t *dst) {
+    const int TW = tile_words(d, bits);
+    const int W = lane_words(d, bits);
+    const int P = 16 / bits;
+    const int total = ntiles * TW;
+    for (int wi = threadIdx.x; wi < total; wi += blockDim.x) {
+        const int tile = wi / TW;
+        const int w = wi - tile * TW;
+        const int lane = w / W;
+        const int wl = w - lane * W;
+        uint32_t word = 0;
+        for (int pi = 0; pi < P; ++pi) {
+            const int pair = wl * P + pi;
+            const int j = pair >> 2, k = pair & 3;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                // fragment table: row = lane/4 + 8*(k%2), col = 2*(lane%4) + h + 8*(k/2)
+                const int row = (lane >> 2) + 8 * (k & 1);
+                const int col = 2 * (lane & 3) + h + 8 * (k >> 1);
+                const int t = tile * 16 + (is_v ? col : row);
+                const int c = 16 * j + (is_v ? row : col);
+                word |= static_cast<uint32_t>(codes[t * d + c]) << (16 * h + bits * pi);
+            }
+        }
+        dst[wi] = word;
+    }
+}
+
+// Copy G*d contiguous 16-bit elements into shared memory with 16-byte loads.
+__device__ void load_group(const uint16_t *src, uint16_t *dst, int n) {
+    const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+    for (int i = threadIdx.x; i < n / 8; i += blockDim.x) d4[i] = s4[i];
+}
+
+__global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const QuantizeArgs a) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int d = a.d, G = a.G, bits = a.bits;
+    uint16_t *xs = reinterpret_cast<uint16_t *>(smem);                       // [G][d]
+    uint8_t *codes = smem + static_cast<size_t>(G) * d * 2;                  // [G][d]
+    float *red = reinterpret_cast<float *>(codes + static_cast<size_t>(G) * d);  // 2*256
+    float *ch_s = red + 2 * kQuantThreads;                                   // [d]
+    int *ch_z = reinterpret_cast<int *>(ch_s + d);                           // [d]
+
+    const int64_t grp = blockIdx.x;
+    const int64_t bh = blockIdx.y;
+    const int64_t in_tok = a.in_tok0 + grp * G;
+    const int64_t out_tok = a.out_tok0 + grp * G;
+    const int TW = tile_words(d, bits);
+    const int64_t words_per_slice = a.cap / 16 * TW;
+    const int64_t groups_cap = a.cap / G;
+
+    // ------------------------------ keys ------------------------------
+    load_group(a.xk + bh * a.in_bh_stride + in_tok * d, xs, G * d);
+    __syncthreads();
+    {
+        const int parts = kQuantThreads / d;         // d divides 256
+        const int c = threadIdx.x % d;
+        const int part = threadIdx.x / d;
+        const int per = (G + parts - 1) / parts;
+        float mn = FLT_MAX, mx = -FLT_MAX;
+        for (int t = part * per; t < min(G, (part + 1) * per); ++t) {
+            const float x = widen(xs[t * d + c], a.bf16);
+            if (a.sym) {
+                mx = fmaxf(mx, fabsf(x));
+            } else {
+                mn = fminf(mn, x);
+                mx = fmaxf(mx, x);
+            }
+        }
+        red[threadIdx.x] = mn;
+        red[kQuantThreads + threadIdx.x] = mx;
+        __syncthreads();
+        if (threadIdx.x < d) {
+            for (int p = 1; p < parts; ++p) {
+                mn = fminf(mn, red[p * d + c]);
+                mx = fmaxf(mx, red[kQuantThreads + p * d + c]);
+            }
+            float s;
+            int z;
+            if (a.sym) {
+                s = sym_scale(mx, bits);
+                z = 1 << (bits - 1);
+            } else {
+                const GroupParams gp = asym_params(mn, mx, bits);
+                s = gp.s;
+                z = gp.z;
+                a.kz[(bh * groups_cap + out_tok / G) * d + c] = static_cast<int16_t>(z);
+            }
+            a.ks[(bh * groups_cap + out_tok / G) * d + c] = s;
+            ch_s[c] = s;
+            ch_z[c] = z;
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < G * d; e += blockDim.x) {
+            const int c2 = e % d;
+            const float x = widen(xs[e], a.bf16);
+            codes[e] = static_cast<uint8_t>(
+                a.sym ? sym_code(x, ch_s[c2], bits) : asym_code(x, {ch_s[c2], ch_z[c2]}, bits));
+        }
+        __syncthreads();
+        pack_tiles(codes, G / 16, d, bits, false,
+                   a.kc + bh * words_per_slice + (out_tok / 16) * TW);
+        __syncthreads();
+    }
+
+    // ------------------------------ values ----------------------------
+    load_group(a.xv + bh * a.in_bh_stride + in_tok * d, xs, G * d);
+    __syncthreads();
+    {
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        const int per_lane = d / 32;                 // contiguous channels per lane
+        const int seg = a.Gv / per_lane;             // lanes per value group (power of 2)
+        const int ngv = d / a.Gv;
+        for (int t = warp; t < G; t += kQuantThreads / 32) {
+            float x[8];
+            float mn = FLT_MAX, mx = -FLT_MAX;
+            for (int e = 0; e < per_lane; ++e) {
+                x[e] = widen(xs[t * d + lane * per_lane + e], a.bf16);
+                if (a.sym) {
+                    mx = fmaxf(mx, fabsf(x[e]));
+                } else {
+                    mn = fminf(mn, x[e]);
+                    mx = fmaxf(mx, x[e]);
+                }
+            }
+            for (int off = seg >> 1; off > 0; off >>= 1) {
+                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            }
+            float s;
+            int z;
+            if (a.sym) {
+                s = sym_scale(mx, bits);
+                z = 0;
+            } else {
+                const GroupParams gp = asym_params(mn, mx, bits);
+                s = gp.s;
+                z = gp.z;
+            }
+            const int j = lane / seg;
+            if (lane % seg == 0) {
+                const int64_t mi = (bh * a.cap + out_tok + t) * ngv + j;
+                a.vs[mi] = s;
+                if (!a.sym) a.vz[mi] = static_cast<int16_t>(z);
+            }
+            for (int e = 0; e < per_lane; ++e)
+                codes[t * d + lane * per_lane + e] = static_cast<uint8_t>(
+                    a.sym ? sym_code(x[e], s, bits) : asym_code(x[e], {s, z}, bits));
+        }
+        __syncthreads();
+        pack_tiles(codes, G / 16, d, bits, true,
+                   a.vc + bh * words_per_slice + (out_tok / 16) * TW);
+    }
+}
+
+__global__ void copy_rows_kernel(const uint16_t *src, int64_t src_bh_stride, int64_t src_row0,
+                                 uint16_t *dst, int64_t dst_bh_stride, int64_t dst_row0,
+                                 int64_t rows, int64_t BH, int d) {
+    const int64_t vec_per_row = d / 8;
+    const int64_t total = BH * rows * vec_per_row;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t v = i % vec_per_row;
+        const int64_t row = (i / vec_per_row) % rows;
+        const int64_t bh = i / (vec_per_row * rows);
+        const uint4 *s = reinterpret_cast<const uint4 *>(src + bh * src_bh_stride +
+                                                         (src_row0 + row) * d) + v;
+        uint4 *t = reinterpret_cast<uint4 *>(dst + bh * dst_bh_stride + (dst_row0 + row) * d) + v;
+        *t = *s;
+    }
+}
+
+}  // namespace
+
+size_t quantize_smem_bytes(int d, int G) {
+    return static_cast<size_t>(G) * d * 3 + 2 * kQuantThreads * sizeof(float) +
+           static_cast<size_t>(d) * 8;
+}
+
+cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s) {
+    if (a.n_groups == 0 || a.BH == 0) return cudaSuccess;
+    const size_t smem = quantize_smem_bytes(a.d, a.G);
+    cudaError_t e = cudaFuncSetAttribute(quantize_pack_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    dim3 grid(static_cast<unsigned>(a.n_groups), static_cast<unsigned>(a.BH));
+    quantize_pack_kernel<<<grid, kQuantThreads, smem, s>>>(a);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_copy_rows(const uint16_t *src, int64_t src_bh_stride, int64_t src_row0,
+                             uint16_t *dst, int64_t dst_bh_stride, int64_t dst_row0,
+                             int64_t rows, int64_t BH, int d, cudaStream_t s) {
+    const int64_t total = BH * rows * (d / 8);
+    if (total == 0) return cudaSuccess;
+    const int threads = 256;
+    const int64_t blocks = (total + threads - 1) / threads;
+    copy_rows_kernel<<<static_cast<unsigned>(blocks < 65536 ? blocks : 65536), threads, 0, s>>>(
+        src, src_bh_stride, src_row0, dst, dst_bh_stride, dst_row0, rows, BH, d);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace kvq

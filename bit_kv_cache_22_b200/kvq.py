@@ -1,0 +1,277 @@
+"""Python binding of libkvq (include/kvq.h): argument marshalling only.
+
+PyTorch provides device memory and the current CUDA stream; every step of
+the computation runs in the library's CUDA kernels.  If the library cannot
+be loaded this module raises -- there is no CPU or PyTorch fallback.
+
+Typical use, with the names of the operations on the KIVI page ("LLM系列：
+KVCache量化1 KIVI ...", section 1)::
+
+    cache = prefill_quantize(X_K, X_V, G=32, R=128, bits=2, q_heads=32)
+    append(cache, t_K, t_V)
+    t_O = decode_attention(cache, t_Q)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import build as _build
+
+_lock = threading.Lock()
+_lib = None
+
+KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_STATE, KVQ_ERR_CUDA = range(6)
+KVQ_FP16, KVQ_BF16 = 0, 1
+
+EXPORTED = ("kvq_get_sizes", "kvq_create", "kvq_destroy", "kvq_reset", "kvq_prefill_quantize",
+            "kvq_append", "kvq_decode_attention", "kvq_cache_state", "kvq_set_split_limit",
+            "kvq_decode_splits", "kvq_kernel_launches",
+            "kvq_last_error", "kvq_layout_version")
+
+
+class KVQError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"kvq status {status}: {message}")
+        self.status = status
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("q_heads", ctypes.c_int32),
+                ("kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("group_k", ctypes.c_int32), ("group_v", ctypes.c_int32),
+                ("residual", ctypes.c_int32), ("bits", ctypes.c_int32),
+                ("symmetric", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("capacity", ctypes.c_int64)]
+
+
+class Sizes(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in
+                ("k_codes", "k_scales", "k_zeros", "v_codes", "v_scales", "v_zeros",
+                 "k_residual", "v_residual", "workspace")]
+
+
+class Buffers(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("k_codes", "k_scales", "k_zeros", "v_codes", "v_scales", "v_zeros",
+                 "k_residual", "v_residual")]
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def load() -> ctypes.CDLL:
+    """Load libkvq.so (building it in-tree first if it is missing or stale)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = _build.build()
+        if not os.path.exists(path):
+            raise ImportError(f"libkvq.so not found at {path}")
+        lib = ctypes.CDLL(path)
+        P, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+        lib.kvq_get_sizes.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(Sizes)]
+        lib.kvq_create.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(Buffers),
+                                   ctypes.POINTER(P)]
+        lib.kvq_destroy.argtypes = [P]
+        lib.kvq_destroy.restype = None
+        lib.kvq_reset.argtypes = [P]
+        lib.kvq_prefill_quantize.argtypes = [P, P, P, i64, P]
+        lib.kvq_append.argtypes = [P, P, P, P]
+        lib.kvq_decode_attention.argtypes = [P, P, P, P, sz, P]
+        lib.kvq_cache_state.argtypes = [P, ctypes.POINTER(i64), ctypes.POINTER(i32)]
+        lib.kvq_set_split_limit.argtypes = [P, i32]
+        lib.kvq_decode_splits.argtypes = [P]
+        lib.kvq_decode_splits.restype = i32
+        lib.kvq_kernel_launches.argtypes = []
+        lib.kvq_kernel_launches.restype = ctypes.c_uint64
+        lib.kvq_last_error.argtypes = []
+        lib.kvq_last_error.restype = ctypes.c_char_p
+        lib.kvq_layout_version.argtypes = []
+        lib.kvq_layout_version.restype = i32
+        for name in ("kvq_get_sizes", "kvq_create", "kvq_reset", "kvq_prefill_quantize",
+                     "kvq_append", "kvq_decode_attention", "kvq_cache_state", "kvq_set_split_limit"):
+            getattr(lib, name).restype = ctypes.c_int
+        _lib = lib
+        return lib
+
+
+def _check(status: int):
+    if status != KVQ_OK:
+        msg = load().kvq_last_error().decode(errors="replace")
+        raise KVQError(status, msg)
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float16:
+        return KVQ_FP16
+    if dt == torch.bfloat16:
+        return KVQ_BF16
+    raise TypeError(f"element type must be float16 or bfloat16, got {dt}")
+
+
+def make_config(batch, q_heads, kv_heads, head_dim, group_k, group_v, residual, bits,
+                symmetric, dtype, capacity) -> Config:
+    return Config(batch, q_heads, kv_heads, head_dim, group_k, group_v, residual, bits,
+                  int(bool(symmetric)), dtype if isinstance(dtype, int) else _dtype_code(dtype),
+                  capacity)
+
+
+def get_sizes(cfg: Config) -> Sizes:
+    s = Sizes()
+    _check(load().kvq_get_sizes(ctypes.byref(cfg), ctypes.byref(s)))
+    return s
+
+
+def _stream_ptr(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+class KVQCache:
+    """A quantized KV cache whose device buffers are torch tensors.
+
+    Shapes (e = fp16 or bf16): prompt X_K, X_V [B, Hkv, T, d]; new token
+    t_K, t_V [B, Hkv, d]; query t_Q [B, Hq, d]; output t_O float32 [B, Hq, d].
+    Inputs on the host are copied to the device first (plumbing only).
+    """
+
+    def __init__(self, batch, q_heads, kv_heads, head_dim, group_k, group_v, residual, bits,
+                 symmetric=False, dtype=torch.bfloat16, capacity=None, device=None):
+        if capacity is None:
+            raise ValueError("capacity (quantized tokens per sequence) is required")
+        capacity = -(-capacity // residual) * residual
+        dev = torch.device(device if device is not None else "cuda")
+        if dev.type != "cuda":
+            raise ValueError("the cache lives on a CUDA device")
+        self.device = dev if dev.index is not None else torch.device("cuda", torch.cuda.current_device())
+        self.dtype = dtype
+        self.cfg = make_config(batch, q_heads, kv_heads, head_dim, group_k, group_v, residual,
+                               bits, symmetric, dtype, capacity)
+        self.sizes = get_sizes(self.cfg)
+        BH = batch * kv_heads
+        dev = self.device
+        words = capacity * head_dim * bits // 32
+        self.k_codes = torch.empty((BH, words), dtype=torch.int32, device=dev)
+        self.v_codes = torch.empty((BH, words), dtype=torch.int32, device=dev)
+        self.k_scales = torch.empty((BH, capacity // group_k, head_dim), dtype=torch.float32, device=dev)
+        self.v_scales = torch.empty((BH, capacity, head_dim // group_v), dtype=torch.float32, device=dev)
+        if symmetric:
+            self.k_zeros = self.v_zeros = None
+        else:
+            self.k_zeros = torch.empty((BH, capacity // group_k, head_dim), dtype=torch.int16, device=dev)
+            self.v_zeros = torch.empty((BH, capacity, head_dim // group_v), dtype=torch.int16, device=dev)
+        self.k_residual = torch.zeros((BH, residual, head_dim), dtype=dtype, device=dev)
+        self.v_residual = torch.zeros((BH, residual, head_dim), dtype=dtype, device=dev)
+        self.workspace = torch.empty(self.sizes.workspace // 4, dtype=torch.float32, device=dev)
+        bufs = Buffers(self.k_codes.data_ptr(), self.k_scales.data_ptr(),
+                       self.k_zeros.data_ptr() if self.k_zeros is not None else None,
+                       self.v_codes.data_ptr(), self.v_scales.data_ptr(),
+                       self.v_zeros.data_ptr() if self.v_zeros is not None else None,
+                       self.k_residual.data_ptr(), self.v_residual.data_ptr())
+        self._lib = load()
+        h = ctypes.c_void_p()
+        with torch.cuda.device(dev):
+            _check(self._lib.kvq_create(ctypes.byref(self.cfg), ctypes.byref(bufs), ctypes.byref(h)))
+        self._h = h
+
+    # ------------------------------------------------------------------
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            self._lib.kvq_destroy(h)
+            self._h = None
+
+    def _dev(self, t: torch.Tensor) -> torch.Tensor:
+        if t.dtype != self.dtype:
+            raise TypeError(f"expected {self.dtype}, got {t.dtype}")
+        if t.device != self.device:
+            t = t.to(self.device, non_blocking=True)
+        return t.contiguous()
+
+    def state(self):
+        tq = ctypes.c_int64()
+        r = ctypes.c_int32()
+        _check(self._lib.kvq_cache_state(self._h, ctypes.byref(tq), ctypes.byref(r)))
+        return int(tq.value), int(r.value)
+
+    def set_split_limit(self, max_splits: int):
+        _check(self._lib.kvq_set_split_limit(self._h, max_splits))
+
+    def splits(self) -> int:
+        return int(self._lib.kvq_decode_splits(self._h))
+
+    def reset(self):
+        _check(self._lib.kvq_reset(self._h))
+
+    def prefill_quantize(self, X_K: torch.Tensor, X_V: torch.Tensor, stream=None):
+        X_K, X_V = self._dev(X_K), self._dev(X_V)
+        c = self.cfg
+        if X_K.shape != X_V.shape or X_K.dim() != 4 or X_K.shape[0] != c.batch or \
+                X_K.shape[1] != c.kv_heads or X_K.shape[3] != c.head_dim:
+            raise ValueError(f"X_K/X_V must be [B={c.batch}, Hkv={c.kv_heads}, T, d={c.head_dim}]")
+        _check(self._lib.kvq_prefill_quantize(self._h, X_K.data_ptr(), X_V.data_ptr(),
+                                              X_K.shape[2], _stream_ptr(stream)))
+        self._keep = (X_K, X_V)
+        return self
+
+    def append(self, t_K: torch.Tensor, t_V: torch.Tensor, stream=None):
+        t_K, t_V = self._dev(t_K), self._dev(t_V)
+        c = self.cfg
+        want = (c.batch, c.kv_heads, c.head_dim)
+        if tuple(t_K.shape) != want or tuple(t_V.shape) != want:
+            raise ValueError(f"t_K/t_V must be {list(want)}")
+        _check(self._lib.kvq_append(self._h, t_K.data_ptr(), t_V.data_ptr(), _stream_ptr(stream)))
+        self._keep = (t_K, t_V)
+        return self
+
+    def decode_attention(self, t_Q: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+        t_Q = self._dev(t_Q)
+        c = self.cfg
+        if tuple(t_Q.shape) != (c.batch, c.q_heads, c.head_dim):
+            raise ValueError(f"t_Q must be [{c.batch}, {c.q_heads}, {c.head_dim}]")
+        host_out = out is not None and not out.is_cuda
+        dev_out = torch.empty((c.batch, c.q_heads, c.head_dim), dtype=torch.float32,
+                              device=self.device) if (out is None or host_out) else out
+        _check(self._lib.kvq_decode_attention(self._h, t_Q.data_ptr(), dev_out.data_ptr(),
+                                              self.workspace.data_ptr(),
+                                              self.workspace.numel() * 4, _stream_ptr(stream)))
+        if host_out:
+            out.copy_(dev_out, non_blocking=True)
+            return out
+        return dev_out
+
+
+# ----------------------------------------------------------------------------
+# function-style API with the operation names of the method
+# ----------------------------------------------------------------------------
+
+def prefill_quantize(X_K: torch.Tensor, X_V: torch.Tensor, G: int, R: int, bits: int, *,
+                     q_heads: int | None = None, group_v: int | None = None,
+                     symmetric: bool = False, capacity: int | None = None,
+                     device=None) -> KVQCache:
+    """Create a cache sized for the prompt (plus `capacity`) and quantize X_K, X_V [B, Hkv, T, d]."""
+    B, Hkv, T, d = X_K.shape
+    cap = capacity if capacity is not None else max(T, 1) + R
+    dev = device if device is not None else (X_K.device if X_K.is_cuda else "cuda")
+    gv = group_v if group_v is not None else min(G, d)
+    cache = KVQCache(B, q_heads or Hkv, Hkv, d, G, gv, R, bits, symmetric, X_K.dtype, cap, dev)
+    return cache.prefill_quantize(X_K, X_V)
+
+
+def append(cache: KVQCache, t_K: torch.Tensor, t_V: torch.Tensor) -> KVQCache:
+    return cache.append(t_K, t_V)
+
+
+def decode_attention(cache: KVQCache, t_Q: torch.Tensor, out=None) -> torch.Tensor:
+    return cache.decode_attention(t_Q, out)
+
+
+def kernel_launches() -> int:
+    """Kernels libkvq has launched in this process so far."""
+    return int(load().kvq_kernel_launches())

@@ -1,0 +1,194 @@
+/*
+ * kvq.h -- C ABI of libkvq: decode-phase attention over a KIVI-style low-bit
+ * quantized KV cache on NVIDIA B200 (sm_100a).
+ *
+ * What is computed (web pages the operations follow):
+ *  - "LLM系列：KVCache量化1 KIVI: A Tuning-Free Asymmetric 2bit Quantization
+ *    for KV Cache", section 1: keys are quantized per channel in groups of G
+ *    tokens, values per token; the newest tokens stay in a full-precision
+ *    residual X_Kr that is quantized and appended when it holds R tokens;
+ *    A = Concat(A_g, A_r), t_O = A X_V.
+ *  - "Atom: Low-bit Quantization for Efficient and Accurate LLM Serving",
+ *    section 核心公式 / 量化基础: asymmetric s = (max-min)/(2^n-1),
+ *    z = round(-min/s), code = clamp(round(x/s) + z, 0, 2^n-1); symmetric
+ *    s = 2 max|x| / (2^n-1), code = clamp(round(x/s), -2^(n-1), 2^(n-1)-1).
+ *  - "KV Cache的Int4量化…", section 2 (x' = (q - z) s) and section 3
+ *    (softmax(Q K^T / sqrt(d_k)) V).
+ * Rounding is half-to-even in IEEE fp32; a constant group uses s = |min|
+ * (1 when min = 0) so that it reconstructs exactly; the symmetric variant
+ * stores u = q + 2^(n-1) and has no zero-point tensors.
+ *
+ * Conventions for every call:
+ *  - Device memory (cache buffers, inputs, outputs, workspace) is owned and
+ *    allocated by the caller.  The library allocates no device memory; it
+ *    only keeps a small host-side handle with the cache geometry and the
+ *    two counters Tq (quantized tokens) and r (residual tokens).
+ *  - Work is enqueued asynchronously on the caller's CUDA stream (`stream`
+ *    is a cudaStream_t, NULL for the legacy default stream).  Host counters
+ *    advance when a call is enqueued, so a sequence of calls needs no
+ *    device-to-host synchronisation.
+ *  - A call that returns an error has launched nothing and changed no state;
+ *    kvq_last_error() then describes the cause (thread-local string).
+ *  - Device pointers must be 16-byte aligned; tensors are dense and
+ *    row-major in the shapes given below.  Element type `e` is fp16 or bf16
+ *    (kvq_config.dtype) and is passed as raw 16-bit patterns.
+ *  - Query head i reads kv head i / (Hq / Hkv).
+ *  - No C++ exception crosses this interface.
+ *
+ * Storage format of the cache (this library's own; the pages fix none):
+ *  - k_codes, v_codes: uint32 [B][Hkv][capacity * d * n / 32].  Tokens are cut
+ *    into tiles of 16 and channels into chunks of 16.  A tile occupies
+ *    d*n/2 consecutive words; inside it 32 lanes own W = d*n/64 words each.
+ *    In chunk j, a 16x16 block indexed (row, col) -- keys (token%16,
+ *    channel%16), values (channel%16, token%16) -- places element (row, col)
+ *    in lane 4*(row%8) + (col%8)/2, half col%2, register k = row/8 +
+ *    2*(col/8): the A-operand fragment of a 16x16x16 tensor-core MMA.  Pair
+ *    p = 4*j + k lives in word p/(16/n) of the lane at bit
+ *    16*half + n*(p % (16/n)).
+ *  - k_scales float / k_zeros int16: [B][Hkv][capacity/G][d]   (group, channel)
+ *  - v_scales float / v_zeros int16: [B][Hkv][capacity][d/Gv]  (token, group)
+ *  - k_residual, v_residual: e [B][Hkv][R][d]  (rows 0..r-1 valid)
+ *  Symmetric caches have no zero tensors (pass NULL).
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KVQ_OK = 0,
+    KVQ_ERR_INVALID_ARG = 1,   /* bad pointer, alignment, shape or parameter   */
+    KVQ_ERR_UNSUPPORTED = 2,   /* valid but not built (e.g. head_dim 96)        */
+    KVQ_ERR_CAPACITY = 3,      /* the call would exceed the token capacity      */
+    KVQ_ERR_STATE = 4,         /* call out of order (prefill twice, empty cache) */
+    KVQ_ERR_CUDA = 5           /* a CUDA runtime call or launch failed          */
+} kvq_status;
+
+typedef enum { KVQ_FP16 = 0, KVQ_BF16 = 1 } kvq_dtype;
+
+/* Cache geometry and quantiser settings. */
+typedef struct {
+    int32_t batch;       /* B                                                   */
+    int32_t q_heads;     /* Hq                                                  */
+    int32_t kv_heads;    /* Hkv, divides Hq                                     */
+    int32_t head_dim;    /* d: 64 or 128                                        */
+    int32_t group_k;     /* G: tokens per key group, multiple of 16, <= 256,
+                            G * d <= 32768                                      */
+    int32_t group_v;     /* Gv: channels per value group: 16, 32, 64 or 128, <= d */
+    int32_t residual;    /* R: residual capacity, multiple of G                 */
+    int32_t bits;        /* n: 2 or 4                                           */
+    int32_t symmetric;   /* 0 asymmetric min-max, 1 symmetric (offset codes)    */
+    int32_t dtype;       /* kvq_dtype of every e tensor                         */
+    int64_t capacity;    /* quantized-token capacity per sequence, multiple of R */
+} kvq_config;
+
+/* Byte sizes of the caller-allocated device buffers. */
+typedef struct {
+    size_t k_codes, k_scales, k_zeros;
+    size_t v_codes, v_scales, v_zeros;
+    size_t k_residual, v_residual;
+    size_t workspace;    /* scratch needed by kvq_decode_attention              */
+} kvq_sizes;
+
+/* Caller-owned device buffers of one cache (layout above). */
+typedef struct {
+    void *k_codes;
+    float *k_scales;
+    int16_t *k_zeros;    /* NULL when symmetric                                 */
+    void *v_codes;
+    float *v_scales;
+    int16_t *v_zeros;    /* NULL when symmetric                                 */
+    void *k_residual;
+    void *v_residual;
+} kvq_buffers;
+
+typedef struct kvq_cache kvq_cache;   /* opaque host-side handle */
+
+/* Validates `cfg` and fills `out` with the buffer sizes.  No device needed. */
+KVQ_API kvq_status kvq_get_sizes(const kvq_config *cfg, kvq_sizes *out);
+
+/*
+ * Creates a handle over caller-owned buffers (not copied, not freed).  The
+ * cache starts empty (Tq = 0, r = 0).  Reads device properties of the current
+ * device; all later calls must run with that device current.
+ */
+KVQ_API kvq_status kvq_create(const kvq_config *cfg, const kvq_buffers *bufs, kvq_cache **out);
+
+/* Frees the host handle only.  NULL is ignored. */
+KVQ_API void kvq_destroy(kvq_cache *cache);
+
+/* Empties the cache (Tq = r = 0) without touching device memory. */
+KVQ_API kvq_status kvq_reset(kvq_cache *cache);
+
+/*
+ * Prefill (KIVI section 1, prefill phase): X_K, X_V are e [B][Hkv][T][d]
+ * device tensors of the prompt's keys and values.  The first
+ * Tq = floor(T/R)*R tokens are quantized (keys per channel over G tokens,
+ * values per token over Gv channels) and packed; the remaining T - Tq
+ * tokens are copied into the residual.  Only allowed on an empty cache
+ * (KVQ_ERR_STATE otherwise); Tq > capacity gives KVQ_ERR_CAPACITY.
+ * T = 0 is accepted and does nothing.
+ */
+KVQ_API kvq_status kvq_prefill_quantize(kvq_cache *cache, const void *X_K, const void *X_V,
+                                int64_t T, void *stream);
+
+/*
+ * Decode-phase append (KIVI section 1): t_K, t_V are e [B][Hkv][d] device
+ * tensors of one new token per sequence.  They are written to residual row
+ * r and r is incremented; when r reaches R the R residual rows are quantized
+ * into tokens [Tq, Tq+R) of the quantized cache, Tq += R and r = 0.  A flush
+ * that would exceed the capacity gives KVQ_ERR_CAPACITY (nothing written).
+ */
+KVQ_API kvq_status kvq_append(kvq_cache *cache, const void *t_K, const void *t_V, void *stream);
+
+/*
+ * Decode attention (KIVI section 1: A = Concat(A_g, A_r), t_O = A X_V with
+ * the 1/sqrt(d) scaling): t_Q is e [B][Hq][d]; t_O receives float
+ * [B][Hq][d] = softmax(t_Q [deq(K_g); K_r]^T / sqrt(d)) [deq(V_g); V_r].
+ * `workspace` is device scratch of at least kvq_sizes.workspace bytes
+ * (holds per-split partial results; contents on entry are ignored).
+ * An empty cache gives KVQ_ERR_STATE.
+ */
+KVQ_API kvq_status kvq_decode_attention(kvq_cache *cache, const void *t_Q, float *t_O,
+                                void *workspace, size_t workspace_bytes, void *stream);
+
+/* Current counters: quantized tokens Tq and residual tokens r. */
+KVQ_API kvq_status kvq_cache_state(const kvq_cache *cache, int64_t *quantized_tokens,
+                           int32_t *residual_tokens);
+
+/*
+ * Upper bound on the token splits of kvq_decode_attention (1 .. 64; 0 restores
+ * the default of 64).  Fewer splits mean fewer partial results to merge, more
+ * splits more parallelism for short batches; the result is the same up to
+ * fp32 rounding.
+ */
+KVQ_API kvq_status kvq_set_split_limit(kvq_cache *cache, int32_t max_splits);
+
+/* Number of token splits the next kvq_decode_attention would use (>= 1). */
+KVQ_API int32_t kvq_decode_splits(const kvq_cache *cache);
+
+/* Kernels this library has launched in the process so far (all devices). */
+KVQ_API uint64_t kvq_kernel_launches(void);
+
+/* Description of the last error on the calling thread ("" if none). */
+KVQ_API const char *kvq_last_error(void);
+
+/* Version of the storage format described above (currently 1). */
+KVQ_API int32_t kvq_layout_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

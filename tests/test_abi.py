@@ -1,0 +1,101 @@
+"""The C ABI without a GPU: the library loads, exports what include/kvq.h declares,
+and validates configurations on the host."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from bit_kv_cache_22_b200 import kvq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kvq.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"KVQ_API\s+[\w\s\*]+?\b(kvq_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_three_operations():
+    names = declared_symbols()
+    for op in ("kvq_prefill_quantize", "kvq_append", "kvq_decode_attention"):
+        assert op in names
+    assert set(names) == set(kvq.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = kvq.load()
+    out = subprocess.run(["nm", "-D", "--defined-only", kvq.library_path()],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (kvq_\w+)", out))
+    for name in declared_symbols():
+        assert name in exported, name
+        assert hasattr(lib, name)
+    # nothing else with the public prefix leaks out
+    assert exported == set(declared_symbols())
+
+
+def test_library_is_sm100a_only():
+    out = subprocess.run(["/usr/local/cuda/bin/cuobjdump", "--list-elf", kvq.library_path()],
+                         capture_output=True, text=True)
+    if out.returncode != 0:
+        pytest.skip("cuobjdump unavailable")
+    arches = set(re.findall(r"sm_(\d+a?)", out.stdout))
+    assert arches == {"100a"}
+
+
+def _cfg(**kw):
+    base = dict(batch=1, q_heads=4, kv_heads=2, head_dim=128, group_k=32, group_v=32,
+                residual=128, bits=2, symmetric=0, dtype=kvq.KVQ_BF16, capacity=1024)
+    base.update(kw)
+    return kvq.Config(**base)
+
+
+def test_sizes_match_layout():
+    s = kvq.get_sizes(_cfg())
+    BH, cap, d = 2, 1024, 128
+    assert s.k_codes == s.v_codes == BH * cap * d * 2 // 8
+    assert s.k_scales == BH * (cap // 32) * d * 4 and s.k_zeros == BH * (cap // 32) * d * 2
+    assert s.v_scales == BH * cap * (d // 32) * 4 and s.v_zeros == BH * cap * (d // 32) * 2
+    assert s.k_residual == s.v_residual == BH * 128 * d * 2
+    assert s.workspace > 0
+    sym = kvq.get_sizes(_cfg(symmetric=1, bits=4))
+    assert sym.k_zeros == 0 and sym.v_zeros == 0
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(head_dim=96), kvq.KVQ_ERR_UNSUPPORTED),
+    (dict(bits=3), kvq.KVQ_ERR_UNSUPPORTED),
+    (dict(q_heads=3), kvq.KVQ_ERR_INVALID_ARG),
+    (dict(group_k=24), kvq.KVQ_ERR_INVALID_ARG),
+    (dict(group_v=48), kvq.KVQ_ERR_INVALID_ARG),
+    (dict(residual=48), kvq.KVQ_ERR_INVALID_ARG),
+    (dict(capacity=1000), kvq.KVQ_ERR_INVALID_ARG),
+    (dict(dtype=7), kvq.KVQ_ERR_INVALID_ARG),
+    (dict(batch=0), kvq.KVQ_ERR_INVALID_ARG),
+    (dict(group_v=256, head_dim=128), kvq.KVQ_ERR_INVALID_ARG),
+])
+def test_invalid_configs_are_rejected(bad, status):
+    with pytest.raises(kvq.KVQError) as ei:
+        kvq.get_sizes(_cfg(**bad))
+    assert ei.value.status == status
+    assert kvq.load().kvq_last_error()
+
+
+def test_null_arguments_are_rejected_without_a_device():
+    lib = kvq.load()
+    assert lib.kvq_get_sizes(None, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_prefill_quantize(None, None, None, 0, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_append(None, None, None, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_decode_attention(None, None, None, None, 0, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_decode_splits(None) == 0
+    lib.kvq_destroy(None)
+    h = ctypes.c_void_p()
+    cfg = _cfg()
+    bufs = kvq.Buffers()
+    assert lib.kvq_create(ctypes.byref(cfg), ctypes.byref(bufs), ctypes.byref(h)) == \
+        kvq.KVQ_ERR_INVALID_ARG
+    assert not h.value
+    assert lib.kvq_layout_version() == 1
