@@ -214,10 +214,10 @@ def run_kvq(args):
         for s in range(w.steps):
             cache.append(tK[s], tV[s])
             if ev is not None:
-                ev[s][0].record(stream)
+                ev[s][0].record()
             cache.decode_attention(tQ[s], out=out)
             if ev is not None:
-                ev[s][1].record(stream)
+                ev[s][1].record()
 
     def barrier():
         if world > 1:
@@ -226,22 +226,33 @@ def run_kvq(args):
     for _ in range(args.warmup):
         episode()
     torch.cuda.synchronize()
-    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(w.steps)] for _ in range(args.steps)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # One episode is captured once as a CUDA graph (with timing events around
+    # every decode_attention call) and replayed: the host-side launch cost of
+    # ~640 small kernels per episode would otherwise starve the GPU.
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(w.steps)]
     launches0 = kvq.kernel_launches()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        episode(evs)
+    launches_per_episode = kvq.kernel_launches() - launches0
+    graph.replay()
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
+    decode_ms = 0.0
     with ClockSampler(local) as clk:
         start.record(stream)
         for k in range(args.steps):
-            episode(evs[k])
+            graph.replay()
         stop.record(stream)
         torch.cuda.synchronize()
         barrier()
-    launches = kvq.kernel_launches() - launches0
+    launches = launches_per_episode * args.steps
     ms = start.elapsed_time(stop)
-    decode_ms = sum(a.elapsed_time(b) for ev in evs for a, b in ev)
+    # decode_attention durations of the last replay (the events are graph nodes)
+    decode_ms = sum(a.elapsed_time(b) for a, b in evs) * args.steps
     t = torch.tensor([ms, decode_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -263,11 +274,16 @@ def run_kvq(args):
         for _ in range(max(1, args.warmup)):
             e2e_episode()
         torch.cuda.synchronize()
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2):
+            e2e_episode()
+        g2.replay()
+        torch.cuda.synchronize()
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(args.steps):
-            e2e_episode()
+            g2.replay()
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()

@@ -1,4 +1,4 @@
-// decode.cu -- split-K decode attention over the packed low-bit cache.
+// decode.cu -- split-K decode attention over the packed low-bit cache (CUDA cores).
 //
 // Computes, for every (batch, query head), one decode step of
 //   A = softmax(q [deq(K_g); K_r]^T / sqrt(d)),   t_O = A [deq(V_g); V_r]
@@ -7,23 +7,30 @@
 //
 // Split-K (flash-decoding): the token axis -- quantized 16-token tiles followed
 // by the residual rows, cut into 16-row tiles -- is divided into S contiguous
-// splits; a CTA owns one (batch, query head, split) and its four warps take the
-// split's tiles round-robin.  Token order does not change the result
+// splits; a CTA owns one (batch, query head, split) and each of its four warps a
+// contiguous share of the split's tiles, streamed through a per-warp cp.async
+// ring of shared-memory stages.  Token order does not change the result
 // (A . V = A_P . V_P, "Resumo Técnico: LogQuant", section 4), which is what
 // allows the splits and the residual to be folded into one online-softmax pass.
 // Each CTA writes an unnormalised partial (o, m, l); combine_kernel merges the
 // S partials with a log-sum-exp reduction.
 //
-// Inner loop, per lane and tile (lane = 4*r8 + l4 owns the A-fragment slots of
-// the packed layout):
-//   keys   : logit_t = sum_c q_c s_{g,c} (code - z_{g,c}) / sqrt(d)
-//            = sum_c M_c code_{t,c} - bias_g, with M_c = q_c s_{g,c} log2(e)/sqrt(d)
-//            refreshed once per key group and bias_g = sum_c M_c z_{g,c};
-//   values : o_c += sum_t p_t s_{t,gv} code_{t,c} - sum_t p_t s_{t,gv} z_{t,gv}.
-// Codes are turned into floats with the exponent trick: (word & mask) | 0x4B000000
-// is the float 2^23 + code * 2^pos exactly; one packed fp32x2 add removes 2^23
-// and one packed fp32x2 FMA accumulates two codes, the 2^pos factors being
-// folded into the multipliers (exact powers of two).
+// Lane = 4*g8 + t4.  In a tile it holds, per 16-channel chunk j, the codes of
+// rows g8 and g8+8 at columns 4*t4 .. 4*t4+3 (keys: rows = tokens, columns =
+// channels; values: rows = channels, columns = tokens); (word >> n*slot) with
+// the low n bits of each byte kept is four such codes, one per byte.
+//   keys   : logit_t = sum_c q_c s_{g,c} (code - z_{g,c}) log2(e)/sqrt(d)
+//            = 2^-e sum_c Q_c code_{t,c} - bias_g.  Once per key group the
+//            multipliers q_c s_{g,c} log2(e)/sqrt(d) are rounded to 22-bit fixed
+//            point Q_c = round(2^e q'_c) (e from the group's largest |q'|), split
+//            into three byte digits, and the integer dot products run as
+//            byte dot products (dp4a) with exact int32 accumulation;
+//            bias_g = sum_c q'_c z_{g,c} in fp32.
+//   values : o_c += sum_t p_t s_{t,gv} code_{t,c} - sum_t p_t s_{t,gv} z_{t,gv} in fp32:
+//            (word & mask) | 0x4B000000 is the float 2^23 + code * 2^pos exactly
+//            (one lop3); a packed fp32x2 add removes 2^23 and a packed fp32x2
+//            FMA accumulates two codes, the 2^pos factors folded into the
+//            multipliers and accumulators (exact powers of two).
 #include <cfloat>
 #include <cmath>
 #include <cstdint>
@@ -65,133 +72,265 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
     return upk(d);
 }
 
-// Load the W words a lane owns in one tile with the widest aligned loads.
+// (a & b) | c in one lop3.
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+    return r;
+}
+
+// byte dot products with int32 accumulation: bytes of a unsigned, of b unsigned / signed
+__device__ __forceinline__ int dp4a_uu(uint32_t a, uint32_t b, int c) {
+    int d;
+    asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+    int d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// 2^x (ex2.approx.ftz: relative error ~2^-22, 2^-inf = 0)
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Exact int -> float for |x| < 2^22: 1.5 * 2^23 + x as a bit pattern, minus 1.5 * 2^23.
+__device__ __forceinline__ float small_int_to_float(int x) {
+    return __int_as_float(0x4B400000 + x) - 12582912.0f;
+}
+// round(x) for |x| < 2^22, exactly (round half to even), without the XU pipe
+__device__ __forceinline__ int round_small(float x) {
+    return __float_as_int(x + 12582912.0f) - 0x4B400000;
+}
+
+// The lane's W words of one stage array (chunk-major, see Stage).
 template <int W>
-__device__ __forceinline__ void load_lane_words(const uint32_t *p, uint32_t (&w)[W]) {
+__device__ __forceinline__ void load_stage_words(const uint32_t *base, int lane, uint32_t (&w)[W]) {
     if constexpr (W % 4 == 0) {
 #pragma unroll
         for (int i = 0; i < W / 4; ++i) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p) + i);
+            const uint4 v = reinterpret_cast<const uint4 *>(base)[32 * i + lane];
             w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
         }
-    } else if constexpr (W % 2 == 0) {
-#pragma unroll
-        for (int i = 0; i < W / 2; ++i) {
-            const uint2 v = __ldg(reinterpret_cast<const uint2 *>(p) + i);
-            w[2 * i] = v.x; w[2 * i + 1] = v.y;
-        }
     } else {
-#pragma unroll
-        for (int i = 0; i < W; ++i) w[i] = __ldg(p + i);
+        const uint2 v = reinterpret_cast<const uint2 *>(base)[lane];
+        w[0] = v.x; w[1] = v.y;
     }
 }
 
-// Code pair (half 0 from the low 16 bits, half 1 from the high) at slot pi,
-// as floats code * 2^(N*pi).
-template <int N>
-__device__ __forceinline__ float2 code_pair(uint32_t lo, uint32_t hi, int pi) {
-    const uint32_t msk = ((1u << N) - 1u) << (N * pi);
-    float2 v = make_float2(__uint_as_float((lo & msk) | kMagicBits),
-                           __uint_as_float((hi & msk) | kMagicBits));
-    return add2(v, make_float2(-kMagic, -kMagic));
+// cp.async (global -> shared, bypassing L1) and its group bookkeeping.
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+    const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem));
 }
+__device__ __forceinline__ void cp_async8(void *smem, const void *gmem) {
+    const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(s), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
+template <int PENDING>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(PENDING));
+}
+
+// Shared-memory stage of one 16-token tile, owned by one warp:
+//   [K codes][V codes], each as (W/4 chunks) x (32 lanes) x 16 bytes, chunk-major so
+//   that a warp's 16-byte loads of one chunk hit 32 consecutive 16-byte slots
+//   (W = 2: 32 lanes x 8 bytes)
+//   [value scales 16 x NGV f32][value zeros 16 x NGV i16]
+//   [key scales D f32][key zeros D i16]   (filled only when the tile opens a key group)
+template <int N, int D, int GV>
+struct Stage {
+    static constexpr int W = D * N / 64;
+    static constexpr int NGV = D / GV;
+    static constexpr int kCodes = 32 * W * 4;          // bytes of one code array
+    static constexpr int kVs = 2 * kCodes;
+    static constexpr int kVz = kVs + 16 * NGV * 4;
+    static constexpr int kKs = kVz + 16 * NGV * 2;
+    static constexpr int kKz = kKs + D * 4;
+    static constexpr int kBytes = kKz + D * 2;
+    static_assert(kVz % 16 == 0 && kKs % 16 == 0 && kKz % 16 == 0 && kBytes % 16 == 0, "align");
+};
+
+constexpr int kStages = 4;
 
 template <int N, int D, int GV>
 __global__ void __launch_bounds__(kDecodeThreads, 4) decode_split_kernel(const DecodeArgs a) {
-    constexpr int P = 16 / N;         // code pairs per word
     constexpr int W = D * N / 64;     // words per lane per tile
     constexpr int TW = D * N / 2;     // words per tile
     constexpr int NJ = D / 16;        // 16-channel chunks
+    constexpr int BPW = 4 / N;        // chunks per word
+    constexpr int SLOTS = 2 * BPW;    // byte groups per word
     constexpr int NGV = D / GV;       // value groups per token
-    constexpr float kInvN = 1.0f / (1 << N);
+    constexpr uint32_t BYTE_MASK = ((1u << N) - 1u) * 0x01010101u;
+    using St = Stage<N, D, GV>;
 
     __shared__ float q_s[D];
     __shared__ float o_s[kDecodeWarps][D];
     __shared__ float ml_s[kDecodeWarps][2];
+    extern __shared__ __align__(128) unsigned char stage_mem[];
 
     const int sigma = blockIdx.x, qi = blockIdx.y, b = blockIdx.z;
     const int g = a.Hq / a.Hkv;
     const int64_t bh = static_cast<int64_t>(b) * a.Hkv + qi / g;
     const int64_t bq = static_cast<int64_t>(b) * a.Hq + qi;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int r8 = lane >> 2, l4 = lane & 3;
+    const int g8 = lane >> 2, t4 = lane & 3;
+    unsigned char *wmem = stage_mem + static_cast<size_t>(warp) * kStages * St::kBytes;
+    const uint32_t magic = kMagicBits;
 
     for (int c = threadIdx.x; c < D; c += kDecodeThreads)
         q_s[c] = widen(a.q[bq * D + c], a.bf16) * a.qscale;
     __syncthreads();
 
+    // this warp's contiguous share of the split's tiles
     const int total_tiles = a.n_qtiles + (a.r + 15) / 16;
     const int t_begin = sigma * a.tiles_per_split;
     const int t_end = min(total_tiles, t_begin + a.tiles_per_split);
+    const int per_w = (t_end - t_begin + kDecodeWarps - 1) / kDecodeWarps;
+    const int wb = t_begin + warp * per_w;
+    const int we = min(t_end, wb + per_w);
+    const int qe = min(we, a.n_qtiles);
     const int64_t groups_cap = a.cap / a.G;
     const uint32_t *kc = a.kc + bh * (a.cap / 16) * TW;
     const uint32_t *vc = a.vc + bh * (a.cap / 16) * TW;
+    const float *vs_g = a.vs + bh * a.cap * NGV;
+    const int16_t *vz_g = a.vz + bh * a.cap * NGV;
     const int zsym = 1 << (N - 1);
+    const int gmask = (1 << a.gshift) - 1;   // tiles per key group - 1
+
+    // producer: stage the tile's lane segments, value meta and (at a group start) key meta
+    auto issue = [&](int ti) {
+        if (ti >= qe) return;
+        unsigned char *st = wmem + ((ti - wb) % kStages) * St::kBytes;
+        const uint32_t *ksrc = kc + static_cast<int64_t>(ti) * TW + lane * W;
+        const uint32_t *vsrc = vc + static_cast<int64_t>(ti) * TW + lane * W;
+        if constexpr (W % 4 == 0) {
+            uint32_t *kdst = reinterpret_cast<uint32_t *>(st) + 4 * lane;
+            uint32_t *vdst = reinterpret_cast<uint32_t *>(st + St::kCodes) + 4 * lane;
+#pragma unroll
+            for (int i = 0; i < W / 4; ++i) {
+                cp_async16(kdst + 128 * i, ksrc + 4 * i);
+                cp_async16(vdst + 128 * i, vsrc + 4 * i);
+            }
+        } else {
+            static_assert(W == 2, "lane segment of 8 bytes");
+            cp_async8(reinterpret_cast<uint32_t *>(st) + lane * W, ksrc);
+            cp_async8(reinterpret_cast<uint32_t *>(st + St::kCodes) + lane * W, vsrc);
+        }
+        const int64_t tok0 = static_cast<int64_t>(ti) * 16;
+        for (int c = lane; c < NGV * 4; c += 32)
+            cp_async16(st + St::kVs + 16 * c, vs_g + tok0 * NGV + 4 * c);
+        if (!a.sym)
+            for (int c = lane; c < NGV * 2; c += 32)
+                cp_async16(st + St::kVz + 16 * c, vz_g + tok0 * NGV + 8 * c);
+        if (ti == wb || (ti & gmask) == 0) {
+            const int64_t gofs = (bh * groups_cap + (ti >> a.gshift)) * D;
+            for (int c = lane; c < D / 4; c += 32) cp_async16(st + St::kKs + 16 * c, a.ks + gofs + 4 * c);
+            if (!a.sym)
+                for (int c = lane; c < D / 8; c += 32) cp_async16(st + St::kKz + 16 * c, a.kz + gofs + 8 * c);
+        }
+    };
 
     float m = -INFINITY, lsum = 0.0f;
-    float2 acc[NJ][2];
+    float2 acc[NJ][2];       // value accumulators, channel 16j + g8 + 8h, x: tokens 4t4+{0,1}, y: +{2,3}
     float zsum[NGV];
 #pragma unroll
     for (int j = 0; j < NJ; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
 #pragma unroll
     for (int v = 0; v < NGV; ++v) zsum[v] = 0.f;
-    float2 mk[NJ][2];
-    float kbias = 0.f;
-    int64_t cur_group = -1;
+    uint32_t kdig[NJ][3];    // key multiplier digits, channels 16j + 4t4 + {0..3}
+    float kbias = 0.f, kinv = 0.f;
 
-    for (int ti = t_begin + warp; ti < t_end; ti += kDecodeWarps) {
+#pragma unroll
+    for (int s = 0; s < kStages - 1; ++s) {
+        issue(wb + s);
+        cp_async_commit();
+    }
+
+    for (int ti = wb; ti < we; ++ti) {
+        issue(ti + kStages - 1);
+        cp_async_commit();
+        cp_async_wait<kStages - 1>();
+        __syncwarp();
+        const unsigned char *st = wmem + ((ti - wb) % kStages) * St::kBytes;
         const bool quant = ti < a.n_qtiles;
-        float lg0, lg1;   // log2-domain logits of tokens r8 and r8 + 8 of the tile
+        float lg0, lg1;   // log2-domain logits of tokens g8 and g8 + 8 of the tile
         if (quant) {
-            const int64_t tok0 = static_cast<int64_t>(ti) * 16;
-            const int64_t grp = tok0 / a.G;
-            if (grp != cur_group) {
-                // key multipliers and bias of the new group
-                const int64_t gofs = (bh * groups_cap + grp) * D;
-                float kb = 0.f;
+            if (ti == wb || (ti & gmask) == 0) {
+                // fixed-point key multipliers and bias of the group this tile opens
+                const float *ks_s = reinterpret_cast<const float *>(st + St::kKs);
+                const int16_t *kz_s = reinterpret_cast<const int16_t *>(st + St::kKz);
+                float qs[NJ][4];
+                float kb = 0.f, mx = 0.f;
 #pragma unroll
                 for (int j = 0; j < NJ; ++j) {
+                    const int c0 = 16 * j + 4 * t4;
+                    const float4 sc = *reinterpret_cast<const float4 *>(ks_s + c0);
+                    const float4 qq = *reinterpret_cast<const float4 *>(q_s + c0);
+                    qs[j][0] = qq.x * sc.x; qs[j][1] = qq.y * sc.y;
+                    qs[j][2] = qq.z * sc.z; qs[j][3] = qq.w * sc.w;
+                    float z[4] = {static_cast<float>(zsym), static_cast<float>(zsym),
+                                  static_cast<float>(zsym), static_cast<float>(zsym)};
+                    if (!a.sym) {
+                        const uint2 zz = *reinterpret_cast<const uint2 *>(kz_s + c0);
+                        z[0] = small_int_to_float(static_cast<int16_t>(zz.x & 0xffffu));
+                        z[1] = small_int_to_float(static_cast<int16_t>(zz.x >> 16));
+                        z[2] = small_int_to_float(static_cast<int16_t>(zz.y & 0xffffu));
+                        z[3] = small_int_to_float(static_cast<int16_t>(zz.y >> 16));
+                    }
 #pragma unroll
-                    for (int s = 0; s < 2; ++s) {
-                        const int c0 = 16 * j + 2 * l4 + 8 * s;
-                        const float2 sc = *reinterpret_cast<const float2 *>(a.ks + gofs + c0);
-                        const float2 qs = make_float2(q_s[c0] * sc.x, q_s[c0 + 1] * sc.y);
-                        float z0 = static_cast<float>(zsym), z1 = z0;
-                        if (!a.sym) {
-                            const uint32_t zz = *reinterpret_cast<const uint32_t *>(a.kz + gofs + c0);
-                            z0 = static_cast<float>(static_cast<int16_t>(zz & 0xffffu));
-                            z1 = static_cast<float>(static_cast<int16_t>(zz >> 16));
-                        }
-                        kb = fmaf(qs.x, z0, kb);
-                        kb = fmaf(qs.y, z1, kb);
-                        const int pos = (4 * j + 2 * s) % P;
-                        const float f = 1.0f / static_cast<float>(1u << (N * pos));
-                        mk[j][s] = make_float2(qs.x * f, qs.y * f);
+                    for (int i = 0; i < 4; ++i) {
+                        kb = fmaf(qs[j][i], z[i], kb);
+                        mx = fmaxf(mx, fabsf(qs[j][i]));
                     }
                 }
                 kb += __shfl_xor_sync(0xffffffffu, kb, 1);
                 kb += __shfl_xor_sync(0xffffffffu, kb, 2);
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                // 2^e with |q'| * 2^e < 2^21: exponent of mx plus one, subtracted from 21
+                int e = 0;
+                if (mx > 0.f) e = 21 - (static_cast<int>((__float_as_uint(mx) >> 23) & 0xff) - 126);
+                e = max(-120, min(120, e));
+                const float scale = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+                kinv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+#pragma unroll
+                for (int j = 0; j < NJ; ++j) {
+                    const int Q0 = round_small(qs[j][0] * scale), Q1 = round_small(qs[j][1] * scale);
+                    const int Q2 = round_small(qs[j][2] * scale), Q3 = round_small(qs[j][3] * scale);
+#pragma unroll
+                    for (int k = 0; k < 3; ++k) {
+                        const uint32_t sel = static_cast<uint32_t>(k | ((k + 4) << 4));
+                        const uint32_t lo = __byte_perm(Q0, Q1, sel);
+                        const uint32_t hi = __byte_perm(Q2, Q3, sel);
+                        kdig[j][k] = __byte_perm(lo, hi, 0x5410);
+                    }
+                }
                 kbias = kb;
-                cur_group = grp;
             }
             uint32_t kw[W];
-            load_lane_words<W>(kc + static_cast<int64_t>(ti) * TW + lane * W, kw);
-            float2 s0 = make_float2(0.f, 0.f), s1 = s0;
+            load_stage_words<W>(reinterpret_cast<const uint32_t *>(st), lane, kw);
+            int ak[2][3] = {{0, 0, 0}, {0, 0, 0}};
 #pragma unroll
             for (int wi = 0; wi < W; ++wi) {
-                const uint32_t lo = kw[wi], hi = kw[wi] >> 16;
 #pragma unroll
-                for (int pi = 0; pi < P; ++pi) {
-                    const int psi = wi * P + pi;
-                    const int j = psi >> 2, k = psi & 3;
-                    const float2 v = code_pair<N>(lo, hi, pi);
-                    if ((k & 1) == 0)
-                        s0 = fma2(v, mk[j][k >> 1], s0);
-                    else
-                        s1 = fma2(v, mk[j][k >> 1], s1);
+                for (int sl = 0; sl < SLOTS; ++sl) {
+                    const uint32_t x = (kw[wi] >> (N * sl)) & BYTE_MASK;
+                    const int j = wi * BPW + (sl >> 1), h = sl & 1;
+                    ak[h][0] = dp4a_uu(x, kdig[j][0], ak[h][0]);
+                    ak[h][1] = dp4a_uu(x, kdig[j][1], ak[h][1]);
+                    ak[h][2] = dp4a_us(x, kdig[j][2], ak[h][2]);
                 }
             }
-            float x0 = s0.x + s0.y, x1 = (s1.x + s1.y) * kInvN;
+            float x0 = (small_int_to_float(ak[0][0]) + 256.f * small_int_to_float(ak[0][1]) +
+                        65536.f * small_int_to_float(ak[0][2])) * kinv;
+            float x1 = (small_int_to_float(ak[1][0]) + 256.f * small_int_to_float(ak[1][1]) +
+                        65536.f * small_int_to_float(ak[1][2])) * kinv;
             x0 += __shfl_xor_sync(0xffffffffu, x0, 1);
             x1 += __shfl_xor_sync(0xffffffffu, x1, 1);
             x0 += __shfl_xor_sync(0xffffffffu, x0, 2);
@@ -200,24 +339,26 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_split_kernel(const D
             lg1 = x1 - kbias;
         } else {
             // residual rows: exact e values
-            const int row0 = (ti - a.n_qtiles) * 16 + r8, row1 = row0 + 8;
+            const int row0 = (ti - a.n_qtiles) * 16 + g8, row1 = row0 + 8;
             float x0 = 0.f, x1 = 0.f;
             const uint16_t *kr = a.kr + bh * a.R * D;
 #pragma unroll
             for (int j = 0; j < NJ; ++j) {
-#pragma unroll
-                for (int s = 0; s < 2; ++s) {
-                    const int c0 = 16 * j + 2 * l4 + 8 * s;
-                    if (row0 < a.r) {
-                        const uint32_t two = *reinterpret_cast<const uint32_t *>(kr + row0 * D + c0);
-                        x0 = fmaf(q_s[c0], widen(two & 0xffffu, a.bf16), x0);
-                        x0 = fmaf(q_s[c0 + 1], widen(two >> 16, a.bf16), x0);
-                    }
-                    if (row1 < a.r) {
-                        const uint32_t two = *reinterpret_cast<const uint32_t *>(kr + row1 * D + c0);
-                        x1 = fmaf(q_s[c0], widen(two & 0xffffu, a.bf16), x1);
-                        x1 = fmaf(q_s[c0 + 1], widen(two >> 16, a.bf16), x1);
-                    }
+                const int c0 = 16 * j + 4 * t4;
+                const float4 qq = *reinterpret_cast<const float4 *>(q_s + c0);
+                if (row0 < a.r) {
+                    const uint2 kk = *reinterpret_cast<const uint2 *>(kr + row0 * D + c0);
+                    x0 = fmaf(qq.x, widen(kk.x & 0xffffu, a.bf16), x0);
+                    x0 = fmaf(qq.y, widen(kk.x >> 16, a.bf16), x0);
+                    x0 = fmaf(qq.z, widen(kk.y & 0xffffu, a.bf16), x0);
+                    x0 = fmaf(qq.w, widen(kk.y >> 16, a.bf16), x0);
+                }
+                if (row1 < a.r) {
+                    const uint2 kk = *reinterpret_cast<const uint2 *>(kr + row1 * D + c0);
+                    x1 = fmaf(qq.x, widen(kk.x & 0xffffu, a.bf16), x1);
+                    x1 = fmaf(qq.y, widen(kk.x >> 16, a.bf16), x1);
+                    x1 = fmaf(qq.z, widen(kk.y & 0xffffu, a.bf16), x1);
+                    x1 = fmaf(qq.w, widen(kk.y >> 16, a.bf16), x1);
                 }
             }
             x0 += __shfl_xor_sync(0xffffffffu, x0, 1);
@@ -234,7 +375,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_split_kernel(const D
         tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
         tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
         if (tmax > m) {
-            const float alpha = exp2f(m - tmax);
+            const float alpha = fast_exp2(m - tmax);
             lsum *= alpha;
 #pragma unroll
             for (int j = 0; j < NJ; ++j) {
@@ -245,86 +386,84 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_split_kernel(const D
             for (int v = 0; v < NGV; ++v) zsum[v] *= alpha;
             m = tmax;
         }
-        const float p0 = exp2f(lg0 - m), p1 = exp2f(lg1 - m);
+        const float p0 = fast_exp2(lg0 - m), p1 = fast_exp2(lg1 - m);
         lsum += p0 + p1;
-        // probabilities of the lane's value tokens 2*l4, 2*l4+1, 2*l4+8, 2*l4+9
-        const float pa = __shfl_sync(0xffffffffu, p0, 8 * l4);
-        const float pb = __shfl_sync(0xffffffffu, p0, 8 * l4 + 4);
-        const float pc = __shfl_sync(0xffffffffu, p1, 8 * l4);
-        const float pd = __shfl_sync(0xffffffffu, p1, 8 * l4 + 4);
+        // probabilities of the lane's value tokens 4*t4 + i (rows g8 + 8*(t4/2))
+        const float pexp = (t4 & 2) ? p1 : p0;
+        float pt[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            pt[i] = __shfl_sync(0xffffffffu, pexp, 4 * ((4 * t4 + i) & 7) + 2 * (t4 >> 1));
 
         if (quant) {
-            const int64_t ta = static_cast<int64_t>(ti) * 16 + 2 * l4;
-            const float *vsp = a.vs + (bh * a.cap + ta) * NGV;
-            const int16_t *vzp = a.vz + (bh * a.cap + ta) * NGV;
-            float2 pm[NGV][2];
+            const float *vsp = reinterpret_cast<const float *>(st + St::kVs) + 4 * t4 * NGV;
+            const int16_t *vzp = reinterpret_cast<const int16_t *>(st + St::kVz) + 4 * t4 * NGV;
+            float2 pm[NGV][2];   // (tokens i, i+2) x value scale x 2^-8i
 #pragma unroll
             for (int v = 0; v < NGV; ++v) {
-                const float sa = vsp[v], sb = vsp[NGV + v];
-                const float sc = vsp[8 * NGV + v], sd = vsp[9 * NGV + v];
-                const float2 plo = make_float2(pa * sa, pb * sb);
-                const float2 phi = make_float2(pc * sc, pd * sd);
-                float za, zb, zc, zd;
-                if (a.sym) {
-                    za = zb = zc = zd = static_cast<float>(zsym);
-                } else {
-                    za = vzp[v]; zb = vzp[NGV + v]; zc = vzp[8 * NGV + v]; zd = vzp[9 * NGV + v];
+                float ps[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    ps[i] = pt[i] * vsp[i * NGV + v];
+                    const float z = a.sym ? static_cast<float>(zsym) : small_int_to_float(vzp[i * NGV + v]);
+                    zsum[v] = fmaf(ps[i], z, zsum[v]);
                 }
-                zsum[v] = fmaf(plo.x, za, zsum[v]);
-                zsum[v] = fmaf(plo.y, zb, zsum[v]);
-                zsum[v] = fmaf(phi.x, zc, zsum[v]);
-                zsum[v] = fmaf(phi.y, zd, zsum[v]);
-                pm[v][0] = plo;
-                pm[v][1] = mul2(phi, make_float2(1.0f / (1 << (2 * N)), 1.0f / (1 << (2 * N))));
+                pm[v][0] = make_float2(ps[0], ps[2]);
+                pm[v][1] = make_float2(ps[1] * (1.0f / 256.0f), ps[3] * (1.0f / 256.0f));
             }
             uint32_t vw[W];
-            load_lane_words<W>(vc + static_cast<int64_t>(ti) * TW + lane * W, vw);
+            load_stage_words<W>(reinterpret_cast<const uint32_t *>(st + St::kCodes), lane, vw);
 #pragma unroll
             for (int wi = 0; wi < W; ++wi) {
                 const uint32_t lo = vw[wi], hi = vw[wi] >> 16;
 #pragma unroll
-                for (int pi = 0; pi < P; ++pi) {
-                    const int psi = wi * P + pi;
-                    const int j = psi >> 2, k = psi & 3;
-                    const float2 v = code_pair<N>(lo, hi, pi);
-                    acc[j][k & 1] = fma2(v, pm[(16 * j) / GV][k >> 1], acc[j][k & 1]);
+                for (int sl = 0; sl < SLOTS; ++sl) {
+                    const int j = wi * BPW + (sl >> 1), h = sl & 1;
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const uint32_t msk = ((1u << N) - 1u) << (8 * i + N * sl);
+                        float2 v = make_float2(__uint_as_float(and_or(lo, msk, magic)),
+                                               __uint_as_float(and_or(hi, msk, magic)));
+                        v = add2(v, make_float2(-kMagic, -kMagic));
+                        acc[j][h] = fma2(v, pm[(16 * j) / GV][i], acc[j][h]);
+                    }
                 }
             }
         } else {
-            const int ra = (ti - a.n_qtiles) * 16 + 2 * l4;
+            const int ra = (ti - a.n_qtiles) * 16 + 4 * t4;
             const uint16_t *vr = a.vr + bh * a.R * D;
 #pragma unroll
             for (int j = 0; j < NJ; ++j) {
-                const int base = (4 * j) % P;
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int c = 16 * j + r8 + 8 * e;
-                    const float f = static_cast<float>(1u << (N * (base + e)));
-                    float2 add = make_float2(0.f, 0.f);
-                    if (ra < a.r) add.x = fmaf(pa, widen(vr[ra * D + c], a.bf16), add.x);
-                    if (ra + 1 < a.r) add.y = fmaf(pb, widen(vr[(ra + 1) * D + c], a.bf16), add.y);
-                    if (ra + 8 < a.r) add.x = fmaf(pc, widen(vr[(ra + 8) * D + c], a.bf16), add.x);
-                    if (ra + 9 < a.r) add.y = fmaf(pd, widen(vr[(ra + 9) * D + c], a.bf16), add.y);
-                    acc[j][e] = fma2(add, make_float2(f, f), acc[j][e]);
+                for (int h = 0; h < 2; ++h) {
+                    const int c = 16 * j + g8 + 8 * h;
+                    const float f = static_cast<float>(1u << (N * (2 * (j % BPW) + h)));
+                    float vv[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        vv[i] = (ra + i < a.r) ? pt[i] * widen(vr[(ra + i) * D + c], a.bf16) : 0.f;
+                    acc[j][h] = fma2(make_float2(vv[0] + vv[1], vv[2] + vv[3]), make_float2(f, f),
+                                     acc[j][h]);
                 }
             }
         }
+        __syncwarp();   // every lane is done with this stage before it is refilled
     }
+    cp_async_wait<0>();
 
-    // ---- warp epilogue: o for channels 16j + r8 + 8e, unnormalised ----
+    // ---- warp epilogue: o for channels 16j + g8 + 8h, unnormalised ----
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
-        const int base = (4 * j) % P;
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const float f = 1.0f / static_cast<float>(1u << (N * (base + e)));
-            float val = (acc[j][e].x + acc[j][e].y) * f - zsum[(16 * j) / GV];
+        for (int h = 0; h < 2; ++h) {
+            const float f = 1.0f / static_cast<float>(1u << (N * (2 * (j % BPW) + h)));
+            float val = (acc[j][h].x + acc[j][h].y) * f - zsum[(16 * j) / GV];
             val += __shfl_xor_sync(0xffffffffu, val, 1);
             val += __shfl_xor_sync(0xffffffffu, val, 2);
-            if (l4 == 0) o_s[warp][16 * j + r8 + 8 * e] = val;
+            if (t4 == 0) o_s[warp][16 * j + g8 + 8 * h] = val;
         }
     }
     if (lane == 0) {
@@ -374,9 +513,24 @@ __global__ void combine_kernel(const float *o_part, const float *m_part, const f
 }
 
 template <int N, int D, int GV>
+constexpr int split_smem() { return kDecodeWarps * kStages * Stage<N, D, GV>::kBytes; }
+
+template <int N, int D, int GV>
 cudaError_t launch_split(const DecodeArgs &a, cudaStream_t s) {
+    // the dynamic shared-memory opt-in is per device; do it once per device
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 64 || !configured[dev]) {
+        e = cudaFuncSetAttribute(decode_split_kernel<N, D, GV>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 split_smem<N, D, GV>());
+        if (e != cudaSuccess) return e;
+        if (dev < 64) configured[dev] = true;
+    }
     dim3 grid(a.S, a.Hq, a.B);
-    decode_split_kernel<N, D, GV><<<grid, kDecodeThreads, 0, s>>>(a);
+    decode_split_kernel<N, D, GV><<<grid, kDecodeThreads, split_smem<N, D, GV>(), s>>>(a);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -384,8 +538,13 @@ cudaError_t launch_split(const DecodeArgs &a, cudaStream_t s) {
 template <int N, int D, int GV>
 int occupancy() {
     int n = 0;
+    if (cudaFuncSetAttribute(decode_split_kernel<N, D, GV>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             split_smem<N, D, GV>()) != cudaSuccess)
+        return 1;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_split_kernel<N, D, GV>,
-                                                      kDecodeThreads, 0) != cudaSuccess)
+                                                      kDecodeThreads, split_smem<N, D, GV>()) !=
+        cudaSuccess)
         return 1;
     return n > 0 ? n : 1;
 }

@@ -67,10 +67,11 @@ kvq_status validate(const kvq_config *c) {
         return fail(KVQ_ERR_UNSUPPORTED, "bits must be 2 or 4 (got %d)", c->bits);
     if (c->head_dim != 64 && c->head_dim != 128)
         return fail(KVQ_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", c->head_dim);
-    if (c->group_k < 16 || c->group_k % 16 != 0 || c->group_k > 256 ||
+    if (!(c->group_k == 16 || c->group_k == 32 || c->group_k == 64 || c->group_k == 128 ||
+          c->group_k == 256) ||
         c->group_k * c->head_dim > 32768)
         return fail(KVQ_ERR_INVALID_ARG,
-                    "group_k must be a multiple of 16, <= 256, with group_k*head_dim <= 32768");
+                    "group_k must be 16, 32, 64, 128 or 256 with group_k*head_dim <= 32768");
     if (!(c->group_v == 16 || c->group_v == 32 || c->group_v == 64 || c->group_v == 128) ||
         c->group_v > c->head_dim)
         return fail(KVQ_ERR_INVALID_ARG, "group_v must be 16, 32, 64 or 128 and <= head_dim");
@@ -107,25 +108,36 @@ struct kvq_cache {
 
 namespace {
 
-// Split count for the current cache length: enough CTAs to fill the GPU once,
-// at least kMinTilesPerSplit tiles each, at most kMaxSplits.
+// Split count for the current cache length.  A CTA's time is modelled as its
+// tiles per warp plus a fixed start/finish cost of ~3 tiles; the kernel's time
+// as that times the number of waves of CTAs over the GPU's resident slots.
+// The split count with the lowest modelled time wins (ties: fewer splits).
 void plan_splits(const kvq_cache *h, int *S_out, int *tiles_per_split) {
     const kvq_config &c = h->cfg;
     const int64_t tiles = h->Tq / 16 + (h->r + 15) / 16;
     const int64_t units = static_cast<int64_t>(c.batch) * c.q_heads;
-    const int64_t target = static_cast<int64_t>(h->num_sms) * h->ctas_per_sm;
-    int64_t S = (target + units - 1) / units;
-    const int64_t by_tiles = (tiles + kMinTilesPerSplit - 1) / kMinTilesPerSplit;
-    if (S > by_tiles) S = by_tiles;
-    if (S > max_splits(&c)) S = max_splits(&c);
-    if (S > h->split_limit) S = h->split_limit;
-    if (S < 1) S = 1;
-    int64_t per = (tiles + S - 1) / S;
-    if (per < 1) per = 1;
-    S = (tiles + per - 1) / per;
-    if (S < 1) S = 1;
-    *S_out = static_cast<int>(S);
-    *tiles_per_split = static_cast<int>(per);
+    const int64_t slots = static_cast<int64_t>(h->num_sms) * h->ctas_per_sm;
+    int64_t cap = (tiles + kMinTilesPerSplit - 1) / kMinTilesPerSplit;
+    if (cap > max_splits(&c)) cap = max_splits(&c);
+    if (cap > h->split_limit) cap = h->split_limit;
+    if (cap < 1) cap = 1;
+    int64_t best_S = 1, best_per = tiles > 0 ? tiles : 1;
+    double best_cost = -1.0;
+    for (int64_t S = 1; S <= cap; ++S) {
+        int64_t per = (tiles + S - 1) / S;
+        if (per < 1) per = 1;
+        const int64_t S_eff = (tiles + per - 1) / per;
+        if (S_eff != S) continue;
+        const int64_t waves = (units * S + slots - 1) / slots;
+        const double cost = static_cast<double>(waves) * ((per + 3) / 4 + 3);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best_S = S;
+            best_per = per;
+        }
+    }
+    *S_out = static_cast<int>(best_S);
+    *tiles_per_split = static_cast<int>(best_per);
 }
 
 kvq::DecodeArgs decode_args(const kvq_cache *h) {
@@ -150,6 +162,8 @@ kvq::DecodeArgs decode_args(const kvq_cache *h) {
     a.bits = c.bits;
     a.sym = c.symmetric != 0;
     a.bf16 = c.dtype == KVQ_BF16;
+    a.gshift = 0;
+    while ((16 << a.gshift) < c.group_k) ++a.gshift;
     a.qscale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c.head_dim)));
     return a;
 }
@@ -369,6 +383,6 @@ uint64_t kvq_kernel_launches(void) { return g_launches.load(); }
 
 const char *kvq_last_error(void) { return g_last_error.c_str(); }
 
-int32_t kvq_layout_version(void) { return 1; }
+int32_t kvq_layout_version(void) { return 2; }
 
 }  // extern "C"

@@ -61,6 +61,7 @@ struct DecodeArgs {
     float *out;                  // [B][Hq][d]
     int64_t cap;
     int B, Hq, Hkv, d, G, Gv, R, bits;
+    int gshift;                  // log2(G / 16): key groups are 2^gshift tiles
     bool sym, bf16;
     int n_qtiles;                // Tq / 16
     int r;                       // residual rows

@@ -15,8 +15,9 @@
 // reconstructs it exactly.
 //
 // Packing writes the library's tile layout (see include/kvq.h): each output
-// word is assembled from the 16x16 tensor-core A-fragment table, so writes are
-// fully coalesced and each thread produces whole words.
+// word is assembled from the 8-bit MMA A-fragment table (four codes of one
+// row per byte group), so writes are fully coalesced and each thread produces
+// whole words.
 #include <cfloat>
 #include <cstdint>
 
@@ -64,11 +65,14 @@ __device__ __forceinline__ int sym_code(float x, float s, int bits) {
 
 // Assemble the packed words of `ntiles` 16-token tiles from byte codes
 // codes[t * d + c] (t relative to the first tile) and store them at dst.
+// Word w of a tile belongs to lane w / W; its slot s (0 .. 8/n - 1) holds, in
+// byte b, the element (row = lane/4 + 8*(s%2), col = 4*(lane%4) + b) of block
+// (chunk) j = (w % W) * (4/n) + s/2 at bit 8*b + n*s.
 __device__ void pack_tiles(const uint8_t *codes, int ntiles, int d, int bits, bool is_v,
                            uint32_t *dst) {
     const int TW = tile_words(d, bits);
     const int W = lane_words(d, bits);
-    const int P = 16 / bits;
+    const int B = 4 / bits;               // blocks per word
     const int total = ntiles * TW;
     for (int wi = threadIdx.x; wi < total; wi += blockDim.x) {
         const int tile = wi / TW;
@@ -76,17 +80,15 @@ __device__ void pack_tiles(const uint8_t *codes, int ntiles, int d, int bits, bo
         const int lane = w / W;
         const int wl = w - lane * W;
         uint32_t word = 0;
-        for (int pi = 0; pi < P; ++pi) {
-            const int pair = wl * P + pi;
-            const int j = pair >> 2, k = pair & 3;
+        for (int slot = 0; slot < 2 * B; ++slot) {
+            const int j = wl * B + (slot >> 1);
+            const int row = (lane >> 2) + 8 * (slot & 1);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                // fragment table: row = lane/4 + 8*(k%2), col = 2*(lane%4) + h + 8*(k/2)
-                const int row = (lane >> 2) + 8 * (k & 1);
-                const int col = 2 * (lane & 3) + h + 8 * (k >> 1);
+            for (int b = 0; b < 4; ++b) {
+                const int col = 4 * (lane & 3) + b;
                 const int t = tile * 16 + (is_v ? col : row);
                 const int c = 16 * j + (is_v ? row : col);
-                word |= static_cast<uint32_t>(codes[t * d + c]) << (16 * h + bits * pi);
+                word |= static_cast<uint32_t>(codes[t * d + c]) << (8 * b + bits * slot);
             }
         }
         dst[wi] = word;
@@ -248,10 +250,17 @@ size_t quantize_smem_bytes(int d, int G) {
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s) {
     if (a.n_groups == 0 || a.BH == 0) return cudaSuccess;
     const size_t smem = quantize_smem_bytes(a.d, a.G);
-    cudaError_t e = cudaFuncSetAttribute(quantize_pack_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    // opt in to the largest dynamic shared memory any configuration needs, once per device
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    if (dev >= 64 || !configured[dev]) {
+        e = cudaFuncSetAttribute(quantize_pack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(quantize_smem_bytes(256, 128)));
+        if (e != cudaSuccess) return e;
+        if (dev < 64) configured[dev] = true;
+    }
     dim3 grid(static_cast<unsigned>(a.n_groups), static_cast<unsigned>(a.BH));
     quantize_pack_kernel<<<grid, kQuantThreads, smem, s>>>(a);
     count_launches(1);

@@ -41,10 +41,12 @@
  *    d*n/2 consecutive words; inside it 32 lanes own W = d*n/64 words each.
  *    In chunk j, a 16x16 block indexed (row, col) -- keys (token%16,
  *    channel%16), values (channel%16, token%16) -- places element (row, col)
- *    in lane 4*(row%8) + (col%8)/2, half col%2, register k = row/8 +
- *    2*(col/8): the A-operand fragment of a 16x16x16 tensor-core MMA.  Pair
- *    p = 4*j + k lives in word p/(16/n) of the lane at bit
- *    16*half + n*(p % (16/n)).
+ *    in lane 4*(row%8) + col/4, byte col%4, half row/8.  A lane's word holds
+ *    B = 4/n blocks: block j in word j/B, element at bit
+ *    8*byte + n*(2*(j%B) + half).  Keeping the low n bits of every byte of
+ *    (word >> n*slot) gives four codes of one row, one per byte: the operand
+ *    of a 4-way byte dot product and the A fragment of an 8-bit 16x8x32
+ *    tensor-core MMA.
  *  - k_scales float / k_zeros int16: [B][Hkv][capacity/G][d]   (group, channel)
  *  - v_scales float / v_zeros int16: [B][Hkv][capacity][d/Gv]  (token, group)
  *  - k_residual, v_residual: e [B][Hkv][R][d]  (rows 0..r-1 valid)
@@ -83,7 +85,7 @@ typedef struct {
     int32_t q_heads;     /* Hq                                                  */
     int32_t kv_heads;    /* Hkv, divides Hq                                     */
     int32_t head_dim;    /* d: 64 or 128                                        */
-    int32_t group_k;     /* G: tokens per key group, multiple of 16, <= 256,
+    int32_t group_k;     /* G: tokens per key group: 16, 32, 64, 128 or 256,
                             G * d <= 32768                                      */
     int32_t group_v;     /* Gv: channels per value group: 16, 32, 64 or 128, <= d */
     int32_t residual;    /* R: residual capacity, multiple of G                 */
@@ -184,7 +186,7 @@ KVQ_API uint64_t kvq_kernel_launches(void);
 /* Description of the last error on the calling thread ("" if none). */
 KVQ_API const char *kvq_last_error(void);
 
-/* Version of the storage format described above (currently 1). */
+/* Version of the storage format described above (currently 2). */
 KVQ_API int32_t kvq_layout_version(void);
 
 #ifdef __cplusplus

@@ -276,10 +276,11 @@ int oracle_quantize_kv(const uint16_t *XK, const uint16_t *XV, int dtype,
  *  - inside a tile, 32 "lanes" own W = d*n/64 consecutive words each;
  *  - within chunk j, a 16x16 block is indexed (row, col): keys use
  *    (row, col) = (t%16, c%16), values use (row, col) = (c%16, t%16);
- *  - lane = 4*(row%8) + (col%8)/2, half = col%2,
- *    k = row/8 + 2*(col/8), pair = 4*j + k;
- *  - a word holds P = 16/n pairs; pair p sits in word p/P of the lane and
- *    its code at bit 16*half + n*(p%P).
+ *  - lane = 4*(row%8) + col/4, byte = col%4, half = row/8;
+ *  - a word holds B = 4/n blocks of a lane: block j sits in word j/B,
+ *    slot s = 2*(j%B) + half, and the code at bit 8*byte + n*s.
+ * So (word >> n*s) masked to the low n bits of every byte yields four codes
+ * of one row, one per byte.
  */
 void oracle_code_position(int64_t t, int c, int is_v, int d, int bits,
                           int64_t *word, int *bit)
@@ -288,14 +289,14 @@ void oracle_code_position(int64_t t, int c, int is_v, int d, int bits,
     int row = is_v ? (c % 16) : (int)(t % 16);
     int col = is_v ? (int)(t % 16) : (c % 16);
     int j = c / 16;
-    int lane = 4 * (row % 8) + (col % 8) / 2;
-    int half = col % 2;
-    int k = row / 8 + 2 * (col / 8);
-    int pair = 4 * j + k;
-    int P = 16 / bits;
+    int lane = 4 * (row % 8) + col / 4;
+    int byte = col % 4;
+    int half = row / 8;
+    int B = 4 / bits;
     int W = d * bits / 64;
-    *word = tile * (int64_t)(d * bits / 2) + (int64_t)lane * W + pair / P;
-    *bit = 16 * half + bits * (pair % P);
+    int slot = 2 * (j % B) + half;
+    *word = tile * (int64_t)(d * bits / 2) + (int64_t)lane * W + j / B;
+    *bit = 8 * byte + bits * slot;
 }
 
 /* Pack codes q [BH][T][d] (T a multiple of 16) into words [BH][T*d*n/32]. */

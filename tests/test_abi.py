@@ -70,6 +70,7 @@ def test_sizes_match_layout():
     (dict(bits=3), kvq.KVQ_ERR_UNSUPPORTED),
     (dict(q_heads=3), kvq.KVQ_ERR_INVALID_ARG),
     (dict(group_k=24), kvq.KVQ_ERR_INVALID_ARG),
+    (dict(group_k=48, residual=96), kvq.KVQ_ERR_INVALID_ARG),
     (dict(group_v=48), kvq.KVQ_ERR_INVALID_ARG),
     (dict(residual=48), kvq.KVQ_ERR_INVALID_ARG),
     (dict(capacity=1000), kvq.KVQ_ERR_INVALID_ARG),
@@ -98,4 +99,4 @@ def test_null_arguments_are_rejected_without_a_device():
     assert lib.kvq_create(ctypes.byref(cfg), ctypes.byref(bufs), ctypes.byref(h)) == \
         kvq.KVQ_ERR_INVALID_ARG
     assert not h.value
-    assert lib.kvq_layout_version() == 1
+    assert lib.kvq_layout_version() == 2

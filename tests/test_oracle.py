@@ -188,23 +188,28 @@ def test_layout_hand_positions(oracle_mod, case):
 
 
 @pytest.mark.parametrize("d,bits", [(32, 2), (64, 2), (128, 2), (64, 4), (128, 4)])
-def test_layout_is_the_mma_a_fragment(oracle_mod, d, bits):
-    """Restates the PTX ISA table of the m16n8k16 f16 A operand (lane l holds,
-    in register a_i, half h: row = l/4 + 8*(i%2), col = 2*(l%4) + h + 8*(i/2))
-    and checks that the packed layout stores each 16x16 block that way."""
-    P = 16 // bits
+def test_layout_is_the_int8_mma_a_fragment(oracle_mod, d, bits):
+    """Restates the PTX ISA table of the m16n8k32 8-bit A operand (lane l holds,
+    in register a_i, byte b: row = l/4 + 8*(i%2), col = 4*(l%4) + b + 16*(i/2))
+    and checks that shifting the lane's word right by n*(2*(j%B) + i%2) and
+    keeping the low n bits of each byte yields that register: for keys a 16x32
+    block spans chunks 2m, 2m+1 of one tile, for values tiles 2m, 2m+1 of one
+    chunk."""
+    B = 4 // bits
     W = d * bits // 64
+    TW = d * bits // 2
     for lane in range(32):
         for i in range(4):
-            for h in range(2):
+            for b in range(4):
                 row = lane // 4 + 8 * (i % 2)
-                col = 2 * (lane % 4) + h + 8 * (i // 2)
+                col = 4 * (lane % 4) + b + 16 * (i // 2)
+                for m in range(d // 32):
+                    j = 2 * m + i // 2                 # keys: chunk of this column
+                    want = (lane * W + j // B, 8 * b + bits * (2 * (j % B) + i % 2))
+                    assert oracle_mod.code_position(row, 32 * m + col, False, d, bits) == want
                 for j in range(d // 16):
-                    pair = 4 * j + i
-                    want = (lane * W + pair // P, 16 * h + bits * (pair % P))
-                    # keys: row = token, col = channel
-                    assert oracle_mod.code_position(row, 16 * j + col, False, d, bits) == want
-                    # values: row = channel, col = token
+                    tile = i // 2                      # values: tile of this column
+                    want = (tile * TW + lane * W + j // B, 8 * b + bits * (2 * (j % B) + i % 2))
                     assert oracle_mod.code_position(col, 16 * j + row, True, d, bits) == want
 
 
