@@ -208,16 +208,12 @@ def run_kvq(args):
     tokens_per_episode = sum(w.B * (tq + r) for tq, r in ctx)
     bytes_per_episode = sum(algorithmic_bytes(w, tq, r) for tq, r in ctx)
 
-    def episode(ev=None):
+    def episode():
         cache.reset()
         cache.prefill_quantize(XK, XV)
         for s in range(w.steps):
             cache.append(tK[s], tV[s])
-            if ev is not None:
-                ev[s][0].record()
             cache.decode_attention(tQ[s], out=out)
-            if ev is not None:
-                ev[s][1].record()
 
     def barrier():
         if world > 1:
@@ -226,33 +222,55 @@ def run_kvq(args):
     for _ in range(args.warmup):
         episode()
     torch.cuda.synchronize()
-    # One episode is captured once as a CUDA graph (with timing events around
-    # every decode_attention call) and replayed: the host-side launch cost of
-    # ~640 small kernels per episode would otherwise starve the GPU.
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(w.steps)]
+    # The episode is captured once as a sequence of CUDA graphs -- the prompt
+    # prefill, then per decode step one graph for append (+ flush) and one for
+    # decode_attention -- and replayed in that order: the host-side cost of
+    # ~640 small launches per episode would otherwise starve the GPU.  Timing
+    # events sit between the graph launches, on the capture/replay stream, so
+    # every decode_attention call of the timed region is timed individually.
     launches0 = kvq.kernel_launches()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        episode(evs)
+    pool = torch.cuda.graph_pool_handle()
+    cache.reset()
+    g_pre = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_pre, pool=pool):
+        cache.prefill_quantize(XK, XV)
+    g_app, g_dec = [], []
+    for s_ in range(w.steps):
+        ga, gd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(ga, pool=pool):
+            cache.append(tK[s_], tV[s_])
+        with torch.cuda.graph(gd, pool=pool):
+            cache.decode_attention(tQ[s_], out=out)
+        g_app.append(ga)
+        g_dec.append(gd)
     launches_per_episode = kvq.kernel_launches() - launches0
-    graph.replay()
+    torch.cuda.synchronize()
+
+    def replay_episode(ev):
+        g_pre.replay()
+        for s_ in range(w.steps):
+            g_app[s_].replay()
+            ev[s_][0].record(stream)
+            g_dec[s_].replay()
+            ev[s_][1].record(stream)
+
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(w.steps)] for _ in range(args.steps + 1)]
+    replay_episode(evs[-1])          # graph warm-up
     torch.cuda.synchronize()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
-    decode_ms = 0.0
     with ClockSampler(local) as clk:
         start.record(stream)
         for k in range(args.steps):
-            graph.replay()
+            replay_episode(evs[k])
         stop.record(stream)
         torch.cuda.synchronize()
         barrier()
     launches = launches_per_episode * args.steps
     ms = start.elapsed_time(stop)
-    # decode_attention durations of the last replay (the events are graph nodes)
-    decode_ms = sum(a.elapsed_time(b) for a, b in evs) * args.steps
+    decode_ms = sum(a.elapsed_time(b) for ev in evs[:args.steps] for a, b in ev)
     t = torch.tensor([ms, decode_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)

@@ -5,11 +5,12 @@
 // ("LLM系列：KVCache量化1 KIVI ...", section 1: A = Concat(A_g, A_r), t_O = A X_V;
 //  the 1/sqrt(d_k) of "KV Cache的Int4量化…" section 3), with deq(x) = (code - z) s.
 //
-// Split-K (flash-decoding): the token axis -- quantized 16-token tiles followed
-// by the residual rows, cut into 16-row tiles -- is divided into S contiguous
-// splits; a CTA owns one (batch, query head, split) and each of its four warps a
-// contiguous share of the split's tiles, streamed through a per-warp cp.async
-// ring of shared-memory stages.  Token order does not change the result
+// Split-K (flash-decoding): the quantized 16-token tiles are divided into
+// contiguous splits and the residual rows, cut into 16-row tiles, form one more
+// split of their own (they are read unstaged, so they run beside the others
+// instead of lengthening one of them); a CTA owns one (batch, query head,
+// split) and each of its four warps a contiguous share of the split's tiles,
+// streamed through a per-warp cp.async ring of shared-memory stages.  Token order does not change the result
 // (A . V = A_P . V_P, "Resumo Técnico: LogQuant", section 4), which is what
 // allows the splits and the residual to be folded into one online-softmax pass.
 // Each CTA writes an unnormalised partial (o, m, l); combine_kernel merges the
@@ -187,10 +188,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_split_kernel(const D
         q_s[c] = widen(a.q[bq * D + c], a.bf16) * a.qscale;
     __syncthreads();
 
-    // this warp's contiguous share of the split's tiles
+    // this warp's contiguous share of the split's tiles: splits 0 .. n_qsplits-1 cut the
+    // quantized tiles, the last split (when r > 0) owns the residual tiles alone
     const int total_tiles = a.n_qtiles + (a.r + 15) / 16;
-    const int t_begin = sigma * a.tiles_per_split;
-    const int t_end = min(total_tiles, t_begin + a.tiles_per_split);
+    const int t_begin = sigma < a.n_qsplits ? sigma * a.tiles_per_split : a.n_qtiles;
+    const int t_end = sigma < a.n_qsplits ? min(a.n_qtiles, t_begin + a.tiles_per_split) : total_tiles;
     const int per_w = (t_end - t_begin + kDecodeWarps - 1) / kDecodeWarps;
     const int wb = t_begin + warp * per_w;
     const int we = min(t_end, wb + per_w);
@@ -493,6 +495,510 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_split_kernel(const D
     }
 }
 
+// ---------------------------------------------------------------------------
+// Grouped-query heads (4 query heads per kv head): tensor-core path.
+//
+// A CTA owns one (batch, kv head, split) and serves the 4 query heads that read
+// that kv head, so every code is fetched and unpacked once for all of them.
+// Lane = 4*g8 + t4; query head t4 is "owned" by the lanes with that t4.
+//   keys   : int8 MMA m16n8k32.  A = the byte-masked key codes (rows = tokens,
+//            k = channels) exactly as stored; B = byte digits of the 21-bit
+//            fixed-point multipliers q_c s_{g,c} log2(e)/sqrt(d) (exponent per
+//            key group and head), columns 2h+d (digits 0, 1 of head h) in the
+//            first n-tile and 2h (signed digit 2) in the second; int32 sums,
+//            exact.  The digits are built once per key group, cooperatively by
+//            the warp (lane l: head l/8, 16 channels), in shared memory.
+//   values : f16 MMA m16n8k16.  A = value codes as exact f16 (rows = channels,
+//            k = tokens; bytes 0,2 and 1,3 of a masked word are f16x2 pairs via
+//            the 0x6400 exponent trick); B = p_t s_{t,gv} split into f16 hi +
+//            lo parts (columns 2h, 2h+1), built cooperatively per tile; fp32
+//            accumulators, rescaled when a head's running maximum grows.
+//   z-terms: bias_g = sum_c q'_c z_{g,c} and sum_t p_t s_t z_t in fp32.
+// Residual rows form the last split, where each warp serves one query head
+// with exact e values on CUDA cores.
+// ---------------------------------------------------------------------------
+constexpr int kGqa = 4;
+
+__device__ __forceinline__ void imma_uu(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void imma_us(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void hmma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                     uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// f16x2 arithmetic on raw registers
+__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+// (lo, hi) floats -> f16x2 (round to nearest)
+__device__ __forceinline__ uint32_t f2h2(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+__device__ __forceinline__ float2 h22f(uint32_t h) {
+    __half2_raw r;
+    r.x = static_cast<unsigned short>(h & 0xffffu);
+    r.y = static_cast<unsigned short>(h >> 16);
+    return __half22float2(__half2(r));
+}
+
+// Codes of a masked-word slot as two exact f16x2 registers: (byte 0, byte 2), (byte 1, byte 3).
+// 0x6400 is the f16 1024 with unit mantissa steps; a code OR-ed into the low
+// mantissa bits gives 1024 + code.  For 2-bit codes the byte-1/3 codes sit at
+// mantissa bits 8-9 (1024 + 256 code, rescaled by one f16x2 FMA); 4-bit codes
+// there would reach the exponent, so they are shifted down first.
+template <int N>
+__device__ __forceinline__ void codes_f16(uint32_t xs, uint32_t magic16, uint32_t &r02, uint32_t &r13) {
+    constexpr uint32_t L = (1u << N) - 1u;
+    r02 = hsub2(and_or(xs, L | (L << 16), magic16), magic16);                  // (1024 + c) - 1024
+    if constexpr (N == 2)
+        r13 = hfma2(and_or(xs, (L << 8) | (L << 24), magic16), 0x1C001C00u,    // (1024 + 256c)/256 - 4
+                    0xC400C400u);
+    else
+        r13 = hsub2(and_or(xs >> 8, L | (L << 16), magic16), magic16);
+}
+
+template <int N, int D, int GV>
+struct GqaSmem {
+    static constexpr int NGV = D / GV;
+    static constexpr int kStageBytes = kStages * Stage<N, D, GV>::kBytes;
+    static constexpr int kKd = kStageBytes;                  // key digits [3][4 heads][D] bytes
+    static constexpr int kVb = kKd + 3 * kGqa * D;           // value B [NGV][4][2][16] f16
+    static constexpr int kPs = kVb + NGV * kGqa * 2 * 16 * 2; // p [4][16] f32
+    static constexpr int kAl = kPs + kGqa * 16 * 4;          // alpha [4], key scale [4], bias [4]
+    static constexpr int kWarpBytes = kAl + 16 * 4;
+    static_assert(kKd % 16 == 0 && kVb % 16 == 0 && kPs % 16 == 0 && kAl % 16 == 0, "align");
+};
+
+template <int N, int D, int GV>
+__global__ void __launch_bounds__(kDecodeThreads, 3) decode_gqa_kernel(const DecodeArgs a) {
+    constexpr int W = D * N / 64;
+    constexpr int TW = D * N / 2;
+    constexpr int NJ = D / 16;
+    constexpr int NK = D / 32;        // k32 steps of the key MMA
+    constexpr int BPW = 4 / N;
+    constexpr int NGV = D / GV;
+    constexpr uint32_t BYTE_MASK = ((1u << N) - 1u) * 0x01010101u;
+    using St = Stage<N, D, GV>;
+    using Sm = GqaSmem<N, D, GV>;
+
+    __shared__ __align__(16) float q_s[kGqa][D];
+    __shared__ float ml_s[kDecodeWarps][kGqa][2];
+    extern __shared__ __align__(128) unsigned char stage_mem[];
+
+    const int sigma = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+    const int64_t bh = static_cast<int64_t>(b) * a.Hkv + hk;
+    const int64_t bq0 = static_cast<int64_t>(b) * a.Hq + hk * kGqa;   // first query head
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g8 = lane >> 2, t4 = lane & 3;
+    unsigned char *wmem = stage_mem + static_cast<size_t>(warp) * Sm::kWarpBytes;
+    uint8_t *kd = wmem + Sm::kKd;
+    uint16_t *vb = reinterpret_cast<uint16_t *>(wmem + Sm::kVb);
+    float *ps = reinterpret_cast<float *>(wmem + Sm::kPs);
+    float *al = reinterpret_cast<float *>(wmem + Sm::kAl);
+    const uint32_t magic = kMagicBits;
+    const uint32_t magic16 = 0x64006400u;
+
+    for (int i = threadIdx.x; i < kGqa * D; i += kDecodeThreads)
+        q_s[i / D][i % D] = widen(a.q[bq0 * D + i], a.bf16) * a.qscale;
+    __syncthreads();
+
+    const int total_tiles = a.n_qtiles + (a.r + 15) / 16;
+    const int zsym = 1 << (N - 1);
+
+    if (sigma >= a.n_qsplits) {
+        // ---------------- residual split: warp = query head ----------------
+        const float *qh = q_s[warp];
+        const int64_t bq = bq0 + warp;
+        float m = -INFINITY, lsum = 0.f;
+        float2 acc[NJ][2];
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
+        const uint16_t *kr = a.kr + bh * a.R * D;
+        const uint16_t *vr = a.vr + bh * a.R * D;
+        for (int ti = a.n_qtiles; ti < total_tiles; ++ti) {
+            const int row0 = (ti - a.n_qtiles) * 16 + g8, row1 = row0 + 8;
+            float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+            for (int j = 0; j < NJ; ++j) {
+                const int c0 = 16 * j + 4 * t4;
+                const float4 qq = *reinterpret_cast<const float4 *>(qh + c0);
+                if (row0 < a.r) {
+                    const uint2 kk = *reinterpret_cast<const uint2 *>(kr + row0 * D + c0);
+                    x0 = fmaf(qq.x, widen(kk.x & 0xffffu, a.bf16), x0);
+                    x0 = fmaf(qq.y, widen(kk.x >> 16, a.bf16), x0);
+                    x0 = fmaf(qq.z, widen(kk.y & 0xffffu, a.bf16), x0);
+                    x0 = fmaf(qq.w, widen(kk.y >> 16, a.bf16), x0);
+                }
+                if (row1 < a.r) {
+                    const uint2 kk = *reinterpret_cast<const uint2 *>(kr + row1 * D + c0);
+                    x1 = fmaf(qq.x, widen(kk.x & 0xffffu, a.bf16), x1);
+                    x1 = fmaf(qq.y, widen(kk.x >> 16, a.bf16), x1);
+                    x1 = fmaf(qq.z, widen(kk.y & 0xffffu, a.bf16), x1);
+                    x1 = fmaf(qq.w, widen(kk.y >> 16, a.bf16), x1);
+                }
+            }
+            x0 += __shfl_xor_sync(0xffffffffu, x0, 1);
+            x1 += __shfl_xor_sync(0xffffffffu, x1, 1);
+            x0 += __shfl_xor_sync(0xffffffffu, x0, 2);
+            x1 += __shfl_xor_sync(0xffffffffu, x1, 2);
+            const float lg0 = row0 < a.r ? x0 : -INFINITY;
+            const float lg1 = row1 < a.r ? x1 : -INFINITY;
+            float tmax = fmaxf(lg0, lg1);
+            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
+            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
+            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
+            if (tmax > m) {
+                const float alpha = fast_exp2(m - tmax);
+                lsum *= alpha;
+#pragma unroll
+                for (int j = 0; j < NJ; ++j) {
+                    acc[j][0] = mul2(acc[j][0], make_float2(alpha, alpha));
+                    acc[j][1] = mul2(acc[j][1], make_float2(alpha, alpha));
+                }
+                m = tmax;
+            }
+            const float p0 = fast_exp2(lg0 - m), p1 = fast_exp2(lg1 - m);
+            lsum += p0 + p1;
+            const float pexp = (t4 & 2) ? p1 : p0;
+            float pt[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                pt[i] = __shfl_sync(0xffffffffu, pexp, 4 * ((4 * t4 + i) & 7) + 2 * (t4 >> 1));
+            const int ra = (ti - a.n_qtiles) * 16 + 4 * t4;
+#pragma unroll
+            for (int j = 0; j < NJ; ++j) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int c = 16 * j + g8 + 8 * h;
+                    float vv[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        vv[i] = (ra + i < a.r) ? pt[i] * widen(vr[(ra + i) * D + c], a.bf16) : 0.f;
+                    acc[j][h] = add2(acc[j][h], make_float2(vv[0] + vv[1], vv[2] + vv[3]));
+                }
+            }
+        }
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float val = acc[j][h].x + acc[j][h].y;
+                val += __shfl_xor_sync(0xffffffffu, val, 1);
+                val += __shfl_xor_sync(0xffffffffu, val, 2);
+                if (t4 == 0) a.o_part[(bq * a.S + sigma) * D + 16 * j + g8 + 8 * h] = val;
+            }
+        }
+        if (lane == 0) {
+            a.m_part[bq * a.S + sigma] = m;
+            a.l_part[bq * a.S + sigma] = lsum;
+        }
+        return;
+    }
+
+    // ---------------- quantized split ----------------
+    const int t_begin = sigma * a.tiles_per_split;
+    const int t_end = min(a.n_qtiles, t_begin + a.tiles_per_split);
+    const int per_w = (t_end - t_begin + kDecodeWarps - 1) / kDecodeWarps;
+    const int wb = t_begin + warp * per_w;
+    const int we = min(t_end, wb + per_w);
+    const int64_t groups_cap = a.cap / a.G;
+    const uint32_t *kc = a.kc + bh * (a.cap / 16) * TW;
+    const uint32_t *vc = a.vc + bh * (a.cap / 16) * TW;
+    const float *vs_g = a.vs + bh * a.cap * NGV;
+    const int16_t *vz_g = a.vz + bh * a.cap * NGV;
+    const int gmask = (1 << a.gshift) - 1;
+
+    auto issue = [&](int ti) {
+        if (ti >= we) return;
+        unsigned char *st = wmem + ((ti - wb) % kStages) * St::kBytes;
+        const uint32_t *ksrc = kc + static_cast<int64_t>(ti) * TW + lane * W;
+        const uint32_t *vsrc = vc + static_cast<int64_t>(ti) * TW + lane * W;
+        if constexpr (W % 4 == 0) {
+            uint32_t *kdst = reinterpret_cast<uint32_t *>(st) + 4 * lane;
+            uint32_t *vdst = reinterpret_cast<uint32_t *>(st + St::kCodes) + 4 * lane;
+#pragma unroll
+            for (int i = 0; i < W / 4; ++i) {
+                cp_async16(kdst + 128 * i, ksrc + 4 * i);
+                cp_async16(vdst + 128 * i, vsrc + 4 * i);
+            }
+        } else {
+            static_assert(W == 2, "lane segment of 8 bytes");
+            cp_async8(reinterpret_cast<uint32_t *>(st) + lane * W, ksrc);
+            cp_async8(reinterpret_cast<uint32_t *>(st + St::kCodes) + lane * W, vsrc);
+        }
+        const int64_t tok0 = static_cast<int64_t>(ti) * 16;
+        for (int c = lane; c < NGV * 4; c += 32)
+            cp_async16(st + St::kVs + 16 * c, vs_g + tok0 * NGV + 4 * c);
+        if (!a.sym)
+            for (int c = lane; c < NGV * 2; c += 32)
+                cp_async16(st + St::kVz + 16 * c, vz_g + tok0 * NGV + 8 * c);
+        if (ti == wb || (ti & gmask) == 0) {
+            const int64_t gofs = (bh * groups_cap + (ti >> a.gshift)) * D;
+            for (int c = lane; c < D / 4; c += 32) cp_async16(st + St::kKs + 16 * c, a.ks + gofs + 4 * c);
+            if (!a.sym)
+                for (int c = lane; c < D / 8; c += 32) cp_async16(st + St::kKz + 16 * c, a.kz + gofs + 8 * c);
+        }
+    };
+
+    // owner state (query head t4)
+    float m = -INFINITY, lsum = 0.f;
+    float dv[NJ][4];                  // value accumulators: channel 16j + g8 (+8), head t4 hi / lo
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) dv[j][0] = dv[j][1] = dv[j][2] = dv[j][3] = 0.f;
+    float kinv = 0.f, kbias = 0.f;
+    // builder state (head hb = lane / 8)
+    const int hb = lane >> 3, lb = lane & 7;
+    float zsum[NGV];
+#pragma unroll
+    for (int v = 0; v < NGV; ++v) zsum[v] = 0.f;
+    // B operands of the key MMA for the current group
+    uint32_t kb0[NK][2], kb1[NK][2];
+
+#pragma unroll
+    for (int s = 0; s < kStages - 1; ++s) {
+        issue(wb + s);
+        cp_async_commit();
+    }
+
+    for (int ti = wb; ti < we; ++ti) {
+        issue(ti + kStages - 1);
+        cp_async_commit();
+        cp_async_wait<kStages - 1>();
+        __syncwarp();
+        const unsigned char *st = wmem + ((ti - wb) % kStages) * St::kBytes;
+
+        if (ti == wb || (ti & gmask) == 0) {
+            // ---- key digits of this group: lane builds head hb, channels 16*lb .. +15 ----
+            const float *ks_s = reinterpret_cast<const float *>(st + St::kKs);
+            const int16_t *kz_s = reinterpret_cast<const int16_t *>(st + St::kKz);
+            float qv[16];
+            float mx = 0.f, kbp = 0.f;
+#pragma unroll
+            for (int i4 = 0; i4 < 4; ++i4) {
+                const int c0 = 16 * lb + 4 * i4;
+                const float4 sc = *reinterpret_cast<const float4 *>(ks_s + c0);
+                const float4 qq = *reinterpret_cast<const float4 *>(&q_s[hb][c0]);
+                qv[4 * i4 + 0] = qq.x * sc.x; qv[4 * i4 + 1] = qq.y * sc.y;
+                qv[4 * i4 + 2] = qq.z * sc.z; qv[4 * i4 + 3] = qq.w * sc.w;
+                float z[4] = {static_cast<float>(zsym), static_cast<float>(zsym),
+                              static_cast<float>(zsym), static_cast<float>(zsym)};
+                if (!a.sym) {
+                    const uint2 zz = *reinterpret_cast<const uint2 *>(kz_s + c0);
+                    z[0] = small_int_to_float(static_cast<int16_t>(zz.x & 0xffffu));
+                    z[1] = small_int_to_float(static_cast<int16_t>(zz.x >> 16));
+                    z[2] = small_int_to_float(static_cast<int16_t>(zz.y & 0xffffu));
+                    z[3] = small_int_to_float(static_cast<int16_t>(zz.y >> 16));
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    kbp = fmaf(qv[4 * i4 + i], z[i], kbp);
+                    mx = fmaxf(mx, fabsf(qv[4 * i4 + i]));
+                }
+            }
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1) {
+                kbp += __shfl_xor_sync(0xffffffffu, kbp, o);
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            }
+            int e = 0;
+            if (mx > 0.f) e = 21 - (static_cast<int>((__float_as_uint(mx) >> 23) & 0xff) - 126);
+            e = max(-120, min(120, e));
+            const float scale = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+            uint32_t dw[3][4];
+#pragma unroll
+            for (int i4 = 0; i4 < 4; ++i4) {
+                const int Q0 = round_small(qv[4 * i4 + 0] * scale), Q1 = round_small(qv[4 * i4 + 1] * scale);
+                const int Q2 = round_small(qv[4 * i4 + 2] * scale), Q3 = round_small(qv[4 * i4 + 3] * scale);
+#pragma unroll
+                for (int k = 0; k < 3; ++k) {
+                    const uint32_t sel = static_cast<uint32_t>(k | ((k + 4) << 4));
+                    dw[k][i4] = __byte_perm(__byte_perm(Q0, Q1, sel), __byte_perm(Q2, Q3, sel), 0x5410);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 3; ++k)
+                *reinterpret_cast<uint4 *>(kd + (k * kGqa + hb) * D + 16 * lb) =
+                    make_uint4(dw[k][0], dw[k][1], dw[k][2], dw[k][3]);
+            if (lb == 0) {
+                al[4 + hb] = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+                al[8 + hb] = kbp;
+            }
+            __syncwarp();
+            // B fragments: column g8 = head g8/2, digit g8%2 (first n-tile), digit 2 for even g8
+            const uint32_t *kdw0 = reinterpret_cast<const uint32_t *>(kd + ((g8 & 1) * kGqa + (g8 >> 1)) * D);
+            const uint32_t *kdw2 = reinterpret_cast<const uint32_t *>(kd + (2 * kGqa + (g8 >> 1)) * D);
+#pragma unroll
+            for (int mk = 0; mk < NK; ++mk) {
+                kb0[mk][0] = kdw0[8 * mk + t4];
+                kb0[mk][1] = kdw0[8 * mk + 4 + t4];
+                kb1[mk][0] = (g8 & 1) ? 0u : kdw2[8 * mk + t4];
+                kb1[mk][1] = (g8 & 1) ? 0u : kdw2[8 * mk + 4 + t4];
+            }
+            kinv = al[4 + t4];
+            kbias = al[8 + t4];
+        }
+
+        // ---- key MMA: logits of tokens g8, g8 + 8 for query head t4 ----
+        uint32_t kw[W];
+        load_stage_words<W>(reinterpret_cast<const uint32_t *>(st), lane, kw);
+        int d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int mk = 0; mk < NK; ++mk) {
+            uint32_t af[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int j = 2 * mk + (r >> 1), half = r & 1;
+                af[r] = (kw[j / BPW] >> (N * (2 * (j % BPW) + half))) & BYTE_MASK;
+            }
+            imma_uu(d0, af, kb0[mk][0], kb0[mk][1]);
+            imma_us(d1, af, kb1[mk][0], kb1[mk][1]);
+        }
+        const float lg0 = (small_int_to_float(d0[0]) + 256.f * small_int_to_float(d0[1]) +
+                           65536.f * small_int_to_float(d1[0])) * kinv - kbias;
+        const float lg1 = (small_int_to_float(d0[2]) + 256.f * small_int_to_float(d0[3]) +
+                           65536.f * small_int_to_float(d1[2])) * kinv - kbias;
+
+        // ---- online softmax of head t4 ----
+        float tmax = fmaxf(lg0, lg1);
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
+        const bool grew = tmax > m;
+        if (__any_sync(0xffffffffu, grew)) {
+            const float alpha = grew ? fast_exp2(m - tmax) : 1.f;
+            if (grew) m = tmax;
+            lsum *= alpha;
+#pragma unroll
+            for (int j = 0; j < NJ; ++j) {
+                dv[j][0] *= alpha; dv[j][1] *= alpha; dv[j][2] *= alpha; dv[j][3] *= alpha;
+            }
+            if (g8 == 0) al[t4] = alpha;
+            __syncwarp();
+            const float ab = al[hb];
+#pragma unroll
+            for (int v = 0; v < NGV; ++v) zsum[v] *= ab;
+        }
+        const float p0 = fast_exp2(lg0 - m), p1 = fast_exp2(lg1 - m);
+        lsum += p0 + p1;
+        ps[t4 * 16 + g8] = p0;
+        ps[t4 * 16 + g8 + 8] = p1;
+        __syncwarp();
+
+        // ---- value B: lane builds head hb, tokens 4q + e and 4q + e + 2 ----
+        {
+            const int q4 = lb >> 1, e = lb & 1;
+            const int ta = 4 * q4 + e, tb = ta + 2;
+            const float pa = ps[hb * 16 + ta], pb = ps[hb * 16 + tb];
+            const float *vsp = reinterpret_cast<const float *>(st + St::kVs);
+            const int16_t *vzp = reinterpret_cast<const int16_t *>(st + St::kVz);
+#pragma unroll
+            for (int v = 0; v < NGV; ++v) {
+                const float xa = pa * vsp[ta * NGV + v], xb = pb * vsp[tb * NGV + v];
+                const float za = a.sym ? static_cast<float>(zsym) : small_int_to_float(vzp[ta * NGV + v]);
+                const float zb = a.sym ? static_cast<float>(zsym) : small_int_to_float(vzp[tb * NGV + v]);
+                zsum[v] = fmaf(xa, za, fmaf(xb, zb, zsum[v]));
+                const uint32_t hi = f2h2(xa, xb);
+                const float2 hf = h22f(hi);
+                const uint32_t lo = f2h2(xa - hf.x, xb - hf.y);
+                uint32_t *dst = reinterpret_cast<uint32_t *>(vb + ((v * kGqa + hb) * 2) * 16);
+                dst[(4 * q4 + 2 * e) >> 1] = hi;          // part 0 plane
+                dst[(16 + 4 * q4 + 2 * e) >> 1] = lo;     // part 1 plane
+            }
+        }
+        __syncwarp();
+
+        // ---- value MMA: rows = channels of chunk j, k = the tile's tokens ----
+        uint32_t vw[W];
+        load_stage_words<W>(reinterpret_cast<const uint32_t *>(st + St::kCodes), lane, vw);
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+            const uint32_t x0 = vw[j / BPW] >> (N * (2 * (j % BPW)));
+            const uint32_t x1 = vw[j / BPW] >> (N * (2 * (j % BPW) + 1));
+            uint32_t a02, a13, b02, b13;
+            codes_f16<N>(x0, magic16, a02, a13);      // channel 16j + g8
+            codes_f16<N>(x1, magic16, b02, b13);      // channel 16j + g8 + 8
+            const uint2 bb = *reinterpret_cast<const uint2 *>(
+                vb + (((16 * j) / GV * kGqa + (g8 >> 1)) * 2 + (g8 & 1)) * 16 + 4 * t4);
+            hmma(dv[j], a02, b02, a13, b13, bb.x, bb.y);
+        }
+        __syncwarp();
+    }
+    cp_async_wait<0>();
+    (void)magic;
+
+    // ---- epilogue: reduce per head, subtract the z-terms, merge warps ----
+    lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
+    lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
+    lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
+#pragma unroll
+    for (int v = 0; v < NGV; ++v) {
+        zsum[v] += __shfl_xor_sync(0xffffffffu, zsum[v], 1);
+        zsum[v] += __shfl_xor_sync(0xffffffffu, zsum[v], 2);
+        zsum[v] += __shfl_xor_sync(0xffffffffu, zsum[v], 4);
+    }
+    __syncthreads();   // stage memory is reused for the per-warp outputs below
+    float *o_s = reinterpret_cast<float *>(stage_mem);   // [warp][head][D]
+    float *zs_s = o_s + kDecodeWarps * kGqa * D;          // [warp][head][NGV]
+    if (lb == 0)
+        for (int v = 0; v < NGV; ++v) zs_s[(warp * kGqa + hb) * NGV + v] = zsum[v];
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+        const float z = zs_s[(warp * kGqa + t4) * NGV + (16 * j) / GV];
+        o_s[(warp * kGqa + t4) * D + 16 * j + g8] = dv[j][0] + dv[j][1] - z;
+        o_s[(warp * kGqa + t4) * D + 16 * j + g8 + 8] = dv[j][2] + dv[j][3] - z;
+    }
+    if (g8 == 0) {
+        ml_s[warp][t4][0] = m;
+        ml_s[warp][t4][1] = lsum;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < kGqa * D; i += kDecodeThreads) {
+        const int hh = i / D, c = i % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kDecodeWarps; ++w) M = fmaxf(M, ml_s[w][hh][0]);
+        float o = 0.f, l = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDecodeWarps; ++w) {
+            if (ml_s[w][hh][0] == -INFINITY) continue;
+            const float f = exp2f(ml_s[w][hh][0] - M);
+            o = fmaf(o_s[(w * kGqa + hh) * D + c], f, o);
+            l = fmaf(ml_s[w][hh][1], f, l);
+        }
+        const int64_t bq = bq0 + hh;
+        a.o_part[(bq * a.S + sigma) * D + c] = o;
+        if (c == 0) {
+            a.m_part[bq * a.S + sigma] = M;
+            a.l_part[bq * a.S + sigma] = l;
+        }
+    }
+}
+
 // Log-sum-exp merge of the S split partials of one (batch, query head).
 __global__ void combine_kernel(const float *o_part, const float *m_part, const float *l_part,
                                float *out, int S, int D) {
@@ -536,6 +1042,39 @@ cudaError_t launch_split(const DecodeArgs &a, cudaStream_t s) {
 }
 
 template <int N, int D, int GV>
+constexpr int gqa_smem() { return kDecodeWarps * GqaSmem<N, D, GV>::kWarpBytes; }
+
+template <int N, int D, int GV>
+cudaError_t launch_gqa(const DecodeArgs &a, cudaStream_t s) {
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 64 || !configured[dev]) {
+        e = cudaFuncSetAttribute(decode_gqa_kernel<N, D, GV>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, gqa_smem<N, D, GV>());
+        if (e != cudaSuccess) return e;
+        if (dev < 64) configured[dev] = true;
+    }
+    dim3 grid(a.S, a.Hkv, a.B);
+    decode_gqa_kernel<N, D, GV><<<grid, kDecodeThreads, gqa_smem<N, D, GV>(), s>>>(a);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+template <int N, int D, int GV>
+int gqa_occupancy() {
+    int n = 0;
+    if (cudaFuncSetAttribute(decode_gqa_kernel<N, D, GV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gqa_smem<N, D, GV>()) != cudaSuccess)
+        return 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_gqa_kernel<N, D, GV>, kDecodeThreads,
+                                                      gqa_smem<N, D, GV>()) != cudaSuccess)
+        return 1;
+    return n > 0 ? n : 1;
+}
+
+template <int N, int D, int GV>
 int occupancy() {
     int n = 0;
     if (cudaFuncSetAttribute(decode_split_kernel<N, D, GV>,
@@ -552,8 +1091,12 @@ int occupancy() {
 // Dispatch over the compiled (bits, head_dim, value-group) variants.
 template <int N, int D, int GV>
 struct LaunchF {
-    static cudaError_t run(const DecodeArgs &a, cudaStream_t s) { return launch_split<N, D, GV>(a, s); }
-    static int occ() { return occupancy<N, D, GV>(); }
+    static cudaError_t run(const DecodeArgs &a, cudaStream_t s) {
+        return a.gqa ? launch_gqa<N, D, GV>(a, s) : launch_split<N, D, GV>(a, s);
+    }
+    static int occ(const DecodeArgs &a) {
+        return a.gqa ? gqa_occupancy<N, D, GV>() : occupancy<N, D, GV>();
+    }
 };
 
 template <int N, int D>
@@ -570,10 +1113,10 @@ cudaError_t launch_gv(const DecodeArgs &a, cudaStream_t s) {
 template <int N, int D>
 int occ_gv(const DecodeArgs &a) {
     switch (a.Gv) {
-        case 16: return LaunchF<N, D, 16>::occ();
-        case 32: return LaunchF<N, D, 32>::occ();
-        case 64: return LaunchF<N, D, 64>::occ();
-        default: if constexpr (D >= 128) { if (a.Gv == 128) return LaunchF<N, D, 128>::occ(); }
+        case 16: return LaunchF<N, D, 16>::occ(a);
+        case 32: return LaunchF<N, D, 32>::occ(a);
+        case 64: return LaunchF<N, D, 64>::occ(a);
+        default: if constexpr (D >= 128) { if (a.Gv == 128) return LaunchF<N, D, 128>::occ(a); }
     }
     return 1;
 }

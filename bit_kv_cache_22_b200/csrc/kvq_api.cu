@@ -89,9 +89,10 @@ kvq_status validate(const kvq_config *c) {
     return KVQ_OK;
 }
 
+// Splits over the quantized tiles are at most kMaxSplits; the residual adds one.
 int max_splits(const kvq_config *c) {
-    const int64_t tiles = c->capacity / 16 + c->residual / 16;
-    return static_cast<int>(tiles < kMaxSplits ? tiles : kMaxSplits);
+    const int64_t tiles = c->capacity / 16;
+    return static_cast<int>(tiles < kMaxSplits ? tiles : kMaxSplits) + 1;
 }
 
 }  // namespace
@@ -108,36 +109,42 @@ struct kvq_cache {
 
 namespace {
 
-// Split count for the current cache length.  A CTA's time is modelled as its
-// tiles per warp plus a fixed start/finish cost of ~3 tiles; the kernel's time
-// as that times the number of waves of CTAs over the GPU's resident slots.
-// The split count with the lowest modelled time wins (ties: fewer splits).
-void plan_splits(const kvq_cache *h, int *S_out, int *tiles_per_split) {
+// Split count for the current cache length.  The quantized tiles are cut into
+// n_qsplits contiguous splits; the residual rows (if any) get one split of
+// their own.  A quantized split's time is modelled as its tiles per warp plus a
+// fixed start/finish cost of ~3 tiles, the kernel's time as that times the
+// number of waves of CTAs over the GPU's resident slots; the split count with
+// the lowest modelled time wins (ties: fewer splits).
+void plan_splits(const kvq_cache *h, int *n_qsplits, int *tiles_per_split, int *S_out) {
     const kvq_config &c = h->cfg;
-    const int64_t tiles = h->Tq / 16 + (h->r + 15) / 16;
-    const int64_t units = static_cast<int64_t>(c.batch) * c.q_heads;
+    const int64_t tiles = h->Tq / 16;
+    const int extra = h->r > 0 ? 1 : 0;
+    // CTAs per split: one per query head, or one per kv head on the grouped-query path
+    const int64_t units = static_cast<int64_t>(c.batch) *
+                          (c.q_heads == 4 * c.kv_heads ? c.kv_heads : c.q_heads);
     const int64_t slots = static_cast<int64_t>(h->num_sms) * h->ctas_per_sm;
-    int64_t cap = (tiles + kMinTilesPerSplit - 1) / kMinTilesPerSplit;
-    if (cap > max_splits(&c)) cap = max_splits(&c);
-    if (cap > h->split_limit) cap = h->split_limit;
-    if (cap < 1) cap = 1;
-    int64_t best_S = 1, best_per = tiles > 0 ? tiles : 1;
-    double best_cost = -1.0;
-    for (int64_t S = 1; S <= cap; ++S) {
-        int64_t per = (tiles + S - 1) / S;
-        if (per < 1) per = 1;
-        const int64_t S_eff = (tiles + per - 1) / per;
-        if (S_eff != S) continue;
-        const int64_t waves = (units * S + slots - 1) / slots;
-        const double cost = static_cast<double>(waves) * ((per + 3) / 4 + 3);
-        if (best_cost < 0 || cost < best_cost) {
-            best_cost = cost;
-            best_S = S;
-            best_per = per;
+    int64_t best_S = 0, best_per = 1;
+    if (tiles > 0) {
+        int64_t cap = (tiles + kMinTilesPerSplit - 1) / kMinTilesPerSplit;
+        if (cap > max_splits(&c) - 1) cap = max_splits(&c) - 1;
+        if (cap > h->split_limit) cap = h->split_limit;
+        if (cap < 1) cap = 1;
+        double best_cost = -1.0;
+        for (int64_t S = 1; S <= cap; ++S) {
+            const int64_t per = (tiles + S - 1) / S;
+            if ((tiles + per - 1) / per != S) continue;
+            const int64_t waves = (units * (S + extra) + slots - 1) / slots;
+            const double cost = static_cast<double>(waves) * ((per + 3) / 4 + 3);
+            if (best_cost < 0 || cost < best_cost) {
+                best_cost = cost;
+                best_S = S;
+                best_per = per;
+            }
         }
     }
-    *S_out = static_cast<int>(best_S);
+    *n_qsplits = static_cast<int>(best_S);
     *tiles_per_split = static_cast<int>(best_per);
+    *S_out = static_cast<int>(best_S + extra);
 }
 
 kvq::DecodeArgs decode_args(const kvq_cache *h) {
@@ -162,6 +169,7 @@ kvq::DecodeArgs decode_args(const kvq_cache *h) {
     a.bits = c.bits;
     a.sym = c.symmetric != 0;
     a.bf16 = c.dtype == KVQ_BF16;
+    a.gqa = c.q_heads == 4 * c.kv_heads;
     a.gshift = 0;
     while ((16 << a.gshift) < c.group_k) ++a.gshift;
     a.qscale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c.head_dim)));
@@ -278,13 +286,10 @@ kvq_status kvq_prefill_quantize(kvq_cache *h, const void *X_K, const void *X_V, 
     if (e != cudaSuccess) return cuda_fail(e, "prefill quantize launch");
     const int64_t BH = static_cast<int64_t>(c.batch) * c.kv_heads;
     const int64_t rstride = static_cast<int64_t>(c.residual) * c.head_dim;
-    e = kvq::launch_copy_rows(static_cast<const uint16_t *>(X_K), T * c.head_dim, Tq,
-                              static_cast<uint16_t *>(h->buf.k_residual), rstride, 0, r, BH,
+    e = kvq::launch_copy_rows(static_cast<const uint16_t *>(X_K), static_cast<const uint16_t *>(X_V),
+                              T * c.head_dim, Tq, static_cast<uint16_t *>(h->buf.k_residual),
+                              static_cast<uint16_t *>(h->buf.v_residual), rstride, 0, r, BH,
                               c.head_dim, s);
-    if (e == cudaSuccess)
-        e = kvq::launch_copy_rows(static_cast<const uint16_t *>(X_V), T * c.head_dim, Tq,
-                                  static_cast<uint16_t *>(h->buf.v_residual), rstride, 0, r, BH,
-                                  c.head_dim, s);
     if (e != cudaSuccess) return cuda_fail(e, "prefill residual copy launch");
     h->Tq = Tq;
     h->r = static_cast<int32_t>(r);
@@ -303,13 +308,10 @@ kvq_status kvq_append(kvq_cache *h, const void *t_K, const void *t_V, void *stre
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t BH = static_cast<int64_t>(c.batch) * c.kv_heads;
     const int64_t rstride = static_cast<int64_t>(c.residual) * c.head_dim;
-    cudaError_t e = kvq::launch_copy_rows(static_cast<const uint16_t *>(t_K), c.head_dim, 0,
-                                          static_cast<uint16_t *>(h->buf.k_residual), rstride,
-                                          h->r, 1, BH, c.head_dim, s);
-    if (e == cudaSuccess)
-        e = kvq::launch_copy_rows(static_cast<const uint16_t *>(t_V), c.head_dim, 0,
-                                  static_cast<uint16_t *>(h->buf.v_residual), rstride, h->r, 1, BH,
-                                  c.head_dim, s);
+    cudaError_t e = kvq::launch_copy_rows(
+        static_cast<const uint16_t *>(t_K), static_cast<const uint16_t *>(t_V), c.head_dim, 0,
+        static_cast<uint16_t *>(h->buf.k_residual), static_cast<uint16_t *>(h->buf.v_residual),
+        rstride, h->r, 1, BH, c.head_dim, s);
     if (e != cudaSuccess) return cuda_fail(e, "append launch");
     if (flush) {
         kvq::QuantizeArgs q = quantize_args(h);
@@ -339,8 +341,8 @@ kvq_status kvq_set_split_limit(kvq_cache *h, int32_t max_splits) {
 
 int32_t kvq_decode_splits(const kvq_cache *h) {
     if (!h) return 0;
-    int S, per;
-    plan_splits(h, &S, &per);
+    int nq, per, S;
+    plan_splits(h, &nq, &per, &S);
     return S;
 }
 
@@ -357,7 +359,7 @@ kvq_status kvq_decode_attention(kvq_cache *h, const void *t_Q, float *t_O, void 
         return fail(KVQ_ERR_INVALID_ARG, "workspace needs %zu bytes, got %zu", sz.workspace,
                     workspace_bytes);
     kvq::DecodeArgs a = decode_args(h);
-    plan_splits(h, &a.S, &a.tiles_per_split);
+    plan_splits(h, &a.n_qsplits, &a.tiles_per_split, &a.S);
     const int64_t units = static_cast<int64_t>(c.batch) * c.q_heads;
     float *ws = static_cast<float *>(workspace);
     a.o_part = ws;

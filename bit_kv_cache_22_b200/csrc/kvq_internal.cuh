@@ -46,10 +46,12 @@ struct QuantizeArgs {
 };
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s);
 
-// dst[bh][dst_row0 + i][:] = src[bh][src_row0 + i][:] for i < rows (e elements)
-cudaError_t launch_copy_rows(const uint16_t *src, int64_t src_bh_stride, int64_t src_row0,
-                             uint16_t *dst, int64_t dst_bh_stride, int64_t dst_row0,
-                             int64_t rows, int64_t BH, int d, cudaStream_t s);
+// For both (src, dst) pairs: dst[bh][dst_row0 + i][:] = src[bh][src_row0 + i][:],
+// i < rows (e elements); one launch.
+cudaError_t launch_copy_rows(const uint16_t *src0, const uint16_t *src1, int64_t src_bh_stride,
+                             int64_t src_row0, uint16_t *dst0, uint16_t *dst1,
+                             int64_t dst_bh_stride, int64_t dst_row0, int64_t rows, int64_t BH,
+                             int d, cudaStream_t s);
 
 struct DecodeArgs {
     const uint32_t *kc, *vc;
@@ -63,10 +65,12 @@ struct DecodeArgs {
     int B, Hq, Hkv, d, G, Gv, R, bits;
     int gshift;                  // log2(G / 16): key groups are 2^gshift tiles
     bool sym, bf16;
+    bool gqa;                    // 4 query heads per kv head: tensor-core kernel, grid over kv heads
     int n_qtiles;                // Tq / 16
     int r;                       // residual rows
-    int tiles_per_split;
-    int S;
+    int tiles_per_split;         // quantized tiles per split
+    int n_qsplits;               // splits over the quantized tiles
+    int S;                       // n_qsplits + (r > 0)
     float qscale;                // log2(e) / sqrt(d)
 };
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);

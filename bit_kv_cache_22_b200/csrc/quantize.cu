@@ -44,9 +44,24 @@ __device__ __forceinline__ GroupParams asym_params(float mn, float mx, int bits)
     return {s, static_cast<int>(zf)};
 }
 
-__device__ __forceinline__ int asym_code(float x, GroupParams p, int bits) {
+// round(x / s) (half to even, of the correctly rounded fp32 quotient) as an int,
+// for |x / s| < 2^21.  With rinv = RN(1/s), q = RN(x * rinv) is within
+// |q| * 2^-22 of RN(x / s), so both round to the same integer unless q lies
+// within that distance of a half-integer; only those elements (margin 4x) pay
+// for the IEEE division.
+__device__ __forceinline__ int rint_quotient(float x, float s, float rinv) {
+    const float q = x * rinv;
+    const float t = q + 12582912.0f;                  // 1.5 * 2^23: rounds q to an integer
+    const float k = t - 12582912.0f;
+    const float dist = fabsf(fabsf(q - k) - 0.5f);
+    if (dist <= fabsf(q) * 0x1p-20f + 0x1p-126f)
+        return static_cast<int>(rintf(__fdiv_rn(x, s)));
+    return __float_as_int(t) - 0x4B400000;
+}
+
+__device__ __forceinline__ int asym_code(float x, GroupParams p, float rinv, int bits) {
     const int L = (1 << bits) - 1;
-    int q = static_cast<int>(rintf(__fdiv_rn(x, p.s))) + p.z;
+    int q = rint_quotient(x, p.s, rinv) + p.z;
     return min(max(q, 0), L);
 }
 
@@ -55,10 +70,10 @@ __device__ __forceinline__ float sym_scale(float amax, int bits) {
     return __fdiv_rn(__fmul_rn(2.0f, amax), L);
 }
 
-__device__ __forceinline__ int sym_code(float x, float s, int bits) {
+__device__ __forceinline__ int sym_code(float x, float s, float rinv, int bits) {
     const int half = 1 << (bits - 1);
     if (s == 0.0f) return half;
-    int q = static_cast<int>(rintf(__fdiv_rn(x, s)));
+    int q = rint_quotient(x, s, rinv);
     q = min(max(q, -half), half - 1);
     return q + half;
 }
@@ -110,6 +125,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
     float *red = reinterpret_cast<float *>(codes + static_cast<size_t>(G) * d);  // 2*256
     float *ch_s = red + 2 * kQuantThreads;                                   // [d]
     int *ch_z = reinterpret_cast<int *>(ch_s + d);                           // [d]
+    float *ch_r = reinterpret_cast<float *>(ch_z + d);                       // [d] 1/s
 
     const int64_t grp = blockIdx.x;
     const int64_t bh = blockIdx.y;
@@ -159,13 +175,15 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
             a.ks[(bh * groups_cap + out_tok / G) * d + c] = s;
             ch_s[c] = s;
             ch_z[c] = z;
+            ch_r[c] = s != 0.0f ? __frcp_rn(s) : 0.0f;
         }
         __syncthreads();
         for (int e = threadIdx.x; e < G * d; e += blockDim.x) {
             const int c2 = e % d;
             const float x = widen(xs[e], a.bf16);
-            codes[e] = static_cast<uint8_t>(
-                a.sym ? sym_code(x, ch_s[c2], bits) : asym_code(x, {ch_s[c2], ch_z[c2]}, bits));
+            const float sc = ch_s[c2], ri = ch_r[c2];
+            codes[e] = static_cast<uint8_t>(a.sym ? sym_code(x, sc, ri, bits)
+                                                  : asym_code(x, {sc, ch_z[c2]}, ri, bits));
         }
         __syncthreads();
         pack_tiles(codes, G / 16, d, bits, false,
@@ -213,9 +231,10 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
                 a.vs[mi] = s;
                 if (!a.sym) a.vz[mi] = static_cast<int16_t>(z);
             }
+            const float ri = s != 0.0f ? __frcp_rn(s) : 0.0f;
             for (int e = 0; e < per_lane; ++e)
                 codes[t * d + lane * per_lane + e] = static_cast<uint8_t>(
-                    a.sym ? sym_code(x[e], s, bits) : asym_code(x[e], {s, z}, bits));
+                    a.sym ? sym_code(x[e], s, ri, bits) : asym_code(x[e], {s, z}, ri, bits));
         }
         __syncthreads();
         pack_tiles(codes, G / 16, d, bits, true,
@@ -223,20 +242,25 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
     }
 }
 
-__global__ void copy_rows_kernel(const uint16_t *src, int64_t src_bh_stride, int64_t src_row0,
-                                 uint16_t *dst, int64_t dst_bh_stride, int64_t dst_row0,
-                                 int64_t rows, int64_t BH, int d) {
+__global__ void copy_rows_kernel(const uint16_t *src0, const uint16_t *src1, int64_t src_bh_stride,
+                                 int64_t src_row0, uint16_t *dst0, uint16_t *dst1,
+                                 int64_t dst_bh_stride, int64_t dst_row0, int64_t rows,
+                                 int64_t BH, int d) {
     const int64_t vec_per_row = d / 8;
-    const int64_t total = BH * rows * vec_per_row;
-    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+    const int64_t per_pair = BH * rows * vec_per_row;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < 2 * per_pair;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t v = i % vec_per_row;
-        const int64_t row = (i / vec_per_row) % rows;
-        const int64_t bh = i / (vec_per_row * rows);
-        const uint4 *s = reinterpret_cast<const uint4 *>(src + bh * src_bh_stride +
-                                                         (src_row0 + row) * d) + v;
-        uint4 *t = reinterpret_cast<uint4 *>(dst + bh * dst_bh_stride + (dst_row0 + row) * d) + v;
-        *t = *s;
+        const bool second = i >= per_pair;
+        const int64_t k = second ? i - per_pair : i;
+        const int64_t v = k % vec_per_row;
+        const int64_t row = (k / vec_per_row) % rows;
+        const int64_t bh = k / (vec_per_row * rows);
+        const uint16_t *src = second ? src1 : src0;
+        uint16_t *dst = second ? dst1 : dst0;
+        const uint4 *sp = reinterpret_cast<const uint4 *>(src + bh * src_bh_stride +
+                                                          (src_row0 + row) * d) + v;
+        uint4 *tp = reinterpret_cast<uint4 *>(dst + bh * dst_bh_stride + (dst_row0 + row) * d) + v;
+        *tp = *sp;
     }
 }
 
@@ -244,7 +268,7 @@ __global__ void copy_rows_kernel(const uint16_t *src, int64_t src_bh_stride, int
 
 size_t quantize_smem_bytes(int d, int G) {
     return static_cast<size_t>(G) * d * 3 + 2 * kQuantThreads * sizeof(float) +
-           static_cast<size_t>(d) * 8;
+           static_cast<size_t>(d) * 12;
 }
 
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s) {
@@ -267,15 +291,16 @@ cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_copy_rows(const uint16_t *src, int64_t src_bh_stride, int64_t src_row0,
-                             uint16_t *dst, int64_t dst_bh_stride, int64_t dst_row0,
-                             int64_t rows, int64_t BH, int d, cudaStream_t s) {
-    const int64_t total = BH * rows * (d / 8);
+cudaError_t launch_copy_rows(const uint16_t *src0, const uint16_t *src1, int64_t src_bh_stride,
+                             int64_t src_row0, uint16_t *dst0, uint16_t *dst1,
+                             int64_t dst_bh_stride, int64_t dst_row0, int64_t rows, int64_t BH,
+                             int d, cudaStream_t s) {
+    const int64_t total = 2 * BH * rows * (d / 8);
     if (total == 0) return cudaSuccess;
     const int threads = 256;
     const int64_t blocks = (total + threads - 1) / threads;
     copy_rows_kernel<<<static_cast<unsigned>(blocks < 65536 ? blocks : 65536), threads, 0, s>>>(
-        src, src_bh_stride, src_row0, dst, dst_bh_stride, dst_row0, rows, BH, d);
+        src0, src1, src_bh_stride, src_row0, dst0, dst1, dst_bh_stride, dst_row0, rows, BH, d);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -170,10 +170,11 @@ KVQ_API kvq_status kvq_cache_state(const kvq_cache *cache, int64_t *quantized_to
                            int32_t *residual_tokens);
 
 /*
- * Upper bound on the token splits of kvq_decode_attention (1 .. 64; 0 restores
- * the default of 64).  Fewer splits mean fewer partial results to merge, more
- * splits more parallelism for short batches; the result is the same up to
- * fp32 rounding.
+ * Upper bound on the splits kvq_decode_attention cuts the quantized tokens into
+ * (1 .. 64; 0 restores the default of 64); the residual tokens, when there are
+ * any, always form one more split of their own.  Fewer splits mean fewer
+ * partial results to merge, more splits more parallelism for short batches;
+ * the result is the same up to fp32 rounding.
  */
 KVQ_API kvq_status kvq_set_split_limit(kvq_cache *cache, int32_t max_splits);
 
