@@ -508,11 +508,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_split_kernel(const D
 //            first n-tile and 2h (signed digit 2) in the second; int32 sums,
 //            exact.  The digits are built once per key group, cooperatively by
 //            the warp (lane l: head l/8, 16 channels), in shared memory.
-//   values : f16 MMA m16n8k16.  A = value codes as exact f16 (rows = channels,
-//            k = tokens; bytes 0,2 and 1,3 of a masked word are f16x2 pairs via
-//            the 0x6400 exponent trick); B = p_t s_{t,gv} split into f16 hi +
-//            lo parts (columns 2h, 2h+1), built cooperatively per tile; fp32
-//            accumulators, rescaled when a head's running maximum grows.
+//   values : bf16 MMA m16n8k16.  A = value codes as exact bf16 (rows = channels,
+//            k = tokens; bytes 0,2 and 1,3 of a word slot are bf16x2 pairs via
+//            the 0x4300 exponent trick); B = p_t s_{t,gv} split into bf16 hi +
+//            lo parts (columns 2h, 2h+1; bf16 keeps fp32's exponent range, so
+//            the tiny probabilities of long contexts do not underflow), built
+//            cooperatively per tile; fp32 accumulators, rescaled when a head's
+//            running maximum grows.
 //   z-terms: bias_g = sum_c q'_c z_{g,c} and sum_t p_t s_t z_t in fp32.
 // Residual rows form the last split, where each warp serves one query head
 // with exact e values on CUDA cores.
@@ -533,57 +535,43 @@ __device__ __forceinline__ void imma_us(int (&d)[4], const uint32_t (&a)[4], uin
 }
 __device__ __forceinline__ void hmma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                      uint32_t b0, uint32_t b1) {
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-// f16x2 arithmetic on raw registers
-__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
+// (lo, hi) floats -> bf16x2 (round to nearest)
+__device__ __forceinline__ uint32_t f2bf2(float lo, float hi) {
     uint32_t d;
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
     return d;
-}
-__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
-    uint32_t d;
-    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
-}
-// (lo, hi) floats -> f16x2 (round to nearest)
-__device__ __forceinline__ uint32_t f2h2(float lo, float hi) {
-    uint32_t d;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
-    return d;
-}
-__device__ __forceinline__ float2 h22f(uint32_t h) {
-    __half2_raw r;
-    r.x = static_cast<unsigned short>(h & 0xffffu);
-    r.y = static_cast<unsigned short>(h >> 16);
-    return __half22float2(__half2(r));
 }
 
-// Codes of a masked-word slot as two exact f16x2 registers: (byte 0, byte 2), (byte 1, byte 3).
-// 0x6400 is the f16 1024 with unit mantissa steps; a code OR-ed into the low
-// mantissa bits gives 1024 + code.  For 2-bit codes the byte-1/3 codes sit at
-// mantissa bits 8-9 (1024 + 256 code, rescaled by one f16x2 FMA); 4-bit codes
-// there would reach the exponent, so they are shifted down first.
+// Codes of one slot of a value word as two bf16x2 registers, (byte 0, byte 2)
+// and (byte 1, byte 3), each element equal to 2^(7-N) * (2^N + code) exactly:
+// the code is shifted to the top N mantissa bits of 0x4300 (bf16 128, unit
+// mantissa steps).  The 2^N offset is small next to the code range, so it is
+// kept: the value MMA accumulates sum_t b_t (2^N + code) and the z-term uses
+// z + 2^N instead of z; the 2^(7-N) factor is folded into the B operand.
 template <int N>
-__device__ __forceinline__ void codes_f16(uint32_t xs, uint32_t magic16, uint32_t &r02, uint32_t &r13) {
+__device__ __forceinline__ void codes_bf16(uint32_t w, int slot, uint32_t magic16, uint32_t &r02,
+                                           uint32_t &r13) {
     constexpr uint32_t L = (1u << N) - 1u;
-    r02 = hsub2(and_or(xs, L | (L << 16), magic16), magic16);                  // (1024 + c) - 1024
-    if constexpr (N == 2)
-        r13 = hfma2(and_or(xs, (L << 8) | (L << 24), magic16), 0x1C001C00u,    // (1024 + 256c)/256 - 4
-                    0xC400C400u);
-    else
-        r13 = hsub2(and_or(xs >> 8, L | (L << 16), magic16), magic16);
+    constexpr uint32_t M = (L << (7 - N)) | (L << (23 - N));
+    const int up = 7 - N - N * slot;                  // byte 0/2 code: bit N*slot -> 7 - N
+    const uint32_t x02 = up >= 0 ? (w << up) : (w >> -up);
+    const uint32_t x13 = w >> (N * slot + N + 1);     // byte 1/3 code: bit 8 + N*slot -> 7 - N
+    r02 = and_or(x02, M, magic16);
+    r13 = and_or(x13, M, magic16);
 }
 
 template <int N, int D, int GV>
 struct GqaSmem {
     static constexpr int NGV = D / GV;
     static constexpr int kStageBytes = kStages * Stage<N, D, GV>::kBytes;
-    static constexpr int kKd = kStageBytes;                  // key digits [3][4 heads][D] bytes
-    static constexpr int kVb = kKd + 3 * kGqa * D;           // value B [NGV][4][2][16] f16
+    static constexpr int kKdRow = D + 16;                    // padded: the 8 B-fragment rows hit distinct banks
+    static constexpr int kKd = kStageBytes;                  // key digits [3][4 heads][kKdRow] bytes
+    static constexpr int kVb = kKd + 3 * kGqa * kKdRow;      // value B [NGV][4][2][16] bf16
     static constexpr int kPs = kVb + NGV * kGqa * 2 * 16 * 2; // p [4][16] f32
     static constexpr int kAl = kPs + kGqa * 16 * 4;          // alpha [4], key scale [4], bias [4]
     static constexpr int kWarpBytes = kAl + 16 * 4;
@@ -617,7 +605,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_gqa_kernel(const Dec
     float *ps = reinterpret_cast<float *>(wmem + Sm::kPs);
     float *al = reinterpret_cast<float *>(wmem + Sm::kAl);
     const uint32_t magic = kMagicBits;
-    const uint32_t magic16 = 0x64006400u;
+    const uint32_t magic16 = 0x43004300u;    // bf16 128 in both halves
 
     for (int i = threadIdx.x; i < kGqa * D; i += kDecodeThreads)
         q_s[i / D][i % D] = widen(a.q[bq0 * D + i], a.bf16) * a.qscale;
@@ -841,7 +829,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_gqa_kernel(const Dec
             }
 #pragma unroll
             for (int k = 0; k < 3; ++k)
-                *reinterpret_cast<uint4 *>(kd + (k * kGqa + hb) * D + 16 * lb) =
+                *reinterpret_cast<uint4 *>(kd + (k * kGqa + hb) * Sm::kKdRow + 16 * lb) =
                     make_uint4(dw[k][0], dw[k][1], dw[k][2], dw[k][3]);
             if (lb == 0) {
                 al[4 + hb] = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
@@ -849,8 +837,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_gqa_kernel(const Dec
             }
             __syncwarp();
             // B fragments: column g8 = head g8/2, digit g8%2 (first n-tile), digit 2 for even g8
-            const uint32_t *kdw0 = reinterpret_cast<const uint32_t *>(kd + ((g8 & 1) * kGqa + (g8 >> 1)) * D);
-            const uint32_t *kdw2 = reinterpret_cast<const uint32_t *>(kd + (2 * kGqa + (g8 >> 1)) * D);
+            const uint32_t *kdw0 =
+                reinterpret_cast<const uint32_t *>(kd + ((g8 & 1) * kGqa + (g8 >> 1)) * Sm::kKdRow);
+            const uint32_t *kdw2 = reinterpret_cast<const uint32_t *>(kd + (2 * kGqa + (g8 >> 1)) * Sm::kKdRow);
 #pragma unroll
             for (int mk = 0; mk < NK; ++mk) {
                 kb0[mk][0] = kdw0[8 * mk + t4];
@@ -910,20 +899,31 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_gqa_kernel(const Dec
 
         // ---- value B: lane builds head hb, tokens 4q + e and 4q + e + 2 ----
         {
+            constexpr float kBscale = 1.0f / static_cast<float>(1 << (7 - N));
+            constexpr int kOff = 1 << N;              // code offset carried by the f16 A operand
             const int q4 = lb >> 1, e = lb & 1;
             const int ta = 4 * q4 + e, tb = ta + 2;
-            const float pa = ps[hb * 16 + ta], pb = ps[hb * 16 + tb];
+            const float pa = ps[hb * 16 + ta] * kBscale, pb = ps[hb * 16 + tb] * kBscale;
             const float *vsp = reinterpret_cast<const float *>(st + St::kVs);
             const int16_t *vzp = reinterpret_cast<const int16_t *>(st + St::kVz);
+            float sa[NGV], sb[NGV];
+            int16_t zza[NGV], zzb[NGV];
 #pragma unroll
             for (int v = 0; v < NGV; ++v) {
-                const float xa = pa * vsp[ta * NGV + v], xb = pb * vsp[tb * NGV + v];
-                const float za = a.sym ? static_cast<float>(zsym) : small_int_to_float(vzp[ta * NGV + v]);
-                const float zb = a.sym ? static_cast<float>(zsym) : small_int_to_float(vzp[tb * NGV + v]);
+                sa[v] = vsp[ta * NGV + v];
+                sb[v] = vsp[tb * NGV + v];
+                zza[v] = a.sym ? static_cast<int16_t>(zsym) : vzp[ta * NGV + v];
+                zzb[v] = a.sym ? static_cast<int16_t>(zsym) : vzp[tb * NGV + v];
+            }
+#pragma unroll
+            for (int v = 0; v < NGV; ++v) {
+                const float xa = pa * sa[v], xb = pb * sb[v];
+                const float za = small_int_to_float(zza[v] + kOff);
+                const float zb = small_int_to_float(zzb[v] + kOff);
                 zsum[v] = fmaf(xa, za, fmaf(xb, zb, zsum[v]));
-                const uint32_t hi = f2h2(xa, xb);
-                const float2 hf = h22f(hi);
-                const uint32_t lo = f2h2(xa - hf.x, xb - hf.y);
+                const uint32_t hi = f2bf2(xa, xb);
+                const uint32_t lo =
+                    f2bf2(xa - __uint_as_float(hi << 16), xb - __uint_as_float(hi & 0xffff0000u));
                 uint32_t *dst = reinterpret_cast<uint32_t *>(vb + ((v * kGqa + hb) * 2) * 16);
                 dst[(4 * q4 + 2 * e) >> 1] = hi;          // part 0 plane
                 dst[(16 + 4 * q4 + 2 * e) >> 1] = lo;     // part 1 plane
@@ -936,11 +936,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_gqa_kernel(const Dec
         load_stage_words<W>(reinterpret_cast<const uint32_t *>(st + St::kCodes), lane, vw);
 #pragma unroll
         for (int j = 0; j < NJ; ++j) {
-            const uint32_t x0 = vw[j / BPW] >> (N * (2 * (j % BPW)));
-            const uint32_t x1 = vw[j / BPW] >> (N * (2 * (j % BPW) + 1));
             uint32_t a02, a13, b02, b13;
-            codes_f16<N>(x0, magic16, a02, a13);      // channel 16j + g8
-            codes_f16<N>(x1, magic16, b02, b13);      // channel 16j + g8 + 8
+            codes_bf16<N>(vw[j / BPW], 2 * (j % BPW), magic16, a02, a13);       // channel 16j + g8
+            codes_bf16<N>(vw[j / BPW], 2 * (j % BPW) + 1, magic16, b02, b13);   // channel 16j + g8 + 8
             const uint2 bb = *reinterpret_cast<const uint2 *>(
                 vb + (((16 * j) / GV * kGqa + (g8 >> 1)) * 2 + (g8 & 1)) * 16 + 4 * t4);
             hmma(dv[j], a02, b02, a13, b13, bb.x, bb.y);
@@ -965,12 +963,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_gqa_kernel(const Dec
     float *zs_s = o_s + kDecodeWarps * kGqa * D;          // [warp][head][NGV]
     if (lb == 0)
         for (int v = 0; v < NGV; ++v) zs_s[(warp * kGqa + hb) * NGV + v] = zsum[v];
+    // dv sums A * B = (2^N + code) p s; zsum sums b (2^N + z) with b = p s 2^-(7-N)
     __syncwarp();
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
         const float z = zs_s[(warp * kGqa + t4) * NGV + (16 * j) / GV];
-        o_s[(warp * kGqa + t4) * D + 16 * j + g8] = dv[j][0] + dv[j][1] - z;
-        o_s[(warp * kGqa + t4) * D + 16 * j + g8 + 8] = dv[j][2] + dv[j][3] - z;
+        constexpr float kUnscale = static_cast<float>(1 << (7 - N));
+        o_s[(warp * kGqa + t4) * D + 16 * j + g8] = dv[j][0] + dv[j][1] - z * kUnscale;
+        o_s[(warp * kGqa + t4) * D + 16 * j + g8 + 8] = dv[j][2] + dv[j][3] - z * kUnscale;
     }
     if (g8 == 0) {
         ml_s[warp][t4][0] = m;
