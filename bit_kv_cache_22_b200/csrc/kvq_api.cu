@@ -12,6 +12,7 @@
 #include <cstdio>
 #include <cstring>
 #include <atomic>
+#include <mutex>
 #include <new>
 #include <string>
 
@@ -362,6 +363,78 @@ kvq_status kvq_decode_attention(kvq_cache *h, const void *t_Q, float *t_O, void 
     plan_splits(h, &a.n_qsplits, &a.tiles_per_split, &a.S);
     const int64_t units = static_cast<int64_t>(c.batch) * c.q_heads;
     float *ws = static_cast<float *>(workspace);
+    a.o_part = ws;
+    a.m_part = ws + units * a.S * c.head_dim;
+    a.l_part = a.m_part + units * a.S;
+    a.q = static_cast<const uint16_t *>(t_Q);
+    a.out = t_O;
+    a.n_qtiles = static_cast<int>(h->Tq / 16);
+    a.r = h->r;
+    cudaError_t e = kvq::launch_decode(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    return ok();
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode attention without a caller-provided workspace.
+//
+// The split partials live in one file-scope device array instead of caller
+// memory.  Host code cannot use the array's name as a device address (it is a
+// host-side stand-in for the symbol), so the address is looked up with
+// cudaGetSymbolAddress once per device, with that device current, the first
+// time the entry point runs on it.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchFloats = size_t{1} << 20;   // 4 MiB per device
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+
+std::mutex g_noalloc_mutex;
+float *g_noalloc_ptr[kMaxDevices] = {};
+
+kvq_status noalloc_scratch(float **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "querying the current device");
+    if (dev < 0 || dev >= kMaxDevices)
+        return fail(KVQ_ERR_UNSUPPORTED, "device ordinal %d is beyond %d", dev, kMaxDevices);
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "looking up the static decode scratch");
+        g_noalloc_ptr[dev] = static_cast<float *>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return KVQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_decode_attention_noalloc(kvq_cache *h, const void *t_Q, float *t_O, void *stream) {
+    if (!h) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+    if (!t_Q || !t_O || !aligned16(t_Q) || !aligned16(t_O))
+        return fail(KVQ_ERR_INVALID_ARG, "t_Q and t_O must be non-NULL and 16-byte aligned");
+    if (h->Tq == 0 && h->r == 0) return fail(KVQ_ERR_STATE, "the cache is empty");
+    const kvq_config &c = h->cfg;
+    kvq::DecodeArgs a = decode_args(h);
+    plan_splits(h, &a.n_qsplits, &a.tiles_per_split, &a.S);
+    const int64_t units = static_cast<int64_t>(c.batch) * c.q_heads;
+    const size_t need = static_cast<size_t>(units) * a.S * (c.head_dim + 2);
+    if (need > kNoAllocScratchFloats)
+        return fail(KVQ_ERR_CAPACITY,
+                    "this decode needs %zu bytes of scratch but the static scratch holds %zu; "
+                    "use kvq_decode_attention with a workspace",
+                    need * sizeof(float), kNoAllocScratchFloats * sizeof(float));
+    float *ws = nullptr;
+    kvq_status st = noalloc_scratch(&ws);
+    if (st != KVQ_OK) return st;
     a.o_part = ws;
     a.m_part = ws + units * a.S * c.head_dim;
     a.l_part = a.m_part + units * a.S;

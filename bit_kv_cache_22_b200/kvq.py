@@ -29,7 +29,7 @@ KVQ_FP16, KVQ_BF16 = 0, 1
 
 EXPORTED = ("kvq_get_sizes", "kvq_create", "kvq_destroy", "kvq_reset", "kvq_prefill_quantize",
             "kvq_append", "kvq_decode_attention", "kvq_cache_state", "kvq_set_split_limit",
-            "kvq_decode_splits", "kvq_kernel_launches",
+            "kvq_decode_splits", "kvq_kernel_launches", "kvq_decode_attention_noalloc",
             "kvq_last_error", "kvq_layout_version")
 
 
@@ -84,6 +84,8 @@ def load() -> ctypes.CDLL:
         lib.kvq_prefill_quantize.argtypes = [P, P, P, i64, P]
         lib.kvq_append.argtypes = [P, P, P, P]
         lib.kvq_decode_attention.argtypes = [P, P, P, P, sz, P]
+        lib.kvq_decode_attention_noalloc.argtypes = [P, P, P, P]
+        lib.kvq_decode_attention_noalloc.restype = ctypes.c_int
         lib.kvq_cache_state.argtypes = [P, ctypes.POINTER(i64), ctypes.POINTER(i32)]
         lib.kvq_set_split_limit.argtypes = [P, i32]
         lib.kvq_decode_splits.argtypes = [P]

@@ -165,6 +165,28 @@ KVQ_API kvq_status kvq_append(kvq_cache *cache, const void *t_K, const void *t_V
 KVQ_API kvq_status kvq_decode_attention(kvq_cache *cache, const void *t_Q, float *t_O,
                                 void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Decode attention that allocates nothing and takes no workspace (the pages
+ * have no counterpart: this is an interface for callers that cannot allocate
+ * device memory -- for instance code that runs while another framework owns
+ * every allocation on the device, a plugin host that forbids cudaMalloc, or a
+ * latency-bound loop that must not hit the allocator).  Same inputs, outputs
+ * and result as kvq_decode_attention; the per-split partial results go to a
+ * fixed 4 MiB device array inside the library (allocated once per device that
+ * loads the library and held until the process exits).
+ *  - Calls whose partials would exceed 4 MiB (B * Hq * splits * (d + 2) * 4
+ *    bytes, splits as reported by kvq_decode_splits) return KVQ_ERR_CAPACITY
+ *    and launch nothing.
+ *  - All calls on a device share that array: calls whose kernels may overlap
+ *    on the GPU (different streams without ordering) race and give undefined
+ *    results.  Nothing in it needs to start at zero; every call writes the
+ *    partials it reads.
+ *  - The first call on each device looks up the array's device address (with
+ *    that device current); make that first call before any stream capture.
+ */
+KVQ_API kvq_status kvq_decode_attention_noalloc(kvq_cache *cache, const void *t_Q, float *t_O,
+                                                void *stream);
+
 /* Current counters: quantized tokens Tq and residual tokens r. */
 KVQ_API kvq_status kvq_cache_state(const kvq_cache *cache, int64_t *quantized_tokens,
                            int32_t *residual_tokens);
