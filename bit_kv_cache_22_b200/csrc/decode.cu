@@ -565,18 +565,52 @@ __device__ __forceinline__ void codes_bf16(uint32_t w, int slot, uint32_t magic1
     r13 = and_or(x13, M, magic16);
 }
 
+// Shared-memory stages of the grouped-query kernel (it consumes two tiles per
+// iteration, so it keeps a deeper ring when a stage is small).
+template <int N>
+__host__ __device__ constexpr int gqa_stages() { return N == 2 ? 6 : 4; }
+
 template <int N, int D, int GV>
 struct GqaSmem {
     static constexpr int NGV = D / GV;
-    static constexpr int kStageBytes = kStages * Stage<N, D, GV>::kBytes;
+    static constexpr int kStageBytes = gqa_stages<N>() * Stage<N, D, GV>::kBytes;
     static constexpr int kKdRow = D + 16;                    // padded: the 8 B-fragment rows hit distinct banks
     static constexpr int kKd = kStageBytes;                  // key digits [3][4 heads][kKdRow] bytes
-    static constexpr int kVb = kKd + 3 * kGqa * kKdRow;      // value B [NGV][4][2][16] bf16
-    static constexpr int kPs = kVb + NGV * kGqa * 2 * 16 * 2; // p [4][16] f32
-    static constexpr int kAl = kPs + kGqa * 16 * 4;          // alpha [4], key scale [4], bias [4]
+    static constexpr int kVb = kKd + 3 * kGqa * kKdRow;      // value B [2 tiles][NGV][4][2][16] bf16
+    // p [2 tiles][2 token halves][4 heads][8] f32, tokens of a half in (0, 2, 1, 3) order
+    // within each 4-group: owners store and builders read (as pairs) without conflicts
+    static constexpr int kPs = kVb + 2 * NGV * kGqa * 2 * 16 * 2;
+    static constexpr int kAl = kPs + 2 * 2 * kGqa * 8 * 4;   // alpha [4], key scale [4], bias [4]
     static constexpr int kWarpBytes = kAl + 16 * 4;
     static_assert(kKd % 16 == 0 && kVb % 16 == 0 && kPs % 16 == 0 && kAl % 16 == 0, "align");
 };
+
+// One token's value scales and zeros (NGV of each) from a stage, with vector loads.
+template <int NGV>
+__device__ __forceinline__ void load_meta(const float *sp, const int16_t *zp, bool sym, int zsym,
+                                          float (&s)[NGV], int16_t (&z)[NGV]) {
+    if constexpr (NGV == 4) {
+        const float4 v = *reinterpret_cast<const float4 *>(sp);
+        s[0] = v.x; s[1] = v.y; s[2] = v.z; s[3] = v.w;
+    } else if constexpr (NGV == 2) {
+        const float2 v = *reinterpret_cast<const float2 *>(sp);
+        s[0] = v.x; s[1] = v.y;
+    } else {
+#pragma unroll
+        for (int i = 0; i < NGV; ++i) s[i] = sp[i];
+    }
+    if (sym) {
+#pragma unroll
+        for (int i = 0; i < NGV; ++i) z[i] = static_cast<int16_t>(zsym);
+    } else if constexpr (NGV == 4) {
+        const uint2 v = *reinterpret_cast<const uint2 *>(zp);
+        z[0] = static_cast<int16_t>(v.x & 0xffffu); z[1] = static_cast<int16_t>(v.x >> 16);
+        z[2] = static_cast<int16_t>(v.y & 0xffffu); z[3] = static_cast<int16_t>(v.y >> 16);
+    } else {
+#pragma unroll
+        for (int i = 0; i < NGV; ++i) z[i] = zp[i];
+    }
+}
 
 template <int N, int D, int GV>
 __global__ void __launch_bounds__(kDecodeThreads, 3) decode_gqa_kernel(const DecodeArgs a) {
@@ -589,6 +623,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_gqa_kernel(const Dec
     constexpr uint32_t BYTE_MASK = ((1u << N) - 1u) * 0x01010101u;
     using St = Stage<N, D, GV>;
     using Sm = GqaSmem<N, D, GV>;
+    constexpr int kGqaStages = gqa_stages<N>();
 
     __shared__ __align__(16) float q_s[kGqa][D];
     __shared__ float ml_s[kDecodeWarps][kGqa][2];
@@ -722,7 +757,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_gqa_kernel(const Dec
 
     auto issue = [&](int ti) {
         if (ti >= we) return;
-        unsigned char *st = wmem + ((ti - wb) % kStages) * St::kBytes;
+        unsigned char *st = wmem + ((ti - wb) % kGqaStages) * St::kBytes;
         const uint32_t *ksrc = kc + static_cast<int64_t>(ti) * TW + lane * W;
         const uint32_t *vsrc = vc + static_cast<int64_t>(ti) * TW + lane * W;
         if constexpr (W % 4 == 0) {
@@ -766,113 +801,130 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_gqa_kernel(const Dec
     // B operands of the key MMA for the current group
     uint32_t kb0[NK][2], kb1[NK][2];
 
+    // Key digits of the group tile `st` opens: lane builds head hb, channels
+    // 4*lb + 32*i4 + {0..3} (a quarter-warp reads 128 contiguous bytes).
+    auto rebuild_key_digits = [&](const unsigned char *st) {
+        const float *ks_s = reinterpret_cast<const float *>(st + St::kKs);
+        const int16_t *kz_s = reinterpret_cast<const int16_t *>(st + St::kKz);
+        float qv[16];
+        float mx = 0.f, kbp = 0.f;
 #pragma unroll
-    for (int s = 0; s < kStages - 1; ++s) {
+        for (int i4 = 0; i4 < 4; ++i4) {
+            const int c0 = 4 * lb + 32 * i4;
+            const float4 sc = *reinterpret_cast<const float4 *>(ks_s + c0);
+            const float4 qq = *reinterpret_cast<const float4 *>(&q_s[hb][c0]);
+            qv[4 * i4 + 0] = qq.x * sc.x; qv[4 * i4 + 1] = qq.y * sc.y;
+            qv[4 * i4 + 2] = qq.z * sc.z; qv[4 * i4 + 3] = qq.w * sc.w;
+            float z[4] = {static_cast<float>(zsym), static_cast<float>(zsym),
+                          static_cast<float>(zsym), static_cast<float>(zsym)};
+            if (!a.sym) {
+                const uint2 zz = *reinterpret_cast<const uint2 *>(kz_s + c0);
+                z[0] = __int2float_rn(static_cast<int16_t>(zz.x & 0xffffu));
+                z[1] = __int2float_rn(static_cast<int16_t>(zz.x >> 16));
+                z[2] = __int2float_rn(static_cast<int16_t>(zz.y & 0xffffu));
+                z[3] = __int2float_rn(static_cast<int16_t>(zz.y >> 16));
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                kbp = fmaf(qv[4 * i4 + i], z[i], kbp);
+                mx = fmaxf(mx, fabsf(qv[4 * i4 + i]));
+            }
+        }
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) {
+            kbp += __shfl_xor_sync(0xffffffffu, kbp, o);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+        int e = 0;
+        if (mx > 0.f) e = 21 - (static_cast<int>((__float_as_uint(mx) >> 23) & 0xff) - 126);
+        e = max(-120, min(120, e));
+        const float scale = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+        uint32_t dw[3][4];
+#pragma unroll
+        for (int i4 = 0; i4 < 4; ++i4) {
+            const int Q0 = round_small(qv[4 * i4 + 0] * scale), Q1 = round_small(qv[4 * i4 + 1] * scale);
+            const int Q2 = round_small(qv[4 * i4 + 2] * scale), Q3 = round_small(qv[4 * i4 + 3] * scale);
+#pragma unroll
+            for (int k = 0; k < 3; ++k) {
+                const uint32_t sel = static_cast<uint32_t>(k | ((k + 4) << 4));
+                dw[k][i4] = __byte_perm(__byte_perm(Q0, Q1, sel), __byte_perm(Q2, Q3, sel), 0x5410);
+            }
+        }
+        __syncwarp();   // the previous group's digits have been read into registers
+#pragma unroll
+        for (int k = 0; k < 3; ++k)
+#pragma unroll
+            for (int i4 = 0; i4 < 4; ++i4)
+                reinterpret_cast<uint32_t *>(kd + (k * kGqa + hb) * Sm::kKdRow)[lb + 8 * i4] = dw[k][i4];
+        if (lb == 0) {
+            al[4 + hb] = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+            al[8 + hb] = kbp;
+        }
+        __syncwarp();
+        // B fragments: column g8 = head g8/2, digit g8%2 (first n-tile), digit 2 for even g8
+        const uint32_t *kdw0 =
+            reinterpret_cast<const uint32_t *>(kd + ((g8 & 1) * kGqa + (g8 >> 1)) * Sm::kKdRow);
+        const uint32_t *kdw2 = reinterpret_cast<const uint32_t *>(kd + (2 * kGqa + (g8 >> 1)) * Sm::kKdRow);
+#pragma unroll
+        for (int mk = 0; mk < NK; ++mk) {
+            kb0[mk][0] = kdw0[8 * mk + t4];
+            kb0[mk][1] = kdw0[8 * mk + 4 + t4];
+            kb1[mk][0] = (g8 & 1) ? 0u : kdw2[8 * mk + t4];
+            kb1[mk][1] = (g8 & 1) ? 0u : kdw2[8 * mk + 4 + t4];
+        }
+        kinv = al[4 + t4];
+        kbias = al[8 + t4];
+    };
+
+#pragma unroll
+    for (int s = 0; s < kGqaStages - 2; ++s) {
         issue(wb + s);
         cp_async_commit();
     }
 
-    for (int ti = wb; ti < we; ++ti) {
-        issue(ti + kStages - 1);
+    // two tiles per iteration: their key MMAs, one softmax update and their value MMAs
+    // are independent streams of work for the scheduler
+    for (int ti = wb; ti < we; ti += 2) {
+        const int nt = min(2, we - ti);
+        issue(ti + kGqaStages - 2);
         cp_async_commit();
-        cp_async_wait<kStages - 1>();
+        issue(ti + kGqaStages - 1);
+        cp_async_commit();
+        cp_async_wait<kGqaStages - 2>();
         __syncwarp();
-        const unsigned char *st = wmem + ((ti - wb) % kStages) * St::kBytes;
 
-        if (ti == wb || (ti & gmask) == 0) {
-            // ---- key digits of this group: lane builds head hb, channels 16*lb .. +15 ----
-            const float *ks_s = reinterpret_cast<const float *>(st + St::kKs);
-            const int16_t *kz_s = reinterpret_cast<const int16_t *>(st + St::kKz);
-            float qv[16];
-            float mx = 0.f, kbp = 0.f;
+        // ---- key MMAs: logits of tokens g8, g8 + 8 of both tiles, query head t4 ----
+        float lg[2][2];
 #pragma unroll
-            for (int i4 = 0; i4 < 4; ++i4) {
-                const int c0 = 16 * lb + 4 * i4;
-                const float4 sc = *reinterpret_cast<const float4 *>(ks_s + c0);
-                const float4 qq = *reinterpret_cast<const float4 *>(&q_s[hb][c0]);
-                qv[4 * i4 + 0] = qq.x * sc.x; qv[4 * i4 + 1] = qq.y * sc.y;
-                qv[4 * i4 + 2] = qq.z * sc.z; qv[4 * i4 + 3] = qq.w * sc.w;
-                float z[4] = {static_cast<float>(zsym), static_cast<float>(zsym),
-                              static_cast<float>(zsym), static_cast<float>(zsym)};
-                if (!a.sym) {
-                    const uint2 zz = *reinterpret_cast<const uint2 *>(kz_s + c0);
-                    z[0] = small_int_to_float(static_cast<int16_t>(zz.x & 0xffffu));
-                    z[1] = small_int_to_float(static_cast<int16_t>(zz.x >> 16));
-                    z[2] = small_int_to_float(static_cast<int16_t>(zz.y & 0xffffu));
-                    z[3] = small_int_to_float(static_cast<int16_t>(zz.y >> 16));
+        for (int u = 0; u < 2; ++u) {
+            lg[u][0] = lg[u][1] = -INFINITY;
+            if (u < nt) {
+                const int t = ti + u;
+                const unsigned char *st = wmem + ((t - wb) % kGqaStages) * St::kBytes;
+                if (t == wb || (t & gmask) == 0) rebuild_key_digits(st);
+                uint32_t kw[W];
+                load_stage_words<W>(reinterpret_cast<const uint32_t *>(st), lane, kw);
+                int d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0};
+#pragma unroll
+                for (int mk = 0; mk < NK; ++mk) {
+                    uint32_t af[4];
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const int j = 2 * mk + (r >> 1), half = r & 1;
+                        af[r] = (kw[j / BPW] >> (N * (2 * (j % BPW) + half))) & BYTE_MASK;
+                    }
+                    imma_uu(d0, af, kb0[mk][0], kb0[mk][1]);
+                    imma_us(d1, af, kb1[mk][0], kb1[mk][1]);
                 }
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    kbp = fmaf(qv[4 * i4 + i], z[i], kbp);
-                    mx = fmaxf(mx, fabsf(qv[4 * i4 + i]));
-                }
+                lg[u][0] = (small_int_to_float(d0[0]) + 256.f * small_int_to_float(d0[1]) +
+                            65536.f * small_int_to_float(d1[0])) * kinv - kbias;
+                lg[u][1] = (small_int_to_float(d0[2]) + 256.f * small_int_to_float(d0[3]) +
+                            65536.f * small_int_to_float(d1[2])) * kinv - kbias;
             }
-#pragma unroll
-            for (int o = 1; o < 8; o <<= 1) {
-                kbp += __shfl_xor_sync(0xffffffffu, kbp, o);
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            }
-            int e = 0;
-            if (mx > 0.f) e = 21 - (static_cast<int>((__float_as_uint(mx) >> 23) & 0xff) - 126);
-            e = max(-120, min(120, e));
-            const float scale = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
-            uint32_t dw[3][4];
-#pragma unroll
-            for (int i4 = 0; i4 < 4; ++i4) {
-                const int Q0 = round_small(qv[4 * i4 + 0] * scale), Q1 = round_small(qv[4 * i4 + 1] * scale);
-                const int Q2 = round_small(qv[4 * i4 + 2] * scale), Q3 = round_small(qv[4 * i4 + 3] * scale);
-#pragma unroll
-                for (int k = 0; k < 3; ++k) {
-                    const uint32_t sel = static_cast<uint32_t>(k | ((k + 4) << 4));
-                    dw[k][i4] = __byte_perm(__byte_perm(Q0, Q1, sel), __byte_perm(Q2, Q3, sel), 0x5410);
-                }
-            }
-#pragma unroll
-            for (int k = 0; k < 3; ++k)
-                *reinterpret_cast<uint4 *>(kd + (k * kGqa + hb) * Sm::kKdRow + 16 * lb) =
-                    make_uint4(dw[k][0], dw[k][1], dw[k][2], dw[k][3]);
-            if (lb == 0) {
-                al[4 + hb] = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
-                al[8 + hb] = kbp;
-            }
-            __syncwarp();
-            // B fragments: column g8 = head g8/2, digit g8%2 (first n-tile), digit 2 for even g8
-            const uint32_t *kdw0 =
-                reinterpret_cast<const uint32_t *>(kd + ((g8 & 1) * kGqa + (g8 >> 1)) * Sm::kKdRow);
-            const uint32_t *kdw2 = reinterpret_cast<const uint32_t *>(kd + (2 * kGqa + (g8 >> 1)) * Sm::kKdRow);
-#pragma unroll
-            for (int mk = 0; mk < NK; ++mk) {
-                kb0[mk][0] = kdw0[8 * mk + t4];
-                kb0[mk][1] = kdw0[8 * mk + 4 + t4];
-                kb1[mk][0] = (g8 & 1) ? 0u : kdw2[8 * mk + t4];
-                kb1[mk][1] = (g8 & 1) ? 0u : kdw2[8 * mk + 4 + t4];
-            }
-            kinv = al[4 + t4];
-            kbias = al[8 + t4];
         }
 
-        // ---- key MMA: logits of tokens g8, g8 + 8 for query head t4 ----
-        uint32_t kw[W];
-        load_stage_words<W>(reinterpret_cast<const uint32_t *>(st), lane, kw);
-        int d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0};
-#pragma unroll
-        for (int mk = 0; mk < NK; ++mk) {
-            uint32_t af[4];
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int j = 2 * mk + (r >> 1), half = r & 1;
-                af[r] = (kw[j / BPW] >> (N * (2 * (j % BPW) + half))) & BYTE_MASK;
-            }
-            imma_uu(d0, af, kb0[mk][0], kb0[mk][1]);
-            imma_us(d1, af, kb1[mk][0], kb1[mk][1]);
-        }
-        const float lg0 = (small_int_to_float(d0[0]) + 256.f * small_int_to_float(d0[1]) +
-                           65536.f * small_int_to_float(d1[0])) * kinv - kbias;
-        const float lg1 = (small_int_to_float(d0[2]) + 256.f * small_int_to_float(d0[3]) +
-                           65536.f * small_int_to_float(d1[2])) * kinv - kbias;
-
-        // ---- online softmax of head t4 ----
-        float tmax = fmaxf(lg0, lg1);
+        // ---- online softmax of head t4 over both tiles ----
+        float tmax = fmaxf(fmaxf(lg[0][0], lg[0][1]), fmaxf(lg[1][0], lg[1][1]));
         tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
         tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
         tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
@@ -887,61 +939,78 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_gqa_kernel(const Dec
             }
             if (g8 == 0) al[t4] = alpha;
             __syncwarp();
-            const float ab = al[hb];
+            const float ab = al[lane & 3];     // zsum belongs to head lane % 4
 #pragma unroll
             for (int v = 0; v < NGV; ++v) zsum[v] *= ab;
         }
-        const float p0 = fast_exp2(lg0 - m), p1 = fast_exp2(lg1 - m);
-        lsum += p0 + p1;
-        ps[t4 * 16 + g8] = p0;
-        ps[t4 * 16 + g8 + 8] = p1;
+        // position of token g8 (and g8 + 8) inside its half: 4-groups in (0, 2, 1, 3) order
+        const int ppos = (g8 & 4) + ((g8 & 1) << 1) + ((g8 >> 1) & 1);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const float p0 = fast_exp2(lg[u][0] - m), p1 = fast_exp2(lg[u][1] - m);
+            lsum += p0 + p1;
+            ps[((u * 2 + 0) * kGqa + t4) * 8 + ppos] = p0;
+            ps[((u * 2 + 1) * kGqa + t4) * 8 + ppos] = p1;
+        }
         __syncwarp();
 
-        // ---- value B: lane builds head hb, tokens 4q + e and 4q + e + 2 ----
-        {
-            constexpr float kBscale = 1.0f / static_cast<float>(1 << (7 - N));
-            constexpr int kOff = 1 << N;              // code offset carried by the f16 A operand
-            const int q4 = lb >> 1, e = lb & 1;
-            const int ta = 4 * q4 + e, tb = ta + 2;
-            const float pa = ps[hb * 16 + ta] * kBscale, pb = ps[hb * 16 + tb] * kBscale;
-            const float *vsp = reinterpret_cast<const float *>(st + St::kVs);
-            const int16_t *vzp = reinterpret_cast<const int16_t *>(st + St::kVz);
-            float sa[NGV], sb[NGV];
-            int16_t zza[NGV], zzb[NGV];
+        // ---- value B of both tiles: lane l builds head l % 4 for tokens 4q + e and
+        //      4q + e + 2, (q, e) = (l / 8, (l / 4) % 2): a quarter-warp covers one token pair
+        //      of all four heads (broadcast meta reads, distinct p rows and plane words) ----
 #pragma unroll
-            for (int v = 0; v < NGV; ++v) {
-                sa[v] = vsp[ta * NGV + v];
-                sb[v] = vsp[tb * NGV + v];
-                zza[v] = a.sym ? static_cast<int16_t>(zsym) : vzp[ta * NGV + v];
-                zzb[v] = a.sym ? static_cast<int16_t>(zsym) : vzp[tb * NGV + v];
-            }
+        for (int u = 0; u < 2; ++u) {
+            if (u < nt) {
+                const unsigned char *st = wmem + ((ti + u - wb) % kGqaStages) * St::kBytes;
+                constexpr float kBscale = 1.0f / static_cast<float>(1 << (7 - N));
+                constexpr int kOff = 1 << N;          // code offset carried by the bf16 A operand
+                const int hv = lane & 3, q4 = lane >> 3, e = (lane >> 2) & 1;
+                const int ta = 4 * q4 + e, tb = ta + 2;
+                // tokens ta, tb sit side by side: half q4/2, position 4*(q4%2) + 2e (+1)
+                const float2 pr = *reinterpret_cast<const float2 *>(
+                    ps + ((u * 2 + (q4 >> 1)) * kGqa + hv) * 8 + 4 * (q4 & 1) + 2 * e);
+                const float2 pab = make_float2(pr.x * kBscale, pr.y * kBscale);
+                const float *vsp = reinterpret_cast<const float *>(st + St::kVs);
+                const int16_t *vzp = reinterpret_cast<const int16_t *>(st + St::kVz);
+                float sa[NGV], sb[NGV];
+                int16_t zza[NGV], zzb[NGV];
+                load_meta<NGV>(vsp + ta * NGV, vzp + ta * NGV, a.sym, zsym, sa, zza);
+                load_meta<NGV>(vsp + tb * NGV, vzp + tb * NGV, a.sym, zsym, sb, zzb);
 #pragma unroll
-            for (int v = 0; v < NGV; ++v) {
-                const float xa = pa * sa[v], xb = pb * sb[v];
-                const float za = small_int_to_float(zza[v] + kOff);
-                const float zb = small_int_to_float(zzb[v] + kOff);
-                zsum[v] = fmaf(xa, za, fmaf(xb, zb, zsum[v]));
-                const uint32_t hi = f2bf2(xa, xb);
-                const uint32_t lo =
-                    f2bf2(xa - __uint_as_float(hi << 16), xb - __uint_as_float(hi & 0xffff0000u));
-                uint32_t *dst = reinterpret_cast<uint32_t *>(vb + ((v * kGqa + hb) * 2) * 16);
-                dst[(4 * q4 + 2 * e) >> 1] = hi;          // part 0 plane
-                dst[(16 + 4 * q4 + 2 * e) >> 1] = lo;     // part 1 plane
+                for (int v = 0; v < NGV; ++v) {
+                    const float2 x = mul2(pab, make_float2(sa[v], sb[v]));
+                    const float2 z = make_float2(__int2float_rn(zza[v] + kOff), __int2float_rn(zzb[v] + kOff));
+                    zsum[v] = fmaf(x.x, z.x, fmaf(x.y, z.y, zsum[v]));
+                    const uint32_t hi = f2bf2(x.x, x.y);
+                    const float2 lof = add2(x, make_float2(-__uint_as_float(hi << 16),
+                                                           -__uint_as_float(hi & 0xffff0000u)));
+                    const uint32_t lo = f2bf2(lof.x, lof.y);
+                    // planes (part p of head h) at sub-block p ^ (h >> 1): conflict-free stores and loads
+                    uint32_t *dst = reinterpret_cast<uint32_t *>(vb + (((u * NGV + v) * kGqa + hv) * 2) * 16);
+                    dst[((hv >> 1) << 3) + ((4 * q4 + 2 * e) >> 1)] = hi;          // part 0 plane
+                    dst[((1 ^ (hv >> 1)) << 3) + ((4 * q4 + 2 * e) >> 1)] = lo;    // part 1 plane
+                }
             }
         }
         __syncwarp();
 
-        // ---- value MMA: rows = channels of chunk j, k = the tile's tokens ----
-        uint32_t vw[W];
-        load_stage_words<W>(reinterpret_cast<const uint32_t *>(st + St::kCodes), lane, vw);
+        // ---- value MMAs: rows = channels of chunk j, k = a tile's tokens ----
 #pragma unroll
-        for (int j = 0; j < NJ; ++j) {
-            uint32_t a02, a13, b02, b13;
-            codes_bf16<N>(vw[j / BPW], 2 * (j % BPW), magic16, a02, a13);       // channel 16j + g8
-            codes_bf16<N>(vw[j / BPW], 2 * (j % BPW) + 1, magic16, b02, b13);   // channel 16j + g8 + 8
-            const uint2 bb = *reinterpret_cast<const uint2 *>(
-                vb + (((16 * j) / GV * kGqa + (g8 >> 1)) * 2 + (g8 & 1)) * 16 + 4 * t4);
-            hmma(dv[j], a02, b02, a13, b13, bb.x, bb.y);
+        for (int u = 0; u < 2; ++u) {
+            if (u < nt) {
+                const unsigned char *st = wmem + ((ti + u - wb) % kGqaStages) * St::kBytes;
+                uint32_t vw[W];
+                load_stage_words<W>(reinterpret_cast<const uint32_t *>(st + St::kCodes), lane, vw);
+#pragma unroll
+                for (int j = 0; j < NJ; ++j) {
+                    uint32_t a02, a13, b02, b13;
+                    codes_bf16<N>(vw[j / BPW], 2 * (j % BPW), magic16, a02, a13);       // channel 16j + g8
+                    codes_bf16<N>(vw[j / BPW], 2 * (j % BPW) + 1, magic16, b02, b13);   // channel 16j + g8 + 8
+                    const uint2 bb = *reinterpret_cast<const uint2 *>(
+                        vb + ((((u * NGV + (16 * j) / GV) * kGqa + (g8 >> 1)) * 2 + ((g8 & 1) ^ (g8 >> 2))) * 16) +
+                        4 * t4);
+                    hmma(dv[j], a02, b02, a13, b13, bb.x, bb.y);
+                }
+            }
         }
         __syncwarp();
     }
@@ -953,16 +1022,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_gqa_kernel(const Dec
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
 #pragma unroll
-    for (int v = 0; v < NGV; ++v) {
-        zsum[v] += __shfl_xor_sync(0xffffffffu, zsum[v], 1);
-        zsum[v] += __shfl_xor_sync(0xffffffffu, zsum[v], 2);
+    for (int v = 0; v < NGV; ++v) {      // lanes with the same lane % 4 hold one head's partials
         zsum[v] += __shfl_xor_sync(0xffffffffu, zsum[v], 4);
+        zsum[v] += __shfl_xor_sync(0xffffffffu, zsum[v], 8);
+        zsum[v] += __shfl_xor_sync(0xffffffffu, zsum[v], 16);
     }
     __syncthreads();   // stage memory is reused for the per-warp outputs below
     float *o_s = reinterpret_cast<float *>(stage_mem);   // [warp][head][D]
     float *zs_s = o_s + kDecodeWarps * kGqa * D;          // [warp][head][NGV]
-    if (lb == 0)
-        for (int v = 0; v < NGV; ++v) zs_s[(warp * kGqa + hb) * NGV + v] = zsum[v];
+    if (lane < kGqa)
+        for (int v = 0; v < NGV; ++v) zs_s[(warp * kGqa + lane) * NGV + v] = zsum[v];
     // dv sums A * B = (2^N + code) p s; zsum sums b (2^N + z) with b = p s 2^-(7-N)
     __syncwarp();
 #pragma unroll
