@@ -41,7 +41,7 @@ FALLBACK_HBM_GBS = 6650.0
 def _args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--steps", type=int, default=30)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--workload", default="llama7b")
     p.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
@@ -87,10 +87,15 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def ncu_traffic(workload: str):
+def decode_kernel_name(w) -> str:
+    """The decode kernel the library launches for this geometry."""
+    return "decode_gqa_kernel" if w.Hq == 4 * w.Hkv else "decode_split_kernel"
+
+
+def ncu_traffic(w):
     """Per-launch DRAM bytes of the decode kernel from the committed ncu summary,
     if it was taken on the current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", f"decode_split_kernel_{workload}.md")
+    path = os.path.join(ROOT, "profiles", f"{decode_kernel_name(w)}_{w.name}.md")
     src = os.path.join(ROOT, "bit_kv_cache_22_b200", "csrc", "decode.cu")
     try:
         text = open(path).read()
@@ -102,6 +107,26 @@ def ncu_traffic(workload: str):
     except OSError:
         pass
     return None
+
+
+def shard_workload(base, rank: int):
+    """Weak scaling: every rank serves its own batch of sequences (seed offset by rank)."""
+    return base if rank == 0 else base.replace(seed=base.seed + 1000 * rank)
+
+
+def max_over_ranks(values, world: int, device=None):
+    """Element-wise maximum of per-rank values (the job's time is its slowest rank's)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def job_throughput(units_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job rate: the units every rank processed over the slowest rank's time."""
+    return units_per_rank * world / (ms / 1e3)
 
 
 class ClockSampler:
@@ -118,7 +143,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -178,8 +203,7 @@ def run_kvq(args):
         import datetime
         dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
 
-    base = wl.WORKLOADS[args.workload]
-    w = base.replace(seed=base.seed + 1000 * rank) if rank else base
+    w = shard_workload(wl.WORKLOADS[args.workload], rank)
     dt = torch.float16 if w.dtype == wl.FP16 else torch.bfloat16
 
     def to_t(bits, pin=False):
@@ -256,12 +280,12 @@ def run_kvq(args):
 
     evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             for _ in range(w.steps)] for _ in range(args.steps + 1)]
-    replay_episode(evs[-1])          # graph warm-up
-    torch.cuda.synchronize()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
     with ClockSampler(local) as clk:
+        replay_episode(evs[-1])          # graph warm-up (also gives the sampler time to start)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
         start.record(stream)
         for k in range(args.steps):
             replay_episode(evs[k])
@@ -271,10 +295,7 @@ def run_kvq(args):
     launches = launches_per_episode * args.steps
     ms = start.elapsed_time(stop)
     decode_ms = sum(a.elapsed_time(b) for ev in evs[:args.steps] for a, b in ev)
-    t = torch.tensor([ms, decode_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms, decode_ms = float(t[0]), float(t[1])
+    ms, decode_ms = max_over_ranks([ms, decode_ms], world, dev)
 
     # ---- end to end through the public API with pinned host buffers ----
     e2e = None
@@ -305,13 +326,10 @@ def run_kvq(args):
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e_ms = float(te[0])
+        e2e_ms, = max_over_ranks([e0.elapsed_time(e1)], world, dev)
         h2d = XKp.numel() * 2 * 2 + w.steps * (2 * w.B * w.Hkv * w.d + w.B * w.Hq * w.d) * 2
         d2h = w.steps * w.B * w.Hq * w.d * 4
-        e2e = {"value": tokens_per_episode * args.steps * world / (e2e_ms / 1e3), "unit": UNIT,
+        e2e = {"value": job_throughput(tokens_per_episode * args.steps, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms / args.steps}
 
@@ -327,10 +345,10 @@ def run_kvq(args):
     peak, peak_kind = peaks()
     decode_launch_ms = decode_ms / (args.steps * w.steps)
     achieved = bytes_per_episode / w.steps / (decode_launch_ms / 1e3) / 1e9
-    traffic = ncu_traffic(args.workload)
+    traffic = ncu_traffic(w)
     line = {
         "metric": METRIC,
-        "value": tokens_per_episode * args.steps * world / (ms / 1e3),
+        "value": job_throughput(tokens_per_episode * args.steps, world, ms),
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,
@@ -354,9 +372,9 @@ def run_kvq(args):
             "splits": cache.splits(),
         },
         "decode_steps_per_s": w.steps * args.steps / (ms / 1e3),
-        "kv_tokens_per_s_decode_only": tokens_per_episode * args.steps * world / (decode_ms / 1e3),
+        "kv_tokens_per_s_decode_only": job_throughput(tokens_per_episode * args.steps, world, decode_ms),
         "roofline": {
-            "kernel": "decode_attention (split-K kernel + combine), per call",
+            "kernel": f"decode_attention ({decode_kernel_name(w)} + combine), per call",
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
             if peak_kind == "measured" else "fallback 6.65 TB/s",
