@@ -3,7 +3,7 @@
 One step = one full pass of the hot path over one batch: prefill-quantize the
 prompt (keys per channel, values per token, residual tail), then every decode
 step of the workload (append the new token -- flushing the residual when it
-holds R tokens -- and split-K decode attention with its log-sum-exp combine).
+holds R tokens -- and split-K decode attention whose last split merges the partials).
 The metric is KV tokens attended per second: each decode step attends to
 B * (Tq + r) cached tokens.
 
@@ -48,7 +48,7 @@ def _args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--ncu-case", action="store_true",
-                   help="run one prefill and 3 decode steps of the workload, then exit (for ncu)")
+                   help="run one prefill and up to 64 decode steps of the workload, then exit (for ncu)")
     return p.parse_args()
 
 
@@ -89,7 +89,11 @@ def peaks():
 
 def decode_kernel_name(w) -> str:
     """The decode kernel the library launches for this geometry."""
-    return "decode_gqa_kernel" if w.Hq == 4 * w.Hkv else "decode_split_kernel"
+    if w.Hq == 4 * w.Hkv:
+        return "decode_gqa_kernel"
+    if w.Hq == w.Hkv and w.G >= 32:
+        return "decode_mha_kernel"
+    return "decode_split_kernel"
 
 
 def ncu_traffic(w):
@@ -221,7 +225,7 @@ def run_kvq(args):
 
     if args.ncu_case:
         cache.prefill_quantize(XK, XV)
-        for s in range(3):
+        for s in range(min(w.steps, 64)):      # ends with r = 64 residual rows, mid-episode
             cache.append(tK[s], tV[s])
             cache.decode_attention(tQ[s], out=out)
         torch.cuda.synchronize()
@@ -374,7 +378,7 @@ def run_kvq(args):
         "decode_steps_per_s": w.steps * args.steps / (ms / 1e3),
         "kv_tokens_per_s_decode_only": job_throughput(tokens_per_episode * args.steps, world, decode_ms),
         "roofline": {
-            "kernel": f"decode_attention ({decode_kernel_name(w)} + combine), per call",
+            "kernel": f"decode_attention ({decode_kernel_name(w)}, splits merged in-kernel), per call",
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
             if peak_kind == "measured" else "fallback 6.65 TB/s",

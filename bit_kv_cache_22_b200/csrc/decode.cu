@@ -13,8 +13,8 @@
 // streamed through a per-warp cp.async ring of shared-memory stages.  Token order does not change the result
 // (A . V = A_P . V_P, "Resumo Técnico: LogQuant", section 4), which is what
 // allows the splits and the residual to be folded into one online-softmax pass.
-// Each CTA writes an unnormalised partial (o, m, l); combine_kernel merges the
-// S partials with a log-sum-exp reduction.
+// Each CTA merges its warps into an unnormalised partial (o, m, l); the last
+// CTA of each (batch, head) to finish merges the S partials (finish_cta).
 //
 // Lane = 4*g8 + t4.  In a tile it holds, per 16-channel chunk j, the codes of
 // rows g8 and g8+8 at columns 4*t4 .. 4*t4+3 (keys: rows = tokens, columns =
@@ -159,6 +159,83 @@ struct Stage {
 
 constexpr int kStages = 4;
 
+// End of every decode CTA.  o_w [warp][HG][D] and ml_w [warp][HG] = (m, l) are
+// the per-warp partials of the CTA's HG query heads (unnormalised, log2
+// domain; m = -inf for a warp without tokens).  They are merged into the CTA's
+// partial of split `sigma`.  With one split that is the answer and is written
+// out.  Otherwise the partial goes to the workspace, and the CTA that brings
+// the unit's arrival counter to S merges all S partials with a log-sum-exp
+// reduction, writes t_O and puts the counter back to zero for the next call
+// (flash-decoding's reduction, done by the last split instead of a second
+// kernel).  wts is shared scratch of HG * (S + 1) floats that may alias o_w.
+template <int HG, int D>
+__device__ __forceinline__ void finish_cta(const DecodeArgs &a, const float *o_w,
+                                           const float (*ml_w)[HG][2], int64_t unit, int64_t bq0,
+                                           int sigma, int *last, float *wts) {
+    for (int i = threadIdx.x; i < HG * D; i += kDecodeThreads) {
+        const int hh = i / D, c = i % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kDecodeWarps; ++w) M = fmaxf(M, ml_w[w][hh][0]);
+        float o = 0.f, l = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDecodeWarps; ++w) {
+            if (ml_w[w][hh][0] == -INFINITY) continue;
+            const float f = exp2f(ml_w[w][hh][0] - M);
+            o = fmaf(o_w[(w * HG + hh) * D + c], f, o);
+            l = fmaf(ml_w[w][hh][1], f, l);
+        }
+        const int64_t bq = bq0 + hh;
+        if (a.S == 1) {
+            a.out[bq * D + c] = o / l;
+            continue;
+        }
+        a.o_part[(bq * a.S + sigma) * D + c] = o;
+        if (c == 0) {
+            a.m_part[bq * a.S + sigma] = M;
+            a.l_part[bq * a.S + sigma] = l;
+        }
+    }
+    if (a.S == 1) return;
+    __threadfence();   // this CTA's partial is visible before its arrival is counted
+    __syncthreads();
+    if (threadIdx.x == 0)
+        *last = atomicAdd(a.arrivals + unit, 1u) == static_cast<unsigned>(a.S - 1);
+    __syncthreads();
+    if (!*last) return;
+    __threadfence();
+    // split weights 2^(m_s - M) and 1 / sum_s l_s 2^(m_s - M), one warp per head
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int hh = warp; hh < HG; hh += kDecodeWarps) {
+        const int64_t row = (bq0 + hh) * a.S;
+        float M = -INFINITY;
+        for (int s = lane; s < a.S; s += 32) M = fmaxf(M, __ldcg(a.m_part + row + s));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float L = 0.f;
+        for (int s = lane; s < a.S; s += 32) {
+            const float ms = __ldcg(a.m_part + row + s);
+            const float f = ms == -INFINITY ? 0.f : exp2f(ms - M);
+            wts[hh * a.S + s] = f;
+            L = fmaf(__ldcg(a.l_part + row + s), f, L);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        if (lane == 0) wts[HG * a.S + hh] = L;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < HG * D; i += kDecodeThreads) {
+        const int hh = i / D, c = i % D;
+        const float *op = a.o_part + (bq0 + hh) * a.S * D + c;
+        const float *wp = wts + hh * a.S;
+        float o = 0.f;
+#pragma unroll 8
+        for (int s = 0; s < a.S; ++s) o = fmaf(__ldcg(op + static_cast<int64_t>(s) * D), wp[s], o);
+        a.out[(bq0 + hh) * D + c] = o / wts[HG * a.S + hh];
+    }
+    if (threadIdx.x == 0) a.arrivals[unit] = 0u;
+}
+
 template <int N, int D, int GV>
 __global__ void __launch_bounds__(kDecodeThreads, 4) decode_split_kernel(const DecodeArgs a) {
     constexpr int W = D * N / 64;     // words per lane per tile
@@ -173,9 +250,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_split_kernel(const D
     __shared__ float q_s[D];
     __shared__ float o_s[kDecodeWarps][D];
     __shared__ float ml_s[kDecodeWarps][2];
+    __shared__ int last_s;
     extern __shared__ __align__(128) unsigned char stage_mem[];
 
-    const int sigma = blockIdx.x, qi = blockIdx.y, b = blockIdx.z;
+    const int qi = blockIdx.x, b = blockIdx.y, sigma = blockIdx.z;
     const int g = a.Hq / a.Hkv;
     const int64_t bh = static_cast<int64_t>(b) * a.Hkv + qi / g;
     const int64_t bq = static_cast<int64_t>(b) * a.Hq + qi;
@@ -474,25 +552,109 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_split_kernel(const D
     }
     __syncthreads();
 
-    // ---- merge the four warps, write this split's partial ----
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kDecodeWarps; ++w) M = fmaxf(M, ml_s[w][0]);
-    for (int c = threadIdx.x; c < D; c += kDecodeThreads) {
-        float o = 0.f, l = 0.f;
-#pragma unroll
-        for (int w = 0; w < kDecodeWarps; ++w) {
-            if (ml_s[w][0] == -INFINITY) continue;
-            const float f = exp2f(ml_s[w][0] - M);
-            o = fmaf(o_s[w][c], f, o);
-            l = fmaf(ml_s[w][1], f, l);
+    // ---- merge the four warps, finish the split ----
+    finish_cta<1, D>(a, &o_s[0][0], reinterpret_cast<const float(*)[1][2]>(ml_s), bq, bq, sigma,
+                     &last_s, reinterpret_cast<float *>(stage_mem));
+}
+
+// Shared-memory bytes residual_pass needs per warp: one 16-row tile of K and of V,
+// rows padded by 16 bytes so that the 8 row groups of a warp hit distinct banks.
+template <int D>
+__host__ __device__ constexpr int residual_scratch_bytes() { return 2 * 16 * (2 * D + 16); }
+
+// Online-softmax pass of one warp over residual tiles rt0, rt0 + stride, ... < rt1
+// of one query head (16 rows each; rows >= r masked) with the exact e values on
+// CUDA cores.  Each tile's K and V rows are first staged in `scratch`
+// (residual_scratch_bytes<D>() bytes of this warp's shared memory) with
+// coalesced cp.async; the caller must have no cp.async group of its own
+// pending.  qh is the log2-scaled query in shared memory; acc[j][h] accumulates
+// channel 16j + g8 + 8h, x over tokens 4*t4 + {0, 1}, y over 4*t4 + {2, 3}.
+template <int D>
+__device__ __forceinline__ void residual_pass(const DecodeArgs &a, const float *qh, const uint16_t *kr,
+                                              const uint16_t *vr, int rt0, int rt1, int lane, float &m,
+                                              float &lsum, float2 (&acc)[D / 16][2], unsigned char *scratch,
+                                              int stride = 1) {
+    constexpr int NJ = D / 16;
+    constexpr int kRow = 2 * D + 16;          // padded row stride in bytes
+    constexpr int kPieces = 2 * D / 16;       // 16-byte pieces of one row
+    const int g8 = lane >> 2, t4 = lane & 3;
+    unsigned char *ks = scratch, *vs = scratch + 16 * kRow;
+    for (int rt = rt0; rt < rt1; rt += stride) {
+        const int rows = min(16, a.r - 16 * rt);
+        const int n = rows * kPieces;
+        __syncwarp();   // the previous tile's rows have been read
+        for (int c = lane; c < 2 * n; c += 32) {
+            const bool isv = c >= n;
+            const int cc = isv ? c - n : c, row = cc / kPieces, pc = cc % kPieces;
+            cp_async16((isv ? vs : ks) + row * kRow + 16 * pc,
+                       (isv ? vr : kr) + (static_cast<int64_t>(rt) * 16 + row) * D + 8 * pc);
         }
-        a.o_part[(bq * a.S + sigma) * D + c] = o;
-        if (c == 0) {
-            a.m_part[bq * a.S + sigma] = M;
-            a.l_part[bq * a.S + sigma] = l;
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncwarp();
+        const int row0 = g8, row1 = g8 + 8;
+        float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+            const int c0 = 16 * j + 4 * t4;
+            const float4 qq = *reinterpret_cast<const float4 *>(qh + c0);
+            const uint2 k0 = *reinterpret_cast<const uint2 *>(ks + row0 * kRow + 2 * c0);
+            const uint2 k1 = *reinterpret_cast<const uint2 *>(ks + row1 * kRow + 2 * c0);
+            x0 = fmaf(qq.x, widen(k0.x & 0xffffu, a.bf16), x0);
+            x0 = fmaf(qq.y, widen(k0.x >> 16, a.bf16), x0);
+            x0 = fmaf(qq.z, widen(k0.y & 0xffffu, a.bf16), x0);
+            x0 = fmaf(qq.w, widen(k0.y >> 16, a.bf16), x0);
+            x1 = fmaf(qq.x, widen(k1.x & 0xffffu, a.bf16), x1);
+            x1 = fmaf(qq.y, widen(k1.x >> 16, a.bf16), x1);
+            x1 = fmaf(qq.z, widen(k1.y & 0xffffu, a.bf16), x1);
+            x1 = fmaf(qq.w, widen(k1.y >> 16, a.bf16), x1);
         }
+        x0 += __shfl_xor_sync(0xffffffffu, x0, 1);
+        x1 += __shfl_xor_sync(0xffffffffu, x1, 1);
+        x0 += __shfl_xor_sync(0xffffffffu, x0, 2);
+        x1 += __shfl_xor_sync(0xffffffffu, x1, 2);
+        const float lg0 = row0 < rows ? x0 : -INFINITY;
+        const float lg1 = row1 < rows ? x1 : -INFINITY;
+        float tmax = fmaxf(lg0, lg1);
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
+        if (tmax > m) {
+            const float alpha = fast_exp2(m - tmax);
+            lsum *= alpha;
+#pragma unroll
+            for (int j = 0; j < NJ; ++j) {
+                acc[j][0] = mul2(acc[j][0], make_float2(alpha, alpha));
+                acc[j][1] = mul2(acc[j][1], make_float2(alpha, alpha));
+            }
+            m = tmax;
+        }
+        const float p0 = fast_exp2(lg0 - m), p1 = fast_exp2(lg1 - m);
+        lsum += p0 + p1;
+        const float pexp = (t4 & 2) ? p1 : p0;
+        float pt[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            pt[i] = __shfl_sync(0xffffffffu, pexp, 4 * ((4 * t4 + i) & 7) + 2 * (t4 >> 1));
+        // rows >= r hold stale bytes: their p is exactly 0 but 0 * stale could be NaN
+        float vv[NJ][2][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const bool ok = 4 * t4 + i < rows;
+            const uint16_t *vrow = reinterpret_cast<const uint16_t *>(vs + (4 * t4 + i) * kRow);
+#pragma unroll
+            for (int j = 0; j < NJ; ++j)
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    vv[j][h][i] = ok ? pt[i] * widen(vrow[16 * j + g8 + 8 * h], a.bf16) : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < NJ; ++j)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                acc[j][h] = add2(acc[j][h], make_float2(vv[j][h][0] + vv[j][h][1], vv[j][h][2] + vv[j][h][3]));
     }
+    __syncwarp();
 }
 
 // ---------------------------------------------------------------------------
@@ -532,6 +694,13 @@ __device__ __forceinline__ void imma_us(int (&d)[4], const uint32_t (&a)[4], uin
         "{%0,%1,%2,%3};"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// d = A B (no accumulator input)
+__device__ __forceinline__ void imma_us0(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0));
 }
 __device__ __forceinline__ void hmma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                      uint32_t b0, uint32_t b1) {
@@ -627,9 +796,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_gqa_kernel(const Dec
 
     __shared__ __align__(16) float q_s[kGqa][D];
     __shared__ float ml_s[kDecodeWarps][kGqa][2];
+    __shared__ int last_s;
     extern __shared__ __align__(128) unsigned char stage_mem[];
 
-    const int sigma = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+    const int hk = blockIdx.x, b = blockIdx.y, sigma = blockIdx.z;
     const int64_t bh = static_cast<int64_t>(b) * a.Hkv + hk;
     const int64_t bq0 = static_cast<int64_t>(b) * a.Hq + hk * kGqa;   // first query head
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -652,79 +822,18 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_gqa_kernel(const Dec
     if (sigma >= a.n_qsplits) {
         // ---------------- residual split: warp = query head ----------------
         const float *qh = q_s[warp];
-        const int64_t bq = bq0 + warp;
         float m = -INFINITY, lsum = 0.f;
         float2 acc[NJ][2];
 #pragma unroll
         for (int j = 0; j < NJ; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
-        const uint16_t *kr = a.kr + bh * a.R * D;
-        const uint16_t *vr = a.vr + bh * a.R * D;
-        for (int ti = a.n_qtiles; ti < total_tiles; ++ti) {
-            const int row0 = (ti - a.n_qtiles) * 16 + g8, row1 = row0 + 8;
-            float x0 = 0.f, x1 = 0.f;
-#pragma unroll
-            for (int j = 0; j < NJ; ++j) {
-                const int c0 = 16 * j + 4 * t4;
-                const float4 qq = *reinterpret_cast<const float4 *>(qh + c0);
-                if (row0 < a.r) {
-                    const uint2 kk = *reinterpret_cast<const uint2 *>(kr + row0 * D + c0);
-                    x0 = fmaf(qq.x, widen(kk.x & 0xffffu, a.bf16), x0);
-                    x0 = fmaf(qq.y, widen(kk.x >> 16, a.bf16), x0);
-                    x0 = fmaf(qq.z, widen(kk.y & 0xffffu, a.bf16), x0);
-                    x0 = fmaf(qq.w, widen(kk.y >> 16, a.bf16), x0);
-                }
-                if (row1 < a.r) {
-                    const uint2 kk = *reinterpret_cast<const uint2 *>(kr + row1 * D + c0);
-                    x1 = fmaf(qq.x, widen(kk.x & 0xffffu, a.bf16), x1);
-                    x1 = fmaf(qq.y, widen(kk.x >> 16, a.bf16), x1);
-                    x1 = fmaf(qq.z, widen(kk.y & 0xffffu, a.bf16), x1);
-                    x1 = fmaf(qq.w, widen(kk.y >> 16, a.bf16), x1);
-                }
-            }
-            x0 += __shfl_xor_sync(0xffffffffu, x0, 1);
-            x1 += __shfl_xor_sync(0xffffffffu, x1, 1);
-            x0 += __shfl_xor_sync(0xffffffffu, x0, 2);
-            x1 += __shfl_xor_sync(0xffffffffu, x1, 2);
-            const float lg0 = row0 < a.r ? x0 : -INFINITY;
-            const float lg1 = row1 < a.r ? x1 : -INFINITY;
-            float tmax = fmaxf(lg0, lg1);
-            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
-            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
-            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
-            if (tmax > m) {
-                const float alpha = fast_exp2(m - tmax);
-                lsum *= alpha;
-#pragma unroll
-                for (int j = 0; j < NJ; ++j) {
-                    acc[j][0] = mul2(acc[j][0], make_float2(alpha, alpha));
-                    acc[j][1] = mul2(acc[j][1], make_float2(alpha, alpha));
-                }
-                m = tmax;
-            }
-            const float p0 = fast_exp2(lg0 - m), p1 = fast_exp2(lg1 - m);
-            lsum += p0 + p1;
-            const float pexp = (t4 & 2) ? p1 : p0;
-            float pt[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                pt[i] = __shfl_sync(0xffffffffu, pexp, 4 * ((4 * t4 + i) & 7) + 2 * (t4 >> 1));
-            const int ra = (ti - a.n_qtiles) * 16 + 4 * t4;
-#pragma unroll
-            for (int j = 0; j < NJ; ++j) {
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int c = 16 * j + g8 + 8 * h;
-                    float vv[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        vv[i] = (ra + i < a.r) ? pt[i] * widen(vr[(ra + i) * D + c], a.bf16) : 0.f;
-                    acc[j][h] = add2(acc[j][h], make_float2(vv[0] + vv[1], vv[2] + vv[3]));
-                }
-            }
-        }
+        residual_pass<D>(a, qh, a.kr + bh * a.R * D, a.vr + bh * a.R * D, 0, total_tiles - a.n_qtiles,
+                         lane, m, lsum, acc, wmem);
         lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
         lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
         lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
+        static_assert(residual_scratch_bytes<D>() <= Sm::kWarpBytes, "residual staging");
+        __syncthreads();   // every warp is done with its staged rows before o_s overwrites them
+        float *o_s = reinterpret_cast<float *>(stage_mem);   // [warp][head][D]; only head == warp
 #pragma unroll
         for (int j = 0; j < NJ; ++j) {
 #pragma unroll
@@ -732,13 +841,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_gqa_kernel(const Dec
                 float val = acc[j][h].x + acc[j][h].y;
                 val += __shfl_xor_sync(0xffffffffu, val, 1);
                 val += __shfl_xor_sync(0xffffffffu, val, 2);
-                if (t4 == 0) a.o_part[(bq * a.S + sigma) * D + 16 * j + g8 + 8 * h] = val;
+                if (t4 == 0) o_s[(warp * kGqa + warp) * D + 16 * j + g8 + 8 * h] = val;
             }
         }
-        if (lane == 0) {
-            a.m_part[bq * a.S + sigma] = m;
-            a.l_part[bq * a.S + sigma] = lsum;
+        if (lane < kGqa) {
+            ml_s[warp][lane][0] = lane == warp ? m : -INFINITY;
+            ml_s[warp][lane][1] = lane == warp ? lsum : 0.f;
         }
+        __syncthreads();
+        finish_cta<kGqa, D>(a, o_s, ml_s, bh, bq0, sigma, &last_s, o_s + kDecodeWarps * kGqa * D);
         return;
     }
 
@@ -802,14 +913,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_gqa_kernel(const Dec
     uint32_t kb0[NK][2], kb1[NK][2];
 
     // Key digits of the group tile `st` opens: lane builds head hb, channels
-    // 4*lb + 32*i4 + {0..3} (a quarter-warp reads 128 contiguous bytes).
+    // 4*lb + 32*i4 + {0..3}, i4 < D/32 (a quarter-warp reads 128 contiguous bytes).
     auto rebuild_key_digits = [&](const unsigned char *st) {
         const float *ks_s = reinterpret_cast<const float *>(st + St::kKs);
         const int16_t *kz_s = reinterpret_cast<const int16_t *>(st + St::kKz);
-        float qv[16];
+        constexpr int NQ = D / 32;
+        float qv[4 * NQ];
         float mx = 0.f, kbp = 0.f;
 #pragma unroll
-        for (int i4 = 0; i4 < 4; ++i4) {
+        for (int i4 = 0; i4 < NQ; ++i4) {
             const int c0 = 4 * lb + 32 * i4;
             const float4 sc = *reinterpret_cast<const float4 *>(ks_s + c0);
             const float4 qq = *reinterpret_cast<const float4 *>(&q_s[hb][c0]);
@@ -839,9 +951,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_gqa_kernel(const Dec
         if (mx > 0.f) e = 21 - (static_cast<int>((__float_as_uint(mx) >> 23) & 0xff) - 126);
         e = max(-120, min(120, e));
         const float scale = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
-        uint32_t dw[3][4];
+        uint32_t dw[3][NQ];
 #pragma unroll
-        for (int i4 = 0; i4 < 4; ++i4) {
+        for (int i4 = 0; i4 < NQ; ++i4) {
             const int Q0 = round_small(qv[4 * i4 + 0] * scale), Q1 = round_small(qv[4 * i4 + 1] * scale);
             const int Q2 = round_small(qv[4 * i4 + 2] * scale), Q3 = round_small(qv[4 * i4 + 3] * scale);
 #pragma unroll
@@ -854,7 +966,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_gqa_kernel(const Dec
 #pragma unroll
         for (int k = 0; k < 3; ++k)
 #pragma unroll
-            for (int i4 = 0; i4 < 4; ++i4)
+            for (int i4 = 0; i4 < NQ; ++i4)
                 reinterpret_cast<uint32_t *>(kd + (k * kGqa + hb) * Sm::kKdRow)[lb + 8 * i4] = dw[k][i4];
         if (lb == 0) {
             al[4 + hb] = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
@@ -1046,125 +1158,561 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_gqa_kernel(const Dec
         ml_s[warp][t4][1] = lsum;
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < kGqa * D; i += kDecodeThreads) {
-        const int hh = i / D, c = i % D;
-        float M = -INFINITY;
+    finish_cta<kGqa, D>(a, o_s, ml_s, bh, bq0, sigma, &last_s, o_s + kDecodeWarps * kGqa * D);
+}
+
+// ---------------------------------------------------------------------------
+// One query head per kv head: tensor-core path.
+//
+// A CTA owns one (batch, head, split); each warp takes an even-aligned,
+// contiguous share of the split's tiles and walks it in chunks of kMhaChunk
+// tiles: first the keys of the chunk (logits to shared memory, a running
+// maximum per lane), then, with the chunk's maximum fixed, its values.  So the
+// probabilities need no per-tile cross-lane maximum, key and value work form
+// two streams without dependences between tiles, and the accumulators are
+// rescaled at most once per chunk.  Items -- a key tile pair or a value tile
+// pair -- stream through a per-warp ring of cp.async stages; a key pair never
+// straddles a key group (groups of >= 32 tokens).
+//   keys   : int8 MMA m16n8k32, rows = tokens, k = channels.  A is a stored
+//            word masked to one byte slot, without a shift: slot s arrives as
+//            code * 2^(N*s).  The two 16-channel chunks of one MMA are taken
+//            from the same slot class (same 2^(N*s) for its first 8 rows, the
+//            next slot for the other 8), so the factor is constant per row of
+//            the product and is divided out of the row sum exactly.  B holds
+//            the balanced base-256 digits (each in [-128, 127]) of the 22-bit
+//            fixed-point multipliers Q_c = round(2^e q_c s_{g,c} log2(e)/sqrt(d)),
+//            built once per key group: columns 0, 1 hold digits 0, 1 and column
+//            4 digit 2, so lanes t4 = 0 and t4 = 2 of a row group hold the row's
+//            three digit sums; int32 accumulation is exact (|sum| < 2^22).
+//   values : bf16 MMA m16n8k16, rows = channels, k = tokens: A = the codes as
+//            exact bf16 2^(7-N) (2^N + code) (codes_bf16), B = p_t s_t 2^-(7-N)
+//            split into a bf16 hi part (column 0) and lo part (column 1).
+//   z-terms: bias_g = sum_c q'_c z_{g,c} and sum_t p_t s_t (z_t + 2^N) in fp32.
+// The residual rows get no split of their own: their 16-row tiles are dealt
+// round-robin to the warps of all splits, which run them on CUDA cores (staged
+// in their stage memory) before streaming and start their softmax state there.
+// ---------------------------------------------------------------------------
+constexpr int kMhaChunk = 32;     // tiles per key phase / value phase of a warp
+constexpr int kMhaStages = 4;
+
+// cp.async of one tile's code array -- lane-major in global memory, lane l's W
+// words at l*W -- into the chunk-major stage layout (16-byte piece p of lane l
+// at slot 32p + l).  Every instruction reads 512 contiguous bytes; the slots
+// one instruction writes are distinct banks in each quarter.
+template <int W>
+__device__ __forceinline__ void copy_tile_codes(unsigned char *dst, const uint32_t *src, int lane) {
+    if constexpr (W % 4 == 0) {
+        constexpr int P = W / 4;
 #pragma unroll
-        for (int w = 0; w < kDecodeWarps; ++w) M = fmaxf(M, ml_s[w][hh][0]);
-        float o = 0.f, l = 0.f;
-#pragma unroll
-        for (int w = 0; w < kDecodeWarps; ++w) {
-            if (ml_s[w][hh][0] == -INFINITY) continue;
-            const float f = exp2f(ml_s[w][hh][0] - M);
-            o = fmaf(o_s[(w * kGqa + hh) * D + c], f, o);
-            l = fmaf(ml_s[w][hh][1], f, l);
+        for (int i = 0; i < P; ++i) {
+            const int gp = 32 * i + lane;
+            cp_async16(dst + 16 * ((gp % P) * 32 + gp / P), src + 4 * gp);
         }
-        const int64_t bq = bq0 + hh;
-        a.o_part[(bq * a.S + sigma) * D + c] = o;
-        if (c == 0) {
-            a.m_part[bq * a.S + sigma] = M;
-            a.l_part[bq * a.S + sigma] = l;
+    } else {
+        static_assert(W == 2, "lane segment of 8 bytes");
+        cp_async8(dst + 8 * lane, src + 2 * lane);
+    }
+}
+
+template <int N, int D, int GV>
+struct MhaStage {                 // one item: two tiles of one code array and their meta
+    static constexpr int W = D * N / 64;
+    static constexpr int NGV = D / GV;
+    static constexpr int kCodes = 32 * W * 4;            // one tile's code array (chunk-major)
+    static constexpr int kMeta = 2 * kCodes;              // key item: scales [D] f32; value item: [32][NGV] f32
+    static constexpr int kKz = kMeta + D * 4;             // key zeros [D] i16
+    static constexpr int kVz = kMeta + 32 * NGV * 4;      // value zeros [32][NGV] i16
+    static constexpr int kEnd = (kKz + D * 2 > kVz + 32 * NGV * 2) ? kKz + D * 2 : kVz + 32 * NGV * 2;
+    static constexpr int kBytes = (kEnd + 15) / 16 * 16;
+    static_assert(kMeta % 16 == 0 && kKz % 16 == 0 && kVz % 16 == 0, "align");
+};
+
+template <int N, int D, int GV>
+struct MhaSmem {
+    static constexpr int kKdWords = D / 4 + 4;   // one digit row (4 channels a word), padded by 4 banks
+    static constexpr int kLg = kMhaStages * MhaStage<N, D, GV>::kBytes;   // logits [kMhaChunk][16] f32
+    static constexpr int kKd = kLg + kMhaChunk * 16 * 4;
+    static constexpr int kWarpBytes = kKd + 3 * kKdWords * 4;
+    static_assert(kLg % 16 == 0 && kWarpBytes % 16 == 0, "align");
+};
+
+// Value scales and zeros of the four tokens 4*t4 + i of a lane (NGV of each).
+template <int NGV>
+__device__ __forceinline__ void load_meta4(const float *sp, const int16_t *zp, bool sym, int zsym,
+                                           float (&s)[4][NGV], int (&z)[4][NGV]) {
+    if constexpr (NGV == 1) {
+        const float4 v = *reinterpret_cast<const float4 *>(sp);
+        s[0][0] = v.x; s[1][0] = v.y; s[2][0] = v.z; s[3][0] = v.w;
+        if (sym) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) z[i][0] = zsym;
+        } else {
+            const uint2 u = *reinterpret_cast<const uint2 *>(zp);
+            z[0][0] = static_cast<int16_t>(u.x & 0xffffu); z[1][0] = static_cast<int16_t>(u.x >> 16);
+            z[2][0] = static_cast<int16_t>(u.y & 0xffffu); z[3][0] = static_cast<int16_t>(u.y >> 16);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            int16_t zz[NGV];
+            load_meta<NGV>(sp + i * NGV, zp + i * NGV, sym, zsym, s[i], zz);
+#pragma unroll
+            for (int v = 0; v < NGV; ++v) z[i][v] = zz[v];
         }
     }
 }
 
-// Log-sum-exp merge of the S split partials of one (batch, query head).
-__global__ void combine_kernel(const float *o_part, const float *m_part, const float *l_part,
-                               float *out, int S, int D) {
-    const int64_t bq = blockIdx.x;
-    float M = -INFINITY;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, m_part[bq * S + s]);
-    for (int c = threadIdx.x; c < D; c += blockDim.x) {
-        float o = 0.f, l = 0.f;
-        for (int s = 0; s < S; ++s) {
-            const float ms = m_part[bq * S + s];
-            if (ms == -INFINITY) continue;
-            const float f = exp2f(ms - M);
-            o = fmaf(o_part[(bq * S + s) * D + c], f, o);
-            l = fmaf(l_part[bq * S + s], f, l);
+template <int N, int D, int GV>
+__global__ void __launch_bounds__(kDecodeThreads, (D / GV >= 4) ? 3 : 4) decode_mha_kernel(const DecodeArgs a) {
+    constexpr int W = D * N / 64;
+    constexpr int TW = D * N / 2;
+    constexpr int NJ = D / 16;
+    constexpr int BPW = 4 / N;        // slot classes (chunks per word)
+    constexpr int NP = W / 2;         // word pairs; the key MMAs of a tile are (pair, class)
+    constexpr int NGV = D / GV;
+    constexpr uint32_t BYTE_L = ((1u << N) - 1u) * 0x01010101u;
+    constexpr int kSt = kMhaStages;
+    using St = MhaStage<N, D, GV>;
+    using Sm = MhaSmem<N, D, GV>;
+    static_assert(W % 2 == 0, "key MMAs take words in pairs");
+    static_assert(kMhaChunk % 2 == 0 && (kMhaChunk & (kMhaChunk - 1)) == 0, "chunk");
+
+    __shared__ __align__(16) float q_s[D];
+    __shared__ float ml_s[kDecodeWarps][1][2];
+    __shared__ int last_s;
+    extern __shared__ __align__(128) unsigned char stage_mem[];
+
+    const int qi = blockIdx.x, b = blockIdx.y, sigma = blockIdx.z;
+    const int64_t bh = static_cast<int64_t>(b) * a.Hkv + qi;
+    const int64_t bq = static_cast<int64_t>(b) * a.Hq + qi;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g8 = lane >> 2, t4 = lane & 3;
+    unsigned char *wmem = stage_mem + static_cast<size_t>(warp) * Sm::kWarpBytes;
+    float *lgs = reinterpret_cast<float *>(wmem + Sm::kLg);
+    uint32_t *kd = reinterpret_cast<uint32_t *>(wmem + Sm::kKd);
+    const int zsym = 1 << (N - 1);
+
+    for (int c = threadIdx.x; c < D; c += kDecodeThreads)
+        q_s[c] = widen(a.q[bq * D + c], a.bf16) * a.qscale;
+    __syncthreads();
+
+    float m = -INFINITY, lsum = 0.f;
+    float ov[NJ][2];   // channels 16j + g8 (+8), final in lanes t4 == 0
+
+    {
+        // ---------------- quantized split ----------------
+        const int t_begin = sigma * a.tiles_per_split;                 // even
+        const int t_end = min(a.n_qtiles, t_begin + a.tiles_per_split);
+        const int per_w = 2 * ((t_end - t_begin + 2 * kDecodeWarps - 1) / (2 * kDecodeWarps));
+        const int wb = min(t_end, t_begin + warp * per_w);             // even
+        const int ntiles = min(t_end, wb + per_w) - wb;
+        const int nitems = 2 * ((ntiles + 1) / 2);   // one key item and one value item per tile pair
+        const int64_t groups_cap = a.cap / a.G;
+        const int64_t tile0 = bh * (a.cap / 16) + wb;
+        const uint32_t *kp = a.kc + tile0 * TW;
+        const uint32_t *vp = a.vc + tile0 * TW;
+        const float *vsp = a.vs + tile0 * 16 * NGV;
+        const int16_t *vzp = a.sym ? nullptr : a.vz + tile0 * 16 * NGV;
+        const int gmask = (1 << a.gshift) - 1;
+        const int n_vs = 4 * NGV, n_meta = a.sym ? n_vs : 6 * NGV;   // 16-byte pieces per value tile
+
+        // Item cursor: chunk [cb, cb + kMhaChunk) of the warp's tiles holds np tile pairs; items
+        // 0 .. np-1 of a chunk are its key pairs, np .. 2np-1 its value pairs.
+        struct Cursor {
+            int cb, r, np;
+            __device__ void start(int ntiles) { cb = 0; r = 0; np = (min(kMhaChunk, ntiles) + 1) / 2; }
+            __device__ void next(int ntiles) {
+                if (++r == 2 * np) {
+                    cb += kMhaChunk;
+                    r = 0;
+                    np = (min(kMhaChunk, ntiles - cb) + 1) / 2;
+                }
+            }
+            __device__ bool key() const { return r < np; }
+            __device__ int rel() const { return cb + 2 * (r < np ? r : r - np); }
+        };
+
+        Cursor ic;       // producer's cursor, kSt - 1 items ahead
+        ic.start(ntiles);
+        int issued = 0;
+        auto issue_next = [&]() {
+            if (issued < nitems) {
+                unsigned char *st = wmem + (issued % kSt) * St::kBytes;
+                const int rel = ic.rel();
+                const bool two = rel + 1 < ntiles;
+                if (ic.key()) {
+                    const uint32_t *src = kp + static_cast<int64_t>(rel) * TW;
+                    copy_tile_codes<W>(st, src, lane);
+                    if (two) copy_tile_codes<W>(st + St::kCodes, src + TW, lane);
+                    const int ti = wb + rel;
+                    if (rel == 0 || (ti & gmask) == 0) {
+                        const int64_t gofs = (bh * groups_cap + (ti >> a.gshift)) * D;
+                        for (int c = lane; c < (a.sym ? D / 4 : D / 4 + D / 8); c += 32) {
+                            if (c < D / 4) cp_async16(st + St::kMeta + 16 * c, a.ks + gofs + 4 * c);
+                            else cp_async16(st + St::kKz + 16 * (c - D / 4), a.kz + gofs + 8 * (c - D / 4));
+                        }
+                    }
+                } else {
+                    const uint32_t *src = vp + static_cast<int64_t>(rel) * TW;
+                    copy_tile_codes<W>(st, src, lane);
+                    if (two) copy_tile_codes<W>(st + St::kCodes, src + TW, lane);
+                    const int64_t tok = static_cast<int64_t>(rel) * 16 * NGV;
+                    const int nvs = two ? 2 * n_vs : n_vs;
+                    for (int c = lane; c < (two ? 2 * n_meta : n_meta); c += 32) {
+                        if (c < nvs) cp_async16(st + St::kMeta + 16 * c, vsp + tok + 4 * c);
+                        else cp_async16(st + St::kVz + 16 * (c - nvs), vzp + tok + 8 * (c - nvs));
+                    }
+                }
+                ic.next(ntiles);
+            }
+            cp_async_commit();
+            ++issued;
+        };
+
+        float dv[NJ][4];   // value MMA accumulators: rows = channels 16j + g8 (+8), columns 2*t4, 2*t4 + 1
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) dv[j][0] = dv[j][1] = dv[j][2] = dv[j][3] = 0.f;
+        float zsum[NGV];
+#pragma unroll
+        for (int v = 0; v < NGV; ++v) zsum[v] = 0.f;
+        uint32_t kb[NP * BPW][2];   // key MMA B fragments of the current group
+        float klane = 0.f, kbias = 0.f;
+        float mloc = -INFINITY;     // this lane's largest logit of the current chunk
+
+        // Key digits of the group the stage opens: lane l builds channels 4l .. 4l+3.
+        auto rebuild_key_digits = [&](const unsigned char *st) {
+            const int cl = lane % (D / 4);
+            const float4 sc = *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(st + St::kMeta) + 4 * cl);
+            const float4 qq = *reinterpret_cast<const float4 *>(q_s + 4 * cl);
+            const float qv[4] = {qq.x * sc.x, qq.y * sc.y, qq.z * sc.z, qq.w * sc.w};
+            float z[4] = {static_cast<float>(zsym), static_cast<float>(zsym), static_cast<float>(zsym),
+                          static_cast<float>(zsym)};
+            if (!a.sym) {
+                const uint2 zz = *reinterpret_cast<const uint2 *>(reinterpret_cast<const int16_t *>(st + St::kKz) + 4 * cl);
+                z[0] = small_int_to_float(static_cast<int16_t>(zz.x & 0xffffu));
+                z[1] = small_int_to_float(static_cast<int16_t>(zz.x >> 16));
+                z[2] = small_int_to_float(static_cast<int16_t>(zz.y & 0xffffu));
+                z[3] = small_int_to_float(static_cast<int16_t>(zz.y >> 16));
+            }
+            float kbp = 0.f, mx = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                kbp = fmaf(qv[i], z[i], kbp);
+                mx = fmaxf(mx, fabsf(qv[i]));
+            }
+            if (lane >= D / 4) kbp = 0.f;    // d = 64: lanes 16..31 repeat channels
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                kbp += __shfl_xor_sync(0xffffffffu, kbp, o);
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            }
+            // 2^e with |q'| 2^e < 2^21, from the exponent of the largest |q'|
+            int e = 0;
+            if (mx > 0.f) e = 21 - (static_cast<int>((__float_as_uint(mx) >> 23) & 0xff) - 126);
+            e = max(-120, min(120, e));
+            const float scale = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+            // balanced base-256 digits: Q = d0 + 256 d1 + 65536 d2 with d0, d1 in [-128, 127]
+            int dg[3][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int Q = round_small(qv[i] * scale);
+                const int Q1 = (Q + 128) >> 8;
+                dg[0][i] = Q;
+                dg[1][i] = Q1;
+                dg[2][i] = (Q1 + 128) >> 8;
+            }
+            __syncwarp();   // the previous group's digits have been read
+            if (lane < D / 4) {
+#pragma unroll
+                for (int k = 0; k < 3; ++k)
+                    kd[k * Sm::kKdWords + cl] = __byte_perm(__byte_perm(dg[k][0], dg[k][1], 0x0040),
+                                                            __byte_perm(dg[k][2], dg[k][3], 0x0040), 0x5410);
+            }
+            __syncwarp();
+            // B fragments: column g8 holds digit 0 (g8 = 0), 1 (g8 = 1) or 2 (g8 = 4)
+            const int dig = g8 == 0 ? 0 : (g8 == 1 ? 1 : 2);
+            const bool has = g8 == 0 || g8 == 1 || g8 == 4;
+            const uint32_t *row = kd + dig * Sm::kKdWords;
+#pragma unroll
+            for (int pm = 0; pm < NP; ++pm) {
+#pragma unroll
+                for (int c = 0; c < BPW; ++c) {
+                    const int j1 = 2 * pm * BPW + c, j2 = j1 + BPW;
+                    kb[pm * BPW + c][0] = has ? row[4 * j1 + t4] : 0u;
+                    kb[pm * BPW + c][1] = has ? row[4 * j2 + t4] : 0u;
+                }
+            }
+            const float kinv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+            klane = t4 == 2 ? kinv * 65536.f : kinv;
+            kbias = kbp;
+        };
+
+        // This warp's share of the residual tiles (dealt round-robin over the warps of all
+        // splits), on CUDA cores in the stage memory before the stream starts.  Its result
+        // seeds the softmax state: lane t4 = 0 holds channels 16j + g8 (+8) in both layouts,
+        // and lsum carries the B operand's 2^-(7-N).
+        static_assert(residual_scratch_bytes<D>() <= Sm::kWarpBytes, "residual staging");
+        {
+            const int nres = (a.r + 15) / 16;
+            const int gw = sigma * kDecodeWarps + warp, nw = a.S * kDecodeWarps;
+            if (gw < nres) {
+                float lr = 0.f;
+                float2 acc[NJ][2];
+#pragma unroll
+                for (int j = 0; j < NJ; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
+                residual_pass<D>(a, q_s, a.kr + bh * a.R * D, a.vr + bh * a.R * D, gw, nres, lane, m, lr,
+                                 acc, wmem, nw);
+                lr += __shfl_xor_sync(0xffffffffu, lr, 4);     // lanes hold rows g8, g8 + 8
+                lr += __shfl_xor_sync(0xffffffffu, lr, 8);
+                lr += __shfl_xor_sync(0xffffffffu, lr, 16);
+#pragma unroll
+                for (int j = 0; j < NJ; ++j) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        float val = acc[j][h].x + acc[j][h].y;
+                        val += __shfl_xor_sync(0xffffffffu, val, 1);
+                        val += __shfl_xor_sync(0xffffffffu, val, 2);
+                        dv[j][2 * h] = t4 == 0 ? val : 0.f;
+                    }
+                }
+                lsum = t4 == 0 ? lr / static_cast<float>(1 << (7 - N)) : 0.f;
+            }
         }
-        out[bq * D + c] = o / l;
+
+#pragma unroll
+        for (int s = 0; s < kSt - 1; ++s) issue_next();
+
+        Cursor cc;       // consumer's cursor
+        cc.start(ntiles);
+        for (int k = 0; k < nitems; ++k) {
+            issue_next();
+            cp_async_wait<kSt - 1>();
+            __syncwarp();
+            const unsigned char *st = wmem + (k % kSt) * St::kBytes;
+            const int rel = cc.rel();
+            const int nt = rel + 1 < ntiles ? 2 : 1;
+            float *lgc = lgs + (rel % kMhaChunk) * 16;   // logits of tiles rel, rel + 1
+            if (cc.key()) {
+                if (rel == 0 || ((wb + rel) & gmask) == 0) rebuild_key_digits(st);
+                // ---- key MMAs: log2-domain logits of tokens g8 and g8 + 8 ----
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    if (u < nt) {
+                        uint32_t kw[W];
+                        load_stage_words<W>(reinterpret_cast<const uint32_t *>(st + u * St::kCodes), lane, kw);
+                        int acc[2][BPW][4];   // two chains (even / odd word pair)
+#pragma unroll
+                        for (int pm = 0; pm < NP; ++pm) {
+#pragma unroll
+                            for (int c = 0; c < BPW; ++c) {
+                                const uint32_t mlo = BYTE_L << (N * 2 * c), mhi = BYTE_L << (N * (2 * c + 1));
+                                const uint32_t af[4] = {kw[2 * pm] & mlo, kw[2 * pm] & mhi, kw[2 * pm + 1] & mlo,
+                                                        kw[2 * pm + 1] & mhi};
+                                if (pm < 2) imma_us0(acc[pm][c], af, kb[pm * BPW + c][0], kb[pm * BPW + c][1]);
+                                else imma_us(acc[pm & 1][c], af, kb[pm * BPW + c][0], kb[pm * BPW + c][1]);
+                            }
+                        }
+                        float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+                        for (int c = 0; c < BPW; ++c) {   // digit sums d0 + 256 d1 (< 2^31), slot factor out
+                            const float f0 = 1.0f / static_cast<float>(1u << (2 * N * c));
+                            const float f1 = 1.0f / static_cast<float>(1u << (N * (2 * c + 1)));
+                            int r0 = acc[0][c][0] + acc[0][c][1] * 256, r1 = acc[0][c][2] + acc[0][c][3] * 256;
+                            if constexpr (NP > 1) {
+                                r0 += acc[1][c][0] + acc[1][c][1] * 256;
+                                r1 += acc[1][c][2] + acc[1][c][3] * 256;
+                            }
+                            x0 = fmaf(static_cast<float>(r0), f0, x0);
+                            x1 = fmaf(static_cast<float>(r1), f1, x1);
+                        }
+                        x0 *= klane;
+                        x1 *= klane;
+                        x0 += __shfl_xor_sync(0xffffffffu, x0, 1);
+                        x1 += __shfl_xor_sync(0xffffffffu, x1, 1);
+                        x0 += __shfl_xor_sync(0xffffffffu, x0, 2);
+                        x1 += __shfl_xor_sync(0xffffffffu, x1, 2);
+                        const float lg0 = x0 - kbias, lg1 = x1 - kbias;
+                        mloc = fmaxf(mloc, fmaxf(lg0, lg1));
+                        if (t4 == 0) {
+                            lgc[16 * u + g8] = lg0;
+                            lgc[16 * u + g8 + 8] = lg1;
+                        }
+                    }
+                }
+                if (cc.r == cc.np - 1) {
+                    // the chunk's keys are done: fix its maximum, rescale what came before
+                    float cm = mloc;
+                    cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 4));
+                    cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 8));
+                    cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 16));
+                    if (cm > m) {
+                        const float alpha = fast_exp2(m - cm);
+                        m = cm;
+                        lsum *= alpha;
+#pragma unroll
+                        for (int j = 0; j < NJ; ++j) {
+                            dv[j][0] *= alpha; dv[j][1] *= alpha; dv[j][2] *= alpha; dv[j][3] *= alpha;
+                        }
+#pragma unroll
+                        for (int v = 0; v < NGV; ++v) zsum[v] *= alpha;
+                    }
+                    mloc = -INFINITY;
+                }
+            } else {
+                // p 2^-(7-N) of tokens 4*t4 + i (the B scale folded into the exponent)
+                const float mb = m + static_cast<float>(7 - N);
+                constexpr int kOff = 1 << N;
+                const bool lo_part = (g8 & 1) != 0;   // B column g8: hi part (even), lo part (odd)
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    if (u < nt) {
+                        const float4 l4 = *reinterpret_cast<const float4 *>(lgc + 16 * u + 4 * t4);
+                        const float pt[4] = {fast_exp2(l4.x - mb), fast_exp2(l4.y - mb), fast_exp2(l4.z - mb),
+                                             fast_exp2(l4.w - mb)};
+                        lsum += (pt[0] + pt[1]) + (pt[2] + pt[3]);
+                        float sv[4][NGV];
+                        int zv[4][NGV];
+                        load_meta4<NGV>(reinterpret_cast<const float *>(st + St::kMeta) + (16 * u + 4 * t4) * NGV,
+                                        reinterpret_cast<const int16_t *>(st + St::kVz) + (16 * u + 4 * t4) * NGV,
+                                        a.sym, zsym, sv, zv);
+                        uint32_t B0[NGV], B1[NGV];
+#pragma unroll
+                        for (int v = 0; v < NGV; ++v) {
+                            float ps[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                ps[i] = pt[i] * sv[i][v];
+                                zsum[v] = fmaf(ps[i], small_int_to_float(zv[i][v] + kOff), zsum[v]);
+                            }
+                            // k order of the B fragment: (4t4, 4t4+2 | 4t4+1, 4t4+3), as codes_bf16 pairs
+                            // bytes; columns 2..7 repeat columns 0, 1 and their sums are not read
+                            const uint32_t h02 = f2bf2(ps[0], ps[2]), h13 = f2bf2(ps[1], ps[3]);
+                            const uint32_t l02 = f2bf2(ps[0] - __uint_as_float(h02 << 16),
+                                                       ps[2] - __uint_as_float(h02 & 0xffff0000u));
+                            const uint32_t l13 = f2bf2(ps[1] - __uint_as_float(h13 << 16),
+                                                       ps[3] - __uint_as_float(h13 & 0xffff0000u));
+                            B0[v] = lo_part ? l02 : h02;
+                            B1[v] = lo_part ? l13 : h13;
+                        }
+                        // ---- value MMAs: rows = channels of chunk j, k = the tile's tokens ----
+                        uint32_t vw[W];
+                        load_stage_words<W>(reinterpret_cast<const uint32_t *>(st + u * St::kCodes), lane, vw);
+                        const uint32_t magic16 = 0x43004300u;
+#pragma unroll
+                        for (int j = 0; j < NJ; ++j) {
+                            uint32_t a02, a13, b02, b13;
+                            codes_bf16<N>(vw[j / BPW], 2 * (j % BPW), magic16, a02, a13);       // channel 16j + g8
+                            codes_bf16<N>(vw[j / BPW], 2 * (j % BPW) + 1, magic16, b02, b13);   // channel 16j + g8 + 8
+                            hmma(dv[j], a02, b02, a13, b13, B0[(16 * j) / GV], B1[(16 * j) / GV]);
+                        }
+                    }
+                }
+            }
+            cc.next(ntiles);
+            __syncwarp();   // stage consumed and the chunk's logits visible to every lane
+        }
+        cp_async_wait<0>();
+
+        // lanes with the same t4 hold the same token sums: reduce over t4; lsum and zsum carry
+        // the 2^-(7-N) of the B operand, dv sums (2^N + code) p s
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+        lsum *= static_cast<float>(1 << (7 - N));
+#pragma unroll
+        for (int v = 0; v < NGV; ++v) {
+            zsum[v] += __shfl_xor_sync(0xffffffffu, zsum[v], 1);
+            zsum[v] += __shfl_xor_sync(0xffffffffu, zsum[v], 2);
+        }
+        constexpr float kUnscale = static_cast<float>(1 << (7 - N));
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+            const float z = zsum[(16 * j) / GV] * kUnscale;
+            ov[j][0] = dv[j][0] + dv[j][1] - z;
+            ov[j][1] = dv[j][2] + dv[j][3] - z;
+        }
     }
+
+    __syncthreads();   // stage memory is reused for the per-warp outputs
+    float *o_s = reinterpret_cast<float *>(stage_mem);   // [warp][D]
+    if (t4 == 0) {
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+            o_s[warp * D + 16 * j + g8] = ov[j][0];
+            o_s[warp * D + 16 * j + g8 + 8] = ov[j][1];
+        }
+    }
+    if (lane == 0) {
+        ml_s[warp][0][0] = m;
+        ml_s[warp][0][1] = lsum;
+    }
+    __syncthreads();
+    finish_cta<1, D>(a, o_s, ml_s, bq, bq, sigma, &last_s, o_s + kDecodeWarps * D);
 }
 
 template <int N, int D, int GV>
 constexpr int split_smem() { return kDecodeWarps * kStages * Stage<N, D, GV>::kBytes; }
-
-template <int N, int D, int GV>
-cudaError_t launch_split(const DecodeArgs &a, cudaStream_t s) {
-    // the dynamic shared-memory opt-in is per device; do it once per device
-    static bool configured[64] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev >= 64 || !configured[dev]) {
-        e = cudaFuncSetAttribute(decode_split_kernel<N, D, GV>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 split_smem<N, D, GV>());
-        if (e != cudaSuccess) return e;
-        if (dev < 64) configured[dev] = true;
-    }
-    dim3 grid(a.S, a.Hq, a.B);
-    decode_split_kernel<N, D, GV><<<grid, kDecodeThreads, split_smem<N, D, GV>(), s>>>(a);
-    count_launches(1);
-    return cudaGetLastError();
-}
-
 template <int N, int D, int GV>
 constexpr int gqa_smem() { return kDecodeWarps * GqaSmem<N, D, GV>::kWarpBytes; }
-
 template <int N, int D, int GV>
-cudaError_t launch_gqa(const DecodeArgs &a, cudaStream_t s) {
+constexpr int mha_smem() { return kDecodeWarps * MhaSmem<N, D, GV>::kWarpBytes; }
+
+// The opt-in to more than 48 KB of dynamic shared memory is per device and per
+// kernel; it is made once for each.
+template <auto Kernel>
+cudaError_t configure_smem(int smem) {
     static bool configured[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 64 || !configured[dev]) {
-        e = cudaFuncSetAttribute(decode_gqa_kernel<N, D, GV>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, gqa_smem<N, D, GV>());
-        if (e != cudaSuccess) return e;
-        if (dev < 64) configured[dev] = true;
-    }
-    dim3 grid(a.S, a.Hkv, a.B);
-    decode_gqa_kernel<N, D, GV><<<grid, kDecodeThreads, gqa_smem<N, D, GV>(), s>>>(a);
+    if (dev < 64 && configured[dev]) return cudaSuccess;
+    e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess && dev < 64) configured[dev] = true;
+    return e;
+}
+
+template <auto Kernel>
+cudaError_t launch_kernel(const DecodeArgs &a, dim3 grid, int smem, cudaStream_t s) {
+    cudaError_t e = configure_smem<Kernel>(smem);
+    if (e != cudaSuccess) return e;
+    Kernel<<<grid, kDecodeThreads, smem, s>>>(a);
     count_launches(1);
     return cudaGetLastError();
 }
 
-template <int N, int D, int GV>
-int gqa_occupancy() {
+template <auto Kernel>
+int occupancy_of(int smem) {
     int n = 0;
-    if (cudaFuncSetAttribute(decode_gqa_kernel<N, D, GV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             gqa_smem<N, D, GV>()) != cudaSuccess)
-        return 1;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_gqa_kernel<N, D, GV>, kDecodeThreads,
-                                                      gqa_smem<N, D, GV>()) != cudaSuccess)
+    if (configure_smem<Kernel>(smem) != cudaSuccess) return 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kernel, kDecodeThreads, smem) != cudaSuccess)
         return 1;
     return n > 0 ? n : 1;
 }
 
-template <int N, int D, int GV>
-int occupancy() {
-    int n = 0;
-    if (cudaFuncSetAttribute(decode_split_kernel<N, D, GV>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             split_smem<N, D, GV>()) != cudaSuccess)
-        return 1;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_split_kernel<N, D, GV>,
-                                                      kDecodeThreads, split_smem<N, D, GV>()) !=
-        cudaSuccess)
-        return 1;
-    return n > 0 ? n : 1;
-}
-
-// Dispatch over the compiled (bits, head_dim, value-group) variants.
+// Dispatch over the compiled (bits, head_dim, value-group) variants and the three kernels.
+// The split index is the slowest grid dimension: CTAs start in linear order, so every
+// quantized split is resident before the (short) residual-split CTAs fill the slots
+// that remain.
 template <int N, int D, int GV>
 struct LaunchF {
     static cudaError_t run(const DecodeArgs &a, cudaStream_t s) {
-        return a.gqa ? launch_gqa<N, D, GV>(a, s) : launch_split<N, D, GV>(a, s);
+        switch (a.path) {
+            case kPathGqa:
+                return launch_kernel<decode_gqa_kernel<N, D, GV>>(a, dim3(a.Hkv, a.B, a.S),
+                                                                  gqa_smem<N, D, GV>(), s);
+            case kPathMha:
+                return launch_kernel<decode_mha_kernel<N, D, GV>>(a, dim3(a.Hq, a.B, a.S),
+                                                                  mha_smem<N, D, GV>(), s);
+            default:
+                return launch_kernel<decode_split_kernel<N, D, GV>>(a, dim3(a.Hq, a.B, a.S),
+                                                                    split_smem<N, D, GV>(), s);
+        }
     }
     static int occ(const DecodeArgs &a) {
-        return a.gqa ? gqa_occupancy<N, D, GV>() : occupancy<N, D, GV>();
+        switch (a.path) {
+            case kPathGqa: return occupancy_of<decode_gqa_kernel<N, D, GV>>(gqa_smem<N, D, GV>());
+            case kPathMha: return occupancy_of<decode_mha_kernel<N, D, GV>>(mha_smem<N, D, GV>());
+            default: return occupancy_of<decode_split_kernel<N, D, GV>>(split_smem<N, D, GV>());
+        }
     }
 };
 
@@ -1198,11 +1746,7 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
     else if (a.bits == 2 && a.d == 128) e = launch_gv<2, 128>(a, s);
     else if (a.bits == 4 && a.d == 64) e = launch_gv<4, 64>(a, s);
     else if (a.bits == 4 && a.d == 128) e = launch_gv<4, 128>(a, s);
-    if (e != cudaSuccess) return e;
-    combine_kernel<<<static_cast<unsigned>(static_cast<int64_t>(a.B) * a.Hq), a.d, 0, s>>>(
-        a.o_part, a.m_part, a.l_part, a.out, a.S, a.d);
-    count_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 int decode_ctas_per_sm(const DecodeArgs &a) {

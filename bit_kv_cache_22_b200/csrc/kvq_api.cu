@@ -101,6 +101,7 @@ int max_splits(const kvq_config *c) {
 struct kvq_cache {
     kvq_config cfg;
     kvq_buffers buf;
+    unsigned int *arrivals = nullptr;   // device, B * Hq split-arrival counters (library-owned)
     int64_t Tq = 0;
     int32_t r = 0;
     int num_sms = 148;
@@ -111,19 +112,29 @@ struct kvq_cache {
 namespace {
 
 // Split count for the current cache length.  The quantized tiles are cut into
-// n_qsplits contiguous splits; the residual rows (if any) get one split of
-// their own.  A quantized split's time is modelled as its tiles per warp plus a
-// fixed start/finish cost of ~3 tiles, the kernel's time as that times the
-// number of waves of CTAs over the GPU's resident slots; the split count with
-// the lowest modelled time wins (ties: fewer splits).
+// n_qsplits contiguous splits (of a multiple of the path's tile alignment); the
+// residual rows (if any) get one split of their own.  A CTA's time is modelled
+// as a fixed start/finish cost of kCtaFixedTiles tiles plus the tiles its
+// busiest warp streams; the kernel's time as the larger of (the waves of
+// quantized CTAs over the GPU's resident slots x one quantized CTA) and (all
+// CTA time spread evenly over the slots, plus one residual CTA).  The split
+// count with the lowest modelled time wins (ties: fewer splits).
+constexpr double kCtaFixedTiles = 6.0;
+
 void plan_splits(const kvq_cache *h, int *n_qsplits, int *tiles_per_split, int *S_out) {
     const kvq_config &c = h->cfg;
     const int64_t tiles = h->Tq / 16;
-    const int extra = h->r > 0 ? 1 : 0;
+    const int path = kvq::decode_path(c.q_heads, c.kv_heads, c.group_k);
+    // the MHA kernel deals the residual tiles to the warps of the quantized splits
+    const bool res_shared = path == kvq::kPathMha;
+    const int extra = (h->r > 0 && !res_shared) ? 1 : 0;
+    const int64_t align = kvq::split_tile_align(path);
     // CTAs per split: one per query head, or one per kv head on the grouped-query path
-    const int64_t units = static_cast<int64_t>(c.batch) *
-                          (c.q_heads == 4 * c.kv_heads ? c.kv_heads : c.q_heads);
-    const int64_t slots = static_cast<int64_t>(h->num_sms) * h->ctas_per_sm;
+    const int64_t units = static_cast<int64_t>(c.batch) * (path == kvq::kPathGqa ? c.kv_heads : c.q_heads);
+    const double slots = static_cast<double>(h->num_sms) * h->ctas_per_sm;
+    const int64_t nres = (h->r + 15) / 16;
+    // residual CTA: its tiles shared by the 4 warps, or one warp per query head (grouped-query path)
+    const double c_res = kCtaFixedTiles + static_cast<double>(path == kvq::kPathGqa ? nres : (nres + 3) / 4);
     int64_t best_S = 0, best_per = 1;
     if (tiles > 0) {
         int64_t cap = (tiles + kMinTilesPerSplit - 1) / kMinTilesPerSplit;
@@ -132,16 +143,27 @@ void plan_splits(const kvq_cache *h, int *n_qsplits, int *tiles_per_split, int *
         if (cap < 1) cap = 1;
         double best_cost = -1.0;
         for (int64_t S = 1; S <= cap; ++S) {
-            const int64_t per = (tiles + S - 1) / S;
+            const int64_t per = ((tiles + S - 1) / S + align - 1) / align * align;
             if ((tiles + per - 1) / per != S) continue;
-            const int64_t waves = (units * (S + extra) + slots - 1) / slots;
-            const double cost = static_cast<double>(waves) * ((per + 3) / 4 + 3);
-            if (best_cost < 0 || cost < best_cost) {
+            const int64_t per_warp = ((per + 4 * align - 1) / (4 * align)) * align;
+            // a residual tile on CUDA cores costs about two quantized tiles
+            const int64_t res_warp = res_shared ? (nres + 4 * S - 1) / (4 * S) : 0;
+            const double c_q = kCtaFixedTiles + static_cast<double>(per_warp + 2 * res_warp);
+            const double nq = static_cast<double>(units * S);
+            const double t_waves = std::ceil(nq / slots) * c_q;
+            const double t_spread = (nq * c_q + static_cast<double>(units * extra) * c_res) / slots +
+                                    (extra ? c_res : 0.0);
+            const double cost = t_waves > t_spread ? t_waves : t_spread;
+            if (best_cost < 0 || cost < best_cost - 1e-9) {
                 best_cost = cost;
                 best_S = S;
                 best_per = per;
             }
         }
+    }
+    if (res_shared && best_S == 0) {   // residual rows only: one split whose warps share them
+        best_S = 1;
+        best_per = 0;
     }
     *n_qsplits = static_cast<int>(best_S);
     *tiles_per_split = static_cast<int>(best_per);
@@ -170,7 +192,8 @@ kvq::DecodeArgs decode_args(const kvq_cache *h) {
     a.bits = c.bits;
     a.sym = c.symmetric != 0;
     a.bf16 = c.dtype == KVQ_BF16;
-    a.gqa = c.q_heads == 4 * c.kv_heads;
+    a.path = kvq::decode_path(c.q_heads, c.kv_heads, c.group_k);
+    a.arrivals = h->arrivals;
     a.gshift = 0;
     while ((16 << a.gshift) < c.group_k) ++a.gshift;
     a.qscale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c.head_dim)));
@@ -248,11 +271,25 @@ kvq_status kvq_create(const kvq_config *cfg, const kvq_buffers *bufs, kvq_cache 
     }
     h->num_sms = sms > 0 ? sms : 148;
     h->ctas_per_sm = kvq::decode_ctas_per_sm(decode_args(h));
+    // the decode kernels' split-arrival counters: zeroed once here, left at zero by every decode
+    const size_t counter_bytes = static_cast<size_t>(cfg->batch) * cfg->q_heads * sizeof(unsigned int);
+    e = cudaMalloc(&h->arrivals, counter_bytes);
+    if (e == cudaSuccess) e = cudaMemset(h->arrivals, 0, counter_bytes);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) {
+        if (h->arrivals) cudaFree(h->arrivals);
+        delete h;
+        return cuda_fail(e, "allocating the split-arrival counters");
+    }
     *out = h;
     return ok();
 }
 
-void kvq_destroy(kvq_cache *cache) { delete cache; }
+void kvq_destroy(kvq_cache *cache) {
+    if (!cache) return;
+    if (cache->arrivals) cudaFree(cache->arrivals);
+    delete cache;
+}
 
 kvq_status kvq_reset(kvq_cache *cache) {
     if (!cache) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");

@@ -69,6 +69,48 @@ def test_split_count_does_not_change_the_result(limit):
     run_episode(w, split_limit=limit)
 
 
+@pytest.mark.parametrize("limit", [1, 3, 64])
+def test_split_count_does_not_change_the_result_mha(limit):
+    # one query head per kv head: splits cut tile pairs; odd limits give uneven splits
+    w = reduced(wl.WORKLOADS["llama7b"]).replace(steps=3)
+    run_episode(w, split_limit=limit)
+
+
+# (q heads per kv head, d, bits, G, Gv, R): every decode kernel and its ragged shapes --
+# the tensor-core MHA kernel (g = 1, G >= 32), the grouped-query kernel (g = 4) and
+# the CUDA-core split kernel (16-token key groups, any other g)
+PATHS = [(1, 128, 4, 32, 64, 64), (1, 64, 2, 64, 16, 64), (1, 128, 2, 16, 32, 32),
+         (2, 128, 2, 32, 32, 64), (8, 64, 4, 32, 32, 32), (4, 64, 4, 16, 16, 32),
+         (1, 64, 4, 256, 64, 256)]
+
+
+@pytest.mark.parametrize("g,d,bits,G,Gv,R", PATHS)
+def test_every_decode_path(g, d, bits, G, Gv, R):
+    base = wl.WORKLOADS["stream2"]
+    w = base.replace(B=2, Hkv=2, Hq=2 * g, d=d, bits=bits, G=G, Gv=Gv, R=R, T=3 * R + 37,
+                     steps=R + 5, k_outlier_channels=2)
+    run_episode(w, check_every=7)
+
+
+def test_repeated_decodes_are_identical_across_split_counts():
+    """The split-merge counters return to zero after every call: the same query
+    gives the same output call after call, whatever the split count in between."""
+    w = reduced(wl.WORKLOADS["llama7b"]).replace(steps=1)
+    XK, XV = wl.prefill_bits(w)
+    _, _, tQ = wl.decode_bits(w)
+    cache = tl.new_cache(w)
+    cache.prefill_quantize(tl.to_dev(XK, w), tl.to_dev(XV, w))
+    q = tl.to_dev(tQ[0], w)
+    first = cache.decode_attention(q).clone()
+    for limit in (5, 1, 64, 2, 64):
+        cache.set_split_limit(limit)
+        out = cache.decode_attention(q)
+        if limit == 64:
+            assert torch.equal(out, first)
+        else:
+            tl.assert_close(out.cpu().numpy(), first.cpu().numpy().astype(np.float64), f"limit {limit}")
+
+
 def test_prefill_then_append_equals_longer_prefill_on_gpu():
     w = reduced(wl.WORKLOADS["stream2"])
     T, k = 100, 170
@@ -87,10 +129,11 @@ def test_prefill_then_append_equals_longer_prefill_on_gpu():
     assert torch.equal(a.v_residual[:, :r], b.v_residual[:, :r])
 
 
+@pytest.mark.parametrize("name", ["gqa8b", "llama7b"])
 @pytest.mark.parametrize("T", [1, 15, 16, 127])
-def test_all_residual_and_tiny_prompts(T):
+def test_all_residual_and_tiny_prompts(T, name):
     """No quantized token (T < R): plain softmax attention over the residual."""
-    w = reduced(wl.WORKLOADS["gqa8b"]).replace(T=T, steps=2)
+    w = reduced(wl.WORKLOADS[name]).replace(T=T, steps=2)
     run_episode(w)
 
 
