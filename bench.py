@@ -89,11 +89,7 @@ def peaks():
 
 def decode_kernel_name(w) -> str:
     """The decode kernel the library launches for this geometry."""
-    if w.Hq == 4 * w.Hkv:
-        return "decode_gqa_kernel"
-    if w.Hq == w.Hkv and w.G >= 32:
-        return "decode_mha_kernel"
-    return "decode_split_kernel"
+    return "decode_tc_kernel" if w.Hq // w.Hkv in (1, 2, 4) and w.G >= 32 else "decode_split_kernel"
 
 
 def ncu_traffic(w):

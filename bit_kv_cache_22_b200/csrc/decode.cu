@@ -138,6 +138,53 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(PENDING));
 }
 
+// Bulk (TMA) copies global -> shared completing on an mbarrier, and the barrier
+// operations (no cluster multicast anywhere).
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_inval(uint64_t *bar) {
+    asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// barrier initialisations visible to the async proxy
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+// earlier generic-proxy accesses to shared memory ordered before later async-proxy ones
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+// bytes: a multiple of 16; both addresses 16-byte aligned
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Waits for the phase of `parity` to complete, giving up after kSpinLimit polls
+// (each poll may suspend the thread for a while); false when it gave up.
+constexpr uint32_t kSpinLimit = 1u << 22;
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kSpinLimit; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
 // Shared-memory stage of one 16-token tile, owned by one warp:
 //   [K codes][V codes], each as (W/4 chunks) x (32 lanes) x 16 bytes, chunk-major so
 //   that a warp's 16-byte loads of one chunk hit 32 consecutive 16-byte slots
@@ -658,37 +705,8 @@ __device__ __forceinline__ void residual_pass(const DecodeArgs &a, const float *
 }
 
 // ---------------------------------------------------------------------------
-// Grouped-query heads (4 query heads per kv head): tensor-core path.
-//
-// A CTA owns one (batch, kv head, split) and serves the 4 query heads that read
-// that kv head, so every code is fetched and unpacked once for all of them.
-// Lane = 4*g8 + t4; query head t4 is "owned" by the lanes with that t4.
-//   keys   : int8 MMA m16n8k32.  A = the byte-masked key codes (rows = tokens,
-//            k = channels) exactly as stored; B = byte digits of the 21-bit
-//            fixed-point multipliers q_c s_{g,c} log2(e)/sqrt(d) (exponent per
-//            key group and head), columns 2h+d (digits 0, 1 of head h) in the
-//            first n-tile and 2h (signed digit 2) in the second; int32 sums,
-//            exact.  The digits are built once per key group, cooperatively by
-//            the warp (lane l: head l/8, 16 channels), in shared memory.
-//   values : bf16 MMA m16n8k16.  A = value codes as exact bf16 (rows = channels,
-//            k = tokens; bytes 0,2 and 1,3 of a word slot are bf16x2 pairs via
-//            the 0x4300 exponent trick); B = p_t s_{t,gv} split into bf16 hi +
-//            lo parts (columns 2h, 2h+1; bf16 keeps fp32's exponent range, so
-//            the tiny probabilities of long contexts do not underflow), built
-//            cooperatively per tile; fp32 accumulators, rescaled when a head's
-//            running maximum grows.
-//   z-terms: bias_g = sum_c q'_c z_{g,c} and sum_t p_t s_t z_t in fp32.
-// Residual rows form the last split, where each warp serves one query head
-// with exact e values on CUDA cores.
+// Tensor-core helpers (mma.sync).
 // ---------------------------------------------------------------------------
-constexpr int kGqa = 4;
-
-__device__ __forceinline__ void imma_uu(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
 __device__ __forceinline__ void imma_us(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
@@ -715,44 +733,6 @@ __device__ __forceinline__ uint32_t f2bf2(float lo, float hi) {
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
     return d;
 }
-
-// Codes of one slot of a value word as two bf16x2 registers, (byte 0, byte 2)
-// and (byte 1, byte 3), each element equal to 2^(7-N) * (2^N + code) exactly:
-// the code is shifted to the top N mantissa bits of 0x4300 (bf16 128, unit
-// mantissa steps).  The 2^N offset is small next to the code range, so it is
-// kept: the value MMA accumulates sum_t b_t (2^N + code) and the z-term uses
-// z + 2^N instead of z; the 2^(7-N) factor is folded into the B operand.
-template <int N>
-__device__ __forceinline__ void codes_bf16(uint32_t w, int slot, uint32_t magic16, uint32_t &r02,
-                                           uint32_t &r13) {
-    constexpr uint32_t L = (1u << N) - 1u;
-    constexpr uint32_t M = (L << (7 - N)) | (L << (23 - N));
-    const int up = 7 - N - N * slot;                  // byte 0/2 code: bit N*slot -> 7 - N
-    const uint32_t x02 = up >= 0 ? (w << up) : (w >> -up);
-    const uint32_t x13 = w >> (N * slot + N + 1);     // byte 1/3 code: bit 8 + N*slot -> 7 - N
-    r02 = and_or(x02, M, magic16);
-    r13 = and_or(x13, M, magic16);
-}
-
-// Shared-memory stages of the grouped-query kernel (it consumes two tiles per
-// iteration, so it keeps a deeper ring when a stage is small).
-template <int N>
-__host__ __device__ constexpr int gqa_stages() { return N == 2 ? 6 : 4; }
-
-template <int N, int D, int GV>
-struct GqaSmem {
-    static constexpr int NGV = D / GV;
-    static constexpr int kStageBytes = gqa_stages<N>() * Stage<N, D, GV>::kBytes;
-    static constexpr int kKdRow = D + 16;                    // padded: the 8 B-fragment rows hit distinct banks
-    static constexpr int kKd = kStageBytes;                  // key digits [3][4 heads][kKdRow] bytes
-    static constexpr int kVb = kKd + 3 * kGqa * kKdRow;      // value B [2 tiles][NGV][4][2][16] bf16
-    // p [2 tiles][2 token halves][4 heads][8] f32, tokens of a half in (0, 2, 1, 3) order
-    // within each 4-group: owners store and builders read (as pairs) without conflicts
-    static constexpr int kPs = kVb + 2 * NGV * kGqa * 2 * 16 * 2;
-    static constexpr int kAl = kPs + 2 * 2 * kGqa * 8 * 4;   // alpha [4], key scale [4], bias [4]
-    static constexpr int kWarpBytes = kAl + 16 * 4;
-    static_assert(kKd % 16 == 0 && kVb % 16 == 0 && kPs % 16 == 0 && kAl % 16 == 0, "align");
-};
 
 // One token's value scales and zeros (NGV of each) from a stage, with vector loads.
 template <int NGV>
@@ -781,419 +761,49 @@ __device__ __forceinline__ void load_meta(const float *sp, const int16_t *zp, bo
     }
 }
 
-template <int N, int D, int GV>
-__global__ void __launch_bounds__(kDecodeThreads, 3) decode_gqa_kernel(const DecodeArgs a) {
-    constexpr int W = D * N / 64;
-    constexpr int TW = D * N / 2;
-    constexpr int NJ = D / 16;
-    constexpr int NK = D / 32;        // k32 steps of the key MMA
-    constexpr int BPW = 4 / N;
-    constexpr int NGV = D / GV;
-    constexpr uint32_t BYTE_MASK = ((1u << N) - 1u) * 0x01010101u;
-    using St = Stage<N, D, GV>;
-    using Sm = GqaSmem<N, D, GV>;
-    constexpr int kGqaStages = gqa_stages<N>();
-
-    __shared__ __align__(16) float q_s[kGqa][D];
-    __shared__ float ml_s[kDecodeWarps][kGqa][2];
-    __shared__ int last_s;
-    extern __shared__ __align__(128) unsigned char stage_mem[];
-
-    const int hk = blockIdx.x, b = blockIdx.y, sigma = blockIdx.z;
-    const int64_t bh = static_cast<int64_t>(b) * a.Hkv + hk;
-    const int64_t bq0 = static_cast<int64_t>(b) * a.Hq + hk * kGqa;   // first query head
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g8 = lane >> 2, t4 = lane & 3;
-    unsigned char *wmem = stage_mem + static_cast<size_t>(warp) * Sm::kWarpBytes;
-    uint8_t *kd = wmem + Sm::kKd;
-    uint16_t *vb = reinterpret_cast<uint16_t *>(wmem + Sm::kVb);
-    float *ps = reinterpret_cast<float *>(wmem + Sm::kPs);
-    float *al = reinterpret_cast<float *>(wmem + Sm::kAl);
-    const uint32_t magic = kMagicBits;
-    const uint32_t magic16 = 0x43004300u;    // bf16 128 in both halves
-
-    for (int i = threadIdx.x; i < kGqa * D; i += kDecodeThreads)
-        q_s[i / D][i % D] = widen(a.q[bq0 * D + i], a.bf16) * a.qscale;
-    __syncthreads();
-
-    const int total_tiles = a.n_qtiles + (a.r + 15) / 16;
-    const int zsym = 1 << (N - 1);
-
-    if (sigma >= a.n_qsplits) {
-        // ---------------- residual split: warp = query head ----------------
-        const float *qh = q_s[warp];
-        float m = -INFINITY, lsum = 0.f;
-        float2 acc[NJ][2];
-#pragma unroll
-        for (int j = 0; j < NJ; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
-        residual_pass<D>(a, qh, a.kr + bh * a.R * D, a.vr + bh * a.R * D, 0, total_tiles - a.n_qtiles,
-                         lane, m, lsum, acc, wmem);
-        lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
-        lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
-        lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
-        static_assert(residual_scratch_bytes<D>() <= Sm::kWarpBytes, "residual staging");
-        __syncthreads();   // every warp is done with its staged rows before o_s overwrites them
-        float *o_s = reinterpret_cast<float *>(stage_mem);   // [warp][head][D]; only head == warp
-#pragma unroll
-        for (int j = 0; j < NJ; ++j) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float val = acc[j][h].x + acc[j][h].y;
-                val += __shfl_xor_sync(0xffffffffu, val, 1);
-                val += __shfl_xor_sync(0xffffffffu, val, 2);
-                if (t4 == 0) o_s[(warp * kGqa + warp) * D + 16 * j + g8 + 8 * h] = val;
-            }
-        }
-        if (lane < kGqa) {
-            ml_s[warp][lane][0] = lane == warp ? m : -INFINITY;
-            ml_s[warp][lane][1] = lane == warp ? lsum : 0.f;
-        }
-        __syncthreads();
-        finish_cta<kGqa, D>(a, o_s, ml_s, bh, bq0, sigma, &last_s, o_s + kDecodeWarps * kGqa * D);
-        return;
-    }
-
-    // ---------------- quantized split ----------------
-    const int t_begin = sigma * a.tiles_per_split;
-    const int t_end = min(a.n_qtiles, t_begin + a.tiles_per_split);
-    const int per_w = (t_end - t_begin + kDecodeWarps - 1) / kDecodeWarps;
-    const int wb = t_begin + warp * per_w;
-    const int we = min(t_end, wb + per_w);
-    const int64_t groups_cap = a.cap / a.G;
-    const uint32_t *kc = a.kc + bh * (a.cap / 16) * TW;
-    const uint32_t *vc = a.vc + bh * (a.cap / 16) * TW;
-    const float *vs_g = a.vs + bh * a.cap * NGV;
-    const int16_t *vz_g = a.vz + bh * a.cap * NGV;
-    const int gmask = (1 << a.gshift) - 1;
-
-    auto issue = [&](int ti) {
-        if (ti >= we) return;
-        unsigned char *st = wmem + ((ti - wb) % kGqaStages) * St::kBytes;
-        const uint32_t *ksrc = kc + static_cast<int64_t>(ti) * TW + lane * W;
-        const uint32_t *vsrc = vc + static_cast<int64_t>(ti) * TW + lane * W;
-        if constexpr (W % 4 == 0) {
-            uint32_t *kdst = reinterpret_cast<uint32_t *>(st) + 4 * lane;
-            uint32_t *vdst = reinterpret_cast<uint32_t *>(st + St::kCodes) + 4 * lane;
-#pragma unroll
-            for (int i = 0; i < W / 4; ++i) {
-                cp_async16(kdst + 128 * i, ksrc + 4 * i);
-                cp_async16(vdst + 128 * i, vsrc + 4 * i);
-            }
-        } else {
-            static_assert(W == 2, "lane segment of 8 bytes");
-            cp_async8(reinterpret_cast<uint32_t *>(st) + lane * W, ksrc);
-            cp_async8(reinterpret_cast<uint32_t *>(st + St::kCodes) + lane * W, vsrc);
-        }
-        const int64_t tok0 = static_cast<int64_t>(ti) * 16;
-        for (int c = lane; c < NGV * 4; c += 32)
-            cp_async16(st + St::kVs + 16 * c, vs_g + tok0 * NGV + 4 * c);
-        if (!a.sym)
-            for (int c = lane; c < NGV * 2; c += 32)
-                cp_async16(st + St::kVz + 16 * c, vz_g + tok0 * NGV + 8 * c);
-        if (ti == wb || (ti & gmask) == 0) {
-            const int64_t gofs = (bh * groups_cap + (ti >> a.gshift)) * D;
-            for (int c = lane; c < D / 4; c += 32) cp_async16(st + St::kKs + 16 * c, a.ks + gofs + 4 * c);
-            if (!a.sym)
-                for (int c = lane; c < D / 8; c += 32) cp_async16(st + St::kKz + 16 * c, a.kz + gofs + 8 * c);
-        }
-    };
-
-    // owner state (query head t4)
-    float m = -INFINITY, lsum = 0.f;
-    float dv[NJ][4];                  // value accumulators: channel 16j + g8 (+8), head t4 hi / lo
-#pragma unroll
-    for (int j = 0; j < NJ; ++j) dv[j][0] = dv[j][1] = dv[j][2] = dv[j][3] = 0.f;
-    float kinv = 0.f, kbias = 0.f;
-    // builder state (head hb = lane / 8)
-    const int hb = lane >> 3, lb = lane & 7;
-    float zsum[NGV];
-#pragma unroll
-    for (int v = 0; v < NGV; ++v) zsum[v] = 0.f;
-    // B operands of the key MMA for the current group
-    uint32_t kb0[NK][2], kb1[NK][2];
-
-    // Key digits of the group tile `st` opens: lane builds head hb, channels
-    // 4*lb + 32*i4 + {0..3}, i4 < D/32 (a quarter-warp reads 128 contiguous bytes).
-    auto rebuild_key_digits = [&](const unsigned char *st) {
-        const float *ks_s = reinterpret_cast<const float *>(st + St::kKs);
-        const int16_t *kz_s = reinterpret_cast<const int16_t *>(st + St::kKz);
-        constexpr int NQ = D / 32;
-        float qv[4 * NQ];
-        float mx = 0.f, kbp = 0.f;
-#pragma unroll
-        for (int i4 = 0; i4 < NQ; ++i4) {
-            const int c0 = 4 * lb + 32 * i4;
-            const float4 sc = *reinterpret_cast<const float4 *>(ks_s + c0);
-            const float4 qq = *reinterpret_cast<const float4 *>(&q_s[hb][c0]);
-            qv[4 * i4 + 0] = qq.x * sc.x; qv[4 * i4 + 1] = qq.y * sc.y;
-            qv[4 * i4 + 2] = qq.z * sc.z; qv[4 * i4 + 3] = qq.w * sc.w;
-            float z[4] = {static_cast<float>(zsym), static_cast<float>(zsym),
-                          static_cast<float>(zsym), static_cast<float>(zsym)};
-            if (!a.sym) {
-                const uint2 zz = *reinterpret_cast<const uint2 *>(kz_s + c0);
-                z[0] = __int2float_rn(static_cast<int16_t>(zz.x & 0xffffu));
-                z[1] = __int2float_rn(static_cast<int16_t>(zz.x >> 16));
-                z[2] = __int2float_rn(static_cast<int16_t>(zz.y & 0xffffu));
-                z[3] = __int2float_rn(static_cast<int16_t>(zz.y >> 16));
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                kbp = fmaf(qv[4 * i4 + i], z[i], kbp);
-                mx = fmaxf(mx, fabsf(qv[4 * i4 + i]));
-            }
-        }
-#pragma unroll
-        for (int o = 1; o < 8; o <<= 1) {
-            kbp += __shfl_xor_sync(0xffffffffu, kbp, o);
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        }
-        int e = 0;
-        if (mx > 0.f) e = 21 - (static_cast<int>((__float_as_uint(mx) >> 23) & 0xff) - 126);
-        e = max(-120, min(120, e));
-        const float scale = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
-        uint32_t dw[3][NQ];
-#pragma unroll
-        for (int i4 = 0; i4 < NQ; ++i4) {
-            const int Q0 = round_small(qv[4 * i4 + 0] * scale), Q1 = round_small(qv[4 * i4 + 1] * scale);
-            const int Q2 = round_small(qv[4 * i4 + 2] * scale), Q3 = round_small(qv[4 * i4 + 3] * scale);
-#pragma unroll
-            for (int k = 0; k < 3; ++k) {
-                const uint32_t sel = static_cast<uint32_t>(k | ((k + 4) << 4));
-                dw[k][i4] = __byte_perm(__byte_perm(Q0, Q1, sel), __byte_perm(Q2, Q3, sel), 0x5410);
-            }
-        }
-        __syncwarp();   // the previous group's digits have been read into registers
-#pragma unroll
-        for (int k = 0; k < 3; ++k)
-#pragma unroll
-            for (int i4 = 0; i4 < NQ; ++i4)
-                reinterpret_cast<uint32_t *>(kd + (k * kGqa + hb) * Sm::kKdRow)[lb + 8 * i4] = dw[k][i4];
-        if (lb == 0) {
-            al[4 + hb] = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
-            al[8 + hb] = kbp;
-        }
-        __syncwarp();
-        // B fragments: column g8 = head g8/2, digit g8%2 (first n-tile), digit 2 for even g8
-        const uint32_t *kdw0 =
-            reinterpret_cast<const uint32_t *>(kd + ((g8 & 1) * kGqa + (g8 >> 1)) * Sm::kKdRow);
-        const uint32_t *kdw2 = reinterpret_cast<const uint32_t *>(kd + (2 * kGqa + (g8 >> 1)) * Sm::kKdRow);
-#pragma unroll
-        for (int mk = 0; mk < NK; ++mk) {
-            kb0[mk][0] = kdw0[8 * mk + t4];
-            kb0[mk][1] = kdw0[8 * mk + 4 + t4];
-            kb1[mk][0] = (g8 & 1) ? 0u : kdw2[8 * mk + t4];
-            kb1[mk][1] = (g8 & 1) ? 0u : kdw2[8 * mk + 4 + t4];
-        }
-        kinv = al[4 + t4];
-        kbias = al[8 + t4];
-    };
-
-#pragma unroll
-    for (int s = 0; s < kGqaStages - 2; ++s) {
-        issue(wb + s);
-        cp_async_commit();
-    }
-
-    // two tiles per iteration: their key MMAs, one softmax update and their value MMAs
-    // are independent streams of work for the scheduler
-    for (int ti = wb; ti < we; ti += 2) {
-        const int nt = min(2, we - ti);
-        issue(ti + kGqaStages - 2);
-        cp_async_commit();
-        issue(ti + kGqaStages - 1);
-        cp_async_commit();
-        cp_async_wait<kGqaStages - 2>();
-        __syncwarp();
-
-        // ---- key MMAs: logits of tokens g8, g8 + 8 of both tiles, query head t4 ----
-        float lg[2][2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            lg[u][0] = lg[u][1] = -INFINITY;
-            if (u < nt) {
-                const int t = ti + u;
-                const unsigned char *st = wmem + ((t - wb) % kGqaStages) * St::kBytes;
-                if (t == wb || (t & gmask) == 0) rebuild_key_digits(st);
-                uint32_t kw[W];
-                load_stage_words<W>(reinterpret_cast<const uint32_t *>(st), lane, kw);
-                int d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0};
-#pragma unroll
-                for (int mk = 0; mk < NK; ++mk) {
-                    uint32_t af[4];
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        const int j = 2 * mk + (r >> 1), half = r & 1;
-                        af[r] = (kw[j / BPW] >> (N * (2 * (j % BPW) + half))) & BYTE_MASK;
-                    }
-                    imma_uu(d0, af, kb0[mk][0], kb0[mk][1]);
-                    imma_us(d1, af, kb1[mk][0], kb1[mk][1]);
-                }
-                lg[u][0] = (small_int_to_float(d0[0]) + 256.f * small_int_to_float(d0[1]) +
-                            65536.f * small_int_to_float(d1[0])) * kinv - kbias;
-                lg[u][1] = (small_int_to_float(d0[2]) + 256.f * small_int_to_float(d0[3]) +
-                            65536.f * small_int_to_float(d1[2])) * kinv - kbias;
-            }
-        }
-
-        // ---- online softmax of head t4 over both tiles ----
-        float tmax = fmaxf(fmaxf(lg[0][0], lg[0][1]), fmaxf(lg[1][0], lg[1][1]));
-        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
-        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
-        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
-        const bool grew = tmax > m;
-        if (__any_sync(0xffffffffu, grew)) {
-            const float alpha = grew ? fast_exp2(m - tmax) : 1.f;
-            if (grew) m = tmax;
-            lsum *= alpha;
-#pragma unroll
-            for (int j = 0; j < NJ; ++j) {
-                dv[j][0] *= alpha; dv[j][1] *= alpha; dv[j][2] *= alpha; dv[j][3] *= alpha;
-            }
-            if (g8 == 0) al[t4] = alpha;
-            __syncwarp();
-            const float ab = al[lane & 3];     // zsum belongs to head lane % 4
-#pragma unroll
-            for (int v = 0; v < NGV; ++v) zsum[v] *= ab;
-        }
-        // position of token g8 (and g8 + 8) inside its half: 4-groups in (0, 2, 1, 3) order
-        const int ppos = (g8 & 4) + ((g8 & 1) << 1) + ((g8 >> 1) & 1);
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const float p0 = fast_exp2(lg[u][0] - m), p1 = fast_exp2(lg[u][1] - m);
-            lsum += p0 + p1;
-            ps[((u * 2 + 0) * kGqa + t4) * 8 + ppos] = p0;
-            ps[((u * 2 + 1) * kGqa + t4) * 8 + ppos] = p1;
-        }
-        __syncwarp();
-
-        // ---- value B of both tiles: lane l builds head l % 4 for tokens 4q + e and
-        //      4q + e + 2, (q, e) = (l / 8, (l / 4) % 2): a quarter-warp covers one token pair
-        //      of all four heads (broadcast meta reads, distinct p rows and plane words) ----
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            if (u < nt) {
-                const unsigned char *st = wmem + ((ti + u - wb) % kGqaStages) * St::kBytes;
-                constexpr float kBscale = 1.0f / static_cast<float>(1 << (7 - N));
-                constexpr int kOff = 1 << N;          // code offset carried by the bf16 A operand
-                const int hv = lane & 3, q4 = lane >> 3, e = (lane >> 2) & 1;
-                const int ta = 4 * q4 + e, tb = ta + 2;
-                // tokens ta, tb sit side by side: half q4/2, position 4*(q4%2) + 2e (+1)
-                const float2 pr = *reinterpret_cast<const float2 *>(
-                    ps + ((u * 2 + (q4 >> 1)) * kGqa + hv) * 8 + 4 * (q4 & 1) + 2 * e);
-                const float2 pab = make_float2(pr.x * kBscale, pr.y * kBscale);
-                const float *vsp = reinterpret_cast<const float *>(st + St::kVs);
-                const int16_t *vzp = reinterpret_cast<const int16_t *>(st + St::kVz);
-                float sa[NGV], sb[NGV];
-                int16_t zza[NGV], zzb[NGV];
-                load_meta<NGV>(vsp + ta * NGV, vzp + ta * NGV, a.sym, zsym, sa, zza);
-                load_meta<NGV>(vsp + tb * NGV, vzp + tb * NGV, a.sym, zsym, sb, zzb);
-#pragma unroll
-                for (int v = 0; v < NGV; ++v) {
-                    const float2 x = mul2(pab, make_float2(sa[v], sb[v]));
-                    const float2 z = make_float2(__int2float_rn(zza[v] + kOff), __int2float_rn(zzb[v] + kOff));
-                    zsum[v] = fmaf(x.x, z.x, fmaf(x.y, z.y, zsum[v]));
-                    const uint32_t hi = f2bf2(x.x, x.y);
-                    const float2 lof = add2(x, make_float2(-__uint_as_float(hi << 16),
-                                                           -__uint_as_float(hi & 0xffff0000u)));
-                    const uint32_t lo = f2bf2(lof.x, lof.y);
-                    // planes (part p of head h) at sub-block p ^ (h >> 1): conflict-free stores and loads
-                    uint32_t *dst = reinterpret_cast<uint32_t *>(vb + (((u * NGV + v) * kGqa + hv) * 2) * 16);
-                    dst[((hv >> 1) << 3) + ((4 * q4 + 2 * e) >> 1)] = hi;          // part 0 plane
-                    dst[((1 ^ (hv >> 1)) << 3) + ((4 * q4 + 2 * e) >> 1)] = lo;    // part 1 plane
-                }
-            }
-        }
-        __syncwarp();
-
-        // ---- value MMAs: rows = channels of chunk j, k = a tile's tokens ----
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            if (u < nt) {
-                const unsigned char *st = wmem + ((ti + u - wb) % kGqaStages) * St::kBytes;
-                uint32_t vw[W];
-                load_stage_words<W>(reinterpret_cast<const uint32_t *>(st + St::kCodes), lane, vw);
-#pragma unroll
-                for (int j = 0; j < NJ; ++j) {
-                    uint32_t a02, a13, b02, b13;
-                    codes_bf16<N>(vw[j / BPW], 2 * (j % BPW), magic16, a02, a13);       // channel 16j + g8
-                    codes_bf16<N>(vw[j / BPW], 2 * (j % BPW) + 1, magic16, b02, b13);   // channel 16j + g8 + 8
-                    const uint2 bb = *reinterpret_cast<const uint2 *>(
-                        vb + ((((u * NGV + (16 * j) / GV) * kGqa + (g8 >> 1)) * 2 + ((g8 & 1) ^ (g8 >> 2))) * 16) +
-                        4 * t4);
-                    hmma(dv[j], a02, b02, a13, b13, bb.x, bb.y);
-                }
-            }
-        }
-        __syncwarp();
-    }
-    cp_async_wait<0>();
-    (void)magic;
-
-    // ---- epilogue: reduce per head, subtract the z-terms, merge warps ----
-    lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
-    lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
-    lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
-#pragma unroll
-    for (int v = 0; v < NGV; ++v) {      // lanes with the same lane % 4 hold one head's partials
-        zsum[v] += __shfl_xor_sync(0xffffffffu, zsum[v], 4);
-        zsum[v] += __shfl_xor_sync(0xffffffffu, zsum[v], 8);
-        zsum[v] += __shfl_xor_sync(0xffffffffu, zsum[v], 16);
-    }
-    __syncthreads();   // stage memory is reused for the per-warp outputs below
-    float *o_s = reinterpret_cast<float *>(stage_mem);   // [warp][head][D]
-    float *zs_s = o_s + kDecodeWarps * kGqa * D;          // [warp][head][NGV]
-    if (lane < kGqa)
-        for (int v = 0; v < NGV; ++v) zs_s[(warp * kGqa + lane) * NGV + v] = zsum[v];
-    // dv sums A * B = (2^N + code) p s; zsum sums b (2^N + z) with b = p s 2^-(7-N)
-    __syncwarp();
-#pragma unroll
-    for (int j = 0; j < NJ; ++j) {
-        const float z = zs_s[(warp * kGqa + t4) * NGV + (16 * j) / GV];
-        constexpr float kUnscale = static_cast<float>(1 << (7 - N));
-        o_s[(warp * kGqa + t4) * D + 16 * j + g8] = dv[j][0] + dv[j][1] - z * kUnscale;
-        o_s[(warp * kGqa + t4) * D + 16 * j + g8 + 8] = dv[j][2] + dv[j][3] - z * kUnscale;
-    }
-    if (g8 == 0) {
-        ml_s[warp][t4][0] = m;
-        ml_s[warp][t4][1] = lsum;
-    }
-    __syncthreads();
-    finish_cta<kGqa, D>(a, o_s, ml_s, bh, bq0, sigma, &last_s, o_s + kDecodeWarps * kGqa * D);
-}
-
 // ---------------------------------------------------------------------------
-// One query head per kv head: tensor-core path.
+// Tensor-core decode for HG = 1, 2 or 4 query heads per kv head.
 //
-// A CTA owns one (batch, head, split); each warp takes an even-aligned,
-// contiguous share of the split's tiles and walks it in chunks of kMhaChunk
-// tiles: first the keys of the chunk (logits to shared memory, a running
-// maximum per lane), then, with the chunk's maximum fixed, its values.  So the
-// probabilities need no per-tile cross-lane maximum, key and value work form
-// two streams without dependences between tiles, and the accumulators are
-// rescaled at most once per chunk.  Items -- a key tile pair or a value tile
-// pair -- stream through a per-warp ring of cp.async stages; a key pair never
-// straddles a key group (groups of >= 32 tokens).
+// A CTA owns one (batch, kv head, split) and serves the HG query heads that
+// read that kv head, so every code is fetched and unpacked once for all of
+// them.  Each warp takes an even-aligned, contiguous share of the split's tiles
+// and walks it in chunks of tc_chunk<HG>() tiles: first the chunk's keys (the
+// logits of its HG heads go to shared memory, each lane keeps a running
+// maximum), then, with the chunk's maxima fixed, its values.  So probabilities
+// need no per-tile cross-lane maximum, key and value work form two streams
+// without dependences between tiles, and accumulators are rescaled at most once
+// per chunk.  Items -- a key tile pair or a value tile pair -- stream through a
+// per-warp ring of cp.async stages.  Lane = 4*g8 + t4.
 //   keys   : int8 MMA m16n8k32, rows = tokens, k = channels.  A is a stored
 //            word masked to one byte slot, without a shift: slot s arrives as
-//            code * 2^(N*s).  The two 16-channel chunks of one MMA are taken
-//            from the same slot class (same 2^(N*s) for its first 8 rows, the
-//            next slot for the other 8), so the factor is constant per row of
-//            the product and is divided out of the row sum exactly.  B holds
-//            the balanced base-256 digits (each in [-128, 127]) of the 22-bit
-//            fixed-point multipliers Q_c = round(2^e q_c s_{g,c} log2(e)/sqrt(d)),
-//            built once per key group: columns 0, 1 hold digits 0, 1 and column
-//            4 digit 2, so lanes t4 = 0 and t4 = 2 of a row group hold the row's
-//            three digit sums; int32 accumulation is exact (|sum| < 2^22).
-//   values : bf16 MMA m16n8k16, rows = channels, k = tokens: A = the codes as
-//            exact bf16 2^(7-N) (2^N + code) (codes_bf16), B = p_t s_t 2^-(7-N)
-//            split into a bf16 hi part (column 0) and lo part (column 1).
-//   z-terms: bias_g = sum_c q'_c z_{g,c} and sum_t p_t s_t (z_t + 2^N) in fp32.
-// The residual rows get no split of their own: their 16-row tiles are dealt
-// round-robin to the warps of all splits, which run them on CUDA cores (staged
-// in their stage memory) before streaming and start their softmax state there.
+//            code * 2^(N*s); the two 16-channel chunks of one MMA come from the
+//            same slot class, so the factor is constant per row of the product
+//            and divided out exactly.  B holds the balanced base-256 digits
+//            (each in [-128, 127]) of the 22-bit fixed-point multipliers
+//            Q_c = round(2^e q_c s_{g,c} log2(e)/sqrt(d)) of each head (e per
+//            head and key group), built once per key group.  Head h's digits 0
+//            and 1 sit in columns 2h, 2h+1, digit 2 in column 4 + 2h (HG <= 2)
+//            or in column 2h of a second n-tile (HG = 4); int32 sums are exact.
+//   values : bf16 MMA m16n8k16, rows = channels, k = tokens.  A is a stored
+//            word masked to one byte slot (bytes 0, 2 of the word, or 1, 3 after
+//            a shift by 8).  A bf16 pattern whose bits 8..15 are zero is exactly
+//            (bits 0..7) * 2^-133: subnormal, or with bit 7 set the lowest
+//            normal binade, and the two join linearly.  So A = code * 2^(N*s) *
+//            2^-133 with no conversion.  B = p_t s_t 2^96 split into a bf16 hi
+//            part (even columns) and lo part (odd columns) of head (g8/2) mod
+//            HG; products ~ p s code 2^-37 stay well inside fp32's normal range
+//            for value scales in [2^-40, 2^31].
+//   z-terms: bias_{g,h} = sum_c q'_c z_{g,c} and sum_t p_t s_t z_t in fp32.
+// Residual rows: with HG = 1 their tiles are dealt round-robin to the warps of
+// all splits, which run them first on CUDA cores (staged in shared memory) and
+// start their softmax state from them; with HG > 1 they form one more split.
 // ---------------------------------------------------------------------------
-constexpr int kMhaChunk = 32;     // tiles per key phase / value phase of a warp
-constexpr int kMhaStages = 4;
+constexpr int kTcStages = 4;
+constexpr int kVScaleLog2 = 96;   // the value MMA's B operand is p s 2^96
+
+// Tiles per key phase / value phase of a warp (the logits of a chunk take 2 KB).
+template <int HG>
+__host__ __device__ constexpr int tc_chunk() { return 32 / HG; }
 
 // cp.async of one tile's code array -- lane-major in global memory, lane l's W
 // words at l*W -- into the chunk-major stage layout (16-byte piece p of lane l
@@ -1214,27 +824,51 @@ __device__ __forceinline__ void copy_tile_codes(unsigned char *dst, const uint32
     }
 }
 
+// The lane's W words of one tile's code array as stored (lane-major: lane l's words at l*W).
+template <int W>
+__device__ __forceinline__ void load_lane_words(const unsigned char *base, int lane, uint32_t (&w)[W]) {
+    if constexpr (W % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < W / 4; ++i) {
+            const uint4 v = reinterpret_cast<const uint4 *>(base)[lane * (W / 4) + i];
+            w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+        }
+    } else {
+        static_assert(W == 2, "lane segment of 8 bytes");
+        const uint2 v = reinterpret_cast<const uint2 *>(base)[lane];
+        w[0] = v.x; w[1] = v.y;
+    }
+}
+
 template <int N, int D, int GV>
-struct MhaStage {                 // one item: two tiles of one code array and their meta
+struct TcStage {                  // one item: two tiles of one code array and their meta
     static constexpr int W = D * N / 64;
     static constexpr int NGV = D / GV;
-    static constexpr int kCodes = 32 * W * 4;            // one tile's code array (chunk-major)
-    static constexpr int kMeta = 2 * kCodes;              // key item: scales [D] f32; value item: [32][NGV] f32
-    static constexpr int kKz = kMeta + D * 4;             // key zeros [D] i16
-    static constexpr int kVz = kMeta + 32 * NGV * 4;      // value zeros [32][NGV] i16
+    static constexpr int kCodes = 32 * W * 4;            // one tile's code array, as stored (lane-major)
+    static constexpr int kMeta = 2 * kCodes;
+    // key item: the scales [D] f32 (at kMeta) and zeros [D] i16 (at kKz) of the key group its
+    // first tile opens (groups of >= 32 tokens: an even-aligned tile pair opens at most one)
+    static constexpr int kKz = kMeta + D * 4;
+    // value item: scales [32][NGV] f32 at kMeta, zeros [32][NGV] i16 at kVz
+    static constexpr int kVz = kMeta + 32 * NGV * 4;
     static constexpr int kEnd = (kKz + D * 2 > kVz + 32 * NGV * 2) ? kKz + D * 2 : kVz + 32 * NGV * 2;
     static constexpr int kBytes = (kEnd + 15) / 16 * 16;
     static_assert(kMeta % 16 == 0 && kKz % 16 == 0 && kVz % 16 == 0, "align");
 };
 
-template <int N, int D, int GV>
-struct MhaSmem {
+template <int N, int D, int GV, int HG>
+struct TcSmem {
     static constexpr int kKdWords = D / 4 + 4;   // one digit row (4 channels a word), padded by 4 banks
-    static constexpr int kLg = kMhaStages * MhaStage<N, D, GV>::kBytes;   // logits [kMhaChunk][16] f32
-    static constexpr int kKd = kLg + kMhaChunk * 16 * 4;
-    static constexpr int kWarpBytes = kKd + 3 * kKdWords * 4;
-    static_assert(kLg % 16 == 0 && kWarpBytes % 16 == 0, "align");
+    static constexpr int kLg = kTcStages * TcStage<N, D, GV>::kBytes;          // logits [chunk][HG][16] f32
+    static constexpr int kKd = kLg + tc_chunk<HG>() * HG * 16 * 4;             // digits [HG][3][kKdWords]
+    static constexpr int kBars = kKd + HG * 3 * kKdWords * 4;                 // stage barriers [kTcStages]
+    static constexpr int kWarpBytes = (kBars + kTcStages * 8 + 15) / 16 * 16;
+    static_assert(kLg % 16 == 0 && kBars % 16 == 0, "align");
 };
+
+// Position of token t (0..15) of a tile in the logits buffer: tokens 4q + e and 4q + e + 2
+// sit side by side, the pair one lane of the value-B build needs.
+__device__ __forceinline__ int logit_pos(int t) { return 4 * (t >> 2) + 2 * (t & 1) + ((t >> 1) & 1); }
 
 // Value scales and zeros of the four tokens 4*t4 + i of a lane (NGV of each).
 template <int NGV>
@@ -1262,399 +896,533 @@ __device__ __forceinline__ void load_meta4(const float *sp, const int16_t *zp, b
     }
 }
 
-template <int N, int D, int GV>
-__global__ void __launch_bounds__(kDecodeThreads, (D / GV >= 4) ? 3 : 4) decode_mha_kernel(const DecodeArgs a) {
+template <int D, int GV, int HG>
+__host__ __device__ constexpr int tc_min_ctas() { return (HG == 4 || D / GV >= 4) ? 3 : 4; }
+
+template <int N, int D, int GV, int HG>
+__global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) decode_tc_kernel(const DecodeArgs a) {
     constexpr int W = D * N / 64;
     constexpr int TW = D * N / 2;
     constexpr int NJ = D / 16;
     constexpr int BPW = 4 / N;        // slot classes (chunks per word)
     constexpr int NP = W / 2;         // word pairs; the key MMAs of a tile are (pair, class)
     constexpr int NGV = D / GV;
+    constexpr int NTK = HG == 4 ? 2 : 1;                  // n-tiles of the key MMA
+    constexpr int LPH = 32 / HG;                          // lanes per head when building digits
+    constexpr int QPL = (D / 4 + LPH - 1) / LPH;          // channel quads per lane when building digits
+    constexpr int kChunk = tc_chunk<HG>();
     constexpr uint32_t BYTE_L = ((1u << N) - 1u) * 0x01010101u;
-    constexpr int kSt = kMhaStages;
-    using St = MhaStage<N, D, GV>;
-    using Sm = MhaSmem<N, D, GV>;
+    constexpr uint32_t HALF_L = ((1u << N) - 1u) * 0x00010001u;
+    constexpr int kSt = kTcStages;
+    using St = TcStage<N, D, GV>;
+    using Sm = TcSmem<N, D, GV, HG>;
+    static_assert(HG == 1 || HG == 2 || HG == 4, "heads per kv head");
     static_assert(W % 2 == 0, "key MMAs take words in pairs");
-    static_assert(kMhaChunk % 2 == 0 && (kMhaChunk & (kMhaChunk - 1)) == 0, "chunk");
+    static_assert(kChunk % 2 == 0 && (kChunk & (kChunk - 1)) == 0, "chunk");
+    static_assert(residual_scratch_bytes<D>() <= Sm::kBars, "residual staging");
+    static_assert(kDecodeWarps * HG * D * 4 + HG * 66 * 4 <= (kDecodeWarps - 1) * Sm::kWarpBytes + Sm::kBars,
+                  "epilogue");
 
-    __shared__ __align__(16) float q_s[D];
-    __shared__ float ml_s[kDecodeWarps][1][2];
+    __shared__ __align__(16) float q_s[HG][D];
+    __shared__ float ml_s[kDecodeWarps][HG][2];
     __shared__ int last_s;
     extern __shared__ __align__(128) unsigned char stage_mem[];
 
-    const int qi = blockIdx.x, b = blockIdx.y, sigma = blockIdx.z;
-    const int64_t bh = static_cast<int64_t>(b) * a.Hkv + qi;
-    const int64_t bq = static_cast<int64_t>(b) * a.Hq + qi;
+    const int hk = blockIdx.x, b = blockIdx.y, sigma = blockIdx.z;
+    const int64_t bh = static_cast<int64_t>(b) * a.Hkv + hk;
+    const int64_t bq0 = static_cast<int64_t>(b) * a.Hq + static_cast<int64_t>(hk) * HG;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g8 = lane >> 2, t4 = lane & 3;
+    const int hown = t4 & (HG - 1);            // head of this lane's logits and value columns
+    const int hb = (g8 >> 1) & (HG - 1);       // head of this lane's value-B column
     unsigned char *wmem = stage_mem + static_cast<size_t>(warp) * Sm::kWarpBytes;
     float *lgs = reinterpret_cast<float *>(wmem + Sm::kLg);
     uint32_t *kd = reinterpret_cast<uint32_t *>(wmem + Sm::kKd);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(wmem + Sm::kBars);
     const int zsym = 1 << (N - 1);
 
-    for (int c = threadIdx.x; c < D; c += kDecodeThreads)
-        q_s[c] = widen(a.q[bq * D + c], a.bf16) * a.qscale;
+    for (int i = threadIdx.x; i < HG * D; i += kDecodeThreads)
+        q_s[i / D][i % D] = widen(a.q[bq0 * D + i], a.bf16) * a.qscale;
     __syncthreads();
 
-    float m = -INFINITY, lsum = 0.f;
-    float ov[NJ][2];   // channels 16j + g8 (+8), final in lanes t4 == 0
+    float *o_s = reinterpret_cast<float *>(stage_mem);   // epilogue: [warp][HG][D]
 
-    {
-        // ---------------- quantized split ----------------
-        const int t_begin = sigma * a.tiles_per_split;                 // even
-        const int t_end = min(a.n_qtiles, t_begin + a.tiles_per_split);
-        const int per_w = 2 * ((t_end - t_begin + 2 * kDecodeWarps - 1) / (2 * kDecodeWarps));
-        const int wb = min(t_end, t_begin + warp * per_w);             // even
-        const int ntiles = min(t_end, wb + per_w) - wb;
-        const int nitems = 2 * ((ntiles + 1) / 2);   // one key item and one value item per tile pair
-        const int64_t groups_cap = a.cap / a.G;
-        const int64_t tile0 = bh * (a.cap / 16) + wb;
-        const uint32_t *kp = a.kc + tile0 * TW;
-        const uint32_t *vp = a.vc + tile0 * TW;
-        const float *vsp = a.vs + tile0 * 16 * NGV;
-        const int16_t *vzp = a.sym ? nullptr : a.vz + tile0 * 16 * NGV;
-        const int gmask = (1 << a.gshift) - 1;
-        const int n_vs = 4 * NGV, n_meta = a.sym ? n_vs : 6 * NGV;   // 16-byte pieces per value tile
-
-        // Item cursor: chunk [cb, cb + kMhaChunk) of the warp's tiles holds np tile pairs; items
-        // 0 .. np-1 of a chunk are its key pairs, np .. 2np-1 its value pairs.
-        struct Cursor {
-            int cb, r, np;
-            __device__ void start(int ntiles) { cb = 0; r = 0; np = (min(kMhaChunk, ntiles) + 1) / 2; }
-            __device__ void next(int ntiles) {
-                if (++r == 2 * np) {
-                    cb += kMhaChunk;
-                    r = 0;
-                    np = (min(kMhaChunk, ntiles - cb) + 1) / 2;
+    if constexpr (HG > 1) {
+        if (sigma >= a.n_qsplits) {
+            // ---------------- residual split: kDecodeWarps / HG warps per head ----------------
+            constexpr int WPH = kDecodeWarps / HG;
+            const int h = warp / WPH;
+            float m = -INFINITY, lsum = 0.f;
+            float2 acc[NJ][2];
+#pragma unroll
+            for (int j = 0; j < NJ; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
+            residual_pass<D>(a, q_s[h], a.kr + bh * a.R * D, a.vr + bh * a.R * D, warp % WPH, (a.r + 15) / 16,
+                             lane, m, lsum, acc, wmem, WPH);
+            lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
+            lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
+            lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
+            __syncthreads();   // every warp is done with its staged rows before o_s overwrites them
+#pragma unroll
+            for (int j = 0; j < NJ; ++j) {
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float val = acc[j][hh].x + acc[j][hh].y;
+                    val += __shfl_xor_sync(0xffffffffu, val, 1);
+                    val += __shfl_xor_sync(0xffffffffu, val, 2);
+                    if (t4 == 0) o_s[(warp * HG + h) * D + 16 * j + g8 + 8 * hh] = val;
                 }
             }
-            __device__ bool key() const { return r < np; }
-            __device__ int rel() const { return cb + 2 * (r < np ? r : r - np); }
-        };
+            if (lane < HG) {
+                ml_s[warp][lane][0] = lane == h ? m : -INFINITY;
+                ml_s[warp][lane][1] = lane == h ? lsum : 0.f;
+            }
+            __syncthreads();
+            finish_cta<HG, D>(a, o_s, ml_s, bh, bq0, sigma, &last_s, o_s + kDecodeWarps * HG * D);
+            return;
+        }
+    }
 
-        Cursor ic;       // producer's cursor, kSt - 1 items ahead
-        ic.start(ntiles);
-        int issued = 0;
-        auto issue_next = [&]() {
-            if (issued < nitems) {
+    // ---------------- quantized split ----------------
+    const int t_begin = sigma * a.tiles_per_split;                 // even
+    const int t_end = min(a.n_qtiles, t_begin + a.tiles_per_split);
+    const int per_w = 2 * ((t_end - t_begin + 2 * kDecodeWarps - 1) / (2 * kDecodeWarps));
+    const int wb = min(t_end, t_begin + warp * per_w);             // even
+    const int ntiles = min(t_end, wb + per_w) - wb;
+    const int nitems = 2 * ((ntiles + 1) / 2);   // one key item and one value item per tile pair
+    const int64_t groups_cap = a.cap / a.G;
+    const int64_t tile0 = bh * (a.cap / 16) + wb;
+    const uint32_t *kp = a.kc + tile0 * TW;
+    const uint32_t *vp = a.vc + tile0 * TW;
+    const float *vsp = a.vs + tile0 * 16 * NGV;
+    const int16_t *vzp = a.sym ? nullptr : a.vz + tile0 * 16 * NGV;
+    const int gmask = (1 << a.gshift) - 1;
+
+    // Item cursor: chunk [cb, cb + kChunk) of the warp's tiles holds np tile pairs; items
+    // 0 .. np-1 of a chunk are its key pairs, np .. 2np-1 its value pairs.
+    struct Cursor {
+        int cb, r, np;
+        __device__ void start(int n) { cb = 0; r = 0; np = (min(kChunk, n) + 1) / 2; }
+        __device__ void next(int n) {
+            if (++r == 2 * np) {
+                cb += kChunk;
+                r = 0;
+                np = (min(kChunk, n - cb) + 1) / 2;
+            }
+        }
+        __device__ bool key() const { return r < np; }
+        __device__ int rel() const { return cb + 2 * (r < np ? r : r - np); }
+    };
+
+    // Producer: lane 0 loads item `issued` into stage issued % kSt with bulk copies that
+    // complete on the stage's barrier: the tile pair's codes (one contiguous copy), then a
+    // key item's group scales / zeros (of the group its first tile opens, if any) or a value
+    // item's scales / zeros.
+    Cursor ic;       // producer's cursor, kSt - 1 items ahead
+    ic.start(ntiles);
+    int issued = 0;
+    auto issue_next = [&]() {
+        if (issued < nitems) {
+            if (lane == 0) {
                 unsigned char *st = wmem + (issued % kSt) * St::kBytes;
+                uint64_t *bar = bars + issued % kSt;
                 const int rel = ic.rel();
-                const bool two = rel + 1 < ntiles;
+                const int nt = rel + 1 < ntiles ? 2 : 1;
+                const uint32_t cbytes = nt * St::kCodes;
+                fence_proxy_async();   // this stage's earlier reads come before the copies below
                 if (ic.key()) {
-                    const uint32_t *src = kp + static_cast<int64_t>(rel) * TW;
-                    copy_tile_codes<W>(st, src, lane);
-                    if (two) copy_tile_codes<W>(st + St::kCodes, src + TW, lane);
                     const int ti = wb + rel;
-                    if (rel == 0 || (ti & gmask) == 0) {
+                    const bool open = rel == 0 || (ti & gmask) == 0;
+                    const uint32_t sb = open ? static_cast<uint32_t>(D * 4) : 0u;
+                    const uint32_t zb = (open && !a.sym) ? static_cast<uint32_t>(D * 2) : 0u;
+                    mbar_expect_tx(bar, cbytes + sb + zb);
+                    bulk_g2s(st, kp + static_cast<int64_t>(rel) * TW, cbytes, bar);
+                    if (open) {
                         const int64_t gofs = (bh * groups_cap + (ti >> a.gshift)) * D;
-                        for (int c = lane; c < (a.sym ? D / 4 : D / 4 + D / 8); c += 32) {
-                            if (c < D / 4) cp_async16(st + St::kMeta + 16 * c, a.ks + gofs + 4 * c);
-                            else cp_async16(st + St::kKz + 16 * (c - D / 4), a.kz + gofs + 8 * (c - D / 4));
-                        }
+                        bulk_g2s(st + St::kMeta, a.ks + gofs, sb, bar);
+                        if (!a.sym) bulk_g2s(st + St::kKz, a.kz + gofs, zb, bar);
                     }
                 } else {
-                    const uint32_t *src = vp + static_cast<int64_t>(rel) * TW;
-                    copy_tile_codes<W>(st, src, lane);
-                    if (two) copy_tile_codes<W>(st + St::kCodes, src + TW, lane);
+                    const uint32_t sb = static_cast<uint32_t>(nt * 16 * NGV * 4);
+                    const uint32_t zb = a.sym ? 0u : sb / 2;
+                    mbar_expect_tx(bar, cbytes + sb + zb);
+                    bulk_g2s(st, vp + static_cast<int64_t>(rel) * TW, cbytes, bar);
                     const int64_t tok = static_cast<int64_t>(rel) * 16 * NGV;
-                    const int nvs = two ? 2 * n_vs : n_vs;
-                    for (int c = lane; c < (two ? 2 * n_meta : n_meta); c += 32) {
-                        if (c < nvs) cp_async16(st + St::kMeta + 16 * c, vsp + tok + 4 * c);
-                        else cp_async16(st + St::kVz + 16 * (c - nvs), vzp + tok + 8 * (c - nvs));
-                    }
+                    bulk_g2s(st + St::kMeta, vsp + tok, sb, bar);
+                    if (!a.sym) bulk_g2s(st + St::kVz, vzp + tok, zb, bar);
                 }
-                ic.next(ntiles);
             }
-            cp_async_commit();
-            ++issued;
-        };
+            ic.next(ntiles);
+        }
+        ++issued;
+    };
 
-        float dv[NJ][4];   // value MMA accumulators: rows = channels 16j + g8 (+8), columns 2*t4, 2*t4 + 1
+    float m_own = -INFINITY;   // running maximum of head hown (this lane's logits and value columns)
+    float mB = -INFINITY;      // running maximum of head hb (this lane's value-B column)
+    float lsum = 0.f;          // sum of p 2^96 of head hb over this lane's tokens
+    float dv[NJ][4];           // value MMA accumulators: rows = channels 16j + g8 (+8), columns 2*t4, 2*t4 + 1
 #pragma unroll
-        for (int j = 0; j < NJ; ++j) dv[j][0] = dv[j][1] = dv[j][2] = dv[j][3] = 0.f;
-        float zsum[NGV];
+    for (int j = 0; j < NJ; ++j) dv[j][0] = dv[j][1] = dv[j][2] = dv[j][3] = 0.f;
+    float zsum[NGV];           // sum of p s z 2^96 of head hb over this lane's tokens
 #pragma unroll
-        for (int v = 0; v < NGV; ++v) zsum[v] = 0.f;
-        uint32_t kb[NP * BPW][2];   // key MMA B fragments of the current group
-        float klane = 0.f, kbias = 0.f;
-        float mloc = -INFINITY;     // this lane's largest logit of the current chunk
+    for (int v = 0; v < NGV; ++v) zsum[v] = 0.f;
+    uint32_t kb[NTK][NP * BPW][2];   // key MMA B fragments of the current group
+    float klane = 0.f, kinv2 = 0.f, kbias = 0.f;
+    float mloc = -INFINITY;          // this lane's largest logit of the current chunk
 
-        // Key digits of the group the stage opens: lane l builds channels 4l .. 4l+3.
-        auto rebuild_key_digits = [&](const unsigned char *st) {
-            const int cl = lane % (D / 4);
-            const float4 sc = *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(st + St::kMeta) + 4 * cl);
-            const float4 qq = *reinterpret_cast<const float4 *>(q_s + 4 * cl);
-            const float qv[4] = {qq.x * sc.x, qq.y * sc.y, qq.z * sc.z, qq.w * sc.w};
+    // Key digits of a key group (scales [D] f32, zeros [D] i16); lane l builds head
+    // l / LPH, channel quads l % LPH + LPH * i.
+    auto rebuild_key_digits = [&](const float *ks_s, const int16_t *kz_s) {
+        const int hd = lane / LPH, li = lane % LPH;
+        float qv[QPL][4];
+        float kbp = 0.f, mx = 0.f;
+#pragma unroll
+        for (int i = 0; i < QPL; ++i) {
+            const int c4 = li + LPH * i;
+            const bool ok = c4 < D / 4;             // d = 64, HG = 1: lanes 16..31 repeat quads
+            const int cc = ok ? c4 : c4 - D / 4;
+            const float4 sc = *reinterpret_cast<const float4 *>(ks_s + 4 * cc);
+            const float4 qq = *reinterpret_cast<const float4 *>(&q_s[hd][4 * cc]);
+            qv[i][0] = qq.x * sc.x; qv[i][1] = qq.y * sc.y; qv[i][2] = qq.z * sc.z; qv[i][3] = qq.w * sc.w;
             float z[4] = {static_cast<float>(zsym), static_cast<float>(zsym), static_cast<float>(zsym),
                           static_cast<float>(zsym)};
             if (!a.sym) {
-                const uint2 zz = *reinterpret_cast<const uint2 *>(reinterpret_cast<const int16_t *>(st + St::kKz) + 4 * cl);
+                const uint2 zz = *reinterpret_cast<const uint2 *>(kz_s + 4 * cc);
                 z[0] = small_int_to_float(static_cast<int16_t>(zz.x & 0xffffu));
                 z[1] = small_int_to_float(static_cast<int16_t>(zz.x >> 16));
                 z[2] = small_int_to_float(static_cast<int16_t>(zz.y & 0xffffu));
                 z[3] = small_int_to_float(static_cast<int16_t>(zz.y >> 16));
             }
-            float kbp = 0.f, mx = 0.f;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                kbp = fmaf(qv[i], z[i], kbp);
-                mx = fmaxf(mx, fabsf(qv[i]));
+            for (int k = 0; k < 4; ++k) {
+                if (ok) kbp = fmaf(qv[i][k], z[k], kbp);
+                mx = fmaxf(mx, fabsf(qv[i][k]));
             }
-            if (lane >= D / 4) kbp = 0.f;    // d = 64: lanes 16..31 repeat channels
+        }
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                kbp += __shfl_xor_sync(0xffffffffu, kbp, o);
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            }
-            // 2^e with |q'| 2^e < 2^21, from the exponent of the largest |q'|
-            int e = 0;
-            if (mx > 0.f) e = 21 - (static_cast<int>((__float_as_uint(mx) >> 23) & 0xff) - 126);
-            e = max(-120, min(120, e));
-            const float scale = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
-            // balanced base-256 digits: Q = d0 + 256 d1 + 65536 d2 with d0, d1 in [-128, 127]
+        for (int o = 1; o < LPH; o <<= 1) {
+            kbp += __shfl_xor_sync(0xffffffffu, kbp, o);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+        // 2^e with |q'| 2^e < 2^21, from the exponent of the head's largest |q'|
+        int e = 0;
+        if (mx > 0.f) e = 21 - (static_cast<int>((__float_as_uint(mx) >> 23) & 0xff) - 126);
+        e = max(-120, min(120, e));
+        const float scale = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+        // balanced base-256 digits: Q = d0 + 256 d1 + 65536 d2 with d0, d1 in [-128, 127]
+        uint32_t dw[3][QPL];
+#pragma unroll
+        for (int i = 0; i < QPL; ++i) {
             int dg[3][4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int Q = round_small(qv[i] * scale);
+            for (int k = 0; k < 4; ++k) {
+                const int Q = round_small(qv[i][k] * scale);
                 const int Q1 = (Q + 128) >> 8;
-                dg[0][i] = Q;
-                dg[1][i] = Q1;
-                dg[2][i] = (Q1 + 128) >> 8;
+                dg[0][k] = Q;
+                dg[1][k] = Q1;
+                dg[2][k] = (Q1 + 128) >> 8;
             }
-            __syncwarp();   // the previous group's digits have been read
-            if (lane < D / 4) {
 #pragma unroll
-                for (int k = 0; k < 3; ++k)
-                    kd[k * Sm::kKdWords + cl] = __byte_perm(__byte_perm(dg[k][0], dg[k][1], 0x0040),
-                                                            __byte_perm(dg[k][2], dg[k][3], 0x0040), 0x5410);
+            for (int k = 0; k < 3; ++k)
+                dw[k][i] = __byte_perm(__byte_perm(dg[k][0], dg[k][1], 0x0040),
+                                       __byte_perm(dg[k][2], dg[k][3], 0x0040), 0x5410);
+        }
+        __syncwarp();   // the previous group's digits have been read
+#pragma unroll
+        for (int i = 0; i < QPL; ++i) {
+            const int c4 = li + LPH * i;
+            if (c4 < D / 4) {
+#pragma unroll
+                for (int k = 0; k < 3; ++k) kd[(hd * 3 + k) * Sm::kKdWords + c4] = dw[k][i];
             }
-            __syncwarp();
-            // B fragments: column g8 holds digit 0 (g8 = 0), 1 (g8 = 1) or 2 (g8 = 4)
-            const int dig = g8 == 0 ? 0 : (g8 == 1 ? 1 : 2);
-            const bool has = g8 == 0 || g8 == 1 || g8 == 4;
-            const uint32_t *row = kd + dig * Sm::kKdWords;
+        }
+        __syncwarp();
+        // B fragments: column g8 of each n-tile
+#pragma unroll
+        for (int nt = 0; nt < NTK; ++nt) {
+            int hh, dig;
+            bool has;
+            if (HG == 4) {
+                hh = g8 >> 1;
+                dig = nt == 0 ? (g8 & 1) : 2;
+                has = nt == 0 || (g8 & 1) == 0;
+            } else if (g8 < 2 * HG) {
+                hh = g8 >> 1;
+                dig = g8 & 1;
+                has = true;
+            } else {
+                hh = (g8 - 4) >> 1;
+                dig = 2;
+                has = g8 >= 4 && (g8 & 1) == 0 && hh < HG;
+            }
+            const uint32_t *row = kd + ((has ? hh : 0) * 3 + dig) * Sm::kKdWords;
 #pragma unroll
             for (int pm = 0; pm < NP; ++pm) {
 #pragma unroll
                 for (int c = 0; c < BPW; ++c) {
                     const int j1 = 2 * pm * BPW + c, j2 = j1 + BPW;
-                    kb[pm * BPW + c][0] = has ? row[4 * j1 + t4] : 0u;
-                    kb[pm * BPW + c][1] = has ? row[4 * j2 + t4] : 0u;
+                    kb[nt][pm * BPW + c][0] = has ? row[4 * j1 + t4] : 0u;
+                    kb[nt][pm * BPW + c][1] = has ? row[4 * j2 + t4] : 0u;
                 }
-            }
-            const float kinv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
-            klane = t4 == 2 ? kinv * 65536.f : kinv;
-            kbias = kbp;
-        };
-
-        // This warp's share of the residual tiles (dealt round-robin over the warps of all
-        // splits), on CUDA cores in the stage memory before the stream starts.  Its result
-        // seeds the softmax state: lane t4 = 0 holds channels 16j + g8 (+8) in both layouts,
-        // and lsum carries the B operand's 2^-(7-N).
-        static_assert(residual_scratch_bytes<D>() <= Sm::kWarpBytes, "residual staging");
-        {
-            const int nres = (a.r + 15) / 16;
-            const int gw = sigma * kDecodeWarps + warp, nw = a.S * kDecodeWarps;
-            if (gw < nres) {
-                float lr = 0.f;
-                float2 acc[NJ][2];
-#pragma unroll
-                for (int j = 0; j < NJ; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
-                residual_pass<D>(a, q_s, a.kr + bh * a.R * D, a.vr + bh * a.R * D, gw, nres, lane, m, lr,
-                                 acc, wmem, nw);
-                lr += __shfl_xor_sync(0xffffffffu, lr, 4);     // lanes hold rows g8, g8 + 8
-                lr += __shfl_xor_sync(0xffffffffu, lr, 8);
-                lr += __shfl_xor_sync(0xffffffffu, lr, 16);
-#pragma unroll
-                for (int j = 0; j < NJ; ++j) {
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        float val = acc[j][h].x + acc[j][h].y;
-                        val += __shfl_xor_sync(0xffffffffu, val, 1);
-                        val += __shfl_xor_sync(0xffffffffu, val, 2);
-                        dv[j][2 * h] = t4 == 0 ? val : 0.f;
-                    }
-                }
-                lsum = t4 == 0 ? lr / static_cast<float>(1 << (7 - N)) : 0.f;
             }
         }
+        // this lane's head (hown): its exponent and bias from the head's first building lane
+        const float kinv = __shfl_sync(0xffffffffu, __uint_as_float(static_cast<uint32_t>(127 - e) << 23),
+                                       hown * LPH);
+        kbias = __shfl_sync(0xffffffffu, kbp, hown * LPH);
+        if constexpr (HG == 4) {
+            klane = kinv;
+            kinv2 = kinv * 65536.f;
+        } else {
+            klane = t4 >= 2 ? kinv * 65536.f : kinv;   // lanes t4 = 2, 3 hold digit 2
+        }
+    };
 
+    // ---- HG = 1: this warp's share of the residual tiles (dealt round-robin over the
+    //      warps of all splits), on CUDA cores before the stream starts; its result seeds
+    //      the softmax state (lane t4 = 0 holds channels 16j + g8 (+8) in both layouts) ----
+    if constexpr (HG == 1) {
+        const int nres = (a.r + 15) / 16;
+        const int gw = sigma * kDecodeWarps + warp, nw = a.S * kDecodeWarps;
+        if (gw < nres) {
+            float lr = 0.f;
+            float2 acc[NJ][2];
 #pragma unroll
-        for (int s = 0; s < kSt - 1; ++s) issue_next();
+            for (int j = 0; j < NJ; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
+            residual_pass<D>(a, q_s[0], a.kr + bh * a.R * D, a.vr + bh * a.R * D, gw, nres, lane, m_own, lr,
+                             acc, wmem, nw);
+            lr += __shfl_xor_sync(0xffffffffu, lr, 4);     // lanes hold rows g8, g8 + 8
+            lr += __shfl_xor_sync(0xffffffffu, lr, 8);
+            lr += __shfl_xor_sync(0xffffffffu, lr, 16);
+#pragma unroll
+            for (int j = 0; j < NJ; ++j) {
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float val = acc[j][hh].x + acc[j][hh].y;
+                    val += __shfl_xor_sync(0xffffffffu, val, 1);
+                    val += __shfl_xor_sync(0xffffffffu, val, 2);
+                    const int slot = 2 * (j % BPW) + hh;   // value-MMA units: 2^(N slot - 37)
+                    dv[j][2 * hh] = t4 == 0 ? val * __uint_as_float(static_cast<uint32_t>(127 + N * slot - 37) << 23) : 0.f;
+                }
+            }
+            lsum = lane == 0 ? lr * __uint_as_float(static_cast<uint32_t>(127 + kVScaleLog2) << 23) : 0.f;
+            mB = m_own;
+        }
+    }
 
-        Cursor cc;       // consumer's cursor
-        cc.start(ntiles);
-        for (int k = 0; k < nitems; ++k) {
-            issue_next();
-            cp_async_wait<kSt - 1>();
-            __syncwarp();
-            const unsigned char *st = wmem + (k % kSt) * St::kBytes;
-            const int rel = cc.rel();
-            const int nt = rel + 1 < ntiles ? 2 : 1;
-            float *lgc = lgs + (rel % kMhaChunk) * 16;   // logits of tiles rel, rel + 1
-            if (cc.key()) {
-                if (rel == 0 || ((wb + rel) & gmask) == 0) rebuild_key_digits(st);
-                // ---- key MMAs: log2-domain logits of tokens g8 and g8 + 8 ----
+    if (lane == 0) {
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    if (u < nt) {
-                        uint32_t kw[W];
-                        load_stage_words<W>(reinterpret_cast<const uint32_t *>(st + u * St::kCodes), lane, kw);
-                        int acc[2][BPW][4];   // two chains (even / odd word pair)
+        for (int s = 0; s < kSt; ++s) mbar_init(bars + s, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
 #pragma unroll
-                        for (int pm = 0; pm < NP; ++pm) {
+    for (int s = 0; s < kSt - 1; ++s) issue_next();
+
+    Cursor cc;       // consumer's cursor
+    cc.start(ntiles);
+    int k = 0;
+    for (; k < nitems; ++k) {
+        issue_next();
+        // wait for item k; a wait that gives up (never expected) raises the device status flag
+        // and abandons the rest of this warp's items
+        const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bars + k % kSt, (k / kSt) & 1));
+        if (!ok) {
+            if (lane == 0) atomicOr(a.status, 1u);
+            break;
+        }
+        const unsigned char *st = wmem + (k % kSt) * St::kBytes;
+        const int rel = cc.rel();
+        const int nt = rel + 1 < ntiles ? 2 : 1;
+        float *lgc = lgs + (rel % kChunk) * HG * 16;   // logits of tiles rel, rel + 1: [tile][head][16]
+        if (cc.key()) {
+            // ---- key MMAs: log2-domain logits of tokens g8 and g8 + 8, head hown ----
 #pragma unroll
-                            for (int c = 0; c < BPW; ++c) {
-                                const uint32_t mlo = BYTE_L << (N * 2 * c), mhi = BYTE_L << (N * (2 * c + 1));
-                                const uint32_t af[4] = {kw[2 * pm] & mlo, kw[2 * pm] & mhi, kw[2 * pm + 1] & mlo,
-                                                        kw[2 * pm + 1] & mhi};
-                                if (pm < 2) imma_us0(acc[pm][c], af, kb[pm * BPW + c][0], kb[pm * BPW + c][1]);
-                                else imma_us(acc[pm & 1][c], af, kb[pm * BPW + c][0], kb[pm * BPW + c][1]);
+            for (int u = 0; u < 2; ++u) {
+                if (u < nt) {
+                    if (u == 0 && (rel == 0 || ((wb + rel) & gmask) == 0))
+                        rebuild_key_digits(reinterpret_cast<const float *>(st + St::kMeta),
+                                           reinterpret_cast<const int16_t *>(st + St::kKz));
+                    uint32_t kw[W];
+                    load_lane_words<W>(st + u * St::kCodes, lane, kw);
+                    int acc[NTK][2][BPW][4];   // two chains (even / odd word pair) per n-tile
+#pragma unroll
+                    for (int pm = 0; pm < NP; ++pm) {
+#pragma unroll
+                        for (int c = 0; c < BPW; ++c) {
+                            const uint32_t mlo = BYTE_L << (N * 2 * c), mhi = BYTE_L << (N * (2 * c + 1));
+                            const uint32_t af[4] = {kw[2 * pm] & mlo, kw[2 * pm] & mhi, kw[2 * pm + 1] & mlo,
+                                                    kw[2 * pm + 1] & mhi};
+#pragma unroll
+                            for (int n = 0; n < NTK; ++n) {
+                                if (pm < 2) imma_us0(acc[n][pm][c], af, kb[n][pm * BPW + c][0], kb[n][pm * BPW + c][1]);
+                                else imma_us(acc[n][pm & 1][c], af, kb[n][pm * BPW + c][0], kb[n][pm * BPW + c][1]);
                             }
                         }
-                        float x0 = 0.f, x1 = 0.f;
+                    }
+                    float x0 = 0.f, x1 = 0.f;
 #pragma unroll
-                        for (int c = 0; c < BPW; ++c) {   // digit sums d0 + 256 d1 (< 2^31), slot factor out
-                            const float f0 = 1.0f / static_cast<float>(1u << (2 * N * c));
-                            const float f1 = 1.0f / static_cast<float>(1u << (N * (2 * c + 1)));
-                            int r0 = acc[0][c][0] + acc[0][c][1] * 256, r1 = acc[0][c][2] + acc[0][c][3] * 256;
+                    for (int c = 0; c < BPW; ++c) {   // digit sums d0 + 256 d1 (< 2^31), slot factor out
+                        const float f0 = 1.0f / static_cast<float>(1u << (2 * N * c));
+                        const float f1 = 1.0f / static_cast<float>(1u << (N * (2 * c + 1)));
+                        int r0 = acc[0][0][c][0] + acc[0][0][c][1] * 256, r1 = acc[0][0][c][2] + acc[0][0][c][3] * 256;
+                        if constexpr (NP > 1) {
+                            r0 += acc[0][1][c][0] + acc[0][1][c][1] * 256;
+                            r1 += acc[0][1][c][2] + acc[0][1][c][3] * 256;
+                        }
+                        float y0 = static_cast<float>(r0) * klane, y1 = static_cast<float>(r1) * klane;
+                        if constexpr (NTK == 2) {   // digit 2 of head t4 in the second n-tile
+                            int e0 = acc[1][0][c][0], e1 = acc[1][0][c][2];
                             if constexpr (NP > 1) {
-                                r0 += acc[1][c][0] + acc[1][c][1] * 256;
-                                r1 += acc[1][c][2] + acc[1][c][3] * 256;
+                                e0 += acc[1][1][c][0];
+                                e1 += acc[1][1][c][2];
                             }
-                            x0 = fmaf(static_cast<float>(r0), f0, x0);
-                            x1 = fmaf(static_cast<float>(r1), f1, x1);
+                            y0 = fmaf(static_cast<float>(e0), kinv2, y0);
+                            y1 = fmaf(static_cast<float>(e1), kinv2, y1);
                         }
-                        x0 *= klane;
-                        x1 *= klane;
+                        x0 = fmaf(y0, f0, x0);
+                        x1 = fmaf(y1, f1, x1);
+                    }
+                    if constexpr (HG == 1) {   // every lane of a row group gets the logits
                         x0 += __shfl_xor_sync(0xffffffffu, x0, 1);
                         x1 += __shfl_xor_sync(0xffffffffu, x1, 1);
+                    }
+                    if constexpr (HG <= 2) {   // digit 2 from lane t4 ^ 2
                         x0 += __shfl_xor_sync(0xffffffffu, x0, 2);
                         x1 += __shfl_xor_sync(0xffffffffu, x1, 2);
-                        const float lg0 = x0 - kbias, lg1 = x1 - kbias;
-                        mloc = fmaxf(mloc, fmaxf(lg0, lg1));
-                        if (t4 == 0) {
-                            lgc[16 * u + g8] = lg0;
-                            lgc[16 * u + g8 + 8] = lg1;
-                        }
+                    }
+                    const float lg0 = x0 - kbias, lg1 = x1 - kbias;
+                    mloc = fmaxf(mloc, fmaxf(lg0, lg1));
+                    if (t4 < HG) {
+                        lgc[(u * HG + hown) * 16 + logit_pos(g8)] = lg0;
+                        lgc[(u * HG + hown) * 16 + logit_pos(g8 + 8)] = lg1;
                     }
                 }
-                if (cc.r == cc.np - 1) {
-                    // the chunk's keys are done: fix its maximum, rescale what came before
-                    float cm = mloc;
-                    cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 4));
-                    cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 8));
-                    cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 16));
-                    if (cm > m) {
-                        const float alpha = fast_exp2(m - cm);
-                        m = cm;
-                        lsum *= alpha;
+            }
+            if (cc.r == cc.np - 1) {
+                // the chunk's keys are done: fix its maxima, rescale what came before
+                float cm = mloc;
+                cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 4));
+                cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 8));
+                cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 16));
+                const float mo = fmaxf(m_own, cm);
+                const float ao = fast_exp2(m_own - mo);
+                m_own = mo;
+                const float mBn = __shfl_sync(0xffffffffu, m_own, hb);   // lane hb holds head hb
+                const float aB = fast_exp2(mB - mBn);
+                mB = mBn;
+                if (__any_sync(0xffffffffu, ao != 1.f || aB != 1.f)) {
 #pragma unroll
-                        for (int j = 0; j < NJ; ++j) {
-                            dv[j][0] *= alpha; dv[j][1] *= alpha; dv[j][2] *= alpha; dv[j][3] *= alpha;
-                        }
-#pragma unroll
-                        for (int v = 0; v < NGV; ++v) zsum[v] *= alpha;
+                    for (int j = 0; j < NJ; ++j) {
+                        dv[j][0] *= ao; dv[j][1] *= ao; dv[j][2] *= ao; dv[j][3] *= ao;
                     }
-                    mloc = -INFINITY;
+                    lsum *= aB;
+#pragma unroll
+                    for (int v = 0; v < NGV; ++v) zsum[v] *= aB;
                 }
-            } else {
-                // p 2^-(7-N) of tokens 4*t4 + i (the B scale folded into the exponent)
-                const float mb = m + static_cast<float>(7 - N);
-                constexpr int kOff = 1 << N;
-                const bool lo_part = (g8 & 1) != 0;   // B column g8: hi part (even), lo part (odd)
+                mloc = -INFINITY;
+            }
+        } else {
+            // Value B of head hb: lane (g8, t4) owns tokens te = 4*t4 + e and te + 2 (e = g8 & 1),
+            // the k-pair of B register e, and builds both bf16 parts of p s 2^96 for them; the
+            // lane pair (e = 0, 1) then swaps halves: lane e = 0 keeps hi parts (column 2h),
+            // lane e = 1 lo parts (column 2h + 1).
+            const float mb = mB - static_cast<float>(kVScaleLog2);
+            const int e = g8 & 1, te = 4 * t4 + e;
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    if (u < nt) {
-                        const float4 l4 = *reinterpret_cast<const float4 *>(lgc + 16 * u + 4 * t4);
-                        const float pt[4] = {fast_exp2(l4.x - mb), fast_exp2(l4.y - mb), fast_exp2(l4.z - mb),
-                                             fast_exp2(l4.w - mb)};
-                        lsum += (pt[0] + pt[1]) + (pt[2] + pt[3]);
-                        float sv[4][NGV];
-                        int zv[4][NGV];
-                        load_meta4<NGV>(reinterpret_cast<const float *>(st + St::kMeta) + (16 * u + 4 * t4) * NGV,
-                                        reinterpret_cast<const int16_t *>(st + St::kVz) + (16 * u + 4 * t4) * NGV,
-                                        a.sym, zsym, sv, zv);
-                        uint32_t B0[NGV], B1[NGV];
+            for (int u = 0; u < 2; ++u) {
+                if (u < nt) {
+                    const float2 l2 = *reinterpret_cast<const float2 *>(lgc + (u * HG + hb) * 16 + 4 * t4 + 2 * e);
+                    const float p0 = fast_exp2(l2.x - mb), p1 = fast_exp2(l2.y - mb);
+                    lsum += p0 + p1;
+                    const float *sv = reinterpret_cast<const float *>(st + St::kMeta) + (16 * u + te) * NGV;
+                    const int16_t *zv = reinterpret_cast<const int16_t *>(st + St::kVz) + (16 * u + te) * NGV;
+                    uint32_t B0[NGV], B1[NGV];
 #pragma unroll
-                        for (int v = 0; v < NGV; ++v) {
-                            float ps[4];
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                ps[i] = pt[i] * sv[i][v];
-                                zsum[v] = fmaf(ps[i], small_int_to_float(zv[i][v] + kOff), zsum[v]);
-                            }
-                            // k order of the B fragment: (4t4, 4t4+2 | 4t4+1, 4t4+3), as codes_bf16 pairs
-                            // bytes; columns 2..7 repeat columns 0, 1 and their sums are not read
-                            const uint32_t h02 = f2bf2(ps[0], ps[2]), h13 = f2bf2(ps[1], ps[3]);
-                            const uint32_t l02 = f2bf2(ps[0] - __uint_as_float(h02 << 16),
-                                                       ps[2] - __uint_as_float(h02 & 0xffff0000u));
-                            const uint32_t l13 = f2bf2(ps[1] - __uint_as_float(h13 << 16),
-                                                       ps[3] - __uint_as_float(h13 & 0xffff0000u));
-                            B0[v] = lo_part ? l02 : h02;
-                            B1[v] = lo_part ? l13 : h13;
+                    for (int v = 0; v < NGV; ++v) {
+                        const float ps0 = p0 * sv[v], ps1 = p1 * sv[2 * NGV + v];
+                        if (!a.sym) {
+                            zsum[v] = fmaf(ps0, small_int_to_float(zv[v]), zsum[v]);
+                            zsum[v] = fmaf(ps1, small_int_to_float(zv[2 * NGV + v]), zsum[v]);
+                        } else {
+                            zsum[v] = fmaf(ps0 + ps1, static_cast<float>(zsym), zsum[v]);
                         }
-                        // ---- value MMAs: rows = channels of chunk j, k = the tile's tokens ----
-                        uint32_t vw[W];
-                        load_stage_words<W>(reinterpret_cast<const uint32_t *>(st + u * St::kCodes), lane, vw);
-                        const uint32_t magic16 = 0x43004300u;
+                        const uint32_t hi = f2bf2(ps0, ps1);
+                        const uint32_t lo = f2bf2(ps0 - __uint_as_float(hi << 16), ps1 - __uint_as_float(hi & 0xffff0000u));
+                        const uint32_t y = __shfl_xor_sync(0xffffffffu, e ? hi : lo, 4);
+                        B0[v] = e ? y : hi;
+                        B1[v] = e ? lo : y;
+                    }
+                    // ---- value MMAs: rows = channels of chunk j, k = the tile's tokens ----
+                    uint32_t vw[W];
+                    load_lane_words<W>(st + u * St::kCodes, lane, vw);
 #pragma unroll
-                        for (int j = 0; j < NJ; ++j) {
-                            uint32_t a02, a13, b02, b13;
-                            codes_bf16<N>(vw[j / BPW], 2 * (j % BPW), magic16, a02, a13);       // channel 16j + g8
-                            codes_bf16<N>(vw[j / BPW], 2 * (j % BPW) + 1, magic16, b02, b13);   // channel 16j + g8 + 8
-                            hmma(dv[j], a02, b02, a13, b13, B0[(16 * j) / GV], B1[(16 * j) / GV]);
+                    for (int wi = 0; wi < W; ++wi) {
+                        const uint32_t w02 = vw[wi], w13 = vw[wi] >> 8;   // bytes 0, 2 and 1, 3 in bits 0..7 of each half
+#pragma unroll
+                        for (int c = 0; c < BPW; ++c) {
+                            const int j = wi * BPW + c;
+                            const uint32_t m0 = HALF_L << (N * 2 * c), m1 = HALF_L << (N * (2 * c + 1));
+                            hmma(dv[j], w02 & m0, w02 & m1, w13 & m0, w13 & m1, B0[(16 * j) / GV], B1[(16 * j) / GV]);
                         }
                     }
                 }
             }
-            cc.next(ntiles);
-            __syncwarp();   // stage consumed and the chunk's logits visible to every lane
         }
-        cp_async_wait<0>();
+        cc.next(ntiles);
+        __syncwarp();   // stage consumed and the chunk's logits visible to every lane
+    }
+    // after an abandoned wait: give the copies still in flight their (bounded) time to land
+    for (int j = k + 1; j < min(issued, nitems); ++j) mbar_wait_bounded(bars + j % kSt, (j / kSt) & 1);
+    __syncwarp();
+    if (lane == 0) {
+#pragma unroll
+        for (int s = 0; s < kSt; ++s) mbar_inval(bars + s);
+    }
 
-        // lanes with the same t4 hold the same token sums: reduce over t4; lsum and zsum carry
-        // the 2^-(7-N) of the B operand, dv sums (2^N + code) p s
-        lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
-        lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
-        lsum *= static_cast<float>(1 << (7 - N));
+    // head sums of the value-B lanes: lanes g8 = 2h, 2h + 1 hold head h's tokens; reduce over
+    // t4 and the lane pair, then the lanes of head hown read them from lane 8 * hown
 #pragma unroll
-        for (int v = 0; v < NGV; ++v) {
-            zsum[v] += __shfl_xor_sync(0xffffffffu, zsum[v], 1);
-            zsum[v] += __shfl_xor_sync(0xffffffffu, zsum[v], 2);
-        }
-        constexpr float kUnscale = static_cast<float>(1 << (7 - N));
+    for (int o = 1; o <= 4; o <<= 1) {
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
 #pragma unroll
-        for (int j = 0; j < NJ; ++j) {
-            const float z = zsum[(16 * j) / GV] * kUnscale;
-            ov[j][0] = dv[j][0] + dv[j][1] - z;
-            ov[j][1] = dv[j][2] + dv[j][3] - z;
-        }
+        for (int v = 0; v < NGV; ++v) zsum[v] += __shfl_xor_sync(0xffffffffu, zsum[v], o);
+    }
+    constexpr float kUnB = 1.0f / (static_cast<float>(1ull << 48) * static_cast<float>(1ull << 48));   // 2^-96
+    const float l_own = __shfl_sync(0xffffffffu, lsum, 8 * hown) * kUnB;
+    float z_own[NGV];
+#pragma unroll
+    for (int v = 0; v < NGV; ++v) z_own[v] = __shfl_sync(0xffffffffu, zsum[v], 8 * hown) * kUnB;
+    // dv sums code 2^(N slot) 2^-133 p s 2^96 = 2^(N slot - 37) p s code
+    float ov[NJ][2];
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+        const int s0 = 2 * (j % BPW);
+        const float f0 = __uint_as_float(static_cast<uint32_t>(127 + 37 - N * s0) << 23);
+        const float f1 = __uint_as_float(static_cast<uint32_t>(127 + 37 - N * (s0 + 1)) << 23);
+        ov[j][0] = (dv[j][0] + dv[j][1]) * f0 - z_own[(16 * j) / GV];
+        ov[j][1] = (dv[j][2] + dv[j][3]) * f1 - z_own[(16 * j) / GV];
     }
 
     __syncthreads();   // stage memory is reused for the per-warp outputs
-    float *o_s = reinterpret_cast<float *>(stage_mem);   // [warp][D]
-    if (t4 == 0) {
+    if (t4 < HG) {
 #pragma unroll
         for (int j = 0; j < NJ; ++j) {
-            o_s[warp * D + 16 * j + g8] = ov[j][0];
-            o_s[warp * D + 16 * j + g8 + 8] = ov[j][1];
+            o_s[(warp * HG + hown) * D + 16 * j + g8] = ov[j][0];
+            o_s[(warp * HG + hown) * D + 16 * j + g8 + 8] = ov[j][1];
+        }
+        if (g8 == 0) {
+            ml_s[warp][hown][0] = m_own;
+            ml_s[warp][hown][1] = l_own;
         }
     }
-    if (lane == 0) {
-        ml_s[warp][0][0] = m;
-        ml_s[warp][0][1] = lsum;
-    }
     __syncthreads();
-    finish_cta<1, D>(a, o_s, ml_s, bq, bq, sigma, &last_s, o_s + kDecodeWarps * D);
+    finish_cta<HG, D>(a, o_s, ml_s, bh, bq0, sigma, &last_s, o_s + kDecodeWarps * HG * D);
 }
 
 template <int N, int D, int GV>
 constexpr int split_smem() { return kDecodeWarps * kStages * Stage<N, D, GV>::kBytes; }
-template <int N, int D, int GV>
-constexpr int gqa_smem() { return kDecodeWarps * GqaSmem<N, D, GV>::kWarpBytes; }
-template <int N, int D, int GV>
-constexpr int mha_smem() { return kDecodeWarps * MhaSmem<N, D, GV>::kWarpBytes; }
+template <int N, int D, int GV, int HG>
+constexpr int tc_smem() { return kDecodeWarps * TcSmem<N, D, GV, HG>::kWarpBytes; }
 
 // The opt-in to more than 48 KB of dynamic shared memory is per device and per
 // kernel; it is made once for each.
@@ -1688,31 +1456,37 @@ int occupancy_of(int smem) {
     return n > 0 ? n : 1;
 }
 
-// Dispatch over the compiled (bits, head_dim, value-group) variants and the three kernels.
+// Dispatch over the compiled (bits, head_dim, value-group) variants and the kernels.
 // The split index is the slowest grid dimension: CTAs start in linear order, so every
 // quantized split is resident before the (short) residual-split CTAs fill the slots
 // that remain.
 template <int N, int D, int GV>
 struct LaunchF {
+    template <int HG>
+    static cudaError_t tc(const DecodeArgs &a, cudaStream_t s) {
+        return launch_kernel<decode_tc_kernel<N, D, GV, HG>>(a, dim3(a.Hkv, a.B, a.S), tc_smem<N, D, GV, HG>(), s);
+    }
     static cudaError_t run(const DecodeArgs &a, cudaStream_t s) {
-        switch (a.path) {
-            case kPathGqa:
-                return launch_kernel<decode_gqa_kernel<N, D, GV>>(a, dim3(a.Hkv, a.B, a.S),
-                                                                  gqa_smem<N, D, GV>(), s);
-            case kPathMha:
-                return launch_kernel<decode_mha_kernel<N, D, GV>>(a, dim3(a.Hq, a.B, a.S),
-                                                                  mha_smem<N, D, GV>(), s);
-            default:
-                return launch_kernel<decode_split_kernel<N, D, GV>>(a, dim3(a.Hq, a.B, a.S),
-                                                                    split_smem<N, D, GV>(), s);
+        if (a.path == kPathTc) {
+            switch (a.Hq / a.Hkv) {
+                case 1: return tc<1>(a, s);
+                case 2: return tc<2>(a, s);
+                case 4: return tc<4>(a, s);
+                default: return cudaErrorInvalidValue;
+            }
         }
+        return launch_kernel<decode_split_kernel<N, D, GV>>(a, dim3(a.Hq, a.B, a.S), split_smem<N, D, GV>(), s);
     }
     static int occ(const DecodeArgs &a) {
-        switch (a.path) {
-            case kPathGqa: return occupancy_of<decode_gqa_kernel<N, D, GV>>(gqa_smem<N, D, GV>());
-            case kPathMha: return occupancy_of<decode_mha_kernel<N, D, GV>>(mha_smem<N, D, GV>());
-            default: return occupancy_of<decode_split_kernel<N, D, GV>>(split_smem<N, D, GV>());
+        if (a.path == kPathTc) {
+            switch (a.Hq / a.Hkv) {
+                case 1: return occupancy_of<decode_tc_kernel<N, D, GV, 1>>(tc_smem<N, D, GV, 1>());
+                case 2: return occupancy_of<decode_tc_kernel<N, D, GV, 2>>(tc_smem<N, D, GV, 2>());
+                case 4: return occupancy_of<decode_tc_kernel<N, D, GV, 4>>(tc_smem<N, D, GV, 4>());
+                default: return 1;
+            }
         }
+        return occupancy_of<decode_split_kernel<N, D, GV>>(split_smem<N, D, GV>());
     }
 };
 

@@ -125,16 +125,19 @@ void plan_splits(const kvq_cache *h, int *n_qsplits, int *tiles_per_split, int *
     const kvq_config &c = h->cfg;
     const int64_t tiles = h->Tq / 16;
     const int path = kvq::decode_path(c.q_heads, c.kv_heads, c.group_k);
-    // the MHA kernel deals the residual tiles to the warps of the quantized splits
-    const bool res_shared = path == kvq::kPathMha;
+    // with one query head per kv head the tensor-core kernel deals the residual tiles to the
+    // warps of the quantized splits
+    const int hg = c.q_heads / c.kv_heads;
+    const bool res_shared = path == kvq::kPathTc && hg == 1;
     const int extra = (h->r > 0 && !res_shared) ? 1 : 0;
     const int64_t align = kvq::split_tile_align(path);
-    // CTAs per split: one per query head, or one per kv head on the grouped-query path
-    const int64_t units = static_cast<int64_t>(c.batch) * (path == kvq::kPathGqa ? c.kv_heads : c.q_heads);
+    // CTAs per split: one per kv head on the tensor-core path, else one per query head
+    const int64_t units = static_cast<int64_t>(c.batch) * (path == kvq::kPathTc ? c.kv_heads : c.q_heads);
     const double slots = static_cast<double>(h->num_sms) * h->ctas_per_sm;
     const int64_t nres = (h->r + 15) / 16;
-    // residual CTA: its tiles shared by the 4 warps, or one warp per query head (grouped-query path)
-    const double c_res = kCtaFixedTiles + static_cast<double>(path == kvq::kPathGqa ? nres : (nres + 3) / 4);
+    // residual CTA: its tiles shared by the 4 warps of each of its query heads
+    const int heads_per_cta = path == kvq::kPathTc ? hg : 1;
+    const double c_res = kCtaFixedTiles + static_cast<double>((nres * heads_per_cta + 3) / 4);
     int64_t best_S = 0, best_per = 1;
     if (tiles > 0) {
         int64_t cap = (tiles + kMinTilesPerSplit - 1) / kMinTilesPerSplit;
@@ -194,6 +197,7 @@ kvq::DecodeArgs decode_args(const kvq_cache *h) {
     a.bf16 = c.dtype == KVQ_BF16;
     a.path = kvq::decode_path(c.q_heads, c.kv_heads, c.group_k);
     a.arrivals = h->arrivals;
+    a.status = h->arrivals + static_cast<int64_t>(c.batch) * c.q_heads;
     a.gshift = 0;
     while ((16 << a.gshift) < c.group_k) ++a.gshift;
     a.qscale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c.head_dim)));
@@ -271,8 +275,9 @@ kvq_status kvq_create(const kvq_config *cfg, const kvq_buffers *bufs, kvq_cache 
     }
     h->num_sms = sms > 0 ? sms : 148;
     h->ctas_per_sm = kvq::decode_ctas_per_sm(decode_args(h));
-    // the decode kernels' split-arrival counters: zeroed once here, left at zero by every decode
-    const size_t counter_bytes = static_cast<size_t>(cfg->batch) * cfg->q_heads * sizeof(unsigned int);
+    // the decode kernels' split-arrival counters (zeroed once here, left at zero by every
+    // decode) and, after them, their status word
+    const size_t counter_bytes = (static_cast<size_t>(cfg->batch) * cfg->q_heads + 1) * sizeof(unsigned int);
     e = cudaMalloc(&h->arrivals, counter_bytes);
     if (e == cudaSuccess) e = cudaMemset(h->arrivals, 0, counter_bytes);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
@@ -489,6 +494,20 @@ kvq_status kvq_cache_state(const kvq_cache *h, int64_t *quantized_tokens, int32_
     if (quantized_tokens) *quantized_tokens = h->Tq;
     if (residual_tokens) *residual_tokens = h->r;
     return ok();
+}
+
+kvq_status kvq_check_device(kvq_cache *h) {
+    if (!h) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+    unsigned int *word = h->arrivals + static_cast<int64_t>(h->cfg.batch) * h->cfg.q_heads;
+    unsigned int v = 0;
+    cudaError_t e = cudaMemcpy(&v, word, sizeof v, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the decode status word");
+    if (v == 0) return ok();
+    e = cudaMemset(word, 0, sizeof v);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the decode status word");
+    return fail(KVQ_ERR_CUDA, "a decode kernel gave up waiting for a copy into shared memory; "
+                              "outputs since the last check are unreliable");
 }
 
 uint64_t kvq_kernel_launches(void) { return g_launches.load(); }

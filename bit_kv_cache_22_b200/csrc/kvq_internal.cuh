@@ -54,20 +54,19 @@ cudaError_t launch_copy_rows(const uint16_t *src0, const uint16_t *src1, int64_t
                              int d, cudaStream_t s);
 
 // The decode kernel that serves a configuration:
-//  kPathGqa   4 query heads per kv head: tensor cores, one CTA per (batch, kv head, split);
-//  kPathMha   one query head per kv head, key groups of >= 32 tokens: tensor cores;
-//  kPathSplit any other grouping (or 16-token key groups): CUDA cores, one CTA per
+//  kPathTc    1, 2 or 4 query heads per kv head and key groups of >= 32 tokens: tensor
+//             cores, one CTA per (batch, kv head, split) serving those heads;
+//  kPathSplit any other grouping, or 16-token key groups: CUDA cores, one CTA per
 //             (batch, query head, split).
-enum DecodePath : int { kPathSplit = 0, kPathMha = 1, kPathGqa = 2 };
+enum DecodePath : int { kPathSplit = 0, kPathTc = 1 };
 
 inline int decode_path(int q_heads, int kv_heads, int group_k) {
-    if (q_heads == 4 * kv_heads) return kPathGqa;
-    if (q_heads == kv_heads && group_k >= 32) return kPathMha;
-    return kPathSplit;
+    const int g = q_heads / kv_heads;
+    return ((g == 1 || g == 2 || g == 4) && group_k >= 32) ? kPathTc : kPathSplit;
 }
-// Split boundaries must fall on multiples of this many tiles (the MHA kernel
-// stages tile pairs that must not straddle a key group).
-inline int split_tile_align(int path) { return path == kPathMha ? 2 : 1; }
+// Split boundaries must fall on multiples of this many tiles (the tensor-core
+// kernel streams tile pairs).
+inline int split_tile_align(int path) { return path == kPathTc ? 2 : 1; }
 
 struct DecodeArgs {
     const uint32_t *kc, *vc;
@@ -78,6 +77,7 @@ struct DecodeArgs {
     float *o_part, *m_part, *l_part;   // [B*Hq][S][d], [B*Hq][S], [B*Hq][S]
     float *out;                  // [B][Hq][d]
     unsigned int *arrivals;      // [B*Hq] split-arrival counters, zero between calls
+    unsigned int *status;        // nonzero once a bounded wait inside a decode kernel gave up
     int64_t cap;
     int B, Hq, Hkv, d, G, Gv, R, bits;
     int gshift;                  // log2(G / 16): key groups are 2^gshift tiles

@@ -30,7 +30,7 @@ KVQ_FP16, KVQ_BF16 = 0, 1
 EXPORTED = ("kvq_get_sizes", "kvq_create", "kvq_destroy", "kvq_reset", "kvq_prefill_quantize",
             "kvq_append", "kvq_decode_attention", "kvq_cache_state", "kvq_set_split_limit",
             "kvq_decode_splits", "kvq_kernel_launches", "kvq_decode_attention_noalloc",
-            "kvq_last_error", "kvq_layout_version")
+            "kvq_last_error", "kvq_layout_version", "kvq_check_device")
 
 
 class KVQError(RuntimeError):
@@ -96,8 +96,10 @@ def load() -> ctypes.CDLL:
         lib.kvq_last_error.restype = ctypes.c_char_p
         lib.kvq_layout_version.argtypes = []
         lib.kvq_layout_version.restype = i32
+        lib.kvq_check_device.argtypes = [P]
         for name in ("kvq_get_sizes", "kvq_create", "kvq_reset", "kvq_prefill_quantize",
-                     "kvq_append", "kvq_decode_attention", "kvq_cache_state", "kvq_set_split_limit"):
+                     "kvq_append", "kvq_decode_attention", "kvq_cache_state", "kvq_set_split_limit",
+                     "kvq_check_device"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -210,6 +212,10 @@ class KVQCache:
 
     def reset(self):
         _check(self._lib.kvq_reset(self._h))
+
+    def check_device(self):
+        """Raise KVQError if a decode kernel of this cache gave up one of its bounded waits."""
+        _check(self._lib.kvq_check_device(self._h))
 
     def prefill_quantize(self, X_K: torch.Tensor, X_V: torch.Tensor, stream=None):
         X_K, X_V = self._dev(X_K), self._dev(X_V)

@@ -20,9 +20,14 @@
  *
  * Conventions for every call:
  *  - Device memory (cache buffers, inputs, outputs, workspace) is owned and
- *    allocated by the caller.  The library allocates no device memory; it
- *    only keeps a small host-side handle with the cache geometry and the
- *    two counters Tq (quantized tokens) and r (residual tokens).
+ *    allocated by the caller.  The library's own device memory is one small
+ *    array per cache, allocated and zeroed by kvq_create and freed by
+ *    kvq_destroy: a 4-byte split-arrival counter per (batch, query head),
+ *    through which the last split of a decode merges the others, and a status
+ *    word.  Every decode leaves the counters at zero, so decode calls on one
+ *    cache must be ordered (one stream, or synchronised).  The host-side
+ *    handle keeps the cache geometry and the two counters Tq (quantized
+ *    tokens) and r (residual tokens).
  *  - Work is enqueued asynchronously on the caller's CUDA stream (`stream`
  *    is a cudaStream_t, NULL for the legacy default stream).  Host counters
  *    advance when a call is enqueued, so a sequence of calls needs no
@@ -123,11 +128,13 @@ KVQ_API kvq_status kvq_get_sizes(const kvq_config *cfg, kvq_sizes *out);
 /*
  * Creates a handle over caller-owned buffers (not copied, not freed).  The
  * cache starts empty (Tq = 0, r = 0).  Reads device properties of the current
- * device; all later calls must run with that device current.
+ * device, and allocates and zeroes (synchronously) the library's small
+ * per-cache array there; all later calls must run with that device current.
+ * KVQ_ERR_CUDA if that allocation fails.
  */
 KVQ_API kvq_status kvq_create(const kvq_config *cfg, const kvq_buffers *bufs, kvq_cache **out);
 
-/* Frees the host handle only.  NULL is ignored. */
+/* Frees the handle and the library's per-cache array.  NULL is ignored. */
 KVQ_API void kvq_destroy(kvq_cache *cache);
 
 /* Empties the cache (Tq = r = 0) without touching device memory. */
@@ -203,6 +210,17 @@ KVQ_API kvq_status kvq_set_split_limit(kvq_cache *cache, int32_t max_splits);
 
 /* Number of token splits the next kvq_decode_attention would use (>= 1). */
 KVQ_API int32_t kvq_decode_splits(const kvq_cache *cache);
+
+/*
+ * Reads, waiting for the device to finish its queued work, the status word that
+ * this cache's decode kernels raise when one of their bounded waits for a copy
+ * into shared memory gives up (a condition working hardware never reaches; the
+ * wait is bounded so that a fault cannot hang the GPU).  KVQ_OK when the word is
+ * clear; KVQ_ERR_CUDA when it was raised -- the outputs of the decodes since the
+ * last check are then unreliable, and the word is cleared -- or when the read
+ * fails.  The pages have no counterpart.
+ */
+KVQ_API kvq_status kvq_check_device(kvq_cache *cache);
 
 /* Kernels this library has launched in the process so far (all devices). */
 KVQ_API uint64_t kvq_kernel_launches(void);

@@ -92,6 +92,18 @@ def test_every_decode_path(g, d, bits, G, Gv, R):
     run_episode(w, check_every=7)
 
 
+def test_device_status_stays_clear():
+    """No bounded wait gives up in a normal decode; the status read succeeds and clears."""
+    w = reduced(wl.WORKLOADS["gqa8b"]).replace(steps=2)
+    XK, XV = wl.prefill_bits(w)
+    _, _, tQ = wl.decode_bits(w)
+    cache = tl.new_cache(w)
+    cache.prefill_quantize(tl.to_dev(XK, w), tl.to_dev(XV, w))
+    cache.decode_attention(tl.to_dev(tQ[0], w))
+    cache.check_device()
+    assert kvq.load().kvq_check_device(None) == kvq.KVQ_ERR_INVALID_ARG
+
+
 def test_repeated_decodes_are_identical_across_split_counts():
     """The split-merge counters return to zero after every call: the same query
     gives the same output call after call, whatever the split count in between."""
