@@ -268,6 +268,11 @@ def run_kvq(args):
         g_app.append(ga)
         g_dec.append(gd)
     launches_per_episode = kvq.kernel_launches() - launches0
+    # the whole episode as one graph: what `value` times
+    cache.reset()
+    g_ep = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_ep, pool=pool):
+        episode()
     torch.cuda.synchronize()
 
     def replay_episode(ev):
@@ -282,14 +287,22 @@ def run_kvq(args):
             for _ in range(w.steps)] for _ in range(args.steps + 1)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
-        replay_episode(evs[-1])          # graph warm-up (also gives the sampler time to start)
+        g_ep.replay()                    # graph warm-up (also gives the sampler time to start)
+        replay_episode(evs[-1])
         torch.cuda.synchronize()
         barrier()
         torch.cuda.synchronize()
+        # timed region: K episodes, each one whole-episode graph replay
         start.record(stream)
         for k in range(args.steps):
-            replay_episode(evs[k])
+            g_ep.replay()
         stop.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        # the same K episodes replayed step by step, with events around every
+        # decode_attention call: the per-call duration the roofline uses
+        for k in range(args.steps):
+            replay_episode(evs[k])
         torch.cuda.synchronize()
         barrier()
     launches = launches_per_episode * args.steps
@@ -370,6 +383,9 @@ def run_kvq(args):
                   f"{bytes_per_episode / w.steps / 1e6:.0f} MB per decode step, prompt "
                   f"{2 * XK.numel() * 2 / 1e6:.0f} MB per step",
             "splits": cache.splits(),
+            "timing": "value: K whole-episode CUDA-graph replays between two events; roofline: "
+                      "events around every decode_attention graph in K more episodes replayed "
+                      "step by step",
         },
         "decode_steps_per_s": w.steps * args.steps / (ms / 1e3),
         "kv_tokens_per_s_decode_only": job_throughput(tokens_per_episode * args.steps, world, decode_ms),

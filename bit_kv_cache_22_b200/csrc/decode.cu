@@ -897,7 +897,7 @@ __device__ __forceinline__ void load_meta4(const float *sp, const int16_t *zp, b
 }
 
 template <int D, int GV, int HG>
-__host__ __device__ constexpr int tc_min_ctas() { return (HG == 4 || D / GV >= 4) ? 3 : 4; }
+__host__ __device__ constexpr int tc_min_ctas() { return 4; }
 
 template <int N, int D, int GV, int HG>
 __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) decode_tc_kernel(const DecodeArgs a) {
