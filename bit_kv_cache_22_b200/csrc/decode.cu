@@ -167,18 +167,21 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
                  ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
                  : "memory");
 }
+// One poll; the thread may be suspended up to kPollSuspendNs waiting for the phase, so a
+// waiting warp takes (almost) no issue slots from the working ones.
+constexpr uint32_t kPollSuspendNs = 200000;
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "n"(kPollSuspendNs)
         : "memory");
     return ok != 0;
 }
 // Waits for the phase of `parity` to complete, giving up after kSpinLimit polls
-// (each poll may suspend the thread for a while); false when it gave up.
-constexpr uint32_t kSpinLimit = 1u << 22;
+// (at most about kSpinLimit * kPollSuspendNs, a few seconds); false when it gave up.
+constexpr uint32_t kSpinLimit = 1u << 14;
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
     for (uint32_t i = 0; i < kSpinLimit; ++i)
         if (mbar_try_wait(bar, parity)) return true;
@@ -707,6 +710,18 @@ __device__ __forceinline__ void residual_pass(const DecodeArgs &a, const float *
 // ---------------------------------------------------------------------------
 // Tensor-core helpers (mma.sync).
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ void imma_uu(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void imma_uu0(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0));
+}
 __device__ __forceinline__ void imma_us(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
@@ -869,32 +884,6 @@ struct TcSmem {
 // Position of token t (0..15) of a tile in the logits buffer: tokens 4q + e and 4q + e + 2
 // sit side by side, the pair one lane of the value-B build needs.
 __device__ __forceinline__ int logit_pos(int t) { return 4 * (t >> 2) + 2 * (t & 1) + ((t >> 1) & 1); }
-
-// Value scales and zeros of the four tokens 4*t4 + i of a lane (NGV of each).
-template <int NGV>
-__device__ __forceinline__ void load_meta4(const float *sp, const int16_t *zp, bool sym, int zsym,
-                                           float (&s)[4][NGV], int (&z)[4][NGV]) {
-    if constexpr (NGV == 1) {
-        const float4 v = *reinterpret_cast<const float4 *>(sp);
-        s[0][0] = v.x; s[1][0] = v.y; s[2][0] = v.z; s[3][0] = v.w;
-        if (sym) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) z[i][0] = zsym;
-        } else {
-            const uint2 u = *reinterpret_cast<const uint2 *>(zp);
-            z[0][0] = static_cast<int16_t>(u.x & 0xffffu); z[1][0] = static_cast<int16_t>(u.x >> 16);
-            z[2][0] = static_cast<int16_t>(u.y & 0xffffu); z[3][0] = static_cast<int16_t>(u.y >> 16);
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            int16_t zz[NGV];
-            load_meta<NGV>(sp + i * NGV, zp + i * NGV, sym, zsym, s[i], zz);
-#pragma unroll
-            for (int v = 0; v < NGV; ++v) z[i][v] = zz[v];
-        }
-    }
-}
 
 template <int D, int GV, int HG>
 __host__ __device__ constexpr int tc_min_ctas() { return 4; }
@@ -1087,10 +1076,10 @@ __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) deco
                           static_cast<float>(zsym)};
             if (!a.sym) {
                 const uint2 zz = *reinterpret_cast<const uint2 *>(kz_s + 4 * cc);
-                z[0] = small_int_to_float(static_cast<int16_t>(zz.x & 0xffffu));
-                z[1] = small_int_to_float(static_cast<int16_t>(zz.x >> 16));
-                z[2] = small_int_to_float(static_cast<int16_t>(zz.y & 0xffffu));
-                z[3] = small_int_to_float(static_cast<int16_t>(zz.y >> 16));
+                z[0] = static_cast<float>(static_cast<int16_t>(zz.x & 0xffffu));
+                z[1] = static_cast<float>(static_cast<int16_t>(zz.x >> 16));
+                z[2] = static_cast<float>(static_cast<int16_t>(zz.y & 0xffffu));
+                z[3] = static_cast<float>(static_cast<int16_t>(zz.y >> 16));
             }
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -1108,7 +1097,9 @@ __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) deco
         if (mx > 0.f) e = 21 - (static_cast<int>((__float_as_uint(mx) >> 23) & 0xff) - 126);
         e = max(-120, min(120, e));
         const float scale = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
-        // balanced base-256 digits: Q = d0 + 256 d1 + 65536 d2 with d0, d1 in [-128, 127]
+        // base-256 digits Q = d0 + 256 d1 + 65536 d2.  HG = 4: the bytes of Q themselves,
+        // d0 and d1 unsigned and d2 signed (digit 2 has an n-tile, and an MMA type, of its own);
+        // HG <= 2 (all digits in one n-tile, one signed type): balanced d0, d1 in [-128, 127]
         uint32_t dw[3][QPL];
 #pragma unroll
         for (int i = 0; i < QPL; ++i) {
@@ -1116,10 +1107,16 @@ __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) deco
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int Q = round_small(qv[i][k] * scale);
-                const int Q1 = (Q + 128) >> 8;
-                dg[0][k] = Q;
-                dg[1][k] = Q1;
-                dg[2][k] = (Q1 + 128) >> 8;
+                if constexpr (HG == 4) {
+                    dg[0][k] = Q;
+                    dg[1][k] = Q >> 8;
+                    dg[2][k] = Q >> 16;
+                } else {
+                    const int Q1 = (Q + 128) >> 8;
+                    dg[0][k] = Q;
+                    dg[1][k] = Q1;
+                    dg[2][k] = (Q1 + 128) >> 8;
+                }
             }
 #pragma unroll
             for (int k = 0; k < 3; ++k)
@@ -1254,8 +1251,13 @@ __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) deco
                                                     kw[2 * pm + 1] & mhi};
 #pragma unroll
                             for (int n = 0; n < NTK; ++n) {
-                                if (pm < 2) imma_us0(acc[n][pm][c], af, kb[n][pm * BPW + c][0], kb[n][pm * BPW + c][1]);
-                                else imma_us(acc[n][pm & 1][c], af, kb[n][pm * BPW + c][0], kb[n][pm * BPW + c][1]);
+                                if (HG == 4 && n == 0) {   // unsigned digits 0, 1
+                                    if (pm < 2) imma_uu0(acc[n][pm][c], af, kb[n][pm * BPW + c][0], kb[n][pm * BPW + c][1]);
+                                    else imma_uu(acc[n][pm & 1][c], af, kb[n][pm * BPW + c][0], kb[n][pm * BPW + c][1]);
+                                } else {
+                                    if (pm < 2) imma_us0(acc[n][pm][c], af, kb[n][pm * BPW + c][0], kb[n][pm * BPW + c][1]);
+                                    else imma_us(acc[n][pm & 1][c], af, kb[n][pm * BPW + c][0], kb[n][pm * BPW + c][1]);
+                                }
                             }
                         }
                     }
@@ -1264,12 +1266,24 @@ __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) deco
                     for (int c = 0; c < BPW; ++c) {   // digit sums d0 + 256 d1 (< 2^31), slot factor out
                         const float f0 = 1.0f / static_cast<float>(1u << (2 * N * c));
                         const float f1 = 1.0f / static_cast<float>(1u << (N * (2 * c + 1)));
-                        int r0 = acc[0][0][c][0] + acc[0][0][c][1] * 256, r1 = acc[0][0][c][2] + acc[0][0][c][3] * 256;
-                        if constexpr (NP > 1) {
-                            r0 += acc[0][1][c][0] + acc[0][1][c][1] * 256;
-                            r1 += acc[0][1][c][2] + acc[0][1][c][3] * 256;
+                        float y0, y1;
+                        if constexpr (HG == 4) {   // unsigned digit sums (< 2^23 each): convert apart
+                            int s0 = acc[0][0][c][0], s1 = acc[0][0][c][1], s2 = acc[0][0][c][2], s3 = acc[0][0][c][3];
+                            if constexpr (NP > 1) {
+                                s0 += acc[0][1][c][0]; s1 += acc[0][1][c][1];
+                                s2 += acc[0][1][c][2]; s3 += acc[0][1][c][3];
+                            }
+                            y0 = fmaf(static_cast<float>(s1), 256.f, static_cast<float>(s0)) * klane;
+                            y1 = fmaf(static_cast<float>(s3), 256.f, static_cast<float>(s2)) * klane;
+                        } else {
+                            int r0 = acc[0][0][c][0] + acc[0][0][c][1] * 256, r1 = acc[0][0][c][2] + acc[0][0][c][3] * 256;
+                            if constexpr (NP > 1) {
+                                r0 += acc[0][1][c][0] + acc[0][1][c][1] * 256;
+                                r1 += acc[0][1][c][2] + acc[0][1][c][3] * 256;
+                            }
+                            y0 = static_cast<float>(r0) * klane;
+                            y1 = static_cast<float>(r1) * klane;
                         }
-                        float y0 = static_cast<float>(r0) * klane, y1 = static_cast<float>(r1) * klane;
                         if constexpr (NTK == 2) {   // digit 2 of head t4 in the second n-tile
                             int e0 = acc[1][0][c][0], e1 = acc[1][0][c][2];
                             if constexpr (NP > 1) {
@@ -1334,18 +1348,20 @@ __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) deco
                     const float2 l2 = *reinterpret_cast<const float2 *>(lgc + (u * HG + hb) * 16 + 4 * t4 + 2 * e);
                     const float p0 = fast_exp2(l2.x - mb), p1 = fast_exp2(l2.y - mb);
                     lsum += p0 + p1;
-                    const float *sv = reinterpret_cast<const float *>(st + St::kMeta) + (16 * u + te) * NGV;
-                    const int16_t *zv = reinterpret_cast<const int16_t *>(st + St::kVz) + (16 * u + te) * NGV;
+                    float s0[NGV], s1[NGV];
+                    int16_t z0[NGV], z1[NGV];
+                    load_meta<NGV>(reinterpret_cast<const float *>(st + St::kMeta) + (16 * u + te) * NGV,
+                                   reinterpret_cast<const int16_t *>(st + St::kVz) + (16 * u + te) * NGV, a.sym,
+                                   zsym, s0, z0);
+                    load_meta<NGV>(reinterpret_cast<const float *>(st + St::kMeta) + (16 * u + te + 2) * NGV,
+                                   reinterpret_cast<const int16_t *>(st + St::kVz) + (16 * u + te + 2) * NGV, a.sym,
+                                   zsym, s1, z1);
                     uint32_t B0[NGV], B1[NGV];
 #pragma unroll
                     for (int v = 0; v < NGV; ++v) {
-                        const float ps0 = p0 * sv[v], ps1 = p1 * sv[2 * NGV + v];
-                        if (!a.sym) {
-                            zsum[v] = fmaf(ps0, small_int_to_float(zv[v]), zsum[v]);
-                            zsum[v] = fmaf(ps1, small_int_to_float(zv[2 * NGV + v]), zsum[v]);
-                        } else {
-                            zsum[v] = fmaf(ps0 + ps1, static_cast<float>(zsym), zsum[v]);
-                        }
+                        const float ps0 = p0 * s0[v], ps1 = p1 * s1[v];
+                        zsum[v] = fmaf(ps0, static_cast<float>(z0[v]), zsum[v]);
+                        zsum[v] = fmaf(ps1, static_cast<float>(z1[v]), zsum[v]);
                         const uint32_t hi = f2bf2(ps0, ps1);
                         const uint32_t lo = f2bf2(ps0 - __uint_as_float(hi << 16), ps1 - __uint_as_float(hi & 0xffff0000u));
                         const uint32_t y = __shfl_xor_sync(0xffffffffu, e ? hi : lo, 4);
