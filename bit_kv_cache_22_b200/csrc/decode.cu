@@ -781,14 +781,14 @@ __device__ __forceinline__ void load_meta(const float *sp, const int16_t *zp, bo
 //
 // A CTA owns one (batch, kv head, split) and serves the HG query heads that
 // read that kv head, so every code is fetched and unpacked once for all of
-// them.  Each warp takes an even-aligned, contiguous share of the split's tiles
+// them.  Each warp takes a contiguous share of the split's tiles, aligned to items,
 // and walks it in chunks of tc_chunk<HG>() tiles: first the chunk's keys (the
 // logits of its HG heads go to shared memory, each lane keeps a running
 // maximum), then, with the chunk's maxima fixed, its values.  So probabilities
 // need no per-tile cross-lane maximum, key and value work form two streams
 // without dependences between tiles, and accumulators are rescaled at most once
-// per chunk.  Items -- a key tile pair or a value tile pair -- stream through a
-// per-warp ring of cp.async stages.  Lane = 4*g8 + t4.
+// per chunk.  Items -- 4 tiles of keys or 4 tiles of values -- stream through a
+// per-warp ring of bulk-copy stages.  Lane = 4*g8 + t4.
 //   keys   : int8 MMA m16n8k32, rows = tokens, k = channels.  A is a stored
 //            word masked to one byte slot, without a shift: slot s arrives as
 //            code * 2^(N*s); the two 16-channel chunks of one MMA come from the
@@ -813,7 +813,7 @@ __device__ __forceinline__ void load_meta(const float *sp, const int16_t *zp, bo
 // all splits, which run them first on CUDA cores (staged in shared memory) and
 // start their softmax state from them; with HG > 1 they form one more split.
 // ---------------------------------------------------------------------------
-constexpr int kTcStages = 4;
+constexpr int kTcItem = 4;         // tiles per item (stage)
 constexpr int kVScaleLog2 = 96;   // the value MMA's B operand is p s 2^96
 
 // Tiles per key phase / value phase of a warp (the logits of a chunk take 2 KB).
@@ -856,28 +856,36 @@ __device__ __forceinline__ void load_lane_words(const unsigned char *base, int l
 }
 
 template <int N, int D, int GV>
-struct TcStage {                  // one item: two tiles of one code array and their meta
+struct TcStage {                  // one item: kTcItem tiles of one code array and their meta
     static constexpr int W = D * N / 64;
     static constexpr int NGV = D / GV;
     static constexpr int kCodes = 32 * W * 4;            // one tile's code array, as stored (lane-major)
-    static constexpr int kMeta = 2 * kCodes;
-    // key item: the scales [D] f32 (at kMeta) and zeros [D] i16 (at kKz) of the key group its
-    // first tile opens (groups of >= 32 tokens: an even-aligned tile pair opens at most one)
-    static constexpr int kKz = kMeta + D * 4;
-    // value item: scales [32][NGV] f32 at kMeta, zeros [32][NGV] i16 at kVz
-    static constexpr int kVz = kMeta + 32 * NGV * 4;
-    static constexpr int kEnd = (kKz + D * 2 > kVz + 32 * NGV * 2) ? kKz + D * 2 : kVz + 32 * NGV * 2;
+    static constexpr int kMeta = kTcItem * kCodes;
+    // key item: scales [2][D] f32 at kMeta and zeros [2][D] i16 at kKz: slot 0 the group its
+    // first tile opens, slot 1 the group its third tile opens (groups of 32 tokens); groups
+    // of >= 64 tokens start on item boundaries, so they use slot 0 only
+    static constexpr int kKz = kMeta + 2 * D * 4;
+    // value item: scales [16 * kTcItem][NGV] f32 at kMeta, zeros [16 * kTcItem][NGV] i16 at kVz
+    static constexpr int kVz = kMeta + 16 * kTcItem * NGV * 4;
+    static constexpr int kEnd = (kKz + 2 * D * 2 > kVz + 16 * kTcItem * NGV * 2) ? kKz + 2 * D * 2
+                                                                                : kVz + 16 * kTcItem * NGV * 2;
     static constexpr int kBytes = (kEnd + 15) / 16 * 16;
     static_assert(kMeta % 16 == 0 && kKz % 16 == 0 && kVz % 16 == 0, "align");
 };
 
+// Stages per warp ring: two (one in use, one in flight), three when items are small enough
+// for four CTAs of four warps to keep them in shared memory.
+template <int N, int D, int GV>
+__host__ __device__ constexpr int tc_stages() { return TcStage<N, D, GV>::kBytes <= 3072 ? 3 : 2; }
+
 template <int N, int D, int GV, int HG>
 struct TcSmem {
+    static constexpr int kSt = tc_stages<N, D, GV>();
     static constexpr int kKdWords = D / 4 + 4;   // one digit row (4 channels a word), padded by 4 banks
-    static constexpr int kLg = kTcStages * TcStage<N, D, GV>::kBytes;          // logits [chunk][HG][16] f32
+    static constexpr int kLg = kSt * TcStage<N, D, GV>::kBytes;                // logits [chunk][HG][16] f32
     static constexpr int kKd = kLg + tc_chunk<HG>() * HG * 16 * 4;             // digits [HG][3][kKdWords]
-    static constexpr int kBars = kKd + HG * 3 * kKdWords * 4;                 // stage barriers [kTcStages]
-    static constexpr int kWarpBytes = (kBars + kTcStages * 8 + 15) / 16 * 16;
+    static constexpr int kBars = kKd + HG * 3 * kKdWords * 4;                 // stage barriers [kSt]
+    static constexpr int kWarpBytes = (kBars + kSt * 8 + 15) / 16 * 16;
     static_assert(kLg % 16 == 0 && kBars % 16 == 0, "align");
 };
 
@@ -902,12 +910,12 @@ __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) deco
     constexpr int kChunk = tc_chunk<HG>();
     constexpr uint32_t BYTE_L = ((1u << N) - 1u) * 0x01010101u;
     constexpr uint32_t HALF_L = ((1u << N) - 1u) * 0x00010001u;
-    constexpr int kSt = kTcStages;
     using St = TcStage<N, D, GV>;
     using Sm = TcSmem<N, D, GV, HG>;
+    constexpr int kSt = Sm::kSt;
     static_assert(HG == 1 || HG == 2 || HG == 4, "heads per kv head");
     static_assert(W % 2 == 0, "key MMAs take words in pairs");
-    static_assert(kChunk % 2 == 0 && (kChunk & (kChunk - 1)) == 0, "chunk");
+    static_assert(kChunk % kTcItem == 0 && (kChunk & (kChunk - 1)) == 0, "chunk");
     static_assert(residual_scratch_bytes<D>() <= Sm::kBars, "residual staging");
     static_assert(kDecodeWarps * HG * D * 4 + HG * 66 * 4 <= (kDecodeWarps - 1) * Sm::kWarpBytes + Sm::kBars,
                   "epilogue");
@@ -972,73 +980,81 @@ __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) deco
     }
 
     // ---------------- quantized split ----------------
-    const int t_begin = sigma * a.tiles_per_split;                 // even
+    const int t_begin = sigma * a.tiles_per_split;                 // multiple of kTcItem
     const int t_end = min(a.n_qtiles, t_begin + a.tiles_per_split);
-    const int per_w = 2 * ((t_end - t_begin + 2 * kDecodeWarps - 1) / (2 * kDecodeWarps));
-    const int wb = min(t_end, t_begin + warp * per_w);             // even
+    const int per_w = kTcItem * ((t_end - t_begin + kTcItem * kDecodeWarps - 1) / (kTcItem * kDecodeWarps));
+    const int wb = min(t_end, t_begin + warp * per_w);             // multiple of kTcItem
     const int ntiles = min(t_end, wb + per_w) - wb;
-    const int nitems = 2 * ((ntiles + 1) / 2);   // one key item and one value item per tile pair
-    const int64_t groups_cap = a.cap / a.G;
+    const int nitems = 2 * ((ntiles + kTcItem - 1) / kTcItem);     // a key item and a value item per kTcItem tiles
     const int64_t tile0 = bh * (a.cap / 16) + wb;
-    const uint32_t *kp = a.kc + tile0 * TW;
-    const uint32_t *vp = a.vc + tile0 * TW;
-    const float *vsp = a.vs + tile0 * 16 * NGV;
-    const int16_t *vzp = a.sym ? nullptr : a.vz + tile0 * 16 * NGV;
     const int gmask = (1 << a.gshift) - 1;
 
-    // Item cursor: chunk [cb, cb + kChunk) of the warp's tiles holds np tile pairs; items
-    // 0 .. np-1 of a chunk are its key pairs, np .. 2np-1 its value pairs.
+    // Item cursor: chunk [cb, cb + kChunk) of the warp's tiles holds ni items of each kind;
+    // items 0 .. ni-1 of a chunk are its key items, ni .. 2ni-1 its value items.
     struct Cursor {
-        int cb, r, np;
-        __device__ void start(int n) { cb = 0; r = 0; np = (min(kChunk, n) + 1) / 2; }
+        int cb, r, ni;
+        __device__ void start(int n) { cb = 0; r = 0; ni = (min(kChunk, n) + kTcItem - 1) / kTcItem; }
         __device__ void next(int n) {
-            if (++r == 2 * np) {
+            if (++r == 2 * ni) {
                 cb += kChunk;
                 r = 0;
-                np = (min(kChunk, n - cb) + 1) / 2;
+                ni = (min(kChunk, n - cb) + kTcItem - 1) / kTcItem;
             }
         }
-        __device__ bool key() const { return r < np; }
-        __device__ int rel() const { return cb + 2 * (r < np ? r : r - np); }
+        __device__ bool key() const { return r < ni; }
+        __device__ int rel() const { return cb + kTcItem * (r < ni ? r : r - ni); }
     };
 
     // Producer: lane 0 loads item `issued` into stage issued % kSt with bulk copies that
-    // complete on the stage's barrier: the tile pair's codes (one contiguous copy), then a
-    // key item's group scales / zeros (of the group its first tile opens, if any) or a value
-    // item's scales / zeros.
+    // complete on the stage's barrier: the item's codes (one contiguous copy), then a key
+    // item's group scales / zeros (the groups its tiles open, consecutive in memory) or a
+    // value item's scales / zeros.  Key and value items each advance through the warp's tiles
+    // in order, so the sources are running pointers.
     Cursor ic;       // producer's cursor, kSt - 1 items ahead
     ic.start(ntiles);
     int issued = 0;
+    const uint32_t *ksrc = a.kc + tile0 * TW, *vsrc = a.vc + tile0 * TW;
+    const float *vssrc = a.vs + tile0 * 16 * NGV;
+    const int16_t *vzsrc = a.sym ? nullptr : a.vz + tile0 * 16 * NGV;
+    const int64_t gbase = bh * (a.cap / a.G);
     auto issue_next = [&]() {
         if (issued < nitems) {
+            const int rel = ic.rel();
+            const int nt = min(kTcItem, ntiles - rel);
             if (lane == 0) {
                 unsigned char *st = wmem + (issued % kSt) * St::kBytes;
                 uint64_t *bar = bars + issued % kSt;
-                const int rel = ic.rel();
-                const int nt = rel + 1 < ntiles ? 2 : 1;
-                const uint32_t cbytes = nt * St::kCodes;
+                const uint32_t cbytes = static_cast<uint32_t>(nt * St::kCodes);
                 fence_proxy_async();   // this stage's earlier reads come before the copies below
                 if (ic.key()) {
                     const int ti = wb + rel;
-                    const bool open = rel == 0 || (ti & gmask) == 0;
-                    const uint32_t sb = open ? static_cast<uint32_t>(D * 4) : 0u;
-                    const uint32_t zb = (open && !a.sym) ? static_cast<uint32_t>(D * 2) : 0u;
+                    const bool open0 = rel == 0 || (ti & gmask) == 0;
+                    const bool open2 = nt > 2 && ((ti + 2) & gmask) == 0;   // groups of 32 tokens
+                    const int ng = open0 + open2;
+                    const uint32_t sb = static_cast<uint32_t>(ng * D * 4);
+                    const uint32_t zb = a.sym ? 0u : static_cast<uint32_t>(ng * D * 2);
                     mbar_expect_tx(bar, cbytes + sb + zb);
-                    bulk_g2s(st, kp + static_cast<int64_t>(rel) * TW, cbytes, bar);
-                    if (open) {
-                        const int64_t gofs = (bh * groups_cap + (ti >> a.gshift)) * D;
-                        bulk_g2s(st + St::kMeta, a.ks + gofs, sb, bar);
-                        if (!a.sym) bulk_g2s(st + St::kKz, a.kz + gofs, zb, bar);
+                    bulk_g2s(st, ksrc, cbytes, bar);
+                    if (ng > 0) {
+                        const int64_t gofs = (gbase + ((open0 ? ti : ti + 2) >> a.gshift)) * D;
+                        bulk_g2s(st + St::kMeta + (open0 ? 0 : D * 4), a.ks + gofs, sb, bar);
+                        if (!a.sym) bulk_g2s(st + St::kKz + (open0 ? 0 : D * 2), a.kz + gofs, zb, bar);
                     }
                 } else {
                     const uint32_t sb = static_cast<uint32_t>(nt * 16 * NGV * 4);
                     const uint32_t zb = a.sym ? 0u : sb / 2;
                     mbar_expect_tx(bar, cbytes + sb + zb);
-                    bulk_g2s(st, vp + static_cast<int64_t>(rel) * TW, cbytes, bar);
-                    const int64_t tok = static_cast<int64_t>(rel) * 16 * NGV;
-                    bulk_g2s(st + St::kMeta, vsp + tok, sb, bar);
-                    if (!a.sym) bulk_g2s(st + St::kVz, vzp + tok, zb, bar);
+                    bulk_g2s(st, vsrc, cbytes, bar);
+                    bulk_g2s(st + St::kMeta, vssrc, sb, bar);
+                    if (!a.sym) bulk_g2s(st + St::kVz, vzsrc, zb, bar);
                 }
+            }
+            if (ic.key()) {
+                ksrc += kTcItem * TW;
+            } else {
+                vsrc += kTcItem * TW;
+                vssrc += kTcItem * 16 * NGV;
+                if (!a.sym) vzsrc += kTcItem * 16 * NGV;
             }
             ic.next(ntiles);
         }
@@ -1218,6 +1234,7 @@ __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) deco
     Cursor cc;       // consumer's cursor
     cc.start(ntiles);
     int k = 0;
+    const int e = g8 & 1, te = 4 * t4 + e;   // value-B lanes: token pair te, te + 2 (see below)
     for (; k < nitems; ++k) {
         issue_next();
         // wait for item k; a wait that gives up (never expected) raises the device status flag
@@ -1229,16 +1246,18 @@ __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) deco
         }
         const unsigned char *st = wmem + (k % kSt) * St::kBytes;
         const int rel = cc.rel();
-        const int nt = rel + 1 < ntiles ? 2 : 1;
-        float *lgc = lgs + (rel % kChunk) * HG * 16;   // logits of tiles rel, rel + 1: [tile][head][16]
+        const int nt = min(kTcItem, ntiles - rel);
+        float *lgc = lgs + (rel & (kChunk - 1)) * HG * 16;   // logits of the item's tiles: [tile][head][16]
         if (cc.key()) {
             // ---- key MMAs: log2-domain logits of tokens g8 and g8 + 8, head hown ----
+            const bool open0 = rel == 0 || ((wb + rel) & gmask) == 0;
+            const bool open2 = ((wb + rel + 2) & gmask) == 0;
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
+            for (int u = 0; u < kTcItem; ++u) {
                 if (u < nt) {
-                    if (u == 0 && (rel == 0 || ((wb + rel) & gmask) == 0))
-                        rebuild_key_digits(reinterpret_cast<const float *>(st + St::kMeta),
-                                           reinterpret_cast<const int16_t *>(st + St::kKz));
+                    if ((u == 0 && open0) || (u == 2 && open2))
+                        rebuild_key_digits(reinterpret_cast<const float *>(st + St::kMeta) + (u == 2 ? D : 0),
+                                           reinterpret_cast<const int16_t *>(st + St::kKz) + (u == 2 ? D : 0));
                     uint32_t kw[W];
                     load_lane_words<W>(st + u * St::kCodes, lane, kw);
                     int acc[NTK][2][BPW][4];   // two chains (even / odd word pair) per n-tile
@@ -1312,7 +1331,7 @@ __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) deco
                     }
                 }
             }
-            if (cc.r == cc.np - 1) {
+            if (cc.r == cc.ni - 1) {
                 // the chunk's keys are done: fix its maxima, rescale what came before
                 float cm = mloc;
                 cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 4));
@@ -1341,9 +1360,8 @@ __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) deco
             // lane pair (e = 0, 1) then swaps halves: lane e = 0 keeps hi parts (column 2h),
             // lane e = 1 lo parts (column 2h + 1).
             const float mb = mB - static_cast<float>(kVScaleLog2);
-            const int e = g8 & 1, te = 4 * t4 + e;
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
+            for (int u = 0; u < kTcItem; ++u) {
                 if (u < nt) {
                     const float2 l2 = *reinterpret_cast<const float2 *>(lgc + (u * HG + hb) * 16 + 4 * t4 + 2 * e);
                     const float p0 = fast_exp2(l2.x - mb), p1 = fast_exp2(l2.y - mb);

@@ -65,8 +65,8 @@ inline int decode_path(int q_heads, int kv_heads, int group_k) {
     return ((g == 1 || g == 2 || g == 4) && group_k >= 32) ? kPathTc : kPathSplit;
 }
 // Split boundaries must fall on multiples of this many tiles (the tensor-core
-// kernel streams tile pairs).
-inline int split_tile_align(int path) { return path == kPathTc ? 2 : 1; }
+// kernel streams items of 4 tiles).
+inline int split_tile_align(int path) { return path == kPathTc ? 4 : 1; }
 
 struct DecodeArgs {
     const uint32_t *kc, *vc;
