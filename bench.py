@@ -222,8 +222,7 @@ def run_kvq(args):
     if args.ncu_case:
         cache.prefill_quantize(XK, XV)
         for s in range(min(w.steps, 64)):      # ends with r = 64 residual rows, mid-episode
-            cache.append(tK[s], tV[s])
-            cache.decode_attention(tQ[s], out=out)
+            cache.append_decode(tK[s], tV[s], tQ[s], out=out)
         torch.cuda.synchronize()
         print(json.dumps({"ncu_case": args.workload, "state": cache.state()}))
         return
@@ -236,8 +235,7 @@ def run_kvq(args):
         cache.reset()
         cache.prefill_quantize(XK, XV)
         for s in range(w.steps):
-            cache.append(tK[s], tV[s])
-            cache.decode_attention(tQ[s], out=out)
+            cache.append_decode(tK[s], tV[s], tQ[s], out=out)
 
     def barrier():
         if world > 1:
@@ -258,13 +256,20 @@ def run_kvq(args):
     g_pre = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_pre, pool=pool):
         cache.prefill_quantize(XK, XV)
+    # a step whose append flushes the residual gets its own append graph (the quantize is
+    # not part of the timed decode); every other step is one append_decode graph
     g_app, g_dec = [], []
     for s_ in range(w.steps):
-        ga, gd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(ga, pool=pool):
-            cache.append(tK[s_], tV[s_])
-        with torch.cuda.graph(gd, pool=pool):
-            cache.decode_attention(tQ[s_], out=out)
+        flush = cache.state()[1] + 1 == w.R
+        ga, gd = (torch.cuda.CUDAGraph() if flush else None), torch.cuda.CUDAGraph()
+        if flush:
+            with torch.cuda.graph(ga, pool=pool):
+                cache.append(tK[s_], tV[s_])
+            with torch.cuda.graph(gd, pool=pool):
+                cache.decode_attention(tQ[s_], out=out)
+        else:
+            with torch.cuda.graph(gd, pool=pool):
+                cache.append_decode(tK[s_], tV[s_], tQ[s_], out=out)
         g_app.append(ga)
         g_dec.append(gd)
     launches_per_episode = kvq.kernel_launches() - launches0
@@ -278,7 +283,8 @@ def run_kvq(args):
     def replay_episode(ev):
         g_pre.replay()
         for s_ in range(w.steps):
-            g_app[s_].replay()
+            if g_app[s_] is not None:
+                g_app[s_].replay()
             ev[s_][0].record(stream)
             g_dec[s_].replay()
             ev[s_][1].record(stream)
@@ -321,8 +327,7 @@ def run_kvq(args):
             cache.reset()
             cache.prefill_quantize(XKp, XVp)           # host -> device inside the call path
             for s in range(w.steps):
-                cache.append(tKp[s], tVp[s])
-                cache.decode_attention(tQp[s], out=outs[s])   # device -> host of t_O
+                cache.append_decode(tKp[s], tVp[s], tQp[s], out=outs[s])   # device -> host of t_O
         for _ in range(max(1, args.warmup)):
             e2e_episode()
         torch.cuda.synchronize()
@@ -390,7 +395,8 @@ def run_kvq(args):
         "decode_steps_per_s": w.steps * args.steps / (ms / 1e3),
         "kv_tokens_per_s_decode_only": job_throughput(tokens_per_episode * args.steps, world, decode_ms),
         "roofline": {
-            "kernel": f"decode_attention ({decode_kernel_name(w)}, splits merged in-kernel), per call",
+            "kernel": f"append + decode_attention ({decode_kernel_name(w)}: one launch without a flush, "
+                      "splits merged in-kernel), per call",
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
             if peak_kind == "measured" else "fallback 6.65 TB/s",

@@ -620,10 +620,12 @@ __host__ __device__ constexpr int residual_scratch_bytes() { return 2 * 16 * (2 
 // pending.  qh is the log2-scaled query in shared memory; acc[j][h] accumulates
 // channel 16j + g8 + 8h, x over tokens 4*t4 + {0, 1}, y over 4*t4 + {2, 3}.
 template <int D>
-__device__ __forceinline__ void residual_pass(const DecodeArgs &a, const float *qh, const uint16_t *kr,
-                                              const uint16_t *vr, int rt0, int rt1, int lane, float &m,
-                                              float &lsum, float2 (&acc)[D / 16][2], unsigned char *scratch,
-                                              int stride = 1) {
+__device__ __forceinline__ void residual_pass(const DecodeArgs &a, int64_t bh, const float *qh, int rt0, int rt1,
+                                              int lane, float &m, float &lsum, float2 (&acc)[D / 16][2],
+                                              unsigned char *scratch, int stride = 1) {
+    const uint16_t *kr = a.kr + bh * a.R * D, *vr = a.vr + bh * a.R * D;
+    // a fused append: row new_row is read from the new token itself
+    const uint16_t *nk = a.new_k ? a.new_k + bh * D : nullptr, *nv = a.new_v ? a.new_v + bh * D : nullptr;
     constexpr int NJ = D / 16;
     constexpr int kRow = 2 * D + 16;          // padded row stride in bytes
     constexpr int kPieces = 2 * D / 16;       // 16-byte pieces of one row
@@ -636,8 +638,9 @@ __device__ __forceinline__ void residual_pass(const DecodeArgs &a, const float *
         for (int c = lane; c < 2 * n; c += 32) {
             const bool isv = c >= n;
             const int cc = isv ? c - n : c, row = cc / kPieces, pc = cc % kPieces;
-            cp_async16((isv ? vs : ks) + row * kRow + 16 * pc,
-                       (isv ? vr : kr) + (static_cast<int64_t>(rt) * 16 + row) * D + 8 * pc);
+            const int gr = 16 * rt + row;
+            const uint16_t *src = (nk && gr == a.new_row) ? (isv ? nv : nk) : (isv ? vr : kr) + static_cast<int64_t>(gr) * D;
+            cp_async16((isv ? vs : ks) + row * kRow + 16 * pc, src + 8 * pc);
         }
         cp_async_commit();
         cp_async_wait<0>();
@@ -940,6 +943,16 @@ __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) deco
 
     for (int i = threadIdx.x; i < HG * D; i += kDecodeThreads)
         q_s[i / D][i % D] = widen(a.q[bq0 * D + i], a.bf16) * a.qscale;
+    // a fused append: split 0 stores the new token as residual row new_row, for later steps
+    // (every CTA of this call reads that row from the new token itself)
+    if (a.new_k && sigma == 0) {
+        for (int i = threadIdx.x; i < 2 * D / 8; i += kDecodeThreads) {
+            const bool isv = i >= D / 8;
+            const int c = isv ? i - D / 8 : i;
+            const uint4 val = reinterpret_cast<const uint4 *>((isv ? a.new_v : a.new_k) + bh * D)[c];
+            reinterpret_cast<uint4 *>((isv ? a.vr : a.kr) + (bh * a.R + a.new_row) * D)[c] = val;
+        }
+    }
     __syncthreads();
 
     float *o_s = reinterpret_cast<float *>(stage_mem);   // epilogue: [warp][HG][D]
@@ -953,8 +966,7 @@ __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) deco
             float2 acc[NJ][2];
 #pragma unroll
             for (int j = 0; j < NJ; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
-            residual_pass<D>(a, q_s[h], a.kr + bh * a.R * D, a.vr + bh * a.R * D, warp % WPH, (a.r + 15) / 16,
-                             lane, m, lsum, acc, wmem, WPH);
+            residual_pass<D>(a, bh, q_s[h], warp % WPH, (a.r + 15) / 16, lane, m, lsum, acc, wmem, WPH);
             lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
             lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
             lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
@@ -1201,8 +1213,7 @@ __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) deco
             float2 acc[NJ][2];
 #pragma unroll
             for (int j = 0; j < NJ; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
-            residual_pass<D>(a, q_s[0], a.kr + bh * a.R * D, a.vr + bh * a.R * D, gw, nres, lane, m_own, lr,
-                             acc, wmem, nw);
+            residual_pass<D>(a, bh, q_s[0], gw, nres, lane, m_own, lr, acc, wmem, nw);
             lr += __shfl_xor_sync(0xffffffffu, lr, 4);     // lanes hold rows g8, g8 + 8
             lr += __shfl_xor_sync(0xffffffffu, lr, 8);
             lr += __shfl_xor_sync(0xffffffffu, lr, 16);

@@ -182,8 +182,10 @@ kvq::DecodeArgs decode_args(const kvq_cache *h) {
     a.vs = h->buf.v_scales;
     a.kz = h->buf.k_zeros;
     a.vz = h->buf.v_zeros;
-    a.kr = static_cast<const uint16_t *>(h->buf.k_residual);
-    a.vr = static_cast<const uint16_t *>(h->buf.v_residual);
+    a.kr = static_cast<uint16_t *>(h->buf.k_residual);
+    a.vr = static_cast<uint16_t *>(h->buf.v_residual);
+    a.new_k = a.new_v = nullptr;
+    a.new_row = -1;
     a.cap = c.capacity;
     a.B = c.batch;
     a.Hq = c.q_heads;
@@ -223,6 +225,11 @@ kvq::QuantizeArgs quantize_args(const kvq_cache *h) {
     q.cap = c.capacity;
     return q;
 }
+
+kvq_status check_decode_args(const kvq_cache *h, const void *t_Q, const float *t_O, const void *workspace,
+                             size_t workspace_bytes);
+kvq_status launch_decode_call(kvq_cache *h, const void *t_Q, float *t_O, void *workspace,
+                              const uint16_t *new_k, const uint16_t *new_v, void *stream);
 
 }  // namespace
 
@@ -392,15 +399,56 @@ int32_t kvq_decode_splits(const kvq_cache *h) {
 kvq_status kvq_decode_attention(kvq_cache *h, const void *t_Q, float *t_O, void *workspace,
                                 size_t workspace_bytes, void *stream) {
     if (!h) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+    kvq_status st = check_decode_args(h, t_Q, t_O, workspace, workspace_bytes);
+    if (st != KVQ_OK) return st;
+    if (h->Tq == 0 && h->r == 0) return fail(KVQ_ERR_STATE, "the cache is empty");
+    return launch_decode_call(h, t_Q, t_O, workspace, nullptr, nullptr, stream);
+}
+
+kvq_status kvq_append_decode_attention(kvq_cache *h, const void *t_K, const void *t_V, const void *t_Q,
+                                       float *t_O, void *workspace, size_t workspace_bytes, void *stream) {
+    if (!h) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+    if (!t_K || !t_V || !aligned16(t_K) || !aligned16(t_V))
+        return fail(KVQ_ERR_INVALID_ARG, "t_K and t_V must be non-NULL and 16-byte aligned");
+    kvq_status st = check_decode_args(h, t_Q, t_O, workspace, workspace_bytes);
+    if (st != KVQ_OK) return st;
+    const kvq_config &c = h->cfg;
+    const bool flush = h->r + 1 == c.residual;
+    if (flush || kvq::decode_path(c.q_heads, c.kv_heads, c.group_k) != kvq::kPathTc) {
+        // a flush (or the CUDA-core kernel): the append's own launches, then the decode
+        st = kvq_append(h, t_K, t_V, stream);
+        if (st != KVQ_OK) return st;
+        return launch_decode_call(h, t_Q, t_O, workspace, nullptr, nullptr, stream);
+    }
+    // one kernel: the new token is read as residual row r and stored there by split 0
+    h->r += 1;
+    st = launch_decode_call(h, t_Q, t_O, workspace, static_cast<const uint16_t *>(t_K),
+                            static_cast<const uint16_t *>(t_V), stream);
+    if (st != KVQ_OK) h->r -= 1;
+    return st;
+}
+
+}  // extern "C"
+
+namespace {
+
+kvq_status check_decode_args(const kvq_cache *h, const void *t_Q, const float *t_O, const void *workspace,
+                             size_t workspace_bytes) {
     if (!t_Q || !t_O || !workspace || !aligned16(t_Q) || !aligned16(t_O) || !aligned16(workspace))
         return fail(KVQ_ERR_INVALID_ARG, "t_Q, t_O and workspace must be non-NULL and 16-byte aligned");
-    if (h->Tq == 0 && h->r == 0) return fail(KVQ_ERR_STATE, "the cache is empty");
-    const kvq_config &c = h->cfg;
     kvq_sizes sz;
-    kvq_get_sizes(&c, &sz);
+    kvq_get_sizes(&h->cfg, &sz);
     if (workspace_bytes < sz.workspace)
         return fail(KVQ_ERR_INVALID_ARG, "workspace needs %zu bytes, got %zu", sz.workspace,
                     workspace_bytes);
+    return KVQ_OK;
+}
+
+// Launches one decode over the current state; new_k / new_v (or NULL): residual row r - 1
+// is that token, read from it and stored by the kernel.
+kvq_status launch_decode_call(kvq_cache *h, const void *t_Q, float *t_O, void *workspace,
+                              const uint16_t *new_k, const uint16_t *new_v, void *stream) {
+    const kvq_config &c = h->cfg;
     kvq::DecodeArgs a = decode_args(h);
     plan_splits(h, &a.n_qsplits, &a.tiles_per_split, &a.S);
     const int64_t units = static_cast<int64_t>(c.batch) * c.q_heads;
@@ -412,12 +460,15 @@ kvq_status kvq_decode_attention(kvq_cache *h, const void *t_Q, float *t_O, void 
     a.out = t_O;
     a.n_qtiles = static_cast<int>(h->Tq / 16);
     a.r = h->r;
+    a.new_k = new_k;
+    a.new_v = new_v;
+    a.new_row = new_k ? h->r - 1 : -1;
     cudaError_t e = kvq::launch_decode(a, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
     return ok();
 }
 
-}  // extern "C"
+}  // namespace
 
 // ---------------------------------------------------------------------------
 // Decode attention without a caller-provided workspace.

@@ -72,7 +72,9 @@ struct DecodeArgs {
     const uint32_t *kc, *vc;
     const float *ks, *vs;
     const int16_t *kz, *vz;
-    const uint16_t *kr, *vr;     // residual [BH][R][d]
+    uint16_t *kr, *vr;           // residual [BH][R][d]
+    const uint16_t *new_k, *new_v;   // fused append: the new token [BH][d] (row new_row), else NULL
+    int new_row;
     const uint16_t *q;           // [B][Hq][d]
     float *o_part, *m_part, *l_part;   // [B*Hq][S][d], [B*Hq][S], [B*Hq][S]
     float *out;                  // [B][Hq][d]

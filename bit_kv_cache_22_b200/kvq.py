@@ -30,7 +30,7 @@ KVQ_FP16, KVQ_BF16 = 0, 1
 EXPORTED = ("kvq_get_sizes", "kvq_create", "kvq_destroy", "kvq_reset", "kvq_prefill_quantize",
             "kvq_append", "kvq_decode_attention", "kvq_cache_state", "kvq_set_split_limit",
             "kvq_decode_splits", "kvq_kernel_launches", "kvq_decode_attention_noalloc",
-            "kvq_last_error", "kvq_layout_version", "kvq_check_device")
+            "kvq_last_error", "kvq_layout_version", "kvq_check_device", "kvq_append_decode_attention")
 
 
 class KVQError(RuntimeError):
@@ -84,6 +84,8 @@ def load() -> ctypes.CDLL:
         lib.kvq_prefill_quantize.argtypes = [P, P, P, i64, P]
         lib.kvq_append.argtypes = [P, P, P, P]
         lib.kvq_decode_attention.argtypes = [P, P, P, P, sz, P]
+        lib.kvq_append_decode_attention.argtypes = [P, P, P, P, P, P, sz, P]
+        lib.kvq_append_decode_attention.restype = ctypes.c_int
         lib.kvq_decode_attention_noalloc.argtypes = [P, P, P, P]
         lib.kvq_decode_attention_noalloc.restype = ctypes.c_int
         lib.kvq_cache_state.argtypes = [P, ctypes.POINTER(i64), ctypes.POINTER(i32)]
@@ -249,6 +251,29 @@ class KVQCache:
         _check(self._lib.kvq_decode_attention(self._h, t_Q.data_ptr(), dev_out.data_ptr(),
                                               self.workspace.data_ptr(),
                                               self.workspace.numel() * 4, _stream_ptr(stream)))
+        if host_out:
+            out.copy_(dev_out, non_blocking=True)
+            return out
+        return dev_out
+
+    def append_decode(self, t_K: torch.Tensor, t_V: torch.Tensor, t_Q: torch.Tensor,
+                      out: torch.Tensor | None = None, stream=None):
+        """append(t_K, t_V) then decode_attention(t_Q), in one call (one kernel when possible)."""
+        t_K, t_V, t_Q = self._dev(t_K), self._dev(t_V), self._dev(t_Q)
+        c = self.cfg
+        want = (c.batch, c.kv_heads, c.head_dim)
+        if tuple(t_K.shape) != want or tuple(t_V.shape) != want:
+            raise ValueError(f"t_K/t_V must be {list(want)}")
+        if tuple(t_Q.shape) != (c.batch, c.q_heads, c.head_dim):
+            raise ValueError(f"t_Q must be [{c.batch}, {c.q_heads}, {c.head_dim}]")
+        host_out = out is not None and not out.is_cuda
+        dev_out = torch.empty((c.batch, c.q_heads, c.head_dim), dtype=torch.float32,
+                              device=self.device) if (out is None or host_out) else out
+        _check(self._lib.kvq_append_decode_attention(self._h, t_K.data_ptr(), t_V.data_ptr(),
+                                                     t_Q.data_ptr(), dev_out.data_ptr(),
+                                                     self.workspace.data_ptr(),
+                                                     self.workspace.numel() * 4, _stream_ptr(stream)))
+        self._keep = (t_K, t_V)
         if host_out:
             out.copy_(dev_out, non_blocking=True)
             return out

@@ -173,6 +173,21 @@ KVQ_API kvq_status kvq_decode_attention(kvq_cache *cache, const void *t_Q, float
                                 void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * kvq_append(t_K, t_V) followed by kvq_decode_attention(t_Q -> t_O), in one call
+ * (KIVI section 1: each decode step appends its token, then attends over
+ * [deq(K_g); K_r] including it).  Same arguments, state change and result as the
+ * two calls.  On the tensor-core path (1, 2 or 4 query heads per kv head, key
+ * groups of >= 32 tokens), when the append does not flush, it is one kernel
+ * launch: the decode reads the new token straight from t_K / t_V as residual
+ * row r and stores it there for later steps.  Otherwise it makes the two calls'
+ * launches.  Errors as for the two calls; arguments are checked before
+ * anything is launched or changed.
+ */
+KVQ_API kvq_status kvq_append_decode_attention(kvq_cache *cache, const void *t_K, const void *t_V,
+                                               const void *t_Q, float *t_O, void *workspace,
+                                               size_t workspace_bytes, void *stream);
+
+/*
  * Decode attention that allocates nothing and takes no workspace (the pages
  * have no counterpart: this is an interface for callers that cannot allocate
  * device memory -- for instance code that runs while another framework owns

@@ -93,6 +93,8 @@ def test_null_arguments_are_rejected_without_a_device():
     assert lib.kvq_decode_attention(None, None, None, None, 0, None) == kvq.KVQ_ERR_INVALID_ARG
     assert lib.kvq_decode_splits(None) == 0
     assert lib.kvq_check_device(None) == kvq.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_append_decode_attention(None, None, None, None, None, None, 0, None) == \
+        kvq.KVQ_ERR_INVALID_ARG
     lib.kvq_destroy(None)
     h = ctypes.c_void_p()
     cfg = _cfg()

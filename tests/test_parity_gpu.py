@@ -92,6 +92,35 @@ def test_every_decode_path(g, d, bits, G, Gv, R):
     run_episode(w, check_every=7)
 
 
+@pytest.mark.parametrize("name", ["llama7b", "gqa8b", "tiny", "stream4sym"])
+def test_fused_append_decode_equals_separate_calls(name):
+    """append_decode gives the same state, codes and (bit for bit) outputs as append followed
+    by decode_attention, through flushes; and matches the oracle."""
+    base = wl.WORKLOADS[name]
+    w = base if name == "tiny" else reduced(base).replace(steps=base.R + 6)
+    XK, XV = wl.prefill_bits(w)
+    tK, tV, tQ = wl.decode_bits(w)
+    a, b = tl.new_cache(w), tl.new_cache(w)
+    ref = tl.new_oracle(w)
+    a.prefill_quantize(tl.to_dev(XK, w), tl.to_dev(XV, w))
+    b.prefill_quantize(tl.to_dev(XK, w), tl.to_dev(XV, w))
+    ref.prefill(XK, XV)
+    for s in range(w.steps):
+        ka, va, q = tl.to_dev(tK[s], w), tl.to_dev(tV[s], w), tl.to_dev(tQ[s], w)
+        a.append(ka, va)
+        oa = a.decode_attention(q)
+        ob = b.append_decode(ka, va, q)
+        ref.append(tK[s], tV[s])
+        assert a.state() == b.state() == (ref.Tq, ref.r)
+        assert torch.equal(oa, ob), f"step {s}"
+        if s % 9 == 0 or s == w.steps - 1:
+            tl.assert_close(ob.cpu().numpy(), ref.decode(tQ[s]), f"{name} step {s}")
+    Tq, r = b.state()
+    tl.assert_codes_equal(tl.gpu_packed(b, Tq), ref.packed(), w.symmetric)
+    assert torch.equal(a.k_residual[:, :r], b.k_residual[:, :r])
+    assert torch.equal(a.v_residual[:, :r], b.v_residual[:, :r])
+
+
 def test_device_status_stays_clear():
     """No bounded wait gives up in a normal decode; the status read succeeds and clears."""
     w = reduced(wl.WORKLOADS["gqa8b"]).replace(steps=2)
