@@ -237,7 +237,15 @@ __device__ __forceinline__ void finish_cta(const DecodeArgs &a, const float *o_w
         }
         const int64_t bq = bq0 + hh;
         if (a.S == 1) {
-            a.out[bq * D + c] = o / l;
+            if (a.po) {   // the cache's partial (token-split decode)
+                a.po[bq * D + c] = o;
+                if (c == 0) {
+                    a.pm[bq] = M;
+                    a.pl[bq] = l;
+                }
+            } else {
+                a.out[bq * D + c] = o / l;
+            }
             continue;
         }
         a.o_part[(bq * a.S + sigma) * D + c] = o;
@@ -281,7 +289,17 @@ __device__ __forceinline__ void finish_cta(const DecodeArgs &a, const float *o_w
         float o = 0.f;
 #pragma unroll 8
         for (int s = 0; s < a.S; ++s) o = fmaf(__ldcg(op + static_cast<int64_t>(s) * D), wp[s], o);
-        a.out[(bq0 + hh) * D + c] = o / wts[HG * a.S + hh];
+        if (a.po) {   // the cache's partial (token-split decode): o and l relative to M
+            a.po[(bq0 + hh) * D + c] = o;
+            if (c == 0) {
+                float M = -INFINITY;
+                for (int s = 0; s < a.S; ++s) M = fmaxf(M, __ldcg(a.m_part + (bq0 + hh) * a.S + s));
+                a.pm[bq0 + hh] = M;
+                a.pl[bq0 + hh] = wts[HG * a.S + hh];
+            }
+        } else {
+            a.out[(bq0 + hh) * D + c] = o / wts[HG * a.S + hh];
+        }
     }
     if (threadIdx.x == 0) a.arrivals[unit] = 0u;
 }
@@ -1557,7 +1575,38 @@ int occ_gv(const DecodeArgs &a) {
     return 1;
 }
 
+// Token-split decode: t_O row = sum_k o_k 2^(m_k - M) / sum_k l_k 2^(m_k - M), M = max_k m_k,
+// over n partials of caches holding disjoint tokens (o_all [n][rows][d], m_all and l_all
+// [n][rows]); a partial with m = -inf (no tokens) has weight 0.  One CTA per row.
+__global__ void merge_partials_kernel(const float *o_all, const float *m_all, const float *l_all, int n,
+                                      int64_t rows, int d, float *out) {
+    const int64_t row = blockIdx.x;
+    float M = -INFINITY;
+    for (int k = 0; k < n; ++k) M = fmaxf(M, m_all[k * rows + row]);
+    float L = 0.f;
+    for (int k = 0; k < n; ++k) {
+        const float mk = m_all[k * rows + row];
+        if (mk != -INFINITY) L = fmaf(l_all[k * rows + row], exp2f(mk - M), L);
+    }
+    for (int c = threadIdx.x; c < d; c += blockDim.x) {
+        float o = 0.f;
+        for (int k = 0; k < n; ++k) {
+            const float mk = m_all[k * rows + row];
+            if (mk != -INFINITY) o = fmaf(o_all[(k * rows + row) * d + c], exp2f(mk - M), o);
+        }
+        out[row * d + c] = o / L;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_merge_partials(const float *o_all, const float *m_all, const float *l_all, int n,
+                                  int64_t rows, int d, float *out, cudaStream_t s) {
+    if (rows == 0) return cudaSuccess;
+    merge_partials_kernel<<<static_cast<unsigned>(rows), 128, 0, s>>>(o_all, m_all, l_all, n, rows, d, out);
+    count_launches(1);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
     cudaError_t e = cudaErrorInvalidValue;

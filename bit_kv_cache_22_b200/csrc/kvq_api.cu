@@ -229,7 +229,8 @@ kvq::QuantizeArgs quantize_args(const kvq_cache *h) {
 kvq_status check_decode_args(const kvq_cache *h, const void *t_Q, const float *t_O, const void *workspace,
                              size_t workspace_bytes);
 kvq_status launch_decode_call(kvq_cache *h, const void *t_Q, float *t_O, void *workspace,
-                              const uint16_t *new_k, const uint16_t *new_v, void *stream);
+                              const uint16_t *new_k, const uint16_t *new_v, void *stream,
+                              float *po = nullptr, float *pm = nullptr, float *pl = nullptr);
 
 }  // namespace
 
@@ -428,6 +429,29 @@ kvq_status kvq_append_decode_attention(kvq_cache *h, const void *t_K, const void
     return st;
 }
 
+kvq_status kvq_decode_attention_partial(kvq_cache *h, const void *t_Q, float *o_part, float *m_part,
+                                        float *l_part, void *workspace, size_t workspace_bytes, void *stream) {
+    if (!h) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+    if (!m_part || !l_part || !aligned16(m_part) || !aligned16(l_part))
+        return fail(KVQ_ERR_INVALID_ARG, "m_part and l_part must be non-NULL and 16-byte aligned");
+    kvq_status st = check_decode_args(h, t_Q, o_part, workspace, workspace_bytes);
+    if (st != KVQ_OK) return st;
+    if (h->Tq == 0 && h->r == 0) return fail(KVQ_ERR_STATE, "the cache is empty");
+    return launch_decode_call(h, t_Q, nullptr, workspace, nullptr, nullptr, stream, o_part, m_part, l_part);
+}
+
+kvq_status kvq_merge_partials(const float *o_parts, const float *m_parts, const float *l_parts, int32_t n,
+                              int64_t rows, int32_t d, float *t_O, void *stream) {
+    if (n < 1 || rows < 0 || d < 1) return fail(KVQ_ERR_INVALID_ARG, "n, rows and d must be >= 1, >= 0, >= 1");
+    if (rows > 0 && (!o_parts || !m_parts || !l_parts || !t_O))
+        return fail(KVQ_ERR_INVALID_ARG, "partials and t_O must be non-NULL");
+    if (rows > 0x7fffffffLL) return fail(KVQ_ERR_UNSUPPORTED, "rows must be < 2^31");
+    cudaError_t e = kvq::launch_merge_partials(o_parts, m_parts, l_parts, n, rows, d, t_O,
+                                               static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+    return ok();
+}
+
 }  // extern "C"
 
 namespace {
@@ -445,9 +469,11 @@ kvq_status check_decode_args(const kvq_cache *h, const void *t_Q, const float *t
 }
 
 // Launches one decode over the current state; new_k / new_v (or NULL): residual row r - 1
-// is that token, read from it and stored by the kernel.
+// is that token, read from it and stored by the kernel; po / pm / pl (or NULL): write the
+// cache's partial there instead of t_O.
 kvq_status launch_decode_call(kvq_cache *h, const void *t_Q, float *t_O, void *workspace,
-                              const uint16_t *new_k, const uint16_t *new_v, void *stream) {
+                              const uint16_t *new_k, const uint16_t *new_v, void *stream, float *po,
+                              float *pm, float *pl) {
     const kvq_config &c = h->cfg;
     kvq::DecodeArgs a = decode_args(h);
     plan_splits(h, &a.n_qsplits, &a.tiles_per_split, &a.S);
@@ -463,6 +489,9 @@ kvq_status launch_decode_call(kvq_cache *h, const void *t_Q, float *t_O, void *w
     a.new_k = new_k;
     a.new_v = new_v;
     a.new_row = new_k ? h->r - 1 : -1;
+    a.po = po;
+    a.pm = pm;
+    a.pl = pl;
     cudaError_t e = kvq::launch_decode(a, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
     return ok();

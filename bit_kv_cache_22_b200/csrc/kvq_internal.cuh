@@ -78,6 +78,8 @@ struct DecodeArgs {
     const uint16_t *q;           // [B][Hq][d]
     float *o_part, *m_part, *l_part;   // [B*Hq][S][d], [B*Hq][S], [B*Hq][S]
     float *out;                  // [B][Hq][d]
+    float *po, *pm, *pl;         // instead of out (token-split decode): o [B][Hq][d] and m, l [B][Hq]
+                                 // of the whole cache, o and l relative to m (log2 units); else NULL
     unsigned int *arrivals;      // [B*Hq] split-arrival counters, zero between calls
     unsigned int *status;        // nonzero once a bounded wait inside a decode kernel gave up
     int64_t cap;
@@ -93,6 +95,9 @@ struct DecodeArgs {
     float qscale;                // log2(e) / sqrt(d)
 };
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+// t_O [rows][d] from n partials o_all [n][rows][d], m_all / l_all [n][rows] (log2 units).
+cudaError_t launch_merge_partials(const float *o_all, const float *m_all, const float *l_all, int n,
+                                  int64_t rows, int d, float *out, cudaStream_t s);
 // CTAs of the split kernel that fit on one SM for this configuration.
 int decode_ctas_per_sm(const DecodeArgs &a);
 

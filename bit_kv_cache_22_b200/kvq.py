@@ -30,7 +30,8 @@ KVQ_FP16, KVQ_BF16 = 0, 1
 EXPORTED = ("kvq_get_sizes", "kvq_create", "kvq_destroy", "kvq_reset", "kvq_prefill_quantize",
             "kvq_append", "kvq_decode_attention", "kvq_cache_state", "kvq_set_split_limit",
             "kvq_decode_splits", "kvq_kernel_launches", "kvq_decode_attention_noalloc",
-            "kvq_last_error", "kvq_layout_version", "kvq_check_device", "kvq_append_decode_attention")
+            "kvq_last_error", "kvq_layout_version", "kvq_check_device", "kvq_append_decode_attention",
+            "kvq_decode_attention_partial", "kvq_merge_partials")
 
 
 class KVQError(RuntimeError):
@@ -86,6 +87,10 @@ def load() -> ctypes.CDLL:
         lib.kvq_decode_attention.argtypes = [P, P, P, P, sz, P]
         lib.kvq_append_decode_attention.argtypes = [P, P, P, P, P, P, sz, P]
         lib.kvq_append_decode_attention.restype = ctypes.c_int
+        lib.kvq_decode_attention_partial.argtypes = [P, P, P, P, P, P, sz, P]
+        lib.kvq_decode_attention_partial.restype = ctypes.c_int
+        lib.kvq_merge_partials.argtypes = [P, P, P, i32, i64, i32, P, P]
+        lib.kvq_merge_partials.restype = ctypes.c_int
         lib.kvq_decode_attention_noalloc.argtypes = [P, P, P, P]
         lib.kvq_decode_attention_noalloc.restype = ctypes.c_int
         lib.kvq_cache_state.argtypes = [P, ctypes.POINTER(i64), ctypes.POINTER(i32)]
@@ -256,6 +261,21 @@ class KVQCache:
             return out
         return dev_out
 
+    def decode_attention_partial(self, t_Q: torch.Tensor, stream=None):
+        """This cache's unnormalised partial (o [B, Hq, d], m [B, Hq], l [B, Hq]; base-2
+        logits) for a token-split decode; merge with merge_partials."""
+        t_Q = self._dev(t_Q)
+        c = self.cfg
+        if tuple(t_Q.shape) != (c.batch, c.q_heads, c.head_dim):
+            raise ValueError(f"t_Q must be [{c.batch}, {c.q_heads}, {c.head_dim}]")
+        o = torch.empty((c.batch, c.q_heads, c.head_dim), dtype=torch.float32, device=self.device)
+        m = torch.empty((c.batch, c.q_heads), dtype=torch.float32, device=self.device)
+        l = torch.empty((c.batch, c.q_heads), dtype=torch.float32, device=self.device)
+        _check(self._lib.kvq_decode_attention_partial(self._h, t_Q.data_ptr(), o.data_ptr(), m.data_ptr(),
+                                                      l.data_ptr(), self.workspace.data_ptr(),
+                                                      self.workspace.numel() * 4, _stream_ptr(stream)))
+        return o, m, l
+
     def append_decode(self, t_K: torch.Tensor, t_V: torch.Tensor, t_Q: torch.Tensor,
                       out: torch.Tensor | None = None, stream=None):
         """append(t_K, t_V) then decode_attention(t_Q), in one call (one kernel when possible)."""
@@ -303,6 +323,22 @@ def append(cache: KVQCache, t_K: torch.Tensor, t_V: torch.Tensor) -> KVQCache:
 
 def decode_attention(cache: KVQCache, t_Q: torch.Tensor, out=None) -> torch.Tensor:
     return cache.decode_attention(t_Q, out)
+
+
+def merge_partials(o_all: torch.Tensor, m_all: torch.Tensor, l_all: torch.Tensor,
+                   out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Merge n partials (o [n, *rows, d], m and l [n, *rows], float32, one CUDA device) of caches
+    holding disjoint tokens into the output [*rows, d]."""
+    if not (o_all.is_cuda and m_all.is_cuda and l_all.is_cuda):
+        raise ValueError("partials must be CUDA tensors")
+    n, d = o_all.shape[0], o_all.shape[-1]
+    rows = m_all[0].numel()
+    o_all, m_all, l_all = o_all.contiguous(), m_all.contiguous(), l_all.contiguous()
+    if out is None:
+        out = torch.empty(o_all.shape[1:], dtype=torch.float32, device=o_all.device)
+    _check(load().kvq_merge_partials(o_all.data_ptr(), m_all.data_ptr(), l_all.data_ptr(), n, rows, d,
+                                     out.data_ptr(), _stream_ptr(stream)))
+    return out
 
 
 def kernel_launches() -> int:

@@ -188,6 +188,32 @@ KVQ_API kvq_status kvq_append_decode_attention(kvq_cache *cache, const void *t_K
                                                size_t workspace_bytes, void *stream);
 
 /*
+ * Token-split decode (several caches holding disjoint tokens of the same
+ * sequences, e.g. one per GPU; the order of a concatenation does not matter,
+ * "Resumo Técnico: LogQuant", section 4).  Like kvq_decode_attention, but
+ * instead of t_O it writes this cache's unnormalised partial:
+ *   m_part [B][Hq]     = max_t y_t over this cache's tokens,
+ *   l_part [B][Hq]     = sum_t 2^(y_t - m),
+ *   o_part [B][Hq][d]  = sum_t 2^(y_t - m) v_t,
+ * with y_t = log2(e) q.k_t / sqrt(d) (base-2 logits).  All float, 16-byte
+ * aligned, caller-owned.  An empty cache gives KVQ_ERR_STATE (its partial would
+ * be m = -inf, l = 0, o = 0).  The pages have no counterpart for the split.
+ */
+KVQ_API kvq_status kvq_decode_attention_partial(kvq_cache *cache, const void *t_Q, float *o_part,
+                                                float *m_part, float *l_part, void *workspace,
+                                                size_t workspace_bytes, void *stream);
+
+/*
+ * Merges n partials of kvq_decode_attention_partial (from caches holding
+ * disjoint tokens of the same rows): o_parts [n][rows][d], m_parts and l_parts
+ * [n][rows], device, contiguous -> t_O [rows][d] =
+ * sum_k 2^(m_k - M) o_k / sum_k 2^(m_k - M) l_k with M = max_k m_k (partials
+ * with m = -inf count for nothing).  rows = B * Hq.  One kernel launch.
+ */
+KVQ_API kvq_status kvq_merge_partials(const float *o_parts, const float *m_parts, const float *l_parts,
+                                      int32_t n, int64_t rows, int32_t d, float *t_O, void *stream);
+
+/*
  * Decode attention that allocates nothing and takes no workspace (the pages
  * have no counterpart: this is an interface for callers that cannot allocate
  * device memory -- for instance code that runs while another framework owns

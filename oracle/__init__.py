@@ -77,7 +77,7 @@ def _load():
         lib.oracle_dequant.argtypes = [i32, ctypes.c_float, ctypes.c_int32]
         lib.oracle_decode_attention.restype = i32
         lib.oracle_decode_attention.argtypes = [P, P, P, P, P, P, i64, P, P, i64, i64, P,
-                                                i32, i64, i32, i32, i32, i32, i32, i32, i32, P]
+                                                i32, i64, i32, i32, i32, i32, i32, i32, i32, P, P, P]
         lib.oracle_num_threads.restype = i32
         lib.oracle_num_threads.argtypes = []
         _lib = lib
@@ -197,20 +197,37 @@ def unpack(words: np.ndarray, T: int, d: int, bits: int, is_v: bool) -> np.ndarr
 
 def decode_attention(qcache: dict, Tq: int, Kr: np.ndarray, Vr: np.ndarray, r: int,
                      Q: np.ndarray, dtype: int, B: int, Hq: int, Hkv: int, d: int,
-                     G: int, Gv: int, bits: int, symmetric: bool) -> np.ndarray:
-    """fp64 decode attention of queries Q [B, Hq, d] over [deq(quantized); residual]."""
+                     G: int, Gv: int, bits: int, symmetric: bool, stats: bool = False):
+    """fp64 decode attention of queries Q [B, Hq, d] over [deq(quantized); residual].
+
+    With stats=True also returns the softmax statistics (m, l) [B, Hq]: m the
+    largest scaled logit, l = sum_t exp(logit_t - m)."""
     lib = _load()
     Q = np.ascontiguousarray(Q, dtype=np.uint16)
     Kr = np.ascontiguousarray(Kr, dtype=np.uint16)
     Vr = np.ascontiguousarray(Vr, dtype=np.uint16)
     Rcap = Kr.shape[1]
     out = np.zeros((B, Hq, d), np.float64)
+    m = np.zeros((B, Hq), np.float64)
+    l = np.zeros((B, Hq), np.float64)
     arrs = [np.ascontiguousarray(qcache[k]) for k in ("Kq", "Ks", "Kz", "Vq", "Vs", "Vz")]
     rc = lib.oracle_decode_attention(*[_ptr(a) for a in arrs], Tq, _ptr(Kr), _ptr(Vr), Rcap, r,
                                      _ptr(Q), dtype, B, Hq, Hkv, d, G, Gv, bits,
-                                     int(symmetric), _ptr(out))
+                                     int(symmetric), _ptr(out), _ptr(m), _ptr(l))
     _check(rc, "decode_attention")
-    return out
+    return (out, m, l) if stats else out
+
+
+def merge_partials(outs, ms, ls) -> np.ndarray:
+    """Output over the union of disjoint token sets from each set's (normalised) output and
+    softmax statistics: sum_k w_k out_k / sum_k w_k with w_k = l_k exp(m_k - M), M = max_k m_k
+    (log-sum-exp; the token order of a concatenation does not matter, LogQuant summary,
+    section 4)."""
+    ms = np.stack(ms)
+    M = ms.max(axis=0)
+    w = np.stack(ls) * np.exp(ms - M)
+    num = sum(w[k][..., None] * outs[k] for k in range(len(outs)))
+    return num / w.sum(axis=0)[..., None]
 
 
 # ----------------------------------------------------------------------------
@@ -293,8 +310,8 @@ class OracleCache:
         return dict(Kc=pack(qc["Kq"], self.bits, False), Vc=pack(qc["Vq"], self.bits, True),
                     Ks=qc["Ks"], Kz=qc["Kz"], Vs=qc["Vs"], Vz=qc["Vz"])
 
-    def decode(self, Q: np.ndarray) -> np.ndarray:
-        """Q element bits [B, Hq, d] -> fp64 output [B, Hq, d]."""
+    def decode(self, Q: np.ndarray, stats: bool = False):
+        """Q element bits [B, Hq, d] -> fp64 output [B, Hq, d] (and (m, l) with stats=True)."""
         return decode_attention(self.quantized(), self.Tq, self.Kr, self.Vr, self.r, Q,
                                 self.dtype, self.B, self.Hq, self.Hkv, self.d, self.G,
-                                self.Gv, self.bits, self.symmetric)
+                                self.Gv, self.bits, self.symmetric, stats)

@@ -361,13 +361,18 @@ double oracle_dequant(int code, float s, int32_t z)
  *   Vs, Vz  [B*Hkv][Tq][d/Gv];      Kr, Vr element bits [B*Hkv][Rcap][d]
  *   (first r rows valid);  Q element bits [B][Hq][d];  out [B][Hq][d].
  *   Symmetric mode: Kz/Vz ignored, z = 2^(n-1).
+ *   max_out, denom_out [B][Hq] (each may be NULL): the largest scaled logit m
+ *   and sum_t exp(logit_t - m), the statistics with which outputs over
+ *   disjoint token sets merge into the output over their union (the order-free
+ *   concatenation of the LogQuant summary, section 4).
  */
 int oracle_decode_attention(const uint8_t *Kq, const float *Ks, const int16_t *Kz,
                             const uint8_t *Vq, const float *Vs, const int16_t *Vz,
                             int64_t Tq, const uint16_t *Kr, const uint16_t *Vr,
                             int64_t Rcap, int64_t r, const uint16_t *Q,
                             int dtype, int64_t B, int Hq, int Hkv, int d, int G,
-                            int Gv, int bits, int symmetric, double *out)
+                            int Gv, int bits, int symmetric, double *out,
+                            double *max_out, double *denom_out)
 {
     if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || d <= 0) return ORACLE_EINVAL;
     if (Tq < 0 || r < 0 || r > Rcap || (Tq > 0 && (Tq % G != 0 || d % Gv != 0)))
@@ -438,6 +443,9 @@ int oracle_decode_attention(const uint8_t *Kq, const float *Ks, const int16_t *K
                        (double)oracle_widen(Vr[(bh * Rcap + t) * d + c], dtype);
             out[(b * Hq + i) * d + c] = acc / denom;
         }
+        /* the softmax statistics, for merging with other token sets (max_out, denom_out may be NULL) */
+        if (max_out) max_out[b * Hq + i] = mx;
+        if (denom_out) denom_out[b * Hq + i] = denom;
         free(q);
         free(logit);
     }

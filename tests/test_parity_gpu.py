@@ -285,3 +285,56 @@ def _full_size(name, samples):
 def test_full_size_workload_sampled(name):
     w = wl.WORKLOADS[name]
     _full_size(name, [(0, 0), (w.B - 1, w.Hkv - 1)])
+
+
+@pytest.mark.parametrize("name,world", [("llama7b", 2), ("gqa8b", 2), ("tiny", 3)])
+def test_token_split_partials_merge_to_the_full_decode(name, world):
+    """Shard caches of one prompt (token_split.shard_bounds; the last takes the appends):
+    their partials merged by kvq_merge_partials equal the single-cache decode and the oracle."""
+    from bit_kv_cache_22_b200 import token_split
+    base = wl.WORKLOADS[name]
+    w = base.replace(T=3 * base.R + 40, steps=9) if name == "tiny" else \
+        reduced(base).replace(T=3 * base.R + 40, steps=9)
+    XK, XV = wl.prefill_bits(w)
+    tK, tV, tQ = wl.decode_bits(w)
+    full = tl.new_cache(w)
+    full.prefill_quantize(tl.to_dev(XK, w), tl.to_dev(XV, w))
+    shards = []
+    for k, (lo, hi) in enumerate(token_split.shard_bounds(w.T, world, w.R)):
+        last = k == world - 1
+        cap = max(w.R, -(-((hi - lo) + (w.steps if last else 0)) // w.R) * w.R)
+        c = tl.new_cache(w, capacity=cap)
+        if hi > lo:
+            c.prefill_quantize(tl.to_dev(np.ascontiguousarray(XK[:, :, lo:hi]), w),
+                               tl.to_dev(np.ascontiguousarray(XV[:, :, lo:hi]), w))
+        shards.append(c)
+    ref = tl.new_oracle(w)
+    ref.prefill(XK, XV)
+    for s in range(w.steps):
+        kk, vv, q = tl.to_dev(tK[s], w), tl.to_dev(tV[s], w), tl.to_dev(tQ[s], w)
+        full.append(kk, vv)
+        shards[-1].append(kk, vv)
+        ref.append(tK[s], tV[s])
+        parts = [c.decode_attention_partial(q) for c in shards if c.state() != (0, 0)]
+        got = kvq.merge_partials(torch.stack([p[0] for p in parts]), torch.stack([p[1] for p in parts]),
+                                 torch.stack([p[2] for p in parts]))
+        want = full.decode_attention(q)
+        torch.testing.assert_close(got, want, rtol=1e-4, atol=1e-5)
+        if s % 4 == 0:
+            tl.assert_close(got.cpu().numpy(), ref.decode(tQ[s]), f"{name} token split step {s}")
+
+
+def test_merge_partials_of_one_and_of_an_empty_partial():
+    w = reduced(wl.WORKLOADS["gqa8b"]).replace(steps=1)
+    XK, XV = wl.prefill_bits(w)
+    _, _, tQ = wl.decode_bits(w)
+    c = tl.new_cache(w)
+    c.prefill_quantize(tl.to_dev(XK, w), tl.to_dev(XV, w))
+    q = tl.to_dev(tQ[0], w)
+    o, m, l = c.decode_attention_partial(q)
+    want = c.decode_attention(q)
+    one = kvq.merge_partials(o[None], m[None], l[None])
+    torch.testing.assert_close(one, want, rtol=1e-6, atol=1e-7)
+    empty = (torch.zeros_like(o), torch.full_like(m, float("-inf")), torch.zeros_like(l))
+    two = kvq.merge_partials(torch.stack([empty[0], o]), torch.stack([empty[1], m]), torch.stack([empty[2], l]))
+    torch.testing.assert_close(two, want, rtol=1e-6, atol=1e-7)
