@@ -49,6 +49,8 @@ def _args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--ncu-case", action="store_true",
                    help="run one prefill and up to 64 decode steps of the workload, then exit (for ncu)")
+    p.add_argument("--paged", default=None, metavar="RAGGED_WORKLOAD",
+                   help="measure the paged, ragged cache on this ragged batch (e.g. ragged_gqa) instead")
     return p.parse_args()
 
 
@@ -96,11 +98,11 @@ def ncu_traffic(w):
     """Per-launch DRAM bytes of the decode kernel from the committed ncu summary,
     if it was taken on the current kernel source (else None)."""
     path = os.path.join(ROOT, "profiles", f"{decode_kernel_name(w)}_{w.name}.md")
-    src = os.path.join(ROOT, "bit_kv_cache_22_b200", "csrc", "decode.cu")
+    src = os.path.join(ROOT, "bit_kv_cache_22_b200", "csrc", "decode_kernels.cuh")
     try:
         text = open(path).read()
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        m_sha = re.search(r"decode\.cu sha256\[:16\]:\s*([0-9a-f]{16})", text)
+        m_sha = re.search(r"decode_kernels\.cuh sha256\[:16\]:\s*([0-9a-f]{16})", text)
         m_b = re.search(r"dram bytes per launch:\s*([0-9]+)", text)
         if m_sha and m_b and m_sha.group(1) == sha:
             return int(m_b.group(1))
@@ -415,6 +417,123 @@ def run_kvq(args):
 
 
 # ---------------------------------------------------------------------------
+# the paged, ragged cache
+# ---------------------------------------------------------------------------
+
+def run_paged(args):
+    """Decode attention of a ragged batch held in a paged cache.  After the prompts'
+    prefill, every decode step appends one token per slot (eagerly: the page table is
+    written from the host when a flush opens a page) and its decode_attention call is
+    captured as a CUDA graph and replayed `--steps` times between two events on the
+    replay stream.  value = KV tokens attended per second of decode time over all steps;
+    the roofline uses the algorithmic bytes of every slot at its own length."""
+    import torch
+
+    from bit_kv_cache_22_b200 import kvq
+    from bit_kv_cache_22_b200 import workloads as wl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
+    spec = wl.RAGGED[args.paged]
+    w = shard_workload(spec["base"], rank)
+    lens = wl.ragged_lengths(w, spec["lo"], spec["hi"])
+    P = spec["page_tokens"]
+    dt = torch.float16 if w.dtype == wl.FP16 else torch.bfloat16
+
+    def to_t(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(dt).to(dev)
+
+    cap = -(-(max(lens) + w.steps) // P) * P
+    cache = kvq.PagedKVQCache(w.B, w.Hq, w.Hkv, w.d, w.G, w.Gv, w.R, w.bits, w.symmetric, dt, cap, P,
+                              None, dev)
+    np.random.default_rng(w.seed).shuffle(cache.free_pages)     # a scrambled pool
+    for b, T in enumerate(lens):
+        XK, XV = wl.prefill_bits(w, bs=[b], T=T)
+        cache.prefill(b, to_t(XK[0]), to_t(XV[0]))
+    tK, tV, tQ = (to_t(x) for x in wl.decode_bits(w))
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    pool = torch.cuda.graph_pool_handle()
+    total_ms, total_tokens, total_bytes, launches = 0.0, 0, 0, 0
+    with ClockSampler(local) as clk:
+        for s in range(w.steps):
+            cache.append(tK[s], tV[s])
+            torch.cuda.synchronize()
+            l0 = kvq.kernel_launches()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, pool=pool):
+                cache.decode_attention(tQ[s], out=out)
+            per_call = kvq.kernel_launches() - l0
+            for _ in range(max(1, args.warmup)):
+                g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            total_ms += e0.elapsed_time(e1)
+            launches += per_call * args.steps
+            n = [cache.lens[b] for b in range(w.B)]
+            total_tokens += sum(n) * args.steps
+            w1 = w.replace(B=1)
+            total_bytes += sum(algorithmic_bytes(w1, x // w.R * w.R, x % w.R) for x in n) * args.steps
+            del g
+    ms, = max_over_ranks([total_ms], world, dev)
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+    calls = w.steps * args.steps
+    peak, peak_kind = peaks()
+    achieved = total_bytes / (total_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": job_throughput(total_tokens, world, ms), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / calls,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": f"u{w.bits} codes, f32 accumulate",
+        "data": "synthetic (seeded; distributions of the workload definition)",
+        "config": {
+            "workload": f"{args.paged} (paged, ragged)", "slots_per_gpu": w.B, "q_heads": w.Hq,
+            "kv_heads": w.Hkv, "head_dim": w.d, "prompt_tokens": f"{min(lens)}..{max(lens)} "
+            f"(mean {sum(lens) / len(lens):.0f})", "page_tokens": P, "decode_steps": w.steps,
+            "bits": w.bits, "group_k": w.G, "group_v": w.Gv, "residual": w.R,
+            "elem": "fp16" if w.dtype == wl.FP16 else "bf16", "parallelism": f"dp{world}",
+            "l2": "inputs larger than L2: packed cache "
+                  f"{total_bytes / calls / 1e6:.0f} MB per decode call",
+            "splits": cache.splits(),
+            "timing": "per decode step: its decode_attention graph replayed --steps times between "
+                      "two events (value and roofline: decode time only; appends run eagerly between)",
+        },
+        "roofline": {
+            "kernel": f"paged decode_attention ({decode_kernel_name(w)}, paged instance), per call",
+            "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+            else "fallback 6.65 TB/s",
+            "algorithmic_bytes_per_launch": total_bytes / calls, "avg_launch_us": total_ms / calls * 1e3,
+            "traffic": None,
+        },
+        "cpu_baseline": None,
+        "e2e": None,
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
 # the CPU oracle (cpu_baseline leg and --impl reference)
 # ---------------------------------------------------------------------------
 
@@ -470,6 +589,8 @@ def main():
     args = _args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.paged:
+        run_paged(args)
     else:
         run_kvq(args)
 

@@ -37,15 +37,31 @@ def _stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every translation unit (in parallel) and link libkvq.so."""
     if not force and not _stale():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [NVCC, *NVCC_FLAGS, "-shared", "-I", os.path.join(ROOT, "include"), "-o", tmp,
-           *sources()]
-    if verbose:
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
+    objdir = os.path.join(PKG, "_build")
+    os.makedirs(objdir, exist_ok=True)
+    tag = os.getpid()
+    procs = []
+    for src in sources():
+        obj = os.path.join(objdir, os.path.basename(src) + f".{tag}.o")
+        cmd = [NVCC, *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-c", src, "-o", obj]
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        procs.append((subprocess.Popen(cmd), obj))
+    failed = [p.args for p, _ in procs if p.wait() != 0]
+    objs = [o for _, o in procs]
+    try:
+        if failed:
+            raise subprocess.CalledProcessError(1, failed[0])
+        tmp = LIB + f".tmp{tag}"
+        subprocess.run([NVCC, *NVCC_FLAGS, "-shared", "-o", tmp, *objs], check=True)
+        os.replace(tmp, LIB)
+    finally:
+        for o in objs:
+            if os.path.exists(o):
+                os.remove(o)
     return LIB
 
 

@@ -15,6 +15,7 @@
 #include <mutex>
 #include <new>
 #include <string>
+#include <vector>
 
 #include "../../include/kvq.h"
 #include "kvq_internal.cuh"
@@ -111,30 +112,46 @@ struct kvq_cache {
 
 namespace {
 
-// Split count for the current cache length.  The quantized tiles are cut into
-// n_qsplits contiguous splits (of a multiple of the path's tile alignment); the
-// residual rows (if any) get one split of their own.  A CTA's time is modelled
-// as a fixed start/finish cost of kCtaFixedTiles tiles plus the tiles its
-// busiest warp streams; the kernel's time as the larger of (the waves of
-// quantized CTAs over the GPU's resident slots x one quantized CTA) and (all
-// CTA time spread evenly over the slots, plus one residual CTA).  The split
-// count with the lowest modelled time wins (ties: fewer splits).
+// Split count for a decode.  The quantized tiles of every sequence are cut into
+// splits of tiles_per_split tiles (a multiple of the path's tile alignment); S
+// covers the longest sequence, and a shorter one leaves its later splits empty.
+// The residual rows (if any) get one split of their own, except on the tensor-core
+// path with one query head per kv head, where they are dealt to the warps of the
+// quantized splits.  A CTA's time is modelled as a fixed start/finish cost of
+// kCtaFixedTiles tiles plus the tiles its busiest warp streams (an empty split
+// costs kEmptyCtaTiles); the kernel's time as the larger of (the waves of quantized
+// CTAs over the GPU's resident slots x one quantized CTA) and (all CTA time spread
+// evenly over the slots, plus one residual CTA).  The split count with the lowest
+// modelled time wins (ties: fewer splits).
 constexpr double kCtaFixedTiles = 6.0;
+constexpr double kEmptyCtaTiles = 1.0;
 
-void plan_splits(const kvq_cache *h, int *n_qsplits, int *tiles_per_split, int *S_out) {
+// The sequences' lengths as the planner sees them: n entries of quantized tiles,
+// each standing for `mult` sequences, and the most residual rows of any sequence.
+struct PlanInput {
+    const int64_t *tiles;
+    int n;
+    int64_t mult;
+    int32_t max_r;
+};
+
+void plan_splits_for(const kvq_cache *h, const PlanInput &in, int *n_qsplits, int *tiles_per_split,
+                     int *S_out) {
     const kvq_config &c = h->cfg;
-    const int64_t tiles = h->Tq / 16;
+    int64_t tiles = 0;
+    for (int i = 0; i < in.n; ++i) tiles = in.tiles[i] > tiles ? in.tiles[i] : tiles;
     const int path = kvq::decode_path(c.q_heads, c.kv_heads, c.group_k);
     // with one query head per kv head the tensor-core kernel deals the residual tiles to the
     // warps of the quantized splits
     const int hg = c.q_heads / c.kv_heads;
     const bool res_shared = path == kvq::kPathTc && hg == 1;
-    const int extra = (h->r > 0 && !res_shared) ? 1 : 0;
+    const int extra = (in.max_r > 0 && !res_shared) ? 1 : 0;
     const int64_t align = kvq::split_tile_align(path);
-    // CTAs per split: one per kv head on the tensor-core path, else one per query head
-    const int64_t units = static_cast<int64_t>(c.batch) * (path == kvq::kPathTc ? c.kv_heads : c.q_heads);
+    // CTAs per split and sequence: one per kv head on the tensor-core path, else one per query head
+    const int64_t per_seq = path == kvq::kPathTc ? c.kv_heads : c.q_heads;
+    const int64_t units = static_cast<int64_t>(c.batch) * per_seq;
     const double slots = static_cast<double>(h->num_sms) * h->ctas_per_sm;
-    const int64_t nres = (h->r + 15) / 16;
+    const int64_t nres = (in.max_r + 15) / 16;
     // residual CTA: its tiles shared by the 4 warps of each of its query heads
     const int heads_per_cta = path == kvq::kPathTc ? hg : 1;
     const double c_res = kCtaFixedTiles + static_cast<double>((nres * heads_per_cta + 3) / 4);
@@ -152,9 +169,13 @@ void plan_splits(const kvq_cache *h, int *n_qsplits, int *tiles_per_split, int *
             // a residual tile on CUDA cores costs about two quantized tiles
             const int64_t res_warp = res_shared ? (nres + 4 * S - 1) / (4 * S) : 0;
             const double c_q = kCtaFixedTiles + static_cast<double>(per_warp + 2 * res_warp);
-            const double nq = static_cast<double>(units * S);
+            int64_t busy = 0;   // non-empty quantized splits over all sequences
+            for (int i = 0; i < in.n; ++i) busy += in.mult * ((in.tiles[i] + per - 1) / per);
+            const double nq = static_cast<double>(per_seq * busy);
+            const double n_empty = static_cast<double>(units * S) - nq;
             const double t_waves = std::ceil(nq / slots) * c_q;
-            const double t_spread = (nq * c_q + static_cast<double>(units * extra) * c_res) / slots +
+            const double t_spread = (nq * c_q + n_empty * kEmptyCtaTiles + static_cast<double>(units * extra) * c_res) /
+                                        slots +
                                     (extra ? c_res : 0.0);
             const double cost = t_waves > t_spread ? t_waves : t_spread;
             if (best_cost < 0 || cost < best_cost - 1e-9) {
@@ -168,9 +189,19 @@ void plan_splits(const kvq_cache *h, int *n_qsplits, int *tiles_per_split, int *
         best_S = 1;
         best_per = 0;
     }
+    if (best_S + extra == 0) {          // nothing in any sequence: one empty split writes zeros
+        best_S = 1;
+        best_per = align;
+    }
     *n_qsplits = static_cast<int>(best_S);
     *tiles_per_split = static_cast<int>(best_per);
     *S_out = static_cast<int>(best_S + extra);
+}
+
+void plan_splits(const kvq_cache *h, int *n_qsplits, int *tiles_per_split, int *S_out) {
+    const int64_t tiles = h->Tq / 16;
+    const PlanInput in{&tiles, 1, h->cfg.batch, h->r};
+    plan_splits_for(h, in, n_qsplits, tiles_per_split, S_out);
 }
 
 kvq::DecodeArgs decode_args(const kvq_cache *h) {
@@ -595,5 +626,322 @@ uint64_t kvq_kernel_launches(void) { return g_launches.load(); }
 const char *kvq_last_error(void) { return g_last_error.c_str(); }
 
 int32_t kvq_layout_version(void) { return 2; }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Paged, ragged cache.
+//
+// The handle wraps a kvq_cache for the geometry, the launch properties and the
+// library-owned counters; its six cache buffers are the pool.  The host keeps
+// every slot's length (-1: inactive) to decide flushes and plan splits; the
+// kernels read the device copy, which the paged append kernel advances in
+// stream order.
+// ---------------------------------------------------------------------------
+struct kvq_paged {
+    kvq_cache base;
+    int32_t page_tokens = 0, num_pages = 0, max_pages = 0;
+    const int32_t *page_table = nullptr;
+    int32_t *seq_len = nullptr;   // device [B], inside base.arrivals' allocation
+    int64_t *len = nullptr;       // host [B]
+};
+
+namespace {
+
+kvq_status validate_paged(const kvq_paged_config *c) {
+    if (!c) return fail(KVQ_ERR_INVALID_ARG, "config is NULL");
+    kvq_status st = validate(&c->geom);
+    if (st != KVQ_OK) return st;
+    const int P = c->page_tokens;
+    if (P < 64 || P % 64 != 0 || P % c->geom.residual != 0)
+        return fail(KVQ_ERR_INVALID_ARG, "page_tokens (%d) must be a positive multiple of 64 and of residual (%d)",
+                    P, c->geom.residual);
+    if (c->geom.capacity % P != 0)
+        return fail(KVQ_ERR_INVALID_ARG, "capacity must be a multiple of page_tokens");
+    if (c->num_pages < 1) return fail(KVQ_ERR_INVALID_ARG, "num_pages must be >= 1");
+    if (static_cast<int64_t>(c->num_pages) * c->geom.kv_heads * (P / 16) > (int64_t{1} << 40))
+        return fail(KVQ_ERR_UNSUPPORTED, "pool too large");
+    if (static_cast<int64_t>(c->geom.batch) * (c->geom.capacity / P) > (int64_t{1} << 31) - 1)
+        return fail(KVQ_ERR_UNSUPPORTED, "page table too large");
+    return KVQ_OK;
+}
+
+kvq::DecodeArgs paged_decode_args(const kvq_paged *h) {
+    kvq::DecodeArgs a = decode_args(&h->base);
+    a.cap = h->page_tokens;
+    a.page_table = h->page_table;
+    a.seq_len = h->seq_len;
+    a.page_tiles = h->page_tokens / 16;
+    a.max_pages = h->max_pages;
+    a.num_pages = h->num_pages;
+    a.n_qtiles = 0;
+    a.r = 0;
+    return a;
+}
+
+kvq::QuantizeArgs paged_quantize_args(const kvq_paged *h) {
+    kvq::QuantizeArgs q = quantize_args(&h->base);
+    q.cap = h->page_tokens;
+    q.page_table = h->page_table;
+    q.max_pages = h->max_pages;
+    q.num_pages = h->num_pages;
+    q.Hkv = h->base.cfg.kv_heads;
+    q.status = h->base.arrivals + static_cast<int64_t>(h->base.cfg.batch) * h->base.cfg.q_heads;
+    return q;
+}
+
+void paged_plan(const kvq_paged *h, int *n_qsplits, int *tiles_per_split, int *S) {
+    const kvq_config &c = h->base.cfg;
+    // lengths of the active slots (tiles per slot) and the most residual rows
+    std::vector<int64_t> tiles(static_cast<size_t>(c.batch));
+    int32_t max_r = 0;
+    for (int b = 0; b < c.batch; ++b) {
+        const int64_t len = h->len[b] > 0 ? h->len[b] : 0;
+        tiles[b] = (len / c.residual) * c.residual / 16;
+        const int32_t r = static_cast<int32_t>(len % c.residual);
+        max_r = r > max_r ? r : max_r;
+    }
+    const PlanInput in{tiles.data(), c.batch, 1, max_r};
+    plan_splits_for(&h->base, in, n_qsplits, tiles_per_split, S);
+}
+
+kvq_status check_status_word(unsigned int *word) {
+    unsigned int v = 0;
+    cudaError_t e = cudaMemcpy(&v, word, sizeof v, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
+    if (v == 0) return ok();
+    e = cudaMemset(word, 0, sizeof v);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
+    if (v & 2u)
+        return fail(KVQ_ERR_INVALID_ARG, "a kernel met a page-table entry outside the pool; "
+                                         "outputs since the last check are unreliable");
+    return fail(KVQ_ERR_CUDA, "a decode kernel gave up waiting for a copy into shared memory; "
+                              "outputs since the last check are unreliable");
+}
+
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_paged_get_sizes(const kvq_paged_config *cfg, kvq_paged_sizes *out) {
+    if (!out) return fail(KVQ_ERR_INVALID_ARG, "out is NULL");
+    kvq_status st = validate_paged(cfg);
+    if (st != KVQ_OK) return st;
+    const kvq_config &g = cfg->geom;
+    const int64_t slices = static_cast<int64_t>(cfg->num_pages) * g.kv_heads;
+    const int64_t P = cfg->page_tokens, d = g.head_dim;
+    std::memset(out, 0, sizeof *out);
+    out->k_codes = out->v_codes = static_cast<size_t>(slices * P * d * g.bits / 8);
+    out->k_scales = static_cast<size_t>(slices * (P / g.group_k) * d * 4);
+    out->k_zeros = g.symmetric ? 0 : static_cast<size_t>(slices * (P / g.group_k) * d * 2);
+    out->v_scales = static_cast<size_t>(slices * P * (d / g.group_v) * 4);
+    out->v_zeros = g.symmetric ? 0 : static_cast<size_t>(slices * P * (d / g.group_v) * 2);
+    const int64_t BH = static_cast<int64_t>(g.batch) * g.kv_heads;
+    out->k_residual = out->v_residual = static_cast<size_t>(BH * g.residual * d * 2);
+    out->page_table = static_cast<size_t>(static_cast<int64_t>(g.batch) * (g.capacity / P) * 4);
+    const int64_t units = static_cast<int64_t>(g.batch) * g.q_heads;
+    out->workspace = static_cast<size_t>(units * max_splits(&g) * (d + 2) * 4);
+    return ok();
+}
+
+kvq_status kvq_paged_create(const kvq_paged_config *cfg, const kvq_buffers *bufs, const int32_t *page_table,
+                            kvq_paged **out) {
+    if (!out) return fail(KVQ_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    kvq_status st = validate_paged(cfg);
+    if (st != KVQ_OK) return st;
+    if (!bufs) return fail(KVQ_ERR_INVALID_ARG, "buffers are NULL");
+    if (!page_table || !aligned16(page_table))
+        return fail(KVQ_ERR_INVALID_ARG, "page_table must be non-NULL and 16-byte aligned");
+    const void *need[] = {bufs->k_codes, bufs->k_scales, bufs->v_codes, bufs->v_scales,
+                          bufs->k_residual, bufs->v_residual};
+    for (const void *p : need)
+        if (!p || !aligned16(p))
+            return fail(KVQ_ERR_INVALID_ARG, "cache buffers must be non-NULL and 16-byte aligned");
+    const kvq_config &g = cfg->geom;
+    if (!g.symmetric && (!bufs->k_zeros || !bufs->v_zeros || !aligned16(bufs->k_zeros) ||
+                         !aligned16(bufs->v_zeros)))
+        return fail(KVQ_ERR_INVALID_ARG, "asymmetric caches need 16-byte aligned zero buffers");
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "querying the current device");
+    kvq_paged *h = new (std::nothrow) kvq_paged();
+    int64_t *len = new (std::nothrow) int64_t[g.batch];
+    if (!h || !len) {
+        delete h;
+        delete[] len;
+        return fail(KVQ_ERR_INVALID_ARG, "out of host memory");
+    }
+    for (int b = 0; b < g.batch; ++b) len[b] = -1;
+    h->len = len;
+    h->base.cfg = g;
+    h->base.buf = *bufs;
+    if (g.symmetric) {
+        h->base.buf.k_zeros = nullptr;
+        h->base.buf.v_zeros = nullptr;
+    }
+    h->page_tokens = cfg->page_tokens;
+    h->num_pages = cfg->num_pages;
+    h->max_pages = static_cast<int32_t>(g.capacity / cfg->page_tokens);
+    h->page_table = page_table;
+    h->base.num_sms = sms > 0 ? sms : 148;
+    // counters [B * Hq], status word, slot lengths [B] (all -1: inactive)
+    const size_t counters = static_cast<size_t>(g.batch) * g.q_heads + 1;
+    const size_t bytes = (counters + g.batch) * sizeof(unsigned int);
+    e = cudaMalloc(&h->base.arrivals, bytes);
+    if (e == cudaSuccess) e = cudaMemset(h->base.arrivals, 0, counters * sizeof(unsigned int));
+    if (e == cudaSuccess) e = cudaMemset(h->base.arrivals + counters, 0xff, g.batch * sizeof(unsigned int));
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) {
+        if (h->base.arrivals) cudaFree(h->base.arrivals);
+        delete[] h->len;
+        delete h;
+        return cuda_fail(e, "allocating the paged cache's counters");
+    }
+    h->seq_len = reinterpret_cast<int32_t *>(h->base.arrivals + counters);
+    h->base.ctas_per_sm = kvq::decode_ctas_per_sm(paged_decode_args(h));
+    *out = h;
+    return ok();
+}
+
+void kvq_paged_destroy(kvq_paged *h) {
+    if (!h) return;
+    if (h->base.arrivals) cudaFree(h->base.arrivals);
+    delete[] h->len;
+    delete h;
+}
+
+kvq_status kvq_paged_prefill(kvq_paged *h, int32_t seq, const void *X_K, const void *X_V, int64_t T,
+                             void *stream) {
+    if (!h) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+    const kvq_config &c = h->base.cfg;
+    if (seq < 0 || seq >= c.batch) return fail(KVQ_ERR_INVALID_ARG, "seq must be in 0..%d", c.batch - 1);
+    if (T < 0) return fail(KVQ_ERR_INVALID_ARG, "T must be >= 0");
+    if (h->len[seq] >= 0) return fail(KVQ_ERR_STATE, "slot %d is active; release it first", seq);
+    if (T > 0 && (!X_K || !X_V || !aligned16(X_K) || !aligned16(X_V)))
+        return fail(KVQ_ERR_INVALID_ARG, "X_K and X_V must be non-NULL and 16-byte aligned");
+    const int64_t Tq = (T / c.residual) * c.residual;
+    if (Tq > c.capacity)
+        return fail(KVQ_ERR_CAPACITY, "prefill of %lld tokens exceeds capacity %lld",
+                    static_cast<long long>(Tq), static_cast<long long>(c.capacity));
+    if (T > 0x7fffffffLL) return fail(KVQ_ERR_UNSUPPORTED, "T must be < 2^31");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    kvq::QuantizeArgs q = paged_quantize_args(h);
+    q.xk = static_cast<const uint16_t *>(X_K);
+    q.xv = static_cast<const uint16_t *>(X_V);
+    q.in_bh_stride = T * c.head_dim;
+    q.in_tok0 = 0;
+    q.n_groups = Tq / c.group_k;
+    q.out_tok0 = 0;
+    q.BH = c.kv_heads;
+    q.seq0 = seq;
+    q.seq_len = nullptr;
+    cudaError_t e = kvq::launch_quantize(q, s);
+    if (e != cudaSuccess) return cuda_fail(e, "paged prefill quantize launch");
+    e = kvq::launch_paged_residual(static_cast<const uint16_t *>(X_K), static_cast<const uint16_t *>(X_V), T, Tq,
+                                   T - Tq, static_cast<uint16_t *>(h->base.buf.k_residual),
+                                   static_cast<uint16_t *>(h->base.buf.v_residual), h->seq_len, seq,
+                                   static_cast<int32_t>(T), c.kv_heads, c.residual, c.head_dim, s);
+    if (e != cudaSuccess) return cuda_fail(e, "paged prefill residual launch");
+    h->len[seq] = T;
+    return ok();
+}
+
+kvq_status kvq_paged_append(kvq_paged *h, const void *t_K, const void *t_V, void *stream) {
+    if (!h) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+    if (!t_K || !t_V || !aligned16(t_K) || !aligned16(t_V))
+        return fail(KVQ_ERR_INVALID_ARG, "t_K and t_V must be non-NULL and 16-byte aligned");
+    const kvq_config &c = h->base.cfg;
+    bool any_flush = false;
+    for (int b = 0; b < c.batch; ++b) {
+        if (h->len[b] < 0) continue;
+        const int64_t n = h->len[b] + 1;
+        if (n % c.residual == 0) {
+            if (n > c.capacity)
+                return fail(KVQ_ERR_CAPACITY, "flushing slot %d would exceed capacity %lld", b,
+                            static_cast<long long>(c.capacity));
+            any_flush = true;
+        }
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = kvq::launch_paged_append(static_cast<const uint16_t *>(t_K), static_cast<const uint16_t *>(t_V),
+                                             static_cast<uint16_t *>(h->base.buf.k_residual),
+                                             static_cast<uint16_t *>(h->base.buf.v_residual), h->seq_len, c.batch,
+                                             c.kv_heads, c.residual, c.head_dim, s);
+    if (e != cudaSuccess) return cuda_fail(e, "paged append launch");
+    if (any_flush) {
+        kvq::QuantizeArgs q = paged_quantize_args(h);
+        q.xk = static_cast<const uint16_t *>(h->base.buf.k_residual);
+        q.xv = static_cast<const uint16_t *>(h->base.buf.v_residual);
+        q.in_bh_stride = static_cast<int64_t>(c.residual) * c.head_dim;
+        q.in_tok0 = 0;
+        q.n_groups = c.residual / c.group_k;
+        q.out_tok0 = 0;
+        q.BH = static_cast<int64_t>(c.batch) * c.kv_heads;
+        q.seq0 = 0;
+        q.seq_len = h->seq_len;
+        e = kvq::launch_quantize(q, s);
+        if (e != cudaSuccess) return cuda_fail(e, "paged flush launch");
+    }
+    for (int b = 0; b < c.batch; ++b)
+        if (h->len[b] >= 0) ++h->len[b];
+    return ok();
+}
+
+kvq_status kvq_paged_decode_attention(kvq_paged *h, const void *t_Q, float *t_O, void *workspace,
+                                      size_t workspace_bytes, void *stream) {
+    if (!h) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+    if (!t_Q || !t_O || !workspace || !aligned16(t_Q) || !aligned16(t_O) || !aligned16(workspace))
+        return fail(KVQ_ERR_INVALID_ARG, "t_Q, t_O and workspace must be non-NULL and 16-byte aligned");
+    const kvq_config &c = h->base.cfg;
+    const int64_t units = static_cast<int64_t>(c.batch) * c.q_heads;
+    const size_t need = static_cast<size_t>(units * max_splits(&c) * (c.head_dim + 2) * 4);
+    if (workspace_bytes < need)
+        return fail(KVQ_ERR_INVALID_ARG, "workspace needs %zu bytes, got %zu", need, workspace_bytes);
+    kvq::DecodeArgs a = paged_decode_args(h);
+    paged_plan(h, &a.n_qsplits, &a.tiles_per_split, &a.S);
+    float *ws = static_cast<float *>(workspace);
+    a.o_part = ws;
+    a.m_part = ws + units * a.S * c.head_dim;
+    a.l_part = a.m_part + units * a.S;
+    a.q = static_cast<const uint16_t *>(t_Q);
+    a.out = t_O;
+    cudaError_t e = kvq::launch_decode(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "paged decode launch");
+    return ok();
+}
+
+kvq_status kvq_paged_release(kvq_paged *h, int32_t seq, void *stream) {
+    if (!h) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+    const kvq_config &c = h->base.cfg;
+    if (seq < 0 || seq >= c.batch) return fail(KVQ_ERR_INVALID_ARG, "seq must be in 0..%d", c.batch - 1);
+    cudaError_t e = kvq::launch_paged_residual(nullptr, nullptr, 0, 0, 0, nullptr, nullptr, h->seq_len, seq, -1,
+                                               c.kv_heads, c.residual, c.head_dim, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "paged release launch");
+    h->len[seq] = -1;
+    return ok();
+}
+
+kvq_status kvq_paged_seq_len(const kvq_paged *h, int32_t seq, int64_t *len) {
+    if (!h || !len) return fail(KVQ_ERR_INVALID_ARG, "cache and len must be non-NULL");
+    if (seq < 0 || seq >= h->base.cfg.batch)
+        return fail(KVQ_ERR_INVALID_ARG, "seq must be in 0..%d", h->base.cfg.batch - 1);
+    *len = h->len[seq];
+    return ok();
+}
+
+int32_t kvq_paged_decode_splits(const kvq_paged *h) {
+    if (!h) return 0;
+    int nq, per, S;
+    paged_plan(h, &nq, &per, &S);
+    return S;
+}
+
+kvq_status kvq_paged_check_device(kvq_paged *h) {
+    if (!h) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+    return check_status_word(h->base.arrivals + static_cast<int64_t>(h->base.cfg.batch) * h->base.cfg.q_heads);
+}
 
 }  // extern "C"

@@ -43,6 +43,14 @@ struct QuantizeArgs {
     int16_t *kz, *vz;            // same shapes (unused when sym)
     int64_t cap;                 // token capacity per slice
     int64_t out_tok0;            // first output token (multiple of G)
+    // paged pool (page_table non-NULL): slice (page, kv head) of cap = P tokens; the
+    // slice of output token t of sequence b is page_table[b][t / P] * Hkv + kv head
+    const int32_t *page_table;   // [B][max_pages]
+    int max_pages, num_pages, Hkv;
+    int seq0;                    // first sequence of the launch: CTA y = (seq - seq0) * Hkv + head
+    const int32_t *seq_len;      // flush: tokens of each sequence after the append; only those
+                                 // at a multiple of R flush, to tokens [len - R, len)
+    unsigned int *status;        // bit 2 raised for a page number outside the pool
 };
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s);
 
@@ -93,8 +101,28 @@ struct DecodeArgs {
     int n_qsplits;               // splits over the quantized tiles
     int S;                       // n_qsplits + (r > 0)
     float qscale;                // log2(e) / sqrt(d)
+    // paged, ragged cache (page_table non-NULL): the pool is cut into pages of P tokens per
+    // (page, kv head) slice, laid out like a contiguous cache of capacity P whose batch is
+    // the page; sequence b's tokens [jP, (j+1)P) are in page page_table[b][j], and its token
+    // count is seq_len[b] (Tq = floor(len / R) R, r = len mod R; len < 0: an inactive slot,
+    // treated as empty).  n_qtiles / r above are unused then.
+    const int32_t *page_table;   // [B][max_pages]
+    const int32_t *seq_len;      // [B]
+    int page_tiles;              // P / 16
+    int max_pages, num_pages;
 };
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+cudaError_t launch_decode_paged(const DecodeArgs &a, cudaStream_t s);
+int decode_ctas_per_sm_paged(const DecodeArgs &a);
+// Paged append: for each sequence slot b with seq_len[b] >= 0, rows t_K[b], t_V[b] ([Hkv][d])
+// become residual row seq_len[b] mod R and seq_len[b] grows by one.  One launch.
+cudaError_t launch_paged_append(const uint16_t *tk, const uint16_t *tv, uint16_t *kr, uint16_t *vr,
+                                int32_t *seq_len, int B, int Hkv, int R, int d, cudaStream_t s);
+// Sets seq_len[seq] = value and copies rows [row0, row0 + rows) of X_K / X_V ([Hkv][T][d])
+// to residual rows 0 .. rows-1 of sequence seq.  One launch.
+cudaError_t launch_paged_residual(const uint16_t *xk, const uint16_t *xv, int64_t T, int64_t row0,
+                                  int64_t rows, uint16_t *kr, uint16_t *vr, int32_t *seq_len, int seq,
+                                  int32_t value, int Hkv, int R, int d, cudaStream_t s);
 // t_O [rows][d] from n partials o_all [n][rows][d], m_all / l_all [n][rows] (log2 units).
 cudaError_t launch_merge_partials(const float *o_all, const float *m_all, const float *l_all, int n,
                                   int64_t rows, int d, float *out, cudaStream_t s);

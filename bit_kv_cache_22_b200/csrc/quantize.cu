@@ -128,12 +128,30 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
     float *ch_r = reinterpret_cast<float *>(ch_z + d);                       // [d] 1/s
 
     const int64_t grp = blockIdx.x;
-    const int64_t bh = blockIdx.y;
+    const int64_t bh = blockIdx.y;                 // input slice
     const int64_t in_tok = a.in_tok0 + grp * G;
-    const int64_t out_tok = a.out_tok0 + grp * G;
+    int64_t out_tok = a.out_tok0 + grp * G;
+    int64_t slice = bh, cap = a.cap;               // output slice and its token capacity
+    if (a.page_table) {
+        // paged pool: the group's page of its sequence (groups never straddle pages)
+        const int64_t b = a.seq0 + bh / a.Hkv;
+        if (a.seq_len) {                           // flush: only sequences whose residual just filled
+            const int64_t len = a.seq_len[b], R = a.n_groups * G;
+            if (len <= 0 || len % R != 0) return;
+            out_tok = len - R + grp * G;
+        }
+        const int64_t pi = out_tok / a.cap;
+        const int page = pi < a.max_pages ? a.page_table[b * a.max_pages + pi] : -1;
+        if (page < 0 || page >= a.num_pages) {    // not a page of the pool: write nothing
+            if (threadIdx.x == 0) atomicOr(a.status, 2u);
+            return;
+        }
+        slice = static_cast<int64_t>(page) * a.Hkv + bh % a.Hkv;
+        out_tok -= pi * a.cap;
+    }
     const int TW = tile_words(d, bits);
-    const int64_t words_per_slice = a.cap / 16 * TW;
-    const int64_t groups_cap = a.cap / G;
+    const int64_t words_per_slice = cap / 16 * TW;
+    const int64_t groups_cap = cap / G;
 
     // ------------------------------ keys ------------------------------
     load_group(a.xk + bh * a.in_bh_stride + in_tok * d, xs, G * d);
@@ -170,9 +188,9 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
                 const GroupParams gp = asym_params(mn, mx, bits);
                 s = gp.s;
                 z = gp.z;
-                a.kz[(bh * groups_cap + out_tok / G) * d + c] = static_cast<int16_t>(z);
+                a.kz[(slice * groups_cap + out_tok / G) * d + c] = static_cast<int16_t>(z);
             }
-            a.ks[(bh * groups_cap + out_tok / G) * d + c] = s;
+            a.ks[(slice * groups_cap + out_tok / G) * d + c] = s;
             ch_s[c] = s;
             ch_z[c] = z;
             ch_r[c] = s != 0.0f ? __frcp_rn(s) : 0.0f;
@@ -187,7 +205,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
         }
         __syncthreads();
         pack_tiles(codes, G / 16, d, bits, false,
-                   a.kc + bh * words_per_slice + (out_tok / 16) * TW);
+                   a.kc + slice * words_per_slice + (out_tok / 16) * TW);
         __syncthreads();
     }
 
@@ -227,7 +245,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
             }
             const int j = lane / seg;
             if (lane % seg == 0) {
-                const int64_t mi = (bh * a.cap + out_tok + t) * ngv + j;
+                const int64_t mi = (slice * cap + out_tok + t) * ngv + j;
                 a.vs[mi] = s;
                 if (!a.sym) a.vz[mi] = static_cast<int16_t>(z);
             }
@@ -238,7 +256,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
         }
         __syncthreads();
         pack_tiles(codes, G / 16, d, bits, true,
-                   a.vc + bh * words_per_slice + (out_tok / 16) * TW);
+                   a.vc + slice * words_per_slice + (out_tok / 16) * TW);
     }
 }
 
@@ -262,6 +280,44 @@ __global__ void copy_rows_kernel(const uint16_t *src0, const uint16_t *src1, int
         uint4 *tp = reinterpret_cast<uint4 *>(dst + bh * dst_bh_stride + (dst_row0 + row) * d) + v;
         *tp = *sp;
     }
+}
+
+// Paged append: CTA b copies the new rows of all kv heads of sequence b (if active) into
+// residual row seq_len[b] mod R, then advances seq_len[b].
+__global__ void paged_append_kernel(const uint16_t *tk, const uint16_t *tv, uint16_t *kr, uint16_t *vr,
+                                    int32_t *seq_len, int Hkv, int R, int d) {
+    const int b = blockIdx.x;
+    const int len = seq_len[b];
+    if (len < 0) return;
+    const int row = len % R;
+    const int vec = d / 8, per_seq = Hkv * vec;
+    for (int i = threadIdx.x; i < 2 * per_seq; i += blockDim.x) {
+        const bool isv = i >= per_seq;
+        const int k = isv ? i - per_seq : i;
+        const int h = k / vec, v = k % vec;
+        const int64_t bh = static_cast<int64_t>(b) * Hkv + h;
+        const uint4 x = reinterpret_cast<const uint4 *>((isv ? tv : tk) + bh * d)[v];
+        reinterpret_cast<uint4 *>((isv ? vr : kr) + (bh * R + row) * d)[v] = x;
+    }
+    __syncthreads();   // every thread has read seq_len[b]
+    if (threadIdx.x == 0) seq_len[b] = len + 1;
+}
+
+// Paged prefill tail: rows [row0, row0 + rows) of X_K / X_V ([Hkv][T][d]) become residual
+// rows 0 .. rows-1 of sequence seq; seq_len[seq] = value.
+__global__ void paged_residual_kernel(const uint16_t *xk, const uint16_t *xv, int64_t T, int64_t row0,
+                                      int64_t rows, uint16_t *kr, uint16_t *vr, int32_t *seq_len, int seq,
+                                      int32_t value, int Hkv, int R, int d) {
+    const int64_t vec = d / 8, per = static_cast<int64_t>(Hkv) * rows * vec;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < 2 * per;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const bool isv = i >= per;
+        const int64_t k = isv ? i - per : i;
+        const int64_t v = k % vec, row = (k / vec) % rows, h = k / (vec * rows);
+        const uint4 x = reinterpret_cast<const uint4 *>((isv ? xv : xk) + (h * T + row0 + row) * d)[v];
+        reinterpret_cast<uint4 *>((isv ? vr : kr) + ((static_cast<int64_t>(seq) * Hkv + h) * R + row) * d)[v] = x;
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) seq_len[seq] = value;
 }
 
 }  // namespace
@@ -301,6 +357,29 @@ cudaError_t launch_copy_rows(const uint16_t *src0, const uint16_t *src1, int64_t
     const int64_t blocks = (total + threads - 1) / threads;
     copy_rows_kernel<<<static_cast<unsigned>(blocks < 65536 ? blocks : 65536), threads, 0, s>>>(
         src0, src1, src_bh_stride, src_row0, dst0, dst1, dst_bh_stride, dst_row0, rows, BH, d);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace kvq
+
+namespace kvq {
+
+cudaError_t launch_paged_append(const uint16_t *tk, const uint16_t *tv, uint16_t *kr, uint16_t *vr,
+                                int32_t *seq_len, int B, int Hkv, int R, int d, cudaStream_t s) {
+    if (B == 0) return cudaSuccess;
+    paged_append_kernel<<<B, 128, 0, s>>>(tk, tv, kr, vr, seq_len, Hkv, R, d);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_paged_residual(const uint16_t *xk, const uint16_t *xv, int64_t T, int64_t row0,
+                                  int64_t rows, uint16_t *kr, uint16_t *vr, int32_t *seq_len, int seq,
+                                  int32_t value, int Hkv, int R, int d, cudaStream_t s) {
+    const int64_t total = 2 * static_cast<int64_t>(Hkv) * rows * (d / 8);
+    const int64_t blocks = total > 0 ? (total + 255) / 256 : 1;
+    paged_residual_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(xk, xv, T, row0, rows, kr, vr, seq_len,
+                                                                        seq, value, Hkv, R, d);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -31,7 +31,10 @@ EXPORTED = ("kvq_get_sizes", "kvq_create", "kvq_destroy", "kvq_reset", "kvq_pref
             "kvq_append", "kvq_decode_attention", "kvq_cache_state", "kvq_set_split_limit",
             "kvq_decode_splits", "kvq_kernel_launches", "kvq_decode_attention_noalloc",
             "kvq_last_error", "kvq_layout_version", "kvq_check_device", "kvq_append_decode_attention",
-            "kvq_decode_attention_partial", "kvq_merge_partials")
+            "kvq_decode_attention_partial", "kvq_merge_partials", "kvq_paged_get_sizes",
+            "kvq_paged_create", "kvq_paged_destroy", "kvq_paged_prefill", "kvq_paged_append",
+            "kvq_paged_decode_attention", "kvq_paged_release", "kvq_paged_seq_len",
+            "kvq_paged_decode_splits", "kvq_paged_check_device")
 
 
 class KVQError(RuntimeError):
@@ -59,6 +62,16 @@ class Buffers(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("k_codes", "k_scales", "k_zeros", "v_codes", "v_scales", "v_zeros",
                  "k_residual", "v_residual")]
+
+
+class PagedConfig(ctypes.Structure):
+    _fields_ = [("geom", Config), ("page_tokens", ctypes.c_int32), ("num_pages", ctypes.c_int32)]
+
+
+class PagedSizes(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in
+                ("k_codes", "k_scales", "k_zeros", "v_codes", "v_scales", "v_zeros",
+                 "k_residual", "v_residual", "page_table", "workspace")]
 
 
 def library_path() -> str:
@@ -104,6 +117,23 @@ def load() -> ctypes.CDLL:
         lib.kvq_layout_version.argtypes = []
         lib.kvq_layout_version.restype = i32
         lib.kvq_check_device.argtypes = [P]
+        lib.kvq_paged_get_sizes.argtypes = [ctypes.POINTER(PagedConfig), ctypes.POINTER(PagedSizes)]
+        lib.kvq_paged_create.argtypes = [ctypes.POINTER(PagedConfig), ctypes.POINTER(Buffers), P,
+                                         ctypes.POINTER(P)]
+        lib.kvq_paged_destroy.argtypes = [P]
+        lib.kvq_paged_destroy.restype = None
+        lib.kvq_paged_prefill.argtypes = [P, i32, P, P, i64, P]
+        lib.kvq_paged_append.argtypes = [P, P, P, P]
+        lib.kvq_paged_decode_attention.argtypes = [P, P, P, P, sz, P]
+        lib.kvq_paged_release.argtypes = [P, i32, P]
+        lib.kvq_paged_seq_len.argtypes = [P, i32, ctypes.POINTER(i64)]
+        lib.kvq_paged_decode_splits.argtypes = [P]
+        lib.kvq_paged_decode_splits.restype = i32
+        lib.kvq_paged_check_device.argtypes = [P]
+        for name in ("kvq_paged_get_sizes", "kvq_paged_create", "kvq_paged_prefill", "kvq_paged_append",
+                     "kvq_paged_decode_attention", "kvq_paged_release", "kvq_paged_seq_len",
+                     "kvq_paged_check_device"):
+            getattr(lib, name).restype = ctypes.c_int
         for name in ("kvq_get_sizes", "kvq_create", "kvq_reset", "kvq_prefill_quantize",
                      "kvq_append", "kvq_decode_attention", "kvq_cache_state", "kvq_set_split_limit",
                      "kvq_check_device"):
@@ -298,6 +328,178 @@ class KVQCache:
             out.copy_(dev_out, non_blocking=True)
             return out
         return dev_out
+
+
+class PagedKVQCache:
+    """A paged, ragged cache: `slots` sequences of their own lengths whose quantized tokens
+    live in pages of `page_tokens` tokens of one pool (torch tensors), with a page table
+    per sequence.
+
+    Pages are handed out from a host free list when a prefill or a flush needs them and
+    returned by release(); the page table (int32 [slots, capacity / page_tokens], -1 where
+    unassigned) is written on the stream of the call that needs it.  Shapes: prompt
+    X_K, X_V [Hkv, T, d] of one sequence; new tokens t_K, t_V [slots, Hkv, d]; queries
+    t_Q [slots, Hq, d]; output float32 [slots, Hq, d] (zeros for inactive slots).
+    """
+
+    def __init__(self, slots, q_heads, kv_heads, head_dim, group_k, group_v, residual, bits,
+                 symmetric=False, dtype=torch.bfloat16, capacity=None, page_tokens=None,
+                 num_pages=None, device=None):
+        if capacity is None:
+            raise ValueError("capacity (quantized tokens per sequence) is required")
+        if page_tokens is None:
+            page_tokens = residual * 64 // _gcd(residual, 64)
+        capacity = -(-capacity // page_tokens) * page_tokens
+        max_pages = capacity // page_tokens
+        if num_pages is None:
+            num_pages = slots * max_pages
+        dev = torch.device(device if device is not None else "cuda")
+        if dev.type != "cuda":
+            raise ValueError("the cache lives on a CUDA device")
+        self.device = dev if dev.index is not None else torch.device("cuda", torch.cuda.current_device())
+        self.dtype = dtype
+        self.geom = make_config(slots, q_heads, kv_heads, head_dim, group_k, group_v, residual,
+                                bits, symmetric, dtype, capacity)
+        self.cfg = PagedConfig(self.geom, page_tokens, num_pages)
+        self.sizes = PagedSizes()
+        self._lib = load()
+        _check(self._lib.kvq_paged_get_sizes(ctypes.byref(self.cfg), ctypes.byref(self.sizes)))
+        self.page_tokens, self.num_pages, self.max_pages = page_tokens, num_pages, max_pages
+        dev = self.device
+        NP = num_pages * kv_heads
+        words = page_tokens * head_dim * bits // 32
+        self.k_codes = torch.empty((NP, words), dtype=torch.int32, device=dev)
+        self.v_codes = torch.empty((NP, words), dtype=torch.int32, device=dev)
+        self.k_scales = torch.empty((NP, page_tokens // group_k, head_dim), dtype=torch.float32, device=dev)
+        self.v_scales = torch.empty((NP, page_tokens, head_dim // group_v), dtype=torch.float32, device=dev)
+        if symmetric:
+            self.k_zeros = self.v_zeros = None
+        else:
+            self.k_zeros = torch.empty((NP, page_tokens // group_k, head_dim), dtype=torch.int16, device=dev)
+            self.v_zeros = torch.empty((NP, page_tokens, head_dim // group_v), dtype=torch.int16, device=dev)
+        BH = slots * kv_heads
+        self.k_residual = torch.zeros((BH, residual, head_dim), dtype=dtype, device=dev)
+        self.v_residual = torch.zeros((BH, residual, head_dim), dtype=dtype, device=dev)
+        self.page_table = torch.full((slots, max_pages), -1, dtype=torch.int32, device=dev)
+        self.workspace = torch.empty(self.sizes.workspace // 4, dtype=torch.float32, device=dev)
+        bufs = Buffers(self.k_codes.data_ptr(), self.k_scales.data_ptr(),
+                       self.k_zeros.data_ptr() if self.k_zeros is not None else None,
+                       self.v_codes.data_ptr(), self.v_scales.data_ptr(),
+                       self.v_zeros.data_ptr() if self.v_zeros is not None else None,
+                       self.k_residual.data_ptr(), self.v_residual.data_ptr())
+        h = ctypes.c_void_p()
+        with torch.cuda.device(dev):
+            _check(self._lib.kvq_paged_create(ctypes.byref(self.cfg), ctypes.byref(bufs),
+                                              self.page_table.data_ptr(), ctypes.byref(h)))
+        self._h = h
+        self.free_pages = list(range(num_pages - 1, -1, -1))   # pop() hands out 0, 1, 2, ...
+        self.pages = [[] for _ in range(slots)]
+        self.lens = [-1] * slots
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            self._lib.kvq_paged_destroy(h)
+            self._h = None
+
+    def _dev(self, t: torch.Tensor) -> torch.Tensor:
+        if t.dtype != self.dtype:
+            raise TypeError(f"expected {self.dtype}, got {t.dtype}")
+        if t.device != self.device:
+            t = t.to(self.device, non_blocking=True)
+        return t.contiguous()
+
+    def _grow(self, need: dict, stream):
+        """Give each slot b in `need` pages up to need[b] pages; write the new table entries."""
+        rows, cols, vals = [], [], []
+        for b, n in need.items():
+            while len(self.pages[b]) < n:
+                if not self.free_pages:
+                    raise KVQError(KVQ_ERR_CAPACITY, "the page pool is exhausted")
+                pg = self.free_pages.pop()
+                rows.append(b)
+                cols.append(len(self.pages[b]))
+                vals.append(pg)
+                self.pages[b].append(pg)
+        if vals:
+            s = torch.cuda.current_stream(self.device) if stream is None else stream
+            with torch.cuda.stream(s):
+                self.page_table[torch.tensor(rows, device=self.device), torch.tensor(cols, device=self.device)] = \
+                    torch.tensor(vals, dtype=torch.int32, device=self.device)
+
+    def seq_len(self, seq: int) -> int:
+        n = ctypes.c_int64()
+        _check(self._lib.kvq_paged_seq_len(self._h, seq, ctypes.byref(n)))
+        return int(n.value)
+
+    def splits(self) -> int:
+        return int(self._lib.kvq_paged_decode_splits(self._h))
+
+    def check_device(self):
+        """Raise KVQError if a kernel gave up a bounded wait or met a page outside the pool."""
+        _check(self._lib.kvq_paged_check_device(self._h))
+
+    def prefill(self, seq: int, X_K: torch.Tensor, X_V: torch.Tensor, stream=None):
+        X_K, X_V = self._dev(X_K), self._dev(X_V)
+        g = self.geom
+        if X_K.shape != X_V.shape or X_K.dim() != 3 or X_K.shape[0] != g.kv_heads or \
+                X_K.shape[2] != g.head_dim:
+            raise ValueError(f"X_K/X_V must be [Hkv={g.kv_heads}, T, d={g.head_dim}]")
+        T = X_K.shape[1]
+        Tq = T // g.residual * g.residual
+        if self.lens[seq] >= 0:
+            raise KVQError(KVQ_ERR_STATE, f"slot {seq} is active; release it first")
+        if Tq > g.capacity:
+            raise KVQError(KVQ_ERR_CAPACITY, f"prefill of {T} tokens exceeds capacity {g.capacity}")
+        self._grow({seq: -(-Tq // self.page_tokens)}, stream)
+        _check(self._lib.kvq_paged_prefill(self._h, seq, X_K.data_ptr(), X_V.data_ptr(), T,
+                                           _stream_ptr(stream)))
+        self.lens[seq] = T
+        self._keep = (X_K, X_V)
+        return self
+
+    def append(self, t_K: torch.Tensor, t_V: torch.Tensor, stream=None):
+        t_K, t_V = self._dev(t_K), self._dev(t_V)
+        g = self.geom
+        want = (g.batch, g.kv_heads, g.head_dim)
+        if tuple(t_K.shape) != want or tuple(t_V.shape) != want:
+            raise ValueError(f"t_K/t_V must be {list(want)}")
+        need = {}
+        for b, n in enumerate(self.lens):
+            if n >= 0 and (n + 1) % g.residual == 0 and n + 1 <= g.capacity:
+                need[b] = -(-(n + 1) // self.page_tokens)
+        self._grow(need, stream)
+        _check(self._lib.kvq_paged_append(self._h, t_K.data_ptr(), t_V.data_ptr(), _stream_ptr(stream)))
+        self.lens = [n + 1 if n >= 0 else n for n in self.lens]
+        self._keep = (t_K, t_V)
+        return self
+
+    def decode_attention(self, t_Q: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+        t_Q = self._dev(t_Q)
+        g = self.geom
+        if tuple(t_Q.shape) != (g.batch, g.q_heads, g.head_dim):
+            raise ValueError(f"t_Q must be [{g.batch}, {g.q_heads}, {g.head_dim}]")
+        if out is None:
+            out = torch.empty((g.batch, g.q_heads, g.head_dim), dtype=torch.float32, device=self.device)
+        _check(self._lib.kvq_paged_decode_attention(self._h, t_Q.data_ptr(), out.data_ptr(),
+                                                    self.workspace.data_ptr(), self.workspace.numel() * 4,
+                                                    _stream_ptr(stream)))
+        return out
+
+    def release(self, seq: int, stream=None):
+        """End slot `seq`: it becomes inactive and its pages return to the free list (reused by
+        later calls, which run after this one on the same stream)."""
+        _check(self._lib.kvq_paged_release(self._h, seq, _stream_ptr(stream)))
+        self.free_pages.extend(reversed(self.pages[seq]))
+        self.pages[seq] = []
+        self.lens[seq] = -1
+        return self
+
+
+def _gcd(a: int, b: int) -> int:
+    while b:
+        a, b = b, a % b
+    return a
 
 
 # ----------------------------------------------------------------------------

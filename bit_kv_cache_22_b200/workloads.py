@@ -26,6 +26,14 @@ on (shapes, dtypes, quantiser settings and value distributions):
                  K with 4 channels x10 per head; 256 decode steps (two residual
                  flushes at R=128); 2-bit asym G=Gv=32, or symmetric int4.
 
+A ragged batch for the paged cache (slots of different lengths, the way a
+serving system batches requests) takes one of these workloads' shapes and
+quantiser and draws each sequence's prompt length with ragged_lengths():
+
+* ``ragged_gqa`` the gqa8b geometry and distributions with 32 slots whose
+                 prompt lengths are uniform in [512, 15872] (mean 8192, the
+                 gqa8b prompt); 64 decode steps; pages of 128 tokens.
+
 Decode-step tokens follow the prompt's distribution (outlier channels
 included, sink scaling excluded) except for ``tiny``, whose appended tokens
 are plain N(0,1).  Queries are N(0,1).
@@ -39,7 +47,7 @@ import numpy as np
 FP16, BF16 = 0, 1
 
 # kinds of random streams
-_K, _V, _OUTLIER, _TK, _TV, _TQ = 0, 1, 2, 3, 4, 5
+_K, _V, _OUTLIER, _TK, _TV, _TQ, _LEN = 0, 1, 2, 3, 4, 5, 6
 
 
 @dataclasses.dataclass(frozen=True)
@@ -98,6 +106,18 @@ WORKLOADS = {
                            dtype=BF16, bits=4, G=32, Gv=32, R=128, symmetric=True, seed=4,
                            k_outlier_channels=4, k_outlier_scale=10.0),
 }
+
+
+# ragged batches: base workload, prompt-length range and page size
+RAGGED = {
+    "ragged_gqa": dict(base=WORKLOADS["gqa8b"].replace(name="ragged_gqa", seed=5), lo=512, hi=15872,
+                       page_tokens=128),
+}
+
+
+def ragged_lengths(w: Workload, lo: int, hi: int) -> list[int]:
+    """Prompt length of each of the w.B sequences, uniform integers in [lo, hi]."""
+    return [int(x) for x in _rng(w.seed, _LEN).integers(lo, hi + 1, size=w.B)]
 
 
 def _rng(*key) -> np.random.Generator:

@@ -263,6 +263,116 @@ KVQ_API int32_t kvq_decode_splits(const kvq_cache *cache);
  */
 KVQ_API kvq_status kvq_check_device(kvq_cache *cache);
 
+/*
+ * ---------------------------------------------------------------------------
+ * Paged, ragged cache: sequence slots of different lengths whose quantized tokens
+ * live in pages of one shared pool, each sequence with its own page table (the
+ * way serving systems hold KV caches: "Atom: Low-bit Quantization ...", section
+ * 六 (related work: vLLM's page tables) and Figure 3 (PageAttention)).  Every
+ * sequence is a KIVI cache of its own, with the same quantiser, residual and
+ * flush as above; only the storage is shared.
+ *
+ * Storage:
+ *  - A page holds P = page_tokens tokens of one sequence for every kv head.  The
+ *    pool's six arrays are laid out exactly like a contiguous cache whose batch is
+ *    the page number and whose capacity is P: k_codes [num_pages][Hkv][P*d*n/32],
+ *    k_scales / k_zeros [num_pages][Hkv][P/G][d], v_codes likewise, v_scales /
+ *    v_zeros [num_pages][Hkv][P][d/Gv].
+ *  - k_residual, v_residual: e [B][Hkv][R][d], one residual per slot.
+ *  - page_table: int32 [B][capacity / P], caller-owned device memory.  Entry
+ *    [b][j] is the pool page holding tokens [jP, (j+1)P) of slot b.  The library
+ *    reads it at run time and never writes it.  The caller fills entry j of slot
+ *    b, in stream order, before the first call that writes or reads one of those
+ *    tokens: a prefill (entries 0 .. ceil(Tq/P) - 1), an append whose flush
+ *    reaches a new page (entry Tq/P before the flush), every later decode.  Pages
+ *    of live slots must be distinct.  A kernel that meets an entry outside
+ *    [0, num_pages) touches page 0 instead (reads) or writes nothing (flushes)
+ *    and raises a status bit that kvq_paged_check_device reports.
+ * State: each slot is inactive (after create and release) or active with a length
+ * of len tokens (Tq = floor(len / R) R quantized, r = len mod R residual), kept
+ * on the host for planning and on the device (library-owned) for the kernels.
+ * ---------------------------------------------------------------------------
+ */
+typedef struct {
+    kvq_config geom;      /* batch = sequence slots B; capacity = quantized tokens one
+                             sequence may hold, a multiple of page_tokens           */
+    int32_t page_tokens;  /* P: a multiple of residual (R) and of 64                */
+    int32_t num_pages;    /* pages in the pool, >= 1                                */
+} kvq_paged_config;
+
+typedef struct {
+    size_t k_codes, k_scales, k_zeros;   /* the pool of num_pages pages             */
+    size_t v_codes, v_scales, v_zeros;
+    size_t k_residual, v_residual;       /* [B][Hkv][R][d] e                        */
+    size_t page_table;                   /* int32 [B][capacity / P]                 */
+    size_t workspace;                    /* scratch of kvq_paged_decode_attention   */
+} kvq_paged_sizes;
+
+typedef struct kvq_paged kvq_paged;   /* opaque host-side handle */
+
+/* Validates `cfg` and fills `out` with the buffer sizes.  No device needed. */
+KVQ_API kvq_status kvq_paged_get_sizes(const kvq_paged_config *cfg, kvq_paged_sizes *out);
+
+/*
+ * Creates a handle over the caller's pool, residual and page-table buffers (not
+ * copied, not freed); every slot starts inactive.  Like kvq_create, allocates and
+ * initialises (synchronously) a small library-owned device array: split-arrival
+ * counters, the status word and the slots' lengths.
+ */
+KVQ_API kvq_status kvq_paged_create(const kvq_paged_config *cfg, const kvq_buffers *bufs,
+                                    const int32_t *page_table, kvq_paged **out);
+
+/* Frees the handle and the library's array.  NULL is ignored. */
+KVQ_API void kvq_paged_destroy(kvq_paged *cache);
+
+/*
+ * Prefill of slot `seq` (inactive; KVQ_ERR_STATE otherwise) with the prompt
+ * X_K, X_V: e [Hkv][T][d] device tensors.  As kvq_prefill_quantize for one
+ * sequence: its first Tq = floor(T/R) R tokens are quantized into the pages of
+ * its page table, the rest copied into its residual; the slot becomes active
+ * with len = T (T = 0 allowed).  Tq > capacity gives KVQ_ERR_CAPACITY.
+ */
+KVQ_API kvq_status kvq_paged_prefill(kvq_paged *cache, int32_t seq, const void *X_K, const void *X_V,
+                                     int64_t T, void *stream);
+
+/*
+ * Decode-phase append to every active slot: t_K, t_V are e [B][Hkv][d] (rows of
+ * inactive slots are ignored).  Each active slot's row goes to its residual row r
+ * and its len grows by one; the slots whose residual becomes full (r = R) are
+ * flushed (quantized into tokens [Tq, Tq + R) of their pages).  KVQ_ERR_CAPACITY
+ * (nothing launched) if a flush would pass capacity.  One launch, plus one when
+ * any slot flushes.
+ */
+KVQ_API kvq_status kvq_paged_append(kvq_paged *cache, const void *t_K, const void *t_V, void *stream);
+
+/*
+ * Decode attention of every slot: t_Q e [B][Hq][d] -> t_O float [B][Hq][d] as
+ * kvq_decode_attention, each slot over its own tokens; an inactive or empty slot
+ * gives zeros.  `workspace`: at least kvq_paged_sizes.workspace bytes.  One
+ * launch.
+ */
+KVQ_API kvq_status kvq_paged_decode_attention(kvq_paged *cache, const void *t_Q, float *t_O,
+                                              void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Makes slot `seq` inactive (its pages are the caller's to reuse once the work
+ * queued before this call is done).  One launch (it sets the device length).
+ */
+KVQ_API kvq_status kvq_paged_release(kvq_paged *cache, int32_t seq, void *stream);
+
+/* Length of slot `seq` (-1 when inactive). */
+KVQ_API kvq_status kvq_paged_seq_len(const kvq_paged *cache, int32_t seq, int64_t *len);
+
+/* Number of token splits the next kvq_paged_decode_attention would use (>= 1). */
+KVQ_API int32_t kvq_paged_decode_splits(const kvq_paged *cache);
+
+/*
+ * As kvq_check_device, for a paged cache.  Also reports (KVQ_ERR_INVALID_ARG) a
+ * page-table entry outside the pool met by a kernel since the last check; the
+ * outputs since then are unreliable and the word is cleared.
+ */
+KVQ_API kvq_status kvq_paged_check_device(kvq_paged *cache);
+
 /* Kernels this library has launched in the process so far (all devices). */
 KVQ_API uint64_t kvq_kernel_launches(void);
 

@@ -103,3 +103,50 @@ def test_null_arguments_are_rejected_without_a_device():
         kvq.KVQ_ERR_INVALID_ARG
     assert not h.value
     assert lib.kvq_layout_version() == 2
+
+
+def _paged(page_tokens=128, num_pages=10, **kw):
+    return kvq.PagedConfig(_cfg(**kw), page_tokens, num_pages)
+
+
+def test_paged_sizes_match_layout():
+    lib = kvq.load()
+    s = kvq.PagedSizes()
+    assert lib.kvq_paged_get_sizes(ctypes.byref(_paged()), ctypes.byref(s)) == kvq.KVQ_OK
+    slices, P, d = 10 * 2, 128, 128                 # num_pages * kv_heads
+    assert s.k_codes == s.v_codes == slices * P * d * 2 // 8
+    assert s.k_scales == slices * (P // 32) * d * 4 and s.k_zeros == slices * (P // 32) * d * 2
+    assert s.v_scales == slices * P * (d // 32) * 4 and s.v_zeros == slices * P * (d // 32) * 2
+    assert s.k_residual == s.v_residual == 2 * 128 * d * 2
+    assert s.page_table == 1 * (1024 // 128) * 4
+    assert s.workspace == kvq.get_sizes(_cfg()).workspace
+
+
+@pytest.mark.parametrize("bad", [dict(page_tokens=96), dict(page_tokens=64),   # not a multiple of R = 128
+                                 dict(page_tokens=384), dict(num_pages=0),     # capacity 1024 % 384
+                                 dict(page_tokens=0), dict(head_dim=96)])
+def test_invalid_paged_configs_are_rejected(bad):
+    lib = kvq.load()
+    P = bad.pop("page_tokens", 128)
+    n = bad.pop("num_pages", 10)
+    s = kvq.PagedSizes()
+    assert lib.kvq_paged_get_sizes(ctypes.byref(_paged(P, n, **bad)), ctypes.byref(s)) != kvq.KVQ_OK
+    assert lib.kvq_last_error()
+
+
+def test_paged_null_arguments_are_rejected_without_a_device():
+    lib = kvq.load()
+    assert lib.kvq_paged_get_sizes(None, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_paged_prefill(None, 0, None, None, 0, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_paged_append(None, None, None, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_paged_decode_attention(None, None, None, None, 0, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_paged_release(None, 0, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_paged_seq_len(None, 0, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_paged_check_device(None) == kvq.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_paged_decode_splits(None) == 0
+    lib.kvq_paged_destroy(None)
+    h = ctypes.c_void_p()
+    bufs = kvq.Buffers()
+    assert lib.kvq_paged_create(ctypes.byref(_paged()), ctypes.byref(bufs), None, ctypes.byref(h)) == \
+        kvq.KVQ_ERR_INVALID_ARG
+    assert not h.value
