@@ -315,3 +315,99 @@ class OracleCache:
         return decode_attention(self.quantized(), self.Tq, self.Kr, self.Vr, self.r, Q,
                                 self.dtype, self.B, self.Hq, self.Hkv, self.d, self.G,
                                 self.Gv, self.bits, self.symmetric, stats)
+
+
+# ----------------------------------------------------------------------------
+# LogQuant retention ("Resumo Técnico: LogQuant", section 2, Estratégia de
+# Filtragem Baseada em Logaritmos, and section 4): which tokens stay in full
+# precision.  Reading taken (the summary is terse): the full-precision set F
+# holds at most 3W tokens (the 3W reserve); every new token enters F; when F
+# reaches 3W tokens, the density of its older part is halved -- of its 2W oldest
+# tokens every other one (the 2nd, 4th, ... oldest) leaves F -- which brings the
+# older part from 2W to W tokens before new tokens fill F up again.  The W
+# tokens that leave are quantized together as one block (KIVI's quantiser,
+# groups of G tokens inside the block), appended to the quantized part in the
+# order the blocks leave.  Attention runs over [dequantized blocks; F]: the
+# order of a concatenation does not change it (section 4).  Repeated halving
+# leaves F log-spaced: the newest tokens dense, older ones at strides 2, 4, ...
+# ----------------------------------------------------------------------------
+
+def logquant_step(F: list, t: int, W: int):
+    """Token position t enters F (ascending positions).  Returns the block of W
+    positions that leaves F (ascending), or None."""
+    F.append(t)
+    if len(F) < 3 * W:
+        return None
+    older = F[:2 * W]
+    dropped = older[1::2]
+    F[:] = older[0::2] + F[2 * W:]
+    return dropped
+
+
+class LogQuantCache:
+    """Prefill / append / decode with LogQuant's full-precision retention and
+    KIVI's quantiser for the tokens that leave it.  Element bits as in OracleCache;
+    every token is kept here at full precision too, to quantize it when it leaves."""
+
+    def __init__(self, B, Hq, Hkv, d, G, Gv, W, bits, symmetric=False, dtype=BF16):
+        assert W % G == 0 and d % Gv == 0 and Hq % Hkv == 0
+        self.B, self.Hq, self.Hkv, self.d = B, Hq, Hkv, d
+        self.G, self.Gv, self.W, self.bits = G, Gv, W, bits
+        self.symmetric, self.dtype = symmetric, dtype
+        BH = B * Hkv
+        self.K = np.zeros((BH, 64, d), np.uint16)     # every token so far, by position
+        self.V = np.zeros((BH, 64, d), np.uint16)
+        self.n = 0
+        self.F = []                                  # full-precision positions
+        self.block_positions = []                    # positions of each quantized block
+        self.blocks = []
+        self.Tq = 0
+
+    def _push(self, k: np.ndarray, v: np.ndarray):
+        if self.n == self.K.shape[1]:
+            self.K = np.concatenate([self.K, np.zeros_like(self.K)], axis=1)
+            self.V = np.concatenate([self.V, np.zeros_like(self.V)], axis=1)
+        self.K[:, self.n] = k
+        self.V[:, self.n] = v
+        dropped = logquant_step(self.F, self.n, self.W)
+        self.n += 1
+        if dropped is not None:
+            self.block_positions.append(dropped)
+            self.blocks.append(quantize_kv(self.K[:, dropped], self.V[:, dropped], self.dtype,
+                                           self.G, self.Gv, self.bits, self.symmetric))
+            self.Tq += self.W
+
+    def prefill(self, XK: np.ndarray, XV: np.ndarray):
+        """XK, XV element bits [B, Hkv, T, d]: the tokens enter one by one."""
+        assert self.n == 0
+        B, Hkv, T, d = XK.shape
+        XK = XK.reshape(B * Hkv, T, d)
+        XV = XV.reshape(B * Hkv, T, d)
+        for t in range(T):
+            self._push(XK[:, t], XV[:, t])
+
+    def append(self, tK: np.ndarray, tV: np.ndarray):
+        BH = self.B * self.Hkv
+        self._push(tK.reshape(BH, self.d), tV.reshape(BH, self.d))
+
+    def quantized(self) -> dict:
+        if not self.blocks:
+            BH, d = self.B * self.Hkv, self.d
+            return dict(Kq=np.zeros((BH, 0, d), np.uint8), Ks=np.zeros((BH, 0, d), np.float32),
+                        Kz=np.zeros((BH, 0, d), np.int16), Vq=np.zeros((BH, 0, d), np.uint8),
+                        Vs=np.zeros((BH, 0, d // self.Gv), np.float32),
+                        Vz=np.zeros((BH, 0, d // self.Gv), np.int16))
+        return {k: np.concatenate([b[k] for b in self.blocks], axis=1) for k in self.blocks[0]}
+
+    def packed(self) -> dict:
+        qc = self.quantized()
+        return dict(Kc=pack(qc["Kq"], self.bits, False), Vc=pack(qc["Vq"], self.bits, True),
+                    Ks=qc["Ks"], Kz=qc["Kz"], Vs=qc["Vs"], Vz=qc["Vz"])
+
+    def decode(self, Q: np.ndarray, stats: bool = False):
+        """Q element bits [B, Hq, d] -> fp64 output over [deq(blocks); F]."""
+        Kr = np.ascontiguousarray(self.K[:, self.F])
+        Vr = np.ascontiguousarray(self.V[:, self.F])
+        return decode_attention(self.quantized(), self.Tq, Kr, Vr, len(self.F), Q, self.dtype,
+                                self.B, self.Hq, self.Hkv, self.d, self.G, self.Gv, self.bits,
+                                self.symmetric, stats)
