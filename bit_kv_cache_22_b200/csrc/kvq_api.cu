@@ -108,6 +108,14 @@ struct kvq_cache {
     int num_sms = 148;
     int ctas_per_sm = 4;
     int split_limit = 64;
+    // LogQuant retention (lq_window W > 0): the residual buffer is the full-precision store
+    // of up to 3W rows (cfg.residual = 3W), rows in ascending token position; lq_F holds
+    // those positions, lq_n the tokens seen.  lq_rows (device, library-owned): [0, W) the
+    // rows an event quantizes (1, 3, ..., 2W - 1), then room for a prefill's row lists.
+    int32_t lq_window = 0;
+    int32_t *lq_rows = nullptr;
+    std::vector<int64_t> lq_F;
+    int64_t lq_n = 0;
 };
 
 namespace {
@@ -257,6 +265,22 @@ kvq::QuantizeArgs quantize_args(const kvq_cache *h) {
     return q;
 }
 
+// LogQuant host state: token lq_n enters the full-precision positions; at an event (the
+// store reached 3W) every other one of the 2W oldest leaves ("Resumo Técnico: LogQuant",
+// section 2; the same rule the kernels apply to the rows).
+void lq_push(kvq_cache *h) {
+    if (!h->lq_window) return;
+    const int64_t W = h->lq_window;
+    std::vector<int64_t> &F = h->lq_F;
+    F.push_back(h->lq_n++);
+    if (static_cast<int64_t>(F.size()) < 3 * W) return;
+    for (int64_t i = 0; i < W; ++i) F[i] = F[2 * i];
+    for (int64_t j = 0; j < W; ++j) F[W + j] = F[2 * W + j];
+    F.resize(2 * W);
+}
+
+kvq_status lq_prefill(kvq_cache *h, const void *X_K, const void *X_V, int64_t T, void *stream);
+
 kvq_status check_decode_args(const kvq_cache *h, const void *t_Q, const float *t_O, const void *workspace,
                              size_t workspace_bytes);
 kvq_status launch_decode_call(kvq_cache *h, const void *t_Q, float *t_O, void *workspace,
@@ -332,6 +356,7 @@ kvq_status kvq_create(const kvq_config *cfg, const kvq_buffers *bufs, kvq_cache 
 void kvq_destroy(kvq_cache *cache) {
     if (!cache) return;
     if (cache->arrivals) cudaFree(cache->arrivals);
+    if (cache->lq_rows) cudaFree(cache->lq_rows);
     delete cache;
 }
 
@@ -339,6 +364,8 @@ kvq_status kvq_reset(kvq_cache *cache) {
     if (!cache) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
     cache->Tq = 0;
     cache->r = 0;
+    cache->lq_F.clear();
+    cache->lq_n = 0;
     return ok();
 }
 
@@ -350,6 +377,7 @@ kvq_status kvq_prefill_quantize(kvq_cache *h, const void *X_K, const void *X_V, 
     if (T == 0) return ok();
     if (!X_K || !X_V || !aligned16(X_K) || !aligned16(X_V))
         return fail(KVQ_ERR_INVALID_ARG, "X_K and X_V must be non-NULL and 16-byte aligned");
+    if (h->lq_window) return lq_prefill(h, X_K, X_V, T, stream);
     const kvq_config &c = h->cfg;
     const int64_t Tq = (T / c.residual) * c.residual;
     const int64_t r = T - Tq;
@@ -384,7 +412,8 @@ kvq_status kvq_append(kvq_cache *h, const void *t_K, const void *t_V, void *stre
         return fail(KVQ_ERR_INVALID_ARG, "t_K and t_V must be non-NULL and 16-byte aligned");
     const kvq_config &c = h->cfg;
     const bool flush = h->r + 1 == c.residual;
-    if (flush && h->Tq + c.residual > c.capacity)
+    const int64_t flush_tokens = h->lq_window ? h->lq_window : c.residual;
+    if (flush && h->Tq + flush_tokens > c.capacity)
         return fail(KVQ_ERR_CAPACITY, "flushing the residual would exceed capacity %lld",
                     static_cast<long long>(c.capacity));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -395,7 +424,27 @@ kvq_status kvq_append(kvq_cache *h, const void *t_K, const void *t_V, void *stre
         static_cast<uint16_t *>(h->buf.k_residual), static_cast<uint16_t *>(h->buf.v_residual),
         rstride, h->r, 1, BH, c.head_dim, s);
     if (e != cudaSuccess) return cuda_fail(e, "append launch");
-    if (flush) {
+    if (flush && h->lq_window) {
+        // LogQuant event: the W rows 1, 3, ..., 2W - 1 (every other one of the 2W oldest)
+        // leave the full-precision store as one quantized block; the store is compacted
+        const int W = h->lq_window;
+        kvq::QuantizeArgs q = quantize_args(h);
+        q.xk = static_cast<const uint16_t *>(h->buf.k_residual);
+        q.xv = static_cast<const uint16_t *>(h->buf.v_residual);
+        q.in_bh_stride = rstride;
+        q.in_rows = h->lq_rows;
+        q.n_groups = W / c.group_k;
+        q.out_tok0 = h->Tq;
+        e = kvq::launch_quantize(q, s);
+        if (e == cudaSuccess)
+            e = kvq::launch_lq_compact(static_cast<uint16_t *>(h->buf.k_residual),
+                                       static_cast<uint16_t *>(h->buf.v_residual), BH, c.residual, W,
+                                       c.head_dim, s);
+        if (e != cudaSuccess) return cuda_fail(e, "LogQuant event launch");
+        lq_push(h);
+        h->Tq += W;
+        h->r = 2 * W;
+    } else if (flush) {
         kvq::QuantizeArgs q = quantize_args(h);
         q.xk = static_cast<const uint16_t *>(h->buf.k_residual);
         q.xv = static_cast<const uint16_t *>(h->buf.v_residual);
@@ -408,6 +457,7 @@ kvq_status kvq_append(kvq_cache *h, const void *t_K, const void *t_V, void *stre
         h->Tq += c.residual;
         h->r = 0;
     } else {
+        lq_push(h);
         h->r += 1;
     }
     return ok();
@@ -456,7 +506,11 @@ kvq_status kvq_append_decode_attention(kvq_cache *h, const void *t_K, const void
     h->r += 1;
     st = launch_decode_call(h, t_Q, t_O, workspace, static_cast<const uint16_t *>(t_K),
                             static_cast<const uint16_t *>(t_V), stream);
-    if (st != KVQ_OK) h->r -= 1;
+    if (st != KVQ_OK) {
+        h->r -= 1;
+        return st;
+    }
+    lq_push(h);
     return st;
 }
 
@@ -942,6 +996,136 @@ int32_t kvq_paged_decode_splits(const kvq_paged *h) {
 kvq_status kvq_paged_check_device(kvq_paged *h) {
     if (!h) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
     return check_status_word(h->base.arrivals + static_cast<int64_t>(h->base.cfg.batch) * h->base.cfg.q_heads);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// LogQuant retention ("Resumo Técnico: LogQuant", section 2, Estratégia de
+// Filtragem Baseada em Logaritmos; section 4): a cache whose full-precision
+// store holds up to 3W tokens and, whenever it fills, quantizes every other one
+// of its 2W oldest tokens as a block of W.  It is a kvq_cache whose residual
+// buffer is that store (residual = 3W); kvq_append, kvq_append_decode_attention,
+// the decode calls and kvq_cache_state (r = tokens in the store) serve it as is.
+// ---------------------------------------------------------------------------
+namespace {
+
+kvq_config lq_geometry(const kvq_config *cfg, int32_t W) {
+    kvq_config g = *cfg;
+    const int64_t R = 3 * static_cast<int64_t>(W);
+    g.residual = static_cast<int32_t>(R);
+    g.capacity = (cfg->capacity + R - 1) / R * R;
+    return g;
+}
+
+kvq_status validate_lq(const kvq_config *cfg, int32_t W) {
+    if (!cfg) return fail(KVQ_ERR_INVALID_ARG, "config is NULL");
+    if (W < 16 || W > 4096 || cfg->group_k < 1 || W % cfg->group_k != 0)
+        return fail(KVQ_ERR_INVALID_ARG, "window (%d) must be a multiple of group_k in 16..4096", W);
+    if (cfg->capacity < W || cfg->capacity % W != 0)
+        return fail(KVQ_ERR_INVALID_ARG, "capacity must be a positive multiple of the window");
+    const kvq_config g = lq_geometry(cfg, W);
+    return validate(&g);
+}
+
+kvq_status lq_prefill(kvq_cache *h, const void *X_K, const void *X_V, int64_t T, void *stream) {
+    const kvq_config &c = h->cfg;
+    const int64_t W = h->lq_window;
+    if (T > 0x7fffffffLL) return fail(KVQ_ERR_UNSUPPORTED, "T must be < 2^31");
+    // the tokens enter one by one: the blocks that leave (in the order they leave) and the
+    // positions that stay
+    std::vector<int32_t> lists;
+    std::vector<int64_t> F;
+    F.reserve(3 * W);
+    for (int64_t t = 0; t < T; ++t) {
+        F.push_back(t);
+        if (static_cast<int64_t>(F.size()) == 3 * W) {
+            for (int64_t i = 0; i < W; ++i) lists.push_back(static_cast<int32_t>(F[2 * i + 1]));
+            for (int64_t i = 0; i < W; ++i) F[i] = F[2 * i];
+            for (int64_t j = 0; j < W; ++j) F[W + j] = F[2 * W + j];
+            F.resize(2 * W);
+        }
+    }
+    const int64_t Tq = static_cast<int64_t>(lists.size());
+    if (Tq > c.capacity)
+        return fail(KVQ_ERR_CAPACITY, "prefill of %lld tokens quantizes %lld, beyond capacity %lld",
+                    static_cast<long long>(T), static_cast<long long>(Tq), static_cast<long long>(c.capacity));
+    for (int64_t p : F) lists.push_back(static_cast<int32_t>(p));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t *dev_lists = h->lq_rows + W;
+    // from pageable memory: returns once the list is staged, so the vector may go
+    cudaError_t e = cudaMemcpyAsync(dev_lists, lists.data(), lists.size() * sizeof(int32_t),
+                                    cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "uploading the prefill's row lists");
+    kvq::QuantizeArgs q = quantize_args(h);
+    q.xk = static_cast<const uint16_t *>(X_K);
+    q.xv = static_cast<const uint16_t *>(X_V);
+    q.in_bh_stride = T * c.head_dim;
+    q.in_rows = dev_lists;
+    q.n_groups = Tq / c.group_k;
+    q.out_tok0 = 0;
+    e = kvq::launch_quantize(q, s);
+    if (e != cudaSuccess) return cuda_fail(e, "LogQuant prefill quantize launch");
+    const int64_t BH = static_cast<int64_t>(c.batch) * c.kv_heads;
+    e = kvq::launch_gather_rows(static_cast<const uint16_t *>(X_K), static_cast<const uint16_t *>(X_V),
+                                T * c.head_dim, dev_lists + Tq, static_cast<int>(F.size()),
+                                static_cast<uint16_t *>(h->buf.k_residual), static_cast<uint16_t *>(h->buf.v_residual),
+                                static_cast<int64_t>(c.residual) * c.head_dim, BH, c.head_dim, s);
+    if (e != cudaSuccess) return cuda_fail(e, "LogQuant prefill store launch");
+    h->Tq = Tq;
+    h->r = static_cast<int32_t>(F.size());
+    h->lq_F = F;
+    h->lq_n = T;
+    return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_logquant_get_sizes(const kvq_config *cfg, int32_t window, kvq_sizes *out) {
+    if (!out) return fail(KVQ_ERR_INVALID_ARG, "out is NULL");
+    kvq_status st = validate_lq(cfg, window);
+    if (st != KVQ_OK) return st;
+    const kvq_config g = lq_geometry(cfg, window);
+    return kvq_get_sizes(&g, out);
+}
+
+kvq_status kvq_logquant_create(const kvq_config *cfg, int32_t window, const kvq_buffers *bufs, kvq_cache **out) {
+    if (!out) return fail(KVQ_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    kvq_status st = validate_lq(cfg, window);
+    if (st != KVQ_OK) return st;
+    const kvq_config g = lq_geometry(cfg, window);
+    kvq_cache *h = nullptr;
+    st = kvq_create(&g, bufs, &h);
+    if (st != KVQ_OK) return st;
+    h->lq_window = window;
+    h->lq_F.reserve(3 * static_cast<size_t>(window));
+    // rows 1, 3, ..., 2W - 1, then room for a prefill's lists (capacity + 3W entries)
+    const size_t n = static_cast<size_t>(window) + static_cast<size_t>(g.capacity) + 3 * static_cast<size_t>(window);
+    std::vector<int32_t> odd(static_cast<size_t>(window));
+    for (int32_t i = 0; i < window; ++i) odd[i] = 2 * i + 1;
+    cudaError_t e = cudaMalloc(&h->lq_rows, n * sizeof(int32_t));
+    if (e == cudaSuccess) e = cudaMemcpy(h->lq_rows, odd.data(), odd.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        kvq_destroy(h);
+        return cuda_fail(e, "allocating the LogQuant row lists");
+    }
+    *out = h;
+    return ok();
+}
+
+kvq_status kvq_logquant_retained(const kvq_cache *h, int64_t *positions, int32_t capacity, int32_t *count) {
+    if (!h || !count) return fail(KVQ_ERR_INVALID_ARG, "cache and count must be non-NULL");
+    if (!h->lq_window) return fail(KVQ_ERR_STATE, "not a LogQuant cache");
+    const int32_t n = static_cast<int32_t>(h->lq_F.size());
+    *count = n;
+    if (positions) {
+        if (capacity < n) return fail(KVQ_ERR_INVALID_ARG, "positions holds %d entries, %d needed", capacity, n);
+        for (int32_t i = 0; i < n; ++i) positions[i] = h->lq_F[i];
+    }
+    return ok();
 }
 
 }  // extern "C"

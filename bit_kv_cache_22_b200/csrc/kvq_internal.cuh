@@ -34,6 +34,8 @@ struct QuantizeArgs {
     const uint16_t *xk, *xv;     // e [BH][*][d]; slice stride in elements below
     int64_t in_bh_stride;        // elements between consecutive (b,h) slices
     int64_t in_tok0;             // first input token
+    const int32_t *in_rows;      // or, when non-NULL: input row of token i (device [n_groups * G]);
+                                 // in_tok0 is then unused
     int64_t n_groups;            // key groups to quantize per slice
     int64_t BH;
     int d, G, Gv, bits;
@@ -114,6 +116,15 @@ struct DecodeArgs {
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 cudaError_t launch_decode_paged(const DecodeArgs &a, cudaStream_t s);
 int decode_ctas_per_sm_paged(const DecodeArgs &a);
+// LogQuant retention event: in every (b, h) slice of the full-precision store (rows
+// [0, 3W) of `rows` rows each, ascending positions), rows 2i (i < W) move to row i and rows
+// 2W + j (j < W) to row W + j, for K and V.  One launch.
+cudaError_t launch_lq_compact(uint16_t *kr, uint16_t *vr, int64_t BH, int rows, int W, int d, cudaStream_t s);
+// dst[bh][i] = src[bh][idx[i]] for i < n, K and V (idx device [n]).  One launch.
+cudaError_t launch_gather_rows(const uint16_t *srck, const uint16_t *srcv, int64_t src_bh_stride,
+                               const int32_t *idx, int n, uint16_t *dstk, uint16_t *dstv,
+                               int64_t dst_bh_stride, int64_t BH, int d, cudaStream_t s);
+
 // Paged append: for each sequence slot b with seq_len[b] >= 0, rows t_K[b], t_V[b] ([Hkv][d])
 // become residual row seq_len[b] mod R and seq_len[b] grows by one.  One launch.
 cudaError_t launch_paged_append(const uint16_t *tk, const uint16_t *tv, uint16_t *kr, uint16_t *vr,

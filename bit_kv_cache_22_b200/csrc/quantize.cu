@@ -110,11 +110,17 @@ __device__ void pack_tiles(const uint8_t *codes, int ntiles, int d, int bits, bo
     }
 }
 
-// Copy G*d contiguous 16-bit elements into shared memory with 16-byte loads.
-__device__ void load_group(const uint16_t *src, uint16_t *dst, int n) {
-    const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+// Copy the G rows of d 16-bit elements of one group into shared memory with 16-byte
+// loads: rows tok0 .. tok0+G-1 of `slice`, or rows rows[0 .. G-1] when rows is non-NULL.
+__device__ void load_group(const uint16_t *slice, int64_t tok0, const int32_t *rows, uint16_t *dst, int G,
+                           int d) {
+    const int vec = d / 8;
     uint4 *d4 = reinterpret_cast<uint4 *>(dst);
-    for (int i = threadIdx.x; i < n / 8; i += blockDim.x) d4[i] = s4[i];
+    for (int i = threadIdx.x; i < G * vec; i += blockDim.x) {
+        const int t = i / vec, c = i - t * vec;
+        const int64_t row = rows ? rows[t] : tok0 + t;
+        d4[i] = reinterpret_cast<const uint4 *>(slice + row * d)[c];
+    }
 }
 
 __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const QuantizeArgs a) {
@@ -154,7 +160,8 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
     const int64_t groups_cap = cap / G;
 
     // ------------------------------ keys ------------------------------
-    load_group(a.xk + bh * a.in_bh_stride + in_tok * d, xs, G * d);
+    const int32_t *rows = a.in_rows ? a.in_rows + grp * G : nullptr;
+    load_group(a.xk + bh * a.in_bh_stride, in_tok, rows, xs, G, d);
     __syncthreads();
     {
         const int parts = kQuantThreads / d;         // d divides 256
@@ -210,7 +217,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
     }
 
     // ------------------------------ values ----------------------------
-    load_group(a.xv + bh * a.in_bh_stride + in_tok * d, xs, G * d);
+    load_group(a.xv + bh * a.in_bh_stride, in_tok, rows, xs, G, d);
     __syncthreads();
     {
         const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -279,6 +286,49 @@ __global__ void copy_rows_kernel(const uint16_t *src0, const uint16_t *src1, int
                                                           (src_row0 + row) * d) + v;
         uint4 *tp = reinterpret_cast<uint4 *>(dst + bh * dst_bh_stride + (dst_row0 + row) * d) + v;
         *tp = *sp;
+    }
+}
+
+// LogQuant compaction of one (b, h) slice per CTA, in place: row 2i -> row i (i < W) and
+// row 2W + j -> row W + j (j < W).  Every destination row is at or below its source, so
+// moving the rows in ascending order never overwrites a row before it is read; each
+// wave of rows is read whole before any of it is written.
+__global__ void lq_compact_kernel(uint16_t *kr, uint16_t *vr, int rows, int W, int d) {
+    const int64_t bh = blockIdx.x;
+    const int vec = d / 8;
+    const int per_wave = blockDim.x / vec;                 // destination rows per wave
+    uint4 *k4 = reinterpret_cast<uint4 *>(kr + bh * rows * d);
+    uint4 *v4 = reinterpret_cast<uint4 *>(vr + bh * rows * d);
+    const int r = threadIdx.x / vec, c = threadIdx.x % vec;
+    for (int base = 0; base < 2 * W; base += per_wave) {
+        const int dst = base + r;
+        const bool on = r < per_wave && dst < 2 * W;
+        const int src = dst < W ? 2 * dst : W + dst;
+        uint4 kx = make_uint4(0, 0, 0, 0), vx = kx;
+        if (on) {
+            kx = k4[src * vec + c];
+            vx = v4[src * vec + c];
+        }
+        __syncthreads();
+        if (on) {
+            k4[dst * vec + c] = kx;
+            v4[dst * vec + c] = vx;
+        }
+        __syncthreads();
+    }
+}
+
+__global__ void gather_rows_kernel(const uint16_t *srck, const uint16_t *srcv, int64_t src_bh_stride,
+                                   const int32_t *idx, int n, uint16_t *dstk, uint16_t *dstv,
+                                   int64_t dst_bh_stride, int64_t BH, int d) {
+    const int64_t vec = d / 8, per = BH * n * vec;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < 2 * per;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const bool isv = i >= per;
+        const int64_t k = isv ? i - per : i;
+        const int64_t v = k % vec, row = (k / vec) % n, bh = k / (vec * n);
+        const uint4 x = reinterpret_cast<const uint4 *>((isv ? srcv : srck) + bh * src_bh_stride + idx[row] * d)[v];
+        reinterpret_cast<uint4 *>((isv ? dstv : dstk) + bh * dst_bh_stride + row * d)[v] = x;
     }
 }
 
@@ -380,6 +430,29 @@ cudaError_t launch_paged_residual(const uint16_t *xk, const uint16_t *xv, int64_
     const int64_t blocks = total > 0 ? (total + 255) / 256 : 1;
     paged_residual_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(xk, xv, T, row0, rows, kr, vr, seq_len,
                                                                         seq, value, Hkv, R, d);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace kvq
+
+namespace kvq {
+
+cudaError_t launch_lq_compact(uint16_t *kr, uint16_t *vr, int64_t BH, int rows, int W, int d, cudaStream_t s) {
+    if (BH == 0) return cudaSuccess;
+    lq_compact_kernel<<<static_cast<unsigned>(BH), 256, 0, s>>>(kr, vr, rows, W, d);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(const uint16_t *srck, const uint16_t *srcv, int64_t src_bh_stride,
+                               const int32_t *idx, int n, uint16_t *dstk, uint16_t *dstv,
+                               int64_t dst_bh_stride, int64_t BH, int d, cudaStream_t s) {
+    const int64_t total = 2 * BH * n * (d / 8);
+    if (total == 0) return cudaSuccess;
+    const int64_t blocks = (total + 255) / 256;
+    gather_rows_kernel<<<static_cast<unsigned>(blocks < 65536 ? blocks : 65536), 256, 0, s>>>(
+        srck, srcv, src_bh_stride, idx, n, dstk, dstv, dst_bh_stride, BH, d);
     count_launches(1);
     return cudaGetLastError();
 }

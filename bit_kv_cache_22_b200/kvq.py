@@ -34,7 +34,8 @@ EXPORTED = ("kvq_get_sizes", "kvq_create", "kvq_destroy", "kvq_reset", "kvq_pref
             "kvq_decode_attention_partial", "kvq_merge_partials", "kvq_paged_get_sizes",
             "kvq_paged_create", "kvq_paged_destroy", "kvq_paged_prefill", "kvq_paged_append",
             "kvq_paged_decode_attention", "kvq_paged_release", "kvq_paged_seq_len",
-            "kvq_paged_decode_splits", "kvq_paged_check_device")
+            "kvq_paged_decode_splits", "kvq_paged_check_device", "kvq_logquant_get_sizes",
+            "kvq_logquant_create", "kvq_logquant_retained")
 
 
 class KVQError(RuntimeError):
@@ -130,6 +131,12 @@ def load() -> ctypes.CDLL:
         lib.kvq_paged_decode_splits.argtypes = [P]
         lib.kvq_paged_decode_splits.restype = i32
         lib.kvq_paged_check_device.argtypes = [P]
+        lib.kvq_logquant_get_sizes.argtypes = [ctypes.POINTER(Config), i32, ctypes.POINTER(Sizes)]
+        lib.kvq_logquant_create.argtypes = [ctypes.POINTER(Config), i32, ctypes.POINTER(Buffers),
+                                            ctypes.POINTER(P)]
+        lib.kvq_logquant_retained.argtypes = [P, ctypes.POINTER(i64), i32, ctypes.POINTER(i32)]
+        for name in ("kvq_logquant_get_sizes", "kvq_logquant_create", "kvq_logquant_retained"):
+            getattr(lib, name).restype = ctypes.c_int
         for name in ("kvq_paged_get_sizes", "kvq_paged_create", "kvq_paged_prefill", "kvq_paged_append",
                      "kvq_paged_decode_attention", "kvq_paged_release", "kvq_paged_seq_len",
                      "kvq_paged_check_device"):
@@ -183,9 +190,14 @@ class KVQCache:
     """
 
     def __init__(self, batch, q_heads, kv_heads, head_dim, group_k, group_v, residual, bits,
-                 symmetric=False, dtype=torch.bfloat16, capacity=None, device=None):
+                 symmetric=False, dtype=torch.bfloat16, capacity=None, device=None, window=None):
+        """window: LogQuant retention with window W instead of KIVI's residual (`residual` is
+        then ignored: the full-precision store holds up to 3W tokens)."""
         if capacity is None:
             raise ValueError("capacity (quantized tokens per sequence) is required")
+        self.window = window
+        if window:
+            residual = 3 * window
         capacity = -(-capacity // residual) * residual
         dev = torch.device(device if device is not None else "cuda")
         if dev.type != "cuda":
@@ -194,7 +206,11 @@ class KVQCache:
         self.dtype = dtype
         self.cfg = make_config(batch, q_heads, kv_heads, head_dim, group_k, group_v, residual,
                                bits, symmetric, dtype, capacity)
-        self.sizes = get_sizes(self.cfg)
+        if window:
+            self.sizes = Sizes()
+            _check(load().kvq_logquant_get_sizes(ctypes.byref(self.cfg), window, ctypes.byref(self.sizes)))
+        else:
+            self.sizes = get_sizes(self.cfg)
         BH = batch * kv_heads
         dev = self.device
         words = capacity * head_dim * bits // 32
@@ -218,7 +234,11 @@ class KVQCache:
         self._lib = load()
         h = ctypes.c_void_p()
         with torch.cuda.device(dev):
-            _check(self._lib.kvq_create(ctypes.byref(self.cfg), ctypes.byref(bufs), ctypes.byref(h)))
+            if window:
+                _check(self._lib.kvq_logquant_create(ctypes.byref(self.cfg), window, ctypes.byref(bufs),
+                                                     ctypes.byref(h)))
+            else:
+                _check(self._lib.kvq_create(ctypes.byref(self.cfg), ctypes.byref(bufs), ctypes.byref(h)))
         self._h = h
 
     # ------------------------------------------------------------------
@@ -240,6 +260,14 @@ class KVQCache:
         r = ctypes.c_int32()
         _check(self._lib.kvq_cache_state(self._h, ctypes.byref(tq), ctypes.byref(r)))
         return int(tq.value), int(r.value)
+
+    def retained(self) -> list[int]:
+        """LogQuant cache: token positions of the full-precision store's rows (ascending)."""
+        n = ctypes.c_int32()
+        _check(self._lib.kvq_logquant_retained(self._h, None, 0, ctypes.byref(n)))
+        arr = (ctypes.c_int64 * max(1, n.value))()
+        _check(self._lib.kvq_logquant_retained(self._h, arr, n.value, ctypes.byref(n)))
+        return list(arr[:n.value])
 
     def set_split_limit(self, max_splits: int):
         _check(self._lib.kvq_set_split_limit(self._h, max_splits))

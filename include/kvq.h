@@ -373,6 +373,48 @@ KVQ_API int32_t kvq_paged_decode_splits(const kvq_paged *cache);
  */
 KVQ_API kvq_status kvq_paged_check_device(kvq_paged *cache);
 
+/*
+ * ---------------------------------------------------------------------------
+ * LogQuant retention ("Resumo Técnico: LogQuant", section 2, Estratégia de
+ * Filtragem Baseada em Logaritmos, and section 4).  Instead of KIVI's residual of
+ * the newest < R tokens, a full-precision store keeps up to 3W tokens: every new
+ * token enters it; when it holds 3W, every other one of its 2W oldest tokens (the
+ * 2nd, 4th, ... oldest) leaves it and those W tokens are quantized together as
+ * one block (keys per channel over groups of G tokens inside the block, values
+ * per token), appended to the quantized tokens in the order the blocks leave.
+ * Repeated halving leaves the store log-spaced (the newest tokens dense, older
+ * ones at strides 2, 4, ...; the first token stays).  Attention runs over
+ * [deq(blocks); store], whose order does not matter.
+ *
+ * A LogQuant cache is a kvq_cache: kvq_prefill_quantize (the prompt's tokens
+ * enter one by one), kvq_append, kvq_append_decode_attention, the decode calls,
+ * kvq_cache_state (r = tokens in the store), kvq_reset and kvq_destroy serve it.
+ * Its residual buffers hold the store: e [B][Hkv][3W][d], rows in ascending
+ * token position.  The cache's capacity is rounded up to a multiple of 3W for
+ * the layout (kvq_logquant_get_sizes reports the sizes).  Its prefill uploads
+ * row lists from host memory with one copy (so it cannot be captured in a CUDA
+ * graph); append and decode can.  The library also owns a device array of
+ * (capacity + 4W) int32 row indices per LogQuant cache.
+ * ---------------------------------------------------------------------------
+ */
+
+/* Buffer sizes of a LogQuant cache with window W (W a multiple of group_k in
+ * 16..4096; cfg->residual is ignored; capacity a multiple of W). */
+KVQ_API kvq_status kvq_logquant_get_sizes(const kvq_config *cfg, int32_t window, kvq_sizes *out);
+
+/* Creates a LogQuant cache over caller-owned buffers (sizes as above). */
+KVQ_API kvq_status kvq_logquant_create(const kvq_config *cfg, int32_t window, const kvq_buffers *bufs,
+                                       kvq_cache **out);
+
+/*
+ * Token positions of the rows of the full-precision store, in row order
+ * (ascending): *count receives their number; `positions` (host, `capacity`
+ * entries, or NULL to ask for the count only) receives them.  KVQ_ERR_STATE for
+ * a cache that is not a LogQuant cache.
+ */
+KVQ_API kvq_status kvq_logquant_retained(const kvq_cache *cache, int64_t *positions, int32_t capacity,
+                                         int32_t *count);
+
 /* Kernels this library has launched in the process so far (all devices). */
 KVQ_API uint64_t kvq_kernel_launches(void);
 
