@@ -411,3 +411,110 @@ class LogQuantCache:
         return decode_attention(self.quantized(), self.Tq, Kr, Vr, len(self.F), Q, self.dtype,
                                 self.B, self.Hq, self.Hkv, self.d, self.G, self.Gv, self.bits,
                                 self.symmetric, stats)
+
+
+# ----------------------------------------------------------------------------
+# Dense-and-sparse keys ("LLM系列：KVCache量化…" pages: KVQuant, point (4)
+# Per-Vector Dense-and-Sparse Quantization -- a small share of outliers, e.g.
+# 1%, is kept at full precision in a separate sparse matrix; SqueezeLLM,
+# section (2) Dense-and-Sparse decomposition W = D + S, WX = DX + SX).
+# Reading taken: the vector is one token's key (d channels of one kv head); its
+# n_out entries of largest magnitude (ties: the lower channel first) form the
+# sparse part S and are set to +0 in the dense part D, which KIVI's quantiser
+# then quantizes as usual.  Since D holds that 0, every group that contains it
+# has min <= 0 <= max and quantizes the 0 to code z, which dequantizes to
+# exactly 0; so deq(D) + S is exact at the outliers.  Values are unchanged.
+# ----------------------------------------------------------------------------
+
+def widen_array(bits: np.ndarray, dtype: int) -> np.ndarray:
+    """Exact fp16/bf16 -> fp64 widening of a whole array (bf16: the bits are the high half of
+    an fp32; fp16 through numpy's half type)."""
+    bits = np.ascontiguousarray(bits, dtype=np.uint16)
+    if dtype == FP16:
+        return bits.view(np.float16).astype(np.float64)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def key_outliers(XK: np.ndarray, n_out: int, dtype: int):
+    """XK element bits [BH, T, d] -> (channels [BH, T, n_out], their bits, dense bits)."""
+    XK = np.ascontiguousarray(XK, dtype=np.uint16)
+    mag = np.abs(widen_array(XK, dtype))
+    order = np.argsort(-mag, axis=-1, kind="stable")[..., :n_out]   # equal magnitudes: lower channel first
+    vals = np.take_along_axis(XK, order, axis=-1)
+    dense = XK.copy()
+    np.put_along_axis(dense, order, np.uint16(0), axis=-1)
+    return order, vals, dense
+
+
+def quantize_kv_sparse(XK, XV, dtype, G, Gv, bits, symmetric=False, n_out=0) -> dict:
+    """quantize_kv of the dense keys; "Ko" holds each token's outliers as words
+    (channel << 16) | element bits, [BH, T, n_out], largest magnitude first."""
+    if n_out == 0:
+        q = quantize_kv(XK, XV, dtype, G, Gv, bits, symmetric)
+        q["Ko"] = np.zeros(XK.shape[:2] + (0,), np.uint32)
+        return q
+    idx, vals, dense = key_outliers(XK, n_out, dtype)
+    q = quantize_kv(dense, XV, dtype, G, Gv, bits, symmetric)
+    q["Ko"] = (idx.astype(np.uint32) << 16) | vals.astype(np.uint32)
+    return q
+
+
+def dequantize(qc: dict, G: int, Gv: int, bits: int, symmetric: bool, dtype: int):
+    """fp64 keys and values [BH, T, d] of a quantized block: x' = (q - z) s, plus the
+    sparse key outliers at their channels."""
+    z_sym = 1 << (bits - 1)
+    Kz = np.full(qc["Ks"].shape, z_sym) if symmetric else qc["Kz"]
+    Vz = np.full(qc["Vs"].shape, z_sym) if symmetric else qc["Vz"]
+    K = (qc["Kq"].astype(np.float64) - np.repeat(Kz, G, axis=1)) * np.repeat(qc["Ks"].astype(np.float64), G, axis=1)
+    V = (qc["Vq"].astype(np.float64) - np.repeat(Vz, Gv, axis=2)) * np.repeat(qc["Vs"].astype(np.float64), Gv, axis=2)
+    Ko = qc.get("Ko")
+    if Ko is not None and Ko.shape[-1]:
+        ch = (Ko >> 16).astype(np.int64)
+        x = widen_array((Ko & 0xFFFF).astype(np.uint16), dtype)
+        np.put_along_axis(K, ch, np.take_along_axis(K, ch, axis=-1) + x, axis=-1)
+    return K, V
+
+
+def attend(K: np.ndarray, V: np.ndarray, Q: np.ndarray, dtype: int, B: int, Hq: int, Hkv: int) -> np.ndarray:
+    """fp64 softmax(q k^T / sqrt(d)) v for queries Q bits [B, Hq, d] over K, V [B*Hkv, T, d]."""
+    d = K.shape[-1]
+    g = Hq // Hkv
+    q = widen_array(Q, dtype).reshape(B, Hkv, g, d)
+    K = K.reshape(B, Hkv, -1, d)
+    V = V.reshape(B, Hkv, -1, d)
+    s = np.einsum("bhgd,bhtd->bhgt", q, K) / np.sqrt(d)
+    s -= s.max(axis=-1, keepdims=True)
+    p = np.exp(s)
+    p /= p.sum(axis=-1, keepdims=True)
+    return np.einsum("bhgt,bhtd->bhgd", p, V).reshape(B, Hq, d)
+
+
+class SparseKeyCache(OracleCache):
+    """OracleCache whose quantized keys keep n_out sparse outliers per token."""
+
+    def __init__(self, B, Hq, Hkv, d, G, Gv, R, bits, symmetric=False, dtype=BF16, n_out=1):
+        super().__init__(B, Hq, Hkv, d, G, Gv, R, bits, symmetric, dtype)
+        self.n_out = n_out
+
+    def _quantize_block(self, XK, XV):
+        blk = quantize_kv_sparse(XK, XV, self.dtype, self.G, self.Gv, self.bits, self.symmetric, self.n_out)
+        self.blocks.append(blk)
+        self.Tq += XK.shape[1]
+        self._cat = None
+
+    def packed(self) -> dict:
+        p = super().packed()
+        qc = self.quantized()
+        p["Ko"] = qc["Ko"] if "Ko" in qc else np.zeros((self.B * self.Hkv, 0, self.n_out), np.uint32)
+        return p
+
+    def decode(self, Q: np.ndarray, stats: bool = False):
+        assert not stats
+        BH = self.B * self.Hkv
+        if self.Tq:
+            Kd, Vd = dequantize(self.quantized(), self.G, self.Gv, self.bits, self.symmetric, self.dtype)
+        else:
+            Kd = Vd = np.zeros((BH, 0, self.d))
+        K = np.concatenate([Kd, widen_array(self.Kr[:, :self.r], self.dtype)], axis=1)
+        V = np.concatenate([Vd, widen_array(self.Vr[:, :self.r], self.dtype)], axis=1)
+        return attend(K, V, Q, self.dtype, self.B, self.Hq, self.Hkv)
