@@ -1,6 +1,7 @@
 // decode.cu -- decode attention over contiguous caches, the merge of token-split
-// partials, and the dispatch between contiguous and paged caches.  The kernels are
-// in decode_kernels.cuh; decode_paged.cu holds their paged instances.
+// partials, and the dispatch between contiguous, paged and dense-and-sparse caches.
+// The kernels are in decode_kernels.cuh; decode_paged.cu and decode_sparse.cu hold
+// their other instances.
 #include "decode_kernels.cuh"
 
 namespace kvq {
@@ -41,11 +42,13 @@ cudaError_t launch_merge_partials(const float *o_all, const float *m_all, const 
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
     if (a.page_table) return launch_decode_paged(a, s);
+    if (a.k_out) return launch_decode_sparse(a, s);
     return launch_decode_variant<false>(a, s);
 }
 
 int decode_ctas_per_sm(const DecodeArgs &a) {
     if (a.page_table) return decode_ctas_per_sm_paged(a);
+    if (a.k_out) return decode_ctas_per_sm_sparse(a);
     return ctas_per_sm_variant<false>(a);
 }
 

@@ -967,7 +967,7 @@ __device__ __forceinline__ int logit_pos(int t) { return 4 * (t >> 2) + 2 * (t &
 template <int D, int GV, int HG>
 __host__ __device__ constexpr int tc_min_ctas() { return 4; }
 
-template <int N, int D, int GV, int HG, bool PAGED>
+template <int N, int D, int GV, int HG, bool PAGED, bool SPARSE>
 __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) decode_tc_kernel(const DecodeArgs a) {
     constexpr int W = D * N / 64;
     constexpr int TW = D * N / 2;
@@ -1359,6 +1359,17 @@ __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) deco
                     if ((u == 0 && open0) || (u == 2 && open2))
                         rebuild_key_digits(reinterpret_cast<const float *>(st + St::kMeta) + (u == 2 ? D : 0),
                                            reinterpret_cast<const int16_t *>(st + St::kKz) + (u == 2 ? D : 0));
+                    uint32_t ko[2][2] = {};   // dense-and-sparse keys: outlier words of tokens g8, g8 + 8
+                    if constexpr (SPARSE) {
+                        const int64_t tok = (bh * (a.cap / 16) + wb + rel + u) * 16 + g8;
+#pragma unroll
+                        for (int o = 0; o < 2; ++o) {
+                            if (o < a.n_out) {
+                                ko[0][o] = __ldg(a.k_out + tok * a.n_out + o);
+                                ko[1][o] = __ldg(a.k_out + (tok + 8) * a.n_out + o);
+                            }
+                        }
+                    }
                     uint32_t kw[W];
                     load_lane_words<W>(st + u * St::kCodes, lane, kw);
                     int acc[NTK][2][BPW][4];   // two chains (even / odd word pair) per n-tile
@@ -1424,7 +1435,16 @@ __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) deco
                         x0 += __shfl_xor_sync(0xffffffffu, x0, 2);
                         x1 += __shfl_xor_sync(0xffffffffu, x1, 2);
                     }
-                    const float lg0 = x0 - kbias, lg1 = x1 - kbias;
+                    float lg0 = x0 - kbias, lg1 = x1 - kbias;
+                    if constexpr (SPARSE) {   // the outliers' q_c x_c (the dense part is 0 there)
+#pragma unroll
+                        for (int o = 0; o < 2; ++o) {
+                            if (o < a.n_out) {
+                                lg0 = fmaf(q_s[hown][ko[0][o] >> 16], widen(ko[0][o] & 0xffffu, a.bf16), lg0);
+                                lg1 = fmaf(q_s[hown][ko[1][o] >> 16], widen(ko[1][o] & 0xffffu, a.bf16), lg1);
+                            }
+                        }
+                    }
                     mloc = fmaxf(mloc, fmaxf(lg0, lg1));
                     if (t4 < HG) {
                         lgc[(u * HG + hown) * 16 + logit_pos(g8)] = lg0;
@@ -1595,12 +1615,12 @@ int occupancy_of(int smem) {
 // The split index is the slowest grid dimension: CTAs start in linear order, so every
 // quantized split is resident before the (short) residual-split CTAs fill the slots
 // that remain.
-template <int N, int D, int GV, bool PAGED>
+template <int N, int D, int GV, bool PAGED, bool SPARSE>
 struct LaunchF {
     template <int HG>
     static cudaError_t tc(const DecodeArgs &a, cudaStream_t s) {
-        return launch_kernel<decode_tc_kernel<N, D, GV, HG, PAGED>>(a, dim3(a.Hkv, a.B, a.S),
-                                                                    tc_smem<N, D, GV, HG>(), s);
+        return launch_kernel<decode_tc_kernel<N, D, GV, HG, PAGED, SPARSE>>(a, dim3(a.Hkv, a.B, a.S),
+                                                                            tc_smem<N, D, GV, HG>(), s);
     }
     static cudaError_t run(const DecodeArgs &a, cudaStream_t s) {
         if (a.path == kPathTc) {
@@ -1611,59 +1631,64 @@ struct LaunchF {
                 default: return cudaErrorInvalidValue;
             }
         }
-        return launch_kernel<decode_split_kernel<N, D, GV, PAGED>>(a, dim3(a.Hq, a.B, a.S),
-                                                                   split_smem<N, D, GV>(), s);
+        if constexpr (SPARSE) {
+            return cudaErrorInvalidValue;   // dense-and-sparse keys run on the tensor-core path only
+        } else {
+            return launch_kernel<decode_split_kernel<N, D, GV, PAGED>>(a, dim3(a.Hq, a.B, a.S),
+                                                                       split_smem<N, D, GV>(), s);
+        }
     }
     static int occ(const DecodeArgs &a) {
         if (a.path == kPathTc) {
             switch (a.Hq / a.Hkv) {
-                case 1: return occupancy_of<decode_tc_kernel<N, D, GV, 1, PAGED>>(tc_smem<N, D, GV, 1>());
-                case 2: return occupancy_of<decode_tc_kernel<N, D, GV, 2, PAGED>>(tc_smem<N, D, GV, 2>());
-                case 4: return occupancy_of<decode_tc_kernel<N, D, GV, 4, PAGED>>(tc_smem<N, D, GV, 4>());
+                case 1: return occupancy_of<decode_tc_kernel<N, D, GV, 1, PAGED, SPARSE>>(tc_smem<N, D, GV, 1>());
+                case 2: return occupancy_of<decode_tc_kernel<N, D, GV, 2, PAGED, SPARSE>>(tc_smem<N, D, GV, 2>());
+                case 4: return occupancy_of<decode_tc_kernel<N, D, GV, 4, PAGED, SPARSE>>(tc_smem<N, D, GV, 4>());
                 default: return 1;
             }
         }
-        return occupancy_of<decode_split_kernel<N, D, GV, PAGED>>(split_smem<N, D, GV>());
+        if constexpr (SPARSE) return 1;
+        else return occupancy_of<decode_split_kernel<N, D, GV, PAGED>>(split_smem<N, D, GV>());
     }
 };
 
-template <int N, int D, bool PAGED>
+template <int N, int D, bool PAGED, bool SPARSE>
 cudaError_t launch_gv(const DecodeArgs &a, cudaStream_t s) {
     switch (a.Gv) {
-        case 16: return LaunchF<N, D, 16, PAGED>::run(a, s);
-        case 32: return LaunchF<N, D, 32, PAGED>::run(a, s);
-        case 64: return LaunchF<N, D, 64, PAGED>::run(a, s);
-        default: if constexpr (D >= 128) { if (a.Gv == 128) return LaunchF<N, D, 128, PAGED>::run(a, s); }
+        case 16: return LaunchF<N, D, 16, PAGED, SPARSE>::run(a, s);
+        case 32: return LaunchF<N, D, 32, PAGED, SPARSE>::run(a, s);
+        case 64: return LaunchF<N, D, 64, PAGED, SPARSE>::run(a, s);
+        default: if constexpr (D >= 128) { if (a.Gv == 128) return LaunchF<N, D, 128, PAGED, SPARSE>::run(a, s); }
     }
     return cudaErrorInvalidValue;
 }
 
-template <int N, int D, bool PAGED>
+template <int N, int D, bool PAGED, bool SPARSE>
 int occ_gv(const DecodeArgs &a) {
     switch (a.Gv) {
-        case 16: return LaunchF<N, D, 16, PAGED>::occ(a);
-        case 32: return LaunchF<N, D, 32, PAGED>::occ(a);
-        case 64: return LaunchF<N, D, 64, PAGED>::occ(a);
-        default: if constexpr (D >= 128) { if (a.Gv == 128) return LaunchF<N, D, 128, PAGED>::occ(a); }
+        case 16: return LaunchF<N, D, 16, PAGED, SPARSE>::occ(a);
+        case 32: return LaunchF<N, D, 32, PAGED, SPARSE>::occ(a);
+        case 64: return LaunchF<N, D, 64, PAGED, SPARSE>::occ(a);
+        default: if constexpr (D >= 128) { if (a.Gv == 128) return LaunchF<N, D, 128, PAGED, SPARSE>::occ(a); }
     }
     return 1;
 }
 
-template <bool PAGED>
+template <bool PAGED, bool SPARSE = false>
 cudaError_t launch_decode_variant(const DecodeArgs &a, cudaStream_t s) {
-    if (a.bits == 2 && a.d == 64) return launch_gv<2, 64, PAGED>(a, s);
-    if (a.bits == 2 && a.d == 128) return launch_gv<2, 128, PAGED>(a, s);
-    if (a.bits == 4 && a.d == 64) return launch_gv<4, 64, PAGED>(a, s);
-    if (a.bits == 4 && a.d == 128) return launch_gv<4, 128, PAGED>(a, s);
+    if (a.bits == 2 && a.d == 64) return launch_gv<2, 64, PAGED, SPARSE>(a, s);
+    if (a.bits == 2 && a.d == 128) return launch_gv<2, 128, PAGED, SPARSE>(a, s);
+    if (a.bits == 4 && a.d == 64) return launch_gv<4, 64, PAGED, SPARSE>(a, s);
+    if (a.bits == 4 && a.d == 128) return launch_gv<4, 128, PAGED, SPARSE>(a, s);
     return cudaErrorInvalidValue;
 }
 
-template <bool PAGED>
+template <bool PAGED, bool SPARSE = false>
 int ctas_per_sm_variant(const DecodeArgs &a) {
-    if (a.bits == 2 && a.d == 64) return occ_gv<2, 64, PAGED>(a);
-    if (a.bits == 2 && a.d == 128) return occ_gv<2, 128, PAGED>(a);
-    if (a.bits == 4 && a.d == 64) return occ_gv<4, 64, PAGED>(a);
-    if (a.bits == 4 && a.d == 128) return occ_gv<4, 128, PAGED>(a);
+    if (a.bits == 2 && a.d == 64) return occ_gv<2, 64, PAGED, SPARSE>(a);
+    if (a.bits == 2 && a.d == 128) return occ_gv<2, 128, PAGED, SPARSE>(a);
+    if (a.bits == 4 && a.d == 64) return occ_gv<4, 64, PAGED, SPARSE>(a);
+    if (a.bits == 4 && a.d == 128) return occ_gv<4, 128, PAGED, SPARSE>(a);
     return 1;
 }
 

@@ -114,6 +114,9 @@ struct kvq_cache {
     // rows an event quantizes (1, 3, ..., 2W - 1), then room for a prefill's row lists.
     int32_t lq_window = 0;
     int32_t *lq_rows = nullptr;
+    // dense-and-sparse keys: n_out outlier words per token (caller-owned), or none
+    uint32_t *k_out = nullptr;
+    int32_t n_out = 0;
     std::vector<int64_t> lq_F;
     int64_t lq_n = 0;
 };
@@ -239,6 +242,8 @@ kvq::DecodeArgs decode_args(const kvq_cache *h) {
     a.path = kvq::decode_path(c.q_heads, c.kv_heads, c.group_k);
     a.arrivals = h->arrivals;
     a.status = h->arrivals + static_cast<int64_t>(c.batch) * c.q_heads;
+    a.k_out = h->k_out;
+    a.n_out = h->n_out;
     a.gshift = 0;
     while ((16 << a.gshift) < c.group_k) ++a.gshift;
     a.qscale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c.head_dim)));
@@ -262,6 +267,8 @@ kvq::QuantizeArgs quantize_args(const kvq_cache *h) {
     q.kz = h->buf.k_zeros;
     q.vz = h->buf.v_zeros;
     q.cap = c.capacity;
+    q.k_out = h->k_out;
+    q.n_out = h->n_out;
     return q;
 }
 
@@ -1125,6 +1132,34 @@ kvq_status kvq_logquant_retained(const kvq_cache *h, int64_t *positions, int32_t
         if (capacity < n) return fail(KVQ_ERR_INVALID_ARG, "positions holds %d entries, %d needed", capacity, n);
         for (int32_t i = 0; i < n; ++i) positions[i] = h->lq_F[i];
     }
+    return ok();
+}
+
+}  // extern "C"
+
+extern "C" {
+
+kvq_status kvq_set_key_outliers(kvq_cache *h, int32_t n_out, uint32_t *k_outliers, size_t bytes) {
+    if (!h) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+    if (h->Tq != 0 || h->r != 0) return fail(KVQ_ERR_STATE, "key outliers are set on an empty cache");
+    if (n_out < 0 || n_out > 2) return fail(KVQ_ERR_INVALID_ARG, "n_out must be 0, 1 or 2");
+    const kvq_config &c = h->cfg;
+    if (n_out == 0) {
+        h->k_out = nullptr;
+        h->n_out = 0;
+        h->ctas_per_sm = kvq::decode_ctas_per_sm(decode_args(h));
+        return ok();
+    }
+    if (kvq::decode_path(c.q_heads, c.kv_heads, c.group_k) != kvq::kPathTc)
+        return fail(KVQ_ERR_UNSUPPORTED, "dense-and-sparse keys need 1, 2 or 4 query heads per kv head "
+                                         "and key groups of >= 32 tokens");
+    const size_t need = static_cast<size_t>(c.batch) * c.kv_heads * static_cast<size_t>(c.capacity) * n_out * 4;
+    if (!k_outliers || !aligned16(k_outliers))
+        return fail(KVQ_ERR_INVALID_ARG, "k_outliers must be non-NULL and 16-byte aligned");
+    if (bytes < need) return fail(KVQ_ERR_INVALID_ARG, "k_outliers needs %zu bytes, got %zu", need, bytes);
+    h->k_out = k_outliers;
+    h->n_out = n_out;
+    h->ctas_per_sm = kvq::decode_ctas_per_sm(decode_args(h));
     return ok();
 }
 

@@ -53,6 +53,11 @@ struct QuantizeArgs {
     const int32_t *seq_len;      // flush: tokens of each sequence after the append; only those
                                  // at a multiple of R flush, to tokens [len - R, len)
     unsigned int *status;        // bit 2 raised for a page number outside the pool
+    // dense-and-sparse keys (k_out non-NULL): each token's n_out largest-magnitude key
+    // entries leave the dense part (set to +0 before quantizing) and are written as words
+    // (channel << 16) | element bits to k_out [slice][cap][n_out], largest first
+    uint32_t *k_out;
+    int n_out;
 };
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s);
 
@@ -112,10 +117,16 @@ struct DecodeArgs {
     const int32_t *seq_len;      // [B]
     int page_tiles;              // P / 16
     int max_pages, num_pages;
+    // dense-and-sparse keys (contiguous caches, tensor-core path): outlier words
+    // [BH][cap][n_out] as written by the quantizer, or NULL
+    const uint32_t *k_out;
+    int n_out;
 };
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 cudaError_t launch_decode_paged(const DecodeArgs &a, cudaStream_t s);
 int decode_ctas_per_sm_paged(const DecodeArgs &a);
+cudaError_t launch_decode_sparse(const DecodeArgs &a, cudaStream_t s);
+int decode_ctas_per_sm_sparse(const DecodeArgs &a);
 // LogQuant retention event: in every (b, h) slice of the full-precision store (rows
 // [0, 3W) of `rows` rows each, ascending positions), rows 2i (i < W) move to row i and rows
 // 2W + j (j < W) to row W + j, for K and V.  One launch.

@@ -163,6 +163,39 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
     const int32_t *rows = a.in_rows ? a.in_rows + grp * G : nullptr;
     load_group(a.xk + bh * a.in_bh_stride, in_tok, rows, xs, G, d);
     __syncthreads();
+    if (a.n_out > 0) {
+        // dense-and-sparse keys: per token, the n_out entries of largest magnitude (ties: the
+        // lower channel) are written as outlier words and set to +0 in the dense part
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        const int per_lane = d / 32;                 // 2 or 4
+        for (int t = warp; t < G; t += kQuantThreads / 32) {
+            uint32_t mag[4];
+            for (int e = 0; e < per_lane; ++e)
+                mag[e] = __float_as_uint(fabsf(widen(xs[t * d + lane * per_lane + e], a.bf16)));
+            unsigned picked = 0;
+            for (int o = 0; o < a.n_out; ++o) {
+                uint64_t best = 0;   // (|x| bits << 16) | (0xffff - channel): the larger key wins
+                for (int e = 0; e < per_lane; ++e) {
+                    const uint64_t key = (static_cast<uint64_t>(mag[e]) << 16) |
+                                         static_cast<uint64_t>(0xffff - (lane * per_lane + e));
+                    if (!((picked >> e) & 1u) && key > best) best = key;
+                }
+                for (int off = 16; off > 0; off >>= 1) {
+                    const uint64_t other = __shfl_xor_sync(0xffffffffu, best, off);
+                    best = other > best ? other : best;
+                }
+                const int c = 0xffff - static_cast<int>(best & 0xffffu);
+                if (c / per_lane == lane) picked |= 1u << (c % per_lane);
+                if (lane == 0)
+                    a.k_out[(slice * cap + out_tok + t) * a.n_out + o] =
+                        (static_cast<uint32_t>(c) << 16) | xs[t * d + c];
+            }
+            __syncwarp();    // every lane has read the chosen elements' bits
+            for (int e = 0; e < per_lane; ++e)
+                if ((picked >> e) & 1u) xs[t * d + lane * per_lane + e] = 0;
+        }
+        __syncthreads();
+    }
     {
         const int parts = kQuantThreads / d;         // d divides 256
         const int c = threadIdx.x % d;

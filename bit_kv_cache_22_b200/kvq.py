@@ -35,7 +35,7 @@ EXPORTED = ("kvq_get_sizes", "kvq_create", "kvq_destroy", "kvq_reset", "kvq_pref
             "kvq_paged_create", "kvq_paged_destroy", "kvq_paged_prefill", "kvq_paged_append",
             "kvq_paged_decode_attention", "kvq_paged_release", "kvq_paged_seq_len",
             "kvq_paged_decode_splits", "kvq_paged_check_device", "kvq_logquant_get_sizes",
-            "kvq_logquant_create", "kvq_logquant_retained")
+            "kvq_logquant_create", "kvq_logquant_retained", "kvq_set_key_outliers")
 
 
 class KVQError(RuntimeError):
@@ -135,7 +135,9 @@ def load() -> ctypes.CDLL:
         lib.kvq_logquant_create.argtypes = [ctypes.POINTER(Config), i32, ctypes.POINTER(Buffers),
                                             ctypes.POINTER(P)]
         lib.kvq_logquant_retained.argtypes = [P, ctypes.POINTER(i64), i32, ctypes.POINTER(i32)]
-        for name in ("kvq_logquant_get_sizes", "kvq_logquant_create", "kvq_logquant_retained"):
+        lib.kvq_set_key_outliers.argtypes = [P, i32, P, sz]
+        for name in ("kvq_logquant_get_sizes", "kvq_logquant_create", "kvq_logquant_retained",
+                     "kvq_set_key_outliers"):
             getattr(lib, name).restype = ctypes.c_int
         for name in ("kvq_paged_get_sizes", "kvq_paged_create", "kvq_paged_prefill", "kvq_paged_append",
                      "kvq_paged_decode_attention", "kvq_paged_release", "kvq_paged_seq_len",
@@ -190,9 +192,12 @@ class KVQCache:
     """
 
     def __init__(self, batch, q_heads, kv_heads, head_dim, group_k, group_v, residual, bits,
-                 symmetric=False, dtype=torch.bfloat16, capacity=None, device=None, window=None):
+                 symmetric=False, dtype=torch.bfloat16, capacity=None, device=None, window=None,
+                 key_outliers=0):
         """window: LogQuant retention with window W instead of KIVI's residual (`residual` is
-        then ignored: the full-precision store holds up to 3W tokens)."""
+        then ignored: the full-precision store holds up to 3W tokens).  key_outliers: keep that
+        many largest-magnitude entries of each token's key as sparse full-precision outliers
+        (dense-and-sparse keys; 1 or 2)."""
         if capacity is None:
             raise ValueError("capacity (quantized tokens per sequence) is required")
         self.window = window
@@ -240,6 +245,12 @@ class KVQCache:
             else:
                 _check(self._lib.kvq_create(ctypes.byref(self.cfg), ctypes.byref(bufs), ctypes.byref(h)))
         self._h = h
+        self.key_outliers = key_outliers
+        self.k_outliers = None
+        if key_outliers:
+            self.k_outliers = torch.empty((BH, capacity, key_outliers), dtype=torch.int32, device=dev)
+            _check(self._lib.kvq_set_key_outliers(h, key_outliers, self.k_outliers.data_ptr(),
+                                                  self.k_outliers.numel() * 4))
 
     # ------------------------------------------------------------------
     def __del__(self):

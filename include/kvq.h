@@ -415,6 +415,29 @@ KVQ_API kvq_status kvq_logquant_create(const kvq_config *cfg, int32_t window, co
 KVQ_API kvq_status kvq_logquant_retained(const kvq_cache *cache, int64_t *positions, int32_t capacity,
                                          int32_t *count);
 
+/*
+ * Dense-and-sparse keys (the KV-cache quantization pages: KVQuant's per-vector
+ * dense-and-sparse quantization keeps a small share of outliers, e.g. 1%, at
+ * full precision in a separate sparse matrix; SqueezeLLM's W = D + S).  For each
+ * token's key (d channels of one kv head) the n_out entries of largest magnitude
+ * (ties: the lower channel) form the sparse part; they are set to +0 in the
+ * dense part, which is quantized as usual.  The 0 quantizes to its group's zero
+ * point and dequantizes to exactly 0, so the reconstruction deq(D) + S is exact
+ * at the outliers; the decode adds q_c x_c of each outlier to its token's logit.
+ * Values are unchanged.
+ *
+ * Enables this on an empty cache (KVQ_ERR_STATE otherwise) of the tensor-core
+ * path: 1, 2 or 4 query heads per kv head and key groups of >= 32 tokens
+ * (KVQ_ERR_UNSUPPORTED otherwise); not for paged caches.  n_out: 1 or 2 (about
+ * 1% or 2% of d = 128); 0 turns it off.  k_outliers: caller-owned device memory
+ * of at least `bytes` = B * Hkv * capacity * n_out * 4 bytes (capacity as in the
+ * cache's sizes; a LogQuant cache's is rounded up to a multiple of 3W), holding
+ * uint32 [B][Hkv][capacity][n_out]: per quantized token its outliers, largest
+ * first, each (channel << 16) | element bits.  Applies to every later prefill,
+ * flush (and LogQuant block) of this cache.
+ */
+KVQ_API kvq_status kvq_set_key_outliers(kvq_cache *cache, int32_t n_out, uint32_t *k_outliers, size_t bytes);
+
 /* Kernels this library has launched in the process so far (all devices). */
 KVQ_API uint64_t kvq_kernel_launches(void);
 
