@@ -51,6 +51,10 @@ def _args():
                    help="run one prefill and up to 64 decode steps of the workload, then exit (for ncu)")
     p.add_argument("--paged", default=None, metavar="RAGGED_WORKLOAD",
                    help="measure the paged, ragged cache on this ragged batch (e.g. ragged_gqa) instead")
+    p.add_argument("--window", type=int, default=0,
+                   help="measure LogQuant retention with this window W on the workload instead")
+    p.add_argument("--key-outliers", type=int, default=0,
+                   help="dense-and-sparse keys: keep this many outliers per token (1 or 2)")
     return p.parse_args()
 
 
@@ -217,7 +221,7 @@ def run_kvq(args):
     XK, XV = to_t(XK_h).to(dev), to_t(XV_h).to(dev)
     tK, tV, tQ = to_t(tK_h).to(dev), to_t(tV_h).to(dev), to_t(tQ_h).to(dev)
     cache = kvq.KVQCache(w.B, w.Hq, w.Hkv, w.d, w.G, w.Gv, w.R, w.bits, w.symmetric, dt,
-                         w.capacity, dev)
+                         w.capacity, dev, key_outliers=args.key_outliers)
     out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -232,6 +236,7 @@ def run_kvq(args):
     ctx = episode_contexts(w)
     tokens_per_episode = sum(w.B * (tq + r) for tq, r in ctx)
     bytes_per_episode = sum(algorithmic_bytes(w, tq, r) for tq, r in ctx)
+    bytes_per_episode += sum(w.B * w.Hkv * tq * 4 * args.key_outliers for tq, r in ctx)   # outlier words
 
     def episode():
         cache.reset()
@@ -383,7 +388,7 @@ def run_kvq(args):
             "workload": w.name, "batch_per_gpu": w.B, "global_batch": w.B * world,
             "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d, "prompt_tokens": w.T,
             "decode_steps": w.steps, "bits": w.bits, "group_k": w.G, "group_v": w.Gv,
-            "residual": w.R, "symmetric": w.symmetric,
+            "residual": w.R, "symmetric": w.symmetric, "key_outliers_per_token": args.key_outliers,
             "elem": "fp16" if w.dtype == wl.FP16 else "bf16",
             "parallelism": f"dp{world} (independent sequences per GPU)",
             "l2": "inputs larger than L2: packed cache "
@@ -419,6 +424,115 @@ def run_kvq(args):
 # ---------------------------------------------------------------------------
 # the paged, ragged cache
 # ---------------------------------------------------------------------------
+
+def run_logquant(args):
+    """Decode attention with LogQuant retention (window W) on the workload's batch: the
+    prompt's prefill (eager: it uploads row lists), then per decode step an eager append and
+    the step's decode_attention graph replayed `--steps` times between two events.  value =
+    KV tokens attended per second of decode time; the roofline counts the quantized tokens'
+    bytes and the full-precision store's rows."""
+    import torch
+
+    from bit_kv_cache_22_b200 import kvq
+    from bit_kv_cache_22_b200 import workloads as wl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
+    w = shard_workload(wl.WORKLOADS[args.workload], rank)
+    W = args.window
+    dt = torch.float16 if w.dtype == wl.FP16 else torch.bfloat16
+
+    def to_t(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(dt).to(dev)
+
+    cap = -(-(w.T + w.steps) // W) * W
+    cache = kvq.KVQCache(w.B, w.Hq, w.Hkv, w.d, w.G, w.Gv, w.R, w.bits, w.symmetric, dt, cap, dev,
+                         window=W, key_outliers=args.key_outliers)
+    XK, XV = wl.prefill_bits(w)
+    cache.prefill_quantize(to_t(XK), to_t(XV))
+    del XK, XV
+    tK, tV, tQ = (to_t(x) for x in wl.decode_bits(w))
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    pool = torch.cuda.graph_pool_handle()
+    total_ms, total_tokens, total_bytes, launches = 0.0, 0, 0, 0
+    with ClockSampler(local) as clk:
+        for s in range(w.steps):
+            cache.append(tK[s], tV[s])
+            torch.cuda.synchronize()
+            l0 = kvq.kernel_launches()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, pool=pool):
+                cache.decode_attention(tQ[s], out=out)
+            per_call = kvq.kernel_launches() - l0
+            for _ in range(max(1, args.warmup)):
+                g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            total_ms += e0.elapsed_time(e1)
+            launches += per_call * args.steps
+            tq, r = cache.state()
+            total_tokens += w.B * (tq + r) * args.steps
+            total_bytes += (algorithmic_bytes(w, tq, r) + w.B * w.Hkv * tq * 4 * args.key_outliers) * args.steps
+            del g
+    ms, = max_over_ranks([total_ms], world, dev)
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+    calls = w.steps * args.steps
+    peak, peak_kind = peaks()
+    achieved = total_bytes / (total_ms / 1e3) / 1e9
+    tq, r = cache.state()
+    line = {
+        "metric": METRIC, "value": job_throughput(total_tokens, world, ms), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / calls,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": f"u{w.bits} codes, f32 accumulate",
+        "data": "synthetic (seeded; distributions of the workload definition)",
+        "config": {
+            "workload": f"{w.name} (LogQuant retention, W={W})", "batch_per_gpu": w.B, "q_heads": w.Hq,
+            "kv_heads": w.Hkv, "head_dim": w.d, "prompt_tokens": w.T, "decode_steps": w.steps,
+            "bits": w.bits, "group_k": w.G, "group_v": w.Gv, "window": W,
+            "key_outliers_per_token": args.key_outliers, "full_precision_rows_at_end": r,
+            "elem": "fp16" if w.dtype == wl.FP16 else "bf16", "parallelism": f"dp{world}",
+            "l2": "inputs larger than L2: packed cache "
+                  f"{total_bytes / calls / 1e6:.0f} MB per decode call",
+            "splits": cache.splits(),
+            "timing": "per decode step: its decode_attention graph replayed --steps times between "
+                      "two events (decode time only; appends run eagerly between)",
+        },
+        "roofline": {
+            "kernel": f"decode_attention ({decode_kernel_name(w)}) over a LogQuant cache, per call",
+            "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+            else "fallback 6.65 TB/s",
+            "algorithmic_bytes_per_launch": total_bytes / calls, "avg_launch_us": total_ms / calls * 1e3,
+            "traffic": None,
+        },
+        "cpu_baseline": None,
+        "e2e": None,
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+
 
 def run_paged(args):
     """Decode attention of a ragged batch held in a paged cache.  After the prompts'
@@ -591,6 +705,8 @@ def main():
         run_reference(args)
     elif args.paged:
         run_paged(args)
+    elif args.window:
+        run_logquant(args)
     else:
         run_kvq(args)
 
