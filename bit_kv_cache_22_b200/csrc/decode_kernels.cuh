@@ -1029,14 +1029,17 @@ __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) deco
 
     if constexpr (HG > 1) {
         if (sigma >= a.n_qsplits) {
-            // ---------------- residual split: kDecodeWarps / HG warps per head ----------------
+            // ---------------- residual splits: kDecodeWarps / HG warps per head in each; the
+            //                  residual tiles are dealt round-robin over the warps of all of them ----
             constexpr int WPH = kDecodeWarps / HG;
             const int h = warp / WPH;
+            const int rs = sigma - a.n_qsplits, nrs = a.S - a.n_qsplits;
             float m = -INFINITY, lsum = 0.f;
             float2 acc[NJ][2];
 #pragma unroll
             for (int j = 0; j < NJ; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
-            residual_pass<D>(a, bh, r_rows, q_s[h], warp % WPH, (r_rows + 15) / 16, lane, m, lsum, acc, wmem, WPH);
+            residual_pass<D>(a, bh, r_rows, q_s[h], rs * WPH + warp % WPH, (r_rows + 15) / 16, lane, m, lsum, acc,
+                             wmem, WPH * nrs);
             lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
             lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
             lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);

@@ -53,6 +53,7 @@ kvq_status cuda_fail(cudaError_t e, const char *what) {
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 constexpr int kMaxSplits = 64;
+constexpr int kMaxResidualSplits = 16;
 constexpr int kMinTilesPerSplit = 4;
 
 kvq_status validate(const kvq_config *c) {
@@ -91,10 +92,11 @@ kvq_status validate(const kvq_config *c) {
     return KVQ_OK;
 }
 
-// Splits over the quantized tiles are at most kMaxSplits; the residual adds one.
+// Splits over the quantized tiles are at most kMaxSplits; the residual rows add up to
+// kMaxResidualSplits.
 int max_splits(const kvq_config *c) {
     const int64_t tiles = c->capacity / 16;
-    return static_cast<int>(tiles < kMaxSplits ? tiles : kMaxSplits) + 1;
+    return static_cast<int>(tiles < kMaxSplits ? tiles : kMaxSplits) + kMaxResidualSplits;
 }
 
 }  // namespace
@@ -156,7 +158,8 @@ void plan_splits_for(const kvq_cache *h, const PlanInput &in, int *n_qsplits, in
     // warps of the quantized splits
     const int hg = c.q_heads / c.kv_heads;
     const bool res_shared = path == kvq::kPathTc && hg == 1;
-    const int extra = (in.max_r > 0 && !res_shared) ? 1 : 0;
+    const int extra = (in.max_r > 0 && !res_shared) ? 1 : 0;   // residual splits (the tensor-core
+                                                                // path may take more, below)
     const int64_t align = kvq::split_tile_align(path);
     // CTAs per split and sequence: one per kv head on the tensor-core path, else one per query head
     const int64_t per_seq = path == kvq::kPathTc ? c.kv_heads : c.q_heads;
@@ -165,11 +168,19 @@ void plan_splits_for(const kvq_cache *h, const PlanInput &in, int *n_qsplits, in
     const int64_t nres = (in.max_r + 15) / 16;
     // residual CTA: its tiles shared by the 4 warps of each of its query heads
     const int heads_per_cta = path == kvq::kPathTc ? hg : 1;
-    const double c_res = kCtaFixedTiles + static_cast<double>((nres * heads_per_cta + 3) / 4);
-    int64_t best_S = 0, best_per = 1;
+    const double c_res1 = kCtaFixedTiles + static_cast<double>((nres * heads_per_cta + 3) / 4);
+    // the tensor-core kernel deals the residual tiles over the warps of n_rs residual splits
+    // (4 / HG warps per head in each); a residual tile on CUDA cores costs about two
+    // quantized tiles.  n_rs grows until a residual warp's share costs no more than a
+    // quantized CTA (a long full-precision store, e.g. LogQuant's, then spreads out).
+    const int64_t wph = 4 / heads_per_cta;
+    auto residual_cost = [&](int64_t n_rs) {
+        return kCtaFixedTiles + 2.0 * static_cast<double>((nres + wph * n_rs - 1) / (wph * n_rs));
+    };
+    int64_t best_S = 0, best_per = 1, best_rs = extra;
     if (tiles > 0) {
         int64_t cap = (tiles + kMinTilesPerSplit - 1) / kMinTilesPerSplit;
-        if (cap > max_splits(&c) - 1) cap = max_splits(&c) - 1;
+        if (cap > max_splits(&c) - kMaxResidualSplits) cap = max_splits(&c) - kMaxResidualSplits;
         if (cap > h->split_limit) cap = h->split_limit;
         if (cap < 1) cap = 1;
         double best_cost = -1.0;
@@ -185,14 +196,29 @@ void plan_splits_for(const kvq_cache *h, const PlanInput &in, int *n_qsplits, in
             const double nq = static_cast<double>(per_seq * busy);
             const double n_empty = static_cast<double>(units * S) - nq;
             const double t_waves = std::ceil(nq / slots) * c_q;
-            const double t_spread = (nq * c_q + n_empty * kEmptyCtaTiles + static_cast<double>(units * extra) * c_res) /
-                                        slots +
-                                    (extra ? c_res : 0.0);
-            const double cost = t_waves > t_spread ? t_waves : t_spread;
-            if (best_cost < 0 || cost < best_cost - 1e-9) {
-                best_cost = cost;
-                best_S = S;
-                best_per = per;
+            // residual splits: the tensor-core path tries 1 .. most of them (most: one tile per
+            // residual warp).  Residual CTAs start after every quantized CTA (the grid's order):
+            // when they do not all fit beside the quantized ones, they add to the critical path.
+            int64_t most = 1;
+            if (extra && path == kvq::kPathTc) {
+                most = (nres + wph - 1) / wph;
+                if (most > kMaxResidualSplits) most = kMaxResidualSplits;
+            }
+            for (int64_t n_rs = extra; n_rs <= (extra ? most : 0); ++n_rs) {
+                const double c_res = (path == kvq::kPathTc && n_rs) ? residual_cost(n_rs) : c_res1;
+                const double n_res = static_cast<double>(units * n_rs);
+                const double t_spread =
+                    (nq * c_q + n_empty * kEmptyCtaTiles + n_res * c_res) / slots + (n_rs ? c_res : 0.0);
+                double t_crit = c_q;
+                if (n_rs) t_crit = (nq + n_res > slots) ? c_q + c_res : (c_res > c_q ? c_res : c_q);
+                double cost = t_waves > t_spread ? t_waves : t_spread;
+                cost = cost > t_crit ? cost : t_crit;
+                if (best_cost < 0 || cost < best_cost - 1e-9) {
+                    best_cost = cost;
+                    best_S = S;
+                    best_per = per;
+                    best_rs = n_rs;
+                }
             }
         }
     }
@@ -200,13 +226,20 @@ void plan_splits_for(const kvq_cache *h, const PlanInput &in, int *n_qsplits, in
         best_S = 1;
         best_per = 0;
     }
-    if (best_S + extra == 0) {          // nothing in any sequence: one empty split writes zeros
+    if (best_S == 0 && extra && path == kvq::kPathTc) {   // residual rows only: spread them too
+        int64_t most = (nres + wph - 1) / wph;
+        if (most > kMaxResidualSplits) most = kMaxResidualSplits;
+        const int64_t want = (static_cast<int64_t>(slots) + units - 1) / units;
+        best_rs = want < most ? want : most;
+        if (best_rs < 1) best_rs = 1;
+    }
+    if (best_S + best_rs == 0) {        // nothing in any sequence: one empty split writes zeros
         best_S = 1;
         best_per = align;
     }
     *n_qsplits = static_cast<int>(best_S);
     *tiles_per_split = static_cast<int>(best_per);
-    *S_out = static_cast<int>(best_S + extra);
+    *S_out = static_cast<int>(best_S + best_rs);
 }
 
 void plan_splits(const kvq_cache *h, int *n_qsplits, int *tiles_per_split, int *S_out) {

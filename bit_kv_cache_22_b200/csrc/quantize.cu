@@ -112,14 +112,31 @@ __device__ void pack_tiles(const uint8_t *codes, int ntiles, int d, int bits, bo
 
 // Copy the G rows of d 16-bit elements of one group into shared memory with 16-byte
 // loads: rows tok0 .. tok0+G-1 of `slice`, or rows rows[0 .. G-1] when rows is non-NULL.
+// Each thread issues up to kLoadBatch loads before it stores any, so a group arrives in
+// about one memory latency instead of one per load.
+constexpr int kLoadBatch = 8;
+
 __device__ void load_group(const uint16_t *slice, int64_t tok0, const int32_t *rows, uint16_t *dst, int G,
                            int d) {
-    const int vec = d / 8;
+    const int vec = d / 8, vshift = d == 64 ? 3 : 4;   // d is 64 or 128
+    const int total = G * vec;
     uint4 *d4 = reinterpret_cast<uint4 *>(dst);
-    for (int i = threadIdx.x; i < G * vec; i += blockDim.x) {
-        const int t = i / vec, c = i - t * vec;
-        const int64_t row = rows ? rows[t] : tok0 + t;
-        d4[i] = reinterpret_cast<const uint4 *>(slice + row * d)[c];
+    for (int base = threadIdx.x; base < total; base += kLoadBatch * blockDim.x) {
+        uint4 v[kLoadBatch];
+#pragma unroll
+        for (int k = 0; k < kLoadBatch; ++k) {
+            const int i = base + k * blockDim.x;
+            if (i < total) {
+                const int t = i >> vshift, c = i & (vec - 1);
+                const int64_t row = rows ? rows[t] : tok0 + t;
+                v[k] = __ldcs(reinterpret_cast<const uint4 *>(slice + row * d) + c);   // read once: stream
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kLoadBatch; ++k) {
+            const int i = base + k * blockDim.x;
+            if (i < total) d4[i] = v[k];
+        }
     }
 }
 
