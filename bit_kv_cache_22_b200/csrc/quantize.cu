@@ -79,15 +79,18 @@ __device__ __forceinline__ int sym_code(float x, float s, float rinv, int bits) 
 }
 
 // Assemble the packed words of `ntiles` 16-token tiles from byte codes
-// codes[t * d + c] (t relative to the first tile) and store them at dst.
-// Word w of a tile belongs to lane w / W; its slot s (0 .. 8/n - 1) holds, in
+// codes[t * D + c] (t relative to the first tile) and store them at dst.
+// Word w of a tile belongs to lane w / W; its slot s (0 .. 8/N - 1) holds, in
 // byte b, the element (row = lane/4 + 8*(s%2), col = 4*(lane%4) + b) of block
-// (chunk) j = (w % W) * (4/n) + s/2 at bit 8*b + n*s.
-__device__ void pack_tiles(const uint8_t *codes, int ntiles, int d, int bits, bool is_v,
-                           uint32_t *dst) {
-    const int TW = tile_words(d, bits);
-    const int W = lane_words(d, bits);
-    const int B = 4 / bits;               // blocks per word
+// (chunk) j = (w % W) * (4/N) + s/2 at bit 8*b + N*s.  A key row's four columns
+// are four consecutive channels, one 32-bit load of codes; a value row's are four
+// tokens, four byte loads.  Every code is below 2^N, so a slot's four bytes
+// shifted by N*s stay inside their bytes.
+template <int D, int N, bool IS_V>
+__device__ void pack_tiles(const uint8_t *codes, int ntiles, uint32_t *dst) {
+    constexpr int TW = D * N / 2;        // words per tile
+    constexpr int W = D * N / 64;        // words per lane
+    constexpr int B = 4 / N;             // blocks per word
     const int total = ntiles * TW;
     for (int wi = threadIdx.x; wi < total; wi += blockDim.x) {
         const int tile = wi / TW;
@@ -95,16 +98,20 @@ __device__ void pack_tiles(const uint8_t *codes, int ntiles, int d, int bits, bo
         const int lane = w / W;
         const int wl = w - lane * W;
         uint32_t word = 0;
+#pragma unroll
         for (int slot = 0; slot < 2 * B; ++slot) {
             const int j = wl * B + (slot >> 1);
             const int row = (lane >> 2) + 8 * (slot & 1);
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const int col = 4 * (lane & 3) + b;
-                const int t = tile * 16 + (is_v ? col : row);
-                const int c = 16 * j + (is_v ? row : col);
-                word |= static_cast<uint32_t>(codes[t * d + c]) << (8 * b + bits * slot);
+            const int col0 = 4 * (lane & 3);
+            uint32_t v;
+            if constexpr (IS_V) {
+                const uint8_t *p = codes + (tile * 16 + col0) * D + 16 * j + row;
+                v = static_cast<uint32_t>(p[0]) | (static_cast<uint32_t>(p[D]) << 8) |
+                    (static_cast<uint32_t>(p[2 * D]) << 16) | (static_cast<uint32_t>(p[3 * D]) << 24);
+            } else {
+                v = *reinterpret_cast<const uint32_t *>(codes + (tile * 16 + row) * D + 16 * j + col0);
             }
+            word |= v << (N * slot);
         }
         dst[wi] = word;
     }
@@ -140,9 +147,11 @@ __device__ void load_group(const uint16_t *slice, int64_t tok0, const int32_t *r
     }
 }
 
+template <int D, int N>
 __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const QuantizeArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
-    const int d = a.d, G = a.G, bits = a.bits;
+    constexpr int d = D, bits = N;
+    const int G = a.G;
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem);                       // [G][d]
     uint8_t *codes = smem + static_cast<size_t>(G) * d * 2;                  // [G][d]
     float *red = reinterpret_cast<float *>(codes + static_cast<size_t>(G) * d);  // 2*256
@@ -253,15 +262,17 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
             ch_r[c] = s != 0.0f ? __frcp_rn(s) : 0.0f;
         }
         __syncthreads();
-        for (int e = threadIdx.x; e < G * d; e += blockDim.x) {
-            const int c2 = e % d;
-            const float x = widen(xs[e], a.bf16);
+        {   // d divides the block size: each thread keeps one channel
+            const int c2 = threadIdx.x % d;
             const float sc = ch_s[c2], ri = ch_r[c2];
-            codes[e] = static_cast<uint8_t>(a.sym ? sym_code(x, sc, ri, bits)
-                                                  : asym_code(x, {sc, ch_z[c2]}, ri, bits));
+            const int zc = ch_z[c2];
+            for (int e = threadIdx.x; e < G * d; e += kQuantThreads) {
+                const float x = widen(xs[e], a.bf16);
+                codes[e] = static_cast<uint8_t>(a.sym ? sym_code(x, sc, ri, bits) : asym_code(x, {sc, zc}, ri, bits));
+            }
         }
         __syncthreads();
-        pack_tiles(codes, G / 16, d, bits, false,
+        pack_tiles<D, N, false>(codes, G / 16,
                    a.kc + slice * words_per_slice + (out_tok / 16) * TW);
         __syncthreads();
     }
@@ -270,15 +281,35 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
     load_group(a.xv + bh * a.in_bh_stride, in_tok, rows, xs, G, d);
     __syncthreads();
     {
-        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-        const int per_lane = d / 32;                 // contiguous channels per lane
-        const int seg = a.Gv / per_lane;             // lanes per value group (power of 2)
+        // one token per half-warp (two per warp): the per-token work (segment reductions,
+        // the IEEE divisions of the group parameters) is shared by the two halves
+        constexpr int per_lane = d / 16;             // contiguous channels per lane: 8 or 4
+        const int warp = threadIdx.x >> 5, half = (threadIdx.x >> 4) & 1, hl = threadIdx.x & 15;
+        const int seg = a.Gv / per_lane;             // lanes per value group (power of 2, <= 16)
         const int ngv = d / a.Gv;
-        for (int t = warp; t < G; t += kQuantThreads / 32) {
-            float x[8];
+        for (int tp = warp; tp < G / 2; tp += kQuantThreads / 32) {
+            const int t = 2 * tp + half;
+            float x[per_lane];
             float mn = FLT_MAX, mx = -FLT_MAX;
+            uint16_t xb[per_lane];
+            if constexpr (per_lane == 8) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(xs + t * d + hl * per_lane);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    xb[2 * k] = static_cast<uint16_t>(w[k] & 0xffffu);
+                    xb[2 * k + 1] = static_cast<uint16_t>(w[k] >> 16);
+                }
+            } else {
+                const uint2 v = *reinterpret_cast<const uint2 *>(xs + t * d + hl * per_lane);
+                xb[0] = static_cast<uint16_t>(v.x & 0xffffu);
+                xb[1] = static_cast<uint16_t>(v.x >> 16);
+                xb[2] = static_cast<uint16_t>(v.y & 0xffffu);
+                xb[3] = static_cast<uint16_t>(v.y >> 16);
+            }
+#pragma unroll
             for (int e = 0; e < per_lane; ++e) {
-                x[e] = widen(xs[t * d + lane * per_lane + e], a.bf16);
+                x[e] = widen(xb[e], a.bf16);
                 if (a.sym) {
                     mx = fmaxf(mx, fabsf(x[e]));
                 } else {
@@ -300,19 +331,26 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
                 s = gp.s;
                 z = gp.z;
             }
-            const int j = lane / seg;
-            if (lane % seg == 0) {
+            const int j = hl / seg;
+            if (hl % seg == 0) {
                 const int64_t mi = (slice * cap + out_tok + t) * ngv + j;
                 a.vs[mi] = s;
                 if (!a.sym) a.vz[mi] = static_cast<int16_t>(z);
             }
             const float ri = s != 0.0f ? __frcp_rn(s) : 0.0f;
-            for (int e = 0; e < per_lane; ++e)
-                codes[t * d + lane * per_lane + e] = static_cast<uint8_t>(
+            uint32_t cw[per_lane / 4] = {};
+#pragma unroll
+            for (int e = 0; e < per_lane; ++e) {
+                const uint32_t cq = static_cast<uint32_t>(
                     a.sym ? sym_code(x[e], s, ri, bits) : asym_code(x[e], {s, z}, ri, bits));
+                cw[e / 4] |= cq << (8 * (e % 4));
+            }
+#pragma unroll
+            for (int k = 0; k < per_lane / 4; ++k)
+                reinterpret_cast<uint32_t *>(codes + t * d + hl * per_lane)[k] = cw[k];
         }
         __syncthreads();
-        pack_tiles(codes, G / 16, d, bits, true,
+        pack_tiles<D, N, true>(codes, G / 16,
                    a.vc + slice * words_per_slice + (out_tok / 16) * TW);
     }
 }
@@ -430,19 +468,26 @@ size_t quantize_smem_bytes(int d, int G) {
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s) {
     if (a.n_groups == 0 || a.BH == 0) return cudaSuccess;
     const size_t smem = quantize_smem_bytes(a.d, a.G);
-    // opt in to the largest dynamic shared memory any configuration needs, once per device
-    static bool configured[64] = {};
+    void (*kernel)(const QuantizeArgs) = nullptr;
+    int variant = -1;
+    if (a.d == 64 && a.bits == 2) kernel = quantize_pack_kernel<64, 2>, variant = 0;
+    else if (a.d == 64 && a.bits == 4) kernel = quantize_pack_kernel<64, 4>, variant = 1;
+    else if (a.d == 128 && a.bits == 2) kernel = quantize_pack_kernel<128, 2>, variant = 2;
+    else if (a.d == 128 && a.bits == 4) kernel = quantize_pack_kernel<128, 4>, variant = 3;
+    if (!kernel) return cudaErrorInvalidValue;
+    // opt in to the largest dynamic shared memory any configuration needs, once per device and variant
+    static bool configured[64][4] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 64 || !configured[dev]) {
-        e = cudaFuncSetAttribute(quantize_pack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (dev >= 64 || !configured[dev][variant]) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(quantize_smem_bytes(256, 128)));
         if (e != cudaSuccess) return e;
-        if (dev < 64) configured[dev] = true;
+        if (dev < 64) configured[dev][variant] = true;
     }
     dim3 grid(static_cast<unsigned>(a.n_groups), static_cast<unsigned>(a.BH));
-    quantize_pack_kernel<<<grid, kQuantThreads, smem, s>>>(a);
+    kernel<<<grid, kQuantThreads, smem, s>>>(a);
     count_launches(1);
     return cudaGetLastError();
 }
