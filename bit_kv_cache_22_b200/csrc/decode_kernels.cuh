@@ -172,6 +172,11 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
                  ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
                  : "memory");
 }
+// Hint: bring [src, src + bytes) into L2 (16-byte aligned, a multiple of 16 bytes; no
+// completion to wait for).
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 // One poll; the thread may be suspended up to kPollSuspendNs waiting for the phase, so a
 // waiting warp takes (almost) no issue slots from the working ones.
 constexpr uint32_t kPollSuspendNs = 200000;
@@ -1139,6 +1144,9 @@ __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) deco
                     const uint32_t zb = a.sym ? 0u : static_cast<uint32_t>(ng * D * 2);
                     mbar_expect_tx(bar, cbytes + sb + zb);
                     bulk_g2s(st, ksrc, cbytes, bar);
+                    if constexpr (SPARSE)   // the item's outlier words, read by every lane next to its MMAs
+                        bulk_prefetch_l2(a.k_out + (bh * (a.cap / 16) + ti) * 16 * a.n_out,
+                                         static_cast<uint32_t>(nt * 16 * a.n_out * 4));
                     if (ng > 0) {
                         const int tg = open0 ? ti : ti + 2;
                         const int64_t gofs = (PAGED ? (kt0 + tg) >> a.gshift : gbase + (tg >> a.gshift)) * D;
