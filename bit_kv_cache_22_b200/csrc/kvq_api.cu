@@ -320,6 +320,7 @@ void lq_push(kvq_cache *h) {
 }
 
 kvq_status lq_prefill(kvq_cache *h, const void *X_K, const void *X_V, int64_t T, void *stream);
+kvq_status check_status_word(unsigned int *word);
 
 kvq_status check_decode_args(const kvq_cache *h, const void *t_Q, const float *t_O, const void *workspace,
                              size_t workspace_bytes);
@@ -703,16 +704,7 @@ kvq_status kvq_cache_state(const kvq_cache *h, int64_t *quantized_tokens, int32_
 
 kvq_status kvq_check_device(kvq_cache *h) {
     if (!h) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
-    unsigned int *word = h->arrivals + static_cast<int64_t>(h->cfg.batch) * h->cfg.q_heads;
-    unsigned int v = 0;
-    cudaError_t e = cudaMemcpy(&v, word, sizeof v, cudaMemcpyDeviceToHost);
-    if (e != cudaSuccess) return cuda_fail(e, "reading the decode status word");
-    if (v == 0) return ok();
-    e = cudaMemset(word, 0, sizeof v);
-    if (e == cudaSuccess) e = cudaDeviceSynchronize();
-    if (e != cudaSuccess) return cuda_fail(e, "clearing the decode status word");
-    return fail(KVQ_ERR_CUDA, "a decode kernel gave up waiting for a copy into shared memory; "
-                              "outputs since the last check are unreliable");
+    return check_status_word(h->arrivals + static_cast<int64_t>(h->cfg.batch) * h->cfg.q_heads);
 }
 
 uint64_t kvq_kernel_launches(void) { return g_launches.load(); }

@@ -243,8 +243,8 @@ KVQ_API kvq_status kvq_cache_state(const kvq_cache *cache, int64_t *quantized_to
  * Upper bound on the splits kvq_decode_attention cuts the quantized tokens into
  * (1 .. 64; 0 restores the default of 64).  With one query head per kv head
  * the residual tokens are shared out among those splits; otherwise they form
- * up to 16 more splits of their own when there are any (more for a longer
- * full-precision part, such as a LogQuant store).  Fewer splits mean fewer
+ * 1 to 16 more splits of their own when there are any (more of them for a
+ * longer full-precision part, such as a LogQuant store).  Fewer splits mean fewer
  * partial results to merge, more splits more parallelism for short batches;
  * the result is the same up to fp32 rounding.
  */
