@@ -1,18 +1,19 @@
 // decode_kernels.cuh -- the decode-attention kernels and their launch dispatch, shared by
-// decode.cu (contiguous caches) and decode_paged.cu (paged, ragged caches).
+// decode.cu (contiguous caches), decode_paged.cu (paged, ragged caches) and
+// decode_sparse.cu (dense-and-sparse keys).
 //
-// Split-K decode attention over the packed low-bit cache.
-//
-// Computes, for every (batch, query head), one decode step of
+// Two kernels: decode_split_kernel (CUDA cores, described first, below) and
+// decode_tc_kernel (tensor cores, described above its definition).  Both compute,
+// for every (batch, query head), one decode step of
 //   A = softmax(q [deq(K_g); K_r]^T / sqrt(d)),   t_O = A [deq(V_g); V_r]
 // ("LLM系列：KVCache量化1 KIVI ...", section 1: A = Concat(A_g, A_r), t_O = A X_V;
 //  the 1/sqrt(d_k) of "KV Cache的Int4量化…" section 3), with deq(x) = (code - z) s.
 //
 // Split-K (flash-decoding): the quantized 16-token tiles are divided into
-// contiguous splits and the residual rows, cut into 16-row tiles, form one more
-// split of their own (they are read unstaged, so they run beside the others
-// instead of lengthening one of them); a CTA owns one (batch, query head,
-// split) and each of its four warps a contiguous share of the split's tiles,
+// contiguous splits and the residual rows, cut into 16-row tiles, form splits
+// of their own (one here; up to 16 in the tensor-core kernel), so they run beside
+// the others instead of lengthening one of them; a CTA owns one (batch, query
+// head, split) and each of its four warps a contiguous share of the split's tiles,
 // streamed through a per-warp cp.async ring of shared-memory stages.  Token order does not change the result
 // (A . V = A_P . V_P, "Resumo Técnico: LogQuant", section 4), which is what
 // allows the splits and the residual to be folded into one online-softmax pass.
@@ -887,7 +888,10 @@ __device__ __forceinline__ void load_meta(const float *sp, const int16_t *zp, bo
 //   z-terms: bias_{g,h} = sum_c q'_c z_{g,c} and sum_t p_t s_t z_t in fp32.
 // Residual rows: with HG = 1 their tiles are dealt round-robin to the warps of
 // all splits, which run them first on CUDA cores (staged in shared memory) and
-// start their softmax state from them; with HG > 1 they form one more split.
+// start their softmax state from them; with HG > 1 they form 1 to 16 splits of
+// their own, their tiles dealt round-robin over the warps of all of them.
+// Instances: PAGED reads a paged pool through each sequence's page table and
+// takes each sequence's own length; SPARSE adds each token's key outliers.
 // ---------------------------------------------------------------------------
 constexpr int kTcItem = 4;         // tiles per item (stage)
 constexpr int kVScaleLog2 = 96;   // the value MMA's B operand is p s 2^96

@@ -1,11 +1,13 @@
 // kvq_api.cu -- the C ABI of include/kvq.h: validation, host-side cache state and launches.
 //
-// The handle keeps only geometry, the caller's device pointers and the two
-// counters of the KIVI cache ("LLM系列：KVCache量化1 KIVI ...", section 1):
-// Tq quantized tokens and r < R residual tokens.  Every branch of the
-// streaming logic (when to flush, where a token goes) is decided here on the
-// host from those counters, so the kernels need no device-side control flow
-// and a sequence of calls never waits on the device.
+// A contiguous cache's handle keeps geometry, the caller's device pointers and
+// the two counters of the KIVI cache ("LLM系列：KVCache量化1 KIVI ...", section 1):
+// Tq quantized tokens and r < R residual tokens; a LogQuant cache also keeps
+// the positions of its full-precision store, a paged cache every slot's length.
+// Every branch of the streaming logic (when to flush, where a token goes, how
+// many splits) is decided here on the host from that state, so a sequence of
+// calls never waits on the device.  The kernels read their own copy of the
+// state only where a batch is ragged (the paged cache's slot lengths).
 #include <cmath>
 #include <cstdarg>
 #include <cstdint>

@@ -1,4 +1,5 @@
-// quantize.cu -- KIVI quantize + pack (prefill and residual flush), residual copies.
+// quantize.cu -- KIVI quantize + pack (prefill, residual flush, LogQuant blocks),
+// residual copies, the paged cache's append and the LogQuant store's compaction.
 //
 // One CTA quantizes one key group of G tokens of one (batch, kv-head) slice:
 //   keys   : per channel over the G tokens ("LLM系列：KVCache量化1 KIVI ...",
@@ -17,7 +18,10 @@
 // Packing writes the library's tile layout (see include/kvq.h): each output
 // word is assembled from the 8-bit MMA A-fragment table (four codes of one
 // row per byte group), so writes are fully coalesced and each thread produces
-// whole words.
+// whole words.  The group's rows come from consecutive tokens or from a row
+// list (a LogQuant block); its output slice is a page of a paged pool when a
+// page table is given; dense-and-sparse keys first move each token's largest
+// entries out of the dense part.
 #include <cfloat>
 #include <cstdint>
 
