@@ -8,6 +8,9 @@ fp64 attention), and this module only marshals numpy arrays into it and keeps
 the streaming bookkeeping of the KIVI residual (section 1 of "LLM系列：
 KVCache量化1 KIVI ...": new tokens go to the full-precision residual; when it
 holds R tokens it is quantized, appended to the quantized part and reset).
+It also restates, each in a section of its own below with its sources: the
+merge of token-split partials, LogQuant's full-precision retention
+(LogQuantCache) and dense-and-sparse keys (SparseKeyCache).
 
 It shares no code with the CUDA library and imports nothing from it.
 """
