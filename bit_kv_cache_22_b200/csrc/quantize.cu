@@ -48,38 +48,75 @@ __device__ __forceinline__ GroupParams asym_params(float mn, float mx, int bits)
     return {s, static_cast<int>(zf)};
 }
 
-// round(x / s) (half to even, of the correctly rounded fp32 quotient) as an int,
-// for |x / s| < 2^21.  With rinv = RN(1/s), q = RN(x * rinv) is within
-// |q| * 2^-22 of RN(x / s), so both round to the same integer unless q lies
-// within that distance of a half-integer; only those elements (margin 4x) pay
-// for the IEEE division.
-__device__ __forceinline__ int rint_quotient(float x, float s, float rinv) {
-    const float q = x * rinv;
-    const float t = q + 12582912.0f;                  // 1.5 * 2^23: rounds q to an integer
-    const float k = t - 12582912.0f;
-    const float dist = fabsf(fabsf(q - k) - 0.5f);
-    if (dist <= fabsf(q) * 0x1p-20f + 0x1p-126f)
-        return static_cast<int>(rintf(__fdiv_rn(x, s)));
-    return __float_as_int(t) - 0x4B400000;
-}
-
-__device__ __forceinline__ int asym_code(float x, GroupParams p, float rinv, int bits) {
-    const int L = (1 << bits) - 1;
-    int q = rint_quotient(x, p.s, rinv) + p.z;
-    return min(max(q, 0), L);
-}
-
 __device__ __forceinline__ float sym_scale(float amax, int bits) {
     const float L = static_cast<float>((1 << bits) - 1);
     return __fdiv_rn(__fmul_rn(2.0f, amax), L);
 }
 
-__device__ __forceinline__ int sym_code(float x, float s, float rinv, int bits) {
-    const int half = 1 << (bits - 1);
-    if (s == 0.0f) return half;
-    int q = rint_quotient(x, s, rinv);
-    q = min(max(q, -half), half - 1);
-    return q + half;
+// packed fp32x2 arithmetic (sm_100): two IEEE round-to-nearest operations at once
+__device__ __forceinline__ unsigned long long pack2(float2 v) {
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(v.x), "f"(v.y));
+    return r;
+}
+__device__ __forceinline__ float2 unpack2(unsigned long long r) {
+    float2 v;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+    return v;
+}
+__device__ __forceinline__ float2 mul_x2(float2 a, float2 b) {
+    unsigned long long d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(pack2(a)), "l"(pack2(b)));
+    return unpack2(d);
+}
+__device__ __forceinline__ float2 add_x2(float2 a, float2 b) {
+    unsigned long long d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(pack2(a)), "l"(pack2(b)));
+    return unpack2(d);
+}
+__device__ __forceinline__ float2 fma_x2(float2 a, float2 b, float2 c) {
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(pack2(a)), "l"(pack2(b)), "l"(pack2(c)));
+    return unpack2(d);
+}
+
+// One group's parameters for code_pair: code = clamp(round(x / s) + off, 0, L), with
+// off = z (asymmetric) or 2^(n-1) (symmetric: clamp(round(x/s), -2^(n-1), 2^(n-1)-1) +
+// 2^(n-1) is the same clamp).  ri = RN(1/s) (0 when s = 0, which gives code off).
+// cut2 = (1/2 - 2^-18 qmax)^2 with qmax >= |x / s| over the group.
+struct CodeParams {
+    float s, ri, cut2;
+    int off;
+};
+
+__device__ __forceinline__ CodeParams code_params(float s, int off, float amax) {
+    const float ri = s != 0.0f ? __frcp_rn(s) : 0.0f;
+    const float qmax = amax * ri * 1.0001f;
+    const float cut = fmaxf(0.5f - qmax * 0x1p-18f, 0.0f);   // 0: every element takes the division
+    return {s, ri, cut * cut, off};
+}
+
+// Codes of two elements of one group (byte 0 and byte 1 of the result), where round is
+// half to even of the correctly rounded fp32 quotient RN(x / s).  With ri = RN(1/s),
+// q = RN(x ri) is within |q| 2^-22 of RN(x / s), so both round to the same integer
+// unless q lies within that distance of a half-integer.  r = q - round(q) is exact; while
+// r^2 < cut2, |r| stays more than qmax 2^-20 from 1/2 (the rounding of r^2 and cut2 is
+// covered by the larger margin 2^-18, as qmax >= 1 in every group with a nonzero
+// element; an all-zero group has q = r = 0), so the fast result stands; an element
+// nearer a tie takes the IEEE division.
+template <int N>
+__device__ __forceinline__ uint32_t code_pair(float x0, float x1, const CodeParams &p) {
+    constexpr int L = (1 << N) - 1;
+    const float2 q = mul_x2(make_float2(x0, x1), make_float2(p.ri, p.ri));
+    const float2 t = add_x2(q, make_float2(12582912.0f, 12582912.0f));      // 1.5 * 2^23
+    const float2 k = add_x2(t, make_float2(-12582912.0f, -12582912.0f));
+    const float2 r = fma_x2(k, make_float2(-1.0f, -1.0f), q);
+    const float2 r2 = mul_x2(r, r);
+    int i0 = __float_as_int(t.x) - 0x4B400000, i1 = __float_as_int(t.y) - 0x4B400000;
+    if (r2.x >= p.cut2) i0 = static_cast<int>(rintf(__fdiv_rn(x0, p.s)));
+    if (r2.y >= p.cut2) i1 = static_cast<int>(rintf(__fdiv_rn(x1, p.s)));
+    const int c0 = min(max(i0 + p.off, 0), L), c1 = min(max(i1 + p.off, 0), L);
+    return static_cast<uint32_t>(c0) | (static_cast<uint32_t>(c1) << 8);
 }
 
 // Assemble the packed words of `ntiles` 16-token tiles from byte codes
@@ -162,6 +199,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
     float *ch_s = red + 2 * kQuantThreads;                                   // [d]
     int *ch_z = reinterpret_cast<int *>(ch_s + d);                           // [d]
     float *ch_r = reinterpret_cast<float *>(ch_z + d);                       // [d] 1/s
+    float *ch_c = ch_r + d;                                                  // [d] near-tie bound
 
     const int64_t grp = blockIdx.x;
     const int64_t bh = blockIdx.y;                 // input slice
@@ -261,18 +299,21 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
                 a.kz[(slice * groups_cap + out_tok / G) * d + c] = static_cast<int16_t>(z);
             }
             a.ks[(slice * groups_cap + out_tok / G) * d + c] = s;
+            const CodeParams cp = code_params(s, z, a.sym ? mx : fmaxf(fabsf(mn), fabsf(mx)));
             ch_s[c] = s;
             ch_z[c] = z;
-            ch_r[c] = s != 0.0f ? __frcp_rn(s) : 0.0f;
+            ch_r[c] = cp.ri;
+            ch_c[c] = cp.cut2;
         }
         __syncthreads();
-        {   // d divides the block size: each thread keeps one channel
+        {   // d divides the block size: each thread keeps one channel, two rows at a time
+            constexpr int rstep = kQuantThreads / d;
             const int c2 = threadIdx.x % d;
-            const float sc = ch_s[c2], ri = ch_r[c2];
-            const int zc = ch_z[c2];
-            for (int e = threadIdx.x; e < G * d; e += kQuantThreads) {
-                const float x = widen(xs[e], a.bf16);
-                codes[e] = static_cast<uint8_t>(a.sym ? sym_code(x, sc, ri, bits) : asym_code(x, {sc, zc}, ri, bits));
+            const CodeParams cp{ch_s[c2], ch_r[c2], ch_c[c2], ch_z[c2]};
+            for (int t = threadIdx.x / d; t < G; t += 2 * rstep) {
+                const uint32_t cc = code_pair<N>(widen(xs[t * d + c2], a.bf16), widen(xs[(t + rstep) * d + c2], a.bf16), cp);
+                codes[t * d + c2] = static_cast<uint8_t>(cc & 0xffu);
+                codes[(t + rstep) * d + c2] = static_cast<uint8_t>(cc >> 8);
             }
         }
         __syncthreads();
@@ -341,14 +382,12 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
                 a.vs[mi] = s;
                 if (!a.sym) a.vz[mi] = static_cast<int16_t>(z);
             }
-            const float ri = s != 0.0f ? __frcp_rn(s) : 0.0f;
+            const CodeParams cp = code_params(s, a.sym ? (1 << (bits - 1)) : z,
+                                              a.sym ? mx : fmaxf(fabsf(mn), fabsf(mx)));
             uint32_t cw[per_lane / 4] = {};
 #pragma unroll
-            for (int e = 0; e < per_lane; ++e) {
-                const uint32_t cq = static_cast<uint32_t>(
-                    a.sym ? sym_code(x[e], s, ri, bits) : asym_code(x[e], {s, z}, ri, bits));
-                cw[e / 4] |= cq << (8 * (e % 4));
-            }
+            for (int e = 0; e < per_lane; e += 2)
+                cw[e / 4] |= code_pair<N>(x[e], x[e + 1], cp) << (8 * (e % 4));
 #pragma unroll
             for (int k = 0; k < per_lane / 4; ++k)
                 reinterpret_cast<uint32_t *>(codes + t * d + hl * per_lane)[k] = cw[k];
@@ -466,7 +505,7 @@ __global__ void paged_residual_kernel(const uint16_t *xk, const uint16_t *xv, in
 
 size_t quantize_smem_bytes(int d, int G) {
     return static_cast<size_t>(G) * d * 3 + 2 * kQuantThreads * sizeof(float) +
-           static_cast<size_t>(d) * 12;
+           static_cast<size_t>(d) * 16;
 }
 
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s) {
