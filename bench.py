@@ -422,19 +422,12 @@ def run_kvq(args):
 
 
 # ---------------------------------------------------------------------------
-# the paged, ragged cache
+# decode-only measurements: LogQuant retention and the paged, ragged cache
 # ---------------------------------------------------------------------------
 
-def run_logquant(args):
-    """Decode attention with LogQuant retention (window W) on the workload's batch: the
-    prompt's prefill (eager: it uploads row lists), then per decode step an eager append and
-    the step's decode_attention graph replayed `--steps` times between two events.  value =
-    KV tokens attended per second of decode time; the roofline counts the quantized tokens'
-    bytes and the full-precision store's rows."""
+def _rank_setup(args):
+    """(world, rank, local rank, device) of this process; NCCL process group for N > 1."""
     import torch
-
-    from bit_kv_cache_22_b200 import kvq
-    from bit_kv_cache_22_b200 import workloads as wl
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -447,26 +440,23 @@ def run_logquant(args):
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
-    w = shard_workload(wl.WORKLOADS[args.workload], rank)
-    W = args.window
-    dt = torch.float16 if w.dtype == wl.FP16 else torch.bfloat16
+    return world, rank, local, dev
 
-    def to_t(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(dt).to(dev)
 
-    cap = -(-(w.T + w.steps) // W) * W
-    cache = kvq.KVQCache(w.B, w.Hq, w.Hkv, w.d, w.G, w.Gv, w.R, w.bits, w.symmetric, dt, cap, dev,
-                         window=W, key_outliers=args.key_outliers)
-    XK, XV = wl.prefill_bits(w)
-    cache.prefill_quantize(to_t(XK), to_t(XV))
-    del XK, XV
-    tK, tV, tQ = (to_t(x) for x in wl.decode_bits(w))
-    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
+def _time_decode_steps(args, cache, steps, tK, tV, tQ, out, local, count):
+    """Per decode step: an eager append, then the step's decode_attention captured as a CUDA
+    graph, warmed up and replayed `--steps` times between two events on the replay stream.
+    count() gives (KV tokens, algorithmic bytes) of one decode call at the current state.
+    Returns (decode ms, KV tokens, bytes, kernel launches, clock sampler)."""
+    import torch
+
+    from bit_kv_cache_22_b200 import kvq
+
+    stream = torch.cuda.current_stream()
     pool = torch.cuda.graph_pool_handle()
     total_ms, total_tokens, total_bytes, launches = 0.0, 0, 0, 0
     with ClockSampler(local) as clk:
-        for s in range(w.steps):
+        for s in range(steps):
             cache.append(tK[s], tV[s])
             torch.cuda.synchronize()
             l0 = kvq.kernel_launches()
@@ -485,40 +475,38 @@ def run_logquant(args):
             torch.cuda.synchronize()
             total_ms += e0.elapsed_time(e1)
             launches += per_call * args.steps
-            tq, r = cache.state()
-            total_tokens += w.B * (tq + r) * args.steps
-            total_bytes += (algorithmic_bytes(w, tq, r) + w.B * w.Hkv * tq * 4 * args.key_outliers) * args.steps
+            tokens, nbytes = count()
+            total_tokens += tokens * args.steps
+            total_bytes += nbytes * args.steps
             del g
-    ms, = max_over_ranks([total_ms], world, dev)
-    if rank != 0:
-        if world > 1:
-            dist.destroy_process_group()
-        return
+    return total_ms, total_tokens, total_bytes, launches, clk
+
+
+def _decode_only_line(args, w, world, ms, total_ms, total_tokens, total_bytes, launches, clk, config,
+                      kernel):
+    """The JSON line of a decode-only measurement (rank 0)."""
+    from bit_kv_cache_22_b200 import workloads as wl
+
     calls = w.steps * args.steps
     peak, peak_kind = peaks()
     achieved = total_bytes / (total_ms / 1e3) / 1e9
-    tq, r = cache.state()
-    line = {
+    config = dict(config)
+    config.update({
+        "elem": "fp16" if w.dtype == wl.FP16 else "bf16", "parallelism": f"dp{world}",
+        "l2": f"inputs larger than L2: packed cache {total_bytes / calls / 1e6:.0f} MB per decode call",
+        "timing": "per decode step: its decode_attention graph replayed --steps times between "
+                  "two events (value and roofline: decode time only; appends run eagerly between)",
+    })
+    return {
         "metric": METRIC, "value": job_throughput(total_tokens, world, ms), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / calls,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": f"u{w.bits} codes, f32 accumulate",
         "data": "synthetic (seeded; distributions of the workload definition)",
-        "config": {
-            "workload": f"{w.name} (LogQuant retention, W={W})", "batch_per_gpu": w.B, "q_heads": w.Hq,
-            "kv_heads": w.Hkv, "head_dim": w.d, "prompt_tokens": w.T, "decode_steps": w.steps,
-            "bits": w.bits, "group_k": w.G, "group_v": w.Gv, "window": W,
-            "key_outliers_per_token": args.key_outliers, "full_precision_rows_at_end": r,
-            "elem": "fp16" if w.dtype == wl.FP16 else "bf16", "parallelism": f"dp{world}",
-            "l2": "inputs larger than L2: packed cache "
-                  f"{total_bytes / calls / 1e6:.0f} MB per decode call",
-            "splits": cache.splits(),
-            "timing": "per decode step: its decode_attention graph replayed --steps times between "
-                      "two events (decode time only; appends run eagerly between)",
-        },
+        "config": config,
         "roofline": {
-            "kernel": f"decode_attention ({decode_kernel_name(w)}) over a LogQuant cache, per call",
-            "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "kernel": kernel, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak,
             "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
             else "fallback 6.65 TB/s",
             "algorithmic_bytes_per_launch": total_bytes / calls, "avg_launch_us": total_ms / calls * 1e3,
@@ -529,34 +517,73 @@ def run_logquant(args):
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
     }
-    print(json.dumps(line))
+
+
+def _finish(world, rank, line):
+    if rank == 0:
+        print(json.dumps(line))
     if world > 1:
+        import torch.distributed as dist
         dist.destroy_process_group()
 
 
-def run_paged(args):
-    """Decode attention of a ragged batch held in a paged cache.  After the prompts'
-    prefill, every decode step appends one token per slot (eagerly: the page table is
-    written from the host when a flush opens a page) and its decode_attention call is
-    captured as a CUDA graph and replayed `--steps` times between two events on the
-    replay stream.  value = KV tokens attended per second of decode time over all steps;
-    the roofline uses the algorithmic bytes of every slot at its own length."""
+def run_logquant(args):
+    """Decode attention with LogQuant retention (window W) on the workload's batch: the
+    prompt's prefill (eager: it uploads row lists), then the decode steps timed by
+    _time_decode_steps.  value = KV tokens attended per second of decode time; the roofline
+    counts the quantized tokens' bytes and the full-precision store's rows."""
     import torch
 
     from bit_kv_cache_22_b200 import kvq
     from bit_kv_cache_22_b200 import workloads as wl
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus:
-        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
+    world, rank, local, dev = _rank_setup(args)
+    w = shard_workload(wl.WORKLOADS[args.workload], rank)
+    W = args.window
+    dt = torch.float16 if w.dtype == wl.FP16 else torch.bfloat16
+
+    def to_t(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(dt).to(dev)
+
+    cap = -(-(w.T + w.steps) // W) * W
+    cache = kvq.KVQCache(w.B, w.Hq, w.Hkv, w.d, w.G, w.Gv, w.R, w.bits, w.symmetric, dt, cap, dev,
+                         window=W, key_outliers=args.key_outliers)
+    XK, XV = wl.prefill_bits(w)
+    cache.prefill_quantize(to_t(XK), to_t(XV))
+    del XK, XV
+    tK, tV, tQ = (to_t(x) for x in wl.decode_bits(w))
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
+
+    def count():
+        tq, r = cache.state()
+        return w.B * (tq + r), algorithmic_bytes(w, tq, r) + w.B * w.Hkv * tq * 4 * args.key_outliers
+
+    total_ms, tokens, nbytes, launches, clk = _time_decode_steps(args, cache, w.steps, tK, tV, tQ, out, local,
+                                                                 count)
+    ms, = max_over_ranks([total_ms], world, dev)
+    tq, r = cache.state()
+    config = {"workload": f"{w.name} (LogQuant retention, W={W})", "batch_per_gpu": w.B, "q_heads": w.Hq,
+              "kv_heads": w.Hkv, "head_dim": w.d, "prompt_tokens": w.T, "decode_steps": w.steps,
+              "bits": w.bits, "group_k": w.G, "group_v": w.Gv, "window": W,
+              "key_outliers_per_token": args.key_outliers, "full_precision_rows_at_end": r,
+              "splits": cache.splits()}
+    line = _decode_only_line(args, w, world, ms, total_ms, tokens, nbytes, launches, clk, config,
+                             f"decode_attention ({decode_kernel_name(w)}) over a LogQuant cache, per call")
+    _finish(world, rank, line)
+
+
+def run_paged(args):
+    """Decode attention of a ragged batch held in a paged cache.  After the prompts'
+    prefill, every decode step appends one token per slot (eagerly: the page table is
+    written from the host when a flush opens a page) and is timed by _time_decode_steps.
+    value = KV tokens attended per second of decode time over all steps; the roofline uses
+    the algorithmic bytes of every slot at its own length."""
+    import torch
+
+    from bit_kv_cache_22_b200 import kvq
+    from bit_kv_cache_22_b200 import workloads as wl
+
+    world, rank, local, dev = _rank_setup(args)
     spec = wl.RAGGED[args.paged]
     w = shard_workload(spec["base"], rank)
     lens = wl.ragged_lengths(w, spec["lo"], spec["hi"])
@@ -575,76 +602,23 @@ def run_paged(args):
         cache.prefill(b, to_t(XK[0]), to_t(XV[0]))
     tK, tV, tQ = (to_t(x) for x in wl.decode_bits(w))
     out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    pool = torch.cuda.graph_pool_handle()
-    total_ms, total_tokens, total_bytes, launches = 0.0, 0, 0, 0
-    with ClockSampler(local) as clk:
-        for s in range(w.steps):
-            cache.append(tK[s], tV[s])
-            torch.cuda.synchronize()
-            l0 = kvq.kernel_launches()
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, pool=pool):
-                cache.decode_attention(tQ[s], out=out)
-            per_call = kvq.kernel_launches() - l0
-            for _ in range(max(1, args.warmup)):
-                g.replay()
-            torch.cuda.synchronize()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(args.steps):
-                g.replay()
-            e1.record(stream)
-            torch.cuda.synchronize()
-            total_ms += e0.elapsed_time(e1)
-            launches += per_call * args.steps
-            n = [cache.lens[b] for b in range(w.B)]
-            total_tokens += sum(n) * args.steps
-            w1 = w.replace(B=1)
-            total_bytes += sum(algorithmic_bytes(w1, x // w.R * w.R, x % w.R) for x in n) * args.steps
-            del g
+    w1 = w.replace(B=1)
+
+    def count():
+        n = [cache.lens[b] for b in range(w.B)]
+        return sum(n), sum(algorithmic_bytes(w1, x // w.R * w.R, x % w.R) for x in n)
+
+    total_ms, tokens, nbytes, launches, clk = _time_decode_steps(args, cache, w.steps, tK, tV, tQ, out, local,
+                                                                 count)
     ms, = max_over_ranks([total_ms], world, dev)
-    if rank != 0:
-        if world > 1:
-            dist.destroy_process_group()
-        return
-    calls = w.steps * args.steps
-    peak, peak_kind = peaks()
-    achieved = total_bytes / (total_ms / 1e3) / 1e9
-    line = {
-        "metric": METRIC, "value": job_throughput(total_tokens, world, ms), "unit": UNIT,
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / calls,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": f"u{w.bits} codes, f32 accumulate",
-        "data": "synthetic (seeded; distributions of the workload definition)",
-        "config": {
-            "workload": f"{args.paged} (paged, ragged)", "slots_per_gpu": w.B, "q_heads": w.Hq,
-            "kv_heads": w.Hkv, "head_dim": w.d, "prompt_tokens": f"{min(lens)}..{max(lens)} "
-            f"(mean {sum(lens) / len(lens):.0f})", "page_tokens": P, "decode_steps": w.steps,
-            "bits": w.bits, "group_k": w.G, "group_v": w.Gv, "residual": w.R,
-            "elem": "fp16" if w.dtype == wl.FP16 else "bf16", "parallelism": f"dp{world}",
-            "l2": "inputs larger than L2: packed cache "
-                  f"{total_bytes / calls / 1e6:.0f} MB per decode call",
-            "splits": cache.splits(),
-            "timing": "per decode step: its decode_attention graph replayed --steps times between "
-                      "two events (value and roofline: decode time only; appends run eagerly between)",
-        },
-        "roofline": {
-            "kernel": f"paged decode_attention ({decode_kernel_name(w)}, paged instance), per call",
-            "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-            else "fallback 6.65 TB/s",
-            "algorithmic_bytes_per_launch": total_bytes / calls, "avg_launch_us": total_ms / calls * 1e3,
-            "traffic": None,
-        },
-        "cpu_baseline": None,
-        "e2e": None,
-        "gpu_launches": int(launches),
-        "clocks": clk.summary(),
-    }
-    print(json.dumps(line))
-    if world > 1:
-        dist.destroy_process_group()
+    config = {"workload": f"{args.paged} (paged, ragged)", "slots_per_gpu": w.B, "q_heads": w.Hq,
+              "kv_heads": w.Hkv, "head_dim": w.d,
+              "prompt_tokens": f"{min(lens)}..{max(lens)} (mean {sum(lens) / len(lens):.0f})",
+              "page_tokens": P, "decode_steps": w.steps, "bits": w.bits, "group_k": w.G, "group_v": w.Gv,
+              "residual": w.R, "splits": cache.splits()}
+    line = _decode_only_line(args, w, world, ms, total_ms, tokens, nbytes, launches, clk, config,
+                             f"paged decode_attention ({decode_kernel_name(w)}, paged instance), per call")
+    _finish(world, rank, line)
 
 
 # ---------------------------------------------------------------------------
