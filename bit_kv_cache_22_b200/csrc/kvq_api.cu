@@ -1191,3 +1191,43 @@ kvq_status kvq_set_key_outliers(kvq_cache *h, int32_t n_out, uint32_t *k_outlier
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// The split plan without a device: the same planner the decode calls use, for
+// capacity planning and for tests of its invariants on the host.
+// ---------------------------------------------------------------------------
+extern "C" {
+
+kvq_status kvq_plan_decode(const kvq_config *cfg, const int64_t *lengths, int32_t num_sms, int32_t ctas_per_sm,
+                           int32_t *n_qsplits, int32_t *tiles_per_split, int32_t *splits) {
+    kvq_status st = validate(cfg);
+    if (st != KVQ_OK) return st;
+    if (!lengths || !n_qsplits || !tiles_per_split || !splits)
+        return fail(KVQ_ERR_INVALID_ARG, "lengths and the outputs must be non-NULL");
+    if (num_sms < 1 || ctas_per_sm < 1) return fail(KVQ_ERR_INVALID_ARG, "num_sms and ctas_per_sm must be >= 1");
+    kvq_cache h;
+    h.cfg = *cfg;
+    h.num_sms = num_sms;
+    h.ctas_per_sm = ctas_per_sm;
+    std::vector<int64_t> tiles(static_cast<size_t>(cfg->batch));
+    int32_t max_r = 0;
+    for (int b = 0; b < cfg->batch; ++b) {
+        const int64_t len = lengths[b] > 0 ? lengths[b] : 0;
+        const int64_t tq = (len / cfg->residual) * cfg->residual;
+        if (tq > cfg->capacity)
+            return fail(KVQ_ERR_CAPACITY, "sequence %d: %lld quantized tokens exceed capacity %lld", b,
+                        static_cast<long long>(tq), static_cast<long long>(cfg->capacity));
+        tiles[static_cast<size_t>(b)] = tq / 16;
+        const int32_t r = static_cast<int32_t>(len - tq);
+        max_r = r > max_r ? r : max_r;
+    }
+    const PlanInput in{tiles.data(), cfg->batch, 1, max_r};
+    int nq = 0, per = 0, S = 0;
+    plan_splits_for(&h, in, &nq, &per, &S);
+    *n_qsplits = nq;
+    *tiles_per_split = per;
+    *splits = S;
+    return ok();
+}
+
+}  // extern "C"

@@ -35,7 +35,7 @@ EXPORTED = ("kvq_get_sizes", "kvq_create", "kvq_destroy", "kvq_reset", "kvq_pref
             "kvq_paged_create", "kvq_paged_destroy", "kvq_paged_prefill", "kvq_paged_append",
             "kvq_paged_decode_attention", "kvq_paged_release", "kvq_paged_seq_len",
             "kvq_paged_decode_splits", "kvq_paged_check_device", "kvq_logquant_get_sizes",
-            "kvq_logquant_create", "kvq_logquant_retained", "kvq_set_key_outliers")
+            "kvq_logquant_create", "kvq_logquant_retained", "kvq_set_key_outliers", "kvq_plan_decode")
 
 
 class KVQError(RuntimeError):
@@ -136,6 +136,9 @@ def load() -> ctypes.CDLL:
                                             ctypes.POINTER(P)]
         lib.kvq_logquant_retained.argtypes = [P, ctypes.POINTER(i64), i32, ctypes.POINTER(i32)]
         lib.kvq_set_key_outliers.argtypes = [P, i32, P, sz]
+        lib.kvq_plan_decode.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(i64), i32, i32,
+                                        ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(i32)]
+        lib.kvq_plan_decode.restype = ctypes.c_int
         for name in ("kvq_logquant_get_sizes", "kvq_logquant_create", "kvq_logquant_retained",
                      "kvq_set_key_outliers"):
             getattr(lib, name).restype = ctypes.c_int
@@ -580,6 +583,17 @@ def merge_partials(o_all: torch.Tensor, m_all: torch.Tensor, l_all: torch.Tensor
     _check(load().kvq_merge_partials(o_all.data_ptr(), m_all.data_ptr(), l_all.data_ptr(), n, rows, d,
                                      out.data_ptr(), _stream_ptr(stream)))
     return out
+
+
+def plan_decode(cfg: Config, lengths, num_sms: int = 148, ctas_per_sm: int = 4):
+    """(splits over the quantized tokens, 16-token tiles per split, total splits) that a decode
+    over sequences of these lengths would use; host only."""
+    n = len(lengths)
+    arr = (ctypes.c_int64 * max(1, n))(*lengths)
+    nq, per, S = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    _check(load().kvq_plan_decode(ctypes.byref(cfg), arr, num_sms, ctas_per_sm, ctypes.byref(nq),
+                                  ctypes.byref(per), ctypes.byref(S)))
+    return int(nq.value), int(per.value), int(S.value)
 
 
 def kernel_launches() -> int:

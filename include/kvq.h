@@ -250,6 +250,20 @@ KVQ_API kvq_status kvq_cache_state(const kvq_cache *cache, int64_t *quantized_to
  */
 KVQ_API kvq_status kvq_set_split_limit(kvq_cache *cache, int32_t max_splits);
 
+/*
+ * The split plan of a decode over cfg->batch sequences of lengths[b] tokens each
+ * (host int64; Tq = floor(len/R) R quantized, r = len mod R residual; a length
+ * < 0 counts as empty), on a GPU of num_sms SMs holding ctas_per_sm decode CTAs
+ * each.  Writes the splits over the quantized tokens, the 16-token tiles per
+ * split and the total splits including the residual ones (>= 1): what the
+ * decode calls choose for those lengths (kvq_decode_splits reports a cache's
+ * total on its device).  Host only, no device needed; KVQ_ERR_CAPACITY if a
+ * sequence's Tq exceeds cfg->capacity.
+ */
+KVQ_API kvq_status kvq_plan_decode(const kvq_config *cfg, const int64_t *lengths, int32_t num_sms,
+                                   int32_t ctas_per_sm, int32_t *n_qsplits, int32_t *tiles_per_split,
+                                   int32_t *splits);
+
 /* Number of token splits the next kvq_decode_attention would use (>= 1). */
 KVQ_API int32_t kvq_decode_splits(const kvq_cache *cache);
 
