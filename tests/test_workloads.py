@@ -45,3 +45,13 @@ def test_decode_bits_head_mapping():
     # tiny appends plain N(0,1) tokens: no outlier channel in decode keys
     k, _ = wl.decode_slice(w.replace(steps=4096), 0, 0)
     assert k.std(axis=0).max() < 1.2
+
+
+def test_ragged_lengths_are_seeded_and_in_range():
+    spec = wl.RAGGED["ragged_gqa"]
+    w = spec["base"]
+    a = wl.ragged_lengths(w, spec["lo"], spec["hi"])
+    assert a == wl.ragged_lengths(w, spec["lo"], spec["hi"])
+    assert len(a) == w.B and all(spec["lo"] <= x <= spec["hi"] for x in a)
+    assert a != wl.ragged_lengths(w.replace(seed=w.seed + 1), spec["lo"], spec["hi"])
+    assert spec["page_tokens"] % w.R == 0 and spec["page_tokens"] % 64 == 0
