@@ -7,10 +7,11 @@ holds R tokens -- and split-K decode attention whose last split merges the parti
 The metric is KV tokens attended per second: each decode step attends to
 B * (Tq + r) cached tokens.
 
-Default workload: llama7b (B8, 32 MHA heads, d128, 4096-token prompt bf16,
-4-bit asymmetric, G = Gv = R = 128, 128 decode steps).  Multi-GPU runs are
-weak-scaled: every rank serves its own batch of 8 sequences (no data-path
-collective).
+Default workload: gqa8b, the largest single-GPU configuration (B32, 32 q / 8 kv
+heads, d128, 8192-token prompt bf16, 2-bit asymmetric, G = Gv = 32, R = 128, 64
+decode steps); a 1-GPU run adds long131k, llama7b, stream2 and stream4sym under
+"workloads", each with its own roofline.  Multi-GPU runs are weak-scaled: every
+rank serves its own batch of sequences (no data-path collective).
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
        python bench.py --impl reference ...   (the CPU oracle, rank 0 only)
@@ -43,10 +44,12 @@ def _args():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=30)
     p.add_argument("--warmup", type=int, default=3)
-    p.add_argument("--workload", default="llama7b")
+    p.add_argument("--workload", default="gqa8b")
     p.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-extra", action="store_true",
+                   help="measure the headline workload only (by default a 1-GPU run adds the others)")
     p.add_argument("--ncu-case", action="store_true",
                    help="run one prefill and up to 64 decode steps of the workload, then exit (for ncu)")
     p.add_argument("--paged", default=None, metavar="RAGGED_WORKLOAD",
@@ -191,25 +194,55 @@ class ClockSampler:
 # the library arm
 # ---------------------------------------------------------------------------
 
-def run_kvq(args):
+L2_BYTES = 126 * 1024 * 1024      # B200 L2 (126 MB): per-call inputs below it are timed L2-scrubbed
+EXTRA_WORKLOADS = ("long131k", "llama7b", "stream2", "stream4sym")
+
+
+class L2Scrub:
+    """A read of 2 x L2 bytes: evicts whatever the previous call left in L2 and leaves
+    clean lines behind (nothing to write back during the next timed call)."""
+
+    def __init__(self, dev):
+        import torch
+        self.buf = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+        self.out = torch.empty((), dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        import torch
+        torch.sum(self.buf, dim=0, out=self.out)
+
+
+def _replay_ms(graph, k, stream):
+    """Device time of k back-to-back replays of a CUDA graph (two events on the stream)."""
+    import torch
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(k):
+        graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def measure_workload(w, args, dev, local, world, headline: bool):
+    """One workload on this rank: whole-episode throughput (value), per-decode-call time and
+    the roofline, and (headline only) the end-to-end figure through the public API.
+
+    The episode (prefill + every decode step) is captured as one CUDA graph and replayed
+    K times between two events: `value` and `ms_per_step`.  The decode calls alone -- every
+    step's append_decode (at a flush: append, then decode) after the prompt's prefill -- are
+    a second graph, replayed K times back to back; replaying it is idempotent (every step
+    rewrites the residual row and the flushed tokens it wrote before).  A third graph holds
+    only the flush steps' appends; per call = (decode graph - flush graph) / steps, so
+    avg_launch_us x steps <= ms_per_step.  When one call's cache fits in L2, every decode
+    step in the decode graph is preceded by a read of a 2 x L2 buffer, and the time of a
+    graph of those reads alone is subtracted too: `cold` timing."""
     import torch
     import torch.distributed as dist
 
     from bit_kv_cache_22_b200 import kvq
     from bit_kv_cache_22_b200 import workloads as wl
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus:
-        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
-
-    w = shard_workload(wl.WORKLOADS[args.workload], rank)
     dt = torch.float16 if w.dtype == wl.FP16 else torch.bfloat16
 
     def to_t(bits, pin=False):
@@ -225,18 +258,11 @@ def run_kvq(args):
     out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    if args.ncu_case:
-        cache.prefill_quantize(XK, XV)
-        for s in range(min(w.steps, 64)):      # ends with r = 64 residual rows, mid-episode
-            cache.append_decode(tK[s], tV[s], tQ[s], out=out)
-        torch.cuda.synchronize()
-        print(json.dumps({"ncu_case": args.workload, "state": cache.state()}))
-        return
-
     ctx = episode_contexts(w)
+    call_bytes = [algorithmic_bytes(w, tq, r) + w.B * w.Hkv * tq * 4 * args.key_outliers for tq, r in ctx]
     tokens_per_episode = sum(w.B * (tq + r) for tq, r in ctx)
-    bytes_per_episode = sum(algorithmic_bytes(w, tq, r) for tq, r in ctx)
-    bytes_per_episode += sum(w.B * w.Hkv * tq * 4 * args.key_outliers for tq, r in ctx)   # outlier words
+    cold = max(call_bytes) < L2_BYTES
+    scrub = L2Scrub(dev) if cold else None
 
     def episode():
         cache.reset()
@@ -251,81 +277,86 @@ def run_kvq(args):
     for _ in range(args.warmup):
         episode()
     torch.cuda.synchronize()
-    # The episode is captured once as a sequence of CUDA graphs -- the prompt
-    # prefill, then per decode step one graph for append (+ flush) and one for
-    # decode_attention -- and replayed in that order: the host-side cost of
-    # ~640 small launches per episode would otherwise starve the GPU.  Timing
-    # events sit between the graph launches, on the capture/replay stream, so
-    # every decode_attention call of the timed region is timed individually.
-    launches0 = kvq.kernel_launches()
     pool = torch.cuda.graph_pool_handle()
-    cache.reset()
-    g_pre = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_pre, pool=pool):
-        cache.prefill_quantize(XK, XV)
-    # a step whose append flushes the residual gets its own append graph (the quantize is
-    # not part of the timed decode); every other step is one append_decode graph
-    g_app, g_dec = [], []
-    for s_ in range(w.steps):
-        flush = cache.state()[1] + 1 == w.R
-        ga, gd = (torch.cuda.CUDAGraph() if flush else None), torch.cuda.CUDAGraph()
-        if flush:
-            with torch.cuda.graph(ga, pool=pool):
-                cache.append(tK[s_], tV[s_])
-            with torch.cuda.graph(gd, pool=pool):
-                cache.decode_attention(tQ[s_], out=out)
-        else:
-            with torch.cuda.graph(gd, pool=pool):
-                cache.append_decode(tK[s_], tV[s_], tQ[s_], out=out)
-        g_app.append(ga)
-        g_dec.append(gd)
-    launches_per_episode = kvq.kernel_launches() - launches0
-    # the whole episode as one graph: what `value` times
+    launches0 = kvq.kernel_launches()
     cache.reset()
     g_ep = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_ep, pool=pool):
         episode()
+    launches_per_episode = kvq.kernel_launches() - launches0
+    # the decode calls after an eager prefill, and (separately) the flush steps' appends
+    cache.reset()
+    cache.prefill_quantize(XK, XV)
+    torch.cuda.synchronize()
+    flush_steps = []
+    g_dec = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_dec, pool=pool):
+        for s in range(w.steps):
+            if cache.state()[1] + 1 == w.R:
+                flush_steps.append(s)
+                cache.append(tK[s], tV[s])
+                if scrub:
+                    scrub()
+                cache.decode_attention(tQ[s], out=out)
+            else:
+                if scrub:
+                    scrub()
+                cache.append_decode(tK[s], tV[s], tQ[s], out=out)
+    # what the decode graph holds besides the decode calls: each flush step's append (its own
+    # graph, captured at that step's state: the steps in between run eagerly) and the scrubs
+    side = []
+    if flush_steps:
+        cache.reset()
+        cache.prefill_quantize(XK, XV)
+        for s in range(w.steps):
+            if s in flush_steps:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, pool=pool):
+                    cache.append(tK[s], tV[s])
+                g.replay()
+                side.append(g)
+            else:
+                cache.append(tK[s], tV[s])
+    if scrub:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, pool=pool):
+            for s in range(w.steps):
+                scrub()
+        side.append(g)
     torch.cuda.synchronize()
 
-    def replay_episode(ev):
-        g_pre.replay()
-        for s_ in range(w.steps):
-            if g_app[s_] is not None:
-                g_app[s_].replay()
-            ev[s_][0].record(stream)
-            g_dec[s_].replay()
-            ev[s_][1].record(stream)
+    def replay_side():
+        for g in side:
+            g.replay()
 
-    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(w.steps)] for _ in range(args.steps + 1)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
-        g_ep.replay()                    # graph warm-up (also gives the sampler time to start)
-        replay_episode(evs[-1])
+        g_ep.replay()
+        g_dec.replay()
+        replay_side()
         torch.cuda.synchronize()
         barrier()
         torch.cuda.synchronize()
         # timed region: K episodes, each one whole-episode graph replay
-        start.record(stream)
-        for k in range(args.steps):
-            g_ep.replay()
-        stop.record(stream)
-        torch.cuda.synchronize()
+        ms = _replay_ms(g_ep, args.steps, stream)
         barrier()
-        # the same K episodes replayed step by step, with events around every
-        # decode_attention call: the per-call duration the roofline uses
-        for k in range(args.steps):
-            replay_episode(evs[k])
-        torch.cuda.synchronize()
+        dec_ms = _replay_ms(g_dec, args.steps, stream)
+        side_ms = 0.0
+        if side:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                replay_side()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            side_ms = e0.elapsed_time(e1)
         barrier()
     launches = launches_per_episode * args.steps
-    ms = start.elapsed_time(stop)
-    decode_ms = sum(a.elapsed_time(b) for ev in evs[:args.steps] for a, b in ev)
+    decode_ms = max(dec_ms - side_ms, 1e-6)
     ms, decode_ms = max_over_ranks([ms, decode_ms], world, dev)
+    del g_dec, side
 
-    # ---- end to end through the public API with pinned host buffers ----
     e2e = None
-    if not args.no_e2e:
+    if headline and not args.no_e2e:
         XKp, XVp = to_t(XK_h, True), to_t(XV_h, True)
         tKp, tVp, tQp = to_t(tK_h, True), to_t(tV_h, True), to_t(tQ_h, True)
         outs = torch.empty((w.steps, w.B, w.Hq, w.d), dtype=torch.float32).pin_memory()
@@ -344,19 +375,99 @@ def run_kvq(args):
         g2.replay()
         torch.cuda.synchronize()
         barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            g2.replay()
-        e1.record(stream)
-        torch.cuda.synchronize()
+        e2e_ms, = max_over_ranks([_replay_ms(g2, args.steps, stream)], world, dev)
         barrier()
-        e2e_ms, = max_over_ranks([e0.elapsed_time(e1)], world, dev)
         h2d = XKp.numel() * 2 * 2 + w.steps * (2 * w.B * w.Hkv * w.d + w.B * w.Hq * w.d) * 2
         d2h = w.steps * w.B * w.Hq * w.d * 4
         e2e = {"value": job_throughput(tokens_per_episode * args.steps, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms / args.steps}
+        del g2
+
+    peak, peak_kind = peaks()
+    per_call_ms = decode_ms / (args.steps * w.steps)
+    bytes_per_call = sum(call_bytes) / w.steps
+    achieved = bytes_per_call / (per_call_ms / 1e3) / 1e9
+    res = {
+        "workload": w.name,
+        "value": job_throughput(tokens_per_episode * args.steps, world, ms),
+        "ms_per_step": ms / args.steps,
+        "decode_steps_per_s": w.steps * args.steps / (ms / 1e3),
+        "kv_tokens_per_s_decode_only": job_throughput(tokens_per_episode * args.steps, world, decode_ms),
+        "splits": cache.splits(),
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+        "e2e": e2e,
+        "roofline": {
+            "kernel": f"append + decode_attention ({decode_kernel_name(w)}: one launch without a flush, "
+                      "splits merged in-kernel), per call",
+            "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+            if peak_kind == "measured" else "fallback 6.65 TB/s",
+            "algorithmic_bytes_per_launch": bytes_per_call,
+            "avg_launch_us": per_call_ms * 1e3,
+            "l2": "cold: a read of 2 x L2 before every timed call (its time subtracted)" if cold else
+                  "inputs larger than L2 (calls back to back)",
+            "timing_ms": {"decode_graph": dec_ms, "side_graph": side_ms, "replays": args.steps},
+            "traffic": ncu_traffic(w),
+        },
+        "config": {
+            "workload": w.name, "batch_per_gpu": w.B, "global_batch": w.B * world,
+            "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d, "prompt_tokens": w.T,
+            "decode_steps": w.steps, "bits": w.bits, "group_k": w.G, "group_v": w.Gv,
+            "residual": w.R, "symmetric": w.symmetric, "key_outliers_per_token": args.key_outliers,
+            "elem": "fp16" if w.dtype == wl.FP16 else "bf16",
+        },
+    }
+    del cache, XK, XV, tK, tV, tQ, g_ep, scrub
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_kvq(args):
+    import torch
+    import torch.distributed as dist
+
+    from bit_kv_cache_22_b200 import workloads as wl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
+
+    w = shard_workload(wl.WORKLOADS[args.workload], rank)
+
+    if args.ncu_case:
+        from bit_kv_cache_22_b200 import kvq
+        dt = torch.float16 if w.dtype == wl.FP16 else torch.bfloat16
+
+        def to_t(bits):
+            return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(dt).to(dev)
+        XK, XV = (to_t(x) for x in wl.prefill_bits(w))
+        tK, tV, tQ = (to_t(x) for x in wl.decode_bits(w))
+        cache = kvq.KVQCache(w.B, w.Hq, w.Hkv, w.d, w.G, w.Gv, w.R, w.bits, w.symmetric, dt,
+                             w.capacity, dev, key_outliers=args.key_outliers)
+        out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
+        cache.prefill_quantize(XK, XV)
+        for s in range(min(w.steps, 64)):      # ends mid-episode (r = 64 residual rows at most)
+            cache.append_decode(tK[s], tV[s], tQ[s], out=out)
+        torch.cuda.synchronize()
+        print(json.dumps({"ncu_case": args.workload, "state": cache.state()}))
+        return
+
+    head = measure_workload(w, args, dev, local, world, headline=True)
+    extras = {}
+    if world == 1 and not args.no_extra:
+        for name in EXTRA_WORKLOADS:
+            if name != w.name:
+                extras[name] = measure_workload(wl.WORKLOADS[name], args, dev, local, world, headline=False)
 
     if rank != 0:
         if world > 1:
@@ -367,54 +478,38 @@ def run_kvq(args):
     if world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, budget_s=20.0)
 
-    peak, peak_kind = peaks()
-    decode_launch_ms = decode_ms / (args.steps * w.steps)
-    achieved = bytes_per_episode / w.steps / (decode_launch_ms / 1e3) / 1e9
-    traffic = ncu_traffic(w)
+    config = dict(head["config"])
+    config.update({
+        "parallelism": f"dp{world} (independent sequences per GPU)",
+        "splits": head["splits"],
+        "l2": head["roofline"]["l2"],
+        "timing": "value: K whole-episode CUDA-graph replays (prefill + every decode step) between two "
+                  "events; roofline: events inside one graph of the episode's decode calls, K replays",
+    })
     line = {
         "metric": METRIC,
-        "value": job_throughput(tokens_per_episode * args.steps, world, ms),
+        "value": head["value"],
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": ms / args.steps,
+        "ms_per_step": head["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": f"u{w.bits} codes, f32 accumulate",
         "data": "synthetic (seeded; distributions of the workload definition)",
-        "config": {
-            "workload": w.name, "batch_per_gpu": w.B, "global_batch": w.B * world,
-            "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d, "prompt_tokens": w.T,
-            "decode_steps": w.steps, "bits": w.bits, "group_k": w.G, "group_v": w.Gv,
-            "residual": w.R, "symmetric": w.symmetric, "key_outliers_per_token": args.key_outliers,
-            "elem": "fp16" if w.dtype == wl.FP16 else "bf16",
-            "parallelism": f"dp{world} (independent sequences per GPU)",
-            "l2": "inputs larger than L2: packed cache "
-                  f"{bytes_per_episode / w.steps / 1e6:.0f} MB per decode step, prompt "
-                  f"{2 * XK.numel() * 2 / 1e6:.0f} MB per step",
-            "splits": cache.splits(),
-            "timing": "value: K whole-episode CUDA-graph replays between two events; roofline: "
-                      "events around every decode_attention graph in K more episodes replayed "
-                      "step by step",
-        },
-        "decode_steps_per_s": w.steps * args.steps / (ms / 1e3),
-        "kv_tokens_per_s_decode_only": job_throughput(tokens_per_episode * args.steps, world, decode_ms),
-        "roofline": {
-            "kernel": f"append + decode_attention ({decode_kernel_name(w)}: one launch without a flush, "
-                      "splits merged in-kernel), per call",
-            "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
-            if peak_kind == "measured" else "fallback 6.65 TB/s",
-            "algorithmic_bytes_per_launch": bytes_per_episode / w.steps,
-            "avg_launch_us": decode_launch_ms * 1e3,
-            "traffic": traffic,
-        },
+        "config": config,
+        "decode_steps_per_s": head["decode_steps_per_s"],
+        "kv_tokens_per_s_decode_only": head["kv_tokens_per_s_decode_only"],
+        "roofline": head["roofline"],
         "cpu_baseline": cpu,
-        "e2e": e2e,
-        "gpu_launches": int(launches),
-        "clocks": clk.summary(),
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
+        "clocks": head["clocks"],
+        "workloads": {name: {k: r[k] for k in ("value", "ms_per_step", "decode_steps_per_s", "roofline",
+                                                "splits", "gpu_launches", "clocks", "config")}
+                      for name, r in extras.items()},
     }
     print(json.dumps(line))
     if world > 1:
@@ -625,30 +720,61 @@ def run_paged(args):
 # the CPU oracle (cpu_baseline leg and --impl reference)
 # ---------------------------------------------------------------------------
 
-def cpu_baseline(w, budget_s=20.0, steps=None):
-    """Time the oracle (as it stands) on a bounded sample of the workload: one
-    sequence (all of its kv heads), its prompt prefill and the first decode
-    steps, stopping after ~budget_s seconds.  Returns KV tokens/s for that sample."""
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), or the platform's processor string."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.lower().startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def _oracle_sample(w, budget_s, XK, XV, tK, tV, tQ):
+    """One timed oracle run: prefill of one sequence, then decode steps until budget_s."""
     import oracle
-    from bit_kv_cache_22_b200 import workloads as wl
-    XK, XV = wl.prefill_bits(w, bs=[0])
-    tK, tV, tQ = wl.decode_bits(w, bs=[0])
     t0 = time.perf_counter()
     c = oracle.OracleCache(1, w.Hq, w.Hkv, w.d, w.G, w.Gv, w.R, w.bits, w.symmetric, w.dtype)
     c.prefill(XK, XV)
     tokens, done = 0, 0
-    limit = w.steps if steps is None else steps
-    for s in range(limit):
+    for s in range(w.steps):
         c.append(tK[s], tV[s])
         c.decode(tQ[s])
         tokens += c.Tq + c.r
         done += 1
         if time.perf_counter() - t0 > budget_s:
             break
-    el = time.perf_counter() - t0
-    return {"value": tokens / el, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"1 of {w.B} sequences (all {w.Hkv} kv heads): prefill of {w.T} tokens + "
-                      f"{done} of {w.steps} decode steps, {el:.1f} s, fp64 C oracle with OpenMP"}
+    return tokens, done, time.perf_counter() - t0
+
+
+def cpu_baseline(w, budget_s=20.0, one_core_s=8.0):
+    """Time the oracle (as it stands) on a bounded sample of the workload: one
+    sequence (all of its kv heads), its prompt prefill and the first decode
+    steps, stopping after ~budget_s seconds, on all the threads the oracle uses;
+    then the same sample on one thread for ~one_core_s seconds.  KV tokens/s."""
+    import oracle
+    from bit_kv_cache_22_b200 import workloads as wl
+    XK, XV = wl.prefill_bits(w, bs=[0])
+    tK, tV, tQ = wl.decode_bits(w, bs=[0])
+    threads = oracle.num_threads()
+    tokens, done, el = _oracle_sample(w, budget_s, XK, XV, tK, tV, tQ)
+    res = {"value": tokens / el, "unit": UNIT, "cores": threads, "kind": "oracle",
+           "cpu_model": cpu_model(), "host_cores": len(os.sched_getaffinity(0)),
+           "sample": f"1 of {w.B} sequences (all {w.Hkv} kv heads): prefill of {w.T} tokens + "
+                     f"{done} of {w.steps} decode steps, {el:.1f} s, fp64 C oracle with OpenMP "
+                     f"on {threads} threads"}
+    if one_core_s > 0:
+        old = oracle.set_num_threads(1)
+        try:
+            t1, d1, e1 = _oracle_sample(w, one_core_s, XK, XV, tK, tV, tQ)
+        finally:
+            oracle.set_num_threads(old)
+        res["one_core"] = {"value": t1 / e1, "unit": UNIT, "cores": 1,
+                           "sample": f"the same sample on 1 thread: prefill + {d1} decode steps, {e1:.1f} s"}
+    return res
 
 
 def run_reference(args):
@@ -659,8 +785,8 @@ def run_reference(args):
     w = wl.WORKLOADS[args.workload]
     budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
-        cpu_baseline(w, budget_s=budget)
-    vals = [cpu_baseline(w, budget_s=budget) for _ in range(args.steps)]
+        cpu_baseline(w, budget_s=budget, one_core_s=0)
+    vals = [cpu_baseline(w, budget_s=budget, one_core_s=0) for _ in range(args.steps)]
     v = statistics.mean(x["value"] for x in vals)
     line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
@@ -668,6 +794,7 @@ def run_reference(args):
             "data": "synthetic (seeded)",
             "config": {"workload": w.name, "global_batch": w.B, "note": "CPU oracle, rank 0"},
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": vals[0]["cores"],
+                             "cpu_model": vals[0]["cpu_model"], "host_cores": vals[0]["host_cores"],
                              "kind": "oracle", "sample": vals[0]["sample"]},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))

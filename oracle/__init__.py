@@ -83,6 +83,8 @@ def _load():
                                                 i32, i64, i32, i32, i32, i32, i32, i32, i32, P, P, P]
         lib.oracle_num_threads.restype = i32
         lib.oracle_num_threads.argtypes = []
+        lib.oracle_set_num_threads.restype = i32
+        lib.oracle_set_num_threads.argtypes = [i32]
         _lib = lib
         return lib
 
@@ -99,6 +101,12 @@ def _check(rc: int, what: str):
 
 def num_threads() -> int:
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> int:
+    """Threads the oracle's parallel sections use from now on; returns the previous count.
+    Results do not depend on it (every parallel section writes disjoint outputs)."""
+    return int(_load().oracle_set_num_threads(int(n)))
 
 
 # ----------------------------------------------------------------------------

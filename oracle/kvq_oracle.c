@@ -461,3 +461,17 @@ int oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* Threads of the later parallel sections (n >= 1); returns the previous count.
+ * Only the timing of the oracle depends on it, never a result. */
+int oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    const int old = omp_get_max_threads();
+    if (n >= 1) omp_set_num_threads(n);
+    return old;
+#else
+    (void)n;
+    return 1;
+#endif
+}

@@ -48,3 +48,13 @@ def test_decode_only_line_keys():
     assert r["bound"] == "hbm" and r["unit"] == "GB/s" and abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-12
     assert abs(line["value"] - 10 ** 9 / 0.010) < 1e-3                # tokens over the slowest rank's time
     assert line["config"]["workload"] == "x" and "l2" in line["config"]
+
+
+def test_cpu_baseline_reports_model_cores_and_one_core():
+    w = wl.WORKLOADS["tiny"].replace(steps=2)
+    r = bench.cpu_baseline(w, budget_s=0.5, one_core_s=0.2)
+    assert r["kind"] == "oracle" and r["value"] > 0 and r["cores"] >= 1
+    assert r["cpu_model"] and r["host_cores"] >= 1
+    assert r["one_core"]["cores"] == 1 and r["one_core"]["value"] > 0
+    import oracle
+    assert oracle.num_threads() == r["cores"]          # the thread count is restored
