@@ -1,7 +1,7 @@
 // decode.cu -- decode attention over contiguous caches, the merge of token-split
 // partials, and the dispatch between contiguous, paged and dense-and-sparse caches.
-// The kernels are in decode_kernels.cuh; decode_paged.cu and decode_sparse.cu hold
-// their other instances.
+// The kernels are in decode_kernels.cuh and decode_mma.cuh; decode_paged.cu,
+// decode_sparse.cu and decode_mma.cu hold their other instances.
 #include "decode_kernels.cuh"
 
 namespace kvq {
@@ -40,15 +40,23 @@ cudaError_t launch_merge_partials(const float *o_all, const float *m_all, const 
     return cudaGetLastError();
 }
 
+int binary_version() {
+    cudaFuncAttributes at{};
+    if (cudaFuncGetAttributes(&at, merge_partials_kernel) != cudaSuccess) return -1;
+    return at.binaryVersion;
+}
+
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
     if (a.page_table) return launch_decode_paged(a, s);
     if (a.k_out) return launch_decode_sparse(a, s);
+    if (a.path == kPathMma) return launch_decode_mma(a, s);
     return launch_decode_variant<false>(a, s);
 }
 
 int decode_ctas_per_sm(const DecodeArgs &a) {
     if (a.page_table) return decode_ctas_per_sm_paged(a);
     if (a.k_out) return decode_ctas_per_sm_sparse(a);
+    if (a.path == kPathMma) return decode_ctas_per_sm_mma(a);
     return ctas_per_sm_variant<false>(a);
 }
 

@@ -261,6 +261,11 @@ struct PageWindow {
     }
 };
 
+// Floats of shared scratch finish_cta needs after the per-warp outputs (wts): the split
+// weights HG (S + 1), S <= 80, padded to 4, and the [P][C] float4 sums of the merge.
+template <int HG, int D>
+__host__ __device__ constexpr int finish_scratch_floats() { return (HG * 81 + 3) / 4 * 4 + 4 * kDecodeThreads; }
+
 // End of every decode CTA.  o_w [warp][HG][D] and ml_w [warp][HG] = (m, l) are
 // the per-warp partials of the CTA's HG query heads (unnormalised, log2
 // domain; m = -inf for a warp without tokens).  They are merged into the CTA's
@@ -334,15 +339,39 @@ __device__ __forceinline__ void finish_cta(const DecodeArgs &a, const float *o_w
         if (lane == 0) wts[HG * a.S + hh] = L;
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < HG * D; i += kDecodeThreads) {
-        const int hh = i / D, c = i % D;
-        const float *op = a.o_part + (bq0 + hh) * a.S * D + c;
+    // weighted sum of the S partials: thread t takes 4 channels (float4 column t mod C of the
+    // HG x D outputs) and every P-th split from t / C, with 16 loads in flight; the P partial
+    // sums of a column are then added through shared memory (finish_scratch_floats<HG, D>)
+    constexpr int C = HG * D / 4;                       // float4 columns
+    constexpr int P = kDecodeThreads / C;
+    static_assert(kDecodeThreads % C == 0, "columns");
+    float4 *red = reinterpret_cast<float4 *>(wts + ((HG * (a.S + 1) + 3) & ~3));   // [P][C]
+    {
+        const int col = threadIdx.x % C, part = threadIdx.x / C;
+        const int hh = (4 * col) / D, c = (4 * col) % D;
+        const float4 *op = reinterpret_cast<const float4 *>(a.o_part + (bq0 + hh) * a.S * D + c);
         const float *wp = wts + hh * a.S;
-        float o = 0.f;
-#pragma unroll 8
-        for (int s = 0; s < a.S; ++s) o = fmaf(__ldcg(op + static_cast<int64_t>(s) * D), wp[s], o);
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 16
+        for (int s = part; s < a.S; s += P) {
+            const float4 v = __ldcg(op + static_cast<int64_t>(s) * (D / 4));
+            const float wgt = wp[s];
+            o.x = fmaf(v.x, wgt, o.x); o.y = fmaf(v.y, wgt, o.y);
+            o.z = fmaf(v.z, wgt, o.z); o.w = fmaf(v.w, wgt, o.w);
+        }
+        red[part * C + col] = o;
+    }
+    __syncthreads();
+    for (int col = threadIdx.x; col < C; col += kDecodeThreads) {
+        float4 o = red[col];
+#pragma unroll
+        for (int q = 1; q < P; ++q) {
+            const float4 v = red[q * C + col];
+            o.x += v.x; o.y += v.y; o.z += v.z; o.w += v.w;
+        }
+        const int hh = (4 * col) / D, c = (4 * col) % D;
         if (a.po) {   // the cache's partial (token-split decode): o and l relative to M
-            a.po[(bq0 + hh) * D + c] = o;
+            *reinterpret_cast<float4 *>(a.po + (bq0 + hh) * D + c) = o;
             if (c == 0) {
                 float M = -INFINITY;
                 for (int s = 0; s < a.S; ++s) M = fmaxf(M, __ldcg(a.m_part + (bq0 + hh) * a.S + s));
@@ -351,7 +380,9 @@ __device__ __forceinline__ void finish_cta(const DecodeArgs &a, const float *o_w
             }
         } else {
             const float L = wts[HG * a.S + hh];
-            a.out[(bq0 + hh) * D + c] = L > 0.f ? o / L : 0.f;
+            *reinterpret_cast<float4 *>(a.out + (bq0 + hh) * D + c) =
+                L > 0.f ? make_float4(o.x / L, o.y / L, o.z / L, o.w / L)    // an empty sequence gives 0
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
     if (threadIdx.x == 0) a.arrivals[unit] = 0u;
@@ -367,6 +398,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_split_kernel(const D
     constexpr int NGV = D / GV;       // value groups per token
     constexpr uint32_t BYTE_MASK = ((1u << N) - 1u) * 0x01010101u;
     using St = Stage<N, D, GV>;
+    static_assert(finish_scratch_floats<1, D>() * 4 <= kDecodeWarps * kStages * St::kBytes, "merge scratch");
 
     __shared__ float q_s[D];
     __shared__ float o_s[kDecodeWarps][D];
@@ -997,7 +1029,7 @@ __global__ void __launch_bounds__(kDecodeThreads, tc_min_ctas<D, GV, HG>()) deco
     static_assert(W % 2 == 0, "key MMAs take words in pairs");
     static_assert(kChunk % kTcItem == 0 && (kChunk & (kChunk - 1)) == 0, "chunk");
     static_assert(residual_scratch_bytes<D>() <= Sm::kBars, "residual staging");
-    static_assert(kDecodeWarps * HG * D * 4 + HG * 66 * 4 <= (kDecodeWarps - 1) * Sm::kWarpBytes + Sm::kBars,
+    static_assert((kDecodeWarps * HG * D + finish_scratch_floats<HG, D>()) * 4 <= kDecodeWarps * Sm::kWarpBytes,
                   "epilogue");
 
     __shared__ __align__(16) float q_s[HG][D];

@@ -52,5 +52,5 @@ def test_header_compiles_as_c_and_links():
         assert out.returncode == 0, (out.returncode, out.stderr)
         k_codes, nq, per, S, pt, layout = out.stdout.split()
         assert int(k_codes) == 8 * 32 * 4352 * 128 * 4 // 8      # sizes of the last valid config
-        assert (int(nq), int(per), int(S)) == (2, 128, 2)
+        assert (int(nq), int(per), int(S)) == (2, 128, 3)      # 2 quantized splits + 1 residual split
         assert int(pt) == 8 * (4352 // 128) * 4 and int(layout) == 2
