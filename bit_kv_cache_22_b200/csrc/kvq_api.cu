@@ -101,21 +101,35 @@ int max_splits(const kvq_config *c) {
     return static_cast<int>(tiles < kMaxSplits ? tiles : kMaxSplits) + kMaxResidualSplits;
 }
 
+// The state buffer: split-arrival counters [B * Hq] and the status word (u32), padded to
+// 16 bytes; a LogQuant cache adds its row lists, a paged cache its slots' lengths.
+size_t counter_bytes(const kvq_config *c) {
+    const size_t n = (static_cast<size_t>(c->batch) * c->q_heads + 1) * sizeof(unsigned int);
+    return (n + 15) / 16 * 16;
+}
+size_t lq_list_entries(const kvq_config *g, int32_t W) {
+    return static_cast<size_t>(W) + static_cast<size_t>(g->capacity) + 3 * static_cast<size_t>(W);
+}
+
 }  // namespace
 
 struct kvq_cache {
     kvq_config cfg;
     kvq_buffers buf;
-    unsigned int *arrivals = nullptr;   // device, B * Hq split-arrival counters (library-owned)
+    unsigned int *arrivals = nullptr;   // device, in the caller's state buffer: B * Hq split-arrival
+                                        // counters, then the status word
     int64_t Tq = 0;
     int32_t r = 0;
     int num_sms = 148;
     int ctas_per_sm = 4;
     int split_limit = 64;
+    int path = kvq::kPathSplit;         // the decode kernel (kvq::DecodePath) serving this cache
+    int stall_polls = 0;                // bounds-check builds: see kvq_debug_set_stall
     // LogQuant retention (lq_window W > 0): the residual buffer is the full-precision store
     // of up to 3W rows (cfg.residual = 3W), rows in ascending token position; lq_F holds
-    // those positions, lq_n the tokens seen.  lq_rows (device, library-owned): [0, W) the
-    // rows an event quantizes (1, 3, ..., 2W - 1), then room for a prefill's row lists.
+    // those positions, lq_n the tokens seen.  lq_rows (device, in the caller's state buffer
+    // after the counters): [0, W) the rows an event quantizes (1, 3, ..., 2W - 1), then room
+    // for a prefill's row lists.
     int32_t lq_window = 0;
     int32_t *lq_rows = nullptr;
     // dense-and-sparse keys: n_out outlier words per token (caller-owned), or none
@@ -155,21 +169,22 @@ void plan_splits_for(const kvq_cache *h, const PlanInput &in, int *n_qsplits, in
     const kvq_config &c = h->cfg;
     int64_t tiles = 0;
     for (int i = 0; i < in.n; ++i) tiles = in.tiles[i] > tiles ? in.tiles[i] : tiles;
-    const int path = kvq::decode_path(c.q_heads, c.kv_heads, c.group_k);
-    // with one query head per kv head the tensor-core kernel deals the residual tiles to the
+    const int path = h->path;
+    // with one query head per kv head the integer-MMA kernel deals the residual tiles to the
     // warps of the quantized splits
     const int hg = c.q_heads / c.kv_heads;
     const bool res_shared = path == kvq::kPathTc && hg == 1;
+    const bool per_kv = kvq::path_per_kv_head(path);
     const int extra = (in.max_r > 0 && !res_shared) ? 1 : 0;   // residual splits (the tensor-core
                                                                 // path may take more, below)
     const int64_t align = kvq::split_tile_align(path);
     // CTAs per split and sequence: one per kv head on the tensor-core path, else one per query head
-    const int64_t per_seq = path == kvq::kPathTc ? c.kv_heads : c.q_heads;
+    const int64_t per_seq = per_kv ? c.kv_heads : c.q_heads;
     const int64_t units = static_cast<int64_t>(c.batch) * per_seq;
     const double slots = static_cast<double>(h->num_sms) * h->ctas_per_sm;
     const int64_t nres = (in.max_r + 15) / 16;
     // residual CTA: its tiles shared by the 4 warps of each of its query heads
-    const int heads_per_cta = path == kvq::kPathTc ? hg : 1;
+    const int heads_per_cta = per_kv ? hg : 1;
     const double c_res1 = kCtaFixedTiles + static_cast<double>((nres * heads_per_cta + 3) / 4);
     // the tensor-core kernel deals the residual tiles over the warps of n_rs residual splits
     // (4 / HG warps per head in each); a residual tile on CUDA cores costs about two
@@ -202,12 +217,12 @@ void plan_splits_for(const kvq_cache *h, const PlanInput &in, int *n_qsplits, in
             // residual warp).  Residual CTAs start after every quantized CTA (the grid's order):
             // when they do not all fit beside the quantized ones, they add to the critical path.
             int64_t most = 1;
-            if (extra && path == kvq::kPathTc) {
+            if (extra && per_kv) {
                 most = (nres + wph - 1) / wph;
                 if (most > kMaxResidualSplits) most = kMaxResidualSplits;
             }
             for (int64_t n_rs = extra; n_rs <= (extra ? most : 0); ++n_rs) {
-                const double c_res = (path == kvq::kPathTc && n_rs) ? residual_cost(n_rs) : c_res1;
+                const double c_res = (per_kv && n_rs) ? residual_cost(n_rs) : c_res1;
                 const double n_res = static_cast<double>(units * n_rs);
                 const double t_spread =
                     (nq * c_q + n_empty * kEmptyCtaTiles + n_res * c_res) / slots + (n_rs ? c_res : 0.0);
@@ -228,7 +243,7 @@ void plan_splits_for(const kvq_cache *h, const PlanInput &in, int *n_qsplits, in
         best_S = 1;
         best_per = 0;
     }
-    if (best_S == 0 && extra && path == kvq::kPathTc) {   // residual rows only: spread them too
+    if (best_S == 0 && extra && per_kv) {   // residual rows only: spread them too
         int64_t most = (nres + wph - 1) / wph;
         if (most > kMaxResidualSplits) most = kMaxResidualSplits;
         const int64_t want = (static_cast<int64_t>(slots) + units - 1) / units;
@@ -274,7 +289,7 @@ kvq::DecodeArgs decode_args(const kvq_cache *h) {
     a.bits = c.bits;
     a.sym = c.symmetric != 0;
     a.bf16 = c.dtype == KVQ_BF16;
-    a.path = kvq::decode_path(c.q_heads, c.kv_heads, c.group_k);
+    a.path = h->path;
     a.arrivals = h->arrivals;
     a.status = h->arrivals + static_cast<int64_t>(c.batch) * c.q_heads;
     a.k_out = h->k_out;
@@ -282,6 +297,7 @@ kvq::DecodeArgs decode_args(const kvq_cache *h) {
     a.gshift = 0;
     while ((16 << a.gshift) < c.group_k) ++a.gshift;
     a.qscale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c.head_dim)));
+    a.stall_polls = h->stall_polls;
     return a;
 }
 
@@ -304,6 +320,7 @@ kvq::QuantizeArgs quantize_args(const kvq_cache *h) {
     q.cap = c.capacity;
     q.k_out = h->k_out;
     q.n_out = h->n_out;
+    q.status = h->arrivals + static_cast<int64_t>(c.batch) * c.q_heads;
     return q;
 }
 
@@ -350,6 +367,7 @@ kvq_status kvq_get_sizes(const kvq_config *cfg, kvq_sizes *out) {
     out->k_residual = out->v_residual = static_cast<size_t>(BH * cfg->residual * d * 2);
     const int64_t units = static_cast<int64_t>(cfg->batch) * cfg->q_heads;
     out->workspace = static_cast<size_t>(units * max_splits(cfg) * (d + 2) * 4);
+    out->state = counter_bytes(cfg);
     return ok();
 }
 
@@ -360,10 +378,11 @@ kvq_status kvq_create(const kvq_config *cfg, const kvq_buffers *bufs, kvq_cache 
     if (st != KVQ_OK) return st;
     if (!bufs) return fail(KVQ_ERR_INVALID_ARG, "buffers are NULL");
     const void *need[] = {bufs->k_codes, bufs->k_scales, bufs->v_codes, bufs->v_scales,
-                          bufs->k_residual, bufs->v_residual};
+                          bufs->k_residual, bufs->v_residual, bufs->state};
     for (const void *p : need)
         if (!p || !aligned16(p))
-            return fail(KVQ_ERR_INVALID_ARG, "cache buffers must be non-NULL and 16-byte aligned");
+            return fail(KVQ_ERR_INVALID_ARG, "cache buffers and the state buffer must be non-NULL and "
+                                             "16-byte aligned");
     if (!cfg->symmetric && (!bufs->k_zeros || !bufs->v_zeros || !aligned16(bufs->k_zeros) ||
                             !aligned16(bufs->v_zeros)))
         return fail(KVQ_ERR_INVALID_ARG, "asymmetric caches need 16-byte aligned zero buffers");
@@ -380,28 +399,22 @@ kvq_status kvq_create(const kvq_config *cfg, const kvq_buffers *bufs, kvq_cache 
         h->buf.v_zeros = nullptr;
     }
     h->num_sms = sms > 0 ? sms : 148;
+    h->path = kvq::decode_path(cfg->q_heads, cfg->kv_heads, cfg->group_k);
     h->ctas_per_sm = kvq::decode_ctas_per_sm(decode_args(h));
     // the decode kernels' split-arrival counters (zeroed once here, left at zero by every
-    // decode) and, after them, their status word
-    const size_t counter_bytes = (static_cast<size_t>(cfg->batch) * cfg->q_heads + 1) * sizeof(unsigned int);
-    e = cudaMalloc(&h->arrivals, counter_bytes);
-    if (e == cudaSuccess) e = cudaMemset(h->arrivals, 0, counter_bytes);
+    // decode) and, after them, their status word: the start of the caller's state buffer
+    h->arrivals = static_cast<unsigned int *>(bufs->state);
+    e = cudaMemset(h->arrivals, 0, counter_bytes(cfg));
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) {
-        if (h->arrivals) cudaFree(h->arrivals);
         delete h;
-        return cuda_fail(e, "allocating the split-arrival counters");
+        return cuda_fail(e, "zeroing the state buffer");
     }
     *out = h;
     return ok();
 }
 
-void kvq_destroy(kvq_cache *cache) {
-    if (!cache) return;
-    if (cache->arrivals) cudaFree(cache->arrivals);
-    if (cache->lq_rows) cudaFree(cache->lq_rows);
-    delete cache;
-}
+void kvq_destroy(kvq_cache *cache) { delete cache; }
 
 kvq_status kvq_reset(kvq_cache *cache) {
     if (!cache) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
@@ -476,13 +489,14 @@ kvq_status kvq_append(kvq_cache *h, const void *t_K, const void *t_V, void *stre
         q.xv = static_cast<const uint16_t *>(h->buf.v_residual);
         q.in_bh_stride = rstride;
         q.in_rows = h->lq_rows;
+        q.in_rows_limit = c.residual;
         q.n_groups = W / c.group_k;
         q.out_tok0 = h->Tq;
         e = kvq::launch_quantize(q, s);
         if (e == cudaSuccess)
             e = kvq::launch_lq_compact(static_cast<uint16_t *>(h->buf.k_residual),
                                        static_cast<uint16_t *>(h->buf.v_residual), BH, c.residual, W,
-                                       c.head_dim, s);
+                                       c.head_dim, q.status, s);
         if (e != cudaSuccess) return cuda_fail(e, "LogQuant event launch");
         lq_push(h);
         h->Tq += W;
@@ -539,7 +553,7 @@ kvq_status kvq_append_decode_attention(kvq_cache *h, const void *t_K, const void
     if (st != KVQ_OK) return st;
     const kvq_config &c = h->cfg;
     const bool flush = h->r + 1 == c.residual;
-    if (flush || kvq::decode_path(c.q_heads, c.kv_heads, c.group_k) != kvq::kPathTc) {
+    if (flush || !kvq::path_per_kv_head(h->path)) {
         // a flush (or the CUDA-core kernel): the append's own launches, then the decode
         st = kvq_append(h, t_K, t_V, stream);
         if (st != KVQ_OK) return st;
@@ -632,34 +646,23 @@ kvq_status launch_decode_call(kvq_cache *h, const void *t_Q, float *t_O, void *w
 //
 // The split partials live in one file-scope device array instead of caller
 // memory.  Host code cannot use the array's name as a device address (it is a
-// host-side stand-in for the symbol), so the address is looked up with
-// cudaGetSymbolAddress once per device, with that device current, the first
-// time the entry point runs on it.
+// host-side stand-in for the symbol), so every call looks the address up with
+// cudaGetSymbolAddress in the calling thread's current context: a context made
+// after a device reset, or another context on the same device, gets its own
+// array and never a stale address.  The first lookup in a context may load the
+// library's device code.
 // ---------------------------------------------------------------------------
 namespace {
 
 constexpr size_t kNoAllocScratchFloats = size_t{1} << 20;   // 4 MiB per device
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
 
-std::mutex g_noalloc_mutex;
-float *g_noalloc_ptr[kMaxDevices] = {};
-
 kvq_status noalloc_scratch(float **out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return cuda_fail(e, "querying the current device");
-    if (dev < 0 || dev >= kMaxDevices)
-        return fail(KVQ_ERR_UNSUPPORTED, "device ordinal %d is beyond %d", dev, kMaxDevices);
-    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return cuda_fail(e, "looking up the static decode scratch");
-        g_noalloc_ptr[dev] = static_cast<float *>(p);
-    }
-    *out = g_noalloc_ptr[dev];
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "looking up the static decode scratch");
+    *out = static_cast<float *>(p);
     return KVQ_OK;
 }
 
@@ -714,6 +717,8 @@ uint64_t kvq_kernel_launches(void) { return g_launches.load(); }
 const char *kvq_last_error(void) { return g_last_error.c_str(); }
 
 int32_t kvq_layout_version(void) { return 2; }
+
+int32_t kvq_binary_arch(void) { return kvq::binary_version(); }
 
 }  // extern "C"
 
@@ -801,11 +806,13 @@ kvq_status check_status_word(unsigned int *word) {
     e = cudaMemset(word, 0, sizeof v);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
-    if (v & 2u)
-        return fail(KVQ_ERR_INVALID_ARG, "a kernel met a page-table entry outside the pool; "
-                                         "outputs since the last check are unreliable");
-    return fail(KVQ_ERR_CUDA, "a decode kernel gave up waiting for a copy into shared memory; "
-                              "outputs since the last check are unreliable");
+    std::string why;
+    if (v & 1u) why += " a decode kernel gave up waiting for a copy into shared memory;";
+    if (v & 2u) why += " a kernel met a page-table entry outside the pool;";
+    if (v & 4u) why += " a quantizer met a scale outside the range the decode kernels serve;";
+    if (v & 8u) why += " a kernel met a list index outside its buffer (bounds-check build);";
+    return fail(KVQ_ERR_DEVICE_CHECK, "device check (status 0x%x):%s outputs since the last check are "
+                                      "unreliable", v, why.c_str());
 }
 
 }  // namespace
@@ -830,6 +837,7 @@ kvq_status kvq_paged_get_sizes(const kvq_paged_config *cfg, kvq_paged_sizes *out
     out->page_table = static_cast<size_t>(static_cast<int64_t>(g.batch) * (g.capacity / P) * 4);
     const int64_t units = static_cast<int64_t>(g.batch) * g.q_heads;
     out->workspace = static_cast<size_t>(units * max_splits(&g) * (d + 2) * 4);
+    out->state = counter_bytes(&g) + (static_cast<size_t>(g.batch) * 4 + 15) / 16 * 16;
     return ok();
 }
 
@@ -843,10 +851,11 @@ kvq_status kvq_paged_create(const kvq_paged_config *cfg, const kvq_buffers *bufs
     if (!page_table || !aligned16(page_table))
         return fail(KVQ_ERR_INVALID_ARG, "page_table must be non-NULL and 16-byte aligned");
     const void *need[] = {bufs->k_codes, bufs->k_scales, bufs->v_codes, bufs->v_scales,
-                          bufs->k_residual, bufs->v_residual};
+                          bufs->k_residual, bufs->v_residual, bufs->state};
     for (const void *p : need)
         if (!p || !aligned16(p))
-            return fail(KVQ_ERR_INVALID_ARG, "cache buffers must be non-NULL and 16-byte aligned");
+            return fail(KVQ_ERR_INVALID_ARG, "cache buffers and the state buffer must be non-NULL and "
+                                             "16-byte aligned");
     const kvq_config &g = cfg->geom;
     if (!g.symmetric && (!bufs->k_zeros || !bufs->v_zeros || !aligned16(bufs->k_zeros) ||
                          !aligned16(bufs->v_zeros)))
@@ -875,20 +884,21 @@ kvq_status kvq_paged_create(const kvq_paged_config *cfg, const kvq_buffers *bufs
     h->max_pages = static_cast<int32_t>(g.capacity / cfg->page_tokens);
     h->page_table = page_table;
     h->base.num_sms = sms > 0 ? sms : 148;
-    // counters [B * Hq], status word, slot lengths [B] (all -1: inactive)
-    const size_t counters = static_cast<size_t>(g.batch) * g.q_heads + 1;
-    const size_t bytes = (counters + g.batch) * sizeof(unsigned int);
-    e = cudaMalloc(&h->base.arrivals, bytes);
-    if (e == cudaSuccess) e = cudaMemset(h->base.arrivals, 0, counters * sizeof(unsigned int));
-    if (e == cudaSuccess) e = cudaMemset(h->base.arrivals + counters, 0xff, g.batch * sizeof(unsigned int));
+    h->base.path = kvq::decode_path(g.q_heads, g.kv_heads, g.group_k, false);
+    // the caller's state buffer: counters [B * Hq] and the status word (zeroed), then the
+    // slots' lengths [B] (all -1: inactive)
+    h->base.arrivals = static_cast<unsigned int *>(bufs->state);
+    const size_t cb = counter_bytes(&g);
+    e = cudaMemset(h->base.arrivals, 0, cb);
+    if (e == cudaSuccess)
+        e = cudaMemset(static_cast<unsigned char *>(bufs->state) + cb, 0xff, g.batch * sizeof(unsigned int));
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) {
-        if (h->base.arrivals) cudaFree(h->base.arrivals);
         delete[] h->len;
         delete h;
-        return cuda_fail(e, "allocating the paged cache's counters");
+        return cuda_fail(e, "initialising the paged cache's state buffer");
     }
-    h->seq_len = reinterpret_cast<int32_t *>(h->base.arrivals + counters);
+    h->seq_len = reinterpret_cast<int32_t *>(static_cast<unsigned char *>(bufs->state) + cb);
     h->base.ctas_per_sm = kvq::decode_ctas_per_sm(paged_decode_args(h));
     *out = h;
     return ok();
@@ -896,7 +906,6 @@ kvq_status kvq_paged_create(const kvq_paged_config *cfg, const kvq_buffers *bufs
 
 void kvq_paged_destroy(kvq_paged *h) {
     if (!h) return;
-    if (h->base.arrivals) cudaFree(h->base.arrivals);
     delete[] h->len;
     delete h;
 }
@@ -1096,15 +1105,16 @@ kvq_status lq_prefill(kvq_cache *h, const void *X_K, const void *X_V, int64_t T,
     q.xv = static_cast<const uint16_t *>(X_V);
     q.in_bh_stride = T * c.head_dim;
     q.in_rows = dev_lists;
+    q.in_rows_limit = T;
     q.n_groups = Tq / c.group_k;
     q.out_tok0 = 0;
     e = kvq::launch_quantize(q, s);
     if (e != cudaSuccess) return cuda_fail(e, "LogQuant prefill quantize launch");
     const int64_t BH = static_cast<int64_t>(c.batch) * c.kv_heads;
     e = kvq::launch_gather_rows(static_cast<const uint16_t *>(X_K), static_cast<const uint16_t *>(X_V),
-                                T * c.head_dim, dev_lists + Tq, static_cast<int>(F.size()),
+                                T * c.head_dim, T, dev_lists + Tq, static_cast<int>(F.size()),
                                 static_cast<uint16_t *>(h->buf.k_residual), static_cast<uint16_t *>(h->buf.v_residual),
-                                static_cast<int64_t>(c.residual) * c.head_dim, BH, c.head_dim, s);
+                                static_cast<int64_t>(c.residual) * c.head_dim, BH, c.head_dim, q.status, s);
     if (e != cudaSuccess) return cuda_fail(e, "LogQuant prefill store launch");
     h->Tq = Tq;
     h->r = static_cast<int32_t>(F.size());
@@ -1122,7 +1132,9 @@ kvq_status kvq_logquant_get_sizes(const kvq_config *cfg, int32_t window, kvq_siz
     kvq_status st = validate_lq(cfg, window);
     if (st != KVQ_OK) return st;
     const kvq_config g = lq_geometry(cfg, window);
-    return kvq_get_sizes(&g, out);
+    st = kvq_get_sizes(&g, out);
+    if (st == KVQ_OK) out->state += lq_list_entries(&g, window) * sizeof(int32_t);
+    return st;
 }
 
 kvq_status kvq_logquant_create(const kvq_config *cfg, int32_t window, const kvq_buffers *bufs, kvq_cache **out) {
@@ -1136,15 +1148,15 @@ kvq_status kvq_logquant_create(const kvq_config *cfg, int32_t window, const kvq_
     if (st != KVQ_OK) return st;
     h->lq_window = window;
     h->lq_F.reserve(3 * static_cast<size_t>(window));
-    // rows 1, 3, ..., 2W - 1, then room for a prefill's lists (capacity + 3W entries)
-    const size_t n = static_cast<size_t>(window) + static_cast<size_t>(g.capacity) + 3 * static_cast<size_t>(window);
+    // in the state buffer after the counters: rows 1, 3, ..., 2W - 1, then room for a
+    // prefill's lists (capacity + 3W entries)
+    h->lq_rows = reinterpret_cast<int32_t *>(static_cast<unsigned char *>(bufs->state) + counter_bytes(&g));
     std::vector<int32_t> odd(static_cast<size_t>(window));
     for (int32_t i = 0; i < window; ++i) odd[i] = 2 * i + 1;
-    cudaError_t e = cudaMalloc(&h->lq_rows, n * sizeof(int32_t));
-    if (e == cudaSuccess) e = cudaMemcpy(h->lq_rows, odd.data(), odd.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
+    cudaError_t e = cudaMemcpy(h->lq_rows, odd.data(), odd.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) {
         kvq_destroy(h);
-        return cuda_fail(e, "allocating the LogQuant row lists");
+        return cuda_fail(e, "writing the LogQuant row list");
     }
     *out = h;
     return ok();
@@ -1174,10 +1186,11 @@ kvq_status kvq_set_key_outliers(kvq_cache *h, int32_t n_out, uint32_t *k_outlier
     if (n_out == 0) {
         h->k_out = nullptr;
         h->n_out = 0;
+        h->path = kvq::decode_path(c.q_heads, c.kv_heads, c.group_k);
         h->ctas_per_sm = kvq::decode_ctas_per_sm(decode_args(h));
         return ok();
     }
-    if (kvq::decode_path(c.q_heads, c.kv_heads, c.group_k) != kvq::kPathTc)
+    if (kvq::decode_path(c.q_heads, c.kv_heads, c.group_k, false) != kvq::kPathTc)
         return fail(KVQ_ERR_UNSUPPORTED, "dense-and-sparse keys need 1, 2 or 4 query heads per kv head "
                                          "and key groups of >= 32 tokens");
     const size_t need = static_cast<size_t>(c.batch) * c.kv_heads * static_cast<size_t>(c.capacity) * n_out * 4;
@@ -1186,6 +1199,7 @@ kvq_status kvq_set_key_outliers(kvq_cache *h, int32_t n_out, uint32_t *k_outlier
     if (bytes < need) return fail(KVQ_ERR_INVALID_ARG, "k_outliers needs %zu bytes, got %zu", need, bytes);
     h->k_out = k_outliers;
     h->n_out = n_out;
+    h->path = kvq::kPathTc;   // the integer-MMA kernel's dense-and-sparse instances
     h->ctas_per_sm = kvq::decode_ctas_per_sm(decode_args(h));
     return ok();
 }
@@ -1207,6 +1221,7 @@ kvq_status kvq_plan_decode(const kvq_config *cfg, const int64_t *lengths, int32_
     if (num_sms < 1 || ctas_per_sm < 1) return fail(KVQ_ERR_INVALID_ARG, "num_sms and ctas_per_sm must be >= 1");
     kvq_cache h;
     h.cfg = *cfg;
+    h.path = kvq::decode_path(cfg->q_heads, cfg->kv_heads, cfg->group_k);
     h.num_sms = num_sms;
     h.ctas_per_sm = ctas_per_sm;
     std::vector<int64_t> tiles(static_cast<size_t>(cfg->batch));
@@ -1231,3 +1246,36 @@ kvq_status kvq_plan_decode(const kvq_config *cfg, const int64_t *lengths, int32_
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Bounds-check builds only (libkvq_check.so, include/kvq_check.h): entry points that make
+// the kernels' checks fire, for tests.
+// ---------------------------------------------------------------------------
+#ifdef KVQ_CHECK
+#include "../../include/kvq_check.h"
+
+extern "C" {
+
+kvq_status kvq_debug_set_stall(kvq_cache *h, int32_t polls) {
+    if (!h) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+    if (polls < 0 || polls > 4096) return fail(KVQ_ERR_INVALID_ARG, "polls must be in 0..4096");
+    h->stall_polls = polls;
+    return ok();
+}
+
+kvq_status kvq_debug_gather_rows(kvq_cache *h, const void *src, int64_t src_rows, const int32_t *idx, int32_t n,
+                                 void *dst, void *stream) {
+    if (!h || !src || !idx || !dst || !aligned16(src) || !aligned16(dst) || n < 0 || src_rows < 1)
+        return fail(KVQ_ERR_INVALID_ARG, "bad arguments");
+    const kvq_config &c = h->cfg;
+    unsigned int *status = h->arrivals + static_cast<int64_t>(c.batch) * c.q_heads;
+    const cudaError_t e = kvq::launch_gather_rows(static_cast<const uint16_t *>(src), static_cast<const uint16_t *>(src),
+                                                  src_rows * c.head_dim, src_rows, idx, n, static_cast<uint16_t *>(dst),
+                                                  static_cast<uint16_t *>(dst), static_cast<int64_t>(n) * c.head_dim, 1,
+                                                  c.head_dim, status, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "gather launch");
+    return ok();
+}
+
+}  // extern "C"
+#endif  // KVQ_CHECK

@@ -22,6 +22,16 @@ __device__ __forceinline__ float widen(uint16_t h, bool bf16) {
     return __half2float(__half(r));
 }
 
+// Bounds-check builds (-DKVQ_CHECK: libkvq_check.so).  Kernels that index through a list
+// made on the host or by the caller check every index against its buffer; a bad one raises
+// status bit 3 (value 8) and is replaced by row 0 (reads) or skipped (writes).  The product
+// build compiles these checks out.
+#ifdef KVQ_CHECK
+constexpr bool kCheck = true;
+#else
+constexpr bool kCheck = false;
+#endif
+
 // Record n kernel launches (reported by kvq_kernel_launches()).
 void count_launches(int n);
 
@@ -36,6 +46,7 @@ struct QuantizeArgs {
     int64_t in_tok0;             // first input token
     const int32_t *in_rows;      // or, when non-NULL: input row of token i (device [n_groups * G]);
                                  // in_tok0 is then unused
+    int64_t in_rows_limit;       // rows of each input slice the list may name (bounds-check builds)
     int64_t n_groups;            // key groups to quantize per slice
     int64_t BH;
     int d, G, Gv, bits;
@@ -52,7 +63,8 @@ struct QuantizeArgs {
     int seq0;                    // first sequence of the launch: CTA y = (seq - seq0) * Hkv + head
     const int32_t *seq_len;      // flush: tokens of each sequence after the append; only those
                                  // at a multiple of R flush, to tokens [len - R, len)
-    unsigned int *status;        // bit 2 raised for a page number outside the pool
+    unsigned int *status;        // the cache's status word: bit 2 raised for a page number outside
+                                 // the pool, bit 4 for a scale above the decode kernels' range
     // dense-and-sparse keys (k_out non-NULL): each token's n_out largest-magnitude key
     // entries leave the dense part (set to +0 before quantizing) and are written as words
     // (channel << 16) | element bits to k_out [slice][cap][n_out], largest first
@@ -69,19 +81,25 @@ cudaError_t launch_copy_rows(const uint16_t *src0, const uint16_t *src1, int64_t
                              int d, cudaStream_t s);
 
 // The decode kernel that serves a configuration:
-//  kPathTc    1, 2 or 4 query heads per kv head and key groups of >= 32 tokens: tensor
-//             cores, one CTA per (batch, kv head, split) serving those heads;
+//  kPathMma   contiguous caches with 1, 2 or 4 query heads per kv head and key groups of
+//             >= 32 tokens: decode_mma_kernel (tensor cores, bf16 MMA for keys and values),
+//             one CTA per (batch, kv head, split) serving those heads;
+//  kPathTc    the same geometries for paged caches and dense-and-sparse keys:
+//             decode_tc_kernel (tensor cores, integer MMA for keys);
 //  kPathSplit any other grouping, or 16-token key groups: CUDA cores, one CTA per
 //             (batch, query head, split).
-enum DecodePath : int { kPathSplit = 0, kPathTc = 1 };
+enum DecodePath : int { kPathSplit = 0, kPathTc = 1, kPathMma = 2 };
 
-inline int decode_path(int q_heads, int kv_heads, int group_k) {
+inline int decode_path(int q_heads, int kv_heads, int group_k, bool plain = true) {
     const int g = q_heads / kv_heads;
-    return ((g == 1 || g == 2 || g == 4) && group_k >= 32) ? kPathTc : kPathSplit;
+    if (!((g == 1 || g == 2 || g == 4) && group_k >= 32)) return kPathSplit;
+    return plain ? kPathMma : kPathTc;
 }
 // Split boundaries must fall on multiples of this many tiles (the tensor-core
-// kernel streams items of 4 tiles).
-inline int split_tile_align(int path) { return path == kPathTc ? 4 : 1; }
+// kernels stream items of 4 or 2 tiles).
+inline int split_tile_align(int path) { return path == kPathTc ? 4 : path == kPathMma ? 2 : 1; }
+// Paths whose CTAs serve every query head of one kv head.
+inline bool path_per_kv_head(int path) { return path == kPathTc || path == kPathMma; }
 
 struct DecodeArgs {
     const uint32_t *kc, *vc;
@@ -121,20 +139,26 @@ struct DecodeArgs {
     // [BH][cap][n_out] as written by the quantizer, or NULL
     const uint32_t *k_out;
     int n_out;
+    // bounds-check builds: warp 0 of CTA (0, 0, 0) of the bf16-MMA kernel first waits on a
+    // barrier nothing arrives at, bounded by this many polls, and gives up (0: no wait)
+    int stall_polls;
 };
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 cudaError_t launch_decode_paged(const DecodeArgs &a, cudaStream_t s);
 int decode_ctas_per_sm_paged(const DecodeArgs &a);
 cudaError_t launch_decode_sparse(const DecodeArgs &a, cudaStream_t s);
 int decode_ctas_per_sm_sparse(const DecodeArgs &a);
+cudaError_t launch_decode_mma(const DecodeArgs &a, cudaStream_t s);
+int decode_ctas_per_sm_mma(const DecodeArgs &a);
 // LogQuant retention event: in every (b, h) slice of the full-precision store (rows
 // [0, 3W) of `rows` rows each, ascending positions), rows 2i (i < W) move to row i and rows
 // 2W + j (j < W) to row W + j, for K and V.  One launch.
-cudaError_t launch_lq_compact(uint16_t *kr, uint16_t *vr, int64_t BH, int rows, int W, int d, cudaStream_t s);
+cudaError_t launch_lq_compact(uint16_t *kr, uint16_t *vr, int64_t BH, int rows, int W, int d, unsigned int *status,
+                              cudaStream_t s);
 // dst[bh][i] = src[bh][idx[i]] for i < n, K and V (idx device [n]).  One launch.
 cudaError_t launch_gather_rows(const uint16_t *srck, const uint16_t *srcv, int64_t src_bh_stride,
-                               const int32_t *idx, int n, uint16_t *dstk, uint16_t *dstv,
-                               int64_t dst_bh_stride, int64_t BH, int d, cudaStream_t s);
+                               int64_t src_rows, const int32_t *idx, int n, uint16_t *dstk, uint16_t *dstv,
+                               int64_t dst_bh_stride, int64_t BH, int d, unsigned int *status, cudaStream_t s);
 
 // Paged append: for each sequence slot b with seq_len[b] >= 0, rows t_K[b], t_V[b] ([Hkv][d])
 // become residual row seq_len[b] mod R and seq_len[b] grows by one.  One launch.
@@ -148,6 +172,9 @@ cudaError_t launch_paged_residual(const uint16_t *xk, const uint16_t *xv, int64_
 // t_O [rows][d] from n partials o_all [n][rows][d], m_all / l_all [n][rows] (log2 units).
 cudaError_t launch_merge_partials(const float *o_all, const float *m_all, const float *l_all, int n,
                                   int64_t rows, int d, float *out, cudaStream_t s);
+// The compute capability the library's kernels were compiled for (major * 10 + minor, as
+// the CUDA runtime reports it for a loaded kernel), or -1 when it cannot be read.
+int binary_version();
 // CTAs of the split kernel that fit on one SM for this configuration.
 int decode_ctas_per_sm(const DecodeArgs &a);
 

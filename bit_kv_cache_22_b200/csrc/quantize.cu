@@ -31,6 +31,10 @@ namespace kvq {
 namespace {
 
 constexpr int kQuantThreads = 256;
+// Largest scale the decode kernels serve: their tensor-core operands carry q s and p s times
+// fixed powers of two in bf16 / fp32.  A larger scale still quantizes exactly, but raises
+// status bit 4 (kvq_check_device reports it).
+constexpr float kMaxServedScale = 2147483648.0f;   // 2^31
 
 struct GroupParams {
     float s;
@@ -164,8 +168,8 @@ __device__ void pack_tiles(const uint8_t *codes, int ntiles, uint32_t *dst) {
 // about one memory latency instead of one per load.
 constexpr int kLoadBatch = 8;
 
-__device__ void load_group(const uint16_t *slice, int64_t tok0, const int32_t *rows, uint16_t *dst, int G,
-                           int d) {
+__device__ void load_group(const uint16_t *slice, int64_t tok0, const int32_t *rows, int64_t row_limit,
+                           unsigned int *status, uint16_t *dst, int G, int d) {
     const int vec = d / 8, vshift = d == 64 ? 3 : 4;   // d is 64 or 128
     const int total = G * vec;
     uint4 *d4 = reinterpret_cast<uint4 *>(dst);
@@ -176,7 +180,13 @@ __device__ void load_group(const uint16_t *slice, int64_t tok0, const int32_t *r
             const int i = base + k * blockDim.x;
             if (i < total) {
                 const int t = i >> vshift, c = i & (vec - 1);
-                const int64_t row = rows ? rows[t] : tok0 + t;
+                int64_t row = rows ? rows[t] : tok0 + t;
+                if constexpr (kCheck) {
+                    if (rows && (row < 0 || row >= row_limit)) {
+                        atomicOr(status, 8u);
+                        row = 0;
+                    }
+                }
                 v[k] = __ldcs(reinterpret_cast<const uint4 *>(slice + row * d) + c);   // read once: stream
             }
         }
@@ -229,7 +239,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
 
     // ------------------------------ keys ------------------------------
     const int32_t *rows = a.in_rows ? a.in_rows + grp * G : nullptr;
-    load_group(a.xk + bh * a.in_bh_stride, in_tok, rows, xs, G, d);
+    load_group(a.xk + bh * a.in_bh_stride, in_tok, rows, a.in_rows_limit, a.status, xs, G, d);
     __syncthreads();
     if (a.n_out > 0) {
         // dense-and-sparse keys: per token, the n_out entries of largest magnitude (ties: the
@@ -299,6 +309,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
                 a.kz[(slice * groups_cap + out_tok / G) * d + c] = static_cast<int16_t>(z);
             }
             a.ks[(slice * groups_cap + out_tok / G) * d + c] = s;
+            if (s > kMaxServedScale) atomicOr(a.status, 4u);
             const CodeParams cp = code_params(s, z, a.sym ? mx : fmaxf(fabsf(mn), fabsf(mx)));
             ch_s[c] = s;
             ch_z[c] = z;
@@ -323,7 +334,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
     }
 
     // ------------------------------ values ----------------------------
-    load_group(a.xv + bh * a.in_bh_stride, in_tok, rows, xs, G, d);
+    load_group(a.xv + bh * a.in_bh_stride, in_tok, rows, a.in_rows_limit, a.status, xs, G, d);
     __syncthreads();
     {
         // one token per half-warp (two per warp): the per-token work (segment reductions,
@@ -381,6 +392,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
                 const int64_t mi = (slice * cap + out_tok + t) * ngv + j;
                 a.vs[mi] = s;
                 if (!a.sym) a.vz[mi] = static_cast<int16_t>(z);
+                if (s > kMaxServedScale) atomicOr(a.status, 4u);
             }
             const CodeParams cp = code_params(s, a.sym ? (1 << (bits - 1)) : z,
                                               a.sym ? mx : fmaxf(fabsf(mn), fabsf(mx)));
@@ -424,7 +436,7 @@ __global__ void copy_rows_kernel(const uint16_t *src0, const uint16_t *src1, int
 // row 2W + j -> row W + j (j < W).  Every destination row is at or below its source, so
 // moving the rows in ascending order never overwrites a row before it is read; each
 // wave of rows is read whole before any of it is written.
-__global__ void lq_compact_kernel(uint16_t *kr, uint16_t *vr, int rows, int W, int d) {
+__global__ void lq_compact_kernel(uint16_t *kr, uint16_t *vr, int rows, int W, int d, unsigned int *status) {
     const int64_t bh = blockIdx.x;
     const int vec = d / 8;
     const int per_wave = blockDim.x / vec;                 // destination rows per wave
@@ -433,8 +445,14 @@ __global__ void lq_compact_kernel(uint16_t *kr, uint16_t *vr, int rows, int W, i
     const int r = threadIdx.x / vec, c = threadIdx.x % vec;
     for (int base = 0; base < 2 * W; base += per_wave) {
         const int dst = base + r;
-        const bool on = r < per_wave && dst < 2 * W;
+        bool on = r < per_wave && dst < 2 * W;
         const int src = dst < W ? 2 * dst : W + dst;
+        if constexpr (kCheck) {
+            if (on && (src >= rows || dst >= rows)) {
+                atomicOr(status, 8u);
+                on = false;
+            }
+        }
         uint4 kx = make_uint4(0, 0, 0, 0), vx = kx;
         if (on) {
             kx = k4[src * vec + c];
@@ -450,15 +468,22 @@ __global__ void lq_compact_kernel(uint16_t *kr, uint16_t *vr, int rows, int W, i
 }
 
 __global__ void gather_rows_kernel(const uint16_t *srck, const uint16_t *srcv, int64_t src_bh_stride,
-                                   const int32_t *idx, int n, uint16_t *dstk, uint16_t *dstv,
-                                   int64_t dst_bh_stride, int64_t BH, int d) {
+                                   int64_t src_rows, const int32_t *idx, int n, uint16_t *dstk, uint16_t *dstv,
+                                   int64_t dst_bh_stride, int64_t BH, int d, unsigned int *status) {
     const int64_t vec = d / 8, per = BH * n * vec;
     for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < 2 * per;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const bool isv = i >= per;
         const int64_t k = isv ? i - per : i;
         const int64_t v = k % vec, row = (k / vec) % n, bh = k / (vec * n);
-        const uint4 x = reinterpret_cast<const uint4 *>((isv ? srcv : srck) + bh * src_bh_stride + idx[row] * d)[v];
+        int64_t src = idx[row];
+        if constexpr (kCheck) {
+            if (src < 0 || src >= src_rows) {
+                atomicOr(status, 8u);
+                src = 0;
+            }
+        }
+        const uint4 x = reinterpret_cast<const uint4 *>((isv ? srcv : srck) + bh * src_bh_stride + src * d)[v];
         reinterpret_cast<uint4 *>((isv ? dstv : dstk) + bh * dst_bh_stride + row * d)[v] = x;
     }
 }
@@ -576,21 +601,22 @@ cudaError_t launch_paged_residual(const uint16_t *xk, const uint16_t *xv, int64_
 
 namespace kvq {
 
-cudaError_t launch_lq_compact(uint16_t *kr, uint16_t *vr, int64_t BH, int rows, int W, int d, cudaStream_t s) {
+cudaError_t launch_lq_compact(uint16_t *kr, uint16_t *vr, int64_t BH, int rows, int W, int d, unsigned int *status,
+                              cudaStream_t s) {
     if (BH == 0) return cudaSuccess;
-    lq_compact_kernel<<<static_cast<unsigned>(BH), 256, 0, s>>>(kr, vr, rows, W, d);
+    lq_compact_kernel<<<static_cast<unsigned>(BH), 256, 0, s>>>(kr, vr, rows, W, d, status);
     count_launches(1);
     return cudaGetLastError();
 }
 
 cudaError_t launch_gather_rows(const uint16_t *srck, const uint16_t *srcv, int64_t src_bh_stride,
-                               const int32_t *idx, int n, uint16_t *dstk, uint16_t *dstv,
-                               int64_t dst_bh_stride, int64_t BH, int d, cudaStream_t s) {
+                               int64_t src_rows, const int32_t *idx, int n, uint16_t *dstk, uint16_t *dstv,
+                               int64_t dst_bh_stride, int64_t BH, int d, unsigned int *status, cudaStream_t s) {
     const int64_t total = 2 * BH * n * (d / 8);
     if (total == 0) return cudaSuccess;
     const int64_t blocks = (total + 255) / 256;
     gather_rows_kernel<<<static_cast<unsigned>(blocks < 65536 ? blocks : 65536), 256, 0, s>>>(
-        srck, srcv, src_bh_stride, idx, n, dstk, dstv, dst_bh_stride, BH, d);
+        srck, srcv, src_bh_stride, src_rows, idx, n, dstk, dstv, dst_bh_stride, BH, d, status);
     count_launches(1);
     return cudaGetLastError();
 }

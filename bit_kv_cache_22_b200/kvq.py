@@ -24,7 +24,8 @@ from . import build as _build
 _lock = threading.Lock()
 _lib = None
 
-KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_STATE, KVQ_ERR_CUDA = range(6)
+(KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_STATE, KVQ_ERR_CUDA,
+ KVQ_ERR_DEVICE_CHECK) = range(7)
 KVQ_FP16, KVQ_BF16 = 0, 1
 
 EXPORTED = ("kvq_get_sizes", "kvq_create", "kvq_destroy", "kvq_reset", "kvq_prefill_quantize",
@@ -35,7 +36,8 @@ EXPORTED = ("kvq_get_sizes", "kvq_create", "kvq_destroy", "kvq_reset", "kvq_pref
             "kvq_paged_create", "kvq_paged_destroy", "kvq_paged_prefill", "kvq_paged_append",
             "kvq_paged_decode_attention", "kvq_paged_release", "kvq_paged_seq_len",
             "kvq_paged_decode_splits", "kvq_paged_check_device", "kvq_logquant_get_sizes",
-            "kvq_logquant_create", "kvq_logquant_retained", "kvq_set_key_outliers", "kvq_plan_decode")
+            "kvq_logquant_create", "kvq_logquant_retained", "kvq_set_key_outliers", "kvq_plan_decode",
+            "kvq_binary_arch")
 
 
 class KVQError(RuntimeError):
@@ -56,13 +58,13 @@ class Config(ctypes.Structure):
 class Sizes(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
                 ("k_codes", "k_scales", "k_zeros", "v_codes", "v_scales", "v_zeros",
-                 "k_residual", "v_residual", "workspace")]
+                 "k_residual", "v_residual", "workspace", "state")]
 
 
 class Buffers(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("k_codes", "k_scales", "k_zeros", "v_codes", "v_scales", "v_zeros",
-                 "k_residual", "v_residual")]
+                 "k_residual", "v_residual", "state")]
 
 
 class PagedConfig(ctypes.Structure):
@@ -72,22 +74,28 @@ class PagedConfig(ctypes.Structure):
 class PagedSizes(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
                 ("k_codes", "k_scales", "k_zeros", "v_codes", "v_scales", "v_zeros",
-                 "k_residual", "v_residual", "page_table", "workspace")]
+                 "k_residual", "v_residual", "page_table", "workspace", "state")]
+
+
+def check_build() -> bool:
+    """True when KVQ_LIBRARY=check selects the bounds-check build (libkvq_check.so)."""
+    return os.environ.get("KVQ_LIBRARY", "") == "check"
 
 
 def library_path() -> str:
-    return _build.LIB
+    return _build.LIB_CHECK if check_build() else _build.LIB
 
 
 def load() -> ctypes.CDLL:
-    """Load libkvq.so (building it in-tree first if it is missing or stale)."""
+    """Load libkvq.so -- or, with KVQ_LIBRARY=check, its bounds-check build libkvq_check.so --
+    building it in-tree first if it is missing or stale."""
     global _lib
     with _lock:
         if _lib is not None:
             return _lib
-        path = _build.build()
+        path = _build.build(check=check_build())
         if not os.path.exists(path):
-            raise ImportError(f"libkvq.so not found at {path}")
+            raise ImportError(f"{os.path.basename(path)} not found at {path}")
         lib = ctypes.CDLL(path)
         P, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
         lib.kvq_get_sizes.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(Sizes)]
@@ -117,6 +125,13 @@ def load() -> ctypes.CDLL:
         lib.kvq_last_error.restype = ctypes.c_char_p
         lib.kvq_layout_version.argtypes = []
         lib.kvq_layout_version.restype = i32
+        lib.kvq_binary_arch.argtypes = []
+        lib.kvq_binary_arch.restype = i32
+        if check_build():
+            lib.kvq_debug_set_stall.argtypes = [P, i32]
+            lib.kvq_debug_set_stall.restype = ctypes.c_int
+            lib.kvq_debug_gather_rows.argtypes = [P, P, i64, P, i32, P, P]
+            lib.kvq_debug_gather_rows.restype = ctypes.c_int
         lib.kvq_check_device.argtypes = [P]
         lib.kvq_paged_get_sizes.argtypes = [ctypes.POINTER(PagedConfig), ctypes.POINTER(PagedSizes)]
         lib.kvq_paged_create.argtypes = [ctypes.POINTER(PagedConfig), ctypes.POINTER(Buffers), P,
@@ -234,11 +249,12 @@ class KVQCache:
         self.k_residual = torch.zeros((BH, residual, head_dim), dtype=dtype, device=dev)
         self.v_residual = torch.zeros((BH, residual, head_dim), dtype=dtype, device=dev)
         self.workspace = torch.empty(self.sizes.workspace // 4, dtype=torch.float32, device=dev)
+        self.state_buf = torch.zeros(-(-self.sizes.state // 16) * 4, dtype=torch.int32, device=dev)
         bufs = Buffers(self.k_codes.data_ptr(), self.k_scales.data_ptr(),
                        self.k_zeros.data_ptr() if self.k_zeros is not None else None,
                        self.v_codes.data_ptr(), self.v_scales.data_ptr(),
                        self.v_zeros.data_ptr() if self.v_zeros is not None else None,
-                       self.k_residual.data_ptr(), self.v_residual.data_ptr())
+                       self.k_residual.data_ptr(), self.v_residual.data_ptr(), self.state_buf.data_ptr())
         self._lib = load()
         h = ctypes.c_void_p()
         with torch.cuda.device(dev):
@@ -424,11 +440,12 @@ class PagedKVQCache:
         self.v_residual = torch.zeros((BH, residual, head_dim), dtype=dtype, device=dev)
         self.page_table = torch.full((slots, max_pages), -1, dtype=torch.int32, device=dev)
         self.workspace = torch.empty(self.sizes.workspace // 4, dtype=torch.float32, device=dev)
+        self.state_buf = torch.zeros(-(-self.sizes.state // 16) * 4, dtype=torch.int32, device=dev)
         bufs = Buffers(self.k_codes.data_ptr(), self.k_scales.data_ptr(),
                        self.k_zeros.data_ptr() if self.k_zeros is not None else None,
                        self.v_codes.data_ptr(), self.v_scales.data_ptr(),
                        self.v_zeros.data_ptr() if self.v_zeros is not None else None,
-                       self.k_residual.data_ptr(), self.v_residual.data_ptr())
+                       self.k_residual.data_ptr(), self.v_residual.data_ptr(), self.state_buf.data_ptr())
         h = ctypes.c_void_p()
         with torch.cuda.device(dev):
             _check(self._lib.kvq_paged_create(ctypes.byref(self.cfg), ctypes.byref(bufs),

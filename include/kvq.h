@@ -19,15 +19,16 @@
  * stores u = q + 2^(n-1) and has no zero-point tensors.
  *
  * Conventions for every call:
- *  - Device memory (cache buffers, inputs, outputs, workspace) is owned and
- *    allocated by the caller.  The library's own device memory is one small
- *    array per cache, allocated and zeroed by kvq_create and freed by
- *    kvq_destroy: a 4-byte split-arrival counter per (batch, query head),
- *    through which the last split of a decode merges the others, and a status
- *    word.  Every decode leaves the counters at zero, so decode calls on one
- *    cache must be ordered (one stream, or synchronised).  The host-side
- *    handle keeps the cache geometry and the two counters Tq (quantized
- *    tokens) and r (residual tokens).
+ *  - All device memory (cache buffers, inputs, outputs, workspace and the
+ *    cache's state buffer) is owned and allocated by the caller; the library
+ *    allocates none.  The state buffer (kvq_sizes.state bytes) holds a 4-byte
+ *    split-arrival counter per (batch, query head), through which the last
+ *    split of a decode merges the others, and a status word (a LogQuant cache
+ *    adds its row lists, a paged cache its slots' lengths).  kvq_create
+ *    initialises it; every decode leaves the counters at zero, so decode calls
+ *    on one cache must be ordered (one stream, or synchronised).  The
+ *    host-side handle keeps the cache geometry and the two counters Tq
+ *    (quantized tokens) and r (residual tokens).
  *  - Work is enqueued asynchronously on the caller's CUDA stream (`stream`
  *    is a cudaStream_t, NULL for the legacy default stream).  Host counters
  *    advance when a call is enqueued, so a sequence of calls needs no
@@ -79,7 +80,8 @@ typedef enum {
     KVQ_ERR_UNSUPPORTED = 2,   /* valid but not built (e.g. head_dim 96)        */
     KVQ_ERR_CAPACITY = 3,      /* the call would exceed the token capacity      */
     KVQ_ERR_STATE = 4,         /* call out of order (prefill twice, empty cache) */
-    KVQ_ERR_CUDA = 5           /* a CUDA runtime call or launch failed          */
+    KVQ_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed          */
+    KVQ_ERR_DEVICE_CHECK = 6   /* a check inside a kernel failed (see kvq_check_device) */
 } kvq_status;
 
 typedef enum { KVQ_FP16 = 0, KVQ_BF16 = 1 } kvq_dtype;
@@ -106,6 +108,7 @@ typedef struct {
     size_t v_codes, v_scales, v_zeros;
     size_t k_residual, v_residual;
     size_t workspace;    /* scratch needed by kvq_decode_attention              */
+    size_t state;        /* the cache's state buffer (kvq_buffers.state)        */
 } kvq_sizes;
 
 /* Caller-owned device buffers of one cache (layout above). */
@@ -118,6 +121,8 @@ typedef struct {
     int16_t *v_zeros;    /* NULL when symmetric                                 */
     void *k_residual;
     void *v_residual;
+    void *state;         /* kvq_sizes.state bytes; initialised by the create call,
+                            then the library's for the life of the handle       */
 } kvq_buffers;
 
 typedef struct kvq_cache kvq_cache;   /* opaque host-side handle */
@@ -128,13 +133,14 @@ KVQ_API kvq_status kvq_get_sizes(const kvq_config *cfg, kvq_sizes *out);
 /*
  * Creates a handle over caller-owned buffers (not copied, not freed).  The
  * cache starts empty (Tq = 0, r = 0).  Reads device properties of the current
- * device, and allocates and zeroes (synchronously) the library's small
- * per-cache array there; all later calls must run with that device current.
- * KVQ_ERR_CUDA if that allocation fails.
+ * device and zero-fills the state buffer there (synchronously); allocates no
+ * device memory.  All later calls must run with that device current.
+ * KVQ_ERR_INVALID_ARG for a NULL or misaligned buffer; KVQ_ERR_CUDA if the fill
+ * fails.
  */
 KVQ_API kvq_status kvq_create(const kvq_config *cfg, const kvq_buffers *bufs, kvq_cache **out);
 
-/* Frees the handle and the library's per-cache array.  NULL is ignored. */
+/* Frees the host-side handle (no device memory is the library's).  NULL is ignored. */
 KVQ_API void kvq_destroy(kvq_cache *cache);
 
 /* Empties the cache (Tq = r = 0) without touching device memory. */
@@ -148,6 +154,13 @@ KVQ_API kvq_status kvq_reset(kvq_cache *cache);
  * tokens are copied into the residual.  Only allowed on an empty cache
  * (KVQ_ERR_STATE otherwise); Tq > capacity gives KVQ_ERR_CAPACITY.
  * T = 0 is accepted and does nothing.
+ * Range: the decode kernels serve key and value scales s <= 2^31 (values of
+ * magnitude up to about 2^31 (2^n - 1)) and queries |q| <= 2^30.  A group whose
+ * scale exceeds 2^31 is still quantized exactly, but raises status bit 2 of the
+ * state buffer, which the next kvq_check_device reports as KVQ_ERR_DEVICE_CHECK
+ * (the same holds for the quantization done by kvq_append's flush).  Scales
+ * near 0 need no check: tokens that small only lose contributions below fp32's
+ * normal range.
  */
 KVQ_API kvq_status kvq_prefill_quantize(kvq_cache *cache, const void *X_K, const void *X_V,
                                 int64_t T, void *stream);
@@ -229,8 +242,10 @@ KVQ_API kvq_status kvq_merge_partials(const float *o_parts, const float *m_parts
  *    on the GPU (different streams without ordering) race and give undefined
  *    results.  Nothing in it needs to start at zero; every call writes the
  *    partials it reads.
- *  - The first call on each device looks up the array's device address (with
- *    that device current); make that first call before any stream capture.
+ *  - Every call looks up the array's device address in the calling thread's
+ *    current context, so a context made after a device reset, or another
+ *    context on the device, is served correctly.  The first call in a context
+ *    may load the library's device code: make it before any stream capture.
  */
 KVQ_API kvq_status kvq_decode_attention_noalloc(kvq_cache *cache, const void *t_Q, float *t_O,
                                                 void *stream);
@@ -268,13 +283,18 @@ KVQ_API kvq_status kvq_plan_decode(const kvq_config *cfg, const int64_t *lengths
 KVQ_API int32_t kvq_decode_splits(const kvq_cache *cache);
 
 /*
- * Reads, waiting for the device to finish its queued work, the status word that
- * this cache's decode kernels raise when one of their bounded waits for a copy
- * into shared memory gives up (a condition working hardware never reaches; the
- * wait is bounded so that a fault cannot hang the GPU).  KVQ_OK when the word is
- * clear; KVQ_ERR_CUDA when it was raised -- the outputs of the decodes since the
- * last check are then unreliable, and the word is cleared -- or when the read
- * fails.  The pages have no counterpart.
+ * Reads, waiting for the device to finish its queued work, the status word in
+ * this cache's state buffer, which its kernels raise when a check fails: a
+ * decode kernel's bounded wait for a copy into shared memory gave up (bit 0; a
+ * condition working hardware never reaches -- the wait is bounded so that a
+ * fault cannot hang the GPU), or a quantizer met a scale outside the range the
+ * decode kernels serve (bit 2; see kvq_prefill_quantize), or -- in the
+ * bounds-check build only (include/kvq_check.h) -- a kernel met a list index
+ * outside its buffer (bit 3).  KVQ_OK when the word
+ * is clear; KVQ_ERR_DEVICE_CHECK when it was raised -- the outputs of the calls
+ * since the last check are then unreliable, kvq_last_error() names the checks,
+ * and the word is cleared -- or KVQ_ERR_CUDA when the read fails.  The pages
+ * have no counterpart.
  */
 KVQ_API kvq_status kvq_check_device(kvq_cache *cache);
 
@@ -305,7 +325,7 @@ KVQ_API kvq_status kvq_check_device(kvq_cache *cache);
  *    and raises a status bit that kvq_paged_check_device reports.
  * State: each slot is inactive (after create and release) or active with a length
  * of len tokens (Tq = floor(len / R) R quantized, r = len mod R residual), kept
- * on the host for planning and on the device (library-owned) for the kernels.
+ * on the host for planning and on the device (in the state buffer) for the kernels.
  * ---------------------------------------------------------------------------
  */
 typedef struct {
@@ -321,6 +341,7 @@ typedef struct {
     size_t k_residual, v_residual;       /* [B][Hkv][R][d] e                        */
     size_t page_table;                   /* int32 [B][capacity / P]                 */
     size_t workspace;                    /* scratch of kvq_paged_decode_attention   */
+    size_t state;                        /* kvq_buffers.state of the paged cache    */
 } kvq_paged_sizes;
 
 typedef struct kvq_paged kvq_paged;   /* opaque host-side handle */
@@ -329,10 +350,10 @@ typedef struct kvq_paged kvq_paged;   /* opaque host-side handle */
 KVQ_API kvq_status kvq_paged_get_sizes(const kvq_paged_config *cfg, kvq_paged_sizes *out);
 
 /*
- * Creates a handle over the caller's pool, residual and page-table buffers (not
- * copied, not freed); every slot starts inactive.  Like kvq_create, allocates and
- * initialises (synchronously) a small library-owned device array: split-arrival
- * counters, the status word and the slots' lengths.
+ * Creates a handle over the caller's pool, residual, state and page-table
+ * buffers (not copied, not freed); every slot starts inactive.  Like kvq_create,
+ * initialises the state buffer (synchronously): split-arrival counters, the
+ * status word and the slots' lengths.  Allocates no device memory.
  */
 KVQ_API kvq_status kvq_paged_create(const kvq_paged_config *cfg, const kvq_buffers *bufs,
                                     const int32_t *page_table, kvq_paged **out);
@@ -382,9 +403,9 @@ KVQ_API kvq_status kvq_paged_seq_len(const kvq_paged *cache, int32_t seq, int64_
 KVQ_API int32_t kvq_paged_decode_splits(const kvq_paged *cache);
 
 /*
- * As kvq_check_device, for a paged cache.  Also reports (KVQ_ERR_INVALID_ARG) a
- * page-table entry outside the pool met by a kernel since the last check; the
- * outputs since then are unreliable and the word is cleared.
+ * As kvq_check_device, for a paged cache.  Also reports (KVQ_ERR_DEVICE_CHECK,
+ * bit 1) a page-table entry outside the pool met by a kernel since the last
+ * check; the outputs since then are unreliable and the word is cleared.
  */
 KVQ_API kvq_status kvq_paged_check_device(kvq_paged *cache);
 
@@ -408,8 +429,8 @@ KVQ_API kvq_status kvq_paged_check_device(kvq_paged *cache);
  * token position.  The cache's capacity is rounded up to a multiple of 3W for
  * the layout (kvq_logquant_get_sizes reports the sizes).  Its prefill uploads
  * row lists from host memory with one copy (so it cannot be captured in a CUDA
- * graph); append and decode can.  The library also owns a device array of
- * (capacity + 4W) int32 row indices per LogQuant cache.
+ * graph); append and decode can.  Its state buffer also holds (capacity + 4W)
+ * int32 row indices (kvq_logquant_get_sizes counts them in `state`).
  * ---------------------------------------------------------------------------
  */
 
@@ -461,6 +482,14 @@ KVQ_API const char *kvq_last_error(void);
 
 /* Version of the storage format described above (currently 2). */
 KVQ_API int32_t kvq_layout_version(void);
+
+/*
+ * The GPU architecture the library's kernels were compiled for, as the CUDA
+ * runtime reports it for a loaded kernel (major * 10 + minor: 100 for sm_100a),
+ * or -1 when it cannot be read (no device).  Needs the device the caller uses to
+ * be current.  The pages have no counterpart.
+ */
+KVQ_API int32_t kvq_binary_arch(void);
 
 #ifdef __cplusplus
 }

@@ -37,13 +37,20 @@ def test_library_exports_every_declared_symbol():
     assert exported == set(declared_symbols())
 
 
-def test_library_is_sm100a_only():
-    out = subprocess.run(["/usr/local/cuda/bin/cuobjdump", "--list-elf", kvq.library_path()],
-                         capture_output=True, text=True)
-    if out.returncode != 0:
-        pytest.skip("cuobjdump unavailable")
-    arches = set(re.findall(r"sm_(\d+a?)", out.stdout))
-    assert arches == {"100a"}
+def test_library_is_built_for_sm100a_only():
+    from bit_kv_cache_22_b200 import build
+    flags = build.NVCC_FLAGS
+    targets = [flags[i + 1] for i, f in enumerate(flags) if f == "-gencode"]
+    assert targets == ["arch=compute_100a,code=sm_100a"]
+
+
+@pytest.mark.gpu
+def test_loaded_kernels_are_sm100():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    torch.cuda.init()
+    assert kvq.load().kvq_binary_arch() == 100
 
 
 def _cfg(**kw):
@@ -61,8 +68,31 @@ def test_sizes_match_layout():
     assert s.v_scales == BH * cap * (d // 32) * 4 and s.v_zeros == BH * cap * (d // 32) * 2
     assert s.k_residual == s.v_residual == BH * 128 * d * 2
     assert s.workspace > 0
+    # state: a split-arrival counter per (batch, query head) and the status word, 16-byte padded
+    assert s.state == -(-(1 * 4 + 1) * 4 // 16) * 16
     sym = kvq.get_sizes(_cfg(symmetric=1, bits=4))
     assert sym.k_zeros == 0 and sym.v_zeros == 0
+
+
+def test_logquant_state_holds_the_row_lists():
+    lib = kvq.load()
+    cfg, W = _cfg(capacity=1536), 128
+    s = kvq.Sizes()
+    assert lib.kvq_logquant_get_sizes(ctypes.byref(cfg), W, ctypes.byref(s)) == kvq.KVQ_OK
+    cap = -(-1536 // (3 * W)) * 3 * W
+    assert s.state == 32 + (W + cap + 3 * W) * 4          # counters (5 words, padded) + lists
+
+
+def test_create_needs_a_state_buffer():
+    lib = kvq.load()
+    cfg = _cfg()
+    fake = 1 << 20                                 # aligned, never dereferenced: rejected first
+    bufs = kvq.Buffers(*([fake] * 8), None)
+    h = ctypes.c_void_p()
+    assert lib.kvq_create(ctypes.byref(cfg), ctypes.byref(bufs), ctypes.byref(h)) == kvq.KVQ_ERR_INVALID_ARG
+    assert b"state" in lib.kvq_last_error() and not h.value
+    bufs = kvq.Buffers(*([fake] * 8), fake + 8)    # misaligned state
+    assert lib.kvq_create(ctypes.byref(cfg), ctypes.byref(bufs), ctypes.byref(h)) == kvq.KVQ_ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("bad,status", [
@@ -120,6 +150,7 @@ def test_paged_sizes_match_layout():
     assert s.k_residual == s.v_residual == 2 * 128 * d * 2
     assert s.page_table == 1 * (1024 // 128) * 4
     assert s.workspace == kvq.get_sizes(_cfg()).workspace
+    assert s.state == kvq.get_sizes(_cfg()).state + 16      # + the slots' lengths, padded
 
 
 @pytest.mark.parametrize("bad", [dict(page_tokens=96), dict(page_tokens=64),   # not a multiple of R = 128
