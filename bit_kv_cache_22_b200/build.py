@@ -14,6 +14,9 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libkvq.so")
+# the bounds-check build (-DKVQ_CHECK): kernels check list indices, tests can make bounded waits
+# give up (include/kvq_check.h)
+LIB_CHECK = os.path.join(PKG, "libkvq_check.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 NVCC_FLAGS = [
@@ -28,25 +31,28 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + [os.path.join(ROOT, "include", "kvq.h")]
-    t = os.path.getmtime(LIB)
+    deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(ROOT, "include", "*.h"))
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every translation unit (in parallel) and link libkvq.so."""
-    if not force and not _stale():
-        return LIB
-    objdir = os.path.join(PKG, "_build")
+def build(force: bool = False, verbose: bool = False, check: bool = False) -> str:
+    """Compile every translation unit (in parallel) and link libkvq.so (libkvq_check.so with
+    check=True: the bounds-check build)."""
+    lib = LIB_CHECK if check else LIB
+    if not force and not _stale(lib):
+        return lib
+    flags = NVCC_FLAGS + (["-DKVQ_CHECK"] if check else [])
+    objdir = os.path.join(PKG, "_build_check" if check else "_build")
     os.makedirs(objdir, exist_ok=True)
     tag = os.getpid()
     procs = []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + f".{tag}.o")
-        cmd = [NVCC, *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-c", src, "-o", obj]
+        cmd = [NVCC, *flags, "-I", os.path.join(ROOT, "include"), "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
         procs.append((subprocess.Popen(cmd), obj))
@@ -55,15 +61,15 @@ def build(force: bool = False, verbose: bool = False) -> str:
     try:
         if failed:
             raise subprocess.CalledProcessError(1, failed[0])
-        tmp = LIB + f".tmp{tag}"
-        subprocess.run([NVCC, *NVCC_FLAGS, "-shared", "-o", tmp, *objs], check=True)
-        os.replace(tmp, LIB)
+        tmp = lib + f".tmp{tag}"
+        subprocess.run([NVCC, *flags, "-shared", "-o", tmp, *objs], check=True)
+        os.replace(tmp, lib)
     finally:
         for o in objs:
             if os.path.exists(o):
                 os.remove(o)
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True))
+    print(build(force="--force" in sys.argv, verbose=True, check="--check" in sys.argv))
