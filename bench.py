@@ -96,22 +96,39 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def decode_kernel_name(w) -> str:
+def decode_kernel_name(w, paged: bool = False, key_outliers: int = 0) -> str:
     """The decode kernel the library launches for this geometry."""
-    return "decode_tc_kernel" if w.Hq // w.Hkv in (1, 2, 4) and w.G >= 32 else "decode_split_kernel"
+    if w.Hq // w.Hkv not in (1, 2, 4) or w.G < 32:
+        return "decode_split_kernel"
+    return "decode_tc_kernel" if paged or key_outliers else "decode_mma_kernel"
 
 
-def ncu_traffic(w):
+# the sources a decode kernel's code comes from (a profile names their hash)
+KERNEL_SOURCES = {
+    "decode_mma_kernel": ("decode_mma.cuh", "decode_kernels.cuh"),
+    "decode_tc_kernel": ("decode_kernels.cuh",),
+    "decode_split_kernel": ("decode_kernels.cuh",),
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "bit_kv_cache_22_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(w, kernel=None):
     """Per-launch DRAM bytes of the decode kernel from the committed ncu summary,
     if it was taken on the current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", f"{decode_kernel_name(w)}_{w.name}.md")
-    src = os.path.join(ROOT, "bit_kv_cache_22_b200", "csrc", "decode_kernels.cuh")
+    kernel = kernel or decode_kernel_name(w)
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{w.name}.md")
     try:
         text = open(path).read()
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        m_sha = re.search(r"decode_kernels\.cuh sha256\[:16\]:\s*([0-9a-f]{16})", text)
+        m_sha = re.search(r"kernel source sha256\[:16\]:\s*([0-9a-f]{16})", text)
         m_b = re.search(r"dram bytes per launch:\s*([0-9]+)", text)
-        if m_sha and m_b and m_sha.group(1) == sha:
+        if m_sha and m_b and m_sha.group(1) == kernel_source_hash(kernel):
             return int(m_b.group(1))
     except OSError:
         pass
@@ -399,7 +416,7 @@ def measure_workload(w, args, dev, local, world, headline: bool):
         "clocks": clk.summary(),
         "e2e": e2e,
         "roofline": {
-            "kernel": f"append + decode_attention ({decode_kernel_name(w)}: one launch without a flush, "
+            "kernel": f"append + decode_attention ({decode_kernel_name(w, key_outliers=args.key_outliers)}: one launch without a flush, "
                       "splits merged in-kernel), per call",
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
@@ -409,7 +426,7 @@ def measure_workload(w, args, dev, local, world, headline: bool):
             "l2": "cold: a read of 2 x L2 before every timed call (its time subtracted)" if cold else
                   "inputs larger than L2 (calls back to back)",
             "timing_ms": {"decode_graph": dec_ms, "side_graph": side_ms, "replays": args.steps},
-            "traffic": ncu_traffic(w),
+            "traffic": ncu_traffic(w, decode_kernel_name(w, key_outliers=args.key_outliers)),
         },
         "config": {
             "workload": w.name, "batch_per_gpu": w.B, "global_batch": w.B * world,
@@ -663,7 +680,7 @@ def run_logquant(args):
               "key_outliers_per_token": args.key_outliers, "full_precision_rows_at_end": r,
               "splits": cache.splits()}
     line = _decode_only_line(args, w, world, ms, total_ms, tokens, nbytes, launches, clk, config,
-                             f"decode_attention ({decode_kernel_name(w)}) over a LogQuant cache, per call")
+                             f"decode_attention ({decode_kernel_name(w, key_outliers=args.key_outliers)}) over a LogQuant cache, per call")
     _finish(world, rank, line)
 
 
@@ -712,7 +729,7 @@ def run_paged(args):
               "page_tokens": P, "decode_steps": w.steps, "bits": w.bits, "group_k": w.G, "group_v": w.Gv,
               "residual": w.R, "splits": cache.splits()}
     line = _decode_only_line(args, w, world, ms, total_ms, tokens, nbytes, launches, clk, config,
-                             f"paged decode_attention ({decode_kernel_name(w)}, paged instance), per call")
+                             f"paged decode_attention ({decode_kernel_name(w, paged=True)}, paged instance), per call")
     _finish(world, rank, line)
 
 

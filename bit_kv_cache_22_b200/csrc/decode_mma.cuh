@@ -44,6 +44,7 @@ namespace {
 constexpr int kMmaItemTiles = 2;    // tiles per item (stage)
 constexpr int kKeyScaleLog2 = 64;   // the key MMA's B operand is q' s 2^64
 constexpr int kValScaleLog2 = 80;   // the value MMA's B operand is p s 2^80
+constexpr float kLazyRescale = 8.0f; // log2 units the logits may pass the running maximum by
 
 template <int N, int D, int GV, int HG>
 struct MmaLayout {
@@ -84,6 +85,32 @@ struct MmaLayout {
 
 template <int N, int D, int GV, int HG>
 __host__ __device__ constexpr int mma_smem() { return kDecodeWarps * MmaLayout<N, D, GV, HG>::kWarpBytes; }
+
+// The barrier arm and the bulk copy on 32-bit shared addresses.
+__device__ __forceinline__ void mbar_expect_tx_u32(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_g2s_u32(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_u32(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "n"(kPollSuspendNs)
+        : "memory");
+    return ok != 0;
+}
+// Every lane of the warp waits for the phase of `parity` of barrier `bar`: one poll when the
+// data is there, else bounded polling (false when it gave up).
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
+    if (__all_sync(0xffffffffu, mbar_try_wait_u32(bar, parity))) return true;
+    bool ok = false;
+    for (uint32_t i = 0; i < kSpinLimit && !ok; ++i) ok = mbar_try_wait_u32(bar, parity);
+    return __all_sync(0xffffffffu, ok);
+}
 
 // n consecutive 32-bit values from / to shared memory with the widest vector accesses
 template <int n, typename T>
@@ -192,7 +219,10 @@ __global__ void __launch_bounds__(kDecodeThreads, D / GV >= 8 ? 3 : 4) decode_mm
     const int hk = blockIdx.x, b = blockIdx.y, sigma = blockIdx.z;
     const int64_t bh = static_cast<int64_t>(b) * a.Hkv + hk;
     const int64_t bq0 = static_cast<int64_t>(b) * a.Hq + static_cast<int64_t>(hk) * HG;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // the warp index through a shuffle from lane 0: provably warp-uniform, so everything derived
+    // from it (the warp's tile range, the copy sources) can live in uniform registers
+    const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x >> 5), 0);
+    const int lane = threadIdx.x & 31;
     const int g8 = lane >> 2, t4 = lane & 3;
     unsigned char *wmem = stage_mem + static_cast<size_t>(warp) * L::kWarpBytes;
     const int zsym = 1 << (N - 1);
@@ -277,46 +307,39 @@ __global__ void __launch_bounds__(kDecodeThreads, D / GV >= 8 ? 3 : 4) decode_mm
     }
     __syncwarp();
 
-    // Producer: item k of the warp into stage k % kSt with one bulk copy per array, lanes
-    // 0..5 issuing one each from a descriptor fixed for the warp: the array, its bytes per
-    // tile (per key group for the key meta), where it lands in the stage and its size.
-    // Lane 0 also arms the barrier with the item's byte count.
-    const unsigned char *c_src = nullptr;
-    int64_t c_step = 0;
-    int c_shift = 0;
-    uint32_t c_off = 0, c_bytes = 0;
-    bool c_keymeta = false;
-    {
-        constexpr uint32_t vsb = static_cast<uint32_t>(16 * NGV * 4);   // value scales of one tile
-        switch (lane) {
-            case 0: c_src = reinterpret_cast<const unsigned char *>(a.kc); c_step = TW * 4; c_off = 0;
-                    c_bytes = L::kVc; break;
-            case 1: c_src = reinterpret_cast<const unsigned char *>(a.vc); c_step = TW * 4; c_off = L::kVc;
-                    c_bytes = L::kVc; break;
-            case 2: c_src = reinterpret_cast<const unsigned char *>(a.vs); c_step = vsb; c_off = L::kVs;
-                    c_bytes = kMmaItemTiles * vsb; break;
-            case 3: c_src = reinterpret_cast<const unsigned char *>(a.vz); c_step = vsb / 2; c_off = L::kVz;
-                    c_bytes = a.sym ? 0u : kMmaItemTiles * vsb / 2; break;
-            case 4: c_src = reinterpret_cast<const unsigned char *>(a.ks); c_step = D * 4; c_shift = a.gshift;
-                    c_off = L::kKs; c_bytes = D * 4; c_keymeta = true; break;
-            case 5: c_src = reinterpret_cast<const unsigned char *>(a.kz); c_step = D * 2; c_shift = a.gshift;
-                    c_off = L::kKz; c_bytes = a.sym ? 0u : D * 2; c_keymeta = true; break;
-            default: break;
-        }
-    }
+    // Producer: item k of the warp into stage k % kSt, one bulk copy per array (key codes,
+    // value codes, value scales, value zeros and, when the item opens a key group, the group's
+    // key scales and zeros), all issued by lane 0 after it arms the barrier with the item's
+    // byte count.  Every source, destination and size is warp-uniform, so the copies take
+    // their operands from uniform registers and lane 0 issues them back to back.
+    const uint32_t s_stage0 = smem_u32(wmem), s_bar0 = smem_u32(bars);
+    constexpr int64_t kVsb = 16 * NGV * 4;   // value scales of one tile
+    constexpr int64_t kItemCodes = kMmaItemTiles * TW * 4, kItemVs = kMmaItemTiles * kVsb;
+    const unsigned char *kc0 = reinterpret_cast<const unsigned char *>(a.kc) + tile0 * TW * 4;
+    const unsigned char *vc0 = reinterpret_cast<const unsigned char *>(a.vc) + tile0 * TW * 4;
+    const unsigned char *vs0 = reinterpret_cast<const unsigned char *>(a.vs) + tile0 * kVsb;
+    const unsigned char *vz0 = reinterpret_cast<const unsigned char *>(a.vz) + tile0 * (kVsb / 2);
     const uint32_t tx_item = 2u * L::kVc + kMmaItemTiles * 16 * NGV * (a.sym ? 4u : 6u);
     const uint32_t tx_keymeta = static_cast<uint32_t>(D * (a.sym ? 4 : 6));
     auto issue = [&](int k) {
         if (k >= nitems) return;
-        const int64_t gt = tile0 + kMmaItemTiles * k;
         const bool open = k == 0 || ((wb + kMmaItemTiles * k) & gmask) == 0;
-        unsigned char *st = wmem + (k % kSt) * L::kStage;
-        uint64_t *bar = bars + k % kSt;
-        const uint32_t bytes = (c_keymeta && !open) ? 0u : c_bytes;
-        if (bytes) {
-            fence_proxy_async();   // this stage's earlier reads come before the copies below
-            if (lane == 0) mbar_expect_tx(bar, tx_item + (open ? tx_keymeta : 0u));
-            bulk_g2s(st + c_off, c_src + (gt >> c_shift) * c_step, bytes, bar);
+        const uint32_t slot = static_cast<uint32_t>(k % kSt);
+        const uint32_t bar = s_bar0 + 8u * slot, dst = s_stage0 + slot * L::kStage;
+        fence_proxy_async();   // this stage's earlier reads come before the copies below
+        if (lane == 0) {
+            mbar_expect_tx_u32(bar, tx_item + (open ? tx_keymeta : 0u));
+            bulk_g2s_u32(dst, kc0 + k * kItemCodes, L::kVc, bar);
+            bulk_g2s_u32(dst + L::kVc, vc0 + k * kItemCodes, L::kVc, bar);
+            bulk_g2s_u32(dst + L::kVs, vs0 + k * kItemVs, kItemVs, bar);
+            if (!a.sym) bulk_g2s_u32(dst + L::kVz, vz0 + k * (kItemVs / 2), kItemVs / 2, bar);
+            if (open) {
+                const int64_t g = (tile0 + kMmaItemTiles * k) >> a.gshift;   // the key group
+                bulk_g2s_u32(dst + L::kKs, reinterpret_cast<const unsigned char *>(a.ks) + g * (D * 4), D * 4, bar);
+                if (!a.sym)
+                    bulk_g2s_u32(dst + L::kKz, reinterpret_cast<const unsigned char *>(a.kz) + g * (D * 2), D * 2,
+                                 bar);
+            }
         }
     };
 
@@ -367,8 +390,8 @@ __global__ void __launch_bounds__(kDecodeThreads, D / GV >= 8 ? 3 : 4) decode_mm
                                            __uint_as_float(__float_as_uint(x01.y) & 0xffff0000u));
             const float2 t23 = make_float2(__uint_as_float(__float_as_uint(x23.x) & 0xffff0000u),
                                            __uint_as_float(__float_as_uint(x23.y) & 0xffff0000u));
-            const float2 r01 = add2(x01, make_float2(-t01.x, -t01.y));
-            const float2 r23 = add2(x23, make_float2(-t23.x, -t23.y));
+            const float2 r01 = sub2(x01, t01);
+            const float2 r23 = sub2(x23, t23);
             uint32_t *row = kbs + (hp0 + i) * 4 * L::RS + (quad & 3) * L::RS + 2 * (quad >> 2);
             *reinterpret_cast<uint2 *>(row) = make_uint2(bf16_trunc2(x01.x, x23.x), bf16_trunc2(x01.y, x23.y));
             *reinterpret_cast<uint2 *>(row + L::PS) = make_uint2(f2bf2(r01.x, r23.x), f2bf2(r01.y, r23.y));
@@ -416,7 +439,7 @@ __global__ void __launch_bounds__(kDecodeThreads, D / GV >= 8 ? 3 : 4) decode_mm
     int k = 0;
     for (; k < nitems; ++k) {
         issue(k + kSt - 1);
-        const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bars + k % kSt, (k / kSt) & 1));
+        const bool ok = warp_wait(s_bar0 + 8u * static_cast<uint32_t>(k % kSt), static_cast<uint32_t>(k / kSt) & 1u);
         if (!ok) {
             if (lane == 0) atomicOr(a.status, 1u);
             break;
@@ -454,7 +477,9 @@ __global__ void __launch_bounds__(kDecodeThreads, D / GV >= 8 ? 3 : 4) decode_mm
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-            if (__any_sync(0xffffffffu, mx > m_own)) {
+            // lazily: only when the item's maximum passes the running one by more than
+            // kLazyRescale (p may reach 2^kLazyRescale meanwhile), so rescales stay rare
+            if (__any_sync(0xffffffffu, mx > m_own + kLazyRescale)) {
                 const float mn = fmaxf(m_own, mx);
                 const float alpha = fast_exp2(m_own - mn);
                 m_own = mn;
@@ -486,8 +511,10 @@ __global__ void __launch_bounds__(kDecodeThreads, D / GV >= 8 ? 3 : 4) decode_mm
             int16_t zv[NGV];
             load_meta<NGV>(reinterpret_cast<const float *>(st + L::kVs) + lane * NGV,
                            reinterpret_cast<const int16_t *>(st + L::kVz) + lane * NGV, a.sym, zsym, sv, zv);
+            float uz[NGV];
 #pragma unroll
-            for (int v = 0; v < NGV; ++v) uv[lane * NGV + v] = sv[v] * static_cast<float>(zv[v]);
+            for (int v = 0; v < NGV; ++v) uz[v] = sv[v] * static_cast<float>(zv[v]);
+            store_vec<NGV>(uv + lane * NGV, uz);
         }
         __syncwarp();
 
@@ -504,12 +531,35 @@ __global__ void __launch_bounds__(kDecodeThreads, D / GV >= 8 ? 3 : 4) decode_mm
             load_vec<NGV>(uv + r0 * NGV, u0);
             load_vec<NGV>(uv + r1 * NGV, u1);
             uint32_t hi[NGV], lo[NGV];
+            if constexpr (NGV % 2 == 0) {
+                // packed over value-group pairs: (ps0[v], ps0[v + 1]), (ps1[v], ps1[v + 1])
 #pragma unroll
-            for (int v = 0; v < NGV; ++v) {
-                const float ps0 = pp.x * s0[v], ps1 = pp.y * s1[v];
-                zsum[v] = fmaf(pp.x, u0[v], fmaf(pp.y, u1[v], zsum[v]));
-                hi[v] = bf16_trunc2(ps0, ps1);
-                lo[v] = bf16_rem2(ps0, ps1);
+                for (int v = 0; v < NGV; v += 2) {
+                    const float2 a0 = mul2(make_float2(pp.x, pp.x), make_float2(s0[v], s0[v + 1]));
+                    const float2 a1 = mul2(make_float2(pp.y, pp.y), make_float2(s1[v], s1[v + 1]));
+                    float2 zz = fma2(make_float2(pp.x, pp.x), make_float2(u0[v], u0[v + 1]),
+                                     make_float2(zsum[v], zsum[v + 1]));
+                    zz = fma2(make_float2(pp.y, pp.y), make_float2(u1[v], u1[v + 1]), zz);
+                    zsum[v] = zz.x;
+                    zsum[v + 1] = zz.y;
+                    const float2 t0 = make_float2(__uint_as_float(__float_as_uint(a0.x) & 0xffff0000u),
+                                                  __uint_as_float(__float_as_uint(a0.y) & 0xffff0000u));
+                    const float2 t1 = make_float2(__uint_as_float(__float_as_uint(a1.x) & 0xffff0000u),
+                                                  __uint_as_float(__float_as_uint(a1.y) & 0xffff0000u));
+                    const float2 r0 = sub2(a0, t0), r1 = sub2(a1, t1);
+                    hi[v] = bf16_trunc2(a0.x, a1.x);
+                    hi[v + 1] = bf16_trunc2(a0.y, a1.y);
+                    lo[v] = f2bf2(r0.x, r1.x);
+                    lo[v + 1] = f2bf2(r0.y, r1.y);
+                }
+            } else {
+#pragma unroll
+                for (int v = 0; v < NGV; ++v) {
+                    const float ps0 = pp.x * s0[v], ps1 = pp.y * s1[v];
+                    zsum[v] = fmaf(pp.x, u0[v], fmaf(pp.y, u1[v], zsum[v]));
+                    hi[v] = bf16_trunc2(ps0, ps1);
+                    lo[v] = bf16_rem2(ps0, ps1);
+                }
             }
             uint32_t B0[NGV], B1[NGV];
             if constexpr (NGV >= 4) {
