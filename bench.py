@@ -58,7 +58,14 @@ def _args():
                    help="measure LogQuant retention with this window W on the workload instead")
     p.add_argument("--key-outliers", type=int, default=0,
                    help="dense-and-sparse keys: keep this many outliers per token (1 or 2)")
+    p.add_argument("--decode-kernel", default="auto", choices=list(DECODE_KERNELS),
+                   help="the decode kernel (kvq_set_decode_kernel): the library's choice or one forced")
     return p.parse_args()
+
+
+# --decode-kernel: the kvq_set_decode_kernel value and the kernel it launches
+DECODE_KERNELS = {"auto": (0, None), "cuda-cores": (1, "decode_split_kernel"),
+                  "int8-mma": (2, "decode_tc_kernel"), "bf16-mma": (3, "decode_mma_kernel")}
 
 
 # ---------------------------------------------------------------------------
@@ -96,8 +103,10 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def decode_kernel_name(w, paged: bool = False, key_outliers: int = 0) -> str:
+def decode_kernel_name(w, paged: bool = False, key_outliers: int = 0, forced: str = "auto") -> str:
     """The decode kernel the library launches for this geometry."""
+    if DECODE_KERNELS[forced][1]:
+        return DECODE_KERNELS[forced][1]
     if w.Hq // w.Hkv not in (1, 2, 4) or w.G < 32:
         return "decode_split_kernel"
     return "decode_tc_kernel" if paged or key_outliers else "decode_mma_kernel"
@@ -272,6 +281,7 @@ def measure_workload(w, args, dev, local, world, headline: bool):
     tK, tV, tQ = to_t(tK_h).to(dev), to_t(tV_h).to(dev), to_t(tQ_h).to(dev)
     cache = kvq.KVQCache(w.B, w.Hq, w.Hkv, w.d, w.G, w.Gv, w.R, w.bits, w.symmetric, dt,
                          w.capacity, dev, key_outliers=args.key_outliers)
+    cache.set_decode_kernel(DECODE_KERNELS[args.decode_kernel][0])
     out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -402,6 +412,7 @@ def measure_workload(w, args, dev, local, world, headline: bool):
         del g2
 
     peak, peak_kind = peaks()
+    kname = decode_kernel_name(w, key_outliers=args.key_outliers, forced=args.decode_kernel)
     per_call_ms = decode_ms / (args.steps * w.steps)
     bytes_per_call = sum(call_bytes) / w.steps
     achieved = bytes_per_call / (per_call_ms / 1e3) / 1e9
@@ -416,7 +427,7 @@ def measure_workload(w, args, dev, local, world, headline: bool):
         "clocks": clk.summary(),
         "e2e": e2e,
         "roofline": {
-            "kernel": f"append + decode_attention ({decode_kernel_name(w, key_outliers=args.key_outliers)}: one launch without a flush, "
+            "kernel": f"append + decode_attention ({kname}: one launch without a flush, "
                       "splits merged in-kernel), per call",
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
@@ -426,7 +437,7 @@ def measure_workload(w, args, dev, local, world, headline: bool):
             "l2": "cold: a read of 2 x L2 before every timed call (its time subtracted)" if cold else
                   "inputs larger than L2 (calls back to back)",
             "timing_ms": {"decode_graph": dec_ms, "side_graph": side_ms, "replays": args.steps},
-            "traffic": ncu_traffic(w, decode_kernel_name(w, key_outliers=args.key_outliers)),
+            "traffic": ncu_traffic(w, kname),
         },
         "config": {
             "workload": w.name, "batch_per_gpu": w.B, "global_batch": w.B * world,
@@ -434,6 +445,7 @@ def measure_workload(w, args, dev, local, world, headline: bool):
             "decode_steps": w.steps, "bits": w.bits, "group_k": w.G, "group_v": w.Gv,
             "residual": w.R, "symmetric": w.symmetric, "key_outliers_per_token": args.key_outliers,
             "elem": "fp16" if w.dtype == wl.FP16 else "bf16",
+            "decode_kernel": kname,
         },
     }
     del cache, XK, XV, tK, tV, tQ, g_ep, scrub
@@ -471,6 +483,7 @@ def run_kvq(args):
         tK, tV, tQ = (to_t(x) for x in wl.decode_bits(w))
         cache = kvq.KVQCache(w.B, w.Hq, w.Hkv, w.d, w.G, w.Gv, w.R, w.bits, w.symmetric, dt,
                              w.capacity, dev, key_outliers=args.key_outliers)
+        cache.set_decode_kernel(DECODE_KERNELS[args.decode_kernel][0])
         out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
         cache.prefill_quantize(XK, XV)
         for s in range(min(w.steps, 64)):      # ends mid-episode (r = 64 residual rows at most)
@@ -660,6 +673,8 @@ def run_logquant(args):
     cap = -(-(w.T + w.steps) // W) * W
     cache = kvq.KVQCache(w.B, w.Hq, w.Hkv, w.d, w.G, w.Gv, w.R, w.bits, w.symmetric, dt, cap, dev,
                          window=W, key_outliers=args.key_outliers)
+    cache.set_decode_kernel(DECODE_KERNELS[args.decode_kernel][0])
+    kname = decode_kernel_name(w, key_outliers=args.key_outliers, forced=args.decode_kernel)
     XK, XV = wl.prefill_bits(w)
     cache.prefill_quantize(to_t(XK), to_t(XV))
     del XK, XV
@@ -680,7 +695,7 @@ def run_logquant(args):
               "key_outliers_per_token": args.key_outliers, "full_precision_rows_at_end": r,
               "splits": cache.splits()}
     line = _decode_only_line(args, w, world, ms, total_ms, tokens, nbytes, launches, clk, config,
-                             f"decode_attention ({decode_kernel_name(w, key_outliers=args.key_outliers)}) over a LogQuant cache, per call")
+                             f"decode_attention ({kname}) over a LogQuant cache, per call")
     _finish(world, rank, line)
 
 

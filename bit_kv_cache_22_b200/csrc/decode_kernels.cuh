@@ -267,9 +267,12 @@ struct PageWindow {
 };
 
 // Floats of shared scratch finish_cta needs after the per-warp outputs (wts): the split
-// weights HG (S + 1), S <= 80, padded to 4, and the [P][C] float4 sums of the merge.
+// weights HG (S + 1), S <= kMaxDecodeSplits, padded to 4, and the [P][C] float4 sums of
+// the merge.
 template <int HG, int D>
-__host__ __device__ constexpr int finish_scratch_floats() { return (HG * 81 + 3) / 4 * 4 + 4 * kDecodeThreads; }
+__host__ __device__ constexpr int finish_scratch_floats() {
+    return (HG * (kMaxDecodeSplits + 1) + 3) / 4 * 4 + 4 * kDecodeThreads;
+}
 
 // End of every decode CTA.  o_w [warp][HG][D] and ml_w [warp][HG] = (m, l) are
 // the per-warp partials of the CTA's HG query heads (unnormalised, log2

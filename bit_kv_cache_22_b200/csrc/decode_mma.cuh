@@ -46,7 +46,7 @@ constexpr int kKeyScaleLog2 = 64;   // the key MMA's B operand is q' s 2^64
 constexpr int kValScaleLog2 = 80;   // the value MMA's B operand is p s 2^80
 constexpr float kLazyRescale = 8.0f; // log2 units the logits may pass the running maximum by
 
-template <int N, int D, int GV, int HG>
+template <int N, int D, int GV, int HG, bool RR>
 struct MmaLayout {
     static constexpr int W = D * N / 64;            // code words per lane per tile
     static constexpr int TW = D * N / 2;            // code words per tile
@@ -54,37 +54,51 @@ struct MmaLayout {
     static constexpr int BPW = 4 / N;               // chunks per word (slot classes)
     static constexpr int NGV = D / GV;              // value groups per token
     static constexpr int kTok = 16 * kMmaItemTiles;
-    // stage: one item as it arrives: [key codes][value codes][key scales D f32][key zeros D i16]
-    //        [value scales kTok x NGV f32][value zeros kTok x NGV i16]; codes lane-major per tile
-    static constexpr int kVc = kMmaItemTiles * TW * 4;
-    static constexpr int kKs = 2 * kVc;
-    static constexpr int kKz = kKs + D * 4;
-    static constexpr int kVs = kKz + D * 2;
-    static constexpr int kVz = kVs + kTok * NGV * 4;
-    static constexpr int kStage = (kVz + kTok * NGV * 2 + 15) / 16 * 16;
-    static constexpr int kSt = 2;                            // ring depth: one item in flight
-    // key B operand staging: [part][head][t4][2 NJ words]; rows of 24 words and a part
-    // stride of 4 mod 32 words keep both the producers' 8-byte stores and the consumers'
-    // 16-byte loads free of bank conflicts
+    // A stage holds what arrives for kIPS items, each array as one contiguous block:
+    //   [key codes][value codes][key scales][key zeros][value scales][value zeros],
+    // codes lane-major per tile, and the key scales / zeros of up to kGPS key groups.
+    // RR (round robin, key groups of 2 tiles): one ring shared by the CTA whose stages hold
+    // a round, the kDecodeWarps consecutive items the warps take one each.  A round is
+    // 2 kDecodeWarps tiles from an even tile, so it meets at most kDecodeWarps groups.
+    // Otherwise every warp has a ring of its own whose stages hold one of its items.
+    static constexpr int kIPS = RR ? kDecodeWarps : 1;             // items per stage
+    static constexpr int kGPS = RR ? kDecodeWarps : 1;             // key groups per stage
+    static constexpr int kRings = RR ? 1 : kDecodeWarps;
+    static constexpr int kItemCodes = kMmaItemTiles * TW * 4;   // bytes of one item's key (or value) codes
+    static constexpr int kItemVs = kTok * NGV * 4;              // bytes of one item's value scales
+    static constexpr int kRk = 0;
+    static constexpr int kRv = kIPS * kItemCodes;
+    static constexpr int kRks = 2 * kIPS * kItemCodes;
+    static constexpr int kRkz = kRks + kGPS * D * 4;
+    static constexpr int kRvs = kRkz + kGPS * D * 2;
+    static constexpr int kRvz = kRvs + kIPS * kItemVs;
+    static constexpr int kStage = (kRvz + kIPS * kItemVs / 2 + 127) / 128 * 128;
+    static constexpr int kSt = 2;                            // ring depth: one stage in flight
+    // per-warp scratch.  Key B staging [part][head][t4][2 NJ words]: rows of 24 words and a
+    // part stride of 4 mod 32 words keep both the producers' 8-byte stores and the
+    // consumers' 16-byte loads free of bank conflicts.  It is dead once the fragments are in
+    // registers, so the value-phase buffers share its memory.
     static constexpr int RS = 24;
     static constexpr int PS = HG * 4 * RS + 4;
     // value B exchange (NGV >= 4): [part][head][t4][e][NGV words], part stride 4 mod 32 words
     static constexpr int VXS = HG * 4 * 2 * NGV + 4;
-    static constexpr int kKb = kSt * kStage;                       // u32 [2 * PS]
-    static constexpr int kVx = kKb + 2 * PS * 4;                   // u32 [2 * VXS]
-    static constexpr int kUv = kVx + (NGV >= 4 ? 2 * VXS * 4 : 0); // f32 [kTok][NGV]: s z per (token, group)
-    static constexpr int kPb = kUv + kTok * NGV * 4;               // f32 [2 tiles][HG][18]: p 2^80
-    static constexpr int kBars = kPb + kMmaItemTiles * HG * 18 * 4;
-    // (the residual splits stage one 16-row tile of K and V rows in the same memory)
-    static constexpr int kUsed = (kBars + kSt * 8 + 15) / 16 * 16;
-    static constexpr int kWarpBytes = kUsed > residual_scratch_bytes<D>() ? kUsed : residual_scratch_bytes<D>();
+    static constexpr int kKb = 0;                                    // u32 [2 * PS]
+    static constexpr int kVx = 0;                                    // u32 [2 * VXS]
+    static constexpr int kUv = kVx + (NGV >= 4 ? 2 * VXS * 4 : 0);   // f32 [kTok][NGV]: s z per (token, group)
+    static constexpr int kPb = kUv + kTok * NGV * 4;                 // f32 [2 tiles][HG][18]: p 2^80
+    static constexpr int kValueEnd = kPb + kMmaItemTiles * HG * 18 * 4;
+    static constexpr int kWarpBytes = ((2 * PS * 4 > kValueEnd ? 2 * PS * 4 : kValueEnd) + 15) / 16 * 16;
+    static constexpr int kQuantBytes = kRings * kSt * kStage + kDecodeWarps * kWarpBytes;
+    // (the residual splits stage one 16-row tile of K and V rows per warp in the same memory)
+    static constexpr int kSmem = kQuantBytes > kDecodeWarps * residual_scratch_bytes<D>()
+                                     ? kQuantBytes : kDecodeWarps * residual_scratch_bytes<D>();
     static_assert(2 * NJ <= RS, "row");
-    static_assert(kVc % 16 == 0 && kKs % 16 == 0 && kKz % 16 == 0 && kVs % 16 == 0 && kVz % 16 == 0 &&
-                  kKb % 16 == 0 && kVx % 16 == 0 && kUv % 16 == 0 && kPb % 16 == 0 && kBars % 8 == 0, "align");
+    static_assert(kItemCodes % 16 == 0 && kRv % 16 == 0 && kRks % 16 == 0 && kRkz % 16 == 0 && kRvs % 16 == 0 &&
+                  kRvz % 16 == 0 && (kItemVs / 2) % 16 == 0 && kUv % 16 == 0 && kPb % 16 == 0, "align");
 };
 
-template <int N, int D, int GV, int HG>
-__host__ __device__ constexpr int mma_smem() { return kDecodeWarps * MmaLayout<N, D, GV, HG>::kWarpBytes; }
+template <int N, int D, int GV, int HG, bool RR>
+__host__ __device__ constexpr int mma_smem() { return MmaLayout<N, D, GV, HG, RR>::kSmem; }
 
 // The barrier arm and the bulk copy on 32-bit shared addresses.
 __device__ __forceinline__ void mbar_expect_tx_u32(uint32_t bar, uint32_t bytes) {
@@ -93,6 +107,9 @@ __device__ __forceinline__ void mbar_expect_tx_u32(uint32_t bar, uint32_t bytes)
 __device__ __forceinline__ void bulk_g2s_u32(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                  ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_u32(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait_u32(uint32_t bar, uint32_t parity) {
     uint32_t ok;
@@ -192,9 +209,9 @@ __device__ __forceinline__ float transpose_reduce(const float (&v)[H], int lane)
     }
 }
 
-template <int N, int D, int GV, int HG>
+template <int N, int D, int GV, int HG, bool RR>
 __global__ void __launch_bounds__(kDecodeThreads, D / GV >= 8 ? 3 : 4) decode_mma_kernel(const DecodeArgs a) {
-    using L = MmaLayout<N, D, GV, HG>;
+    using L = MmaLayout<N, D, GV, HG, RR>;
     constexpr int W = L::W, TW = L::TW, NJ = L::NJ, BPW = L::BPW, NGV = L::NGV;
     constexpr int kSt = L::kSt;
     constexpr uint32_t HALF_L = ((1u << N) - 1u) * 0x00010001u;
@@ -205,15 +222,15 @@ __global__ void __launch_bounds__(kDecodeThreads, D / GV >= 8 ? 3 : 4) decode_mm
     constexpr int HPL = HG / LPQ > 0 ? HG / LPQ : 1;      // heads per producer lane
     static_assert(HG == 1 || HG == 2 || HG == 4, "heads per kv head");
     static_assert(W % 2 == 0 || W == 2, "words");
-    static_assert(residual_scratch_bytes<D>() <= L::kWarpBytes, "residual staging");
     // epilogue: per-warp outputs, then finish_cta's scratch
-    static_assert((kDecodeWarps * HG * D + finish_scratch_floats<HG, D>()) * 4 <= kDecodeWarps * L::kWarpBytes,
-                  "epilogue");
+    static_assert((kDecodeWarps * HG * D + finish_scratch_floats<HG, D>()) * 4 <= L::kSmem, "epilogue");
 
     __shared__ __align__(16) float q_s[HG][D];   // q log2(e) / sqrt(d)
     __shared__ __align__(16) float qm_s[HG][D];  // the key MMA's multipliers: q_s 2^64 2^(-2n class)
     __shared__ float ml_s[kDecodeWarps][HG][2];
     __shared__ int last_s;
+    // full barriers (copies landed), [ring][stage]; RR: then the empty barriers (released)
+    __shared__ uint64_t rbar[L::kRings * kSt + (RR ? kSt : 0)];
     extern __shared__ __align__(128) unsigned char stage_mem[];
 
     const int hk = blockIdx.x, b = blockIdx.y, sigma = blockIdx.z;
@@ -224,7 +241,7 @@ __global__ void __launch_bounds__(kDecodeThreads, D / GV >= 8 ? 3 : 4) decode_mm
     const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x >> 5), 0);
     const int lane = threadIdx.x & 31;
     const int g8 = lane >> 2, t4 = lane & 3;
-    unsigned char *wmem = stage_mem + static_cast<size_t>(warp) * L::kWarpBytes;
+    unsigned char *wmem = stage_mem + L::kRings * kSt * L::kStage + static_cast<size_t>(warp) * L::kWarpBytes;
     const int zsym = 1 << (N - 1);
 
     for (int i = threadIdx.x; i < HG * D; i += kDecodeThreads) {
@@ -232,6 +249,15 @@ __global__ void __launch_bounds__(kDecodeThreads, D / GV >= 8 ? 3 : 4) decode_mm
         const int cls = ((i % D) / 16) % BPW;   // slot class of the channel's chunk
         q_s[i / D][i % D] = qv;
         qm_s[i / D][i % D] = qv * __uint_as_float(static_cast<uint32_t>(127 + kKeyScaleLog2 - 2 * N * cls) << 23);
+    }
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int i = 0; i < L::kRings * kSt; ++i) mbar_init(rbar + i, 1);
+        if constexpr (RR) {
+#pragma unroll
+            for (int i = 0; i < kSt; ++i) mbar_init(rbar + kSt + i, kDecodeWarps);
+        }
+        fence_mbar_init();
     }
     // a fused append: split 0 stores the new token as residual row new_row, for later steps
     // (every CTA of this call reads that row from the new token itself)
@@ -260,7 +286,7 @@ __global__ void __launch_bounds__(kDecodeThreads, D / GV >= 8 ? 3 : 4) decode_mm
 #pragma unroll
         for (int j = 0; j < NJ; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
         residual_pass<D>(a, bh, r_rows, q_s[h], rs * WPH + warp % WPH, (r_rows + 15) / 16, lane, m, lsum, acc,
-                         wmem, WPH * nrs);
+                         stage_mem + warp * residual_scratch_bytes<D>(), WPH * nrs);
         lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
         lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
         lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
@@ -287,58 +313,83 @@ __global__ void __launch_bounds__(kDecodeThreads, D / GV >= 8 ? 3 : 4) decode_mm
     }
 
     // ---------------- quantized split ----------------
+    // The CTA's tiles form items of kMmaItemTiles tiles, and round r gives each warp one item.
+    // RR: warp w takes item w of every kDecodeWarps consecutive items, so a round is contiguous
+    // in memory and arrives in one stage of the CTA's ring with one bulk copy per array.
+    // Otherwise warp w takes the w-th contiguous quarter of the items (so it builds each key
+    // group's operand once) and streams them through a ring of its own.
     const int t_begin = min(n_qt, sigma * a.tiles_per_split);      // multiple of kMmaItemTiles
     const int t_end = min(n_qt, t_begin + a.tiles_per_split);
-    constexpr int kWarpAlign = kMmaItemTiles * kDecodeWarps;
-    const int per_w = kMmaItemTiles * ((t_end - t_begin + kWarpAlign - 1) / kWarpAlign);
-    const int wb = min(t_end, t_begin + warp * per_w);
-    const int ntiles = min(t_end, wb + per_w) - wb;                // even (Tq is a multiple of G >= 32)
-    int nitems = ntiles / kMmaItemTiles;
-    const int64_t tile0 = bh * (a.cap / 16) + wb;                 // global tile of the warp's first tile
+    const int n_items = (t_end - t_begin) / kMmaItemTiles;        // (Tq is a multiple of G >= 32)
+    const int n_rounds = (n_items + kDecodeWarps - 1) / kDecodeWarps;
+    const int my_items = RR ? n_items : min(n_rounds, n_items - warp * n_rounds);   // (may be <= 0)
+    auto item_of = [&](int r) { return RR ? r * kDecodeWarps + warp : warp * n_rounds + r; };
+    const int64_t unit_tile0 = bh * (a.cap / 16);                 // global tile of the unit's tile 0
     const int gmask = (1 << a.gshift) - 1;                         // tiles per key group - 1
-    uint64_t *bars = reinterpret_cast<uint64_t *>(wmem + L::kBars);
     uint32_t *kbs = reinterpret_cast<uint32_t *>(wmem + L::kKb);
     float *pb = reinterpret_cast<float *>(wmem + L::kPb);
 
-    if (lane == 0) {
-#pragma unroll
-        for (int s = 0; s < kSt; ++s) mbar_init(bars + s, 1);
-        fence_mbar_init();
-    }
-    __syncwarp();
-
-    // Producer: item k of the warp into stage k % kSt, one bulk copy per array (key codes,
-    // value codes, value scales, value zeros and, when the item opens a key group, the group's
-    // key scales and zeros), all issued by lane 0 after it arms the barrier with the item's
-    // byte count.  Every source, destination and size is warp-uniform, so the copies take
-    // their operands from uniform registers and lane 0 issues them back to back.
-    const uint32_t s_stage0 = smem_u32(wmem), s_bar0 = smem_u32(bars);
-    constexpr int64_t kVsb = 16 * NGV * 4;   // value scales of one tile
-    constexpr int64_t kItemCodes = kMmaItemTiles * TW * 4, kItemVs = kMmaItemTiles * kVsb;
-    const unsigned char *kc0 = reinterpret_cast<const unsigned char *>(a.kc) + tile0 * TW * 4;
-    const unsigned char *vc0 = reinterpret_cast<const unsigned char *>(a.vc) + tile0 * TW * 4;
-    const unsigned char *vs0 = reinterpret_cast<const unsigned char *>(a.vs) + tile0 * kVsb;
-    const unsigned char *vz0 = reinterpret_cast<const unsigned char *>(a.vz) + tile0 * (kVsb / 2);
-    const uint32_t tx_item = 2u * L::kVc + kMmaItemTiles * 16 * NGV * (a.sym ? 4u : 6u);
-    const uint32_t tx_keymeta = static_cast<uint32_t>(D * (a.sym ? 4 : 6));
-    auto issue = [&](int k) {
-        if (k >= nitems) return;
-        const bool open = k == 0 || ((wb + kMmaItemTiles * k) & gmask) == 0;
-        const uint32_t slot = static_cast<uint32_t>(k % kSt);
-        const uint32_t bar = s_bar0 + 8u * slot, dst = s_stage0 + slot * L::kStage;
-        fence_proxy_async();   // this stage's earlier reads come before the copies below
-        if (lane == 0) {
-            mbar_expect_tx_u32(bar, tx_item + (open ? tx_keymeta : 0u));
-            bulk_g2s_u32(dst, kc0 + k * kItemCodes, L::kVc, bar);
-            bulk_g2s_u32(dst + L::kVc, vc0 + k * kItemCodes, L::kVc, bar);
-            bulk_g2s_u32(dst + L::kVs, vs0 + k * kItemVs, kItemVs, bar);
-            if (!a.sym) bulk_g2s_u32(dst + L::kVz, vz0 + k * (kItemVs / 2), kItemVs / 2, bar);
-            if (open) {
-                const int64_t g = (tile0 + kMmaItemTiles * k) >> a.gshift;   // the key group
-                bulk_g2s_u32(dst + L::kKs, reinterpret_cast<const unsigned char *>(a.ks) + g * (D * 4), D * 4, bar);
-                if (!a.sym)
-                    bulk_g2s_u32(dst + L::kKz, reinterpret_cast<const unsigned char *>(a.kz) + g * (D * 2), D * 2,
-                                 bar);
+    // Stage r mod kSt of the ring and its full barrier; RR: the stage's empty barrier, which
+    // every warp arrives at once done with the round.
+    const int ring = RR ? 0 : warp;
+    const uint32_t s_stage0 = smem_u32(stage_mem) + ring * kSt * L::kStage;
+    const uint32_t s_full0 = smem_u32(rbar) + 8u * ring * kSt, s_empty0 = smem_u32(rbar) + 8u * L::kRings * kSt;
+    const unsigned char *kc = reinterpret_cast<const unsigned char *>(a.kc);
+    const unsigned char *vc = reinterpret_cast<const unsigned char *>(a.vc);
+    const unsigned char *vs = reinterpret_cast<const unsigned char *>(a.vs);
+    const unsigned char *vz = reinterpret_cast<const unsigned char *>(a.vz);
+    const unsigned char *ks = reinterpret_cast<const unsigned char *>(a.ks);
+    const unsigned char *kz = reinterpret_cast<const unsigned char *>(a.kz);
+    // Producer of round r (RR: lane 0 of warp r mod kDecodeWarps, the role rotating, once every
+    // warp released the stage's previous round; else lane 0 of the ring's own warp): it arms
+    // the stage's full barrier with the byte count and issues the copies.  Sources,
+    // destinations and sizes are warp-uniform, so the copies take their operands from
+    // uniform registers.
+    auto issue_round = [&](int r) {
+        const uint32_t slot = static_cast<uint32_t>(r % kSt);
+        const uint32_t bar = s_full0 + 8u * slot, dst = s_stage0 + slot * L::kStage;
+        fence_proxy_async();   // the stage's earlier reads come before the copies below
+        if constexpr (RR) {
+            const int i0 = r * kDecodeWarps;
+            const int ni = min(kDecodeWarps, n_items - i0);
+            const int t0 = t_begin + i0 * kMmaItemTiles;               // unit-local tiles [t0, t1)
+            const int t1 = t0 + ni * kMmaItemTiles;
+            const int g0 = t0 >> a.gshift;
+            const uint32_t ng = static_cast<uint32_t>(((t1 - 1) >> a.gshift) - g0 + 1);
+            const uint32_t codes = static_cast<uint32_t>(ni) * L::kItemCodes;
+            const uint32_t vsb = static_cast<uint32_t>(ni) * L::kItemVs, ksb = ng * (D * 4);
+            const uint32_t tx = 2u * codes + vsb + ksb + (a.sym ? 0u : (vsb + ksb) / 2);
+            if (lane == 0) {
+                const int64_t gt = unit_tile0 + t0, gg = (unit_tile0 >> a.gshift) + g0;
+                mbar_expect_tx_u32(bar, tx);
+                bulk_g2s_u32(dst + L::kRk, kc + gt * (TW * 4), codes, bar);
+                bulk_g2s_u32(dst + L::kRv, vc + gt * (TW * 4), codes, bar);
+                bulk_g2s_u32(dst + L::kRvs, vs + gt * (16 * NGV * 4), vsb, bar);
+                bulk_g2s_u32(dst + L::kRks, ks + gg * (D * 4), ksb, bar);
+                if (!a.sym) {
+                    bulk_g2s_u32(dst + L::kRvz, vz + gt * (16 * NGV * 2), vsb / 2, bar);
+                    bulk_g2s_u32(dst + L::kRkz, kz + gg * (D * 2), ksb / 2, bar);
+                }
+            }
+        } else {
+            // the warp's item r; its key group's scales / zeros when it opens a group or
+            // starts the warp's quarter
+            const int t = t_begin + item_of(r) * kMmaItemTiles;
+            const bool open = r == 0 || (t & gmask) == 0;
+            const uint32_t tx = 2u * L::kItemCodes + L::kItemVs + (a.sym ? 0u : L::kItemVs / 2) +
+                                (open ? static_cast<uint32_t>(D * (a.sym ? 4 : 6)) : 0u);
+            if (lane == 0) {
+                const int64_t gt = unit_tile0 + t;
+                mbar_expect_tx_u32(bar, tx);
+                bulk_g2s_u32(dst + L::kRk, kc + gt * (TW * 4), L::kItemCodes, bar);
+                bulk_g2s_u32(dst + L::kRv, vc + gt * (TW * 4), L::kItemCodes, bar);
+                bulk_g2s_u32(dst + L::kRvs, vs + gt * (16 * NGV * 4), L::kItemVs, bar);
+                if (!a.sym) bulk_g2s_u32(dst + L::kRvz, vz + gt * (16 * NGV * 2), L::kItemVs / 2, bar);
+                if (open) {
+                    const int64_t gg = gt >> a.gshift;
+                    bulk_g2s_u32(dst + L::kRks, ks + gg * (D * 4), D * 4, bar);
+                    if (!a.sym) bulk_g2s_u32(dst + L::kRkz, kz + gg * (D * 2), D * 2, bar);
+                }
             }
         }
     };
@@ -364,12 +415,12 @@ __global__ void __launch_bounds__(kDecodeThreads, D / GV >= 8 ? 3 : 4) decode_mm
     const int te = 4 * t4 + e;                 // value-B tokens te, te + 2 of a tile
     const int kb_row = e * L::PS + (hb * 4 + t4) * L::RS;
 
-    // Key B operand and bias of the group whose scales / zeros sit in stage st.
-    auto build_key_b = [&](const unsigned char *st) {
-        const float4 s4 = *reinterpret_cast<const float4 *>(st + L::kKs + 16 * quad);
+    // Key B operand and bias of the group whose scales / zeros sit at ksp / kzp.
+    auto build_key_b = [&](const unsigned char *ksp, const unsigned char *kzp) {
+        const float4 s4 = *reinterpret_cast<const float4 *>(ksp + 16 * quad);
         float2 z01 = make_float2(static_cast<float>(zsym), static_cast<float>(zsym)), z23 = z01;
         if (!a.sym) {
-            const uint2 zz = *reinterpret_cast<const uint2 *>(st + L::kKz + 8 * quad);
+            const uint2 zz = *reinterpret_cast<const uint2 *>(kzp + 8 * quad);
             z01 = make_float2(static_cast<float>(static_cast<int16_t>(zz.x & 0xffffu)),
                               static_cast<float>(static_cast<int16_t>(zz.x >> 16)));
             z23 = make_float2(static_cast<float>(static_cast<int16_t>(zz.y & 0xffffu)),
@@ -410,11 +461,13 @@ __global__ void __launch_bounds__(kDecodeThreads, D / GV >= 8 ? 3 : 4) decode_mm
         // head t4 mod HG: in the lane group of heads (h / HPL), at lane offset (h mod HPL) QUADS / HPL
         const int hh = t4 % HG;
         kbias = __shfl_sync(0xffffffffu, bsum, (hh / HPL) * QUADS + (hh % HPL) * (QUADS / HPL));
+        __syncwarp();   // the staging is read before the value phase reuses its memory
     };
 
+    bool skip = false;
     if constexpr (kCheck) {
         // bounds-check builds: a bounded wait on a barrier nothing arrives at, which gives up
-        // (kvq_debug_set_stall); the warp then streams nothing
+        // (kvq_debug_set_stall); the warp then follows the rounds without doing their work
         __shared__ uint64_t stall_bar;
         if (a.stall_polls > 0 && hk == 0 && b == 0 && sigma == 0 && warp == 0) {
             if (lane == 0) {
@@ -426,183 +479,218 @@ __global__ void __launch_bounds__(kDecodeThreads, D / GV >= 8 ? 3 : 4) decode_mm
             for (int i = 0; i < a.stall_polls && !done; ++i) done = mbar_try_wait(&stall_bar, 0);
             if (!__all_sync(0xffffffffu, done)) {
                 if (lane == 0) atomicOr(a.status, 1u);
-                nitems = 0;
+                skip = true;
             }
             __syncwarp();
             if (lane == 0) mbar_inval(&stall_bar);
         }
     }
 
+    // RR: round j is issued by warp j mod kDecodeWarps, else by the ring's warp; rounds
+    // 0 .. kSt - 2 now, round r + kSt - 1 while round r is consumed
+    const int n_loop = RR ? n_rounds : my_items;   // the rounds this warp takes part in
+    int my_last = -1;   // the last round this warp issued
 #pragma unroll
-    for (int s = 0; s < kSt - 1; ++s) issue(s);
-
-    int k = 0;
-    for (; k < nitems; ++k) {
-        issue(k + kSt - 1);
-        const bool ok = warp_wait(s_bar0 + 8u * static_cast<uint32_t>(k % kSt), static_cast<uint32_t>(k / kSt) & 1u);
-        if (!ok) {
-            if (lane == 0) atomicOr(a.status, 1u);
+    for (int j = 0; j < kSt - 1; ++j) {
+        if (j < n_loop && (!RR || j == warp)) {
+            issue_round(j);
+            my_last = j;
+        }
+    }
+    int g_cur = -1;     // key group of the fragments in kb
+    bool failed = false;
+    int r = 0;
+    for (; r < n_loop; ++r) {
+        const int rn = r + kSt - 1;
+        if (rn < n_loop && (!RR || rn % kDecodeWarps == warp)) {
+            // RR: the stage's previous round, rn - kSt, must have been released by every warp
+            if (RR && rn >= kSt &&
+                !warp_wait(s_empty0 + 8u * static_cast<uint32_t>(rn % kSt), static_cast<uint32_t>(rn / kSt - 1) & 1u)) {
+                failed = true;
+                break;
+            }
+            issue_round(rn);
+            my_last = rn;
+        }
+        const uint32_t slot = static_cast<uint32_t>(r % kSt);
+        if (!warp_wait(s_full0 + 8u * slot, static_cast<uint32_t>(r / kSt) & 1u)) {
+            failed = true;
             break;
         }
-        const unsigned char *st = wmem + (k % kSt) * L::kStage;
-        const int ti = wb + kMmaItemTiles * k;
-        if (k == 0 || (ti & gmask) == 0) build_key_b(st);
-
-        // ---- keys: log2-domain logits of head t4 mod HG, tokens g8 and g8 + 8 of each tile ----
-        float lg[kMmaItemTiles][2];
-#pragma unroll
-        for (int u = 0; u < kMmaItemTiles; ++u) {
-            uint32_t kw[W];
-            load_lane_words<W>(st + u * TW * 4, lane, kw);
-            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-            for (int wi = 0; wi < W; ++wi) {
-                const uint32_t w02 = kw[wi], w13 = kw[wi] >> 8;
-#pragma unroll
-                for (int c = 0; c < BPW; ++c) {
-                    const int j = wi * BPW + c;
-                    const uint32_t m0 = HALF_L << (N * 2 * c), m1 = HALF_L << (N * (2 * c + 1));
-                    hmma(acc[wi & 1], w02 & m0, w02 & m1, w13 & m0, w13 & m1, kb[j][0], kb[j][1]);
-                }
+        const int item = item_of(r);
+        if (item < n_items && !skip) {
+        const unsigned char *st = stage_mem + (ring * kSt + slot) * L::kStage;
+            const int ti = t_begin + item * kMmaItemTiles;   // unit-local tile of the item
+            if ((ti >> a.gshift) != g_cur) {
+                g_cur = ti >> a.gshift;
+                // the group's slot: its place among the round's groups, or the warp's own slot
+                const int gi = RR ? g_cur - ((t_begin + r * kDecodeWarps * kMmaItemTiles) >> a.gshift) : 0;
+                build_key_b(st + L::kRks + gi * (D * 4), st + L::kRkz + gi * (D * 2));
             }
-            constexpr float f0 = static_cast<float>(1ull << 62) * 128.0f;                       // 2^69
-            constexpr float f1 = static_cast<float>(1ull << 62) * static_cast<float>(128 >> N); // 2^(69 - n)
-            lg[u][0] = fmaf((acc[0][0] + acc[1][0]) + (acc[0][1] + acc[1][1]), f0, -kbias);
-            lg[u][1] = fmaf((acc[0][2] + acc[1][2]) + (acc[0][3] + acc[1][3]), f1, -kbias);
-        }
+            const int is = RR ? warp : 0;   // the item's place in the stage
+            const unsigned char *kcp = st + L::kRk + is * L::kItemCodes;
+            const unsigned char *vcp = st + L::kRv + is * L::kItemCodes;
+            const float *vsp = reinterpret_cast<const float *>(st + L::kRvs + is * L::kItemVs);
+            const int16_t *vzp = reinterpret_cast<const int16_t *>(st + L::kRvz + is * (L::kItemVs / 2));
 
-        // ---- online softmax of head t4 mod HG: the item's maximum, rescale, p ----
-        {
-            float mx = fmaxf(fmaxf(lg[0][0], lg[0][1]), fmaxf(lg[1][0], lg[1][1]));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-            // lazily: only when the item's maximum passes the running one by more than
-            // kLazyRescale (p may reach 2^kLazyRescale meanwhile), so rescales stay rare
-            if (__any_sync(0xffffffffu, mx > m_own + kLazyRescale)) {
-                const float mn = fmaxf(m_own, mx);
-                const float alpha = fast_exp2(m_own - mn);
-                m_own = mn;
-#pragma unroll
-                for (int j = 0; j < NJ; ++j) {
-                    dv[j][0] *= alpha; dv[j][1] *= alpha; dv[j][2] *= alpha; dv[j][3] *= alpha;
-                }
-                lsum *= alpha;
-                const float ab = __shfl_sync(0xffffffffu, alpha, hb);   // lane hb holds head hb
-#pragma unroll
-                for (int v = 0; v < NGV; ++v) zsum[v] *= ab;
-            }
-        }
-        // p 2^80 = 2^(logit - (m - 80)): the value MMA's scale comes with the exponential
-        const float m80 = m_own - static_cast<float>(kValScaleLog2);
-        if (t4 < HG) {
+            // ---- keys: log2-domain logits of head t4 mod HG, tokens g8 and g8 + 8 of each tile ----
+            float lg[kMmaItemTiles][2];
 #pragma unroll
             for (int u = 0; u < kMmaItemTiles; ++u) {
-                const float p0 = fast_exp2(lg[u][0] - m80), p1 = fast_exp2(lg[u][1] - m80);
-                lsum += p0 + p1;
-                pb[(u * HG + t4) * 18 + logit_pos(g8)] = p0;
-                pb[(u * HG + t4) * 18 + logit_pos(g8 + 8)] = p1;
-            }
-        }
-        // value meta of the item: lane l computes s z of token l for every value group
-        float *uv = reinterpret_cast<float *>(wmem + L::kUv);
-        {
-            float sv[NGV];
-            int16_t zv[NGV];
-            load_meta<NGV>(reinterpret_cast<const float *>(st + L::kVs) + lane * NGV,
-                           reinterpret_cast<const int16_t *>(st + L::kVz) + lane * NGV, a.sym, zsym, sv, zv);
-            float uz[NGV];
+                uint32_t kw[W];
+                load_lane_words<W>(kcp + u * TW * 4, lane, kw);
+                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-            for (int v = 0; v < NGV; ++v) uz[v] = sv[v] * static_cast<float>(zv[v]);
-            store_vec<NGV>(uv + lane * NGV, uz);
-        }
-        __syncwarp();
+                for (int wi = 0; wi < W; ++wi) {
+                    const uint32_t w02 = kw[wi], w13 = kw[wi] >> 8;
+#pragma unroll
+                    for (int c = 0; c < BPW; ++c) {
+                        const int j = wi * BPW + c;
+                        const uint32_t m0 = HALF_L << (N * 2 * c), m1 = HALF_L << (N * (2 * c + 1));
+                        hmma(acc[wi & 1], w02 & m0, w02 & m1, w13 & m0, w13 & m1, kb[j][0], kb[j][1]);
+                    }
+                }
+                constexpr float f0 = static_cast<float>(1ull << 62) * 128.0f;                       // 2^69
+                constexpr float f1 = static_cast<float>(1ull << 62) * static_cast<float>(128 >> N); // 2^(69 - n)
+                lg[u][0] = fmaf((acc[0][0] + acc[1][0]) + (acc[0][1] + acc[1][1]), f0, -kbias);
+                lg[u][1] = fmaf((acc[0][2] + acc[1][2]) + (acc[0][3] + acc[1][3]), f1, -kbias);
+            }
 
-        // ---- values: B = p s 2^80 of head hb; lane (g8, t4) builds both parts for tokens
-        //      te, te + 2 of a tile (the k pair of B register e) and trades halves with
-        //      lane g8 ^ 1 ----
+            // ---- online softmax of head t4 mod HG: the item's maximum, rescale, p ----
+            {
+                float mx = fmaxf(fmaxf(lg[0][0], lg[0][1]), fmaxf(lg[1][0], lg[1][1]));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                // lazily: only when the item's maximum passes the running one by more than
+                // kLazyRescale (p may reach 2^kLazyRescale meanwhile), so rescales stay rare
+                if (__any_sync(0xffffffffu, mx > m_own + kLazyRescale)) {
+                    const float mn = fmaxf(m_own, mx);
+                    const float alpha = fast_exp2(m_own - mn);
+                    m_own = mn;
 #pragma unroll
-        for (int u = 0; u < kMmaItemTiles; ++u) {
-            const float2 pp = *reinterpret_cast<const float2 *>(pb + (u * HG + hb) * 18 + 4 * t4 + 2 * e);
-            float s0[NGV], s1[NGV], u0[NGV], u1[NGV];
-            const int r0 = 16 * u + te, r1 = r0 + 2;
-            load_vec<NGV>(reinterpret_cast<const float *>(st + L::kVs) + r0 * NGV, s0);
-            load_vec<NGV>(reinterpret_cast<const float *>(st + L::kVs) + r1 * NGV, s1);
-            load_vec<NGV>(uv + r0 * NGV, u0);
-            load_vec<NGV>(uv + r1 * NGV, u1);
-            uint32_t hi[NGV], lo[NGV];
-            if constexpr (NGV % 2 == 0) {
-                // packed over value-group pairs: (ps0[v], ps0[v + 1]), (ps1[v], ps1[v + 1])
+                    for (int j = 0; j < NJ; ++j) {
+                        dv[j][0] *= alpha; dv[j][1] *= alpha; dv[j][2] *= alpha; dv[j][3] *= alpha;
+                    }
+                    lsum *= alpha;
+                    const float ab = __shfl_sync(0xffffffffu, alpha, hb);   // lane hb holds head hb
 #pragma unroll
-                for (int v = 0; v < NGV; v += 2) {
-                    const float2 a0 = mul2(make_float2(pp.x, pp.x), make_float2(s0[v], s0[v + 1]));
-                    const float2 a1 = mul2(make_float2(pp.y, pp.y), make_float2(s1[v], s1[v + 1]));
-                    float2 zz = fma2(make_float2(pp.x, pp.x), make_float2(u0[v], u0[v + 1]),
-                                     make_float2(zsum[v], zsum[v + 1]));
-                    zz = fma2(make_float2(pp.y, pp.y), make_float2(u1[v], u1[v + 1]), zz);
-                    zsum[v] = zz.x;
-                    zsum[v + 1] = zz.y;
-                    const float2 t0 = make_float2(__uint_as_float(__float_as_uint(a0.x) & 0xffff0000u),
-                                                  __uint_as_float(__float_as_uint(a0.y) & 0xffff0000u));
-                    const float2 t1 = make_float2(__uint_as_float(__float_as_uint(a1.x) & 0xffff0000u),
-                                                  __uint_as_float(__float_as_uint(a1.y) & 0xffff0000u));
-                    const float2 r0 = sub2(a0, t0), r1 = sub2(a1, t1);
-                    hi[v] = bf16_trunc2(a0.x, a1.x);
-                    hi[v + 1] = bf16_trunc2(a0.y, a1.y);
-                    lo[v] = f2bf2(r0.x, r1.x);
-                    lo[v + 1] = f2bf2(r0.y, r1.y);
-                }
-            } else {
-#pragma unroll
-                for (int v = 0; v < NGV; ++v) {
-                    const float ps0 = pp.x * s0[v], ps1 = pp.y * s1[v];
-                    zsum[v] = fmaf(pp.x, u0[v], fmaf(pp.y, u1[v], zsum[v]));
-                    hi[v] = bf16_trunc2(ps0, ps1);
-                    lo[v] = bf16_rem2(ps0, ps1);
+                    for (int v = 0; v < NGV; ++v) zsum[v] *= ab;
                 }
             }
-            uint32_t B0[NGV], B1[NGV];
-            if constexpr (NGV >= 4) {
-                // through shared memory: [part][head][t4][e][v]; this lane's B0 is part e of
-                // tokens (4 t4, 4 t4 + 2) (e = 0 row), B1 part e of (4 t4 + 1, 4 t4 + 3)
-                uint32_t *vx = reinterpret_cast<uint32_t *>(wmem + L::kVx);
-                uint32_t *mine = vx + ((hb * 4 + t4) * 2 + e) * NGV;
-                store_vec<NGV>(mine, hi);
-                store_vec<NGV>(mine + L::VXS, lo);
-                __syncwarp();
-                const uint32_t *part = vx + e * L::VXS + (hb * 4 + t4) * 2 * NGV;
-                load_vec<NGV>(part, B0);
-                load_vec<NGV>(part + NGV, B1);
-            } else {
+            // p 2^80 = 2^(logit - (m - 80)): the value MMA's scale comes with the exponential
+            const float m80 = m_own - static_cast<float>(kValScaleLog2);
+            if (t4 < HG) {
 #pragma unroll
-                for (int v = 0; v < NGV; ++v) {
-                    const uint32_t y = __shfl_xor_sync(0xffffffffu, e ? hi[v] : lo[v], 4);
-                    B0[v] = e ? y : hi[v];
-                    B1[v] = e ? lo[v] : y;
+                for (int u = 0; u < kMmaItemTiles; ++u) {
+                    const float p0 = fast_exp2(lg[u][0] - m80), p1 = fast_exp2(lg[u][1] - m80);
+                    lsum += p0 + p1;
+                    pb[(u * HG + t4) * 18 + logit_pos(g8)] = p0;
+                    pb[(u * HG + t4) * 18 + logit_pos(g8 + 8)] = p1;
                 }
             }
-            uint32_t vw[W];
-            load_lane_words<W>(st + L::kVc + u * TW * 4, lane, vw);
+            // value meta of the item: lane l computes s z of token l for every value group
+            float *uv = reinterpret_cast<float *>(wmem + L::kUv);
+            {
+                float sv[NGV];
+                int16_t zv[NGV];
+                load_meta<NGV>(vsp + lane * NGV, vzp + lane * NGV, a.sym, zsym, sv, zv);
+                float uz[NGV];
 #pragma unroll
-            for (int wi = 0; wi < W; ++wi) {
-                const uint32_t w02 = vw[wi], w13 = vw[wi] >> 8;
-#pragma unroll
-                for (int c = 0; c < BPW; ++c) {
-                    const int j = wi * BPW + c;
-                    const uint32_t m0 = HALF_L << (N * 2 * c), m1 = HALF_L << (N * (2 * c + 1));
-                    hmma(dv[j], w02 & m0, w02 & m1, w13 & m0, w13 & m1, B0[(16 * j) / GV], B1[(16 * j) / GV]);
-                }
+                for (int v = 0; v < NGV; ++v) uz[v] = sv[v] * static_cast<float>(zv[v]);
+                store_vec<NGV>(uv + lane * NGV, uz);
             }
-            if constexpr (NGV >= 4) __syncwarp();   // the exchange is read before the next tile writes it
+            __syncwarp();
+
+            // ---- values: B = p s 2^80 of head hb; lane (g8, t4) builds both parts for tokens
+            //      te, te + 2 of a tile (the k pair of B register e) and trades halves with
+            //      lane g8 ^ 1 ----
+#pragma unroll
+            for (int u = 0; u < kMmaItemTiles; ++u) {
+                const float2 pp = *reinterpret_cast<const float2 *>(pb + (u * HG + hb) * 18 + 4 * t4 + 2 * e);
+                float s0[NGV], s1[NGV], u0[NGV], u1[NGV];
+                const int r0 = 16 * u + te, r1 = r0 + 2;
+                load_vec<NGV>(vsp + r0 * NGV, s0);
+                load_vec<NGV>(vsp + r1 * NGV, s1);
+                load_vec<NGV>(uv + r0 * NGV, u0);
+                load_vec<NGV>(uv + r1 * NGV, u1);
+                uint32_t hi[NGV], lo[NGV];
+                if constexpr (NGV % 2 == 0) {
+                    // packed over value-group pairs: (ps0[v], ps0[v + 1]), (ps1[v], ps1[v + 1])
+#pragma unroll
+                    for (int v = 0; v < NGV; v += 2) {
+                        const float2 a0 = mul2(make_float2(pp.x, pp.x), make_float2(s0[v], s0[v + 1]));
+                        const float2 a1 = mul2(make_float2(pp.y, pp.y), make_float2(s1[v], s1[v + 1]));
+                        float2 zz = fma2(make_float2(pp.x, pp.x), make_float2(u0[v], u0[v + 1]),
+                                         make_float2(zsum[v], zsum[v + 1]));
+                        zz = fma2(make_float2(pp.y, pp.y), make_float2(u1[v], u1[v + 1]), zz);
+                        zsum[v] = zz.x;
+                        zsum[v + 1] = zz.y;
+                        const float2 t0 = make_float2(__uint_as_float(__float_as_uint(a0.x) & 0xffff0000u),
+                                                      __uint_as_float(__float_as_uint(a0.y) & 0xffff0000u));
+                        const float2 t1 = make_float2(__uint_as_float(__float_as_uint(a1.x) & 0xffff0000u),
+                                                      __uint_as_float(__float_as_uint(a1.y) & 0xffff0000u));
+                        const float2 r0 = sub2(a0, t0), r1 = sub2(a1, t1);
+                        hi[v] = bf16_trunc2(a0.x, a1.x);
+                        hi[v + 1] = bf16_trunc2(a0.y, a1.y);
+                        lo[v] = f2bf2(r0.x, r1.x);
+                        lo[v + 1] = f2bf2(r0.y, r1.y);
+                    }
+                } else {
+#pragma unroll
+                    for (int v = 0; v < NGV; ++v) {
+                        const float ps0 = pp.x * s0[v], ps1 = pp.y * s1[v];
+                        zsum[v] = fmaf(pp.x, u0[v], fmaf(pp.y, u1[v], zsum[v]));
+                        hi[v] = bf16_trunc2(ps0, ps1);
+                        lo[v] = bf16_rem2(ps0, ps1);
+                    }
+                }
+                uint32_t B0[NGV], B1[NGV];
+                if constexpr (NGV >= 4) {
+                    // through shared memory: [part][head][t4][e][v]; this lane's B0 is part e of
+                    // tokens (4 t4, 4 t4 + 2) (e = 0 row), B1 part e of (4 t4 + 1, 4 t4 + 3)
+                    uint32_t *vx = reinterpret_cast<uint32_t *>(wmem + L::kVx);
+                    uint32_t *mine = vx + ((hb * 4 + t4) * 2 + e) * NGV;
+                    store_vec<NGV>(mine, hi);
+                    store_vec<NGV>(mine + L::VXS, lo);
+                    __syncwarp();
+                    const uint32_t *part = vx + e * L::VXS + (hb * 4 + t4) * 2 * NGV;
+                    load_vec<NGV>(part, B0);
+                    load_vec<NGV>(part + NGV, B1);
+                } else {
+#pragma unroll
+                    for (int v = 0; v < NGV; ++v) {
+                        const uint32_t y = __shfl_xor_sync(0xffffffffu, e ? hi[v] : lo[v], 4);
+                        B0[v] = e ? y : hi[v];
+                        B1[v] = e ? lo[v] : y;
+                    }
+                }
+                uint32_t vw[W];
+                load_lane_words<W>(vcp + u * TW * 4, lane, vw);
+#pragma unroll
+                for (int wi = 0; wi < W; ++wi) {
+                    const uint32_t w02 = vw[wi], w13 = vw[wi] >> 8;
+#pragma unroll
+                    for (int c = 0; c < BPW; ++c) {
+                        const int j = wi * BPW + c;
+                        const uint32_t m0 = HALF_L << (N * 2 * c), m1 = HALF_L << (N * (2 * c + 1));
+                        hmma(dv[j], w02 & m0, w02 & m1, w13 & m0, w13 & m1, B0[(16 * j) / GV], B1[(16 * j) / GV]);
+                    }
+                }
+                if constexpr (NGV >= 4) __syncwarp();   // the exchange is read before the next tile writes it
+            }
         }
-        __syncwarp();   // stage, p buffer and key fragments consumed before they are refilled
+        __syncwarp();   // the warp's reads of the stage and its scratch are done
+        if (RR && lane == 0) mbar_arrive_u32(s_empty0 + 8u * slot);
     }
-    // after an abandoned wait: give the copies still in flight their (bounded) time to land
-    for (int j = k + 1; j < min(k + kSt, nitems); ++j) mbar_wait_bounded(bars + j % kSt, (j / kSt) & 1);
-    __syncwarp();
-    if (lane == 0) {
-#pragma unroll
-        for (int s = 0; s < kSt; ++s) mbar_inval(bars + s);
+    if (failed) {
+        // an abandoned wait: the status word says so; the copies this warp issued for rounds
+        // it has not waited for get their (bounded) time to land before the CTA exits
+        if (lane == 0) atomicOr(a.status, 1u);
+        for (int j = r; j <= my_last; ++j)
+            if (!RR || j % kDecodeWarps == warp)
+                mbar_wait_bounded(rbar + ring * kSt + j % kSt, static_cast<uint32_t>(j / kSt) & 1u);
+        __syncwarp();
     }
 
     // ---- warp epilogue (lsum and zsum carry the factor 2^80 of p) ----
@@ -647,21 +735,27 @@ __global__ void __launch_bounds__(kDecodeThreads, D / GV >= 8 ? 3 : 4) decode_mm
     finish_cta<HG, D>(a, o_s, ml_s, bh, bq0, sigma, &last_s, o_s + kDecodeWarps * HG * D);
 }
 
+// the round-robin instance for key groups of 2 tiles, else the per-warp rings
 template <int N, int D, int GV, int HG>
 cudaError_t launch_mma(const DecodeArgs &a, cudaStream_t s) {
-    return launch_kernel<decode_mma_kernel<N, D, GV, HG>>(a, dim3(a.Hkv, a.B, a.S), mma_smem<N, D, GV, HG>(), s);
+    if (a.gshift == 1)
+        return launch_kernel<decode_mma_kernel<N, D, GV, HG, true>>(a, dim3(a.Hkv, a.B, a.S),
+                                                                      mma_smem<N, D, GV, HG, true>(), s);
+    return launch_kernel<decode_mma_kernel<N, D, GV, HG, false>>(a, dim3(a.Hkv, a.B, a.S),
+                                                                   mma_smem<N, D, GV, HG, false>(), s);
 }
 template <int N, int D, int GV, int HG>
-int occ_mma() {
-    return occupancy_of<decode_mma_kernel<N, D, GV, HG>>(mma_smem<N, D, GV, HG>());
+int occ_mma(const DecodeArgs &a) {
+    if (a.gshift == 1) return occupancy_of<decode_mma_kernel<N, D, GV, HG, true>>(mma_smem<N, D, GV, HG, true>());
+    return occupancy_of<decode_mma_kernel<N, D, GV, HG, false>>(mma_smem<N, D, GV, HG, false>());
 }
 
 template <int N, int D, int GV>
 cudaError_t launch_mma_hg(const DecodeArgs &a, cudaStream_t s, bool occ_only, int *occ) {
     switch (a.Hq / a.Hkv) {
-        case 1: if (occ_only) { *occ = occ_mma<N, D, GV, 1>(); return cudaSuccess; } return launch_mma<N, D, GV, 1>(a, s);
-        case 2: if (occ_only) { *occ = occ_mma<N, D, GV, 2>(); return cudaSuccess; } return launch_mma<N, D, GV, 2>(a, s);
-        case 4: if (occ_only) { *occ = occ_mma<N, D, GV, 4>(); return cudaSuccess; } return launch_mma<N, D, GV, 4>(a, s);
+        case 1: if (occ_only) { *occ = occ_mma<N, D, GV, 1>(a); return cudaSuccess; } return launch_mma<N, D, GV, 1>(a, s);
+        case 2: if (occ_only) { *occ = occ_mma<N, D, GV, 2>(a); return cudaSuccess; } return launch_mma<N, D, GV, 2>(a, s);
+        case 4: if (occ_only) { *occ = occ_mma<N, D, GV, 4>(a); return cudaSuccess; } return launch_mma<N, D, GV, 4>(a, s);
         default: return cudaErrorInvalidValue;
     }
 }

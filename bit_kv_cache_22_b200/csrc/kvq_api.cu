@@ -54,8 +54,9 @@ kvq_status cuda_fail(cudaError_t e, const char *what) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-constexpr int kMaxSplits = 64;
+constexpr int kMaxSplits = 128;
 constexpr int kMaxResidualSplits = 16;
+static_assert(kMaxSplits + kMaxResidualSplits == kvq::kMaxDecodeSplits, "split bound");
 constexpr int kMinTilesPerSplit = 4;
 
 kvq_status validate(const kvq_config *c) {
@@ -122,7 +123,7 @@ struct kvq_cache {
     int32_t r = 0;
     int num_sms = 148;
     int ctas_per_sm = 4;
-    int split_limit = 64;
+    int split_limit = kMaxSplits;
     int path = kvq::kPathSplit;         // the decode kernel (kvq::DecodePath) serving this cache
     int stall_polls = 0;                // bounds-check builds: see kvq_debug_set_stall
     // LogQuant retention (lq_window W > 0): the residual buffer is the full-precision store
@@ -525,6 +526,36 @@ kvq_status kvq_set_split_limit(kvq_cache *h, int32_t max_splits) {
     if (max_splits < 0 || max_splits > kMaxSplits)
         return fail(KVQ_ERR_INVALID_ARG, "max_splits must be in 0..%d", kMaxSplits);
     h->split_limit = max_splits == 0 ? kMaxSplits : max_splits;
+    return ok();
+}
+
+kvq_status kvq_set_decode_kernel(kvq_cache *h, int32_t kernel) {
+    if (!h) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+    const kvq_config &c = h->cfg;
+    const bool mma_geom = kvq::decode_path(c.q_heads, c.kv_heads, c.group_k) != kvq::kPathSplit;
+    int path;
+    switch (kernel) {
+        case KVQ_DECODE_AUTO:
+            path = h->n_out > 0 ? kvq::kPathTc : kvq::decode_path(c.q_heads, c.kv_heads, c.group_k);
+            break;
+        case KVQ_DECODE_CUDA_CORES:
+            if (h->n_out > 0) return fail(KVQ_ERR_UNSUPPORTED, "key outliers are served by the integer-MMA kernel");
+            path = kvq::kPathSplit;
+            break;
+        case KVQ_DECODE_INT8_MMA:
+        case KVQ_DECODE_BF16_MMA:
+            if (!mma_geom)
+                return fail(KVQ_ERR_UNSUPPORTED, "the MMA kernels need 1, 2 or 4 query heads per kv head and "
+                                                 "key groups of >= 32 tokens");
+            if (kernel == KVQ_DECODE_BF16_MMA && h->n_out > 0)
+                return fail(KVQ_ERR_UNSUPPORTED, "key outliers are served by the integer-MMA kernel");
+            path = kernel == KVQ_DECODE_INT8_MMA ? kvq::kPathTc : kvq::kPathMma;
+            break;
+        default:
+            return fail(KVQ_ERR_INVALID_ARG, "unknown decode kernel %d", kernel);
+    }
+    h->path = path;
+    h->ctas_per_sm = kvq::decode_ctas_per_sm(decode_args(h));
     return ok();
 }
 

@@ -89,6 +89,8 @@ cudaError_t launch_copy_rows(const uint16_t *src0, const uint16_t *src1, int64_t
 //  kPathSplit any other grouping, or 16-token key groups: CUDA cores, one CTA per
 //             (batch, query head, split).
 enum DecodePath : int { kPathSplit = 0, kPathTc = 1, kPathMma = 2 };
+// Most splits of one decode: up to 128 over the quantized tiles and 16 residual ones.
+constexpr int kMaxDecodeSplits = 144;
 
 inline int decode_path(int q_heads, int kv_heads, int group_k, bool plain = true) {
     const int g = q_heads / kv_heads;

@@ -27,6 +27,8 @@ _lib = None
 (KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_STATE, KVQ_ERR_CUDA,
  KVQ_ERR_DEVICE_CHECK) = range(7)
 KVQ_FP16, KVQ_BF16 = 0, 1
+# decode kernels (kvq_set_decode_kernel)
+KVQ_DECODE_AUTO, KVQ_DECODE_CUDA_CORES, KVQ_DECODE_INT8_MMA, KVQ_DECODE_BF16_MMA = range(4)
 
 EXPORTED = ("kvq_get_sizes", "kvq_create", "kvq_destroy", "kvq_reset", "kvq_prefill_quantize",
             "kvq_append", "kvq_decode_attention", "kvq_cache_state", "kvq_set_split_limit",
@@ -37,7 +39,7 @@ EXPORTED = ("kvq_get_sizes", "kvq_create", "kvq_destroy", "kvq_reset", "kvq_pref
             "kvq_paged_decode_attention", "kvq_paged_release", "kvq_paged_seq_len",
             "kvq_paged_decode_splits", "kvq_paged_check_device", "kvq_logquant_get_sizes",
             "kvq_logquant_create", "kvq_logquant_retained", "kvq_set_key_outliers", "kvq_plan_decode",
-            "kvq_binary_arch")
+            "kvq_binary_arch", "kvq_set_decode_kernel")
 
 
 class KVQError(RuntimeError):
@@ -117,6 +119,8 @@ def load() -> ctypes.CDLL:
         lib.kvq_decode_attention_noalloc.restype = ctypes.c_int
         lib.kvq_cache_state.argtypes = [P, ctypes.POINTER(i64), ctypes.POINTER(i32)]
         lib.kvq_set_split_limit.argtypes = [P, i32]
+        lib.kvq_set_decode_kernel.argtypes = [P, i32]
+        lib.kvq_set_decode_kernel.restype = ctypes.c_int
         lib.kvq_decode_splits.argtypes = [P]
         lib.kvq_decode_splits.restype = i32
         lib.kvq_kernel_launches.argtypes = []
@@ -301,6 +305,10 @@ class KVQCache:
 
     def set_split_limit(self, max_splits: int):
         _check(self._lib.kvq_set_split_limit(self._h, max_splits))
+
+    def set_decode_kernel(self, kernel: int):
+        """KVQ_DECODE_AUTO, _CUDA_CORES, _INT8_MMA or _BF16_MMA (kvq_set_decode_kernel)."""
+        _check(self._lib.kvq_set_decode_kernel(self._h, kernel))
 
     def splits(self) -> int:
         return int(self._lib.kvq_decode_splits(self._h))

@@ -256,7 +256,7 @@ KVQ_API kvq_status kvq_cache_state(const kvq_cache *cache, int64_t *quantized_to
 
 /*
  * Upper bound on the splits kvq_decode_attention cuts the quantized tokens into
- * (1 .. 64; 0 restores the default of 64).  With one query head per kv head
+ * (1 .. 128; 0 restores the default of 128).  With one query head per kv head
  * the residual tokens are shared out among those splits; otherwise they form
  * 1 to 16 more splits of their own when there are any (more of them for a
  * longer full-precision part, such as a LogQuant store).  Fewer splits mean fewer
@@ -264,6 +264,31 @@ KVQ_API kvq_status kvq_cache_state(const kvq_cache *cache, int64_t *quantized_to
  * the result is the same up to fp32 rounding.
  */
 KVQ_API kvq_status kvq_set_split_limit(kvq_cache *cache, int32_t max_splits);
+
+/*
+ * The decode kernel a cache's decode calls launch (all read the same layout and give the
+ * same result up to fp32 rounding, so this only trades speed; for measurement and A/B
+ * checks):
+ *   KVQ_DECODE_AUTO        the library's choice (the default): KVQ_DECODE_BF16_MMA where it
+ *                          applies, else KVQ_DECODE_INT8_MMA with key outliers, else
+ *                          KVQ_DECODE_CUDA_CORES;
+ *   KVQ_DECODE_CUDA_CORES  decode_split_kernel, CUDA cores only (any geometry);
+ *   KVQ_DECODE_INT8_MMA    decode_tc_kernel: keys on integer mma.sync against fixed-point
+ *                          query digits, values on bf16 mma.sync;
+ *   KVQ_DECODE_BF16_MMA    decode_mma_kernel: keys and values on bf16 mma.sync.
+ * The MMA kernels need 1, 2 or 4 query heads per kv head and key groups of >= 32 tokens;
+ * KVQ_DECODE_BF16_MMA also needs a cache without key outliers (kvq_set_key_outliers),
+ * which serves KVQ_DECODE_AUTO and KVQ_DECODE_INT8_MMA only.  Otherwise
+ * KVQ_ERR_UNSUPPORTED and the cache keeps its kernel.  Host only; takes effect at the next
+ * decode call.
+ */
+enum {
+    KVQ_DECODE_AUTO = 0,
+    KVQ_DECODE_CUDA_CORES = 1,
+    KVQ_DECODE_INT8_MMA = 2,
+    KVQ_DECODE_BF16_MMA = 3
+};
+KVQ_API kvq_status kvq_set_decode_kernel(kvq_cache *cache, int32_t kernel);
 
 /*
  * The split plan of a decode over cfg->batch sequences of lengths[b] tokens each

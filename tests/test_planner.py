@@ -42,8 +42,8 @@ def test_plan_invariants(seed):
     tiles = [max(x, 0) // R * R // 16 for x in lens]
     rres = max(max(x, 0) % R for x in lens)
     tc = g in (1, 2, 4) and G >= 32
-    assert S >= 1 and S - nq <= 16 and nq <= 64
-    assert S <= min(cap // 16, 64) + 16                    # the workspace's bound
+    assert S >= 1 and S - nq <= 16 and nq <= 128
+    assert S <= min(cap // 16, 128) + 16                   # the workspace's bound
     if max(tiles) > 0:
         assert nq * per >= max(tiles) > (nq - 1) * per     # every tile covered, no empty last split
         if tc:
