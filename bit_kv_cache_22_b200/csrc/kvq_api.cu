@@ -151,8 +151,9 @@ namespace {
 // kCtaFixedTiles tiles plus the tiles its busiest warp streams (an empty split
 // costs kEmptyCtaTiles); the kernel's time as the larger of (the waves of quantized
 // CTAs over the GPU's resident slots x one quantized CTA) and (all CTA time spread
-// evenly over the slots, plus one residual CTA).  The split count with the lowest
-// modelled time wins (ties: fewer splits).
+// evenly over the slots, plus one residual CTA); when every CTA is resident at once it
+// is the longest CTA's.  The split count with the lowest modelled time wins (ties:
+// fewer splits).
 constexpr double kCtaFixedTiles = 6.0;
 constexpr double kEmptyCtaTiles = 1.0;
 
@@ -231,6 +232,8 @@ void plan_splits_for(const kvq_cache *h, const PlanInput &in, int *n_qsplits, in
                 if (n_rs) t_crit = (nq + n_res > slots) ? c_q + c_res : (c_res > c_q ? c_res : c_q);
                 double cost = t_waves > t_spread ? t_waves : t_spread;
                 cost = cost > t_crit ? cost : t_crit;
+                // every CTA resident at once (one wave): the longest CTA sets the time
+                if (nq + n_res + n_empty <= slots) cost = t_crit;
                 if (best_cost < 0 || cost < best_cost - 1e-9) {
                     best_cost = cost;
                     best_S = S;

@@ -22,8 +22,12 @@
 // list (a LogQuant block); its output slice is a page of a paged pool when a
 // page table is given; dense-and-sparse keys first move each token's largest
 // entries out of the dense part.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
 #include <cfloat>
 #include <cstdint>
+#include <type_traits>
 
 #include "kvq_internal.cuh"
 
@@ -78,18 +82,21 @@ __device__ __forceinline__ float2 add_x2(float2 a, float2 b) {
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(pack2(a)), "l"(pack2(b)));
     return unpack2(d);
 }
-__device__ __forceinline__ float2 fma_x2(float2 a, float2 b, float2 c) {
+__device__ __forceinline__ float2 sub_x2(float2 a, float2 b) {
     unsigned long long d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(pack2(a)), "l"(pack2(b)), "l"(pack2(c)));
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(pack2(a)), "l"(pack2(b)));
     return unpack2(d);
 }
 
-// One group's parameters for code_pair: code = clamp(round(x / s) + off, 0, L), with
+// One group's parameters for code_quad: code = clamp(round(x / s) + off, 0, L), with
 // off = z (asymmetric) or 2^(n-1) (symmetric: clamp(round(x/s), -2^(n-1), 2^(n-1)-1) +
 // 2^(n-1) is the same clamp).  ri = RN(1/s) (0 when s = 0, which gives code off).
-// cut2 = (1/2 - 2^-18 qmax)^2 with qmax >= |x / s| over the group.
+// cut = 1/2 - 2^-18 qmax with qmax >= |x / s| over the group.  q = RN(x ri) is within
+// |q| 2^-22 of RN(x / s), so both round to the same integer unless q lies within that
+// distance of a half-integer; while |q - round(q)| < cut it is more than qmax 2^-18 away
+// (an all-zero group has q = 0).  An element nearer a tie takes the IEEE division.
 struct CodeParams {
-    float s, ri, cut2;
+    float s, ri, cut;
     int off;
 };
 
@@ -97,30 +104,59 @@ __device__ __forceinline__ CodeParams code_params(float s, int off, float amax) 
     const float ri = s != 0.0f ? __frcp_rn(s) : 0.0f;
     const float qmax = amax * ri * 1.0001f;
     const float cut = fmaxf(0.5f - qmax * 0x1p-18f, 0.0f);   // 0: every element takes the division
-    return {s, ri, cut * cut, off};
+    return {s, ri, cut, off};
 }
 
-// Codes of two elements of one group (byte 0 and byte 1 of the result), where round is
-// half to even of the correctly rounded fp32 quotient RN(x / s).  With ri = RN(1/s),
-// q = RN(x ri) is within |q| 2^-22 of RN(x / s), so both round to the same integer
-// unless q lies within that distance of a half-integer.  r = q - round(q) is exact; while
-// r^2 < cut2, |r| stays more than qmax 2^-20 from 1/2 (the rounding of r^2 and cut2 is
-// covered by the larger margin 2^-18, as qmax >= 1 in every group with a nonzero
-// element; an all-zero group has q = r = 0), so the fast result stands; an element
-// nearer a tie takes the IEEE division.
+// M = 1.5 2^23: RN(q + M + off) holds the integer nearest q + off in its low mantissa bits
+constexpr float kRoundMagic = 12582912.0f;
+
+// Codes of four elements, as the four bytes of a word.  For element i with
+// ri = RN(1/s) and moff = M + off (M = 1.5 2^23), t = RN(RN(x ri) + moff) lies in
+// [2^23, 2^24), so its low byte is the integer nearest RN(x ri) + off.  Away from a tie
+// (|r| < cut for r = RN(x ri) - (t - moff), exact) that is rint(RN(x / s)) + off, as
+// before; an element nearer a tie, or with a non-finite r, takes the IEEE
+// division.  The code is at least 0 (x >= the group's minimum, and rint is odd) and at
+// most L + 1 (s rounds to within 2^-24 of (max - min) / L), so the upper clamp alone
+// remains: a byte with bit n set is L + 1.
+struct QuadParams {
+    float4 ri, moff;   // per element
+    float cut;         // |r| < cut: the fast code stands (0: every element is divided)
+};
+
+// Codes of x.x .. x.w as the four bytes of a word; s4 / off4 (per element) serve the
+// elements that take the division.
 template <int N>
-__device__ __forceinline__ uint32_t code_pair(float x0, float x1, const CodeParams &p) {
+__device__ __forceinline__ uint32_t code_quad(const float4 &x, const QuadParams &p, const float4 &s4,
+                                              const int4 &off4) {
     constexpr int L = (1 << N) - 1;
-    const float2 q = mul_x2(make_float2(x0, x1), make_float2(p.ri, p.ri));
-    const float2 t = add_x2(q, make_float2(12582912.0f, 12582912.0f));      // 1.5 * 2^23
-    const float2 k = add_x2(t, make_float2(-12582912.0f, -12582912.0f));
-    const float2 r = fma_x2(k, make_float2(-1.0f, -1.0f), q);
-    const float2 r2 = mul_x2(r, r);
-    int i0 = __float_as_int(t.x) - 0x4B400000, i1 = __float_as_int(t.y) - 0x4B400000;
-    if (r2.x >= p.cut2) i0 = static_cast<int>(rintf(__fdiv_rn(x0, p.s)));
-    if (r2.y >= p.cut2) i1 = static_cast<int>(rintf(__fdiv_rn(x1, p.s)));
-    const int c0 = min(max(i0 + p.off, 0), L), c1 = min(max(i1 + p.off, 0), L);
-    return static_cast<uint32_t>(c0) | (static_cast<uint32_t>(c1) << 8);
+    const float2 q01 = mul_x2(make_float2(x.x, x.y), make_float2(p.ri.x, p.ri.y));
+    const float2 q23 = mul_x2(make_float2(x.z, x.w), make_float2(p.ri.z, p.ri.w));
+    const float2 t01 = add_x2(q01, make_float2(p.moff.x, p.moff.y));
+    const float2 t23 = add_x2(q23, make_float2(p.moff.z, p.moff.w));
+    const float2 r01 = add_x2(q01, sub_x2(make_float2(p.moff.x, p.moff.y), t01));   // moff - t: exact
+    const float2 r23 = add_x2(q23, sub_x2(make_float2(p.moff.z, p.moff.w), t23));
+    uint32_t w = __byte_perm(__byte_perm(__float_as_uint(t01.x), __float_as_uint(t01.y), 0x0040),
+                             __byte_perm(__float_as_uint(t23.x), __float_as_uint(t23.y), 0x0040), 0x5410);
+    const bool near = !(fabsf(r01.x) < p.cut) || !(fabsf(r01.y) < p.cut) || !(fabsf(r23.x) < p.cut) ||
+                      !(fabsf(r23.y) < p.cut);
+    if (near) {
+        const float xs[4] = {x.x, x.y, x.z, x.w}, ss[4] = {s4.x, s4.y, s4.z, s4.w};
+        const float rs[4] = {r01.x, r01.y, r23.x, r23.y};
+        const int os[4] = {off4.x, off4.y, off4.z, off4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if (!(fabsf(rs[e]) < p.cut)) {
+                const int c = static_cast<int>(rintf(__fdiv_rn(xs[e], ss[e]))) + os[e];
+                w = (w & ~(0xffu << (8 * e))) | (static_cast<uint32_t>(min(max(c, 0), L + 1)) << (8 * e));
+            }
+        }
+    }
+    constexpr uint32_t kOver = 0x01010101u << N;   // bit n of every byte: the code L + 1
+    if (w & kOver) {
+        const uint32_t over = (w & kOver) >> N;     // 1 in each byte to clamp
+        w -= over;                                  // L + 1 -> L
+    }
+    return w;
 }
 
 // Assemble the packed words of `ntiles` 16-token tiles from byte codes
@@ -160,6 +196,33 @@ __device__ void pack_tiles(const uint8_t *codes, int ntiles, uint32_t *dst) {
         }
         dst[wi] = word;
     }
+}
+
+// Two 16-bit elements (a 32-bit word, low half first) as floats.
+__device__ __forceinline__ float2 widen2(uint32_t v, bool bf16) {
+    if (bf16) return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+    return __half22float2(*reinterpret_cast<const __half2 *>(&v));
+}
+
+// Element-wise minimum and maximum (sym: maximum magnitude, returned in hi) of n packed
+// pairs p[0], p[stride], ...: exact in the 16-bit type.
+template <bool BF16>
+__device__ __forceinline__ void pair_minmax(const uint32_t *p, int stride, int n, bool sym, uint32_t &lo,
+                                            uint32_t &hi) {
+    using T2 = typename std::conditional<BF16, __nv_bfloat162, __half2>::type;
+    T2 l = *reinterpret_cast<const T2 *>(p), h = l;
+    if (sym) {
+        h = __habs2(h);
+        for (int i = 1; i < n; ++i) h = __hmax2(h, __habs2(*reinterpret_cast<const T2 *>(p + i * stride)));
+    } else {
+        for (int i = 1; i < n; ++i) {
+            const T2 v = *reinterpret_cast<const T2 *>(p + i * stride);
+            l = __hmin2(l, v);
+            h = __hmax2(h, v);
+        }
+    }
+    lo = *reinterpret_cast<const uint32_t *>(&l);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
 }
 
 // Copy the G rows of d 16-bit elements of one group into shared memory with 16-byte
@@ -275,27 +338,27 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
         __syncthreads();
     }
     {
-        const int parts = kQuantThreads / d;         // d divides 256
-        const int c = threadIdx.x % d;
-        const int part = threadIdx.x / d;
-        const int per = (G + parts - 1) / parts;
-        float mn = FLT_MAX, mx = -FLT_MAX;
-        for (int t = part * per; t < min(G, (part + 1) * per); ++t) {
-            const float x = widen(xs[t * d + c], a.bf16);
-            if (a.sym) {
-                mx = fmaxf(mx, fabsf(x));
-            } else {
-                mn = fminf(mn, x);
-                mx = fmaxf(mx, x);
-            }
-        }
-        red[threadIdx.x] = mn;
-        red[kQuantThreads + threadIdx.x] = mx;
+        // per-channel minimum and maximum (or largest magnitude) over the G tokens: thread
+        // (channel pair cp, part) scans its part with packed 16-bit min / max, which are
+        // exact; the parts meet in shared memory
+        constexpr int NP = D / 2;                    // channel pairs
+        constexpr int parts = kQuantThreads / NP;    // 4 (d = 128) or 8 (d = 64); G >= 16
+        const int cp = threadIdx.x % NP, part = threadIdx.x / NP;
+        const uint32_t *xw = reinterpret_cast<const uint32_t *>(xs);   // [G][NP] pairs
+        const int per = G / parts;
+        uint32_t lo, hi;
+        if (a.bf16) pair_minmax<true>(xw + (part * per) * NP + cp, NP, per, a.sym, lo, hi);
+        else pair_minmax<false>(xw + (part * per) * NP + cp, NP, per, a.sym, lo, hi);
+        uint32_t *redu = reinterpret_cast<uint32_t *>(red);
+        redu[threadIdx.x] = lo;
+        redu[kQuantThreads + threadIdx.x] = hi;
         __syncthreads();
         if (threadIdx.x < d) {
-            for (int p = 1; p < parts; ++p) {
-                mn = fminf(mn, red[p * d + c]);
-                mx = fmaxf(mx, red[kQuantThreads + p * d + c]);
+            const int c = threadIdx.x, pc = c >> 1, sh = 16 * (c & 1);
+            float mn = FLT_MAX, mx = -FLT_MAX;
+            for (int p = 0; p < parts; ++p) {
+                mn = fminf(mn, widen(static_cast<uint16_t>(redu[p * NP + pc] >> sh), a.bf16));
+                mx = fmaxf(mx, widen(static_cast<uint16_t>(redu[kQuantThreads + p * NP + pc] >> sh), a.bf16));
             }
             float s;
             int z;
@@ -314,17 +377,24 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
             ch_s[c] = s;
             ch_z[c] = z;
             ch_r[c] = cp.ri;
-            ch_c[c] = cp.cut2;
+            ch_c[c] = cp.cut;
         }
         __syncthreads();
-        {   // d divides the block size: each thread keeps one channel, two rows at a time
-            constexpr int rstep = kQuantThreads / d;
-            const int c2 = threadIdx.x % d;
-            const CodeParams cp{ch_s[c2], ch_r[c2], ch_c[c2], ch_z[c2]};
-            for (int t = threadIdx.x / d; t < G; t += 2 * rstep) {
-                const uint32_t cc = code_pair<N>(widen(xs[t * d + c2], a.bf16), widen(xs[(t + rstep) * d + c2], a.bf16), cp);
-                codes[t * d + c2] = static_cast<uint8_t>(cc & 0xffu);
-                codes[(t + rstep) * d + c2] = static_cast<uint8_t>(cc >> 8);
+        {   // codes: thread (cp, part) takes channels 2 cp, 2 cp + 1 of rows part, part + parts, ...,
+            // two rows at a time (G / parts is even)
+            QuadParams qp;
+            const float r0 = ch_r[2 * cp], r1 = ch_r[2 * cp + 1];
+            const int z0 = ch_z[2 * cp], z1 = ch_z[2 * cp + 1];
+            qp.ri = make_float4(r0, r1, r0, r1);
+            qp.moff = make_float4(kRoundMagic + z0, kRoundMagic + z1, kRoundMagic + z0, kRoundMagic + z1);
+            qp.cut = fminf(ch_c[2 * cp], ch_c[2 * cp + 1]);
+            const float4 s4 = make_float4(ch_s[2 * cp], ch_s[2 * cp + 1], ch_s[2 * cp], ch_s[2 * cp + 1]);
+            const int4 o4 = make_int4(z0, z1, z0, z1);
+            for (int t = part; t < G; t += 2 * parts) {
+                const float2 x0 = widen2(xw[t * NP + cp], a.bf16), x1 = widen2(xw[(t + parts) * NP + cp], a.bf16);
+                const uint32_t w = code_quad<N>(make_float4(x0.x, x0.y, x1.x, x1.y), qp, s4, o4);
+                *reinterpret_cast<uint16_t *>(codes + t * d + 2 * cp) = static_cast<uint16_t>(w & 0xffffu);
+                *reinterpret_cast<uint16_t *>(codes + (t + parts) * d + 2 * cp) = static_cast<uint16_t>(w >> 16);
             }
         }
         __syncthreads();
@@ -396,13 +466,17 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
             }
             const CodeParams cp = code_params(s, a.sym ? (1 << (bits - 1)) : z,
                                               a.sym ? mx : fmaxf(fabsf(mn), fabsf(mx)));
-            uint32_t cw[per_lane / 4] = {};
-#pragma unroll
-            for (int e = 0; e < per_lane; e += 2)
-                cw[e / 4] |= code_pair<N>(x[e], x[e + 1], cp) << (8 * (e % 4));
+            QuadParams qp;
+            qp.ri = make_float4(cp.ri, cp.ri, cp.ri, cp.ri);
+            const float mo = kRoundMagic + static_cast<float>(cp.off);
+            qp.moff = make_float4(mo, mo, mo, mo);
+            qp.cut = cp.cut;
+            const float4 s4 = make_float4(cp.s, cp.s, cp.s, cp.s);
+            const int4 o4 = make_int4(cp.off, cp.off, cp.off, cp.off);
 #pragma unroll
             for (int k = 0; k < per_lane / 4; ++k)
-                reinterpret_cast<uint32_t *>(codes + t * d + hl * per_lane)[k] = cw[k];
+                reinterpret_cast<uint32_t *>(codes + t * d + hl * per_lane)[k] =
+                    code_quad<N>(make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]), qp, s4, o4);
         }
         __syncthreads();
         pack_tiles<D, N, true>(codes, G / 16,
