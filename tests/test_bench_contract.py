@@ -58,3 +58,28 @@ def test_cpu_baseline_reports_model_cores_and_one_core():
     assert r["one_core"]["cores"] == 1 and r["one_core"]["value"] > 0
     import oracle
     assert oracle.num_threads() == r["cores"]          # the thread count is restored
+
+
+def test_decode_kernel_names_follow_the_library_choice():
+    gqa, llama = wl.WORKLOADS["gqa8b"], wl.WORKLOADS["llama7b"]
+    assert bench.decode_kernel_name(gqa) == "decode_mma_kernel"
+    assert bench.decode_kernel_name(llama) == "decode_mma_kernel"
+    assert bench.decode_kernel_name(gqa, paged=True) == "decode_tc_kernel"
+    assert bench.decode_kernel_name(gqa, key_outliers=1) == "decode_tc_kernel"
+    assert bench.decode_kernel_name(gqa.replace(Hq=64)) == "decode_split_kernel"    # 8 query heads per kv head
+    for name, (value, kernel) in bench.DECODE_KERNELS.items():
+        assert bench.decode_kernel_name(gqa, forced=name) == (kernel or "decode_mma_kernel")
+    assert [v for v, _ in bench.DECODE_KERNELS.values()] == [0, 1, 2, 3]   # kvq_set_decode_kernel's values
+
+
+def test_profile_traffic_is_read_only_for_the_current_source(tmp_path, monkeypatch):
+    w = wl.WORKLOADS["gqa8b"]
+    h = bench.kernel_source_hash("decode_mma_kernel")
+    (tmp_path / "profiles").mkdir()
+    f = tmp_path / "profiles" / "decode_mma_kernel_gqa8b.md"
+    f.write_text(f"kernel source sha256[:16]: {h}\ndram bytes per launch: 1234\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda k: h)
+    assert bench.ncu_traffic(w) == 1234
+    f.write_text("kernel source sha256[:16]: 0000000000000000\ndram bytes per launch: 1234\n")
+    assert bench.ncu_traffic(w) is None
