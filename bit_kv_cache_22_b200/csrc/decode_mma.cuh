@@ -426,6 +426,9 @@ __global__ void __launch_bounds__(kDecodeThreads, D / GV >= 8 ? 3 : 4) decode_mm
             z23 = make_float2(static_cast<float>(static_cast<int16_t>(zz.y & 0xffffu)),
                               static_cast<float>(static_cast<int16_t>(zz.y >> 16)));
         }
+        // the bias scale 2^(-64 + 2nc) (exact) folded into the zeros: bp is the scaled partial
+        z01 = mul2(z01, make_float2(pbias_f, pbias_f));
+        z23 = mul2(z23, make_float2(pbias_f, pbias_f));
         float bp[HPL];
         __syncwarp();   // the previous group's fragments have been read
 #pragma unroll
@@ -455,8 +458,6 @@ __global__ void __launch_bounds__(kDecodeThreads, D / GV >= 8 ? 3 : 4) decode_mm
             kb[2 * i][0] = v.x; kb[2 * i][1] = v.y; kb[2 * i + 1][0] = v.z; kb[2 * i + 1][1] = v.w;
         }
         // bias of each head: the producers' partials summed over the QUADS lanes of its quads
-#pragma unroll
-        for (int i = 0; i < HPL; ++i) bp[i] *= pbias_f;
         const float bsum = transpose_reduce<HPL, QUADS>(bp, lane);
         // head t4 mod HG: in the lane group of heads (h / HPL), at lane offset (h mod HPL) QUADS / HPL
         const int hh = t4 % HG;
@@ -552,19 +553,24 @@ __global__ void __launch_bounds__(kDecodeThreads, D / GV >= 8 ? 3 : 4) decode_mm
                 }
                 constexpr float f0 = static_cast<float>(1ull << 62) * 128.0f;                       // 2^69
                 constexpr float f1 = static_cast<float>(1ull << 62) * static_cast<float>(128 >> N); // 2^(69 - n)
-                lg[u][0] = fmaf((acc[0][0] + acc[1][0]) + (acc[0][1] + acc[1][1]), f0, -kbias);
-                lg[u][1] = fmaf((acc[0][2] + acc[1][2]) + (acc[0][3] + acc[1][3]), f1, -kbias);
+                // rows g8 (.x) and g8 + 8 (.y): (chain 0 + chain 1), column 2 t4 plus column 2 t4 + 1
+                const float2 c0 = add2(make_float2(acc[0][0], acc[0][2]), make_float2(acc[1][0], acc[1][2]));
+                const float2 c1 = add2(make_float2(acc[0][1], acc[0][3]), make_float2(acc[1][1], acc[1][3]));
+                const float2 cs = add2(c0, c1);
+                lg[u][0] = fmaf(cs.x, f0, -kbias);
+                lg[u][1] = fmaf(cs.y, f1, -kbias);
             }
 
             // ---- online softmax of head t4 mod HG: the item's maximum, rescale, p ----
             {
                 float mx = fmaxf(fmaxf(lg[0][0], lg[0][1]), fmaxf(lg[1][0], lg[1][1]));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                // lazily: only when the item's maximum passes the running one by more than
-                // kLazyRescale (p may reach 2^kLazyRescale meanwhile), so rescales stay rare
+                // lazily: only when a logit of the item passes the running maximum by more than
+                // kLazyRescale (p may reach 2^kLazyRescale meanwhile), so rescales stay rare;
+                // the lanes of a head (same t4) agree on m_own, so any lane's logit decides
                 if (__any_sync(0xffffffffu, mx > m_own + kLazyRescale)) {
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));   // the item's maximum of the head
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
                     const float mn = fmaxf(m_own, mx);
                     const float alpha = fast_exp2(m_own - mn);
                     m_own = mn;
@@ -580,7 +586,7 @@ __global__ void __launch_bounds__(kDecodeThreads, D / GV >= 8 ? 3 : 4) decode_mm
             }
             // p 2^80 = 2^(logit - (m - 80)): the value MMA's scale comes with the exponential
             const float m80 = m_own - static_cast<float>(kValScaleLog2);
-            if (t4 < HG) {
+            if (HG == 4 || t4 < HG) {
 #pragma unroll
                 for (int u = 0; u < kMmaItemTiles; ++u) {
                     const float p0 = fast_exp2(lg[u][0] - m80), p1 = fast_exp2(lg[u][1] - m80);
