@@ -225,6 +225,19 @@ __device__ __forceinline__ void pair_minmax(const uint32_t *p, int stride, int n
     hi = *reinterpret_cast<const uint32_t *>(&h);
 }
 
+// n consecutive 32-bit words from shared memory in one vector load (n = 2 or 4)
+template <int n>
+__device__ __forceinline__ void load_words(const uint32_t *p, uint32_t (&w)[n]) {
+    static_assert(n == 2 || n == 4, "words");
+    if constexpr (n == 4) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(p);
+        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+    } else {
+        const uint2 v = *reinterpret_cast<const uint2 *>(p);
+        w[0] = v.x; w[1] = v.y;
+    }
+}
+
 // Copy the G rows of d 16-bit elements of one group into shared memory with 16-byte
 // loads: rows tok0 .. tok0+G-1 of `slice`, or rows rows[0 .. G-1] when rows is non-NULL.
 // Each thread issues up to kLoadBatch loads before it stores any, so a group arrives in
@@ -261,7 +274,9 @@ __device__ void load_group(const uint16_t *slice, int64_t tok0, const int32_t *r
     }
 }
 
-template <int D, int N>
+// BATCH: the value parameters batched per warp (groups of 64 tokens or more, four or more
+// token pairs per warp); else computed per token pair
+template <int D, int N, bool BATCH>
 __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const QuantizeArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
     constexpr int d = D, bits = N;
@@ -273,6 +288,8 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
     int *ch_z = reinterpret_cast<int *>(ch_s + d);                           // [d]
     float *ch_r = reinterpret_cast<float *>(ch_z + d);                       // [d] 1/s
     float *ch_c = ch_r + d;                                                  // [d] near-tie bound
+    // value groups: [G][d / Gv] entries of 4 floats: (min, max), then (RN(1/s), M + off, cut, s)
+    float4 *vg = reinterpret_cast<float4 *>(ch_c + d);
 
     const int64_t grp = blockIdx.x;
     const int64_t bh = blockIdx.y;                 // input slice
@@ -407,76 +424,147 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
     load_group(a.xv + bh * a.in_bh_stride, in_tok, rows, a.in_rows_limit, a.status, xs, G, d);
     __syncthreads();
     {
-        // one token per half-warp (two per warp): the per-token work (segment reductions,
-        // the IEEE divisions of the group parameters) is shared by the two halves
+        // one token per half-warp (two per warp).  With four or more token pairs per warp, a warp
+        // first takes the minimum and maximum of every value group of its tokens (segment
+        // reductions over the lanes of a group), then computes the parameters (the IEEE
+        // divisions) with one lane per (token, group), so that one pass of that code serves up
+        // to 32 groups, then the codes.  With fewer, each token pair's lanes compute their
+        // groups' parameters themselves.
         constexpr int per_lane = d / 16;             // contiguous channels per lane: 8 or 4
-        const int warp = threadIdx.x >> 5, half = (threadIdx.x >> 4) & 1, hl = threadIdx.x & 15;
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        const int half = (threadIdx.x >> 4) & 1, hl = threadIdx.x & 15;
         const int seg = a.Gv / per_lane;             // lanes per value group (power of 2, <= 16)
         const int ngv = d / a.Gv;
-        for (int tp = warp; tp < G / 2; tp += kQuantThreads / 32) {
-            const int t = 2 * tp + half;
-            float x[per_lane];
-            float mn = FLT_MAX, mx = -FLT_MAX;
-            uint16_t xb[per_lane];
-            if constexpr (per_lane == 8) {
-                const uint4 v = *reinterpret_cast<const uint4 *>(xs + t * d + hl * per_lane);
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    xb[2 * k] = static_cast<uint16_t>(w[k] & 0xffffu);
-                    xb[2 * k + 1] = static_cast<uint16_t>(w[k] >> 16);
+        const int j = hl / seg;                      // this lane's group in its token
+        constexpr int kWarps = kQuantThreads / 32;
+        if constexpr (BATCH) {       // four or more token pairs per warp: parameters batched
+            for (int tp = warp; tp < G / 2; tp += kWarps) {
+                const int t = 2 * tp + half;
+                uint32_t w[per_lane / 2];
+                load_words<per_lane / 2>(reinterpret_cast<const uint32_t *>(xs + t * d + hl * per_lane), w);
+                uint32_t lo, hi;
+                if (a.bf16) pair_minmax<true>(w, 1, per_lane / 2, a.sym, lo, hi);
+                else pair_minmax<false>(w, 1, per_lane / 2, a.sym, lo, hi);
+                const float2 l2 = widen2(lo, a.bf16), h2 = widen2(hi, a.bf16);
+                float mn = fminf(l2.x, l2.y), mx = fmaxf(h2.x, h2.y);
+                for (int off = seg >> 1; off > 0; off >>= 1) {
+                    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
                 }
-            } else {
-                const uint2 v = *reinterpret_cast<const uint2 *>(xs + t * d + hl * per_lane);
-                xb[0] = static_cast<uint16_t>(v.x & 0xffffu);
-                xb[1] = static_cast<uint16_t>(v.x >> 16);
-                xb[2] = static_cast<uint16_t>(v.y & 0xffffu);
-                xb[3] = static_cast<uint16_t>(v.y >> 16);
+                if (hl % seg == 0) vg[t * ngv + j] = make_float4(mn, mx, 0.f, 0.f);
             }
-#pragma unroll
-            for (int e = 0; e < per_lane; ++e) {
-                x[e] = widen(xb[e], a.bf16);
+            __syncwarp();
+            // the warp's (token, group) pairs: token pairs tp = warp + kWarps i, both tokens, every group
+            const int n_pairs = ((G / 2 - warp + kWarps - 1) / kWarps) * 2 * ngv;
+            for (int q = lane; q < n_pairs; q += 32) {
+                const int i = q / (2 * ngv), hq = (q / ngv) % 2, jq = q % ngv;
+                const int t = 2 * (warp + kWarps * i) + hq;
+                const float4 e = vg[t * ngv + jq];
+                const float mn = e.x, mx = e.y;
+                float s;
+                int z;
                 if (a.sym) {
-                    mx = fmaxf(mx, fabsf(x[e]));
+                    s = sym_scale(mx, bits);
+                    z = 0;
                 } else {
-                    mn = fminf(mn, x[e]);
-                    mx = fmaxf(mx, x[e]);
+                    const GroupParams gp = asym_params(mn, mx, bits);
+                    s = gp.s;
+                    z = gp.z;
                 }
-            }
-            for (int off = seg >> 1; off > 0; off >>= 1) {
-                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-            }
-            float s;
-            int z;
-            if (a.sym) {
-                s = sym_scale(mx, bits);
-                z = 0;
-            } else {
-                const GroupParams gp = asym_params(mn, mx, bits);
-                s = gp.s;
-                z = gp.z;
-            }
-            const int j = hl / seg;
-            if (hl % seg == 0) {
-                const int64_t mi = (slice * cap + out_tok + t) * ngv + j;
+                const int64_t mi = (slice * cap + out_tok + t) * ngv + jq;
                 a.vs[mi] = s;
                 if (!a.sym) a.vz[mi] = static_cast<int16_t>(z);
                 if (s > kMaxServedScale) atomicOr(a.status, 4u);
+                const CodeParams cp = code_params(s, a.sym ? (1 << (bits - 1)) : z,
+                                                  a.sym ? mx : fmaxf(fabsf(mn), fabsf(mx)));
+                vg[t * ngv + jq] = make_float4(cp.ri, kRoundMagic + static_cast<float>(cp.off), cp.cut, cp.s);
             }
-            const CodeParams cp = code_params(s, a.sym ? (1 << (bits - 1)) : z,
-                                              a.sym ? mx : fmaxf(fabsf(mn), fabsf(mx)));
-            QuadParams qp;
-            qp.ri = make_float4(cp.ri, cp.ri, cp.ri, cp.ri);
-            const float mo = kRoundMagic + static_cast<float>(cp.off);
-            qp.moff = make_float4(mo, mo, mo, mo);
-            qp.cut = cp.cut;
-            const float4 s4 = make_float4(cp.s, cp.s, cp.s, cp.s);
-            const int4 o4 = make_int4(cp.off, cp.off, cp.off, cp.off);
-#pragma unroll
-            for (int k = 0; k < per_lane / 4; ++k)
-                reinterpret_cast<uint32_t *>(codes + t * d + hl * per_lane)[k] =
-                    code_quad<N>(make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]), qp, s4, o4);
+            __syncwarp();
+            for (int tp = warp; tp < G / 2; tp += kWarps) {
+                const int t = 2 * tp + half;
+                uint32_t w[per_lane / 2];
+                load_words<per_lane / 2>(reinterpret_cast<const uint32_t *>(xs + t * d + hl * per_lane), w);
+                const float4 e = vg[t * ngv + j];
+                QuadParams qp;
+                qp.ri = make_float4(e.x, e.x, e.x, e.x);
+                qp.moff = make_float4(e.y, e.y, e.y, e.y);
+                qp.cut = e.z;
+                const float4 s4 = make_float4(e.w, e.w, e.w, e.w);
+                const int off = static_cast<int>(e.y - kRoundMagic);
+                const int4 o4 = make_int4(off, off, off, off);
+    #pragma unroll
+                for (int k = 0; k < per_lane / 4; ++k) {
+                    const float2 x0 = widen2(w[2 * k], a.bf16), x1 = widen2(w[2 * k + 1], a.bf16);
+                    reinterpret_cast<uint32_t *>(codes + t * d + hl * per_lane)[k] =
+                        code_quad<N>(make_float4(x0.x, x0.y, x1.x, x1.y), qp, s4, o4);
+                }
+            }
+        } else {                     // short groups: parameters per token pair, as they come
+            for (int tp = warp; tp < G / 2; tp += kQuantThreads / 32) {
+                const int t = 2 * tp + half;
+                float x[per_lane];
+                float mn = FLT_MAX, mx = -FLT_MAX;
+                uint16_t xb[per_lane];
+                if constexpr (per_lane == 8) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(xs + t * d + hl * per_lane);
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    #pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        xb[2 * k] = static_cast<uint16_t>(w[k] & 0xffffu);
+                        xb[2 * k + 1] = static_cast<uint16_t>(w[k] >> 16);
+                    }
+                } else {
+                    const uint2 v = *reinterpret_cast<const uint2 *>(xs + t * d + hl * per_lane);
+                    xb[0] = static_cast<uint16_t>(v.x & 0xffffu);
+                    xb[1] = static_cast<uint16_t>(v.x >> 16);
+                    xb[2] = static_cast<uint16_t>(v.y & 0xffffu);
+                    xb[3] = static_cast<uint16_t>(v.y >> 16);
+                }
+    #pragma unroll
+                for (int e = 0; e < per_lane; ++e) {
+                    x[e] = widen(xb[e], a.bf16);
+                    if (a.sym) {
+                        mx = fmaxf(mx, fabsf(x[e]));
+                    } else {
+                        mn = fminf(mn, x[e]);
+                        mx = fmaxf(mx, x[e]);
+                    }
+                }
+                for (int off = seg >> 1; off > 0; off >>= 1) {
+                    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                }
+                float s;
+                int z;
+                if (a.sym) {
+                    s = sym_scale(mx, bits);
+                    z = 0;
+                } else {
+                    const GroupParams gp = asym_params(mn, mx, bits);
+                    s = gp.s;
+                    z = gp.z;
+                }
+                const int j = hl / seg;
+                if (hl % seg == 0) {
+                    const int64_t mi = (slice * cap + out_tok + t) * ngv + j;
+                    a.vs[mi] = s;
+                    if (!a.sym) a.vz[mi] = static_cast<int16_t>(z);
+                    if (s > kMaxServedScale) atomicOr(a.status, 4u);
+                }
+                const CodeParams cp = code_params(s, a.sym ? (1 << (bits - 1)) : z,
+                                                  a.sym ? mx : fmaxf(fabsf(mn), fabsf(mx)));
+                QuadParams qp;
+                qp.ri = make_float4(cp.ri, cp.ri, cp.ri, cp.ri);
+                const float mo = kRoundMagic + static_cast<float>(cp.off);
+                qp.moff = make_float4(mo, mo, mo, mo);
+                qp.cut = cp.cut;
+                const float4 s4 = make_float4(cp.s, cp.s, cp.s, cp.s);
+                const int4 o4 = make_int4(cp.off, cp.off, cp.off, cp.off);
+    #pragma unroll
+                for (int k = 0; k < per_lane / 4; ++k)
+                    reinterpret_cast<uint32_t *>(codes + t * d + hl * per_lane)[k] =
+                        code_quad<N>(make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]), qp, s4, o4);
+            }
         }
         __syncthreads();
         pack_tiles<D, N, true>(codes, G / 16,
@@ -602,29 +690,37 @@ __global__ void paged_residual_kernel(const uint16_t *xk, const uint16_t *xv, in
 
 }  // namespace
 
-size_t quantize_smem_bytes(int d, int G) {
+size_t quantize_smem_bytes(int d, int G, int Gv) {
     return static_cast<size_t>(G) * d * 3 + 2 * kQuantThreads * sizeof(float) +
-           static_cast<size_t>(d) * 16;
+           static_cast<size_t>(d) * 16 + static_cast<size_t>(G) * (d / Gv) * 16;
+}
+
+using QuantizeKernel = void (*)(const QuantizeArgs);
+template <int D, int N>
+QuantizeKernel quantize_instance(bool batch) {
+    return batch ? quantize_pack_kernel<D, N, true> : quantize_pack_kernel<D, N, false>;
 }
 
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s) {
     if (a.n_groups == 0 || a.BH == 0) return cudaSuccess;
-    const size_t smem = quantize_smem_bytes(a.d, a.G);
+    const size_t smem = quantize_smem_bytes(a.d, a.G, a.Gv);
     void (*kernel)(const QuantizeArgs) = nullptr;
     int variant = -1;
-    if (a.d == 64 && a.bits == 2) kernel = quantize_pack_kernel<64, 2>, variant = 0;
-    else if (a.d == 64 && a.bits == 4) kernel = quantize_pack_kernel<64, 4>, variant = 1;
-    else if (a.d == 128 && a.bits == 2) kernel = quantize_pack_kernel<128, 2>, variant = 2;
-    else if (a.d == 128 && a.bits == 4) kernel = quantize_pack_kernel<128, 4>, variant = 3;
+    const bool batch = a.G / 2 >= 4 * (kQuantThreads / 32);
+    if (a.d == 64 && a.bits == 2) kernel = quantize_instance<64, 2>(batch), variant = 0;
+    else if (a.d == 64 && a.bits == 4) kernel = quantize_instance<64, 4>(batch), variant = 1;
+    else if (a.d == 128 && a.bits == 2) kernel = quantize_instance<128, 2>(batch), variant = 2;
+    else if (a.d == 128 && a.bits == 4) kernel = quantize_instance<128, 4>(batch), variant = 3;
     if (!kernel) return cudaErrorInvalidValue;
+    variant = 2 * variant + (batch ? 1 : 0);
     // opt in to the largest dynamic shared memory any configuration needs, once per device and variant
-    static bool configured[64][4] = {};
+    static bool configured[64][8] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 64 || !configured[dev][variant]) {
         e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(quantize_smem_bytes(256, 128)));
+                                 static_cast<int>(quantize_smem_bytes(256, 128, 16)));
         if (e != cudaSuccess) return e;
         if (dev < 64) configured[dev][variant] = true;
     }
