@@ -149,10 +149,10 @@ namespace {
 // path with one query head per kv head, where they are dealt to the warps of the
 // quantized splits.  A CTA's time is modelled as a fixed start/finish cost of
 // kCtaFixedTiles tiles plus the tiles its busiest warp streams (an empty split
-// costs kEmptyCtaTiles); the kernel's time as the larger of (the waves of quantized
-// CTAs over the GPU's resident slots x one quantized CTA) and (all CTA time spread
-// evenly over the slots, plus one residual CTA); when every CTA is resident at once it
-// is the longest CTA's.  The split count with the lowest modelled time wins (ties:
+// costs kEmptyCtaTiles); the kernel's time as the largest of (the waves of quantized
+// CTAs over the GPU's resident slots x one quantized CTA), (all CTA time spread evenly
+// over the slots, plus one residual CTA) and the longest chain of CTAs on one slot; when
+// every CTA is resident at once it is the longest CTA's.  The split count with the lowest modelled time wins (ties:
 // fewer splits).
 constexpr double kCtaFixedTiles = 6.0;
 constexpr double kEmptyCtaTiles = 1.0;
@@ -228,8 +228,20 @@ void plan_splits_for(const kvq_cache *h, const PlanInput &in, int *n_qsplits, in
                 const double n_res = static_cast<double>(units * n_rs);
                 const double t_spread =
                     (nq * c_q + n_empty * kEmptyCtaTiles + n_res * c_res) / slots + (n_rs ? c_res : 0.0);
+                // the longest chain of CTAs on one slot: with the quantized CTAs resident in one
+                // wave, the residual CTAs run in turns on the slots left beside them; else
+                // they start after the quantized ones
                 double t_crit = c_q;
-                if (n_rs) t_crit = (nq + n_res > slots) ? c_q + c_res : (c_res > c_q ? c_res : c_q);
+                if (n_rs) {
+                    if (nq + n_res <= slots) {
+                        t_crit = c_res > c_q ? c_res : c_q;
+                    } else if (nq < slots) {
+                        const double turns = std::ceil(n_res / (slots - nq));
+                        t_crit = c_res * turns > c_q ? c_res * turns : c_q;
+                    } else {
+                        t_crit = c_q + c_res;
+                    }
+                }
                 double cost = t_waves > t_spread ? t_waves : t_spread;
                 cost = cost > t_crit ? cost : t_crit;
                 // every CTA resident at once (one wave): the longest CTA sets the time
