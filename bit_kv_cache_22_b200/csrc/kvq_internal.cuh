@@ -70,6 +70,7 @@ struct QuantizeArgs {
     // (channel << 16) | element bits to k_out [slice][cap][n_out], largest first
     uint32_t *k_out;
     int n_out;
+    int gpc;                     // key groups per CTA (1, or 2 for short groups: set by the launch)
 };
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s);
 

@@ -277,10 +277,11 @@ __device__ void load_group(const uint16_t *slice, int64_t tok0, const int32_t *r
 // BATCH: the value parameters batched per warp (groups of 64 tokens or more, four or more
 // token pairs per warp); else computed per token pair
 template <int D, int N, bool BATCH>
-__global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const QuantizeArgs a) {
+__global__ void __launch_bounds__(kQuantThreads, 4) quantize_pack_kernel(const QuantizeArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
     constexpr int d = D, bits = N;
-    const int G = a.G;
+    const int GK = a.G;                            // key group
+    const int G = a.gpc * GK;                      // tokens of the CTA: gpc key groups
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem);                       // [G][d]
     uint8_t *codes = smem + static_cast<size_t>(G) * d * 2;                  // [G][d]
     float *red = reinterpret_cast<float *>(codes + static_cast<size_t>(G) * d);  // 2*256
@@ -300,7 +301,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
         // paged pool: the group's page of its sequence (groups never straddle pages)
         const int64_t b = a.seq0 + bh / a.Hkv;
         if (a.seq_len) {                           // flush: only sequences whose residual just filled
-            const int64_t len = a.seq_len[b], R = a.n_groups * G;
+            const int64_t len = a.seq_len[b], R = a.n_groups * GK;
             if (len <= 0 || len % R != 0) return;
             out_tok = len - R + grp * G;
         }
@@ -315,7 +316,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
     }
     const int TW = tile_words(d, bits);
     const int64_t words_per_slice = cap / 16 * TW;
-    const int64_t groups_cap = cap / G;
+    const int64_t groups_cap = cap / GK;
 
     // ------------------------------ keys ------------------------------
     const int32_t *rows = a.in_rows ? a.in_rows + grp * G : nullptr;
@@ -354,15 +355,16 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
         }
         __syncthreads();
     }
-    {
-        // per-channel minimum and maximum (or largest magnitude) over the G tokens: thread
+    for (int kg = 0; kg < a.gpc; ++kg) {
+        // key group kg of the CTA (rows kg GK .. kg GK + GK - 1)
+        // per-channel minimum and maximum (or largest magnitude) over the GK tokens: thread
         // (channel pair cp, part) scans its part with packed 16-bit min / max, which are
         // exact; the parts meet in shared memory
         constexpr int NP = D / 2;                    // channel pairs
         constexpr int parts = kQuantThreads / NP;    // 4 (d = 128) or 8 (d = 64); G >= 16
         const int cp = threadIdx.x % NP, part = threadIdx.x / NP;
-        const uint32_t *xw = reinterpret_cast<const uint32_t *>(xs);   // [G][NP] pairs
-        const int per = G / parts;
+        const uint32_t *xw = reinterpret_cast<const uint32_t *>(xs) + kg * GK * NP;   // [GK][NP] pairs
+        const int per = GK / parts;
         uint32_t lo, hi;
         if (a.bf16) pair_minmax<true>(xw + (part * per) * NP + cp, NP, per, a.sym, lo, hi);
         else pair_minmax<false>(xw + (part * per) * NP + cp, NP, per, a.sym, lo, hi);
@@ -386,9 +388,9 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
                 const GroupParams gp = asym_params(mn, mx, bits);
                 s = gp.s;
                 z = gp.z;
-                a.kz[(slice * groups_cap + out_tok / G) * d + c] = static_cast<int16_t>(z);
+                a.kz[(slice * groups_cap + out_tok / GK + kg) * d + c] = static_cast<int16_t>(z);
             }
-            a.ks[(slice * groups_cap + out_tok / G) * d + c] = s;
+            a.ks[(slice * groups_cap + out_tok / GK + kg) * d + c] = s;
             if (s > kMaxServedScale) atomicOr(a.status, 4u);
             const CodeParams cp = code_params(s, z, a.sym ? mx : fmaxf(fabsf(mn), fabsf(mx)));
             ch_s[c] = s;
@@ -398,7 +400,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
         }
         __syncthreads();
         {   // codes: thread (cp, part) takes channels 2 cp, 2 cp + 1 of rows part, part + parts, ...,
-            // two rows at a time (G / parts is even)
+            // two rows at a time (GK / parts is even)
             QuadParams qp;
             const float r0 = ch_r[2 * cp], r1 = ch_r[2 * cp + 1];
             const int z0 = ch_z[2 * cp], z1 = ch_z[2 * cp + 1];
@@ -407,18 +409,18 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_pack_kernel(const Quan
             qp.cut = fminf(ch_c[2 * cp], ch_c[2 * cp + 1]);
             const float4 s4 = make_float4(ch_s[2 * cp], ch_s[2 * cp + 1], ch_s[2 * cp], ch_s[2 * cp + 1]);
             const int4 o4 = make_int4(z0, z1, z0, z1);
-            for (int t = part; t < G; t += 2 * parts) {
+            uint8_t *kcodes = codes + kg * GK * d;
+            for (int t = part; t < GK; t += 2 * parts) {
                 const float2 x0 = widen2(xw[t * NP + cp], a.bf16), x1 = widen2(xw[(t + parts) * NP + cp], a.bf16);
                 const uint32_t w = code_quad<N>(make_float4(x0.x, x0.y, x1.x, x1.y), qp, s4, o4);
-                *reinterpret_cast<uint16_t *>(codes + t * d + 2 * cp) = static_cast<uint16_t>(w & 0xffffu);
-                *reinterpret_cast<uint16_t *>(codes + (t + parts) * d + 2 * cp) = static_cast<uint16_t>(w >> 16);
+                *reinterpret_cast<uint16_t *>(kcodes + t * d + 2 * cp) = static_cast<uint16_t>(w & 0xffffu);
+                *reinterpret_cast<uint16_t *>(kcodes + (t + parts) * d + 2 * cp) = static_cast<uint16_t>(w >> 16);
             }
         }
         __syncthreads();
-        pack_tiles<D, N, false>(codes, G / 16,
-                   a.kc + slice * words_per_slice + (out_tok / 16) * TW);
-        __syncthreads();
     }
+    pack_tiles<D, N, false>(codes, G / 16, a.kc + slice * words_per_slice + (out_tok / 16) * TW);
+    __syncthreads();
 
     // ------------------------------ values ----------------------------
     load_group(a.xv + bh * a.in_bh_stride, in_tok, rows, a.in_rows_limit, a.status, xs, G, d);
@@ -703,10 +705,15 @@ QuantizeKernel quantize_instance(bool batch) {
 
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s) {
     if (a.n_groups == 0 || a.BH == 0) return cudaSuccess;
-    const size_t smem = quantize_smem_bytes(a.d, a.G, a.Gv);
+    // short key groups of a contiguous cache go two to a CTA, so a CTA streams 64 tokens and
+    // the value parameters are batched (paged pools and row lists keep one group per CTA)
+    QuantizeArgs b = a;
+    b.gpc = (a.G / 2 < 4 * (kQuantThreads / 32) && a.n_groups % 2 == 0 && !a.page_table && !a.in_rows) ? 2 : 1;
+    const int tokens = b.gpc * a.G;
+    const size_t smem = quantize_smem_bytes(a.d, tokens, a.Gv);
     void (*kernel)(const QuantizeArgs) = nullptr;
     int variant = -1;
-    const bool batch = a.G / 2 >= 4 * (kQuantThreads / 32);
+    const bool batch = tokens / 2 >= 4 * (kQuantThreads / 32);
     if (a.d == 64 && a.bits == 2) kernel = quantize_instance<64, 2>(batch), variant = 0;
     else if (a.d == 64 && a.bits == 4) kernel = quantize_instance<64, 4>(batch), variant = 1;
     else if (a.d == 128 && a.bits == 2) kernel = quantize_instance<128, 2>(batch), variant = 2;
@@ -724,8 +731,8 @@ cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         if (dev < 64) configured[dev][variant] = true;
     }
-    dim3 grid(static_cast<unsigned>(a.n_groups), static_cast<unsigned>(a.BH));
-    kernel<<<grid, kQuantThreads, smem, s>>>(a);
+    dim3 grid(static_cast<unsigned>(a.n_groups / b.gpc), static_cast<unsigned>(a.BH));
+    kernel<<<grid, kQuantThreads, smem, s>>>(b);
     count_launches(1);
     return cudaGetLastError();
 }
