@@ -152,9 +152,12 @@ namespace {
 // costs kEmptyCtaTiles); the kernel's time as the largest of (the waves of quantized
 // CTAs over the GPU's resident slots x one quantized CTA), (all CTA time spread evenly
 // over the slots, plus one residual CTA) and the longest chain of CTAs on one slot; when
-// every CTA is resident at once it is the longest CTA's.  The split count with the lowest modelled time wins (ties:
-// fewer splits).
+// every CTA is resident at once it is the longest CTA's.  The split count with the
+// lowest modelled time wins (ties: fewer splits).
 constexpr double kCtaFixedTiles = 6.0;
+// a residual CTA starts and ends cheaper (no copy pipeline; measured: more, shorter residual
+// CTAs beside a one-wave quantized grid pay on the bf16-MMA kernel)
+constexpr double kResCtaFixedTiles = 2.0;
 constexpr double kEmptyCtaTiles = 1.0;
 
 // The sequences' lengths as the planner sees them: n entries of quantized tiles,
@@ -187,14 +190,14 @@ void plan_splits_for(const kvq_cache *h, const PlanInput &in, int *n_qsplits, in
     const int64_t nres = (in.max_r + 15) / 16;
     // residual CTA: its tiles shared by the 4 warps of each of its query heads
     const int heads_per_cta = per_kv ? hg : 1;
-    const double c_res1 = kCtaFixedTiles + static_cast<double>((nres * heads_per_cta + 3) / 4);
+    const double c_res1 = kResCtaFixedTiles + static_cast<double>((nres * heads_per_cta + 3) / 4);
     // the tensor-core kernel deals the residual tiles over the warps of n_rs residual splits
     // (4 / HG warps per head in each); a residual tile on CUDA cores costs about two
     // quantized tiles.  n_rs grows until a residual warp's share costs no more than a
     // quantized CTA (a long full-precision store, e.g. LogQuant's, then spreads out).
     const int64_t wph = 4 / heads_per_cta;
     auto residual_cost = [&](int64_t n_rs) {
-        return kCtaFixedTiles + 2.0 * static_cast<double>((nres + wph * n_rs - 1) / (wph * n_rs));
+        return kResCtaFixedTiles + 2.0 * static_cast<double>((nres + wph * n_rs - 1) / (wph * n_rs));
     };
     int64_t best_S = 0, best_per = 1, best_rs = extra;
     if (tiles > 0) {
