@@ -163,12 +163,12 @@ __device__ __forceinline__ uint32_t code_quad(const float4 &x, const QuadParams 
 // codes[t * D + c] (t relative to the first tile) and store them at dst.
 // Word w of a tile belongs to lane w / W; its slot s (0 .. 8/N - 1) holds, in
 // byte b, the element (row = lane/4 + 8*(s%2), col = 4*(lane%4) + b) of block
-// (chunk) j = (w % W) * (4/N) + s/2 at bit 8*b + N*s.  A key row's four columns
-// are four consecutive channels, one 32-bit load of codes; a value row's are four
-// tokens, four byte loads.  Every code is below 2^N, so a slot's four bytes
-// shifted by N*s stay inside their bytes.
-template <int D, int N, bool IS_V>
-__device__ void pack_tiles(const uint8_t *codes, int ntiles, uint32_t *dst) {
+// (chunk) j = (w % W) * (4/N) + s/2 at bit 8*b + N*s.  Every code is below 2^N, so a
+// slot's four bytes shifted by N*s stay inside their bytes.  For keys (rows = tokens,
+// columns = channels) a row's four columns are four consecutive channels: one 32-bit
+// load of codes per slot.
+template <int D, int N>
+__device__ void pack_key_tiles(const uint8_t *codes, int ntiles, uint32_t *dst) {
     constexpr int TW = D * N / 2;        // words per tile
     constexpr int W = D * N / 64;        // words per lane
     constexpr int B = 4 / N;             // blocks per word
@@ -184,17 +184,51 @@ __device__ void pack_tiles(const uint8_t *codes, int ntiles, uint32_t *dst) {
             const int j = wl * B + (slot >> 1);
             const int row = (lane >> 2) + 8 * (slot & 1);
             const int col0 = 4 * (lane & 3);
-            uint32_t v;
-            if constexpr (IS_V) {
-                const uint8_t *p = codes + (tile * 16 + col0) * D + 16 * j + row;
-                v = static_cast<uint32_t>(p[0]) | (static_cast<uint32_t>(p[D]) << 8) |
-                    (static_cast<uint32_t>(p[2 * D]) << 16) | (static_cast<uint32_t>(p[3 * D]) << 24);
-            } else {
-                v = *reinterpret_cast<const uint32_t *>(codes + (tile * 16 + row) * D + 16 * j + col0);
-            }
+            const uint32_t v = *reinterpret_cast<const uint32_t *>(codes + (tile * 16 + row) * D + 16 * j + col0);
             word |= v << (N * slot);
         }
         dst[wi] = word;
+    }
+}
+
+// The same words for values (rows = channels, columns = tokens), four at a time.  The words of lanes
+// q + 4k + 16h (k = 0 .. 3) at word wl share their tokens (4q .. 4q + 3) and hold, slot by
+// slot, four consecutive channels c0 + k: one 32-bit load per token brings a 4 x 4 block of
+// codes, and a byte transpose in registers gives the four words' bytes.  Thread (q, h) takes
+// the slots from slot q on, so the loads of a warp spread over the banks.
+template <int D, int N>
+__device__ void pack_value_tiles(const uint8_t *codes, int ntiles, uint32_t *dst) {
+    constexpr int TW = D * N / 2;        // words per tile
+    constexpr int W = D * N / 64;        // words per lane
+    constexpr int B = 4 / N;             // blocks per word
+    constexpr int NS = 2 * B;            // slots per word
+    constexpr int TPT = TW / 4;          // threads per tile: (wl, q, h)
+    const int total = ntiles * TPT;
+    for (int i = threadIdx.x; i < total; i += blockDim.x) {
+        const int tile = i / TPT;
+        const int r = i - tile * TPT;
+        const int wl = r % W, q = (r / W) & 3, h = r / (4 * W);
+        const uint8_t *rows = codes + (tile * 16 + 4 * q) * D;
+        uint32_t word[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int step = 0; step < NS; ++step) {
+            const int slot = (step + q) % NS;
+            const int c0 = 16 * (wl * B + (slot >> 1)) + 8 * (slot & 1) + 4 * h;
+            uint32_t in[4];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) in[b] = *reinterpret_cast<const uint32_t *>(rows + b * D + c0);
+            // out[k] byte b = in[b] byte k
+            const uint32_t t0 = __byte_perm(in[0], in[1], 0x5140), t1 = __byte_perm(in[0], in[1], 0x7362);
+            const uint32_t t2 = __byte_perm(in[2], in[3], 0x5140), t3 = __byte_perm(in[2], in[3], 0x7362);
+            const int sh = N * slot;
+            word[0] |= __byte_perm(t0, t2, 0x5410) << sh;
+            word[1] |= __byte_perm(t0, t2, 0x7632) << sh;
+            word[2] |= __byte_perm(t1, t3, 0x5410) << sh;
+            word[3] |= __byte_perm(t1, t3, 0x7632) << sh;
+        }
+        uint32_t *out = dst + tile * TW + (q + 16 * h) * W + wl;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) out[4 * k * W] = word[k];
     }
 }
 
@@ -275,8 +309,8 @@ __device__ void load_group(const uint16_t *slice, int64_t tok0, const int32_t *r
 }
 
 // BATCH: the value parameters batched per warp (groups of 64 tokens or more, four or more
-// token pairs per warp); else computed per token pair
-template <int D, int N, bool BATCH>
+// token pairs per warp); else computed per token pair.  BF16: the inputs are bf16, else fp16.
+template <int D, int N, bool BATCH, bool BF16>
 __global__ void __launch_bounds__(kQuantThreads, 4) quantize_pack_kernel(const QuantizeArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
     constexpr int d = D, bits = N;
@@ -330,7 +364,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quantize_pack_kernel(const Q
         for (int t = warp; t < G; t += kQuantThreads / 32) {
             uint32_t mag[4];
             for (int e = 0; e < per_lane; ++e)
-                mag[e] = __float_as_uint(fabsf(widen(xs[t * d + lane * per_lane + e], a.bf16)));
+                mag[e] = __float_as_uint(fabsf(widen(xs[t * d + lane * per_lane + e], BF16)));
             unsigned picked = 0;
             for (int o = 0; o < a.n_out; ++o) {
                 uint64_t best = 0;   // (|x| bits << 16) | (0xffff - channel): the larger key wins
@@ -366,8 +400,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quantize_pack_kernel(const Q
         const uint32_t *xw = reinterpret_cast<const uint32_t *>(xs) + kg * GK * NP;   // [GK][NP] pairs
         const int per = GK / parts;
         uint32_t lo, hi;
-        if (a.bf16) pair_minmax<true>(xw + (part * per) * NP + cp, NP, per, a.sym, lo, hi);
-        else pair_minmax<false>(xw + (part * per) * NP + cp, NP, per, a.sym, lo, hi);
+        pair_minmax<BF16>(xw + (part * per) * NP + cp, NP, per, a.sym, lo, hi);
         uint32_t *redu = reinterpret_cast<uint32_t *>(red);
         redu[threadIdx.x] = lo;
         redu[kQuantThreads + threadIdx.x] = hi;
@@ -376,8 +409,8 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quantize_pack_kernel(const Q
             const int c = threadIdx.x, pc = c >> 1, sh = 16 * (c & 1);
             float mn = FLT_MAX, mx = -FLT_MAX;
             for (int p = 0; p < parts; ++p) {
-                mn = fminf(mn, widen(static_cast<uint16_t>(redu[p * NP + pc] >> sh), a.bf16));
-                mx = fmaxf(mx, widen(static_cast<uint16_t>(redu[kQuantThreads + p * NP + pc] >> sh), a.bf16));
+                mn = fminf(mn, widen(static_cast<uint16_t>(redu[p * NP + pc] >> sh), BF16));
+                mx = fmaxf(mx, widen(static_cast<uint16_t>(redu[kQuantThreads + p * NP + pc] >> sh), BF16));
             }
             float s;
             int z;
@@ -411,7 +444,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quantize_pack_kernel(const Q
             const int4 o4 = make_int4(z0, z1, z0, z1);
             uint8_t *kcodes = codes + kg * GK * d;
             for (int t = part; t < GK; t += 2 * parts) {
-                const float2 x0 = widen2(xw[t * NP + cp], a.bf16), x1 = widen2(xw[(t + parts) * NP + cp], a.bf16);
+                const float2 x0 = widen2(xw[t * NP + cp], BF16), x1 = widen2(xw[(t + parts) * NP + cp], BF16);
                 const uint32_t w = code_quad<N>(make_float4(x0.x, x0.y, x1.x, x1.y), qp, s4, o4);
                 *reinterpret_cast<uint16_t *>(kcodes + t * d + 2 * cp) = static_cast<uint16_t>(w & 0xffffu);
                 *reinterpret_cast<uint16_t *>(kcodes + (t + parts) * d + 2 * cp) = static_cast<uint16_t>(w >> 16);
@@ -419,7 +452,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quantize_pack_kernel(const Q
         }
         __syncthreads();
     }
-    pack_tiles<D, N, false>(codes, G / 16, a.kc + slice * words_per_slice + (out_tok / 16) * TW);
+    pack_key_tiles<D, N>(codes, G / 16, a.kc + slice * words_per_slice + (out_tok / 16) * TW);
     __syncthreads();
 
     // ------------------------------ values ----------------------------
@@ -445,9 +478,8 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quantize_pack_kernel(const Q
                 uint32_t w[per_lane / 2];
                 load_words<per_lane / 2>(reinterpret_cast<const uint32_t *>(xs + t * d + hl * per_lane), w);
                 uint32_t lo, hi;
-                if (a.bf16) pair_minmax<true>(w, 1, per_lane / 2, a.sym, lo, hi);
-                else pair_minmax<false>(w, 1, per_lane / 2, a.sym, lo, hi);
-                const float2 l2 = widen2(lo, a.bf16), h2 = widen2(hi, a.bf16);
+                pair_minmax<BF16>(w, 1, per_lane / 2, a.sym, lo, hi);
+                const float2 l2 = widen2(lo, BF16), h2 = widen2(hi, BF16);
                 float mn = fminf(l2.x, l2.y), mx = fmaxf(h2.x, h2.y);
                 for (int off = seg >> 1; off > 0; off >>= 1) {
                     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
@@ -496,7 +528,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quantize_pack_kernel(const Q
                 const int4 o4 = make_int4(off, off, off, off);
     #pragma unroll
                 for (int k = 0; k < per_lane / 4; ++k) {
-                    const float2 x0 = widen2(w[2 * k], a.bf16), x1 = widen2(w[2 * k + 1], a.bf16);
+                    const float2 x0 = widen2(w[2 * k], BF16), x1 = widen2(w[2 * k + 1], BF16);
                     reinterpret_cast<uint32_t *>(codes + t * d + hl * per_lane)[k] =
                         code_quad<N>(make_float4(x0.x, x0.y, x1.x, x1.y), qp, s4, o4);
                 }
@@ -524,7 +556,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quantize_pack_kernel(const Q
                 }
     #pragma unroll
                 for (int e = 0; e < per_lane; ++e) {
-                    x[e] = widen(xb[e], a.bf16);
+                    x[e] = widen(xb[e], BF16);
                     if (a.sym) {
                         mx = fmaxf(mx, fabsf(x[e]));
                     } else {
@@ -569,8 +601,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quantize_pack_kernel(const Q
             }
         }
         __syncthreads();
-        pack_tiles<D, N, true>(codes, G / 16,
-                   a.vc + slice * words_per_slice + (out_tok / 16) * TW);
+        pack_value_tiles<D, N>(codes, G / 16, a.vc + slice * words_per_slice + (out_tok / 16) * TW);
     }
 }
 
@@ -699,8 +730,9 @@ size_t quantize_smem_bytes(int d, int G, int Gv) {
 
 using QuantizeKernel = void (*)(const QuantizeArgs);
 template <int D, int N>
-QuantizeKernel quantize_instance(bool batch) {
-    return batch ? quantize_pack_kernel<D, N, true> : quantize_pack_kernel<D, N, false>;
+QuantizeKernel quantize_instance(bool batch, bool bf16) {
+    if (bf16) return batch ? quantize_pack_kernel<D, N, true, true> : quantize_pack_kernel<D, N, false, true>;
+    return batch ? quantize_pack_kernel<D, N, true, false> : quantize_pack_kernel<D, N, false, false>;
 }
 
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s) {
@@ -714,14 +746,14 @@ cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s) {
     void (*kernel)(const QuantizeArgs) = nullptr;
     int variant = -1;
     const bool batch = tokens / 2 >= 4 * (kQuantThreads / 32);
-    if (a.d == 64 && a.bits == 2) kernel = quantize_instance<64, 2>(batch), variant = 0;
-    else if (a.d == 64 && a.bits == 4) kernel = quantize_instance<64, 4>(batch), variant = 1;
-    else if (a.d == 128 && a.bits == 2) kernel = quantize_instance<128, 2>(batch), variant = 2;
-    else if (a.d == 128 && a.bits == 4) kernel = quantize_instance<128, 4>(batch), variant = 3;
+    if (a.d == 64 && a.bits == 2) kernel = quantize_instance<64, 2>(batch, a.bf16), variant = 0;
+    else if (a.d == 64 && a.bits == 4) kernel = quantize_instance<64, 4>(batch, a.bf16), variant = 1;
+    else if (a.d == 128 && a.bits == 2) kernel = quantize_instance<128, 2>(batch, a.bf16), variant = 2;
+    else if (a.d == 128 && a.bits == 4) kernel = quantize_instance<128, 4>(batch, a.bf16), variant = 3;
     if (!kernel) return cudaErrorInvalidValue;
-    variant = 2 * variant + (batch ? 1 : 0);
+    variant = 4 * variant + (a.bf16 ? 2 : 0) + (batch ? 1 : 0);
     // opt in to the largest dynamic shared memory any configuration needs, once per device and variant
-    static bool configured[64][8] = {};
+    static bool configured[64][16] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
