@@ -132,6 +132,8 @@ GEOMS = [  # bits, symmetric, dtype, G, Gv, d, R
     (2, False, wl.FP16, 32, 16, 64, 32),
     (4, False, wl.FP16, 16, 16, 64, 16),
     (4, True, wl.FP16, 32, 32, 128, 32),
+    (2, False, wl.FP16, 32, 32, 128, 64),   # two key groups per CTA, batched value parameters
+    (2, False, wl.BF16, 32, 32, 128, 32),   # a flush of one key group: one group per CTA
 ]
 
 
