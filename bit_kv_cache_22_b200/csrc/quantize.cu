@@ -152,11 +152,7 @@ __device__ __forceinline__ uint32_t code_quad(const float4 &x, const QuadParams 
         }
     }
     constexpr uint32_t kOver = 0x01010101u << N;   // bit n of every byte: the code L + 1
-    if (w & kOver) {
-        const uint32_t over = (w & kOver) >> N;     // 1 in each byte to clamp
-        w -= over;                                  // L + 1 -> L
-    }
-    return w;
+    return w - ((w & kOver) >> N);                 // L + 1 -> L: 1 off each such byte, no borrow
 }
 
 // Assemble the packed words of `ntiles` 16-token tiles from byte codes
