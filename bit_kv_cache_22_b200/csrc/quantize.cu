@@ -305,8 +305,10 @@ __device__ void load_group(const uint16_t *slice, int64_t tok0, const int32_t *r
 }
 
 // BATCH: the value parameters batched per warp (groups of 64 tokens or more, four or more
-// token pairs per warp); else computed per token pair.  BF16: the inputs are bf16, else fp16.
-template <int D, int N, bool BATCH, bool BF16>
+// token pairs per warp); else computed per token pair.  UNROLL: the value phase's token-pair
+// loops unrolled by two (eight or more token pairs per warp).  BF16: the inputs are bf16, else
+// fp16.
+template <int D, int N, bool BATCH, bool UNROLL, bool BF16>
 __global__ void __launch_bounds__(kQuantThreads, 4) quantize_pack_kernel(const QuantizeArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
     constexpr int d = D, bits = N;
@@ -469,6 +471,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quantize_pack_kernel(const Q
         const int j = hl / seg;                      // this lane's group in its token
         constexpr int kWarps = kQuantThreads / 32;
         if constexpr (BATCH) {       // four or more token pairs per warp: parameters batched
+#pragma unroll(UNROLL ? 2 : 1)
             for (int tp = warp; tp < G / 2; tp += kWarps) {
                 const int t = 2 * tp + half;
                 uint32_t w[per_lane / 2];
@@ -510,6 +513,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4) quantize_pack_kernel(const Q
                 vg[t * ngv + jq] = make_float4(cp.ri, kRoundMagic + static_cast<float>(cp.off), cp.cut, cp.s);
             }
             __syncwarp();
+#pragma unroll(UNROLL ? 2 : 1)
             for (int tp = warp; tp < G / 2; tp += kWarps) {
                 const int t = 2 * tp + half;
                 uint32_t w[per_lane / 2];
@@ -726,9 +730,13 @@ size_t quantize_smem_bytes(int d, int G, int Gv) {
 
 using QuantizeKernel = void (*)(const QuantizeArgs);
 template <int D, int N>
-QuantizeKernel quantize_instance(bool batch, bool bf16) {
-    if (bf16) return batch ? quantize_pack_kernel<D, N, true, true> : quantize_pack_kernel<D, N, false, true>;
-    return batch ? quantize_pack_kernel<D, N, true, false> : quantize_pack_kernel<D, N, false, false>;
+QuantizeKernel quantize_instance(bool batch, bool unroll, bool bf16) {
+    if (bf16) {
+        if (!batch) return quantize_pack_kernel<D, N, false, false, true>;
+        return unroll ? quantize_pack_kernel<D, N, true, true, true> : quantize_pack_kernel<D, N, true, false, true>;
+    }
+    if (!batch) return quantize_pack_kernel<D, N, false, false, false>;
+    return unroll ? quantize_pack_kernel<D, N, true, true, false> : quantize_pack_kernel<D, N, true, false, false>;
 }
 
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s) {
@@ -742,14 +750,15 @@ cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s) {
     void (*kernel)(const QuantizeArgs) = nullptr;
     int variant = -1;
     const bool batch = tokens / 2 >= 4 * (kQuantThreads / 32);
-    if (a.d == 64 && a.bits == 2) kernel = quantize_instance<64, 2>(batch, a.bf16), variant = 0;
-    else if (a.d == 64 && a.bits == 4) kernel = quantize_instance<64, 4>(batch, a.bf16), variant = 1;
-    else if (a.d == 128 && a.bits == 2) kernel = quantize_instance<128, 2>(batch, a.bf16), variant = 2;
-    else if (a.d == 128 && a.bits == 4) kernel = quantize_instance<128, 4>(batch, a.bf16), variant = 3;
+    const bool unroll = tokens / 2 >= 8 * (kQuantThreads / 32);
+    if (a.d == 64 && a.bits == 2) kernel = quantize_instance<64, 2>(batch, unroll, a.bf16), variant = 0;
+    else if (a.d == 64 && a.bits == 4) kernel = quantize_instance<64, 4>(batch, unroll, a.bf16), variant = 1;
+    else if (a.d == 128 && a.bits == 2) kernel = quantize_instance<128, 2>(batch, unroll, a.bf16), variant = 2;
+    else if (a.d == 128 && a.bits == 4) kernel = quantize_instance<128, 4>(batch, unroll, a.bf16), variant = 3;
     if (!kernel) return cudaErrorInvalidValue;
-    variant = 4 * variant + (a.bf16 ? 2 : 0) + (batch ? 1 : 0);
+    variant = 6 * variant + (a.bf16 ? 3 : 0) + (batch ? (unroll ? 2 : 1) : 0);
     // opt in to the largest dynamic shared memory any configuration needs, once per device and variant
-    static bool configured[64][16] = {};
+    static bool configured[64][24] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
